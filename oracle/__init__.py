@@ -1,0 +1,250 @@
+"""CPU oracle of the W4A8-FP8 routed MoE layer (plain C, fp32), with numpy wrappers.
+
+TEST INFRASTRUCTURE ONLY: imported by tests/, ``__graft_entry__.smoke()`` and
+the cpu_baseline / reference leg of ``bench.py``.  The CUDA library never
+imports, links or calls it, and it shares no code with the CUDA library.
+
+Every function cites, in ``oracle.c``, the page passage it follows.  Parity of
+the fp32 accumulation order inside the GPU's tensor-core sums (and of expf's
+last ulp) is not pinned by any page: those differences are covered only by
+the layer's stated tolerances (see tests/).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SO = os.path.join(_HERE, "liboracle.so")
+_SRC = os.path.join(_HERE, "oracle.c")
+
+
+def build(verbose: bool = False) -> None:
+    if os.path.exists(_SO) and os.path.getmtime(_SO) >= os.path.getmtime(_SRC):
+        return
+    cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-ffp-contract=off",
+           "-fno-fast-math", _SRC, "-o", _SO, "-lm"]
+    if verbose:
+        print(" ".join(cmd))
+    subprocess.run(cmd, check=True)
+
+
+class _Layer(ctypes.Structure):
+    _fields_ = [("E", ctypes.c_int), ("H", ctypes.c_int), ("N", ctypes.c_int),
+                ("group", ctypes.c_int),
+                ("gate_packed", ctypes.c_void_p), ("up_packed", ctypes.c_void_p),
+                ("down_packed", ctypes.c_void_p),
+                ("gate_scales", ctypes.c_void_p), ("up_scales", ctypes.c_void_p),
+                ("down_scales", ctypes.c_void_p),
+                ("n_shared", ctypes.c_int), ("shared_N", ctypes.c_int),
+                ("sh_gate", ctypes.c_void_p), ("sh_up", ctypes.c_void_p),
+                ("sh_down", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        build()
+        L = ctypes.CDLL(_SO)
+        vp, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+        L.or_bf16_to_f32.argtypes = [ctypes.c_uint16]
+        L.or_bf16_to_f32.restype = ctypes.c_float
+        L.or_f32_to_bf16.argtypes = [ctypes.c_float]
+        L.or_f32_to_bf16.restype = ctypes.c_uint16
+        L.or_e4m3_decode.argtypes = [ctypes.c_uint8]
+        L.or_e4m3_decode.restype = ctypes.c_float
+        L.or_e4m3_encode.argtypes = [ctypes.c_float]
+        L.or_e4m3_encode.restype = ctypes.c_uint8
+        L.or_rtn_pack.argtypes = [vp, i64, i64, i32, vp, vp, vp]
+        L.or_rtn_pack.restype = i32
+        L.or_unpack.argtypes = [vp, i64, i64, vp]
+        L.or_unpack.restype = None
+        L.or_quant_tokens.argtypes = [vp, i64, i64, vp, vp]
+        L.or_quant_tokens.restype = None
+        L.or_route_topk.argtypes = [vp, i64, i32, i32, vp, vp]
+        L.or_route_topk.restype = None
+        L.or_permute.argtypes = [vp, i64, i32, i32, vp, vp, vp]
+        L.or_permute.restype = None
+        L.or_moe_forward.argtypes = [ctypes.POINTER(_Layer), vp, vp, i64, i32, vp] + [vp] * 11
+        L.or_moe_forward.restype = i32
+        L.or_moe_forward_dense.argtypes = [ctypes.POINTER(_Layer), vp, vp, i64, i32, vp, vp, vp,
+                                           vp, vp]
+        L.or_moe_forward_dense.restype = i32
+        _lib = L
+    return _lib
+
+
+def _p(a):
+    if a is None:
+        return None
+    assert a.flags["C_CONTIGUOUS"], "arrays passed to the oracle must be C-contiguous"
+    return ctypes.c_void_p(a.ctypes.data)
+
+
+# ---- scalars --------------------------------------------------------------------------------
+
+def bf16_to_f32(h: np.ndarray) -> np.ndarray:
+    return (np.asarray(h, np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+def e4m3_decode(c: int) -> float:
+    return float(lib().or_e4m3_decode(int(c)))
+
+
+def e4m3_encode(x: float) -> int:
+    return int(lib().or_e4m3_encode(float(x)))
+
+
+def e4m3_decode_table() -> np.ndarray:
+    return np.array([e4m3_decode(c) for c in range(256)], np.float32)
+
+
+# ---- S0..S3 ---------------------------------------------------------------------------------
+
+def rtn_pack(w_bf16: np.ndarray, group: int = 128):
+    """bf16 bits [rows, K] -> (packed int32 [rows, K/8], scales bf16 bits [rows, K/g], codes int8)."""
+    w = np.ascontiguousarray(w_bf16, np.uint16)
+    rows, K = w.shape
+    packed = np.zeros((rows, K // 8), np.int32)
+    scales = np.zeros((rows, K // group), np.uint16)
+    codes = np.zeros((rows, K), np.int8)
+    rc = lib().or_rtn_pack(_p(w), rows, K, group, _p(packed), _p(scales), _p(codes))
+    if rc != 0:
+        raise ValueError("or_rtn_pack: bad shape or code out of range")
+    return packed, scales, codes
+
+
+def unpack(packed: np.ndarray, K: int) -> np.ndarray:
+    packed = np.ascontiguousarray(packed, np.int32)
+    rows = packed.shape[0]
+    codes = np.zeros((rows, K), np.int8)
+    lib().or_unpack(_p(packed), rows, K, _p(codes))
+    return codes
+
+
+def quant_tokens(x_bf16: np.ndarray):
+    x = np.ascontiguousarray(x_bf16, np.uint16)
+    T, H = x.shape
+    q = np.zeros((T, H), np.uint8)
+    s = np.zeros(T, np.float32)
+    lib().or_quant_tokens(_p(x), T, H, _p(q), _p(s))
+    return q, s
+
+
+def route_topk(logits: np.ndarray, k: int):
+    l = np.ascontiguousarray(logits, np.float32)
+    T, E = l.shape
+    ids = np.zeros((T, k), np.int32)
+    gates = np.zeros((T, k), np.float32)
+    lib().or_route_topk(_p(l), T, E, k, _p(ids), _p(gates))
+    return ids, gates
+
+
+def permute(ids: np.ndarray, E: int):
+    ids = np.ascontiguousarray(ids, np.int32)
+    T, k = ids.shape
+    P = T * k
+    offsets = np.zeros(E + 1, np.int32)
+    sorted_pairs = np.zeros(P, np.int32)
+    row_of_pair = np.zeros(P, np.int32)
+    lib().or_permute(_p(ids), T, k, E, _p(offsets), _p(sorted_pairs), _p(row_of_pair))
+    return offsets, sorted_pairs, row_of_pair
+
+
+# ---- the layer ------------------------------------------------------------------------------
+
+class Layer:
+    """Host copy of one layer's packed weights (numpy), laid out like the C ABI's layer."""
+
+    def __init__(self, E, H, N, gate_packed, up_packed, down_packed, gate_scales, up_scales,
+                 down_scales, group=128, sh_gate=None, sh_up=None, sh_down=None):
+        self.E, self.H, self.N, self.group = E, H, N, group
+        self.gate_packed = np.ascontiguousarray(gate_packed, np.int32)
+        self.up_packed = np.ascontiguousarray(up_packed, np.int32)
+        self.down_packed = np.ascontiguousarray(down_packed, np.int32)
+        self.gate_scales = np.ascontiguousarray(gate_scales, np.uint16)
+        self.up_scales = np.ascontiguousarray(up_scales, np.uint16)
+        self.down_scales = np.ascontiguousarray(down_scales, np.uint16)
+        self.sh_gate = None if sh_gate is None else np.ascontiguousarray(sh_gate, np.uint16)
+        self.sh_up = None if sh_up is None else np.ascontiguousarray(sh_up, np.uint16)
+        self.sh_down = None if sh_down is None else np.ascontiguousarray(sh_down, np.uint16)
+        self.n_shared = 0 if sh_gate is None else sh_gate.shape[0]
+        self.shared_N = 0 if sh_gate is None else sh_gate.shape[1]
+
+    def _c(self):
+        return _Layer(self.E, self.H, self.N, self.group,
+                      _p(self.gate_packed), _p(self.up_packed), _p(self.down_packed),
+                      _p(self.gate_scales), _p(self.up_scales), _p(self.down_scales),
+                      self.n_shared, self.shared_N,
+                      _p(self.sh_gate), _p(self.sh_up), _p(self.sh_down))
+
+
+def moe_forward(layer: Layer, x_bf16: np.ndarray, logits: np.ndarray, k: int):
+    """Run the layer; returns a dict with out (bf16 bits) and every intermediate."""
+    x = np.ascontiguousarray(x_bf16, np.uint16)
+    l = np.ascontiguousarray(logits, np.float32)
+    T, H = x.shape
+    E, N = layer.E, layer.N
+    P = T * k
+    r = dict(out=np.zeros((T, H), np.uint16), ids=np.zeros((T, k), np.int32),
+             gates=np.zeros((T, k), np.float32), offsets=np.zeros(E + 1, np.int32),
+             sorted_pairs=np.zeros(P, np.int32), row_of_pair=np.zeros(P, np.int32),
+             xq=np.zeros((T, H), np.uint8), s_x=np.zeros(T, np.float32),
+             hq=np.zeros((P, N), np.uint8), s_h=np.zeros(P, np.float32),
+             y=np.zeros((P, H), np.float32), out_f32=np.zeros((T, H), np.float32))
+    L = layer._c()
+    rc = lib().or_moe_forward(ctypes.byref(L), _p(x), _p(l), T, k, _p(r["out"]), _p(r["ids"]),
+                              _p(r["gates"]), _p(r["offsets"]), _p(r["sorted_pairs"]),
+                              _p(r["row_of_pair"]), _p(r["xq"]), _p(r["s_x"]), _p(r["hq"]),
+                              _p(r["s_h"]), _p(r["y"]), _p(r["out_f32"]))
+    if rc != 0:
+        raise ValueError("or_moe_forward: bad shape")
+    return r
+
+
+def moe_forward_dense(layer: Layer, x_bf16: np.ndarray, logits: np.ndarray, k: int):
+    x = np.ascontiguousarray(x_bf16, np.uint16)
+    l = np.ascontiguousarray(logits, np.float32)
+    T, H = x.shape
+    E, N = layer.E, layer.N
+    r = dict(out=np.zeros((T, H), np.uint16), out_f32=np.zeros((T, H), np.float32),
+             hq=np.zeros((T, E, N), np.uint8), s_h=np.zeros((T, E), np.float32),
+             y=np.zeros((T, E, H), np.float32))
+    L = layer._c()
+    rc = lib().or_moe_forward_dense(ctypes.byref(L), _p(x), _p(l), T, k, _p(r["out"]),
+                                    _p(r["out_f32"]), _p(r["hq"]), _p(r["s_h"]), _p(r["y"]))
+    if rc != 0:
+        raise ValueError("or_moe_forward_dense: bad shape")
+    return r
+
+
+def pack_workload_layer(wl, experts=None, with_shared=True):
+    """Pack (RTN, oracle side) the seeded weights of workload `wl`.
+
+    Only experts in `experts` (default: all) are drawn and packed; the others stay zero,
+    which is enough when the caller knows which experts its tokens route to.
+    """
+    import synth
+    E, H, N, g = wl.E, wl.H, wl.N, wl.group
+    gp = np.zeros((E, N, H // 8), np.int32)
+    up = np.zeros((E, N, H // 8), np.int32)
+    dp = np.zeros((E, H, N // 8), np.int32)
+    gs = np.zeros((E, N, H // g), np.uint16)
+    us = np.zeros((E, N, H // g), np.uint16)
+    ds = np.zeros((E, H, N // g), np.uint16)
+    for e in (range(E) if experts is None else experts):
+        gp[e], gs[e], _ = rtn_pack(synth.expert_weight(wl, e, "gate"), g)
+        up[e], us[e], _ = rtn_pack(synth.expert_weight(wl, e, "up"), g)
+        dp[e], ds[e], _ = rtn_pack(synth.expert_weight(wl, e, "down"), g)
+    sh = {}
+    if with_shared and wl.n_shared:
+        sh = dict(sh_gate=np.stack([synth.shared_weight(wl, s, "gate") for s in range(wl.n_shared)]),
+                  sh_up=np.stack([synth.shared_weight(wl, s, "up") for s in range(wl.n_shared)]),
+                  sh_down=np.stack([synth.shared_weight(wl, s, "down") for s in range(wl.n_shared)]))
+    return Layer(E, H, N, gp, up, dp, gs, us, ds, group=g, **sh)

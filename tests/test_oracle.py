@@ -1,0 +1,386 @@
+"""Pins of the CPU oracle against facts fixed by the pages and by mathematics.
+
+Each test checks the oracle against something other than itself: hand-worked
+values under tests/golden/ (derived from the pages' rules), exhaustive
+brute-force searches, independent library routines (numpy sorts, fp64
+softmax, an fp64 dense MLP) and invariants.
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from conftest import golden_lines
+
+
+# ------------------------------------------------------------------------------------------------
+# E4M3
+# ------------------------------------------------------------------------------------------------
+
+def _all_finite_codes():
+    return [c for c in range(256) if (c & 0x7F) != 0x7F]
+
+
+def test_e4m3_decode_table_shape():
+    vals = oracle.e4m3_decode_table()
+    nan_codes = [c for c in range(256) if np.isnan(vals[c])]
+    assert nan_codes == [0x7F, 0xFF]
+    finite = vals[~np.isnan(vals)]
+    assert len(finite) == 254
+    assert len(set(finite.tolist())) == 253          # +0 and -0 compare equal
+    assert finite.max() == 448.0 and finite.min() == -448.0
+    pos = np.sort(np.unique(np.abs(finite)))
+    assert pos[1] == 2.0 ** -9                        # smallest subnormal
+    # subnormals + first binade are the equally spaced ladder 0..15 * 2^-9
+    assert np.array_equal(pos[:16], np.arange(16) * 2.0 ** -9)
+
+
+@pytest.mark.parametrize("line", list(golden_lines("e4m3_worked.txt")))
+def test_e4m3_worked_values(line):
+    x, code = line.split()
+    assert oracle.e4m3_encode(float(x)) == int(code, 16)
+
+
+def test_e4m3_roundtrip_all_codes():
+    for c in _all_finite_codes():
+        v = oracle.e4m3_decode(c)
+        assert oracle.e4m3_encode(v) == c, hex(c)
+
+
+def test_int4_codes_exact_in_e4m3():
+    for i in range(-8, 8):
+        c = oracle.e4m3_encode(float(i))
+        assert oracle.e4m3_decode(c) == float(i)
+
+
+def _brute_nearest(xs):
+    """Nearest finite E4M3 code by exhaustive search; ties to the even code; saturate."""
+    codes = np.array([c for c in range(128) if c != 0x7F], np.int64)   # non-negative magnitudes
+    mags = np.array([oracle.e4m3_decode(int(c)) for c in codes], np.float64)
+    out = []
+    for x in xs:
+        a = min(abs(float(x)), 448.0)
+        d = np.abs(mags - a)
+        best = np.flatnonzero(d == d.min())
+        if len(best) > 1:
+            best = [b for b in best if codes[b] % 2 == 0]
+        c = int(codes[best[0]])
+        if np.signbit(np.float32(x)):
+            c |= 0x80
+        out.append(c)
+    return out
+
+
+def test_e4m3_encode_vs_brute_force():
+    rng = np.random.default_rng(1)
+    mags = np.array(sorted(set(abs(oracle.e4m3_decode(c)) for c in _all_finite_codes())),
+                    np.float64)
+    mids = (mags[1:] + mags[:-1]) / 2
+    probes = []
+    for m in np.concatenate([mids, mags]):
+        f = np.float32(m)
+        probes += [f, np.nextafter(f, np.float32(np.inf)), np.nextafter(f, np.float32(0))]
+    probes += list(rng.standard_normal(4000).astype(np.float32) * 30)
+    probes += list((rng.standard_normal(2000) * 0.01).astype(np.float32))
+    probes += list(np.float32(2.0) ** rng.uniform(-14, 10, 2000).astype(np.float32))
+    probes = np.array(probes, np.float32)
+    probes = np.concatenate([probes, -probes])
+    got = [oracle.e4m3_encode(float(x)) for x in probes]
+    want = _brute_nearest(probes)
+    bad = [(float(p), g, w) for p, g, w in zip(probes, got, want) if g != w]
+    assert not bad, bad[:10]
+
+
+# ------------------------------------------------------------------------------------------------
+# INT4 RTN + pack-quantized storage
+# ------------------------------------------------------------------------------------------------
+
+def _f32_to_bf16_bits(x):
+    u = np.asarray(x, np.float32).view(np.uint32).astype(np.uint64)
+    return ((u + 0x7FFF + ((u >> 16) & 1)) >> 16).astype(np.uint16)
+
+
+@pytest.mark.parametrize("line", list(golden_lines("pack_words.txt")))
+def test_pack_words_golden(line):
+    f = line.split()
+    codes = np.array([int(v) for v in f[:8]], np.int8)
+    word = np.array([int(f[8], 16)], np.uint32).view(np.int32)
+    # the inverse (unpack) holds for every word, -8 included
+    assert np.array_equal(oracle.unpack(np.array([[word[0]]], np.int32), 8)[0], codes)
+    if codes.min() < -7:
+        return      # RTN with scale amax/7 never yields -8; packing it is covered via unpack
+    # build one 128-element group whose RTN codes are exactly `codes` in its first word:
+    # scale 2^-4 forced by a +-7*2^-4 element elsewhere in the group.
+    w = np.zeros((1, 128), np.float32)
+    w[0, :8] = codes.astype(np.float32) * 0.0625
+    w[0, 100] = 7 * 0.0625
+    packed, scales, got_codes = oracle.rtn_pack(_f32_to_bf16_bits(w))
+    assert oracle.bf16_to_f32(scales)[0, 0] == 0.0625
+    assert np.array_equal(got_codes[0, :8], codes)
+    assert packed[0, 0] == word[0]
+
+
+def test_unpack_every_nibble_every_position():
+    for pos in range(8):
+        for nib in range(16):
+            word = np.array([0x88888888 & ~(0xF << (4 * pos)) | (nib << (4 * pos))],
+                            np.uint32).view(np.int32)
+            codes = oracle.unpack(word.reshape(1, 1), 8)[0]
+            want = np.zeros(8, np.int8)
+            want[pos] = nib - 8
+            assert np.array_equal(codes, want), (pos, nib)
+
+
+def test_pack_roundtrip_random():
+    rng = np.random.default_rng(2)
+    w = _f32_to_bf16_bits(rng.standard_normal((64, 512)).astype(np.float32) * 0.02)
+    packed, scales, codes = oracle.rtn_pack(w)
+    assert codes.min() >= -8 and codes.max() <= 7
+    assert np.array_equal(oracle.unpack(packed, 512), codes)
+
+
+def test_rtn_worked_case():
+    groups = {}
+    scales_want = {}
+    for line in golden_lines("rtn_worked_case.txt"):
+        f = line.split()
+        if f[1] == "scale":
+            scales_want[f[0]] = float(f[2])
+        else:
+            groups.setdefault(f[0], []).append((int(f[1]), float(f[2]), int(f[3])))
+    names = sorted(groups)
+    w = np.zeros((len(names), 128), np.float32)
+    for gi, name in enumerate(names):
+        for idx, val, _ in groups[name]:
+            w[gi, idx] = val
+    wb = _f32_to_bf16_bits(w)
+    assert np.array_equal(oracle.bf16_to_f32(wb), w)      # listed values are exact bf16
+    packed, scales, codes = oracle.rtn_pack(wb)
+    for gi, name in enumerate(names):
+        assert oracle.bf16_to_f32(scales)[gi, 0] == scales_want[name]
+        for idx, _, code in groups[name]:
+            assert codes[gi, idx] == code, (name, idx)
+
+
+def test_rtn_error_bound_and_zero_group():
+    rng = np.random.default_rng(3)
+    w = rng.standard_normal((32, 1024)).astype(np.float32) * 0.02
+    w[5, 128:256] = 0.0                                  # an all-zero group
+    wb = _f32_to_bf16_bits(w)
+    packed, scales, codes = oracle.rtn_pack(wb)
+    wf = oracle.bf16_to_f32(wb).astype(np.float64)
+    s = np.repeat(oracle.bf16_to_f32(scales).astype(np.float64), 128, axis=1)
+    assert scales[5, 1] == 0 and not codes[5, 128:256].any()
+    nz = s > 0
+    # amax/s <= 7*(1+2^-8) so no code is clamped, and rounding error is at most half a step
+    assert np.all(np.abs(wf - codes * s)[nz] <= 0.5 * s[nz] * (1 + 2 ** -20))
+    assert codes.min() >= -7                              # RTN with scale amax/7 never gives -8
+
+
+# ------------------------------------------------------------------------------------------------
+# per-token FP8
+# ------------------------------------------------------------------------------------------------
+
+def test_token_quant_closed_form():
+    x = np.zeros((3, 256), np.float32)
+    x[0, 0] = 1.0                 # amax 1 -> s = fp32(1/448)
+    x[0, 1] = 0.5                 # 0.5*448 = 224 exactly representable -> 0x76
+    x[0, 2] = 0.30078125          # bf16(0.3): 134.75 -> 128 (spacing 16) -> 0x70
+    x[0, 3] = -1.0
+    x[2, :] = 0.875               # s = 2^-9 exactly, all codes 0x7e
+    q, s = oracle.quant_tokens(_f32_to_bf16_bits(x))
+    assert s[0] == np.float32(1.0) / np.float32(448.0)
+    assert list(q[0, :4]) == [0x7E, 0x76, 0x70, 0xFE]
+    assert s[1] == 0.0 and not q[1].any()                # zero row
+    assert s[2] == 2.0 ** -9 and np.all(q[2] == 0x7E)
+
+
+def test_token_quant_properties():
+    wl = synth.WORKLOADS["decode_t8"]
+    x = synth.tokens(wl)
+    q, s = oracle.quant_tokens(x)
+    xf = oracle.bf16_to_f32(x)
+    amax = np.abs(xf).max(axis=1)
+    assert np.array_equal(s, (amax / np.float32(448)).astype(np.float32))
+    dec = oracle.e4m3_decode_table()
+    for t in range(x.shape[0]):
+        i = np.argmax(np.abs(xf[t]))
+        assert q[t, i] in (0x7E, 0xFE)
+        # dequantized value within half an E4M3 step (relative 2^-4 for normals) of x
+        d = dec[q[t]].astype(np.float64) * s[t]
+        err = np.abs(d - xf[t])
+        bound = np.maximum(np.abs(xf[t]) * 2.0 ** -4, 2.0 ** -10 * s[t]) * (1 + 1e-6)
+        assert np.all(err <= bound)
+
+
+# ------------------------------------------------------------------------------------------------
+# routing + permutation
+# ------------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("line", list(golden_lines("routing_worked.txt")))
+def test_routing_worked(line):
+    k, l, ids, gates = [p.split() for p in line.split("|")]
+    k = int(k[0])
+    got_ids, got_g = oracle.route_topk(np.array([[float(v) for v in l]], np.float32), k)
+    assert got_ids[0].tolist() == [int(v) for v in ids]
+    assert np.array_equal(got_g[0], np.array([float(v) for v in gates], np.float32))
+
+
+def test_routing_vs_sort_and_softmax():
+    rng = np.random.default_rng(4)
+    logits = rng.standard_normal((300, 64)).astype(np.float32)
+    logits[:10, 5] = logits[:10, 9]                      # planted ties
+    for k in (1, 2, 6, 64):
+        ids, gates = oracle.route_topk(logits, k)
+        for t in range(logits.shape[0]):
+            order = np.lexsort((np.arange(64), -logits[t].astype(np.float64)))
+            assert ids[t].tolist() == order[:k].tolist()
+            sel = logits[t, order[:k]].astype(np.float64)
+            ref = np.exp(sel - sel.max())
+            ref /= ref.sum()
+            assert np.allclose(gates[t], ref, rtol=2e-6, atol=1e-7)
+            assert abs(float(gates[t].astype(np.float64).sum()) - 1.0) < 1e-6 * k
+        if k == 64:   # k = E: the gate is the full softmax
+            full = np.exp(logits - logits.max(1, keepdims=True))
+            full /= full.sum(1, keepdims=True)
+            back = np.zeros_like(full)
+            np.put_along_axis(back, ids, gates, 1)
+            assert np.allclose(back, full, rtol=2e-6, atol=1e-7)
+
+
+def test_permutation_vs_stable_sort():
+    rng = np.random.default_rng(5)
+    for T, k, E in ((50, 6, 256), (16, 2, 8), (1, 1, 1), (0, 2, 8), (333, 3, 17)):
+        ids = rng.integers(0, E, (T, k)).astype(np.int32) if T else np.zeros((0, k), np.int32)
+        offsets, sorted_pairs, rop = oracle.permute(ids, E)
+        flat = ids.reshape(-1)
+        ref = np.argsort(flat, kind="stable")
+        assert np.array_equal(sorted_pairs, ref)
+        assert np.array_equal(offsets, np.concatenate([[0], np.cumsum(np.bincount(flat, minlength=E))]))
+        assert offsets[-1] == T * k and np.all(np.diff(offsets) >= 0)
+        assert np.array_equal(rop[sorted_pairs], np.arange(T * k))
+
+
+# ------------------------------------------------------------------------------------------------
+# the layer
+# ------------------------------------------------------------------------------------------------
+
+def _tiny_layer(wl):
+    return oracle.pack_workload_layer(wl)
+
+
+def test_layer_dense_brute_force_matches_permuted():
+    wl = synth.WORKLOADS["tiny"]
+    layer = _tiny_layer(wl)
+    x, lg = synth.tokens(wl), synth.logits(wl)
+    r = oracle.moe_forward(layer, x, lg, wl.k)
+    d = oracle.moe_forward_dense(layer, x, lg, wl.k)
+    assert np.array_equal(r["out"], d["out"])
+    assert np.array_equal(r["out_f32"], d["out_f32"])
+    for p in range(wl.P):
+        t, j = divmod(p, wl.k)
+        e = r["ids"][t, j]
+        row = r["row_of_pair"][p]
+        assert np.array_equal(r["hq"][row], d["hq"][t, e])
+        assert r["s_h"][row] == d["s_h"][t, e]
+        assert np.array_equal(r["y"][row], d["y"][t, e])
+
+
+def test_layer_constant_closed_form():
+    want = {}
+    for line in golden_lines("constant_layer.txt"):
+        t, o, hq = line.split()
+        want[int(t)] = (float(o), int(hq, 16))
+    T, H, N, E, k = 4, 128, 128, 2, 1
+    w0 = 0.02734375
+    def packed(sign, rows, K):
+        wb = _f32_to_bf16_bits(np.full((rows, K), sign * w0, np.float32))
+        return oracle.rtn_pack(wb)
+    gp = np.stack([packed(+1, N, H)[0], packed(-1, N, H)[0]])
+    gs = np.stack([packed(+1, N, H)[1], packed(-1, N, H)[1]])
+    dp = np.stack([packed(+1, H, N)[0], packed(-1, H, N)[0]])
+    ds = np.stack([packed(+1, H, N)[1], packed(-1, H, N)[1]])
+    layer = oracle.Layer(E, H, N, gp, gp, dp, gs, gs, ds)
+    x = _f32_to_bf16_bits(np.full((T, H), 0.875, np.float32))
+    lg = np.array([[1, 0], [0, 1], [1, 0], [0, 1]], np.float32)
+    r = oracle.moe_forward(layer, x, lg, k)
+    out = oracle.bf16_to_f32(r["out"])
+    for t in range(T):
+        assert np.all(out[t] == want[t][0]), (t, out[t, :4])
+        assert np.all(r["hq"][r["row_of_pair"][t]] == want[t][1])
+    assert np.all(r["s_x"] == 2.0 ** -9)
+    # closed form of the float result before the final rounding: y = +-3.5 * 9.37890625 * sigmoid(+-3.0625)
+    sig = lambda v: 1.0 / (1.0 + math.exp(-v))
+    for t in range(T):
+        s = 1.0 if t % 2 == 0 else -1.0
+        ref = s * 3.5 * 9.37890625 * sig(s * 3.0625)
+        assert np.allclose(r["out_f32"][t], ref, rtol=1e-6)
+
+
+def test_layer_single_expert_vs_fp64_mlp():
+    """E = 1, k = 1: the layer is one quantized SwiGLU MLP.  Compare with a textbook fp64
+    MLP on the dequantized weights and the unquantized input: the difference is the FP8
+    activation quantization error only (relative step 2^-4 per element, averaged)."""
+    rng = np.random.default_rng(6)
+    T, H, N = 24, 512, 256
+    def wts(rows, K):
+        return _f32_to_bf16_bits(rng.standard_normal((rows, K)).astype(np.float32) * 0.02)
+    Wg, Wu, Wd = wts(N, H), wts(N, H), wts(H, N)
+    pg, sg, cg = oracle.rtn_pack(Wg)
+    pu, su, cu = oracle.rtn_pack(Wu)
+    pd, sd, cd = oracle.rtn_pack(Wd)
+    layer = oracle.Layer(1, H, N, pg[None], pu[None], pd[None], sg[None], su[None], sd[None])
+    x = _f32_to_bf16_bits(rng.standard_normal((T, H)).astype(np.float32))
+    lg = np.zeros((T, 1), np.float32)
+    r = oracle.moe_forward(layer, x, lg, 1)
+    deq = lambda c, s: c.astype(np.float64) * np.repeat(oracle.bf16_to_f32(s).astype(np.float64), 128, 1)
+    Dg, Du, Dd = deq(cg, sg), deq(cu, su), deq(cd, sd)
+    xf = oracle.bf16_to_f32(x).astype(np.float64)
+    g = xf @ Dg.T
+    u = xf @ Du.T
+    h = g / (1 + np.exp(-g)) * u
+    ref = h @ Dd.T
+    got = r["out_f32"].astype(np.float64)
+    rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
+    assert rel < 0.05, rel
+    assert np.corrcoef(got.ravel(), ref.ravel())[0, 1] > 0.998
+    # a wrong sign of the SwiGLU or a transposed weight would be far outside this band
+    assert r["gates"].min() == 1.0
+
+
+def test_layer_empty_batch():
+    wl = synth.WORKLOADS["tiny"]
+    layer = _tiny_layer(wl)
+    r = oracle.moe_forward(layer, np.zeros((0, wl.H), np.uint16), np.zeros((0, wl.E), np.float32),
+                           wl.k)
+    assert r["out"].shape == (0, wl.H)
+    assert np.all(r["offsets"] == 0)
+
+
+# ------------------------------------------------------------------------------------------------
+# the generator (input recipe)
+# ------------------------------------------------------------------------------------------------
+
+def test_generator_moments_and_determinism():
+    a = synth.normal_f32(0, 77, 2_000_000)
+    b = synth.normal_f32(0, 77, 1000, start=500)
+    assert np.array_equal(a[500:1500], b)
+    assert abs(a.mean()) < 3e-3 and abs(a.std() - 1) < 3e-3
+    assert abs((a.astype(np.float64) ** 4).mean() - 3) < 0.03
+    assert not np.array_equal(a[:100], synth.normal_f32(1, 77, 100))
+
+
+def test_workload_recipe():
+    wl = synth.WORKLOADS["decode_t8"]
+    m = synth.outlier_mask(wl)
+    assert int(m.sum()) == 41
+    x = oracle.bf16_to_f32(synth.tokens(wl))
+    assert x.shape == (8, 4096)
+    assert np.abs(x[:, m == 1]).mean() > 10 * np.abs(x[:, m == 0]).mean()
+    z = synth.WORKLOADS["prefill_t2048_zipf"]
+    ranks = synth.expert_ranks(z)
+    assert sorted(ranks.tolist()) == list(range(1, 257))
+    b = synth.logit_bias(z)
+    assert np.allclose(b, -1.1 * np.log(ranks), rtol=0, atol=1e-12)
