@@ -1,0 +1,349 @@
+"""Throughput of the W4A8-FP8 routed MoE layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one moe_w4a8_forward over a T-token batch (routing, FP8 quantization, grouped
+gate/up GEMM, SwiGLU requantization, grouped down GEMM, shared experts if any, combine), with
+inputs already in HBM.  Batches rotate over 8 distinct seeded token sets, so the experts a
+step touches change from step to step; the touched expert weights of one step (~0.57 GB at
+T=8) already exceed the 126 MB L2.  Ranks (torchrun) are independent replicas, each with its
+own batches: weak scaling, no data-path collective.
+
+`--impl reference` times the CPU oracle on the host cores instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "MoE-layer tokens/s; % HBM roofline (decode) / % FP8 TC peak (prefill)"
+DEFAULT_WORKLOAD = "decode_t8"
+N_BATCHES = 8
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def expert_bytes(wl):
+    """Algorithmic bytes of one routed expert: packed INT4 codes + bf16 group scales."""
+    gate = wl.N * wl.H // 2 + wl.N * (wl.H // wl.group) * 2
+    down = wl.H * wl.N // 2 + wl.H * (wl.N // wl.group) * 2
+    return 2 * gate, down            # (gate+up, down)
+
+
+def flops_per_pair(wl):
+    return 2 * wl.H * 2 * wl.N + 2 * wl.N * wl.H
+
+
+def peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.idx = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out = ""
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+# ------------------------------------------------------------------------------------------------
+# our implementation
+# ------------------------------------------------------------------------------------------------
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    import bit_quantized_moe_token_b200 as moe
+    from bit_quantized_moe_token_b200.synthetic import device_inputs, device_layer
+
+    world, rank, local = dist_setup()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    wl = synth.WORKLOADS[args.workload]
+    layer = device_layer(wl, device=dev)
+    if not wl.n_shared:
+        layer.sh_gate = layer.sh_up = layer.sh_down = None
+    T, k = wl.T, wl.k
+    batches = []
+    for b in range(N_BATCHES):
+        t0 = (rank * N_BATCHES + b) * T
+        batches.append(device_inputs(wl, device=dev, t0=t0, T=T))
+    out = torch.empty(T, wl.H, dtype=torch.bfloat16, device=dev)
+    ws = moe.alloc_workspace(layer, T, k, dev)
+    stream = torch.cuda.current_stream(dev)
+
+    # touched experts per batch (for the algorithmic byte count), from the routing outputs
+    lay = moe.moe_w4a8_workspace_layout(layer, T, k)
+    touched = []
+    for x, lg in batches:
+        moe.forward(layer, x, lg, k, out=out, ws=ws)
+        offs = ws[lay["expert_offsets"]:lay["expert_offsets"] + 4 * (wl.E + 1)].view(torch.int32)
+        touched.append(int((offs[1:] - offs[:-1] > 0).sum().item()))
+    torch.cuda.synchronize()
+    if moe.moe_last_device_status() != 0:
+        raise RuntimeError("device status: timeout during warm-up")
+
+    for i in range(args.warmup):
+        x, lg = batches[i % N_BATCHES]
+        moe.forward(layer, x, lg, k, out=out, ws=ws)
+    torch.cuda.synchronize()
+
+    # ---- device-timed region ----
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(moe.N_STAGE_EVENTS)]
+          for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches = 0
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        start.record(stream)
+        for i in range(args.steps):
+            x, lg = batches[i % N_BATCHES]
+            launches += moe.moe_w4a8_forward_profiled(layer, x, lg, k, out, ws, ev[i])
+        end.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    total_ms = start.elapsed_time(end)
+    if moe.moe_last_device_status() != 0:
+        raise RuntimeError("device status: timeout in the timed region")
+    stage_ms = {s: 0.0 for s in moe.STAGES}
+    for i in range(args.steps):
+        for j, s in enumerate(moe.STAGES):
+            stage_ms[s] += ev[i][j].elapsed_time(ev[i][j + 1]) / args.steps
+    t_max = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
+    total_ms = float(t_max.item())
+
+    # ---- end to end through the public API with host buffers ----
+    hx = [b[0].cpu().pin_memory() for b in batches]
+    hl = [b[1].cpu().pin_memory() for b in batches]
+    hout = torch.empty(T, wl.H, dtype=torch.bfloat16).pin_memory()
+    dx = torch.empty_like(batches[0][0])
+    dl = torch.empty_like(batches[0][1])
+    for i in range(2):
+        dx.copy_(hx[i], non_blocking=True)
+        dl.copy_(hl[i], non_blocking=True)
+        moe.moe_w4a8_forward(layer, dx, dl, k, out, ws)
+        hout.copy_(out, non_blocking=True)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for i in range(args.steps):
+        dx.copy_(hx[i % N_BATCHES], non_blocking=True)
+        dl.copy_(hl[i % N_BATCHES], non_blocking=True)
+        moe.moe_w4a8_forward(layer, dx, dl, k, out, ws)
+        hout.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+    e2e_ms = float(e2e_ms.item())
+
+    tokens = world * T * args.steps
+    value = tokens / (total_ms / 1e3)
+    hbm, bf16, peak_kind = peaks()
+    gu_bytes, down_bytes = expert_bytes(wl)
+    mean_touched = sum(touched[i % N_BATCHES] for i in range(args.steps)) / args.steps
+    dom = "gateup_gemm"
+    dom_ms = stage_ms[dom]
+    dom_bytes = mean_touched * gu_bytes
+    achieved = dom_bytes / (dom_ms / 1e3) / 1e9
+    roofline = {"bound": "hbm", "kernel": "grouped gate/up W4A8 GEMM (stage)",
+                "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                "frac": round(achieved / hbm, 4), "traffic": None,
+                "peak_source": f"{peak_kind} hbm_gbs",
+                "algorithmic_bytes_per_launch": int(dom_bytes),
+                "units": f"{mean_touched:.1f} touched experts x {gu_bytes} B (gate+up codes+scales)"}
+    layer_bytes = mean_touched * (gu_bytes + down_bytes)
+    result = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3 x int4 -> f32", "data": "synthetic",
+        "config": {"workload": wl.name, "T": T, "H": wl.H, "N": wl.N, "E": wl.E, "k": k,
+                   "routing": wl.routing, "n_shared": wl.n_shared, "seed": wl.seed,
+                   "batches": N_BATCHES, "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2: touched expert weights per step "
+                         f"{layer_bytes / 1e9:.2f} GB vs 126 MB L2; {N_BATCHES} rotating batches"},
+        "layer_hbm_gbs": round(layer_bytes / (total_ms / args.steps / 1e3) / 1e9, 1),
+        "roofline": roofline,
+        "stages_ms": {s: round(v, 4) for s, v in stage_ms.items()},
+        "gpu_launches": launches,
+        "e2e": {"value": round(tokens / (e2e_ms / 1e3), 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": T * wl.H * 2 + T * wl.E * 4,
+                "d2h_bytes_per_step": T * wl.H * 2},
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(wl, batches_t0=0)
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
+# ------------------------------------------------------------------------------------------------
+# the CPU oracle
+# ------------------------------------------------------------------------------------------------
+
+def oracle_sample(wl, t0, max_tokens):
+    """A bounded sample of the workload for the CPU oracle: the first tokens of one batch,
+    with the experts they route to packed (untimed setup)."""
+    import oracle
+    n = min(wl.T, max_tokens)
+    x = synth.tokens(wl, t0, n)
+    lg = synth.logits(wl, t0, n)
+    ids, _ = oracle.route_topk(lg, wl.k)
+    layer = oracle.pack_workload_layer(wl, experts=sorted(set(ids.reshape(-1).tolist())))
+    return layer, x, lg, n
+
+
+def cores_used():
+    try:
+        return int(os.environ.get("OMP_NUM_THREADS") or len(os.sched_getaffinity(0)))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(wl, batches_t0=0, max_tokens=8):
+    import oracle
+    layer, x, lg, n = oracle_sample(wl, batches_t0, max_tokens)
+    t = time.perf_counter()
+    oracle.moe_forward(layer, x, lg, wl.k)
+    dt = time.perf_counter() - t
+    return {"value": round(n / dt, 3), "unit": "tokens/s", "cores": cores_used(), "kind": "oracle",
+            "sample": f"{n} tokens of {wl.name} (one forward of the C oracle, fp32, OpenMP over "
+                      f"experts), {dt:.2f} s"}
+
+
+def run_reference(args):
+    world, rank, _ = dist_setup()
+    if rank != 0:
+        return
+    import oracle
+    wl = synth.WORKLOADS[args.workload]
+    layer, x, lg, n = oracle_sample(wl, 0, args.ref_tokens)
+    for _ in range(args.warmup):
+        oracle.moe_forward(layer, x, lg, wl.k)
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.moe_forward(layer, x, lg, wl.k)
+    dt = time.perf_counter() - t
+    value = n * args.steps / dt
+    result = {
+        "metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic", "impl": "reference",
+        "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "N": wl.N, "E": wl.E, "k": wl.k,
+                   "routing": wl.routing, "n_shared": wl.n_shared, "seed": wl.seed,
+                   "parallelism": "host cores"},
+        "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": cores_used(),
+                         "kind": "oracle",
+                         "sample": f"{n} tokens of {wl.name} per step (C oracle, fp32)"},
+        "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(result), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--ref-tokens", type=int, default=8)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,232 @@
+"""ctypes binding of libmoe_w4a8.so — argument marshalling only.
+
+Every function has the name of the C entry point it calls.  Tensors are torch CUDA tensors;
+their data pointers go straight to the library, which runs every step on the GPU.  There is
+no CPU or PyTorch fallback: if the library cannot be loaded, the import fails.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+from . import build as _build
+
+MOE_OK = 0
+STATUS = {0: "MOE_OK", -1: "MOE_ERR_INVALID_ARG", -2: "MOE_ERR_UNSUPPORTED_SHAPE",
+          -3: "MOE_ERR_MISALIGNED", -4: "MOE_ERR_WORKSPACE", -5: "MOE_ERR_CUDA",
+          -6: "MOE_ERR_TIMEOUT", -7: "MOE_ERR_NO_DEVICE"}
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)} ({moe_status_string(status)})")
+
+
+class _CLayer(ctypes.Structure):
+    _fields_ = [("E", ctypes.c_int), ("H", ctypes.c_int), ("N", ctypes.c_int),
+                ("group", ctypes.c_int),
+                ("gate_packed", ctypes.c_void_p), ("up_packed", ctypes.c_void_p),
+                ("down_packed", ctypes.c_void_p),
+                ("gate_scales", ctypes.c_void_p), ("up_scales", ctypes.c_void_p),
+                ("down_scales", ctypes.c_void_p),
+                ("n_shared", ctypes.c_int), ("shared_N", ctypes.c_int),
+                ("sh_gate", ctypes.c_void_p), ("sh_up", ctypes.c_void_p),
+                ("sh_down", ctypes.c_void_p)]
+
+
+class _CLayout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_size_t) for n in
+                ("topk_ids", "topk_w", "expert_offsets", "sorted_pairs", "row_of_pair",
+                 "x_sorted", "s_x_sorted", "hq", "s_h", "total")]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load (building first if the sources are newer) libmoe_w4a8.so."""
+    global _lib
+    if _lib is None:
+        path = _build.LIB
+        try:
+            if _build.stale():
+                _build.build()
+        except Exception:
+            if not os.path.exists(path):
+                raise
+        L = ctypes.CDLL(path)
+        vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+        L.w4a8_pack_weights.argtypes = [vp, i64, i64, i32, vp, vp, vp]
+        L.fp8_quant_tokens.argtypes = [vp, i64, i64, vp, vp, vp]
+        L.moe_route_workspace_bytes.argtypes = [i64, i32, i32]
+        L.moe_route_workspace_bytes.restype = sz
+        L.moe_route_topk.argtypes = [vp, i64, i32, i32, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.moe_w4a8_workspace_bytes.argtypes = [ctypes.POINTER(_CLayer), i64, i32]
+        L.moe_w4a8_workspace_bytes.restype = sz
+        L.moe_w4a8_workspace_layout.argtypes = [ctypes.POINTER(_CLayer), i64, i32,
+                                                ctypes.POINTER(_CLayout)]
+        L.moe_w4a8_forward.argtypes = [ctypes.POINTER(_CLayer), vp, vp, i64, i32, vp, vp, sz, vp]
+        L.moe_w4a8_forward_profiled.argtypes = [ctypes.POINTER(_CLayer), vp, vp, i64, i32, vp, vp,
+                                                sz, vp, vp, i32, ctypes.POINTER(ctypes.c_int)]
+        L.moe_last_device_status.argtypes = [vp]
+        L.moe_status_string.argtypes = [i32]
+        L.moe_status_string.restype = ctypes.c_char_p
+        for f in (L.w4a8_pack_weights, L.fp8_quant_tokens, L.moe_route_topk,
+                  L.moe_w4a8_workspace_layout, L.moe_w4a8_forward, L.moe_w4a8_forward_profiled,
+                  L.moe_last_device_status):
+            f.restype = i32
+        _lib = L
+    return _lib
+
+
+def moe_status_string(status: int) -> str:
+    return lib().moe_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != MOE_OK:
+        raise MoeError(status, where)
+
+
+def _ptr(t) -> Optional[ctypes.c_void_p]:
+    """Device pointer of a torch tensor (or pass an int / None through)."""
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return ctypes.c_void_p(t)
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+# ----------------------------------------------------------------------------------------------
+# entry points
+# ----------------------------------------------------------------------------------------------
+
+def w4a8_pack_weights(w, packed, scales, group: int = 128, stream=None) -> None:
+    """w bf16 [rows, K] -> packed int32 [rows, K/8], scales bf16 [rows, K/group]."""
+    rows, K = w.shape[-2] if w.dim() > 1 else 1, w.shape[-1]
+    rows = w.numel() // K
+    _check(lib().w4a8_pack_weights(_ptr(w), rows, K, group, _ptr(packed), _ptr(scales),
+                                   _stream(stream)), "w4a8_pack_weights")
+
+
+def fp8_quant_tokens(x, q, scale, stream=None) -> None:
+    """x bf16 [T, H] -> q uint8 (E4M3 codes) [T, H], scale fp32 [T]."""
+    T, H = x.shape
+    _check(lib().fp8_quant_tokens(_ptr(x), T, H, _ptr(q), _ptr(scale), _stream(stream)),
+           "fp8_quant_tokens")
+
+
+def moe_route_workspace_bytes(T: int, E: int, k: int) -> int:
+    return int(lib().moe_route_workspace_bytes(T, E, k))
+
+
+def moe_route_topk(logits, k: int, topk_ids, topk_w, expert_offsets, sorted_pairs, row_of_pair,
+                   ws, stream=None) -> None:
+    T, E = logits.shape
+    nbytes = ws.numel() * ws.element_size() if ws is not None else 0
+    _check(lib().moe_route_topk(_ptr(logits), T, E, k, _ptr(topk_ids), _ptr(topk_w),
+                                _ptr(expert_offsets), _ptr(sorted_pairs), _ptr(row_of_pair),
+                                _ptr(ws), nbytes, _stream(stream)), "moe_route_topk")
+
+
+@dataclass
+class Layer:
+    """Device tensors of one layer (see moe_w4a8_layer in include/moe_w4a8.h)."""
+    E: int
+    H: int
+    N: int
+    gate_packed: object
+    up_packed: object
+    down_packed: object
+    gate_scales: object
+    up_scales: object
+    down_scales: object
+    group: int = 128
+    sh_gate: object = None
+    sh_up: object = None
+    sh_down: object = None
+
+    @property
+    def n_shared(self) -> int:
+        return 0 if self.sh_gate is None else int(self.sh_gate.shape[0])
+
+    @property
+    def shared_N(self) -> int:
+        return 0 if self.sh_gate is None else int(self.sh_gate.shape[1])
+
+    def c_struct(self) -> _CLayer:
+        return _CLayer(self.E, self.H, self.N, self.group,
+                       _ptr(self.gate_packed), _ptr(self.up_packed), _ptr(self.down_packed),
+                       _ptr(self.gate_scales), _ptr(self.up_scales), _ptr(self.down_scales),
+                       self.n_shared, self.shared_N,
+                       _ptr(self.sh_gate), _ptr(self.sh_up), _ptr(self.sh_down))
+
+    def shape_struct(self) -> _CLayer:
+        """The same struct with null pointers: enough for the size/layout queries."""
+        return _CLayer(self.E, self.H, self.N, self.group, None, None, None, None, None, None,
+                       self.n_shared, self.shared_N, None, None, None)
+
+
+def layer_struct(E, H, N, group=128, n_shared=0, shared_N=0) -> _CLayer:
+    return _CLayer(E, H, N, group, None, None, None, None, None, None, n_shared, shared_N,
+                   None, None, None)
+
+
+def moe_w4a8_workspace_bytes(layer, T: int, k: int) -> int:
+    s = layer if isinstance(layer, _CLayer) else layer.shape_struct()
+    return int(lib().moe_w4a8_workspace_bytes(ctypes.byref(s), T, k))
+
+
+def moe_w4a8_workspace_layout(layer, T: int, k: int) -> dict:
+    s = layer if isinstance(layer, _CLayer) else layer.shape_struct()
+    out = _CLayout()
+    _check(lib().moe_w4a8_workspace_layout(ctypes.byref(s), T, k, ctypes.byref(out)),
+           "moe_w4a8_workspace_layout")
+    return {n: int(getattr(out, n)) for n, _ in _CLayout._fields_}
+
+
+def moe_w4a8_forward(layer: Layer, x, logits, k: int, out, ws, stream=None) -> None:
+    """out bf16 [T, H] = the routed W4A8 MoE layer (+ shared experts) applied to x."""
+    T = x.shape[0]
+    s = layer.c_struct()
+    nbytes = ws.numel() * ws.element_size() if ws is not None else 0
+    _check(lib().moe_w4a8_forward(ctypes.byref(s), _ptr(x), _ptr(logits), T, k, _ptr(out),
+                                  _ptr(ws), nbytes, _stream(stream)), "moe_w4a8_forward")
+
+
+N_STAGE_EVENTS = 8
+STAGES = ("route", "quant", "gateup_gemm", "swiglu_requant", "down_gemm", "shared", "combine")
+
+
+def moe_w4a8_forward_profiled(layer: Layer, x, logits, k: int, out, ws, events, stream=None) -> int:
+    """moe_w4a8_forward that also records `events` (8 torch.cuda.Event with timing) at the stage
+    boundaries; returns the number of kernels launched."""
+    T = x.shape[0]
+    s = layer.c_struct()
+    nbytes = ws.numel() * ws.element_size() if ws is not None else 0
+    arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    n = ctypes.c_int(0)
+    _check(lib().moe_w4a8_forward_profiled(ctypes.byref(s), _ptr(x), _ptr(logits), T, k, _ptr(out),
+                                           _ptr(ws), nbytes, _stream(stream), arr, len(events),
+                                           ctypes.byref(n)), "moe_w4a8_forward_profiled")
+    return int(n.value)
+
+
+def moe_last_device_status(stream=None) -> int:
+    return int(lib().moe_last_device_status(_stream(stream)))

@@ -1,0 +1,63 @@
+// common.cuh — small device helpers shared by the kernels of libmoe_w4a8.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <stdint.h>
+
+#include "moe_w4a8.h"
+
+namespace moe {
+
+constexpr int kGroup = 128;   // K-group of the INT4 scales
+constexpr float kFp8Max = 448.0f;
+
+// ---- host-side argument checks ---------------------------------------------------------------
+
+inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+inline int launch_status() {
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// ---- conversions -------------------------------------------------------------------------------
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint16_t h) {
+    return __uint_as_float(static_cast<uint32_t>(h) << 16);
+}
+
+// Round to nearest even, subnormals kept (hardware cvt.rn.bf16.f32).
+__device__ __forceinline__ uint16_t f32_to_bf16_bits(float f) {
+    __nv_bfloat16 b = __float2bfloat16_rn(f);
+    return *reinterpret_cast<uint16_t*>(&b);
+}
+
+// Two floats -> two E4M3 bytes, round to nearest even with saturation to +-448 (the
+// hardware cvt.rn.satfinite.e4m3x2.f32).  Byte 0 holds `lo`.
+__device__ __forceinline__ uint16_t f32x2_to_e4m3x2(float lo, float hi) {
+    __nv_fp8x2_storage_t r = __nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3);
+    return static_cast<uint16_t>(r);
+}
+
+// E4M3 byte -> float (exact).
+__device__ __forceinline__ float e4m3_to_f32(uint8_t c) {
+    __half_raw h = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(c), __NV_E4M3);
+    return __half2float(*reinterpret_cast<__half*>(&h));
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+__device__ __forceinline__ float silu(float g) {
+    // g * sigmoid(g) with IEEE division; expf is CUDA's (max 2 ulp).
+    return g * __fdiv_rn(1.0f, 1.0f + expf(-g));
+}
+
+}  // namespace moe

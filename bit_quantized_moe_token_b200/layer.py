@@ -1,0 +1,44 @@
+"""Convenience wrappers: torch allocation around the C entry points."""
+from __future__ import annotations
+
+from ._binding import (Layer, moe_w4a8_forward, moe_w4a8_workspace_bytes, w4a8_pack_weights)
+
+
+def pack_expert_weights(w, group: int = 128, stream=None):
+    """bf16 weights [..., rows, K] on the GPU -> (int32 packed [..., rows, K/8],
+    bf16 scales [..., rows, K/group]) in pack-quantized storage."""
+    import torch
+    *lead, rows, K = w.shape
+    packed = torch.empty(*lead, rows, K // 8, dtype=torch.int32, device=w.device)
+    scales = torch.empty(*lead, rows, K // group, dtype=torch.bfloat16, device=w.device)
+    w4a8_pack_weights(w.contiguous(), packed, scales, group=group, stream=stream)
+    return packed, scales
+
+
+def make_layer(gate_w, up_w, down_w, sh_gate=None, sh_up=None, sh_down=None,
+               stream=None) -> Layer:
+    """Quantize and pack bf16 expert weights gate/up [E, N, H], down [E, H, N]."""
+    E, N, H = gate_w.shape
+    gp, gs = pack_expert_weights(gate_w, stream=stream)
+    up, us = pack_expert_weights(up_w, stream=stream)
+    dp, ds = pack_expert_weights(down_w, stream=stream)
+    return Layer(E, H, N, gp, up, dp, gs, us, ds, sh_gate=sh_gate, sh_up=sh_up, sh_down=sh_down)
+
+
+def alloc_workspace(layer: Layer, T: int, k: int, device=None):
+    import torch
+    n = moe_w4a8_workspace_bytes(layer, T, k)
+    if n == 0 and T > 0:
+        raise ValueError("unsupported layer shape for moe_w4a8_forward")
+    dev = device if device is not None else layer.gate_packed.device
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=dev)
+
+
+def forward(layer: Layer, x, logits, k: int, out=None, ws=None, stream=None):
+    import torch
+    if out is None:
+        out = torch.empty_like(x)
+    if ws is None:
+        ws = alloc_workspace(layer, x.shape[0], k, x.device)
+    moe_w4a8_forward(layer, x, logits, k, out, ws, stream=stream)
+    return out

@@ -1,0 +1,191 @@
+/*
+ * moe_w4a8.h — C ABI of the B200 (sm_100a) W4A8-FP8 routed mixture-of-experts layer.
+ *
+ * The layer is the routed MoE block of an Inkling-class model whose experts are stored as
+ * symmetric INT4 weights in K-groups of 128 and run on FP8 E4M3 activations quantized per
+ * token ("Inkling-Small: GPTQ W4A8-FP8 creation and INT4 export recovery" model card,
+ * section 1 "What is being created?": "Symmetric INT4, groups of 128", "Dynamic FP8, token
+ * strategy"; W4A8-FP8 = four-bit integer weights with eight-bit floating-point input
+ * activations).  256 routed experts with 6 active per token and the gate|up / down expert
+ * projections come from the "Inkling-512k-NVFP4-AQLM-hybrid" model card (opening paragraph
+ * and "On-disk tensor format").
+ *
+ * Conventions for every call:
+ *   - All data pointers are DEVICE pointers owned by the caller (for example PyTorch
+ *     tensors).  The library never allocates, frees or synchronises inside a call, and keeps
+ *     no per-call host state, so calls can be captured in a CUDA graph.
+ *   - Work is enqueued on `stream` (NULL = legacy default stream) and runs asynchronously.
+ *     The return value reports argument validation and launch errors only; faults detected
+ *     on the device are reported by moe_last_device_status().
+ *   - bf16 values are passed as their 16-bit patterns (uint16_t), FP8 as E4M3 bytes
+ *     (uint8_t, OCP E4M3FN: bias 7, max 448, no infinities).
+ *   - Matrices are row-major with the last index contiguous.  Pointers to bf16 / fp8 /
+ *     int32 matrices must be 16-byte aligned; other pointers need their type's alignment.
+ *   - Calls on different streams are independent; a call does not touch memory it was not
+ *     given, except the library's sticky device-status word (see moe_last_device_status).
+ */
+#ifndef MOE_W4A8_H
+#define MOE_W4A8_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* The same type as cudaStream_t. */
+typedef struct CUstream_st* moe_stream_t;
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = -1,       /* null pointer, negative size, k outside [1, min(E, 8)] */
+    MOE_ERR_UNSUPPORTED_SHAPE = -2, /* a dimension the kernels do not cover (see each call) */
+    MOE_ERR_MISALIGNED = -3,        /* a pointer below its required alignment */
+    MOE_ERR_WORKSPACE = -4,         /* workspace missing or smaller than required */
+    MOE_ERR_CUDA = -5,              /* a CUDA runtime error at launch */
+    MOE_ERR_TIMEOUT = -6,           /* a bounded device-side wait gave up (device status) */
+    MOE_ERR_NO_DEVICE = -7          /* no sm_100 device current */
+} moe_status;
+
+/* ---------------------------------------------------------------------------------------
+ * S0. Offline weight quantization to pack-quantized INT4.
+ *
+ * Defined by the "Inkling-Small ... model card", section 1 ("Symmetric INT4, groups of 128")
+ * and section 7 "Recover and physically pack INT4" (codes in [-8,7] stored as the nibble
+ * code+8; eight consecutive codes along the last dimension in one little-endian I32 word,
+ * the first code in the least significant nibble; `.weight_packed` I32 of shape
+ * [rows, K/8]).  Scales are stored as bf16 [rows, K/group] (the export's non-I8 payload is
+ * BF16, section 5).  Per group of `group` consecutive K:
+ *     amax = max |w|,  scale = bf16_rn(amax / 7),  code = clamp(rint(w / scale), -8, 7)
+ * (round half to even; an all-zero group gets scale 0 and codes 0).
+ *
+ *   w_bf16      [rows, K] bf16 weights (out-features x in-features), 16-byte aligned
+ *   rows, K     rows >= 0; K a positive multiple of `group`
+ *   group       must be 128
+ *   packed      [rows, K/8] int32 output, 16-byte aligned
+ *   scales_bf16 [rows, K/group] bf16 output
+ * Returns MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED_SHAPE, MOE_ERR_MISALIGNED or
+ * MOE_ERR_CUDA.  rows == 0 is a no-op.
+ * --------------------------------------------------------------------------------------- */
+int w4a8_pack_weights(const uint16_t* w_bf16, int64_t rows, int64_t K, int group,
+                      int32_t* packed, uint16_t* scales_bf16, moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------
+ * S1. Dynamic per-token FP8 quantization ("Dynamic FP8, token strategy", section 1 of the
+ * Inkling-Small card).  For each row t:
+ *     amax = max |x[t,:]|,  scale[t] = amax / 448,  q[t,h] = e4m3_rn_satfinite(x[t,h] / scale[t])
+ * with IEEE fp32 division; a row with amax == 0 gets scale 0 and all-zero codes.
+ *
+ *   x_bf16  [T, H] bf16, 16-byte aligned;  H a positive multiple of 8, at most 65536
+ *   q_e4m3  [T, H] E4M3 output, 16-byte aligned
+ *   scale   [T] fp32 output
+ * T == 0 is a no-op.
+ * --------------------------------------------------------------------------------------- */
+int fp8_quant_tokens(const uint16_t* x_bf16, int64_t T, int64_t H, uint8_t* q_e4m3,
+                     float* scale, moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------
+ * S2 + S3. Top-k routing and the stable token permutation.
+ *
+ * Top-k of each row of the router logits ("256 routed experts/layer, 6 active",
+ * Inkling-512k card): experts are ranked by (logit descending, index ascending); the first
+ * k are the selection, in that order.  Gates are a softmax over the selected logits:
+ *     gate_j = exp(l_j - l_0) / sum_i exp(l_i - l_0)   (fp32, i, j < k).
+ * The routed pairs p = t*k + j are then grouped by expert into one contiguous segment per
+ * expert, segments in expert order, pairs ascending in p inside a segment:
+ *     expert_offsets[e] = number of pairs routed to experts < e   (expert_offsets[E] = T*k)
+ *     sorted_pairs[r]   = the pair at sorted row r;  row_of_pair[p] = its row.
+ *
+ *   logits          [T, E] fp32;  E in [1, 1024];  k in [1, min(E, 8)]
+ *   topk_ids        [T, k] int32 out      topk_w [T, k] fp32 out
+ *   expert_offsets  [E + 1] int32 out
+ *   sorted_pairs    [T*k] int32 out       row_of_pair [T*k] int32 out
+ *   ws, ws_bytes    device scratch of at least moe_route_workspace_bytes(T, E, k) bytes,
+ *                   256-byte aligned; contents on entry are ignored
+ * --------------------------------------------------------------------------------------- */
+size_t moe_route_workspace_bytes(int64_t T, int E, int k);
+int moe_route_topk(const float* logits, int64_t T, int E, int k, int32_t* topk_ids,
+                   float* topk_w, int32_t* expert_offsets, int32_t* sorted_pairs,
+                   int32_t* row_of_pair, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------
+ * S4..S8. The layer.
+ *
+ * Weights of the routed experts in the pack-quantized layout of w4a8_pack_weights, gate and
+ * up as separate projections (Inkling-Small card, section 6: the recovered checkpoint keeps
+ * separate gate/up projections), stacked over experts:
+ *   gate_packed, up_packed  [E, N, H/8] int32     gate_scales, up_scales  [E, N, H/128] bf16
+ *   down_packed             [E, H, N/8] int32     down_scales             [E, H, N/128] bf16
+ * Shared experts (always on, kept in bf16 — Inkling-Small card section 1: "retained
+ * multimodal/shared-expert parameters" stay BF16), n_shared may be 0 and the pointers NULL:
+ *   sh_gate, sh_up          [n_shared, shared_N, H] bf16
+ *   sh_down                 [n_shared, H, shared_N] bf16
+ * --------------------------------------------------------------------------------------- */
+typedef struct {
+    int E, H, N, group;
+    const int32_t *gate_packed, *up_packed, *down_packed;
+    const uint16_t *gate_scales, *up_scales, *down_scales;
+    int n_shared, shared_N;
+    const uint16_t *sh_gate, *sh_up, *sh_down;
+} moe_w4a8_layer;
+
+/* Bytes of device workspace moe_w4a8_forward needs for T tokens and top-k (0 on bad args). */
+size_t moe_w4a8_workspace_bytes(const moe_w4a8_layer* layer, int64_t T, int k);
+
+/* Byte offsets, inside the forward workspace, of the intermediates a caller may inspect
+ * after the forward completes (all in expert-sorted row order r, P = T*k rows):
+ *   topk_ids [T,k] i32, topk_w [T,k] f32, expert_offsets [E+1] i32, sorted_pairs [P] i32,
+ *   row_of_pair [P] i32, x_sorted [P,H] e4m3 (token codes of the row's token), s_x_sorted [P]
+ *   f32, hq [P,N] e4m3 (requantized SwiGLU activations), s_h [P] f32. */
+typedef struct {
+    size_t topk_ids, topk_w, expert_offsets, sorted_pairs, row_of_pair;
+    size_t x_sorted, s_x_sorted, hq, s_h;
+    size_t total;
+} moe_w4a8_ws_layout;
+int moe_w4a8_workspace_layout(const moe_w4a8_layer* layer, int64_t T, int k,
+                              moe_w4a8_ws_layout* out);
+
+/*
+ * out[t,:] = bf16_rn( sum_{j<k} gate[t,j] * Y[(t,j),:]  +  sum_s shared_s(x[t,:]) ) with, for
+ * the pair (t,j) routed to expert e:
+ *   G[n] = s_x[t] * sum_g s_gate[e,n,g] * sum_{k in g} Xq[t,k] * Cgate[e,n,k]   (likewise U)
+ *   h    = silu(G) * U;   s_h = max|h| / 448;   Hq = e4m3(h / s_h)
+ *   Y[m] = s_h * sum_g s_down[e,m,g] * sum_{k in g} Hq[k] * Cdown[e,m,k]
+ * (Xq, s_x from S1; the routing and permutation of S2/S3).
+ *
+ *   x_bf16         [T, H] bf16 hidden states        router_logits [T, E] fp32
+ *   out_bf16       [T, H] bf16 output
+ *   ws, ws_bytes   device scratch, >= moe_w4a8_workspace_bytes(layer, T, k), 256-byte aligned
+ * Supported shapes: H and N multiples of 128 (H <= 16384, N <= 8192), group 128, E <= 1024,
+ * 1 <= k <= min(E, 8), shared_N a multiple of 128.  T == 0 is a no-op.
+ */
+int moe_w4a8_forward(const moe_w4a8_layer* layer, const uint16_t* x_bf16,
+                     const float* router_logits, int64_t T, int k, uint16_t* out_bf16, void* ws,
+                     size_t ws_bytes, moe_stream_t stream);
+
+/* Profiling variant of moe_w4a8_forward: the same work, plus `events[i]` (caller-created
+ * cudaEvent_t handles, n_events >= MOE_W4A8_N_STAGE_EVENTS) recorded on `stream` at the stage
+ * boundaries below, and the number of kernels the call launched in *n_launches (may be NULL).
+ *   0 start  1 routed (top-k + permutation)  2 tokens quantized  3 gate/up GEMM done
+ *   4 SwiGLU requant done  5 down GEMM done  6 shared experts done  7 combined (end) */
+#define MOE_W4A8_N_STAGE_EVENTS 8
+int moe_w4a8_forward_profiled(const moe_w4a8_layer* layer, const uint16_t* x_bf16,
+                              const float* router_logits, int64_t T, int k, uint16_t* out_bf16,
+                              void* ws, size_t ws_bytes, moe_stream_t stream,
+                              void* const* events, int n_events, int* n_launches);
+
+/* Waits for `stream`, then returns and clears the library's sticky device-status word for
+ * the current device: MOE_OK, or MOE_ERR_TIMEOUT when a bounded device-side wait gave up
+ * (its kernel then skipped the rest of its work and returned), or MOE_ERR_CUDA when the
+ * stream itself reports an error. */
+int moe_last_device_status(moe_stream_t stream);
+
+/* Static description of a status code. */
+const char* moe_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_W4A8_H */

@@ -1,0 +1,47 @@
+"""The layer's three parity rules, as reusable checks.
+
+1. Routing indices, permutation, packed codes, and first-stage FP8 codes and scales:
+   bit-exact.
+2. Intermediate FP8 codes (the requantized SwiGLU activations): at most 0.1% differ, and
+   those by at most one E4M3 step.
+3. Each bf16 output element within 1e-2 * max(|ref|, rms(ref row)).
+
+Where fp32 arithmetic decides an integer (an FP8 code after a GPU sum with a different
+accumulation order than the oracle's), rule 2 is what allows the difference.
+"""
+import numpy as np
+
+OUT_RTOL = 1e-2
+HQ_MAX_FRACTION = 1e-3
+
+
+def e4m3_ordinal(c: np.ndarray) -> np.ndarray:
+    """Monotone integer position of an E4M3 code (+0 and -0 both 0)."""
+    c = np.asarray(c, np.int32)
+    mag = c & 0x7F
+    return np.where(c & 0x80, -mag, mag)
+
+
+def check_fp8_codes(got: np.ndarray, want: np.ndarray, max_fraction=HQ_MAX_FRACTION):
+    d = np.abs(e4m3_ordinal(got) - e4m3_ordinal(want))
+    n_diff = int((d != 0).sum())
+    frac = n_diff / max(d.size, 1)
+    assert d.max(initial=0) <= 1, f"an FP8 code differs by {d.max()} steps"
+    assert frac <= max_fraction, f"{n_diff} of {d.size} FP8 codes differ ({frac:.2e})"
+    return n_diff, frac
+
+
+def bf16_to_f32(h: np.ndarray) -> np.ndarray:
+    return (np.asarray(h, np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+def check_output(got_bf16: np.ndarray, ref_bf16: np.ndarray, rtol=OUT_RTOL):
+    g = bf16_to_f32(got_bf16).astype(np.float64)
+    r = bf16_to_f32(ref_bf16).astype(np.float64)
+    rms = np.sqrt((r ** 2).mean(axis=1, keepdims=True))
+    tol = rtol * np.maximum(np.abs(r), rms)
+    err = np.abs(g - r)
+    bad = err > tol
+    assert not bad.any(), (f"{int(bad.sum())} outputs out of tolerance; worst "
+                           f"{float((err / np.maximum(tol, 1e-30)).max()):.3f}x tol")
+    return float((err / np.maximum(np.maximum(np.abs(r), rms), 1e-30)).max())

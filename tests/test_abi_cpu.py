@@ -1,0 +1,123 @@
+"""Host-side checks of the C ABI: the library loads, exports every declared entry point, and
+rejects bad arguments before touching the GPU (no compute call is made here)."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+import bit_quantized_moe_token_b200 as moe
+from conftest import ROOT
+
+
+def _declared_functions():
+    names = []
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        for m in re.finditer(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b([a-z_][a-z0-9_]*)\s*\(", src,
+                             flags=re.M):
+            name = m.group(1)
+            if name not in ("if", "while", "for", "sizeof"):
+                names.append(name)
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for n in ("w4a8_pack_weights", "fp8_quant_tokens", "moe_route_topk", "moe_w4a8_forward",
+              "moe_w4a8_workspace_bytes", "moe_last_device_status", "moe_status_string"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    L = moe.lib()
+    for n in _declared_functions():
+        assert hasattr(L, n), n
+        assert ctypes.cast(getattr(L, n), ctypes.c_void_p).value
+
+
+def test_status_strings():
+    assert moe.moe_status_string(0) == "ok"
+    assert "workspace" in moe.moe_status_string(-4)
+    assert moe.moe_status_string(12345) == "unknown status"
+
+
+def _L():
+    return moe.lib()
+
+
+def test_pack_rejects_bad_args():
+    L = _L()
+    p = ctypes.c_void_p(4096)
+    assert L.w4a8_pack_weights(p, 10, 100, 128, p, p, None) == -2      # K not multiple of 128
+    assert L.w4a8_pack_weights(p, 10, 256, 64, p, p, None) == -2       # group != 128
+    assert L.w4a8_pack_weights(p, -1, 256, 128, p, p, None) == -1
+    assert L.w4a8_pack_weights(None, 10, 256, 128, p, p, None) == -1
+    assert L.w4a8_pack_weights(ctypes.c_void_p(4100), 10, 256, 128, p, p, None) == -3
+    assert L.w4a8_pack_weights(p, 0, 256, 128, p, p, None) == 0          # no-op
+
+
+def test_quant_rejects_bad_args():
+    L = _L()
+    p = ctypes.c_void_p(4096)
+    assert L.fp8_quant_tokens(p, 4, 12, p, p, None) == -2                # H % 8
+    assert L.fp8_quant_tokens(None, 4, 16, p, p, None) == -1
+    assert L.fp8_quant_tokens(ctypes.c_void_p(4104), 4, 16, p, p, None) == -3
+    assert L.fp8_quant_tokens(p, 0, 16, p, p, None) == 0
+
+
+def test_route_rejects_bad_args():
+    L = _L()
+    p = ctypes.c_void_p(4096)
+    ws = moe.moe_route_workspace_bytes(64, 256, 6)
+    assert ws >= 256 and ws % 256 == 0
+    assert moe.moe_route_workspace_bytes(64, 256, 9) == 0                # k > 8
+    assert L.moe_route_topk(p, 64, 256, 9, p, p, p, p, p, p, ws, None) == -2
+    assert L.moe_route_topk(p, 64, 4, 6, p, p, p, p, p, p, ws, None) == -2   # k > E
+    assert L.moe_route_topk(p, 64, 2048, 6, p, p, p, p, p, p, ws, None) == -2
+    assert L.moe_route_topk(p, 64, 256, 6, p, p, p, p, p, p, ws - 1, None) == -4
+    assert L.moe_route_topk(p, 64, 256, 6, p, p, p, p, p, None, ws, None) == -4
+    assert L.moe_route_topk(p, 64, 256, 6, p, p, p, p, p, ctypes.c_void_p(4096 + 16), ws, None) == -3
+    assert L.moe_route_topk(None, 64, 256, 6, p, p, p, p, p, p, ws, None) == -1
+
+
+def test_forward_workspace_and_layout():
+    s = moe.layer_struct(256, 4096, 2048)
+    n8 = moe.moe_w4a8_workspace_bytes(s, 8, 6)
+    n64 = moe.moe_w4a8_workspace_bytes(s, 64, 6)
+    assert 0 < n8 < n64
+    lay = moe.moe_w4a8_workspace_layout(s, 8, 6)
+    assert lay["total"] == n8
+    offs = [lay[k] for k in ("topk_ids", "topk_w", "expert_offsets", "sorted_pairs", "row_of_pair",
+                             "x_sorted", "s_x_sorted", "hq", "s_h")]
+    assert all(o % 256 == 0 for o in offs) and len(set(offs)) == len(offs)
+    assert max(offs) < n8
+    assert moe.moe_w4a8_workspace_bytes(moe.layer_struct(256, 4000, 2048), 8, 6) == 0  # H % 128
+    assert moe.moe_w4a8_workspace_bytes(moe.layer_struct(256, 4096, 2048, group=64), 8, 6) == 0
+    shared = moe.layer_struct(256, 4096, 2048, n_shared=2, shared_N=2048)
+    assert moe.moe_w4a8_workspace_bytes(shared, 8, 6) > n8
+
+
+def test_forward_rejects_bad_args():
+    L = _L()
+    s = moe.layer_struct(8, 256, 128)
+    p = ctypes.c_void_p(4096)
+    # null weights
+    assert L.moe_w4a8_forward(ctypes.byref(s), p, p, 4, 2, p, p, 1 << 20, None) == -1
+    full = moe._binding._CLayer(8, 256, 128, 128, p, p, p, p, p, p, 0, 0, None, None, None)
+    need = moe.moe_w4a8_workspace_bytes(full, 4, 2)
+    assert L.moe_w4a8_forward(ctypes.byref(full), p, p, 4, 2, p, p, need - 1, None) == -4
+    assert L.moe_w4a8_forward(ctypes.byref(full), p, p, 4, 2, p, ctypes.c_void_p(4096 + 128),
+                              need, None) == -3
+    assert L.moe_w4a8_forward(ctypes.byref(full), p, p, 4, 0, p, p, need, None) == -1
+    assert L.moe_w4a8_forward(ctypes.byref(full), p, p, 0, 2, p, p, need, None) == 0
+    assert L.moe_w4a8_forward(None, p, p, 4, 2, p, p, need, None) == -1
+
+
+def test_binding_has_no_fallback():
+    src = open(os.path.join(ROOT, "bit_quantized_moe_token_b200", "_binding.py")).read()
+    assert "oracle" not in src and "numpy" not in src
+    for f in glob.glob(os.path.join(ROOT, "bit_quantized_moe_token_b200", "*.py")):
+        assert "import oracle" not in open(f).read(), f

@@ -1,0 +1,323 @@
+"""GPU parity: every entry point of libmoe_w4a8 (called through the C ABI) against the CPU
+oracle on the same seeded inputs, under the layer's three rules (tests/parity.py)."""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from conftest import cuda_ok
+from parity import bf16_to_f32, check_fp8_codes, check_output
+
+pytestmark = pytest.mark.gpu
+
+if cuda_ok():
+    import torch
+    import bit_quantized_moe_token_b200 as moe
+    from bit_quantized_moe_token_b200.synthetic import device_inputs, device_layer
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _need_gpu():
+    if not cuda_ok():
+        pytest.skip("no CUDA device")
+
+
+# ---- host <-> device helpers -------------------------------------------------------------------
+
+def to_dev_bf16(a_u16):
+    return torch.from_numpy(np.ascontiguousarray(a_u16).view(np.int16)).cuda().view(torch.bfloat16)
+
+
+def bits(t):
+    """bf16 tensor -> uint16 numpy bits."""
+    return t.detach().contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def ws_views(layer, ws, T, k):
+    lay = moe.moe_w4a8_workspace_layout(layer, T, k)
+    P = T * k
+    b = ws.cpu().numpy()
+    def arr(off, dtype, n):
+        return np.frombuffer(b[off:off + n * np.dtype(dtype).itemsize].tobytes(), dtype=dtype).copy()
+    return dict(ids=arr(lay["topk_ids"], np.int32, P).reshape(T, k),
+                gates=arr(lay["topk_w"], np.float32, P).reshape(T, k),
+                offsets=arr(lay["expert_offsets"], np.int32, layer.E + 1),
+                sorted_pairs=arr(lay["sorted_pairs"], np.int32, P),
+                row_of_pair=arr(lay["row_of_pair"], np.int32, P),
+                x_sorted=arr(lay["x_sorted"], np.uint8, P * layer.H).reshape(P, layer.H),
+                s_x_sorted=arr(lay["s_x_sorted"], np.float32, P),
+                hq=arr(lay["hq"], np.uint8, P * layer.N).reshape(P, layer.N),
+                s_h=arr(lay["s_h"], np.float32, P))
+
+
+# ---- generator -----------------------------------------------------------------------------------
+
+def test_device_generator_matches_host():
+    for name in ("tiny", "decode_t8", "prefill_t2048_zipf"):
+        wl = synth.WORKLOADS[name]
+        n = min(wl.T, 64)
+        x, lg = device_inputs(wl, T=n)
+        assert np.array_equal(bits(x), synth.tokens(wl, 0, n)), name
+        assert np.array_equal(lg.cpu().numpy(), synth.logits(wl, 0, n)), name
+    wl = synth.WORKLOADS["decode_t8"]
+    w = torch.empty(wl.N, wl.H, dtype=torch.bfloat16, device="cuda")
+    synth.dev_weight(wl.seed, synth.weight_stream(5, "gate"), w)
+    torch.cuda.synchronize()
+    assert np.array_equal(bits(w), synth.expert_weight(wl, 5, "gate"))
+
+
+# ---- S0 ----------------------------------------------------------------------------------------
+
+def _f32_to_bf16_bits(x):
+    u = np.asarray(x, np.float32).view(np.uint32).astype(np.uint64)
+    return ((u + 0x7FFF + ((u >> 16) & 1)) >> 16).astype(np.uint16)
+
+
+def test_pack_bitexact_random_and_edge_groups():
+    rng = np.random.default_rng(11)
+    w = (rng.standard_normal((300, 1024)) * 0.02).astype(np.float32)
+    w[0, :128] = 0.0                                   # zero group -> scale 0, codes 0
+    w[1, :128] = 0.0
+    w[1, 5] = 1e-40                                    # subnormal amax: bf16(amax/7) rounds to 0
+    w[2, 128:256] *= 1e30                              # huge values
+    w[3, :128] = -0.0                                  # negative zeros
+    w[4, :8] = np.array([0.4375, 0.21875, 0.15625, -0.03125, -0.4375, 0, 0, 0])  # exact ties
+    w[4, 8:128] = 0
+    w[5, :128] = rng.choice([-1.0, 1.0], 128) * 7 * 2.0 ** -8   # all codes +-7
+    wb = _f32_to_bf16_bits(w)
+    packed_ref, scales_ref, _ = oracle.rtn_pack(wb)
+    wd = to_dev_bf16(wb)
+    packed, scales = moe.pack_expert_weights(wd)
+    torch.cuda.synchronize()
+    assert np.array_equal(packed.cpu().numpy(), packed_ref)
+    assert np.array_equal(bits(scales), scales_ref)
+
+
+def test_pack_bitexact_seeded_expert():
+    wl = synth.WORKLOADS["decode_t8"]
+    for proj in ("gate", "down"):
+        wb = synth.expert_weight(wl, 17, proj)
+        p_ref, s_ref, _ = oracle.rtn_pack(wb)
+        p, s = moe.pack_expert_weights(to_dev_bf16(wb))
+        assert np.array_equal(p.cpu().numpy(), p_ref)
+        assert np.array_equal(bits(s), s_ref)
+
+
+# ---- S1 ----------------------------------------------------------------------------------------
+
+def test_quant_tokens_bitexact():
+    wl = synth.WORKLOADS["decode_t64"]
+    x = synth.tokens(wl)
+    xo = synth.tokens(synth.WORKLOADS["decode_t8"])
+    extra = np.zeros((4, wl.H), np.float32)
+    extra[1, :] = 1e-30                                # tiny row
+    extra[2, :] = np.linspace(-3, 3, wl.H)
+    extra[3, ::2] = 1.0
+    extra[3, 1::2] = 2.0 ** -12                        # values that underflow to +-0 codes
+    extra[3, 3] = -(2.0 ** -12)
+    xs = np.concatenate([x, xo, _f32_to_bf16_bits(extra)])
+    q_ref, s_ref = oracle.quant_tokens(xs)
+    xd = to_dev_bf16(xs)
+    q = torch.empty(xs.shape, dtype=torch.uint8, device="cuda")
+    s = torch.empty(xs.shape[0], dtype=torch.float32, device="cuda")
+    moe.fp8_quant_tokens(xd, q, s)
+    assert np.array_equal(s.cpu().numpy(), s_ref)
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+    tiny = synth.tokens(synth.WORKLOADS["tiny"])
+    q_ref, s_ref = oracle.quant_tokens(tiny)
+    q = torch.empty(tiny.shape, dtype=torch.uint8, device="cuda")
+    s = torch.empty(tiny.shape[0], dtype=torch.float32, device="cuda")
+    moe.fp8_quant_tokens(to_dev_bf16(tiny), q, s)
+    assert np.array_equal(q.cpu().numpy(), q_ref) and np.array_equal(s.cpu().numpy(), s_ref)
+
+
+# ---- S2 + S3 -----------------------------------------------------------------------------------
+
+ROUTE_CASES = [(16, 8, 2, None), (8, 256, 6, None), (64, 256, 6, None), (700, 256, 6, None),
+               (2048, 256, 6, "prefill_t2048_zipf"), (3, 1, 1, None), (5, 1024, 8, None),
+               (1000, 33, 3, None), (1, 256, 6, None), (4097, 7, 1, None)]
+
+
+@pytest.mark.parametrize("T,E,k,wlname", ROUTE_CASES)
+def test_route_bitexact(T, E, k, wlname):
+    if wlname:
+        logits = synth.logits(synth.WORKLOADS[wlname])
+    else:
+        logits = synth.normal_f32(0, 9000 + T * 7 + E, T * E).reshape(T, E)
+        if E >= 4:
+            logits[: T // 2, 1] = logits[: T // 2, 3]     # ties, lower index first
+    ids_ref, g_ref = oracle.route_topk(logits, k)
+    off_ref, sp_ref, rop_ref = oracle.permute(ids_ref, E)
+    ld = torch.from_numpy(logits).cuda()
+    P = T * k
+    ids = torch.empty(T, k, dtype=torch.int32, device="cuda")
+    g = torch.empty(T, k, dtype=torch.float32, device="cuda")
+    off = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    sp = torch.empty(P, dtype=torch.int32, device="cuda")
+    rop = torch.empty(P, dtype=torch.int32, device="cuda")
+    ws = torch.empty(moe.moe_route_workspace_bytes(T, E, k), dtype=torch.uint8, device="cuda")
+    moe.moe_route_topk(ld, k, ids, g, off, sp, rop, ws)
+    assert np.array_equal(ids.cpu().numpy(), ids_ref)
+    assert np.array_equal(off.cpu().numpy(), off_ref)
+    assert np.array_equal(sp.cpu().numpy(), sp_ref)
+    assert np.array_equal(rop.cpu().numpy(), rop_ref)
+    np.testing.assert_allclose(g.cpu().numpy(), g_ref, rtol=1e-6, atol=0)
+
+
+# ---- the layer: small shapes, everything compared ------------------------------------------------
+
+def _host_layer_and_dev(E, H, N, seed, n_shared=0, shared_N=0):
+    """Seeded random layer: packed on the host by the oracle and on the GPU by the library."""
+    rng_stream = 50_000 + seed * 10
+    gw = synth.normal_bf16(seed, rng_stream + 0, E * N * H, 0.02).reshape(E, N, H)
+    uw = synth.normal_bf16(seed, rng_stream + 1, E * N * H, 0.02).reshape(E, N, H)
+    dw = synth.normal_bf16(seed, rng_stream + 2, E * H * N, 0.02).reshape(E, H, N)
+    g = 128
+    gp, gs = zip(*[oracle.rtn_pack(gw[e], g)[:2] for e in range(E)])
+    up, us = zip(*[oracle.rtn_pack(uw[e], g)[:2] for e in range(E)])
+    dp, ds = zip(*[oracle.rtn_pack(dw[e], g)[:2] for e in range(E)])
+    sh = {}
+    shd = {}
+    if n_shared:
+        for i, key in enumerate(("sh_gate", "sh_up", "sh_down")):
+            shape = (n_shared, shared_N, H) if i < 2 else (n_shared, H, shared_N)
+            a = synth.normal_bf16(seed, rng_stream + 3 + i, int(np.prod(shape)), 0.02).reshape(shape)
+            sh[key] = a
+            shd[key] = to_dev_bf16(a)
+    hl = oracle.Layer(E, H, N, np.stack(gp), np.stack(up), np.stack(dp), np.stack(gs),
+                      np.stack(us), np.stack(ds), **sh)
+    dl = moe.make_layer(to_dev_bf16(gw), to_dev_bf16(uw), to_dev_bf16(dw), **shd)
+    torch.cuda.synchronize()
+    assert np.array_equal(dl.gate_packed.cpu().numpy(), hl.gate_packed)
+    assert np.array_equal(bits(dl.down_scales), hl.down_scales)
+    return hl, dl
+
+
+def _run_and_compare(hl, dl, x, logits, k, check_all=True):
+    T = x.shape[0]
+    ref = oracle.moe_forward(hl, x, logits, k)
+    xd, ld = to_dev_bf16(x), torch.from_numpy(logits).cuda()
+    ws = moe.alloc_workspace(dl, T, k)
+    out = moe.forward(dl, xd, ld, k, ws=ws)
+    torch.cuda.synchronize()
+    assert moe.moe_last_device_status() == 0
+    v = ws_views(dl, ws, T, k)
+    for key in ("ids", "offsets", "sorted_pairs", "row_of_pair"):
+        assert np.array_equal(v[key], ref[key]), key
+    np.testing.assert_allclose(v["gates"], ref["gates"], rtol=1e-6)
+    # first-stage FP8: codes and scales of each sorted row's token are exact
+    tok = ref["sorted_pairs"] // k
+    assert np.array_equal(v["x_sorted"], ref["xq"][tok])
+    assert np.array_equal(v["s_x_sorted"], ref["s_x"][tok])
+    n_diff, frac = check_fp8_codes(v["hq"], ref["hq"])
+    np.testing.assert_allclose(v["s_h"], ref["s_h"], rtol=2e-5)
+    err = check_output(bits(out), ref["out"])
+    return dict(hq_diff=n_diff, hq_frac=frac, out_err=err, out=bits(out))
+
+
+def test_forward_tiny_workload():
+    wl = synth.WORKLOADS["tiny"]
+    hl = oracle.pack_workload_layer(wl)
+    dl = device_layer(wl)
+    assert np.array_equal(dl.up_packed.cpu().numpy(), hl.up_packed)
+    r1 = _run_and_compare(hl, dl, synth.tokens(wl), synth.logits(wl), wl.k)
+    r2 = _run_and_compare(hl, dl, synth.tokens(wl), synth.logits(wl), wl.k)
+    assert np.array_equal(r1["out"], r2["out"])        # deterministic
+
+
+@pytest.mark.parametrize("E,H,N,k,T", [(5, 384, 256, 3, 37), (1, 256, 128, 1, 9), (8, 256, 128, 2, 1),
+                                       (16, 512, 384, 8, 130), (3, 1024, 128, 2, 700)])
+def test_forward_ragged_shapes(E, H, N, k, T):
+    hl, dl = _host_layer_and_dev(E, H, N, seed=E * 7 + T)
+    x = synth.normal_bf16(3, 777 + T, T * H).reshape(T, H)
+    logits = synth.normal_f32(3, 778 + T, T * E).reshape(T, E)
+    _run_and_compare(hl, dl, x, logits, k)
+
+
+def test_forward_shared_experts_small():
+    hl, dl = _host_layer_and_dev(4, 256, 128, seed=5, n_shared=2, shared_N=256)
+    T = 21
+    x = synth.normal_bf16(4, 901, T * 256).reshape(T, 256)
+    logits = synth.normal_f32(4, 902, T * 4).reshape(T, 4)
+    _run_and_compare(hl, dl, x, logits, 2)
+
+
+def test_forward_zero_tokens_and_zero_rows():
+    hl, dl = _host_layer_and_dev(4, 256, 128, seed=9)
+    x = synth.normal_bf16(5, 903, 6 * 256).reshape(6, 256)
+    x[2, :] = 0                                        # zero row: s_x = 0, codes 0, output 0
+    logits = synth.normal_f32(5, 904, 6 * 4).reshape(6, 4)
+    r = _run_and_compare(hl, dl, x, logits, 2)
+    assert not bf16_to_f32(r["out"][2]).any()
+    xd = torch.empty(0, 256, dtype=torch.bfloat16, device="cuda")
+    ld = torch.empty(0, 4, dtype=torch.float32, device="cuda")
+    out = torch.empty(0, 256, dtype=torch.bfloat16, device="cuda")
+    moe.moe_w4a8_forward(dl, xd, ld, 2, out, torch.empty(256, dtype=torch.uint8, device="cuda"))
+
+
+# ---- the layer at full size: sampled tokens -----------------------------------------------------
+
+FULL = ["decode_t8", "decode_t64", "prefill_t2048_zipf", "prefill_t16384_shared"]
+
+
+@pytest.fixture(scope="module")
+def full_layer():
+    wl = synth.WORKLOADS["prefill_t16384_shared"]     # same weights for all full-size configs
+    return device_layer(wl)
+
+
+def _sample_tokens(wl, n=4):
+    rng = np.random.default_rng(wl.T)
+    picks = {0, wl.T - 1}
+    while len(picks) < min(n, wl.T):
+        picks.add(int(rng.integers(0, wl.T)))
+    return sorted(picks)
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_forward_full_size_sampled(name, full_layer):
+    wl = synth.WORKLOADS[name]
+    dl = full_layer
+    if not wl.n_shared:
+        dl = moe.Layer(dl.E, dl.H, dl.N, dl.gate_packed, dl.up_packed, dl.down_packed,
+                       dl.gate_scales, dl.up_scales, dl.down_scales)
+    x, lg = device_inputs(wl)
+    ws = moe.alloc_workspace(dl, wl.T, wl.k)
+    out = moe.forward(dl, x, lg, wl.k, ws=ws)
+    torch.cuda.synchronize()
+    assert moe.moe_last_device_status() == 0
+    v = ws_views(dl, ws, wl.T, wl.k)
+    P = wl.P
+    # properties at full size
+    off = v["offsets"]
+    assert off[0] == 0 and off[-1] == P and np.all(np.diff(off) >= 0)
+    assert np.array_equal(np.sort(v["sorted_pairs"]), np.arange(P))
+    assert np.array_equal(v["row_of_pair"][v["sorted_pairs"]], np.arange(P))
+    seg = np.repeat(np.arange(wl.E), np.diff(off))
+    assert np.array_equal(v["ids"].reshape(-1)[v["sorted_pairs"]], seg)
+    for e in range(wl.E):
+        s = v["sorted_pairs"][off[e]:off[e + 1]]
+        assert np.all(np.diff(s) > 0)
+    outb = bits(out)
+    assert np.isfinite(bf16_to_f32(outb)).all()
+
+    # the oracle on sampled tokens (tokens are independent, so a sub-batch gives the same rows)
+    toks = _sample_tokens(wl)
+    xs = np.stack([synth.tokens(wl, t, 1)[0] for t in toks])
+    ls = np.stack([synth.logits(wl, t, 1)[0] for t in toks])
+    ids_ref, _ = oracle.route_topk(ls, wl.k)
+    experts = sorted(set(ids_ref.reshape(-1).tolist()))
+    hl = oracle.pack_workload_layer(wl, experts=experts)
+    # S0 parity on the experts the sample touches
+    for e in experts[:3]:
+        assert np.array_equal(dl.gate_packed[e].cpu().numpy(), hl.gate_packed[e])
+        assert np.array_equal(bits(dl.down_scales[e]), hl.down_scales[e])
+    ref = oracle.moe_forward(hl, xs, ls, wl.k)
+    assert np.array_equal(v["ids"][toks], ref["ids"])
+    np.testing.assert_allclose(v["gates"][toks], ref["gates"], rtol=1e-6)
+    gpu_rows = v["row_of_pair"].reshape(wl.T, wl.k)[toks].reshape(-1)
+    ref_rows = ref["row_of_pair"]
+    assert np.array_equal(v["x_sorted"][gpu_rows], ref["xq"][np.repeat(np.arange(len(toks)), wl.k)])
+    check_fp8_codes(v["hq"][gpu_rows], ref["hq"][ref_rows])
+    np.testing.assert_allclose(v["s_h"][gpu_rows], ref["s_h"][ref_rows], rtol=2e-5)
+    check_output(outb[toks], ref["out"])
