@@ -57,55 +57,85 @@ def peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """nvidia-smi clocks and throttle reasons, sampled every 100 ms by a background reader that
+    stamps each line; summary() keeps the samples within 0.25 s of the marked timed region."""
+    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
     def __init__(self, gpu_index):
-        self.idx = gpu_index
-        self.proc = None
+        import threading
+        self.idx, self.samples, self.proc = gpu_index, [], None
+        self.t0 = self.t1 = None
+        self._lock = threading.Lock()
+        self._thread = None
 
-    def __enter__(self):
+    def start(self):
+        import threading
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
+            return self
+        self._thread = threading.Thread(target=self._read, daemon=True)
+        self._thread.start()
+        deadline = time.monotonic() + 5.0
+        while time.monotonic() < deadline and not self.samples:
+            time.sleep(0.02)
         return self
 
-    def __exit__(self, *exc):
-        self.lines = []
-        if self.proc:
-            self.proc.terminate()
-            try:
-                out, _ = self.proc.communicate(timeout=5)
-            except Exception:
-                self.proc.kill()
-                out = ""
-            self.lines = [l for l in out.splitlines() if l.strip()]
+    def _read(self):
+        for line in self.proc.stdout:
+            with self._lock:
+                self.samples.append((time.monotonic(), line.strip()))
+
+    def mark_start(self):
+        self.t0 = time.monotonic()
+
+    def mark_end(self):
+        self.t1 = time.monotonic()
+
+    def stop(self):
+        if not self.proc:
+            return
+        deadline = time.monotonic() + 1.0
+        while time.monotonic() < deadline:
+            with self._lock:
+                if self.samples and self.samples[-1][0] > (self.t1 or 0):
+                    break
+            time.sleep(0.02)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
 
     def summary(self):
+        if self.t0 is None or self.t1 is None:
+            return None
         sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for l in getattr(self, "lines", []):
+        with self._lock:
+            picked = [l for t, l in self.samples if self.t0 - 0.25 <= t <= self.t1 + 0.25]
+        for l in picked:
             f = [x.strip() for x in l.split(",")]
-            if len(f) < 9:
+            if len(f) < 7:
                 continue
             try:
-                sm.append(float(f[1]))
-                mx = float(f[2])
+                sm.append(float(f[0]))
+                mx = float(f[1])
             except ValueError:
                 continue
-            for n, v in zip(names, f[5:9]):
+            for n, v in zip(self.NAMES, f[3:7]):
                 if v.lower() == "active":
                     reasons.add(n)
         if not sm:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "window_s": round(self.t1 - self.t0, 4)}
 
 
 def dist_setup():
@@ -156,35 +186,59 @@ def run_ours(args):
     if moe.moe_last_device_status() != 0:
         raise RuntimeError("device status: timeout during warm-up")
 
+    clk = ClockSampler(local).start()
     for i in range(args.warmup):
         x, lg = batches[i % N_BATCHES]
         moe.forward(layer, x, lg, k, out=out, ws=ws)
     torch.cuda.synchronize()
 
     # ---- device-timed region ----
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(moe.N_STAGE_EVENTS)]
-          for _ in range(args.steps)]
+    def make_events(n):
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        for e in evs:                 # torch creates the CUDA event on first record
+            e.record(stream)
+        return evs
+
+    # stage breakdown: an untimed pass with every stage boundary marked
+    full = [make_events(moe.N_STAGE_EVENTS) for _ in range(N_BATCHES)]
+    torch.cuda.synchronize()
+    for i in range(N_BATCHES):
+        x, lg = batches[i]
+        moe.moe_w4a8_forward_profiled(layer, x, lg, k, out, ws, full[i])
+    torch.cuda.synchronize()
+    stage_ms = {s: 0.0 for s in moe.STAGES}
+    for i in range(N_BATCHES):
+        for j, s in enumerate(moe.STAGES):
+            stage_ms[s] += full[i][j].elapsed_time(full[i][j + 1]) / N_BATCHES
+    # timed region: only the dominant kernel's boundaries are marked (2 events per step)
+    DOM_A, DOM_B = 2, 3               # gate/up GEMM
+    ev = []
+    for _ in range(args.steps):
+        pair = make_events(2)
+        row = [None] * moe.N_STAGE_EVENTS
+        row[DOM_A], row[DOM_B] = pair
+        ev.append(row)
+    torch.cuda.synchronize()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     launches = 0
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
-        start.record(stream)
-        for i in range(args.steps):
-            x, lg = batches[i % N_BATCHES]
-            launches += moe.moe_w4a8_forward_profiled(layer, x, lg, k, out, ws, ev[i])
-        end.record(stream)
-        torch.cuda.synchronize()
+    clk.mark_start()
+    start.record(stream)
+    for i in range(args.steps):
+        x, lg = batches[i % N_BATCHES]
+        launches += moe.moe_w4a8_forward_profiled(layer, x, lg, k, out, ws, ev[i])
+    end.record(stream)
+    torch.cuda.synchronize()
+    clk.mark_end()
+    clk.stop()
     if world > 1:
         dist.barrier()
     total_ms = start.elapsed_time(end)
     if moe.moe_last_device_status() != 0:
         raise RuntimeError("device status: timeout in the timed region")
-    stage_ms = {s: 0.0 for s in moe.STAGES}
-    for i in range(args.steps):
-        for j, s in enumerate(moe.STAGES):
-            stage_ms[s] += ev[i][j].elapsed_time(ev[i][j + 1]) / args.steps
+    dom_ms = sum(ev[i][DOM_A].elapsed_time(ev[i][DOM_B]) for i in range(args.steps)) / args.steps
     t_max = torch.tensor([total_ms], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
@@ -224,8 +278,6 @@ def run_ours(args):
     hbm, bf16, peak_kind = peaks()
     gu_bytes, down_bytes = expert_bytes(wl)
     mean_touched = sum(touched[i % N_BATCHES] for i in range(args.steps)) / args.steps
-    dom = "gateup_gemm"
-    dom_ms = stage_ms[dom]
     dom_bytes = mean_touched * gu_bytes
     achieved = dom_bytes / (dom_ms / 1e3) / 1e9
     roofline = {"bound": "hbm", "kernel": "grouped gate/up W4A8 GEMM (stage)",

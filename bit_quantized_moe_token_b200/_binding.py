@@ -215,12 +215,13 @@ STAGES = ("route", "quant", "gateup_gemm", "swiglu_requant", "down_gemm", "share
 
 
 def moe_w4a8_forward_profiled(layer: Layer, x, logits, k: int, out, ws, events, stream=None) -> int:
-    """moe_w4a8_forward that also records `events` (8 torch.cuda.Event with timing) at the stage
-    boundaries; returns the number of kernels launched."""
+    """moe_w4a8_forward that also records `events` (8 entries: torch.cuda.Event with timing, or
+    None to skip that boundary) at the stage boundaries; returns the number of kernels launched."""
     T = x.shape[0]
     s = layer.c_struct()
     nbytes = ws.numel() * ws.element_size() if ws is not None else 0
-    arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    arr = (ctypes.c_void_p * len(events))(
+        *[ctypes.c_void_p(e.cuda_event if e is not None else 0) for e in events])
     n = ctypes.c_int(0)
     _check(lib().moe_w4a8_forward_profiled(ctypes.byref(s), _ptr(x), _ptr(logits), T, k, _ptr(out),
                                            _ptr(ws), nbytes, _stream(stream), arr, len(events),

@@ -5,50 +5,73 @@
 #include "quant.cuh"
 #include "route.cuh"
 #include "gemm_simple.cuh"
+#include "gemm_tc.cuh"
 
 namespace moe {
 
-// h = silu(G) * U over one expert-sorted row, then Hq = e4m3(h / s_h), s_h = max|h| / 448.
-// G and U are rows of GU: gate in columns [0, N), up in [N, 2N).  One CTA per row; h is
-// recomputed in the second pass (same inputs, same result) instead of being stored.
-__global__ void __launch_bounds__(256) k_swiglu_requant(const float* __restrict__ GU, int N,
-                                                        uint8_t* __restrict__ hq,
-                                                        float* __restrict__ s_h) {
-    __shared__ float red[32];
+// S5 requantization of the SwiGLU activations h (fp32, one expert-sorted row per CTA, written
+// by the gate/up GEMM together with max|h| per row): s_h = max|h| / 448, Hq = e4m3(h / s_h),
+// and the per-group code sums the down GEMM's unsigned widening needs.
+__global__ void __launch_bounds__(256) k_requant(const float* __restrict__ h, int N,
+                                                 const unsigned* __restrict__ amax,
+                                                 uint8_t* __restrict__ hq, float* __restrict__ s_h,
+                                                 float* __restrict__ csum) {
     const int64_t r = blockIdx.x;
-    const float* g = GU + r * 2 * N;
-    const float* u = g + N;
-    float a = 0.0f;
-    for (int n = threadIdx.x; n < N; n += blockDim.x)
-        a = fmaxf(a, fabsf(__fmul_rn(silu(g[n]), u[n])));
-    a = block_max(a, red);
-    const float s = __fdiv_rn(a, kFp8Max);
-    for (int n2 = threadIdx.x * 2; n2 < N; n2 += blockDim.x * 2) {
-        uint16_t c = 0;
-        if (s != 0.0f) {
-            const float h0 = __fmul_rn(silu(g[n2]), u[n2]);
-            const float h1 = __fmul_rn(silu(g[n2 + 1]), u[n2 + 1]);
-            c = f32x2_to_e4m3x2(__fdiv_rn(h0, s), __fdiv_rn(h1, s));
+    const float s = __fdiv_rn(__uint_as_float(amax[r]), kFp8Max);
+    const int chunks = N >> 3, G = N / kGroup;
+    const float4* src = reinterpret_cast<const float4*>(h + r * N);
+    for (int base = 0; base < chunks; base += blockDim.x) {
+        const int c = base + threadIdx.x;
+        const bool live = c < chunks;
+        uint2 codes = make_uint2(0u, 0u);
+        if (live && s != 0.0f) {
+            const float4 a = src[2 * c], b = src[2 * c + 1];
+            codes.x = static_cast<uint32_t>(f32x2_to_e4m3x2(__fdiv_rn(a.x, s), __fdiv_rn(a.y, s))) |
+                      (static_cast<uint32_t>(f32x2_to_e4m3x2(__fdiv_rn(a.z, s), __fdiv_rn(a.w, s))) << 16);
+            codes.y = static_cast<uint32_t>(f32x2_to_e4m3x2(__fdiv_rn(b.x, s), __fdiv_rn(b.y, s))) |
+                      (static_cast<uint32_t>(f32x2_to_e4m3x2(__fdiv_rn(b.z, s), __fdiv_rn(b.w, s))) << 16);
         }
-        *reinterpret_cast<uint16_t*>(hq + r * N + n2) = c;
+        const float gs = half_warp_sum(sum8_e4m3(codes)) * 0.015625f;
+        if (live) {
+            reinterpret_cast<uint2*>(hq + r * N)[c] = codes;
+            if ((c & 15) == 0) csum[r * G + (c >> 4)] = gs;
+        }
     }
     if (threadIdx.x == 0) s_h[r] = s;
 }
 
-// out[t, m] = bf16( sum_j gate[t,j] * Y[row(t,j), m]  (+ shared[t, m]) ).
+// out[t, m] = bf16( sum_j gate[t,j] * Y[row(t,j), m]  (+ shared[t, m]) ), j in selection
+// order.  One thread per (token, 4 consecutive m): float4 loads of the k routed rows.
 __global__ void __launch_bounds__(256) k_combine(const float* __restrict__ Y,
                                                  const float* __restrict__ gates,
                                                  const int32_t* __restrict__ rop, int k, int H,
-                                                 const float* __restrict__ shared,
+                                                 int64_t T, const float* __restrict__ shared,
                                                  uint16_t* __restrict__ out) {
-    const int64_t t = blockIdx.x;
-    for (int m = threadIdx.x; m < H; m += blockDim.x) {
-        float o = 0.0f;
-        for (int j = 0; j < k; ++j)
-            o = __fadd_rn(o, __fmul_rn(gates[t * k + j], Y[(int64_t)rop[t * k + j] * H + m]));
-        if (shared) o = __fadd_rn(o, shared[t * H + m]);
-        out[t * H + m] = f32_to_bf16_bits(o);
+    const int q = H >> 2;
+    const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    if (i >= T * q) return;
+    const int64_t t = i / q;
+    const int m4 = static_cast<int>(i % q);
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j = 0; j < k; ++j) {
+        const float g = gates[t * k + j];
+        const float4 y = reinterpret_cast<const float4*>(Y + (int64_t)rop[t * k + j] * H)[m4];
+        o.x = __fadd_rn(o.x, __fmul_rn(g, y.x));
+        o.y = __fadd_rn(o.y, __fmul_rn(g, y.y));
+        o.z = __fadd_rn(o.z, __fmul_rn(g, y.z));
+        o.w = __fadd_rn(o.w, __fmul_rn(g, y.w));
     }
+    if (shared) {
+        const float4 sh = reinterpret_cast<const float4*>(shared + t * H)[m4];
+        o.x = __fadd_rn(o.x, sh.x);
+        o.y = __fadd_rn(o.y, sh.y);
+        o.z = __fadd_rn(o.z, sh.z);
+        o.w = __fadd_rn(o.w, sh.w);
+    }
+    uint2 packed;
+    packed.x = static_cast<uint32_t>(f32_to_bf16_bits(o.x)) | (static_cast<uint32_t>(f32_to_bf16_bits(o.y)) << 16);
+    packed.y = static_cast<uint32_t>(f32_to_bf16_bits(o.z)) | (static_cast<uint32_t>(f32_to_bf16_bits(o.w)) << 16);
+    reinterpret_cast<uint2*>(out + t * H)[m4] = packed;
 }
 
 // s_out[t, n] = silu(g[t, n]) * u[t, n]   (shared-expert activation, fp32)
@@ -64,7 +87,7 @@ __global__ void k_swiglu_f32(const float* __restrict__ g, const float* __restric
 // ------------------------------------------------------------------------------------------
 struct WsPlan {
     size_t topk_ids, topk_w, offsets, sorted, rop, route_ws;
-    size_t x_sorted, s_x_sorted, gu, hq, s_h, y;
+    size_t x_sorted, s_x_sorted, csum_x, h, amax, hq, s_h, csum_h, y;
     size_t sh_g, sh_u, sh_a, sh_y;
     size_t total;
 };
@@ -86,9 +109,12 @@ inline WsPlan plan_workspace(const moe_w4a8_layer& L, int64_t T, int k) {
     p.route_ws = take(route_ws_bytes(T, L.E, k));
     p.x_sorted = take((size_t)P * L.H);
     p.s_x_sorted = take(P * 4);
-    p.gu = take((size_t)P * 2 * L.N * 4);
+    p.csum_x = take((size_t)P * (L.H / kGroup) * 4);
+    p.h = take((size_t)P * L.N * 4);
+    p.amax = take(P * 4);
     p.hq = take((size_t)P * L.N);
     p.s_h = take(P * 4);
+    p.csum_h = take((size_t)P * (L.N / kGroup) * 4);
     p.y = take((size_t)P * L.H * 4);
     if (L.n_shared > 0) {
         p.sh_g = take((size_t)T * L.shared_N * 4);
@@ -109,7 +135,6 @@ inline int layer_args_ok(const moe_w4a8_layer* L, int64_t T, int k) {
     if (st != MOE_OK) return st;
     if (L->n_shared < 0) return MOE_ERR_INVALID_ARG;
     if (L->n_shared > 0 && (L->shared_N <= 0 || L->shared_N % 128)) return MOE_ERR_UNSUPPORTED_SHAPE;
-    if ((T * k + kSimpleRows - 1) / kSimpleRows + L->E > 65535) return MOE_ERR_UNSUPPORTED_SHAPE;
     return MOE_OK;
 }
 
@@ -206,9 +231,12 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const uint16_t* x_bf16,
     int32_t* rop = (int32_t*)at(p.rop);
     uint8_t* xs = (uint8_t*)at(p.x_sorted);
     float* sxs = (float*)at(p.s_x_sorted);
-    float* gu = (float*)at(p.gu);
+    float* csx = (float*)at(p.csum_x);
+    float* h = (float*)at(p.h);
+    unsigned* amax = (unsigned*)at(p.amax);
     uint8_t* hq = (uint8_t*)at(p.hq);
     float* sh = (float*)at(p.s_h);
+    float* csh = (float*)at(p.csum_h);
     float* y = (float*)at(p.y);
     const int64_t P = T * k;
 
@@ -219,28 +247,30 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const uint16_t* x_bf16,
         return st;
     sm.launches += 1 + (P <= kSinglePassMaxP ? 1 : 3);
     sm.mark(1, stream);
-    // S1, written straight into the expert-sorted rows
-    if ((st = launch_quant_tokens(x_bf16, T, L.H, xs, sxs, rop, k, stream))) return st;
+    // S1, written straight into the expert-sorted rows (+ per-group code sums)
+    if ((st = launch_quant_tokens(x_bf16, T, L.H, xs, sxs, rop, k, stream, csx))) return st;
+    if (cudaMemsetAsync(amax, 0, P * sizeof(unsigned), stream) != cudaSuccess) return MOE_ERR_CUDA;
     sm.launches += 1;
     sm.mark(2, stream);
-    // S4: gate -> columns [0, N), up -> [N, 2N)
-    if ((st = launch_gemm_w4a8_simple(xs, sxs, L.gate_packed, L.gate_scales, offsets, L.E, L.N, L.H,
-                                      P, gu, 2 * L.N, stream)))
-        return st;
-    if ((st = launch_gemm_w4a8_simple(xs, sxs, L.up_packed, L.up_scales, offsets, L.E, L.N, L.H, P,
-                                      gu + L.N, 2 * L.N, stream)))
-        return st;
-    sm.launches += 2;
+    // S4 + SwiGLU: h = silu(G) * U, max|h| per row
+    {
+        TcGemmArgs a{xs, sxs, csx, L.gate_packed, L.gate_scales, L.up_packed, L.up_scales,
+                     offsets, L.E, L.N, L.H, h, L.N, amax};
+        if ((st = launch_gemm_tc<true>(a, P, stream))) return st;
+    }
+    sm.launches += 1;
     sm.mark(3, stream);
     // S5
-    k_swiglu_requant<<<static_cast<unsigned>(P), 256, 0, stream>>>(gu, L.N, hq, sh);
+    k_requant<<<static_cast<unsigned>(P), 256, 0, stream>>>(h, L.N, amax, hq, sh, csh);
     if ((st = launch_status())) return st;
     sm.launches += 1;
     sm.mark(4, stream);
     // S6
-    if ((st = launch_gemm_w4a8_simple(hq, sh, L.down_packed, L.down_scales, offsets, L.E, L.H, L.N,
-                                      P, y, L.H, stream)))
-        return st;
+    {
+        TcGemmArgs a{hq, sh, csh, L.down_packed, L.down_scales, nullptr, nullptr,
+                     offsets, L.E, L.H, L.N, y, L.H, nullptr};
+        if ((st = launch_gemm_tc<false>(a, P, stream))) return st;
+    }
     sm.launches += 1;
     sm.mark(5, stream);
     // S8
@@ -270,7 +300,11 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const uint16_t* x_bf16,
     }
     sm.mark(6, stream);
     // S7
-    k_combine<<<static_cast<unsigned>(T), 256, 0, stream>>>(y, gates, rop, k, L.H, shared, out_bf16);
+    {
+        const int64_t n = T * (L.H / 4);
+        k_combine<<<static_cast<unsigned>((n + 255) / 256), 256, 0, stream>>>(y, gates, rop, k, L.H, T,
+                                                                            shared, out_bf16);
+    }
     if ((st = launch_status())) return st;
     sm.launches += 1;
     sm.mark(7, stream);
