@@ -7,7 +7,8 @@ from ._binding import (MOE_OK, Layer, MoeError, fp8_quant_tokens, layer_struct, 
                        moe_last_device_status, moe_route_topk, moe_route_workspace_bytes,
                        moe_status_string, moe_w4a8_forward, moe_w4a8_forward_profiled,
                        moe_w4a8_workspace_bytes, STAGES, N_STAGE_EVENTS,
-                       moe_w4a8_workspace_layout, w4a8_pack_weights)
+                       moe_w4a8_workspace_layout, w4a8_pack_weights,
+                       moe_selftest_bounded_wait)
 from .layer import alloc_workspace, forward, make_layer, pack_expert_weights
 
 __all__ = ["MOE_OK", "Layer", "MoeError", "fp8_quant_tokens", "layer_struct", "lib",
@@ -15,4 +16,4 @@ __all__ = ["MOE_OK", "Layer", "MoeError", "fp8_quant_tokens", "layer_struct", "l
            "moe_status_string", "moe_w4a8_forward", "moe_w4a8_forward_profiled", "STAGES",
            "N_STAGE_EVENTS", "moe_w4a8_workspace_bytes",
            "moe_w4a8_workspace_layout", "w4a8_pack_weights", "alloc_workspace", "forward",
-           "make_layer", "pack_expert_weights"]
+           "make_layer", "pack_expert_weights", "moe_selftest_bounded_wait"]

@@ -72,11 +72,12 @@ def lib() -> ctypes.CDLL:
         L.moe_w4a8_forward_profiled.argtypes = [ctypes.POINTER(_CLayer), vp, vp, i64, i32, vp, vp,
                                                 sz, vp, vp, i32, ctypes.POINTER(ctypes.c_int)]
         L.moe_last_device_status.argtypes = [vp]
+        L.moe_selftest_bounded_wait.argtypes = [i64, vp]
         L.moe_status_string.argtypes = [i32]
         L.moe_status_string.restype = ctypes.c_char_p
         for f in (L.w4a8_pack_weights, L.fp8_quant_tokens, L.moe_route_topk,
                   L.moe_w4a8_workspace_layout, L.moe_w4a8_forward, L.moe_w4a8_forward_profiled,
-                  L.moe_last_device_status):
+                  L.moe_last_device_status, L.moe_selftest_bounded_wait):
             f.restype = i32
         _lib = L
     return _lib
@@ -231,3 +232,8 @@ def moe_w4a8_forward_profiled(layer: Layer, x, logits, k: int, out, ws, events, 
 
 def moe_last_device_status(stream=None) -> int:
     return int(lib().moe_last_device_status(_stream(stream)))
+
+
+def moe_selftest_bounded_wait(limit_ns: int, stream=None) -> None:
+    _check(lib().moe_selftest_bounded_wait(int(limit_ns), _stream(stream)),
+           "moe_selftest_bounded_wait")

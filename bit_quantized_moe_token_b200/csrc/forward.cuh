@@ -6,36 +6,28 @@
 #include "route.cuh"
 #include "gemm_simple.cuh"
 #include "gemm_tc.cuh"
+#include "gemm_ws.cuh"
 
 namespace moe {
 
 // S5 requantization of the SwiGLU activations h (fp32, one expert-sorted row per CTA, written
-// by the gate/up GEMM together with max|h| per row): s_h = max|h| / 448, Hq = e4m3(h / s_h),
-// and the per-group code sums the down GEMM's unsigned widening needs.
+// by the gate/up GEMM together with max|h| per row): s_h = max|h| / 448, Hq = e4m3(h / s_h).
 __global__ void __launch_bounds__(256) k_requant(const float* __restrict__ h, int N,
                                                  const unsigned* __restrict__ amax,
-                                                 uint8_t* __restrict__ hq, float* __restrict__ s_h,
-                                                 float* __restrict__ csum) {
+                                                 uint8_t* __restrict__ hq, float* __restrict__ s_h) {
     const int64_t r = blockIdx.x;
     const float s = __fdiv_rn(__uint_as_float(amax[r]), kFp8Max);
-    const int chunks = N >> 3, G = N / kGroup;
     const float4* src = reinterpret_cast<const float4*>(h + r * N);
-    for (int base = 0; base < chunks; base += blockDim.x) {
-        const int c = base + threadIdx.x;
-        const bool live = c < chunks;
+    for (int c = threadIdx.x; c < (N >> 3); c += blockDim.x) {
         uint2 codes = make_uint2(0u, 0u);
-        if (live && s != 0.0f) {
+        if (s != 0.0f) {
             const float4 a = src[2 * c], b = src[2 * c + 1];
             codes.x = static_cast<uint32_t>(f32x2_to_e4m3x2(__fdiv_rn(a.x, s), __fdiv_rn(a.y, s))) |
                       (static_cast<uint32_t>(f32x2_to_e4m3x2(__fdiv_rn(a.z, s), __fdiv_rn(a.w, s))) << 16);
             codes.y = static_cast<uint32_t>(f32x2_to_e4m3x2(__fdiv_rn(b.x, s), __fdiv_rn(b.y, s))) |
                       (static_cast<uint32_t>(f32x2_to_e4m3x2(__fdiv_rn(b.z, s), __fdiv_rn(b.w, s))) << 16);
         }
-        const float gs = half_warp_sum(sum8_e4m3(codes)) * 0.015625f;
-        if (live) {
-            reinterpret_cast<uint2*>(hq + r * N)[c] = codes;
-            if ((c & 15) == 0) csum[r * G + (c >> 4)] = gs;
-        }
+        reinterpret_cast<uint2*>(hq + r * N)[c] = codes;
     }
     if (threadIdx.x == 0) s_h[r] = s;
 }
@@ -87,7 +79,7 @@ __global__ void k_swiglu_f32(const float* __restrict__ g, const float* __restric
 // ------------------------------------------------------------------------------------------
 struct WsPlan {
     size_t topk_ids, topk_w, offsets, sorted, rop, route_ws;
-    size_t x_sorted, s_x_sorted, csum_x, h, amax, hq, s_h, csum_h, y;
+    size_t x_sorted, s_x_sorted, h, amax, hq, s_h, y;
     size_t sh_g, sh_u, sh_a, sh_y;
     size_t total;
 };
@@ -109,12 +101,10 @@ inline WsPlan plan_workspace(const moe_w4a8_layer& L, int64_t T, int k) {
     p.route_ws = take(route_ws_bytes(T, L.E, k));
     p.x_sorted = take((size_t)P * L.H);
     p.s_x_sorted = take(P * 4);
-    p.csum_x = take((size_t)P * (L.H / kGroup) * 4);
     p.h = take((size_t)P * L.N * 4);
     p.amax = take(P * 4);
     p.hq = take((size_t)P * L.N);
     p.s_h = take(P * 4);
-    p.csum_h = take((size_t)P * (L.N / kGroup) * 4);
     p.y = take((size_t)P * L.H * 4);
     if (L.n_shared > 0) {
         p.sh_g = take((size_t)T * L.shared_N * 4);
@@ -231,12 +221,10 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const uint16_t* x_bf16,
     int32_t* rop = (int32_t*)at(p.rop);
     uint8_t* xs = (uint8_t*)at(p.x_sorted);
     float* sxs = (float*)at(p.s_x_sorted);
-    float* csx = (float*)at(p.csum_x);
     float* h = (float*)at(p.h);
     unsigned* amax = (unsigned*)at(p.amax);
     uint8_t* hq = (uint8_t*)at(p.hq);
     float* sh = (float*)at(p.s_h);
-    float* csh = (float*)at(p.csum_h);
     float* y = (float*)at(p.y);
     const int64_t P = T * k;
 
@@ -247,29 +235,27 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const uint16_t* x_bf16,
         return st;
     sm.launches += 1 + (P <= kSinglePassMaxP ? 1 : 3);
     sm.mark(1, stream);
-    // S1, written straight into the expert-sorted rows (+ per-group code sums)
-    if ((st = launch_quant_tokens(x_bf16, T, L.H, xs, sxs, rop, k, stream, csx))) return st;
+    // S1, written straight into the expert-sorted rows
+    if ((st = launch_quant_tokens(x_bf16, T, L.H, xs, sxs, rop, k, stream))) return st;
     if (cudaMemsetAsync(amax, 0, P * sizeof(unsigned), stream) != cudaSuccess) return MOE_ERR_CUDA;
     sm.launches += 1;
     sm.mark(2, stream);
     // S4 + SwiGLU: h = silu(G) * U, max|h| per row
     {
-        TcGemmArgs a{xs, sxs, csx, L.gate_packed, L.gate_scales, L.up_packed, L.up_scales,
-                     offsets, L.E, L.N, L.H, h, L.N, amax};
-        if ((st = launch_gemm_tc<true>(a, P, stream))) return st;
+        WsGemmArgs a{sxs, L.gate_scales, L.up_scales, offsets, L.E, L.N, L.H, (int)P, h, L.N, amax};
+        if ((st = launch_gemm_ws<true>(a, xs, L.gate_packed, L.up_packed, stream))) return st;
     }
     sm.launches += 1;
     sm.mark(3, stream);
     // S5
-    k_requant<<<static_cast<unsigned>(P), 256, 0, stream>>>(h, L.N, amax, hq, sh, csh);
+    k_requant<<<static_cast<unsigned>(P), 256, 0, stream>>>(h, L.N, amax, hq, sh);
     if ((st = launch_status())) return st;
     sm.launches += 1;
     sm.mark(4, stream);
     // S6
     {
-        TcGemmArgs a{hq, sh, csh, L.down_packed, L.down_scales, nullptr, nullptr,
-                     offsets, L.E, L.H, L.N, y, L.H, nullptr};
-        if ((st = launch_gemm_tc<false>(a, P, stream))) return st;
+        WsGemmArgs a{sh, L.down_scales, nullptr, offsets, L.E, L.H, L.N, (int)P, y, L.H, nullptr};
+        if ((st = launch_gemm_ws<false>(a, hq, L.down_packed, nullptr, stream))) return st;
     }
     sm.launches += 1;
     sm.mark(5, stream);

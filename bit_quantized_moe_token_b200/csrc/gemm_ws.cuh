@@ -1,0 +1,406 @@
+// gemm_ws.cuh — S4/S6: warp-specialised grouped W4A8 GEMM on tcgen05 with a TMA ring.
+//
+// Roles (192 threads, one persistent CTA per SM):
+//   warps 0-3  math: thread i owns A row i = TMEM lane i.  Per K-group it widens its row of
+//              packed INT4 codes (64 B, from the TMA ring) to 128 E4M3 bytes in a 128-byte-
+//              swizzled A stage, then promotes the previous group's TMEM partial into its fp32
+//              register accumulator with the group scale; at a tile's end it runs the epilogue.
+//   warp 4     TMA producer: streams each group's packed weight tile (128 rows x 64 B) and the
+//              activation tile (BN rows x 128 B, landing pre-swizzled for the MMA) into a ring
+//              of RS stages.
+//   warp 5     MMA issuer (one lane) and TMEM owner: four (or eight) tcgen05.mma.kind::f8f6f4
+//              per group into a double-buffered TMEM partial, then commits to the barriers that
+//              release the TMEM buffer to the math warps and the ring / A stages to their
+//              producers.
+//
+// Widening (see gemm_tc.cuh for the arithmetic):
+//   kUnsigned (narrow token tiles, decode): byte = nibble = E4M3 of (code+8)*2^-9; four more
+//     MMAs per group with a constant A tile of -2^-6 (E4M3 0x88) against the same activation
+//     tile add -8*2^-9*sum_k q_k, so TMEM holds exactly 2^-9 * sum_k q_k*code_k and the
+//     promotion is one FMA with 512*scale.  The tensor core has ample headroom at decode sizes.
+//   signed (wide token tiles, prefill): byte = E4M3(code) by byte-permute lookup.
+//
+// Every mbarrier wait is bounded; a timeout sets a CTA-wide abort flag that turns all later
+// waits into no-ops (so the named barrier among the math warps stays uniform), records the
+// device status, and the CTA frees its TMEM and exits.
+#pragma once
+#include <cuda.h>
+#include "common.cuh"
+#include "tc_ptx.cuh"
+#include "gemm_tc.cuh"
+
+namespace moe {
+
+struct WsGemmArgs {
+    const float* s_row;     // [P] per-row activation scale
+    const uint16_t* s0;     // [E, R0, K/128] bf16 scales of w0 (gate, or down)
+    const uint16_t* s1;     // up scales (SwiGLU instance)
+    const int32_t* offsets; // [E + 1]
+    int E, R0, K, P;
+    float* out;             // SwiGLU: h [P, R0]; plain: Y [P, ldo]
+    int ldo;
+    unsigned* amax;         // SwiGLU: [P] float bits of max|h| per row
+};
+
+namespace ws {
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
+                                            uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];"
+        ::"r"(tc::smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(tc::smem_u32(bar)),
+          "r"(x), "r"(y)
+        : "memory");
+}
+
+__device__ __forceinline__ void prefetch_map(const CUtensorMap* map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+__device__ __forceinline__ void named_sync_math() {
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+
+// Bounded wait that gives up at once after an abort.
+__device__ __forceinline__ bool wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+    if (*abort) return false;
+    if (tc::mbar_wait(bar, parity)) return true;
+    *abort = 1;
+    return false;
+}
+
+}  // namespace ws
+
+template <int BN, bool kUnsigned>
+struct WsCfg {
+    static constexpr int kRaw = 128 * 64;                       // packed codes of one group tile
+    static constexpr int kB = BN * 128;                         // activation tile
+    static constexpr int kStage = ((kB + kRaw + 1023) / 1024) * 1024;
+    static constexpr int kRS = 4;                               // ring stages
+    static constexpr int kCtasPerSm = (BN <= 32) ? 2 : 1;       // narrow tiles: 2 CTAs per SM
+    static constexpr int kAS = 2;                               // widened A stages
+    static constexpr int kA = 128 * 128;
+    static constexpr int kUsStride = BN + 1;
+    static constexpr int kOffRing = 0;
+    static constexpr int kOffA = kOffRing + kRS * kStage;
+    static constexpr int kOffConst = kOffA + kAS * kA;          // constant -2^-6 A tile (unsigned)
+    static constexpr int kOffUs = kOffConst + (kUnsigned ? kA : 0);
+    static constexpr int kOffPre = kOffUs + 64 * kUsStride * 4;
+    static constexpr int kOffBar = ((kOffPre + 1025 * 4 + 7) / 8) * 8;
+    static constexpr int kNumBars = 2 * kRS + 2 * kAS + 4;
+    static constexpr int kOffMisc = kOffBar + kNumBars * 8;     // TMEM slot, abort flag
+    static constexpr int kBytes = kOffMisc + 16;
+    static constexpr int kAlloc = kBytes + 1024;
+    static constexpr int kTmemCols = (2 * BN < 32) ? 32 : 2 * BN;
+    static constexpr int kThreads = 192;
+};
+
+template <int BN, bool kUnsigned, bool kSwiGLU>
+__global__ void __launch_bounds__(192, WsCfg<BN, kUnsigned>::kCtasPerSm)
+    k_gemm_w4a8_ws(const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__ CUtensorMap tm_w1,
+                   const __grid_constant__ CUtensorMap tm_act, const WsGemmArgs a) {
+    using C = WsCfg<BN, kUnsigned>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* ring = sm + C::kOffRing;
+    uint8_t* sA = sm + C::kOffA;
+    uint8_t* sConst = sm + C::kOffConst;
+    float* sUs = reinterpret_cast<float*>(sm + C::kOffUs);
+    int* pre = reinterpret_cast<int*>(sm + C::kOffPre);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + C::kOffBar);
+    uint64_t* raw_full = bar;
+    uint64_t* raw_empty = bar + C::kRS;
+    uint64_t* a_full = bar + 2 * C::kRS;
+    uint64_t* a_empty = a_full + C::kAS;
+    uint64_t* t_full = a_empty + C::kAS;
+    uint64_t* t_empty = t_full + 2;
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + C::kOffMisc);
+    volatile int* abort = reinterpret_cast<volatile int*>(sm + C::kOffMisc + 4);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int G = a.K / kGroup;
+    const int m_tiles = kSwiGLU ? a.R0 / 64 : a.R0 / 128;
+    const int row_tiles = row_tile_prefix(a.offsets, a.E, BN, pre);
+    const int64_t n_tiles = (int64_t)row_tiles * m_tiles;
+    if ((int64_t)blockIdx.x >= n_tiles) return;
+
+    if (tid == 0) {
+        for (int i = 0; i < C::kRS; ++i) { tc::mbar_init(&raw_full[i], 1); tc::mbar_init(&raw_empty[i], 1); }
+        for (int i = 0; i < C::kAS; ++i) { tc::mbar_init(&a_full[i], 128); tc::mbar_init(&a_empty[i], 1); }
+        for (int i = 0; i < 2; ++i) { tc::mbar_init(&t_full[i], 1); tc::mbar_init(&t_empty[i], 128); }
+        *abort = 0;
+        tc::fence_mbar_init();
+    }
+    if (warp == 5) {
+        tc::tmem_alloc(tslot, C::kTmemCols);
+        tc::tmem_relinquish();
+    }
+    if (kUnsigned && tid < 128) {   // constant A tile: every byte E4M3(-2^-6) = 0x88
+        uint4* c4 = reinterpret_cast<uint4*>(sConst);
+        for (int i = tid; i < C::kA / 16; i += 128) c4[i] = make_uint4(0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u);
+        tc::fence_proxy_async_smem();
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem = *tslot;
+
+    if (warp == 4) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            ws::prefetch_map(&tm_w0);
+            if (kSwiGLU) ws::prefetch_map(&tm_w1);
+            ws::prefetch_map(&tm_act);
+            uint32_t it = 0;
+            for (int64_t tile = blockIdx.x; tile < n_tiles && !*abort; tile += gridDim.x) {
+                const int rt = static_cast<int>(tile / m_tiles), mt = static_cast<int>(tile % m_tiles);
+                const int e = expert_of_tile(pre, a.E, rt);
+                const int row0 = a.offsets[e] + (rt - pre[e]) * BN;
+                for (int g = 0; g < G; ++g, ++it) {
+                    const int s = it % C::kRS;
+                    if (!ws::wait(&raw_empty[s], ((it / C::kRS) & 1) ^ 1, abort)) break;
+                    uint8_t* st = ring + s * C::kStage;
+                    tc::mbar_arrive_expect_tx(&raw_full[s], C::kB + C::kRaw);
+                    ws::tma_load_2d(st, &tm_act, g * kGroup, row0, &raw_full[s]);
+                    if (kSwiGLU) {
+                        const int y = e * a.R0 + mt * 64;
+                        ws::tma_load_2d(st + C::kB, &tm_w0, g * 64, y, &raw_full[s]);
+                        ws::tma_load_2d(st + C::kB + 64 * 64, &tm_w1, g * 64, y, &raw_full[s]);
+                    } else {
+                        ws::tma_load_2d(st + C::kB, &tm_w0, g * 64, e * a.R0 + mt * 128, &raw_full[s]);
+                    }
+                }
+            }
+        }
+    } else if (warp == 5) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = tc::idesc_e4m3_f32(128, BN);
+            uint32_t it = 0;
+            for (int64_t tile = blockIdx.x; tile < n_tiles && !*abort; tile += gridDim.x) {
+                for (int g = 0; g < G; ++g, ++it) {
+                    const int s = it % C::kRS, as = it % C::kAS, tb = it & 1;
+                    if (!ws::wait(&raw_full[s], (it / C::kRS) & 1, abort)) break;
+                    if (!ws::wait(&a_full[as], (it / C::kAS) & 1, abort)) break;
+                    if (!ws::wait(&t_empty[tb], ((it >> 1) & 1) ^ 1, abort)) break;
+                    tc::tc_fence_after();
+                    const uint32_t b_addr = tc::smem_u32(ring + s * C::kStage);
+                    const uint32_t a_addr = tc::smem_u32(sA + as * C::kA);
+                    const uint32_t d = tmem + tb * BN;
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        tc::mma_e4m3(d, tc::sdesc_sw128(a_addr + kk * 32), tc::sdesc_sw128(b_addr + kk * 32),
+                                     idesc, kk > 0 ? 1u : 0u);
+                    if (kUnsigned) {
+                        const uint32_t c_addr = tc::smem_u32(sConst);
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            tc::mma_e4m3(d, tc::sdesc_sw128(c_addr + kk * 32),
+                                         tc::sdesc_sw128(b_addr + kk * 32), idesc, 1u);
+                    }
+                    tc::mma_commit(&t_full[tb]);
+                    tc::mma_commit(&a_empty[as]);
+                    tc::mma_commit(&raw_empty[s]);
+                }
+            }
+            // the commits complete in order: once the last one has arrived, no tensor-core
+            // arrive on this CTA's barriers is still pending
+            if (it > 0) ws::wait(&raw_empty[(it - 1) % C::kRS], ((it - 1) / C::kRS) & 1, abort);
+        }
+    } else {
+        // ------------------------------------------------------------ math warps 0-3
+        const uint32_t t_lane = static_cast<uint32_t>(warp * 32) << 16;
+        uint32_t it = 0;
+        for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+            const int rt = static_cast<int>(tile / m_tiles), mt = static_cast<int>(tile % m_tiles);
+            const int e = expert_of_tile(pre, a.E, rt);
+            const int seg0 = a.offsets[e];
+            const int r0 = (rt - pre[e]) * BN;
+            const int nrows = min(BN, a.offsets[e + 1] - seg0 - r0);
+            const int64_t row0 = seg0 + r0;
+            const uint16_t* ssrc;
+            if (kSwiGLU) {
+                const int n = mt * 64 + (tid & 63);
+                ssrc = (tid < 64 ? a.s0 : a.s1) + ((int64_t)e * a.R0 + n) * G;
+            } else {
+                ssrc = a.s0 + ((int64_t)e * a.R0 + mt * 128 + tid) * G;
+            }
+            float acc[BN];
+#pragma unroll
+            for (int j = 0; j < BN; ++j) acc[j] = 0.0f;
+            float sc_next = bf16_bits_to_f32(__ldg(ssrc));
+
+            auto promote = [&](uint32_t itp, float sc) {
+                const int tb = itp & 1;
+                ws::wait(&t_full[tb], (itp >> 1) & 1, abort);
+                tc::tc_fence_after();
+                if (kUnsigned) sc *= 512.0f;
+#pragma unroll
+                for (int c0 = 0; c0 < BN; c0 += (BN >= 32 ? 32 : 16)) {
+                    if constexpr (BN >= 32) {
+                        uint32_t v[32];
+                        tc::tmem_ld32(tmem + t_lane + tb * BN + c0, v);
+                        tc::tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) acc[c0 + j] = fmaf(sc, __uint_as_float(v[j]), acc[c0 + j]);
+                    } else {
+                        uint32_t v[16];
+                        tc::tmem_ld16(tmem + t_lane + tb * BN + c0, v);
+                        tc::tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) acc[c0 + j] = fmaf(sc, __uint_as_float(v[j]), acc[c0 + j]);
+                    }
+                }
+                tc::tc_fence_before();
+                tc::mbar_arrive(&t_empty[tb]);
+            };
+
+            float sc_prev = 0.0f;
+            for (int g = 0; g < G; ++g, ++it) {
+                const int s = it % C::kRS, as = it % C::kAS;
+                const float sc = sc_next;
+                if (g + 1 < G) sc_next = bf16_bits_to_f32(__ldg(ssrc + g + 1));
+                // ---- widen group g into A stage `as` ----
+                ws::wait(&raw_full[s], (it / C::kRS) & 1, abort);
+                ws::wait(&a_empty[as], ((it / C::kAS) & 1) ^ 1, abort);
+                // four consecutive threads widen the four 16-byte chunks of one row: a quarter warp
+                // reads 128 contiguous bytes and writes two rows whose swizzled chunks differ
+                const uint8_t* raw = ring + s * C::kStage + C::kB;
+                uint8_t* a_st = sA + as * C::kA;
+                const int q = tid & 3;
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {
+                    const int row = (tid >> 2) + 32 * p;
+                    const uint4 w = *reinterpret_cast<const uint4*>(raw + row * 64 + q * 16);
+                    const uint2 w0 = widen8<kUnsigned>(w.x), w1 = widen8<kUnsigned>(w.y);
+                    const uint2 w2 = widen8<kUnsigned>(w.z), w3 = widen8<kUnsigned>(w.w);
+                    *reinterpret_cast<uint4*>(a_st + sw128_off(row, 2 * q)) = make_uint4(w0.x, w0.y, w1.x, w1.y);
+                    *reinterpret_cast<uint4*>(a_st + sw128_off(row, 2 * q + 1)) = make_uint4(w2.x, w2.y, w3.x, w3.y);
+                }
+                tc::fence_proxy_async_smem();
+                tc::mbar_arrive(&a_full[as]);
+                // ---- promote group g-1 while the tensor core runs group g ----
+                if (g > 0) promote(it - 1, sc_prev);
+                sc_prev = sc;
+            }
+            promote(it - 1, sc_prev);
+
+            // ---- epilogue (static indices keep acc[] in registers) ----
+            if constexpr (kSwiGLU) {
+                if (tid >= 64) {
+#pragma unroll
+                    for (int j = 0; j < BN; ++j) sUs[(tid - 64) * C::kUsStride + j] = acc[j];
+                }
+                ws::named_sync_math();
+                if (tid < 64) {
+                    const int n = mt * 64 + tid;
+#pragma unroll
+                    for (int j = 0; j < BN; ++j) {
+                        if (j < nrows) {
+                            const float sr = a.s_row[row0 + j];
+                            const float h = silu(acc[j] * sr) * (sUs[tid * C::kUsStride + j] * sr);
+                            a.out[(row0 + j) * a.ldo + n] = h;
+                            const float m = warp_max(fabsf(h));
+                            if (lane == 0) atomicMax(a.amax + row0 + j, __float_as_uint(m));
+                        }
+                    }
+                }
+                ws::named_sync_math();
+            } else {
+                const int m = mt * 128 + tid;
+#pragma unroll
+                for (int j = 0; j < BN; ++j)
+                    if (j < nrows) a.out[(row0 + j) * a.ldo + m] = acc[j] * a.s_row[row0 + j];
+            }
+        }
+    }
+
+    __syncwarp();          // single-lane roles reconverge before the CTA-wide barrier
+    __syncthreads();
+    if (*abort && tid == 0) atomicExch(&g_device_status, 1);
+    if (warp == 5) {
+        tc::tc_fence_after();
+        tc::tmem_dealloc(tmem, C::kTmemCols);
+    }
+}
+
+// ---- host side --------------------------------------------------------------------------------
+
+using PFN_encodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                     const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                     const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                     CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+inline PFN_encodeTiled encode_fn() {
+    static PFN_encodeTiled fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        fn = reinterpret_cast<PFN_encodeTiled>(p);
+    }
+    return fn;
+}
+
+// 2D byte tensor [rows, row_bytes] (row-major) with a box of box_rows x box_bytes.
+inline bool make_map_u8(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t rows,
+                        uint32_t box_bytes, uint32_t box_rows, bool swizzle128) {
+    PFN_encodeTiled fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {row_bytes, rows};
+    const cuuint64_t strides[1] = {row_bytes};
+    const cuuint32_t box[2] = {box_bytes, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE,
+              swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BN, bool kUnsigned, bool kSwiGLU>
+int launch_gemm_ws_inst(const WsGemmArgs& a, const void* act, const void* w0, const void* w1,
+                        int64_t max_row_tiles, cudaStream_t stream) {
+    using C = WsCfg<BN, kUnsigned>;
+    static TcLaunchShape cache[16];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+    auto kern = k_gemm_w4a8_ws<BN, kUnsigned, kSwiGLU>;
+    TcLaunchShape& c = cache[dev & 15];
+    if (c.sms == 0) {
+        int sms = 0;
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kAlloc) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        c.ctas_per_sm = C::kCtasPerSm;
+        c.sms = sms;
+    }
+    CUtensorMap m0, m1, mact;
+    const int rows_per_load = kSwiGLU ? 64 : 128;
+    if (!make_map_u8(&m0, w0, a.K / 2, (uint64_t)a.E * a.R0, 64, rows_per_load, false) ||
+        !make_map_u8(&m1, kSwiGLU ? w1 : w0, a.K / 2, (uint64_t)a.E * a.R0, 64, rows_per_load, false) ||
+        !make_map_u8(&mact, act, a.K, (uint64_t)a.P, 128, BN, true))
+        return MOE_ERR_CUDA;
+    const int m_tiles = kSwiGLU ? a.R0 / 64 : a.R0 / 128;
+    const int64_t grid = std::max<int64_t>(
+        1, std::min<int64_t>(max_row_tiles * m_tiles, (int64_t)c.sms * c.ctas_per_sm));
+    kern<<<static_cast<unsigned>(grid), C::kThreads, C::kAlloc, stream>>>(m0, m1, mact, a);
+    return launch_status();
+}
+
+template <bool kSwiGLU>
+int launch_gemm_ws(const WsGemmArgs& a, const void* act, const void* w0, const void* w1,
+                   cudaStream_t stream) {
+    const int BN = tc_tile_rows(a.P, a.E);
+    const int64_t max_row_tiles = ((int64_t)a.P + BN - 1) / BN + a.E;
+    switch (BN) {
+        case 16: return launch_gemm_ws_inst<16, true, kSwiGLU>(a, act, w0, w1, max_row_tiles, stream);
+        case 32: return launch_gemm_ws_inst<32, true, kSwiGLU>(a, act, w0, w1, max_row_tiles, stream);
+        case 64: return launch_gemm_ws_inst<64, false, kSwiGLU>(a, act, w0, w1, max_row_tiles, stream);
+        default: return launch_gemm_ws_inst<128, false, kSwiGLU>(a, act, w0, w1, max_row_tiles, stream);
+    }
+}
+
+}  // namespace moe

@@ -17,6 +17,25 @@ __device__ int g_device_status = 0;
 #include "route.cuh"
 #include "gemm_simple.cuh"
 #include "forward.cuh"
+#include "tc_ptx.cuh"
+
+namespace moe {
+// An mbarrier that nothing arrives on: the bounded wait must give up after `limit_ns`.
+__global__ void k_selftest_bounded_wait(uint64_t limit_ns) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        tc::mbar_init(&bar, 1);
+        tc::fence_mbar_init();
+        if (!tc::mbar_wait(&bar, 0, limit_ns)) atomicExch(&g_device_status, 1);
+    }
+}
+}  // namespace moe
+
+extern "C" int moe_selftest_bounded_wait(int64_t limit_ns, moe_stream_t stream) {
+    if (limit_ns < 1000 || limit_ns > 1000000000) return MOE_ERR_INVALID_ARG;
+    moe::k_selftest_bounded_wait<<<1, 32, 0, stream>>>(static_cast<uint64_t>(limit_ns));
+    return moe::launch_status();
+}
 
 extern "C" int moe_last_device_status(moe_stream_t stream) {
     if (cudaStreamSynchronize(stream) != cudaSuccess) return MOE_ERR_CUDA;

@@ -46,40 +46,14 @@ __device__ __forceinline__ float amax8(uint4 v) {
     return a;
 }
 
-// Sum of the values of eight E4M3 codes (exact per pair, fp32 adds).
-__device__ __forceinline__ float sum8_e4m3(uint2 c) {
-    const uint32_t u[2] = {c.x, c.y};
-    float s = 0.0f;
-#pragma unroll
-    for (int q = 0; q < 2; ++q) {
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const __half2_raw r = __nv_cvt_fp8x2_to_halfraw2(
-                static_cast<__nv_fp8x2_storage_t>((u[q] >> (16 * h)) & 0xFFFFu), __NV_E4M3);
-            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&r));
-            s += f.x + f.y;
-        }
-    }
-    return s;
-}
-
-// Per-(row, K-group of 128) sum of the code values divided by 64, written by the 16 threads
-// that hold one group's 16 chunks of 8 (lane-aligned half warps).  Used by the tensor-core
-// GEMM's unsigned widening to remove the +8 offset of the stored nibbles.
-__device__ __forceinline__ float half_warp_sum(float v) {
-#pragma unroll
-    for (int o = 8; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    return v;
-}
-
 // One CTA per token row.  With `row_of_pair` non-null the codes and scale of token t are
-// written to its k expert-sorted rows (the forward's gathered activation matrix), together
-// with the group sums when `csum` is non-null; otherwise to row t.
+// written to its k expert-sorted rows (the forward's gathered activation matrix); otherwise
+// to row t.
 __global__ void __launch_bounds__(256) k_quant_tokens(const uint16_t* __restrict__ x, int H,
                                                       uint8_t* __restrict__ q,
                                                       float* __restrict__ scale,
                                                       const int32_t* __restrict__ row_of_pair,
-                                                      int k, float* __restrict__ csum) {
+                                                      int k) {
     __shared__ float red[32];
     const int64_t t = blockIdx.x;
     const uint4* row = reinterpret_cast<const uint4*>(x + t * H);
@@ -89,19 +63,11 @@ __global__ void __launch_bounds__(256) k_quant_tokens(const uint16_t* __restrict
     a = block_max(a, red);
     const float s = __fdiv_rn(a, kFp8Max);
     const int ncopy = row_of_pair ? k : 1;
-    const int G = H / kGroup;
-    for (int base = 0; base < chunks; base += blockDim.x) {   // uniform trip count (shuffles)
-        const int c = base + threadIdx.x;
-        const bool live = c < chunks;
-        const uint2 codes = live ? quant8(__ldg(row + c), s) : make_uint2(0u, 0u);
-        float gs = 0.0f;
-        if (csum) gs = half_warp_sum(sum8_e4m3(codes)) * 0.015625f;
-        if (live) {
-            for (int j = 0; j < ncopy; ++j) {
-                const int64_t r = row_of_pair ? row_of_pair[t * k + j] : t;
-                reinterpret_cast<uint2*>(q + r * H)[c] = codes;
-                if (csum && (c & 15) == 0) csum[r * G + (c >> 4)] = gs;
-            }
+    for (int c = threadIdx.x; c < chunks; c += blockDim.x) {
+        const uint2 codes = quant8(__ldg(row + c), s);
+        for (int j = 0; j < ncopy; ++j) {
+            const int64_t r = row_of_pair ? row_of_pair[t * k + j] : t;
+            reinterpret_cast<uint2*>(q + r * H)[c] = codes;
         }
     }
     if (threadIdx.x == 0)
@@ -109,11 +75,10 @@ __global__ void __launch_bounds__(256) k_quant_tokens(const uint16_t* __restrict
 }
 
 inline int launch_quant_tokens(const uint16_t* x, int64_t T, int64_t H, uint8_t* q, float* s,
-                               const int32_t* row_of_pair, int k, cudaStream_t stream,
-                               float* csum = nullptr) {
+                               const int32_t* row_of_pair, int k, cudaStream_t stream) {
     if (T == 0) return MOE_OK;
     k_quant_tokens<<<static_cast<unsigned>(T), 256, 0, stream>>>(x, static_cast<int>(H), q, s,
-                                                                 row_of_pair, k, csum);
+                                                                 row_of_pair, k);
     return launch_status();
 }
 

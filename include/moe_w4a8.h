@@ -181,6 +181,14 @@ int moe_w4a8_forward_profiled(const moe_w4a8_layer* layer, const uint16_t* x_bf1
  * stream itself reports an error. */
 int moe_last_device_status(moe_stream_t stream);
 
+/* Diagnostic for the failure-detection path: launches one CTA that waits, with the same
+ * bounded wait the GEMM kernels use but a limit of `limit_ns` nanoseconds (1 us .. 1 s), on an
+ * mbarrier that nothing ever arrives on.  The wait gives up, the kernel sets the sticky
+ * device-status word and returns; moe_last_device_status() then reports MOE_ERR_TIMEOUT and the
+ * context stays usable.  No page describes this; it exists so the timeout path can be tested
+ * without hanging a GPU. */
+int moe_selftest_bounded_wait(int64_t limit_ns, moe_stream_t stream);
+
 /* Static description of a status code. */
 const char* moe_status_string(int status);
 

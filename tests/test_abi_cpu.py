@@ -38,6 +38,12 @@ def test_library_exports_every_declared_symbol():
         assert ctypes.cast(getattr(L, n), ctypes.c_void_p).value
 
 
+def test_selftest_rejects_bad_limits():
+    L = _L()
+    assert L.moe_selftest_bounded_wait(10, None) == -1
+    assert L.moe_selftest_bounded_wait(2_000_000_000, None) == -1
+
+
 def test_status_strings():
     assert moe.moe_status_string(0) == "ok"
     assert "workspace" in moe.moe_status_string(-4)

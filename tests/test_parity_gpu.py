@@ -321,3 +321,16 @@ def test_forward_full_size_sampled(name, full_layer):
     check_fp8_codes(v["hq"][gpu_rows], ref["hq"][ref_rows])
     np.testing.assert_allclose(v["s_h"][gpu_rows], ref["s_h"][ref_rows], rtol=2e-5)
     check_output(outb[toks], ref["out"])
+
+
+# ---- failure detection: a bounded device wait that runs out -------------------------------------
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    assert moe.moe_last_device_status() == 0
+    moe.moe_selftest_bounded_wait(50_000_000)          # 50 ms on a barrier nothing completes
+    assert moe.moe_last_device_status() == -6          # MOE_ERR_TIMEOUT
+    assert moe.moe_last_device_status() == 0          # read-and-clear
+    wl = synth.WORKLOADS["tiny"]                        # the context is still usable
+    hl = oracle.pack_workload_layer(wl)
+    dl = device_layer(wl)
+    _run_and_compare(hl, dl, synth.tokens(wl), synth.logits(wl), wl.k)
