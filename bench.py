@@ -211,7 +211,7 @@ def run_ours(args):
         for j, s in enumerate(moe.STAGES):
             stage_ms[s] += full[i][j].elapsed_time(full[i][j + 1]) / N_BATCHES
     # timed region: only the dominant kernel's boundaries are marked (2 events per step)
-    DOM_A, DOM_B = 2, 3               # gate/up GEMM
+    DOM_A, DOM_B = 3, 4               # gate/up GEMM (stage boundaries, moe_w4a8.h)
     ev = []
     for _ in range(args.steps):
         pair = make_events(2)

@@ -212,7 +212,7 @@ def moe_w4a8_forward(layer: Layer, x, logits, k: int, out, ws, stream=None) -> N
 
 
 N_STAGE_EVENTS = 8
-STAGES = ("route", "quant", "gateup_gemm", "swiglu_requant", "down_gemm", "shared", "combine")
+STAGES = ("route", "quant", "shared", "gateup_gemm", "swiglu_requant", "down_gemm", "combine")
 
 
 def moe_w4a8_forward_profiled(layer: Layer, x, logits, k: int, out, ws, events, stream=None) -> int:

@@ -4,9 +4,8 @@
 #include "common.cuh"
 #include "quant.cuh"
 #include "route.cuh"
-#include "gemm_simple.cuh"
-#include "gemm_tc.cuh"
 #include "gemm_ws.cuh"
+#include "gemm_bf16_tc.cuh"
 
 namespace moe {
 
@@ -66,12 +65,66 @@ __global__ void __launch_bounds__(256) k_combine(const float* __restrict__ Y,
     reinterpret_cast<uint2*>(out + t * H)[m4] = packed;
 }
 
-// s_out[t, n] = silu(g[t, n]) * u[t, n]   (shared-expert activation, fp32)
-__global__ void k_swiglu_f32(const float* __restrict__ g, const float* __restrict__ u,
-                             float* __restrict__ a, int64_t n) {
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
-         i += (int64_t)gridDim.x * blockDim.x)
-        a[i] = __fmul_rn(silu(g[i]), u[i]);
+// Decode front end, one CTA of 1024 threads: S2 top-k (a warp per token), S3 the
+// permutation, S1 per-token FP8 quantization written straight into the token's k sorted rows
+// (a warp per token), and zeroing of the per-row / per-token counters and maxima the fused
+// GEMM epilogues accumulate into.  The arithmetic is that of k_topk / k_permute_single /
+// k_quant_tokens.
+template <int EPL>
+__global__ void __launch_bounds__(1024) k_front(const float* __restrict__ logits,
+                                                const uint16_t* __restrict__ x, int T, int E,
+                                                int k, int H, int32_t* __restrict__ ids,
+                                                float* __restrict__ gates,
+                                                int32_t* __restrict__ offsets,
+                                                int32_t* __restrict__ sorted,
+                                                int32_t* __restrict__ rop, uint8_t* __restrict__ xs,
+                                                float* __restrict__ sxs,
+                                                unsigned* __restrict__ zero, int n_zero) {
+    extern __shared__ int sm[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int P = T * k;
+    for (int t = warp; t < T; t += 32) topk_row<EPL>(logits + (int64_t)t * E, E, k, ids + t * k, gates + t * k, lane);
+    for (int i = threadIdx.x; i < n_zero; i += blockDim.x) zero[i] = 0u;
+    __syncthreads();
+    permute_block(ids, P, E, offsets, sorted, rop, sm);
+    __syncthreads();
+    const int chunks = H >> 3;
+    for (int t = warp; t < T; t += 32) {
+        const uint4* row = reinterpret_cast<const uint4*>(x + (int64_t)t * H);
+        float a = 0.0f;
+        for (int c = lane; c < chunks; c += 32) a = fmaxf(a, amax8(__ldg(row + c)));
+        a = warp_max(a);
+        const float s = __fdiv_rn(a, kFp8Max);
+        for (int c = lane; c < chunks; c += 32) {
+            const uint2 codes = quant8(__ldg(row + c), s);
+            for (int j = 0; j < k; ++j)
+                reinterpret_cast<uint2*>(xs + (int64_t)rop[t * k + j] * H)[c] = codes;
+        }
+        if (lane < k) sxs[rop[t * k + lane]] = s;
+    }
+}
+
+inline bool front_fits(int64_t T, int k) { return T <= 256 && T * k <= kSinglePassMaxP; }
+
+inline int launch_front(const float* logits, const uint16_t* x, int T, int E, int k, int H,
+                        int32_t* ids, float* gates, int32_t* offsets, int32_t* sorted, int32_t* rop,
+                        uint8_t* xs, float* sxs, unsigned* zero, int n_zero, cudaStream_t stream) {
+    const size_t smem = permute_block_smem(E);
+    const int epl = (E + 31) / 32;
+#define MOE_FRONT(N)                                                                             \
+    do {                                                                                         \
+        if (set_smem((const void*)k_front<N>, smem)) return MOE_ERR_CUDA;                        \
+        k_front<N><<<1, 1024, smem, stream>>>(logits, x, T, E, k, H, ids, gates, offsets, sorted, \
+                                              rop, xs, sxs, zero, n_zero);                       \
+    } while (0)
+    if (epl <= 1) MOE_FRONT(1);
+    else if (epl <= 2) MOE_FRONT(2);
+    else if (epl <= 4) MOE_FRONT(4);
+    else if (epl <= 8) MOE_FRONT(8);
+    else if (epl <= 16) MOE_FRONT(16);
+    else MOE_FRONT(32);
+#undef MOE_FRONT
+    return launch_status();
 }
 
 // ------------------------------------------------------------------------------------------
@@ -79,8 +132,9 @@ __global__ void k_swiglu_f32(const float* __restrict__ g, const float* __restric
 // ------------------------------------------------------------------------------------------
 struct WsPlan {
     size_t topk_ids, topk_w, offsets, sorted, rop, route_ws;
-    size_t x_sorted, s_x_sorted, h, amax, hq, s_h, y;
-    size_t sh_g, sh_u, sh_a, sh_y;
+    size_t x_sorted, s_x_sorted, h, zero, hq, s_h, y;
+    int64_t n_zero;   // u32 words at `zero`: max|h| per row [P], row counters [P], token counters
+    size_t sh_a, sh_y;
     size_t total;
 };
 
@@ -102,14 +156,13 @@ inline WsPlan plan_workspace(const moe_w4a8_layer& L, int64_t T, int k) {
     p.x_sorted = take((size_t)P * L.H);
     p.s_x_sorted = take(P * 4);
     p.h = take((size_t)P * L.N * 4);
-    p.amax = take(P * 4);
+    p.n_zero = 2 * P + T * (L.H / 128);
+    p.zero = take((size_t)p.n_zero * 4);
     p.hq = take((size_t)P * L.N);
     p.s_h = take(P * 4);
     p.y = take((size_t)P * L.H * 4);
     if (L.n_shared > 0) {
-        p.sh_g = take((size_t)T * L.shared_N * 4);
-        p.sh_u = take((size_t)T * L.shared_N * 4);
-        p.sh_a = take((size_t)T * L.shared_N * 4);
+        p.sh_a = take((size_t)T * L.n_shared * L.shared_N * 2);
         p.sh_y = take((size_t)T * L.H * 4);
     }
     p.total = off;
@@ -204,6 +257,8 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const uint16_t* x_bf16,
         !L.down_packed || !L.gate_scales || !L.up_scales || !L.down_scales)
         return MOE_ERR_INVALID_ARG;
     if (L.n_shared > 0 && (!L.sh_gate || !L.sh_up || !L.sh_down)) return MOE_ERR_INVALID_ARG;
+    if (L.n_shared > 0 && (!aligned(L.sh_gate, 16) || !aligned(L.sh_up, 16) || !aligned(L.sh_down, 16)))
+        return MOE_ERR_MISALIGNED;
     const WsPlan p = plan_workspace(L, T, k);
     if (!ws || ws_bytes < p.total) return MOE_ERR_WORKSPACE;
     if (!aligned(ws, 256) || !aligned(x_bf16, 16) || !aligned(out_bf16, 16) ||
@@ -212,6 +267,7 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const uint16_t* x_bf16,
         !aligned(L.down_scales, 2))
         return MOE_ERR_MISALIGNED;
 
+    const int64_t P = T * k;
     char* w = static_cast<char*>(ws);
     auto at = [&](size_t off) { return static_cast<void*>(w + off); };
     int32_t* ids = (int32_t*)at(p.topk_ids);
@@ -222,77 +278,80 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const uint16_t* x_bf16,
     uint8_t* xs = (uint8_t*)at(p.x_sorted);
     float* sxs = (float*)at(p.s_x_sorted);
     float* h = (float*)at(p.h);
-    unsigned* amax = (unsigned*)at(p.amax);
+    unsigned* zero = (unsigned*)at(p.zero);
+    unsigned* amax = zero;
+    unsigned* rowcnt = zero + P;
+    unsigned* tokcnt = zero + 2 * P;
     uint8_t* hq = (uint8_t*)at(p.hq);
     float* sh = (float*)at(p.s_h);
     float* y = (float*)at(p.y);
-    const int64_t P = T * k;
+    const bool fused = ws_fused(tc_tile_rows(P, L.E));
 
     sm.mark(0, stream);
-    // S2 + S3
-    if ((st = launch_topk(router_logits, T, L.E, k, ids, gates, stream))) return st;
-    if ((st = launch_permute(ids, T, L.E, k, offsets, sorted, rop, (int32_t*)at(p.route_ws), stream)))
-        return st;
-    sm.launches += 1 + (P <= kSinglePassMaxP ? 1 : 3);
-    sm.mark(1, stream);
-    // S1, written straight into the expert-sorted rows
-    if ((st = launch_quant_tokens(x_bf16, T, L.H, xs, sxs, rop, k, stream))) return st;
-    if (cudaMemsetAsync(amax, 0, P * sizeof(unsigned), stream) != cudaSuccess) return MOE_ERR_CUDA;
-    sm.launches += 1;
-    sm.mark(2, stream);
-    // S4 + SwiGLU: h = silu(G) * U, max|h| per row
-    {
-        WsGemmArgs a{sxs, L.gate_scales, L.up_scales, offsets, L.E, L.N, L.H, (int)P, h, L.N, amax};
-        if ((st = launch_gemm_ws<true>(a, xs, L.gate_packed, L.up_packed, stream))) return st;
+    if (front_fits(T, k)) {
+        // S2 + S3 + S1 in one CTA
+        if ((st = launch_front(router_logits, x_bf16, (int)T, L.E, k, L.H, ids, gates, offsets, sorted,
+                               rop, xs, sxs, zero, (int)p.n_zero, stream)))
+            return st;
+        sm.launches += 1;
+        sm.mark(1, stream);
+        sm.mark(2, stream);
+    } else {
+        if ((st = launch_topk(router_logits, T, L.E, k, ids, gates, stream))) return st;
+        if ((st = launch_permute(ids, T, L.E, k, offsets, sorted, rop, (int32_t*)at(p.route_ws), stream)))
+            return st;
+        sm.launches += 1 + (P <= kSinglePassMaxP ? 1 : 3);
+        sm.mark(1, stream);
+        // S1, written straight into the expert-sorted rows
+        if ((st = launch_quant_tokens(x_bf16, T, L.H, xs, sxs, rop, k, stream))) return st;
+        if (cudaMemsetAsync(zero, 0, p.n_zero * sizeof(unsigned), stream) != cudaSuccess) return MOE_ERR_CUDA;
+        sm.launches += 1;
+        sm.mark(2, stream);
     }
-    sm.launches += 1;
-    sm.mark(3, stream);
-    // S5
-    k_requant<<<static_cast<unsigned>(P), 256, 0, stream>>>(h, L.N, amax, hq, sh);
-    if ((st = launch_status())) return st;
-    sm.launches += 1;
-    sm.mark(4, stream);
-    // S6
-    {
-        WsGemmArgs a{sh, L.down_scales, nullptr, offsets, L.E, L.H, L.N, (int)P, y, L.H, nullptr};
-        if ((st = launch_gemm_ws<false>(a, hq, L.down_packed, nullptr, stream))) return st;
-    }
-    sm.launches += 1;
-    sm.mark(5, stream);
-    // S8
+    // S8: shared experts, summed = one SwiGLU MLP of width n_shared * shared_N
     float* shared = nullptr;
     if (L.n_shared > 0) {
-        const int Ns = L.shared_N;
-        float* sg = (float*)at(p.sh_g);
-        float* su = (float*)at(p.sh_u);
-        float* sa = (float*)at(p.sh_a);
+        const int Wsh = L.n_shared * L.shared_N;
+        uint16_t* sa = (uint16_t*)at(p.sh_a);
         shared = (float*)at(p.sh_y);
-        for (int s = 0; s < L.n_shared; ++s) {
-            const uint16_t* wg = L.sh_gate + (int64_t)s * Ns * L.H;
-            const uint16_t* wu = L.sh_up + (int64_t)s * Ns * L.H;
-            const uint16_t* wd = L.sh_down + (int64_t)s * L.H * Ns;
-            if ((st = launch_gemm_bf16_simple<uint16_t>(x_bf16, wg, (int)T, Ns, L.H, sg, Ns, false, stream)))
-                return st;
-            if ((st = launch_gemm_bf16_simple<uint16_t>(x_bf16, wu, (int)T, Ns, L.H, su, Ns, false, stream)))
-                return st;
-            const int64_t n = T * Ns;
-            k_swiglu_f32<<<static_cast<unsigned>(std::min<int64_t>((n + 255) / 256, 148 * 32)), 256, 0,
-                           stream>>>(sg, su, sa, n);
-            if ((st = launch_status())) return st;
-            if ((st = launch_gemm_bf16_simple<float>(sa, wd, (int)T, L.H, Ns, shared, L.H, s > 0, stream)))
-                return st;
-            sm.launches += 4;
-        }
+        Bf16GemmArgs g{Wsh, (int)T, L.H, 0, sa, Wsh};
+        if ((st = launch_gemm_bf16_ws<true>(g, x_bf16, L.sh_gate, L.sh_up, L.n_shared, stream))) return st;
+        Bf16GemmArgs d{L.H, (int)T, Wsh, L.shared_N, shared, L.H};
+        if ((st = launch_gemm_bf16_ws<false>(d, sa, L.sh_down, nullptr, L.n_shared, stream))) return st;
+        sm.launches += 2;
+    }
+    sm.mark(3, stream);
+    // S4 + SwiGLU (+ S5 when fused): h = silu(G) * U, max|h| per row
+    {
+        WsGemmArgs a{sxs, L.gate_scales, L.up_scales, offsets, L.E, L.N, L.H, (int)P, h, L.N, amax,
+                     rowcnt, hq, sh, nullptr, nullptr, nullptr, k, nullptr, nullptr};
+        if ((st = launch_gemm_ws<true>(a, xs, L.gate_packed, L.up_packed, stream))) return st;
+        sm.launches += 1;
+    }
+    sm.mark(4, stream);
+    // S5
+    if (!fused) {
+        k_requant<<<static_cast<unsigned>(P), 256, 0, stream>>>(h, L.N, amax, hq, sh);
+        if ((st = launch_status())) return st;
+        sm.launches += 1;
+    }
+    sm.mark(5, stream);
+    // S6 (+ S7 when fused)
+    {
+        WsGemmArgs a{sh, L.down_scales, nullptr, offsets, L.E, L.H, L.N, (int)P, y, L.H, nullptr,
+                     tokcnt, nullptr, nullptr, sorted, rop, gates, k, shared, out_bf16};
+        if ((st = launch_gemm_ws<false>(a, hq, L.down_packed, nullptr, stream))) return st;
+        sm.launches += 1;
     }
     sm.mark(6, stream);
     // S7
-    {
+    if (!fused) {
         const int64_t n = T * (L.H / 4);
         k_combine<<<static_cast<unsigned>((n + 255) / 256), 256, 0, stream>>>(y, gates, rop, k, L.H, T,
                                                                             shared, out_bf16);
+        if ((st = launch_status())) return st;
+        sm.launches += 1;
     }
-    if ((st = launch_status())) return st;
-    sm.launches += 1;
     sm.mark(7, stream);
     return MOE_OK;
 }

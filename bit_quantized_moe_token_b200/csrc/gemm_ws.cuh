@@ -1,19 +1,21 @@
 // gemm_ws.cuh — S4/S6: warp-specialised grouped W4A8 GEMM on tcgen05 with a TMA ring.
 //
-// Roles (192 threads, one persistent CTA per SM):
-//   warps 0-3  math: thread i owns A row i = TMEM lane i.  Per K-group it widens its row of
-//              packed INT4 codes (64 B, from the TMA ring) to 128 E4M3 bytes in a 128-byte-
-//              swizzled A stage, then promotes the previous group's TMEM partial into its fp32
-//              register accumulator with the group scale; at a tile's end it runs the epilogue.
-//   warp 4     TMA producer: streams each group's packed weight tile (128 rows x 64 B) and the
-//              activation tile (BN rows x 128 B, landing pre-swizzled for the MMA) into a ring
-//              of RS stages.
-//   warp 5     MMA issuer (one lane) and TMEM owner: four (or eight) tcgen05.mma.kind::f8f6f4
-//              per group into a double-buffered TMEM partial, then commits to the barriers that
-//              release the TMEM buffer to the math warps and the ring / A stages to their
-//              producers.
+// Roles (one or two persistent CTAs per SM):
+//   widening warps (8 for narrow token tiles, 4 for wide ones): per K-group they turn the
+//              tile's packed INT4 codes (128 rows x 64 B, from the TMA ring) into 128 x 128 E4M3
+//              bytes in a 128-byte-swizzled A stage.  Four consecutive threads take the four
+//              16-byte chunks of a row, so shared-memory reads and the swizzled writes are both
+//              free of bank conflicts.  They never wait on the tensor core, only on free stages.
+//   promotion warps (4): thread i owns TMEM lane i = A row i.  Per K-group they fold the
+//              group's TMEM partial into an fp32 register accumulator with the group scale
+//              (acc += s[n,g] * partial), then run the tile's epilogue.
+//   TMA warp:  streams each group's packed weight tile and the activation tile (BN rows x
+//              128 B, landing pre-swizzled for the MMA) into a ring of RS stages.
+//   MMA warp:  one lane issues four (or eight) tcgen05.mma.kind::f8f6f4 per group into one of
+//              two TMEM partial buffers and commits to the barriers that hand the buffer to the
+//              promotion warps and release the ring / A stages; the warp also owns the TMEM.
 //
-// Widening (see gemm_tc.cuh for the arithmetic):
+// Widening (see tc_tiles.cuh for the arithmetic):
 //   kUnsigned (narrow token tiles, decode): byte = nibble = E4M3 of (code+8)*2^-9; four more
 //     MMAs per group with a constant A tile of -2^-6 (E4M3 0x88) against the same activation
 //     tile add -8*2^-9*sum_k q_k, so TMEM holds exactly 2^-9 * sum_k q_k*code_k and the
@@ -21,13 +23,13 @@
 //   signed (wide token tiles, prefill): byte = E4M3(code) by byte-permute lookup.
 //
 // Every mbarrier wait is bounded; a timeout sets a CTA-wide abort flag that turns all later
-// waits into no-ops (so the named barrier among the math warps stays uniform), records the
-// device status, and the CTA frees its TMEM and exits.
+// waits into no-ops (so the named barrier among the promotion warps stays uniform), records
+// the device status, and the CTA frees its TMEM and exits.
 #pragma once
 #include <cuda.h>
 #include "common.cuh"
 #include "tc_ptx.cuh"
-#include "gemm_tc.cuh"
+#include "tc_tiles.cuh"
 
 namespace moe {
 
@@ -40,6 +42,16 @@ struct WsGemmArgs {
     float* out;             // SwiGLU: h [P, R0]; plain: Y [P, ldo]
     int ldo;
     unsigned* amax;         // SwiGLU: [P] float bits of max|h| per row
+    // fused epilogues (narrow tiles): counters zeroed by the front kernel
+    unsigned* cnt;          // SwiGLU: [P] finished M tiles per row; plain: [T * m_tiles] per token
+    uint8_t* hq;            // SwiGLU: [P, R0] requantized activations
+    float* s_h;             // SwiGLU: [P]
+    const int32_t* sorted;  // plain: [P] pair of each sorted row
+    const int32_t* rop;     // plain: [P] sorted row of each pair
+    const float* gates;     // plain: [T, k]
+    int k;
+    const float* shared;    // plain: [T, ldo] shared-expert output or null
+    uint16_t* out_bf16;     // plain: [T, ldo] layer output
 };
 
 namespace ws {
@@ -87,17 +99,43 @@ struct WsCfg {
     static constexpr int kOffConst = kOffA + kAS * kA;          // constant -2^-6 A tile (unsigned)
     static constexpr int kOffUs = kOffConst + (kUnsigned ? kA : 0);
     static constexpr int kOffPre = kOffUs + 64 * kUsStride * 4;
-    static constexpr int kOffBar = ((kOffPre + 1025 * 4 + 7) / 8) * 8;
+    static constexpr int kOffFlag = kOffPre + 1025 * 4;          // BN ints (fused epilogues)
+    static constexpr int kOffBar = ((kOffFlag + BN * 4 + 7) / 8) * 8;
     static constexpr int kNumBars = 2 * kRS + 2 * kAS + 4;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;     // TMEM slot, abort flag
     static constexpr int kBytes = kOffMisc + 16;
     static constexpr int kAlloc = kBytes + 1024;
     static constexpr int kTmemCols = (2 * BN < 32) ? 32 : 2 * BN;
-    static constexpr int kThreads = 192;
+    static constexpr int kNW = (BN <= 32) ? 8 : 4;              // widening warps
+    static constexpr int kNP = 4;                               // promotion / epilogue warps
+    static constexpr int kWarpTma = kNW + kNP, kWarpMma = kNW + kNP + 1;
+    static constexpr int kThreads = 32 * (kNW + kNP + 2);
 };
 
-template <int BN, bool kUnsigned, bool kSwiGLU>
-__global__ void __launch_bounds__(192, WsCfg<BN, kUnsigned>::kCtasPerSm)
+// Fused decode epilogues.  Requantization (S5) of a row needs max|h| over all of its M tiles,
+// and the combine (S7) of a token needs all k routed rows: the CTA that finishes the last
+// contribution (counted with a device-scope atomic after a fence) does that work, reading the
+// other CTAs' outputs through L2.  The result does not depend on which CTA finishes last.
+__device__ __forceinline__ void requant_row(const float* __restrict__ h, int N, unsigned amax_bits,
+                                            uint8_t* __restrict__ hq, float* __restrict__ s_h, int tid) {
+    const float s = __fdiv_rn(__uint_as_float(amax_bits), kFp8Max);
+    for (int c = tid; c < (N >> 3); c += 128) {
+        uint2 codes = make_uint2(0u, 0u);
+        if (s != 0.0f) {
+            const float4 a = __ldcg(reinterpret_cast<const float4*>(h) + 2 * c);
+            const float4 b = __ldcg(reinterpret_cast<const float4*>(h) + 2 * c + 1);
+            codes.x = static_cast<uint32_t>(f32x2_to_e4m3x2(__fdiv_rn(a.x, s), __fdiv_rn(a.y, s))) |
+                      (static_cast<uint32_t>(f32x2_to_e4m3x2(__fdiv_rn(a.z, s), __fdiv_rn(a.w, s))) << 16);
+            codes.y = static_cast<uint32_t>(f32x2_to_e4m3x2(__fdiv_rn(b.x, s), __fdiv_rn(b.y, s))) |
+                      (static_cast<uint32_t>(f32x2_to_e4m3x2(__fdiv_rn(b.z, s), __fdiv_rn(b.w, s))) << 16);
+        }
+        reinterpret_cast<uint2*>(hq)[c] = codes;
+    }
+    if (tid == 0) *s_h = s;
+}
+
+template <int BN, bool kUnsigned, bool kSwiGLU, bool kFused>
+__global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUnsigned>::kCtasPerSm)
     k_gemm_w4a8_ws(const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__ CUtensorMap tm_w1,
                    const __grid_constant__ CUtensorMap tm_act, const WsGemmArgs a) {
     using C = WsCfg<BN, kUnsigned>;
@@ -108,6 +146,7 @@ __global__ void __launch_bounds__(192, WsCfg<BN, kUnsigned>::kCtasPerSm)
     uint8_t* sConst = sm + C::kOffConst;
     float* sUs = reinterpret_cast<float*>(sm + C::kOffUs);
     int* pre = reinterpret_cast<int*>(sm + C::kOffPre);
+    int* flag = reinterpret_cast<int*>(sm + C::kOffFlag);
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + C::kOffBar);
     uint64_t* raw_full = bar;
     uint64_t* raw_empty = bar + C::kRS;
@@ -127,18 +166,19 @@ __global__ void __launch_bounds__(192, WsCfg<BN, kUnsigned>::kCtasPerSm)
 
     if (tid == 0) {
         for (int i = 0; i < C::kRS; ++i) { tc::mbar_init(&raw_full[i], 1); tc::mbar_init(&raw_empty[i], 1); }
-        for (int i = 0; i < C::kAS; ++i) { tc::mbar_init(&a_full[i], 128); tc::mbar_init(&a_empty[i], 1); }
-        for (int i = 0; i < 2; ++i) { tc::mbar_init(&t_full[i], 1); tc::mbar_init(&t_empty[i], 128); }
+        for (int i = 0; i < C::kAS; ++i) { tc::mbar_init(&a_full[i], C::kNW); tc::mbar_init(&a_empty[i], 1); }
+        for (int i = 0; i < 2; ++i) { tc::mbar_init(&t_full[i], 1); tc::mbar_init(&t_empty[i], C::kNP); }
         *abort = 0;
         tc::fence_mbar_init();
     }
-    if (warp == 5) {
+    if (warp == C::kWarpMma) {
         tc::tmem_alloc(tslot, C::kTmemCols);
         tc::tmem_relinquish();
     }
-    if (kUnsigned && tid < 128) {   // constant A tile: every byte E4M3(-2^-6) = 0x88
+    if (kUnsigned && warp < C::kNW) {   // constant A tile: every byte E4M3(-2^-6) = 0x88
         uint4* c4 = reinterpret_cast<uint4*>(sConst);
-        for (int i = tid; i < C::kA / 16; i += 128) c4[i] = make_uint4(0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u);
+        for (int i = tid; i < C::kA / 16; i += 32 * C::kNW)
+            c4[i] = make_uint4(0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u);
         tc::fence_proxy_async_smem();
     }
     tc::tc_fence_before();
@@ -146,7 +186,7 @@ __global__ void __launch_bounds__(192, WsCfg<BN, kUnsigned>::kCtasPerSm)
     tc::tc_fence_after();
     const uint32_t tmem = *tslot;
 
-    if (warp == 4) {
+    if (warp == C::kWarpTma) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             ws::prefetch_map(&tm_w0);
@@ -173,7 +213,7 @@ __global__ void __launch_bounds__(192, WsCfg<BN, kUnsigned>::kCtasPerSm)
                 }
             }
         }
-    } else if (warp == 5) {
+    } else if (warp == C::kWarpMma) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc = tc::idesc_e4m3_f32(128, BN);
@@ -208,9 +248,43 @@ __global__ void __launch_bounds__(192, WsCfg<BN, kUnsigned>::kCtasPerSm)
             // arrive on this CTA's barriers is still pending
             if (it > 0) ws::wait(&raw_empty[(it - 1) % C::kRS], ((it - 1) / C::kRS) & 1, abort);
         }
+    } else if (warp < C::kNW) {
+        // ------------------------------------------------------------ widening warps
+        // Four consecutive threads widen the four 16-byte chunks of one row: a quarter warp reads
+        // 128 contiguous bytes and writes two rows whose swizzled chunks all differ.
+        constexpr int kRowsPerThread = 128 * 4 / (32 * C::kNW);
+        const int q = tid & 3;
+        const int rbase = tid >> 2;
+        uint32_t it = 0;
+        for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+            for (int g = 0; g < G; ++g, ++it) {
+                const int s = it % C::kRS, as = it % C::kAS;
+                ws::wait(&raw_full[s], (it / C::kRS) & 1, abort);
+                ws::wait(&a_empty[as], ((it / C::kAS) & 1) ^ 1, abort);
+                const uint8_t* raw = ring + s * C::kStage + C::kB;
+                uint8_t* a_st = sA + as * C::kA;
+                uint4 w[kRowsPerThread];
+#pragma unroll
+                for (int p = 0; p < kRowsPerThread; ++p)
+                    w[p] = *reinterpret_cast<const uint4*>(raw + (rbase + p * (128 / kRowsPerThread)) * 64 + q * 16);
+#pragma unroll
+                for (int p = 0; p < kRowsPerThread; ++p) {
+                    const int row = rbase + p * (128 / kRowsPerThread);
+                    const uint2 w0 = widen8<kUnsigned>(w[p].x), w1 = widen8<kUnsigned>(w[p].y);
+                    const uint2 w2 = widen8<kUnsigned>(w[p].z), w3 = widen8<kUnsigned>(w[p].w);
+                    *reinterpret_cast<uint4*>(a_st + sw128_off(row, 2 * q)) = make_uint4(w0.x, w0.y, w1.x, w1.y);
+                    *reinterpret_cast<uint4*>(a_st + sw128_off(row, 2 * q + 1)) = make_uint4(w2.x, w2.y, w3.x, w3.y);
+                }
+                tc::fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(&a_full[as]);
+            }
+        }
     } else {
-        // ------------------------------------------------------------ math warps 0-3
-        const uint32_t t_lane = static_cast<uint32_t>(warp * 32) << 16;
+        // ------------------------------------------------------------ promotion + epilogue warps
+        // Promotion warp i owns TMEM lanes 32*(i % 4) .. +31 (warp id % 4 selects the lanes).
+        const int pt = tid - 32 * C::kNW;                 // 0..127: TMEM lane = A row
+        const uint32_t t_lane = static_cast<uint32_t>((warp & 3) * 32) << 16;
         uint32_t it = 0;
         for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
             const int rt = static_cast<int>(tile / m_tiles), mt = static_cast<int>(tile % m_tiles);
@@ -219,99 +293,100 @@ __global__ void __launch_bounds__(192, WsCfg<BN, kUnsigned>::kCtasPerSm)
             const int r0 = (rt - pre[e]) * BN;
             const int nrows = min(BN, a.offsets[e + 1] - seg0 - r0);
             const int64_t row0 = seg0 + r0;
+            const int lrow = (warp & 3) * 32 + lane;       // this thread's A row / TMEM lane
             const uint16_t* ssrc;
             if (kSwiGLU) {
-                const int n = mt * 64 + (tid & 63);
-                ssrc = (tid < 64 ? a.s0 : a.s1) + ((int64_t)e * a.R0 + n) * G;
+                const int n = mt * 64 + (lrow & 63);
+                ssrc = (lrow < 64 ? a.s0 : a.s1) + ((int64_t)e * a.R0 + n) * G;
             } else {
-                ssrc = a.s0 + ((int64_t)e * a.R0 + mt * 128 + tid) * G;
+                ssrc = a.s0 + ((int64_t)e * a.R0 + mt * 128 + lrow) * G;
             }
             float acc[BN];
 #pragma unroll
             for (int j = 0; j < BN; ++j) acc[j] = 0.0f;
             float sc_next = bf16_bits_to_f32(__ldg(ssrc));
-
-            auto promote = [&](uint32_t itp, float sc) {
-                const int tb = itp & 1;
-                ws::wait(&t_full[tb], (itp >> 1) & 1, abort);
-                tc::tc_fence_after();
+            for (int g = 0; g < G; ++g, ++it) {
+                float sc = sc_next;
+                if (g + 1 < G) sc_next = bf16_bits_to_f32(__ldg(ssrc + g + 1));
                 if (kUnsigned) sc *= 512.0f;
+                const int tb = it & 1;
+                ws::wait(&t_full[tb], (it >> 1) & 1, abort);
+                tc::tc_fence_after();
 #pragma unroll
-                for (int c0 = 0; c0 < BN; c0 += (BN >= 32 ? 32 : 16)) {
-                    if constexpr (BN >= 32) {
-                        uint32_t v[32];
-                        tc::tmem_ld32(tmem + t_lane + tb * BN + c0, v);
-                        tc::tmem_wait_ld();
+                for (int c0 = 0; c0 < BN; c0 += 16) {      // 16-column loads keep few registers live
+                    uint32_t v[16];
+                    tc::tmem_ld16(tmem + t_lane + tb * BN + c0, v);
+                    tc::tmem_wait_ld();
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) acc[c0 + j] = fmaf(sc, __uint_as_float(v[j]), acc[c0 + j]);
-                    } else {
-                        uint32_t v[16];
-                        tc::tmem_ld16(tmem + t_lane + tb * BN + c0, v);
-                        tc::tmem_wait_ld();
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) acc[c0 + j] = fmaf(sc, __uint_as_float(v[j]), acc[c0 + j]);
-                    }
+                    for (int j = 0; j < 16; ++j) acc[c0 + j] = fmaf(sc, __uint_as_float(v[j]), acc[c0 + j]);
                 }
                 tc::tc_fence_before();
-                tc::mbar_arrive(&t_empty[tb]);
-            };
-
-            float sc_prev = 0.0f;
-            for (int g = 0; g < G; ++g, ++it) {
-                const int s = it % C::kRS, as = it % C::kAS;
-                const float sc = sc_next;
-                if (g + 1 < G) sc_next = bf16_bits_to_f32(__ldg(ssrc + g + 1));
-                // ---- widen group g into A stage `as` ----
-                ws::wait(&raw_full[s], (it / C::kRS) & 1, abort);
-                ws::wait(&a_empty[as], ((it / C::kAS) & 1) ^ 1, abort);
-                // four consecutive threads widen the four 16-byte chunks of one row: a quarter warp
-                // reads 128 contiguous bytes and writes two rows whose swizzled chunks differ
-                const uint8_t* raw = ring + s * C::kStage + C::kB;
-                uint8_t* a_st = sA + as * C::kA;
-                const int q = tid & 3;
-#pragma unroll
-                for (int p = 0; p < 4; ++p) {
-                    const int row = (tid >> 2) + 32 * p;
-                    const uint4 w = *reinterpret_cast<const uint4*>(raw + row * 64 + q * 16);
-                    const uint2 w0 = widen8<kUnsigned>(w.x), w1 = widen8<kUnsigned>(w.y);
-                    const uint2 w2 = widen8<kUnsigned>(w.z), w3 = widen8<kUnsigned>(w.w);
-                    *reinterpret_cast<uint4*>(a_st + sw128_off(row, 2 * q)) = make_uint4(w0.x, w0.y, w1.x, w1.y);
-                    *reinterpret_cast<uint4*>(a_st + sw128_off(row, 2 * q + 1)) = make_uint4(w2.x, w2.y, w3.x, w3.y);
-                }
-                tc::fence_proxy_async_smem();
-                tc::mbar_arrive(&a_full[as]);
-                // ---- promote group g-1 while the tensor core runs group g ----
-                if (g > 0) promote(it - 1, sc_prev);
-                sc_prev = sc;
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(&t_empty[tb]);
             }
-            promote(it - 1, sc_prev);
 
             // ---- epilogue (static indices keep acc[] in registers) ----
             if constexpr (kSwiGLU) {
-                if (tid >= 64) {
+                if (lrow >= 64) {
 #pragma unroll
-                    for (int j = 0; j < BN; ++j) sUs[(tid - 64) * C::kUsStride + j] = acc[j];
+                    for (int j = 0; j < BN; ++j) sUs[(lrow - 64) * C::kUsStride + j] = acc[j];
                 }
                 ws::named_sync_math();
-                if (tid < 64) {
-                    const int n = mt * 64 + tid;
+                if (lrow < 64) {
+                    const int n = mt * 64 + lrow;
 #pragma unroll
                     for (int j = 0; j < BN; ++j) {
                         if (j < nrows) {
                             const float sr = a.s_row[row0 + j];
-                            const float h = silu(acc[j] * sr) * (sUs[tid * C::kUsStride + j] * sr);
+                            const float h = silu(acc[j] * sr) * (sUs[lrow * C::kUsStride + j] * sr);
                             a.out[(row0 + j) * a.ldo + n] = h;
                             const float m = warp_max(fabsf(h));
                             if (lane == 0) atomicMax(a.amax + row0 + j, __float_as_uint(m));
                         }
                     }
                 }
+                if constexpr (kFused) {
+                    __threadfence();
+                    ws::named_sync_math();
+                    if (pt < nrows) flag[pt] = atomicAdd(a.cnt + row0 + pt, 1u) == (unsigned)(m_tiles - 1);
+                    ws::named_sync_math();
+                    for (int j = 0; j < nrows; ++j) {
+                        if (flag[j]) {
+                            __threadfence();
+                            const int64_t r = row0 + j;
+                            requant_row(a.out + r * a.ldo, a.ldo, __ldcg(a.amax + r), a.hq + r * a.ldo,
+                                        a.s_h + r, pt);
+                        }
+                    }
+                }
                 ws::named_sync_math();
             } else {
-                const int m = mt * 128 + tid;
+                const int m = mt * 128 + lrow;
 #pragma unroll
                 for (int j = 0; j < BN; ++j)
                     if (j < nrows) a.out[(row0 + j) * a.ldo + m] = acc[j] * a.s_row[row0 + j];
+                if constexpr (kFused) {
+                    __threadfence();
+                    ws::named_sync_math();
+                    if (pt < nrows) {
+                        const int t = a.sorted[row0 + pt] / a.k;
+                        flag[pt] = atomicAdd(a.cnt + (int64_t)t * m_tiles + mt, 1u) == (unsigned)(a.k - 1) ? t : -1;
+                    }
+                    ws::named_sync_math();
+                    for (int j = 0; j < nrows; ++j) {
+                        const int t = flag[j];
+                        if (t >= 0) {
+                            __threadfence();
+                            float o = 0.0f;
+                            for (int jj = 0; jj < a.k; ++jj)
+                                o = __fadd_rn(o, __fmul_rn(a.gates[t * a.k + jj],
+                                                           __ldcg(a.out + (int64_t)a.rop[t * a.k + jj] * a.ldo + m)));
+                            if (a.shared) o = __fadd_rn(o, a.shared[(int64_t)t * a.ldo + m]);
+                            a.out_bf16[(int64_t)t * a.ldo + m] = f32_to_bf16_bits(o);
+                        }
+                    }
+                    ws::named_sync_math();
+                }
             }
         }
     }
@@ -319,7 +394,7 @@ __global__ void __launch_bounds__(192, WsCfg<BN, kUnsigned>::kCtasPerSm)
     __syncwarp();          // single-lane roles reconverge before the CTA-wide barrier
     __syncthreads();
     if (*abort && tid == 0) atomicExch(&g_device_status, 1);
-    if (warp == 5) {
+    if (warp == C::kWarpMma) {
         tc::tc_fence_after();
         tc::tmem_dealloc(tmem, C::kTmemCols);
     }
@@ -360,14 +435,14 @@ inline bool make_map_u8(CUtensorMap* m, const void* base, uint64_t row_bytes, ui
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN, bool kUnsigned, bool kSwiGLU>
+template <int BN, bool kUnsigned, bool kSwiGLU, bool kFused>
 int launch_gemm_ws_inst(const WsGemmArgs& a, const void* act, const void* w0, const void* w1,
                         int64_t max_row_tiles, cudaStream_t stream) {
     using C = WsCfg<BN, kUnsigned>;
     static TcLaunchShape cache[16];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
-    auto kern = k_gemm_w4a8_ws<BN, kUnsigned, kSwiGLU>;
+    auto kern = k_gemm_w4a8_ws<BN, kUnsigned, kSwiGLU, kFused>;
     TcLaunchShape& c = cache[dev & 15];
     if (c.sms == 0) {
         int sms = 0;
@@ -390,16 +465,19 @@ int launch_gemm_ws_inst(const WsGemmArgs& a, const void* act, const void* w0, co
     return launch_status();
 }
 
+// Narrow token tiles (decode) fuse the requantization / combine into the GEMM epilogues.
+inline bool ws_fused(int BN) { return BN <= 32; }
+
 template <bool kSwiGLU>
 int launch_gemm_ws(const WsGemmArgs& a, const void* act, const void* w0, const void* w1,
                    cudaStream_t stream) {
     const int BN = tc_tile_rows(a.P, a.E);
     const int64_t max_row_tiles = ((int64_t)a.P + BN - 1) / BN + a.E;
     switch (BN) {
-        case 16: return launch_gemm_ws_inst<16, true, kSwiGLU>(a, act, w0, w1, max_row_tiles, stream);
-        case 32: return launch_gemm_ws_inst<32, true, kSwiGLU>(a, act, w0, w1, max_row_tiles, stream);
-        case 64: return launch_gemm_ws_inst<64, false, kSwiGLU>(a, act, w0, w1, max_row_tiles, stream);
-        default: return launch_gemm_ws_inst<128, false, kSwiGLU>(a, act, w0, w1, max_row_tiles, stream);
+        case 16: return launch_gemm_ws_inst<16, true, kSwiGLU, true>(a, act, w0, w1, max_row_tiles, stream);
+        case 32: return launch_gemm_ws_inst<32, true, kSwiGLU, true>(a, act, w0, w1, max_row_tiles, stream);
+        case 64: return launch_gemm_ws_inst<64, false, kSwiGLU, false>(a, act, w0, w1, max_row_tiles, stream);
+        default: return launch_gemm_ws_inst<128, false, kSwiGLU, false>(a, act, w0, w1, max_row_tiles, stream);
     }
 }
 

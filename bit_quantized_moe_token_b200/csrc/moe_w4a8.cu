@@ -15,7 +15,6 @@ __device__ int g_device_status = 0;
 #include "pack.cuh"
 #include "quant.cuh"
 #include "route.cuh"
-#include "gemm_simple.cuh"
 #include "forward.cuh"
 #include "tc_ptx.cuh"
 

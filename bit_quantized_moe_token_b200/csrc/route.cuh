@@ -16,13 +16,9 @@ constexpr int kSinglePassMaxP = 4096; // above this the permutation runs on one 
 // top-k: one warp per token; lane l holds experts l, l+32, ..., (EPL slots)
 // ------------------------------------------------------------------------------------------
 template <int EPL>
-__global__ void __launch_bounds__(256) k_topk(const float* __restrict__ logits, int64_t T, int E,
-                                              int k, int32_t* __restrict__ ids,
-                                              float* __restrict__ gates) {
-    const int64_t t = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
-    const int lane = threadIdx.x & 31;
-    if (t >= T) return;  // uniform per warp
-    const float* l = logits + t * E;
+__device__ __forceinline__ void topk_row(const float* __restrict__ l, int E, int k,
+                                         int32_t* __restrict__ ids, float* __restrict__ gates,
+                                         int lane) {
     float v[EPL];
     uint32_t taken = 0;
 #pragma unroll
@@ -54,7 +50,7 @@ __global__ void __launch_bounds__(256) k_topk(const float* __restrict__ logits, 
             }
         }
         if (lane == (bi & 31)) taken |= 1u << (bi >> 5);
-        if (lane == 0) ids[t * k + j] = bi;
+        if (lane == 0) ids[j] = bi;
         sel[j] = bv;
     }
     if (lane == 0) {
@@ -70,8 +66,17 @@ __global__ void __launch_bounds__(256) k_topk(const float* __restrict__ logits, 
         }
 #pragma unroll
         for (int j = 0; j < kMaxK; ++j)
-            if (j < k) gates[t * k + j] = __fdiv_rn(ex[j], sum);
+            if (j < k) gates[j] = __fdiv_rn(ex[j], sum);
     }
+}
+
+template <int EPL>
+__global__ void __launch_bounds__(256) k_topk(const float* __restrict__ logits, int64_t T, int E,
+                                              int k, int32_t* __restrict__ ids,
+                                              float* __restrict__ gates) {
+    const int64_t t = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+    if (t >= T) return;  // uniform per warp
+    topk_row<EPL>(logits + t * E, E, k, ids + t * k, gates + t * k, threadIdx.x & 31);
 }
 
 inline int launch_topk(const float* logits, int64_t T, int E, int k, int32_t* ids, float* gates,
@@ -157,12 +162,10 @@ __device__ void scatter_chunk(const int32_t* __restrict__ ids, int64_t P, int64_
     __syncthreads();
 }
 
-// Whole permutation in one CTA of 1024 threads (small P).
-__global__ void __launch_bounds__(1024) k_permute_single(const int32_t* __restrict__ ids, int64_t P,
-                                                         int E, int32_t* __restrict__ offsets,
-                                                         int32_t* __restrict__ sorted,
-                                                         int32_t* __restrict__ rop) {
-    extern __shared__ int sm[];
+// Whole permutation inside one CTA of 1024 threads (small P); `sm` holds (2E + 33 + 32E) ints.
+__device__ void permute_block(const int32_t* __restrict__ ids, int64_t P, int E,
+                              int32_t* __restrict__ offsets, int32_t* __restrict__ sorted,
+                              int32_t* __restrict__ rop, int* sm) {
     int* cnt = sm;            // E
     int* base = cnt + E;      // E
     int* wt = base + E;       // 33
@@ -175,6 +178,16 @@ __global__ void __launch_bounds__(1024) k_permute_single(const int32_t* __restri
     for (int i = threadIdx.x; i < E; i += blockDim.x) offsets[i] = base[i];
     if (threadIdx.x == 0) offsets[E] = static_cast<int32_t>(P);
     for (int64_t p0 = 0; p0 < P; p0 += kChunk) scatter_chunk(ids, P, p0, E, base, wc, sorted, rop);
+}
+
+inline size_t permute_block_smem(int E) { return (2 * E + 33 + 32 * E) * sizeof(int); }
+
+__global__ void __launch_bounds__(1024) k_permute_single(const int32_t* __restrict__ ids, int64_t P,
+                                                         int E, int32_t* __restrict__ offsets,
+                                                         int32_t* __restrict__ sorted,
+                                                         int32_t* __restrict__ rop) {
+    extern __shared__ int sm[];
+    permute_block(ids, P, E, offsets, sorted, rop, sm);
 }
 
 // Large P, pass 1: per-chunk expert histogram -> counts[c][E].
@@ -245,7 +258,7 @@ inline int launch_permute(const int32_t* ids, int64_t T, int E, int k, int32_t* 
                           int32_t* sorted, int32_t* rop, int32_t* counts, cudaStream_t stream) {
     const int64_t P = T * k;
     if (P <= kSinglePassMaxP) {
-        const size_t smem = (2 * E + 33 + 32 * E) * sizeof(int);
+        const size_t smem = permute_block_smem(E);
         if (set_smem((const void*)k_permute_single, smem)) return MOE_ERR_CUDA;
         k_permute_single<<<1, 1024, smem, stream>>>(ids, P, E, offsets, sorted, rop);
         return launch_status();

@@ -1,0 +1,101 @@
+// tc_tiles.cuh — pieces shared by the tensor-core GEMMs: INT4 -> E4M3 widening, the
+// 128-byte-swizzle address of a K-major tile, the expert-segment tile map and the token-tile
+// width choice.
+//
+// Widening.  The MMA's A operand is the group's weight tile in E4M3 (every INT4 code -8..7 is
+// an E4M3 value, so the widening is exact):
+//  * signed: byte = E4M3(code) through two byte-permute table lookups (12 integer ops per
+//    8 codes); one FMA per element promotes the group.  Used for wide token tiles (prefill).
+//  * unsigned: byte = the stored nibble itself (code + 8).  Bytes 0x00..0x0F are the E4M3
+//    values 0..15 x 2^-9 (the subnormals and the first normal binade form one equally spaced
+//    ladder), so the MMA sees 2^-9 * (code + 8) with 2-5 integer ops per 8 codes; the GEMM
+//    removes the +8 offset exactly (see gemm_ws.cuh).  Used for narrow token tiles (decode),
+//    where the widening dominates the issue slots.
+#pragma once
+#include "common.cuh"
+
+namespace moe {
+
+// ---- widening ------------------------------------------------------------------------------
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+// Eight codes of one packed word -> eight E4M3 bytes in K order (lo = codes 0..3).
+template <bool kUnsigned>
+__device__ __forceinline__ uint2 widen8(uint32_t w) {
+    if constexpr (kUnsigned) {
+        const uint32_t e = w & 0x0F0F0F0Fu;          // nibbles 0, 2, 4, 6
+        const uint32_t o = (w >> 4) & 0x0F0F0F0Fu;   // nibbles 1, 3, 5, 7
+        return make_uint2(prmt(e, o, 0x5140u), prmt(e, o, 0x7362u));
+    } else {
+        // E4M3 of code = nibble - 8: nibbles 0..7 (negative codes) and 8..15 (0..7)
+        constexpr uint32_t kNeg0 = 0xCACCCED0u, kNeg1 = 0xB8C0C4C8u;
+        constexpr uint32_t kPos0 = 0x44403800u, kPos1 = 0x4E4C4A48u;
+        const uint32_t ws = w << 4;
+        const uint32_t sl = w & 0x7777u, sh = (w >> 16) & 0x7777u;
+        // byte masks: 0xFF where the nibble's bit 3 is set (sign-replicate mode of prmt)
+        const uint32_t ml = prmt(ws, w, 0xD9C8u), mh = prmt(ws, w, 0xFBEAu);
+        const uint32_t lo = (prmt(kPos0, kPos1, sl) & ml) | (prmt(kNeg0, kNeg1, sl) & ~ml);
+        const uint32_t hi = (prmt(kPos0, kPos1, sh) & mh) | (prmt(kNeg0, kNeg1, sh) & ~mh);
+        return make_uint2(lo, hi);
+    }
+}
+
+// Byte offset of 16-byte chunk j (0..7) of row r in a K-major 128-byte-swizzled tile.
+__device__ __forceinline__ uint32_t sw128_off(int r, int j) {
+    return static_cast<uint32_t>((r >> 3) * 1024 + (r & 7) * 128 + ((j ^ (r & 7)) << 4));
+}
+
+// ---- tile map ------------------------------------------------------------------------------
+
+// Per-expert prefix of row tiles (ceil(len / BN)) into shared `pre[0..E]`; returns the total.
+__device__ int row_tile_prefix(const int32_t* __restrict__ offsets, int E, int BN, int* pre) {
+    __shared__ int s_total;
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        int run = 0;
+        for (int e0 = 0; e0 < E; e0 += 32) {
+            const int e = e0 + lane;
+            const int n = (e < E) ? (offsets[e + 1] - offsets[e] + BN - 1) / BN : 0;
+            int inc = n;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, inc, o);
+                if (lane >= o) inc += v;
+            }
+            if (e < E) pre[e] = run + inc - n;
+            run += __shfl_sync(0xffffffffu, inc, 31);
+        }
+        if (lane == 0) { pre[E] = run; s_total = run; }
+    }
+    __syncthreads();
+    return s_total;
+}
+
+// Expert owning row tile `rt` (pre[e] <= rt < pre[e+1]).
+__device__ __forceinline__ int expert_of_tile(const int* pre, int E, int rt) {
+    int lo = 0, hi = E - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (pre[mid] <= rt) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+// Launch shape of one kernel instance on one device (set once; later calls only read it).
+struct TcLaunchShape {
+    int sms = 0, ctas_per_sm = 0;
+};
+
+// Token-tile width for the expected rows per expert; narrow tiles use the unsigned widening.
+inline int tc_tile_rows(int64_t P, int E) {
+    const int64_t avg = (P + E - 1) / E;
+    return avg <= 8 ? 16 : avg <= 24 ? 32 : avg <= 64 ? 64 : 128;
+}
+inline bool tc_unsigned(int BN) { return BN <= 32; }
+
+}  // namespace moe
