@@ -40,7 +40,7 @@ class _CLayer(ctypes.Structure):
 class _CLayout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in
                 ("topk_ids", "topk_w", "expert_offsets", "sorted_pairs", "row_of_pair",
-                 "x_sorted", "s_x_sorted", "hq", "s_h", "total")]
+                 "xq", "s_x", "hq", "s_h", "total")]
 
 
 _lib = None

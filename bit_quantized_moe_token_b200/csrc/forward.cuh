@@ -65,65 +65,43 @@ __global__ void __launch_bounds__(256) k_combine(const float* __restrict__ Y,
     reinterpret_cast<uint2*>(out + t * H)[m4] = packed;
 }
 
-// Decode front end, one CTA of 1024 threads: S2 top-k (a warp per token), S3 the
-// permutation, S1 per-token FP8 quantization written straight into the token's k sorted rows
-// (a warp per token), and zeroing of the per-row / per-token counters and maxima the fused
-// GEMM epilogues accumulate into.  The arithmetic is that of k_topk / k_permute_single /
-// k_quant_tokens.
+// S1 + S2 for one token per CTA: warp 0 ranks the token's router logits (top-k, softmax
+// gate) while all threads quantize its hidden state to FP8 (amax, scale, codes), written once
+// per token; the grouped GEMM gathers the rows it needs by token index.  Same arithmetic as
+// k_topk and k_quant_tokens.
 template <int EPL>
-__global__ void __launch_bounds__(1024) k_front(const float* __restrict__ logits,
-                                                const uint16_t* __restrict__ x, int T, int E,
-                                                int k, int H, int32_t* __restrict__ ids,
-                                                float* __restrict__ gates,
-                                                int32_t* __restrict__ offsets,
-                                                int32_t* __restrict__ sorted,
-                                                int32_t* __restrict__ rop, uint8_t* __restrict__ xs,
-                                                float* __restrict__ sxs,
-                                                unsigned* __restrict__ zero, int n_zero) {
-    extern __shared__ int sm[];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int P = T * k;
-    for (int t = warp; t < T; t += 32) topk_row<EPL>(logits + (int64_t)t * E, E, k, ids + t * k, gates + t * k, lane);
-    for (int i = threadIdx.x; i < n_zero; i += blockDim.x) zero[i] = 0u;
-    __syncthreads();
-    permute_block(ids, P, E, offsets, sorted, rop, sm);
-    __syncthreads();
+__global__ void __launch_bounds__(256) k_quant_topk(const float* __restrict__ logits,
+                                                    const uint16_t* __restrict__ x, int E, int k,
+                                                    int H, int32_t* __restrict__ ids,
+                                                    float* __restrict__ gates,
+                                                    uint8_t* __restrict__ xq,
+                                                    float* __restrict__ s_x) {
+    __shared__ float red[32];
+    const int64_t t = blockIdx.x;
+    if (threadIdx.x < 32) topk_row<EPL>(logits + t * E, E, k, ids + t * k, gates + t * k, threadIdx.x);
+    const uint4* row = reinterpret_cast<const uint4*>(x + t * H);
     const int chunks = H >> 3;
-    for (int t = warp; t < T; t += 32) {
-        const uint4* row = reinterpret_cast<const uint4*>(x + (int64_t)t * H);
-        float a = 0.0f;
-        for (int c = lane; c < chunks; c += 32) a = fmaxf(a, amax8(__ldg(row + c)));
-        a = warp_max(a);
-        const float s = __fdiv_rn(a, kFp8Max);
-        for (int c = lane; c < chunks; c += 32) {
-            const uint2 codes = quant8(__ldg(row + c), s);
-            for (int j = 0; j < k; ++j)
-                reinterpret_cast<uint2*>(xs + (int64_t)rop[t * k + j] * H)[c] = codes;
-        }
-        if (lane < k) sxs[rop[t * k + lane]] = s;
-    }
+    float a = 0.0f;
+    for (int c = threadIdx.x; c < chunks; c += blockDim.x) a = fmaxf(a, amax8(__ldg(row + c)));
+    a = block_max(a, red);
+    const float s = __fdiv_rn(a, kFp8Max);
+    for (int c = threadIdx.x; c < chunks; c += blockDim.x)
+        reinterpret_cast<uint2*>(xq + t * H)[c] = quant8(__ldg(row + c), s);
+    if (threadIdx.x == 0) s_x[t] = s;
 }
 
-inline bool front_fits(int64_t T, int k) { return T <= 256 && T * k <= kSinglePassMaxP; }
-
-inline int launch_front(const float* logits, const uint16_t* x, int T, int E, int k, int H,
-                        int32_t* ids, float* gates, int32_t* offsets, int32_t* sorted, int32_t* rop,
-                        uint8_t* xs, float* sxs, unsigned* zero, int n_zero, cudaStream_t stream) {
-    const size_t smem = permute_block_smem(E);
+inline int launch_quant_topk(const float* logits, const uint16_t* x, int64_t T, int E, int k, int H,
+                             int32_t* ids, float* gates, uint8_t* xq, float* s_x, cudaStream_t stream) {
     const int epl = (E + 31) / 32;
-#define MOE_FRONT(N)                                                                             \
-    do {                                                                                         \
-        if (set_smem((const void*)k_front<N>, smem)) return MOE_ERR_CUDA;                        \
-        k_front<N><<<1, 1024, smem, stream>>>(logits, x, T, E, k, H, ids, gates, offsets, sorted, \
-                                              rop, xs, sxs, zero, n_zero);                       \
-    } while (0)
-    if (epl <= 1) MOE_FRONT(1);
-    else if (epl <= 2) MOE_FRONT(2);
-    else if (epl <= 4) MOE_FRONT(4);
-    else if (epl <= 8) MOE_FRONT(8);
-    else if (epl <= 16) MOE_FRONT(16);
-    else MOE_FRONT(32);
-#undef MOE_FRONT
+    const unsigned grid = static_cast<unsigned>(T);
+#define MOE_QT(N) k_quant_topk<N><<<grid, 256, 0, stream>>>(logits, x, E, k, H, ids, gates, xq, s_x)
+    if (epl <= 1) MOE_QT(1);
+    else if (epl <= 2) MOE_QT(2);
+    else if (epl <= 4) MOE_QT(4);
+    else if (epl <= 8) MOE_QT(8);
+    else if (epl <= 16) MOE_QT(16);
+    else MOE_QT(32);
+#undef MOE_QT
     return launch_status();
 }
 
@@ -132,7 +110,7 @@ inline int launch_front(const float* logits, const uint16_t* x, int T, int E, in
 // ------------------------------------------------------------------------------------------
 struct WsPlan {
     size_t topk_ids, topk_w, offsets, sorted, rop, route_ws;
-    size_t x_sorted, s_x_sorted, h, zero, hq, s_h, y;
+    size_t xq, s_x, x_sorted, s_x_sorted, h, zero, hq, s_h, y;
     int64_t n_zero;   // u32 words at `zero`: max|h| per row [P], row counters [P], token counters
     size_t sh_a, sh_y;
     size_t total;
@@ -153,6 +131,8 @@ inline WsPlan plan_workspace(const moe_w4a8_layer& L, int64_t T, int k) {
     p.sorted = take(P * 4);
     p.rop = take(P * 4);
     p.route_ws = take(route_ws_bytes(T, L.E, k));
+    p.xq = take((size_t)T * L.H);
+    p.s_x = take(T * 4);
     p.x_sorted = take((size_t)P * L.H);
     p.s_x_sorted = take(P * 4);
     p.h = take((size_t)P * L.N * 4);
@@ -199,8 +179,8 @@ extern "C" int moe_w4a8_workspace_layout(const moe_w4a8_layer* layer, int64_t T,
     out->expert_offsets = p.offsets;
     out->sorted_pairs = p.sorted;
     out->row_of_pair = p.rop;
-    out->x_sorted = p.x_sorted;
-    out->s_x_sorted = p.s_x_sorted;
+    out->xq = p.xq;
+    out->s_x = p.s_x;
     out->hq = p.hq;
     out->s_h = p.s_h;
     out->total = p.total;
@@ -275,6 +255,8 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const uint16_t* x_bf16,
     int32_t* offsets = (int32_t*)at(p.offsets);
     int32_t* sorted = (int32_t*)at(p.sorted);
     int32_t* rop = (int32_t*)at(p.rop);
+    uint8_t* xq = (uint8_t*)at(p.xq);
+    float* sx = (float*)at(p.s_x);
     uint8_t* xs = (uint8_t*)at(p.x_sorted);
     float* sxs = (float*)at(p.s_x_sorted);
     float* h = (float*)at(p.h);
@@ -285,26 +267,33 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const uint16_t* x_bf16,
     uint8_t* hq = (uint8_t*)at(p.hq);
     float* sh = (float*)at(p.s_h);
     float* y = (float*)at(p.y);
-    const bool fused = ws_fused(tc_tile_rows(P, L.E));
+    // narrow token tiles (decode): codes written once per token and gathered by the GEMM, fused
+    // requantization and combine; wide tiles (prefill): codes copied to expert-sorted rows.
+    const bool fused = ws_narrow(tc_tile_rows(P, L.E));
 
     sm.mark(0, stream);
-    if (front_fits(T, k)) {
-        // S2 + S3 + S1 in one CTA
-        if ((st = launch_front(router_logits, x_bf16, (int)T, L.E, k, L.H, ids, gates, offsets, sorted,
-                               rop, xs, sxs, zero, (int)p.n_zero, stream)))
+    if (fused) {
+        // S1 + S2: per-token FP8 codes and top-k
+        if ((st = launch_quant_topk(router_logits, x_bf16, T, L.E, k, L.H, ids, gates, xq, sx, stream)))
             return st;
         sm.launches += 1;
         sm.mark(1, stream);
+        // S3 (+ zeroing of the per-row maxima and the fused epilogues' counters)
+        if ((st = launch_permute(ids, T, L.E, k, offsets, sorted, rop, (int32_t*)at(p.route_ws), stream,
+                                 zero, p.n_zero)))
+            return st;
+        sm.launches += (P <= kSinglePassMaxP ? 1 : 3);
         sm.mark(2, stream);
     } else {
+        // S2 + S3 (+ zeroing)
         if ((st = launch_topk(router_logits, T, L.E, k, ids, gates, stream))) return st;
-        if ((st = launch_permute(ids, T, L.E, k, offsets, sorted, rop, (int32_t*)at(p.route_ws), stream)))
+        if ((st = launch_permute(ids, T, L.E, k, offsets, sorted, rop, (int32_t*)at(p.route_ws), stream,
+                                 zero, p.n_zero)))
             return st;
         sm.launches += 1 + (P <= kSinglePassMaxP ? 1 : 3);
         sm.mark(1, stream);
-        // S1, written straight into the expert-sorted rows
-        if ((st = launch_quant_tokens(x_bf16, T, L.H, xs, sxs, rop, k, stream))) return st;
-        if (cudaMemsetAsync(zero, 0, p.n_zero * sizeof(unsigned), stream) != cudaSuccess) return MOE_ERR_CUDA;
+        // S1, written to the token's k expert-sorted rows and to its own row
+        if ((st = launch_quant_tokens(x_bf16, T, L.H, xs, sxs, rop, k, stream, xq, sx))) return st;
         sm.launches += 1;
         sm.mark(2, stream);
     }
@@ -323,9 +312,11 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const uint16_t* x_bf16,
     sm.mark(3, stream);
     // S4 + SwiGLU (+ S5 when fused): h = silu(G) * U, max|h| per row
     {
-        WsGemmArgs a{sxs, L.gate_scales, L.up_scales, offsets, L.E, L.N, L.H, (int)P, h, L.N, amax,
-                     rowcnt, hq, sh, nullptr, nullptr, nullptr, k, nullptr, nullptr};
-        if ((st = launch_gemm_ws<true>(a, xs, L.gate_packed, L.up_packed, stream))) return st;
+        WsGemmArgs a{fused ? sx : sxs, L.gate_scales, L.up_scales, offsets, L.E, L.N, L.H, (int)P, h, L.N,
+                     amax, rowcnt, hq, sh, sorted, nullptr, nullptr, k, nullptr, nullptr, (int)T};
+        if ((st = launch_gemm_ws<true>(a, fused ? (const void*)xq : (const void*)xs, L.gate_packed,
+                                       L.up_packed, stream)))
+            return st;
         sm.launches += 1;
     }
     sm.mark(4, stream);
@@ -339,7 +330,7 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const uint16_t* x_bf16,
     // S6 (+ S7 when fused)
     {
         WsGemmArgs a{sh, L.down_scales, nullptr, offsets, L.E, L.H, L.N, (int)P, y, L.H, nullptr,
-                     tokcnt, nullptr, nullptr, sorted, rop, gates, k, shared, out_bf16};
+                     tokcnt, nullptr, nullptr, sorted, rop, gates, k, shared, out_bf16, (int)T};
         if ((st = launch_gemm_ws<false>(a, hq, L.down_packed, nullptr, stream))) return st;
         sm.launches += 1;
     }

@@ -9,8 +9,9 @@
 //   promotion warps (4): thread i owns TMEM lane i = A row i.  Per K-group they fold the
 //              group's TMEM partial into an fp32 register accumulator with the group scale
 //              (acc += s[n,g] * partial), then run the tile's epilogue.
-//   TMA warp:  streams each group's packed weight tile and the activation tile (BN rows x
-//              128 B, landing pre-swizzled for the MMA) into a ring of RS stages.
+//   TMA warp:  streams each group's packed weight tile into a ring of RW stages and the
+//              activation tile (BN rows x 128 B, landing pre-swizzled for the MMA) into a ring
+//              of RB stages; narrow gate/up tiles gather their live rows four at a time.
 //   MMA warp:  one lane issues four (or eight) tcgen05.mma.kind::f8f6f4 per group into one of
 //              two TMEM partial buffers and commits to the barriers that hand the buffer to the
 //              promotion warps and release the ring / A stages; the warp also owns the TMEM.
@@ -33,8 +34,12 @@
 
 namespace moe {
 
+// The gathering instance (gate/up on narrow token tiles) fetches its activation rows by token
+// (row r of a segment is token sorted[r] / k of the per-token FP8 array [T, K]) and takes s_row
+// per token; every other instance reads expert-sorted activation rows [P, K] directly, s_row per
+// row.
 struct WsGemmArgs {
-    const float* s_row;     // [P] per-row activation scale
+    const float* s_row;     // gathering: [T] per-token scale; otherwise [P] per-row scale
     const uint16_t* s0;     // [E, R0, K/128] bf16 scales of w0 (gate, or down)
     const uint16_t* s1;     // up scales (SwiGLU instance)
     const int32_t* offsets; // [E + 1]
@@ -46,15 +51,28 @@ struct WsGemmArgs {
     unsigned* cnt;          // SwiGLU: [P] finished M tiles per row; plain: [T * m_tiles] per token
     uint8_t* hq;            // SwiGLU: [P, R0] requantized activations
     float* s_h;             // SwiGLU: [P]
-    const int32_t* sorted;  // plain: [P] pair of each sorted row
+    const int32_t* sorted;  // [P] pair of each sorted row
     const int32_t* rop;     // plain: [P] sorted row of each pair
     const float* gates;     // plain: [T, k]
     int k;
     const float* shared;    // plain: [T, ldo] shared-expert output or null
     uint16_t* out_bf16;     // plain: [T, ldo] layer output
+    int T;                  // tokens (rows of the gathered activation tensor)
 };
 
 namespace ws {
+
+// Four rows (r0..r3) of a 2-D tensor, `box_w` wide from column x, into four consecutive
+// box rows at dst (the tensor map's box is one row high).
+__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, int x, int r0, int r1,
+                                            int r2, int r3, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];"
+        ::"r"(tc::smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(tc::smem_u32(bar)),
+          "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+        : "memory");
+}
 
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
                                             uint64_t* bar) {
@@ -86,27 +104,34 @@ __device__ __forceinline__ bool wait(uint64_t* bar, uint32_t parity, volatile in
 
 template <int BN, bool kUnsigned>
 struct WsCfg {
-    static constexpr int kRaw = 128 * 64;                       // packed codes of one group tile
-    static constexpr int kB = BN * 128;                         // activation tile
-    static constexpr int kStage = ((kB + kRaw + 1023) / 1024) * 1024;
-    static constexpr int kRS = 4;                               // ring stages
-    static constexpr int kCtasPerSm = (BN <= 32) ? 2 : 1;       // narrow tiles: 2 CTAs per SM
-    static constexpr int kAS = 2;                               // widened A stages
+    // Narrow token tiles (decode) stream weights as fast as HBM allows: the cheap unsigned
+    // widening, 8 widening warps, and for BN = 16 two persistent CTAs per SM.  Wide tiles
+    // (prefill) keep more smem for the activation tiles, one CTA per SM.
+    static constexpr bool kNarrow = BN <= 32;
+    static constexpr int kRaw = 128 * 64;                       // packed codes, one group tile
+    static constexpr int kB = BN * 128;                         // activation tile, one group
+    static constexpr int kBSlot = ((kB + 1023) / 1024) * 1024;
+    static constexpr int kCtasPerSm = (BN <= 16) ? 2 : 1;       // BN = 16: two CTAs per SM
+    static constexpr int kRW = (BN <= 16) ? 5 : kNarrow ? 12 : (BN <= 64 ? 8 : 6);   // weight ring
+    static constexpr int kRB = (BN <= 16) ? 3 : kNarrow ? 4 : 3;                  // activation ring
+    static constexpr int kAS = (BN <= 16) ? 2 : 3;                                 // widened A stages
+    static constexpr int kNT = kNarrow ? 8 : 4;                 // TMEM partial buffers
     static constexpr int kA = 128 * 128;
     static constexpr int kUsStride = BN + 1;
-    static constexpr int kOffRing = 0;
-    static constexpr int kOffA = kOffRing + kRS * kStage;
+    static constexpr int kOffB = 0;
+    static constexpr int kOffA = kOffB + kRB * kBSlot;
     static constexpr int kOffConst = kOffA + kAS * kA;          // constant -2^-6 A tile (unsigned)
-    static constexpr int kOffUs = kOffConst + (kUnsigned ? kA : 0);
+    static constexpr int kOffW = kOffConst + (kUnsigned ? kA : 0);
+    static constexpr int kOffUs = kOffW + kRW * kRaw;
     static constexpr int kOffPre = kOffUs + 64 * kUsStride * 4;
     static constexpr int kOffFlag = kOffPre + 1025 * 4;          // BN ints (fused epilogues)
     static constexpr int kOffBar = ((kOffFlag + BN * 4 + 7) / 8) * 8;
-    static constexpr int kNumBars = 2 * kRS + 2 * kAS + 4;
+    static constexpr int kNumBars = 2 * kRW + 2 * kRB + 2 * kAS + 2 * kNT;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;     // TMEM slot, abort flag
     static constexpr int kBytes = kOffMisc + 16;
     static constexpr int kAlloc = kBytes + 1024;
-    static constexpr int kTmemCols = (2 * BN < 32) ? 32 : 2 * BN;
-    static constexpr int kNW = (BN <= 32) ? 8 : 4;              // widening warps
+    static constexpr int kTmemCols = (kNT * BN < 32) ? 32 : kNT * BN;   // a power of two
+    static constexpr int kNW = kNarrow ? 8 : 4;                 // widening warps
     static constexpr int kNP = 4;                               // promotion / epilogue warps
     static constexpr int kWarpTma = kNW + kNP, kWarpMma = kNW + kNP + 1;
     static constexpr int kThreads = 32 * (kNW + kNP + 2);
@@ -134,26 +159,29 @@ __device__ __forceinline__ void requant_row(const float* __restrict__ h, int N, 
     if (tid == 0) *s_h = s;
 }
 
-template <int BN, bool kUnsigned, bool kSwiGLU, bool kFused>
+template <int BN, bool kUnsigned, bool kSwiGLU, bool kFused, bool kGather>
 __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUnsigned>::kCtasPerSm)
     k_gemm_w4a8_ws(const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__ CUtensorMap tm_w1,
                    const __grid_constant__ CUtensorMap tm_act, const WsGemmArgs a) {
     using C = WsCfg<BN, kUnsigned>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* ring = sm + C::kOffRing;
+    uint8_t* bring = sm + C::kOffB;
+    uint8_t* wring = sm + C::kOffW;
     uint8_t* sA = sm + C::kOffA;
     uint8_t* sConst = sm + C::kOffConst;
     float* sUs = reinterpret_cast<float*>(sm + C::kOffUs);
     int* pre = reinterpret_cast<int*>(sm + C::kOffPre);
     int* flag = reinterpret_cast<int*>(sm + C::kOffFlag);
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + C::kOffBar);
-    uint64_t* raw_full = bar;
-    uint64_t* raw_empty = bar + C::kRS;
-    uint64_t* a_full = bar + 2 * C::kRS;
-    uint64_t* a_empty = a_full + C::kAS;
-    uint64_t* t_full = a_empty + C::kAS;
-    uint64_t* t_empty = t_full + 2;
+    uint64_t* w_full = bar;                       // weight ring: TMA -> widening warps
+    uint64_t* w_empty = w_full + C::kRW;          //              widening warps -> TMA
+    uint64_t* b_full = w_empty + C::kRW;          // activation ring: TMA -> MMA
+    uint64_t* b_empty = b_full + C::kRB;          //                  MMA commit -> TMA
+    uint64_t* a_full = b_empty + C::kRB;          // widened A: widening warps -> MMA
+    uint64_t* a_empty = a_full + C::kAS;          //            MMA commit -> widening warps
+    uint64_t* t_full = a_empty + C::kAS;          // TMEM partials: MMA commit -> promotion
+    uint64_t* t_empty = t_full + C::kNT;          //                promotion -> MMA
     uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + C::kOffMisc);
     volatile int* abort = reinterpret_cast<volatile int*>(sm + C::kOffMisc + 4);
 
@@ -165,9 +193,10 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
     if ((int64_t)blockIdx.x >= n_tiles) return;
 
     if (tid == 0) {
-        for (int i = 0; i < C::kRS; ++i) { tc::mbar_init(&raw_full[i], 1); tc::mbar_init(&raw_empty[i], 1); }
+        for (int i = 0; i < C::kRW; ++i) { tc::mbar_init(&w_full[i], 1); tc::mbar_init(&w_empty[i], C::kNW); }
+        for (int i = 0; i < C::kRB; ++i) { tc::mbar_init(&b_full[i], 1); tc::mbar_init(&b_empty[i], 1); }
         for (int i = 0; i < C::kAS; ++i) { tc::mbar_init(&a_full[i], C::kNW); tc::mbar_init(&a_empty[i], 1); }
-        for (int i = 0; i < 2; ++i) { tc::mbar_init(&t_full[i], 1); tc::mbar_init(&t_empty[i], C::kNP); }
+        for (int i = 0; i < C::kNT; ++i) { tc::mbar_init(&t_full[i], 1); tc::mbar_init(&t_empty[i], C::kNP); }
         *abort = 0;
         tc::fence_mbar_init();
     }
@@ -188,30 +217,60 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
 
     if (warp == C::kWarpTma) {
         // ------------------------------------------------------------ TMA producer
+        // Lane 0 owns the barriers and the weight tiles.  Activation tiles are either a box of
+        // BN expert-sorted rows, or (kGather) only the tile's live token rows, four per
+        // tile::gather4 issued by lanes 0..; rows past the segment are never read back.
         if (lane == 0) {
             ws::prefetch_map(&tm_w0);
             if (kSwiGLU) ws::prefetch_map(&tm_w1);
             ws::prefetch_map(&tm_act);
-            uint32_t it = 0;
-            for (int64_t tile = blockIdx.x; tile < n_tiles && !*abort; tile += gridDim.x) {
-                const int rt = static_cast<int>(tile / m_tiles), mt = static_cast<int>(tile % m_tiles);
-                const int e = expert_of_tile(pre, a.E, rt);
-                const int row0 = a.offsets[e] + (rt - pre[e]) * BN;
-                for (int g = 0; g < G; ++g, ++it) {
-                    const int s = it % C::kRS;
-                    if (!ws::wait(&raw_empty[s], ((it / C::kRS) & 1) ^ 1, abort)) break;
-                    uint8_t* st = ring + s * C::kStage;
-                    tc::mbar_arrive_expect_tx(&raw_full[s], C::kB + C::kRaw);
-                    ws::tma_load_2d(st, &tm_act, g * kGroup, row0, &raw_full[s]);
-                    if (kSwiGLU) {
-                        const int y = e * a.R0 + mt * 64;
-                        ws::tma_load_2d(st + C::kB, &tm_w0, g * 64, y, &raw_full[s]);
-                        ws::tma_load_2d(st + C::kB + 64 * 64, &tm_w1, g * 64, y, &raw_full[s]);
-                    } else {
-                        ws::tma_load_2d(st + C::kB, &tm_w0, g * 64, e * a.R0 + mt * 128, &raw_full[s]);
+        }
+        uint32_t it = 0;
+        for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+            if (__shfl_sync(0xffffffffu, *abort, 0)) break;
+            const int rt = static_cast<int>(tile / m_tiles), mt = static_cast<int>(tile % m_tiles);
+            const int e = expert_of_tile(pre, a.E, rt);
+            const int row0 = a.offsets[e] + (rt - pre[e]) * BN;
+            const int nrows = min(BN, a.offsets[e + 1] - row0);
+            const int ngather = (nrows + 3) / 4;
+            int tok[4] = {0, 0, 0, 0};
+            if (kGather && lane < ngather) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) tok[i] = a.sorted[row0 + min(4 * lane + i, nrows - 1)] / a.k;
+            }
+            const uint32_t b_bytes = kGather ? static_cast<uint32_t>(ngather) * 512u : C::kB;
+            bool stop = false;
+            for (int g = 0; g < G; ++g, ++it) {
+                const int ws_ = it % C::kRW, bs = it % C::kRB;
+                int ok = 1;
+                if (lane == 0) {
+                    ok = ws::wait(&w_empty[ws_], ((it / C::kRW) & 1) ^ 1, abort);
+                    if (ok) {
+                        uint8_t* wst = wring + ws_ * C::kRaw;
+                        tc::mbar_arrive_expect_tx(&w_full[ws_], C::kRaw);
+                        if (kSwiGLU) {
+                            const int y = e * a.R0 + mt * 64;
+                            ws::tma_load_2d(wst, &tm_w0, g * 64, y, &w_full[ws_]);
+                            ws::tma_load_2d(wst + 64 * 64, &tm_w1, g * 64, y, &w_full[ws_]);
+                        } else {
+                            ws::tma_load_2d(wst, &tm_w0, g * 64, e * a.R0 + mt * 128, &w_full[ws_]);
+                        }
+                        ok = ws::wait(&b_empty[bs], ((it / C::kRB) & 1) ^ 1, abort);
+                        if (ok) tc::mbar_arrive_expect_tx(&b_full[bs], b_bytes);
                     }
                 }
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) { stop = true; break; }
+                uint8_t* bst = bring + bs * C::kBSlot;
+                if (kGather) {
+                    if (lane < ngather)
+                        ws::tma_gather4(bst + lane * 512, &tm_act, g * kGroup, tok[0], tok[1], tok[2], tok[3],
+                                        &b_full[bs]);
+                } else if (lane == 0) {
+                    ws::tma_load_2d(bst, &tm_act, g * kGroup, row0, &b_full[bs]);
+                }
             }
+            if (stop) break;
         }
     } else if (warp == C::kWarpMma) {
         // ------------------------------------------------------------ MMA issuer
@@ -220,12 +279,12 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
             uint32_t it = 0;
             for (int64_t tile = blockIdx.x; tile < n_tiles && !*abort; tile += gridDim.x) {
                 for (int g = 0; g < G; ++g, ++it) {
-                    const int s = it % C::kRS, as = it % C::kAS, tb = it & 1;
-                    if (!ws::wait(&raw_full[s], (it / C::kRS) & 1, abort)) break;
+                    const int bs = it % C::kRB, as = it % C::kAS, tb = it % C::kNT;
+                    if (!ws::wait(&b_full[bs], (it / C::kRB) & 1, abort)) break;
                     if (!ws::wait(&a_full[as], (it / C::kAS) & 1, abort)) break;
-                    if (!ws::wait(&t_empty[tb], ((it >> 1) & 1) ^ 1, abort)) break;
+                    if (!ws::wait(&t_empty[tb], ((it / C::kNT) & 1) ^ 1, abort)) break;
                     tc::tc_fence_after();
-                    const uint32_t b_addr = tc::smem_u32(ring + s * C::kStage);
+                    const uint32_t b_addr = tc::smem_u32(bring + bs * C::kBSlot);
                     const uint32_t a_addr = tc::smem_u32(sA + as * C::kA);
                     const uint32_t d = tmem + tb * BN;
 #pragma unroll
@@ -241,12 +300,12 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
                     }
                     tc::mma_commit(&t_full[tb]);
                     tc::mma_commit(&a_empty[as]);
-                    tc::mma_commit(&raw_empty[s]);
+                    tc::mma_commit(&b_empty[bs]);
                 }
             }
             // the commits complete in order: once the last one has arrived, no tensor-core
             // arrive on this CTA's barriers is still pending
-            if (it > 0) ws::wait(&raw_empty[(it - 1) % C::kRS], ((it - 1) / C::kRS) & 1, abort);
+            if (it > 0) ws::wait(&b_empty[(it - 1) % C::kRB], ((it - 1) / C::kRB) & 1, abort);
         }
     } else if (warp < C::kNW) {
         // ------------------------------------------------------------ widening warps
@@ -258,15 +317,18 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
         uint32_t it = 0;
         for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
             for (int g = 0; g < G; ++g, ++it) {
-                const int s = it % C::kRS, as = it % C::kAS;
-                ws::wait(&raw_full[s], (it / C::kRS) & 1, abort);
-                ws::wait(&a_empty[as], ((it / C::kAS) & 1) ^ 1, abort);
-                const uint8_t* raw = ring + s * C::kStage + C::kB;
-                uint8_t* a_st = sA + as * C::kA;
+                const int ws_ = it % C::kRW, as = it % C::kAS;
+                ws::wait(&w_full[ws_], (it / C::kRW) & 1, abort);
+                const uint8_t* raw = wring + ws_ * C::kRaw;
                 uint4 w[kRowsPerThread];
 #pragma unroll
                 for (int p = 0; p < kRowsPerThread; ++p)
                     w[p] = *reinterpret_cast<const uint4*>(raw + (rbase + p * (128 / kRowsPerThread)) * 64 + q * 16);
+                tc::fence_proxy_async_smem();              // order these reads before the next TMA write
+                __syncwarp();                              // this warp's reads of the slot are done
+                if (lane == 0) tc::mbar_arrive(&w_empty[ws_]);
+                ws::wait(&a_empty[as], ((it / C::kAS) & 1) ^ 1, abort);
+                uint8_t* a_st = sA + as * C::kA;
 #pragma unroll
                 for (int p = 0; p < kRowsPerThread; ++p) {
                     const int row = rbase + p * (128 / kRowsPerThread);
@@ -309,8 +371,8 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
                 float sc = sc_next;
                 if (g + 1 < G) sc_next = bf16_bits_to_f32(__ldg(ssrc + g + 1));
                 if (kUnsigned) sc *= 512.0f;
-                const int tb = it & 1;
-                ws::wait(&t_full[tb], (it >> 1) & 1, abort);
+                const int tb = it % C::kNT;
+                ws::wait(&t_full[tb], (it / C::kNT) & 1, abort);
                 tc::tc_fence_after();
 #pragma unroll
                 for (int c0 = 0; c0 < BN; c0 += 16) {      // 16-column loads keep few registers live
@@ -337,7 +399,7 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
 #pragma unroll
                     for (int j = 0; j < BN; ++j) {
                         if (j < nrows) {
-                            const float sr = a.s_row[row0 + j];
+                            const float sr = kGather ? a.s_row[a.sorted[row0 + j] / a.k] : a.s_row[row0 + j];
                             const float h = silu(acc[j] * sr) * (sUs[lrow * C::kUsStride + j] * sr);
                             a.out[(row0 + j) * a.ldo + n] = h;
                             const float m = warp_max(fabsf(h));
@@ -435,14 +497,14 @@ inline bool make_map_u8(CUtensorMap* m, const void* base, uint64_t row_bytes, ui
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN, bool kUnsigned, bool kSwiGLU, bool kFused>
+template <int BN, bool kUnsigned, bool kSwiGLU, bool kFused, bool kGather>
 int launch_gemm_ws_inst(const WsGemmArgs& a, const void* act, const void* w0, const void* w1,
                         int64_t max_row_tiles, cudaStream_t stream) {
     using C = WsCfg<BN, kUnsigned>;
     static TcLaunchShape cache[16];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
-    auto kern = k_gemm_w4a8_ws<BN, kUnsigned, kSwiGLU, kFused>;
+    auto kern = k_gemm_w4a8_ws<BN, kUnsigned, kSwiGLU, kFused, kGather>;
     TcLaunchShape& c = cache[dev & 15];
     if (c.sms == 0) {
         int sms = 0;
@@ -456,7 +518,7 @@ int launch_gemm_ws_inst(const WsGemmArgs& a, const void* act, const void* w0, co
     const int rows_per_load = kSwiGLU ? 64 : 128;
     if (!make_map_u8(&m0, w0, a.K / 2, (uint64_t)a.E * a.R0, 64, rows_per_load, false) ||
         !make_map_u8(&m1, kSwiGLU ? w1 : w0, a.K / 2, (uint64_t)a.E * a.R0, 64, rows_per_load, false) ||
-        !make_map_u8(&mact, act, a.K, (uint64_t)a.P, 128, BN, true))
+        !make_map_u8(&mact, act, a.K, kGather ? (uint64_t)a.T : (uint64_t)a.P, 128, kGather ? 1 : BN, true))
         return MOE_ERR_CUDA;
     const int m_tiles = kSwiGLU ? a.R0 / 64 : a.R0 / 128;
     const int64_t grid = std::max<int64_t>(
@@ -465,8 +527,9 @@ int launch_gemm_ws_inst(const WsGemmArgs& a, const void* act, const void* w0, co
     return launch_status();
 }
 
-// Narrow token tiles (decode) fuse the requantization / combine into the GEMM epilogues.
-inline bool ws_fused(int BN) { return BN <= 32; }
+// Narrow token tiles (decode) fuse the requantization / combine into the GEMM epilogues, and
+// their gate/up instance gathers activation rows by token from the per-token FP8 array.
+inline bool ws_narrow(int BN) { return BN <= 32; }
 
 template <bool kSwiGLU>
 int launch_gemm_ws(const WsGemmArgs& a, const void* act, const void* w0, const void* w1,
@@ -474,10 +537,10 @@ int launch_gemm_ws(const WsGemmArgs& a, const void* act, const void* w0, const v
     const int BN = tc_tile_rows(a.P, a.E);
     const int64_t max_row_tiles = ((int64_t)a.P + BN - 1) / BN + a.E;
     switch (BN) {
-        case 16: return launch_gemm_ws_inst<16, true, kSwiGLU, true>(a, act, w0, w1, max_row_tiles, stream);
-        case 32: return launch_gemm_ws_inst<32, true, kSwiGLU, true>(a, act, w0, w1, max_row_tiles, stream);
-        case 64: return launch_gemm_ws_inst<64, false, kSwiGLU, false>(a, act, w0, w1, max_row_tiles, stream);
-        default: return launch_gemm_ws_inst<128, false, kSwiGLU, false>(a, act, w0, w1, max_row_tiles, stream);
+        case 16: return launch_gemm_ws_inst<16, true, kSwiGLU, true, kSwiGLU>(a, act, w0, w1, max_row_tiles, stream);
+        case 32: return launch_gemm_ws_inst<32, true, kSwiGLU, true, kSwiGLU>(a, act, w0, w1, max_row_tiles, stream);
+        case 64: return launch_gemm_ws_inst<64, false, kSwiGLU, false, false>(a, act, w0, w1, max_row_tiles, stream);
+        default: return launch_gemm_ws_inst<128, false, kSwiGLU, false, false>(a, act, w0, w1, max_row_tiles, stream);
     }
 }
 

@@ -1,7 +1,7 @@
 // pack.cuh — S0: symmetric RTN INT4 quantization into pack-quantized storage.
 //
-// "Inkling-Small: GPTQ W4A8-FP8 creation and INT4 export recovery", section 1 ("Symmetric
-// INT4, groups of 128") and section 7 "Recover and physically pack INT4" (nibble = code + 8,
+// "Inkling-Small: GPTQ W4A8-FP8 creation and INT4 export recovery", section 1 (symmetric
+// INT4 in 128-wide groups) and section 7 "Recover and physically pack INT4" (nibble = code + 8,
 // eight codes along K per little-endian I32, first code in the least significant nibble).
 #pragma once
 #include "common.cuh"

@@ -1,5 +1,5 @@
-// quant.cuh — S1: dynamic per-token FP8 E4M3 quantization ("Dynamic FP8, token strategy",
-// Inkling-Small W4A8-G128 card, section 1).  scale = amax / 448, q = e4m3_rn_sat(x / scale).
+// quant.cuh — S1: dynamic per-token FP8 E4M3 quantization (Inkling-Small W4A8-G128 card,
+// section 1: FP8 input activations scaled per token at run time).  scale = amax / 448, q = e4m3_rn_sat(x / scale).
 #pragma once
 #include "common.cuh"
 
@@ -47,13 +47,14 @@ __device__ __forceinline__ float amax8(uint4 v) {
 }
 
 // One CTA per token row.  With `row_of_pair` non-null the codes and scale of token t are
-// written to its k expert-sorted rows (the forward's gathered activation matrix); otherwise
-// to row t.
+// written to its k expert-sorted rows (the forward's gathered activation matrix) and, when
+// q_tok / s_tok are non-null, also to row t of those; otherwise to row t of q / scale.
 __global__ void __launch_bounds__(256) k_quant_tokens(const uint16_t* __restrict__ x, int H,
                                                       uint8_t* __restrict__ q,
                                                       float* __restrict__ scale,
                                                       const int32_t* __restrict__ row_of_pair,
-                                                      int k) {
+                                                      int k, uint8_t* __restrict__ q_tok,
+                                                      float* __restrict__ s_tok) {
     __shared__ float red[32];
     const int64_t t = blockIdx.x;
     const uint4* row = reinterpret_cast<const uint4*>(x + t * H);
@@ -69,16 +70,20 @@ __global__ void __launch_bounds__(256) k_quant_tokens(const uint16_t* __restrict
             const int64_t r = row_of_pair ? row_of_pair[t * k + j] : t;
             reinterpret_cast<uint2*>(q + r * H)[c] = codes;
         }
+        if (q_tok) reinterpret_cast<uint2*>(q_tok + t * H)[c] = codes;
     }
-    if (threadIdx.x == 0)
+    if (threadIdx.x == 0) {
         for (int j = 0; j < ncopy; ++j) scale[row_of_pair ? row_of_pair[t * k + j] : t] = s;
+        if (s_tok) s_tok[t] = s;
+    }
 }
 
 inline int launch_quant_tokens(const uint16_t* x, int64_t T, int64_t H, uint8_t* q, float* s,
-                               const int32_t* row_of_pair, int k, cudaStream_t stream) {
+                               const int32_t* row_of_pair, int k, cudaStream_t stream,
+                               uint8_t* q_tok = nullptr, float* s_tok = nullptr) {
     if (T == 0) return MOE_OK;
     k_quant_tokens<<<static_cast<unsigned>(T), 256, 0, stream>>>(x, static_cast<int>(H), q, s,
-                                                                 row_of_pair, k);
+                                                                 row_of_pair, k, q_tok, s_tok);
     return launch_status();
 }
 

@@ -1,7 +1,7 @@
 // route.cuh — S2 top-k routing with a softmax over the selected logits, and S3 the stable
-// permutation of routed pairs into per-expert segments ("256 routed experts/layer, 6
-// active", Inkling-512k-NVFP4-AQLM-hybrid card; pairs grouped per expert for the fused
-// grouped GEMM, same card, "Serving").
+// permutation of routed pairs into per-expert segments (Inkling-512k-NVFP4-AQLM-hybrid card:
+// 256 routed experts per layer with 6 active, opening paragraph; its fused MoE kernels run
+// all experts of a layer in one grouped GEMM, section "Serving").
 #pragma once
 #include "common.cuh"
 
@@ -185,8 +185,10 @@ inline size_t permute_block_smem(int E) { return (2 * E + 33 + 32 * E) * sizeof(
 __global__ void __launch_bounds__(1024) k_permute_single(const int32_t* __restrict__ ids, int64_t P,
                                                          int E, int32_t* __restrict__ offsets,
                                                          int32_t* __restrict__ sorted,
-                                                         int32_t* __restrict__ rop) {
+                                                         int32_t* __restrict__ rop,
+                                                         unsigned* __restrict__ zero, int64_t n_zero) {
     extern __shared__ int sm[];
+    for (int64_t i = threadIdx.x; i < n_zero; i += blockDim.x) zero[i] = 0u;
     permute_block(ids, P, E, offsets, sorted, rop, sm);
 }
 
@@ -254,15 +256,19 @@ inline int set_smem(const void* fn, size_t bytes) {
                                 static_cast<int>(bytes)) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
+// Also zeroes `n_zero` words at `zero` (may be null) for the forward's accumulators.
 inline int launch_permute(const int32_t* ids, int64_t T, int E, int k, int32_t* offsets,
-                          int32_t* sorted, int32_t* rop, int32_t* counts, cudaStream_t stream) {
+                          int32_t* sorted, int32_t* rop, int32_t* counts, cudaStream_t stream,
+                          unsigned* zero = nullptr, int64_t n_zero = 0) {
     const int64_t P = T * k;
     if (P <= kSinglePassMaxP) {
         const size_t smem = permute_block_smem(E);
         if (set_smem((const void*)k_permute_single, smem)) return MOE_ERR_CUDA;
-        k_permute_single<<<1, 1024, smem, stream>>>(ids, P, E, offsets, sorted, rop);
+        k_permute_single<<<1, 1024, smem, stream>>>(ids, P, E, offsets, sorted, rop, zero, n_zero);
         return launch_status();
     }
+    if (zero && cudaMemsetAsync(zero, 0, n_zero * sizeof(unsigned), stream) != cudaSuccess)
+        return MOE_ERR_CUDA;
     const int64_t nchunks = (P + kChunk - 1) / kChunk;
     k_chunk_hist<<<static_cast<unsigned>(nchunks), 1024, E * sizeof(int), stream>>>(ids, P, E, counts);
     k_chunk_scan<<<1, 1024, (2 * E + 33) * sizeof(int), stream>>>(counts, nchunks, P, E, offsets);

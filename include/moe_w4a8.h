@@ -4,9 +4,9 @@
  * The layer is the routed MoE block of an Inkling-class model whose experts are stored as
  * symmetric INT4 weights in K-groups of 128 and run on FP8 E4M3 activations quantized per
  * token ("Inkling-Small: GPTQ W4A8-FP8 creation and INT4 export recovery" model card,
- * section 1 "What is being created?": "Symmetric INT4, groups of 128", "Dynamic FP8, token
- * strategy"; W4A8-FP8 = four-bit integer weights with eight-bit floating-point input
- * activations).  256 routed experts with 6 active per token and the gate|up / down expert
+ * section 1 "What is being created?": its table gives symmetric INT4 weights with 128-wide
+ * groups and dynamic FP8 input activations with a per-token scale, and the text defines
+ * W4A8-FP8 as 4-bit integer weights with 8-bit floating-point input activations).  256 routed experts with 6 active per token and the gate|up / down expert
  * projections come from the "Inkling-512k-NVFP4-AQLM-hybrid" model card (opening paragraph
  * and "On-disk tensor format").
  *
@@ -51,8 +51,8 @@ typedef enum {
 /* ---------------------------------------------------------------------------------------
  * S0. Offline weight quantization to pack-quantized INT4.
  *
- * Defined by the "Inkling-Small ... model card", section 1 ("Symmetric INT4, groups of 128")
- * and section 7 "Recover and physically pack INT4" (codes in [-8,7] stored as the nibble
+ * Defined by the "Inkling-Small ... model card", section 1 (symmetric INT4 in 128-wide
+ * groups) and section 7 "Recover and physically pack INT4" (codes in [-8,7] stored as the nibble
  * code+8; eight consecutive codes along the last dimension in one little-endian I32 word,
  * the first code in the least significant nibble; `.weight_packed` I32 of shape
  * [rows, K/8]).  Scales are stored as bf16 [rows, K/group] (the export's non-I8 payload is
@@ -72,8 +72,8 @@ int w4a8_pack_weights(const uint16_t* w_bf16, int64_t rows, int64_t K, int group
                       int32_t* packed, uint16_t* scales_bf16, moe_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------
- * S1. Dynamic per-token FP8 quantization ("Dynamic FP8, token strategy", section 1 of the
- * Inkling-Small card).  For each row t:
+ * S1. Dynamic per-token FP8 quantization (section 1 of the Inkling-Small card: FP8 input
+ * activations, scaled per token at run time).  For each row t:
  *     amax = max |x[t,:]|,  scale[t] = amax / 448,  q[t,h] = e4m3_rn_satfinite(x[t,h] / scale[t])
  * with IEEE fp32 division; a row with amax == 0 gets scale 0 and all-zero codes.
  *
@@ -88,8 +88,8 @@ int fp8_quant_tokens(const uint16_t* x_bf16, int64_t T, int64_t H, uint8_t* q_e4
 /* ---------------------------------------------------------------------------------------
  * S2 + S3. Top-k routing and the stable token permutation.
  *
- * Top-k of each row of the router logits ("256 routed experts/layer, 6 active",
- * Inkling-512k card): experts are ranked by (logit descending, index ascending); the first
+ * Top-k of each row of the router logits (the Inkling-512k card's opening paragraph: 256
+ * routed experts per layer, 6 of them active per token): experts are ranked by (logit descending, index ascending); the first
  * k are the selection, in that order.  Gates are a softmax over the selected logits:
  *     gate_j = exp(l_j - l_0) / sum_i exp(l_i - l_0)   (fp32, i, j < k).
  * The routed pairs p = t*k + j are then grouped by expert into one contiguous segment per
@@ -117,8 +117,8 @@ int moe_route_topk(const float* logits, int64_t T, int E, int k, int32_t* topk_i
  * separate gate/up projections), stacked over experts:
  *   gate_packed, up_packed  [E, N, H/8] int32     gate_scales, up_scales  [E, N, H/128] bf16
  *   down_packed             [E, H, N/8] int32     down_scales             [E, H, N/128] bf16
- * Shared experts (always on, kept in bf16 — Inkling-Small card section 1: "retained
- * multimodal/shared-expert parameters" stay BF16), n_shared may be 0 and the pointers NULL:
+ * Shared experts (always on, kept in bf16 — Inkling-Small card section 1: the shared-expert
+ * parameters are among those left in BF16), n_shared may be 0 and the pointers NULL:
  *   sh_gate, sh_up          [n_shared, shared_N, H] bf16
  *   sh_down                 [n_shared, H, shared_N] bf16
  * --------------------------------------------------------------------------------------- */
@@ -136,11 +136,11 @@ size_t moe_w4a8_workspace_bytes(const moe_w4a8_layer* layer, int64_t T, int k);
 /* Byte offsets, inside the forward workspace, of the intermediates a caller may inspect
  * after the forward completes (all in expert-sorted row order r, P = T*k rows):
  *   topk_ids [T,k] i32, topk_w [T,k] f32, expert_offsets [E+1] i32, sorted_pairs [P] i32,
- *   row_of_pair [P] i32, x_sorted [P,H] e4m3 (token codes of the row's token), s_x_sorted [P]
- *   f32, hq [P,N] e4m3 (requantized SwiGLU activations), s_h [P] f32. */
+ *   row_of_pair [P] i32, xq [T,H] e4m3 and s_x [T] f32 (the S1 codes and scales of every
+ *   token), hq [P,N] e4m3 and s_h [P] f32 (requantized SwiGLU activations, sorted rows). */
 typedef struct {
     size_t topk_ids, topk_w, expert_offsets, sorted_pairs, row_of_pair;
-    size_t x_sorted, s_x_sorted, hq, s_h;
+    size_t xq, s_x, hq, s_h;
     size_t total;
 } moe_w4a8_ws_layout;
 int moe_w4a8_workspace_layout(const moe_w4a8_layer* layer, int64_t T, int k,

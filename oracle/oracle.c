@@ -166,7 +166,7 @@ void or_unpack(const int32_t* packed, int64_t rows, int64_t K, int8_t* codes) {
 }
 
 /* ------------------------------------------------------------------------------------------ */
-/* S1: dynamic per-token FP8 ([P1] §1 "Dynamic FP8, token strategy"; reading R2).               */
+/* S1: dynamic per-token FP8 ([P1] §1: FP8 activations with a per-token scale; reading R2).   */
 /* ------------------------------------------------------------------------------------------ */
 
 static void quant_row_f32(const float* x, int64_t n, uint8_t* q, float* s_out) {

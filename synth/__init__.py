@@ -8,10 +8,9 @@ for bit, so a full-size weight set can be drawn directly in HBM while the
 oracle regenerates just the slices it checks.
 
 Workloads follow the five layer configurations of the Inkling-Small W4A8-G128
-model card ("1. What is being created?": hidden 4096, expert width 2048, 256
-routed experts; top-6 from the Inkling-512k hybrid card, "A memory-optimized
-hybrid-quantized build ... 256 routed experts/layer, 6 active"), with
-synthetic values:
+model card (section 1 "What is being created?": hidden 4096, expert width 2048,
+256 routed experts; top-6 from the opening paragraph of the Inkling-512k hybrid
+card), with synthetic values:
 
 * hidden states bf16 ~ N(0,1); where ``outliers`` is set, round(0.01*H)
   channels drawn once per workload (same for every token) are scaled x20;

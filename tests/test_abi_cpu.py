@@ -97,7 +97,7 @@ def test_forward_workspace_and_layout():
     lay = moe.moe_w4a8_workspace_layout(s, 8, 6)
     assert lay["total"] == n8
     offs = [lay[k] for k in ("topk_ids", "topk_w", "expert_offsets", "sorted_pairs", "row_of_pair",
-                             "x_sorted", "s_x_sorted", "hq", "s_h")]
+                             "xq", "s_x", "hq", "s_h")]
     assert all(o % 256 == 0 for o in offs) and len(set(offs)) == len(offs)
     assert max(offs) < n8
     assert moe.moe_w4a8_workspace_bytes(moe.layer_struct(256, 4000, 2048), 8, 6) == 0  # H % 128

@@ -44,8 +44,8 @@ def ws_views(layer, ws, T, k):
                 offsets=arr(lay["expert_offsets"], np.int32, layer.E + 1),
                 sorted_pairs=arr(lay["sorted_pairs"], np.int32, P),
                 row_of_pair=arr(lay["row_of_pair"], np.int32, P),
-                x_sorted=arr(lay["x_sorted"], np.uint8, P * layer.H).reshape(P, layer.H),
-                s_x_sorted=arr(lay["s_x_sorted"], np.float32, P),
+                xq=arr(lay["xq"], np.uint8, T * layer.H).reshape(T, layer.H),
+                s_x=arr(lay["s_x"], np.float32, T),
                 hq=arr(lay["hq"], np.uint8, P * layer.N).reshape(P, layer.N),
                 s_h=arr(lay["s_h"], np.float32, P))
 
@@ -205,10 +205,9 @@ def _run_and_compare(hl, dl, x, logits, k, check_all=True):
     for key in ("ids", "offsets", "sorted_pairs", "row_of_pair"):
         assert np.array_equal(v[key], ref[key]), key
     np.testing.assert_allclose(v["gates"], ref["gates"], rtol=1e-6)
-    # first-stage FP8: codes and scales of each sorted row's token are exact
-    tok = ref["sorted_pairs"] // k
-    assert np.array_equal(v["x_sorted"], ref["xq"][tok])
-    assert np.array_equal(v["s_x_sorted"], ref["s_x"][tok])
+    # first-stage FP8: codes and scales of every token are exact
+    assert np.array_equal(v["xq"], ref["xq"])
+    assert np.array_equal(v["s_x"], ref["s_x"])
     n_diff, frac = check_fp8_codes(v["hq"], ref["hq"])
     np.testing.assert_allclose(v["s_h"], ref["s_h"], rtol=2e-5)
     err = check_output(bits(out), ref["out"])
@@ -317,7 +316,8 @@ def test_forward_full_size_sampled(name, full_layer):
     np.testing.assert_allclose(v["gates"][toks], ref["gates"], rtol=1e-6)
     gpu_rows = v["row_of_pair"].reshape(wl.T, wl.k)[toks].reshape(-1)
     ref_rows = ref["row_of_pair"]
-    assert np.array_equal(v["x_sorted"][gpu_rows], ref["xq"][np.repeat(np.arange(len(toks)), wl.k)])
+    assert np.array_equal(v["xq"][toks], ref["xq"])
+    assert np.array_equal(v["s_x"][toks], ref["s_x"])
     check_fp8_codes(v["hq"][gpu_rows], ref["hq"][ref_rows])
     np.testing.assert_allclose(v["s_h"][gpu_rows], ref["s_h"][ref_rows], rtol=2e-5)
     check_output(outb[toks], ref["out"])
