@@ -62,3 +62,62 @@ extern "C" const char* moe_status_string(int status) {
         default: return "unknown status";
     }
 }
+
+// ---------------------------------------------------------------------------------------------
+// Allocation-free routing.  Some callers cannot allocate device memory at all (an engine whose
+// own allocator has reserved every byte of the GPU up front, a C caller with no device allocator
+// to link), so this variant of moe_route_topk takes its permutation scratch from a fixed array
+// compiled into the library instead of a caller buffer.
+// ---------------------------------------------------------------------------------------------
+namespace moe {
+
+// Per-chunk expert counts of the multi-chunk permutation: (ceil(T*k / 1024) * E) int32 words.
+constexpr size_t kRouteStaticBytes = 256 * 1024;
+static __device__ __align__(256) int32_t g_route_static_scratch[kRouteStaticBytes / sizeof(int32_t)];
+
+// Device address of the array on the current device, looked up once per device.  Host code may
+// not pass `g_route_static_scratch` itself to a kernel: on the host that name is only a stand-in.
+static int route_static_scratch(int32_t** out) {
+    static int32_t* cache[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+    if (dev < 0 || dev >= 64) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (!cache[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_route_static_scratch) != cudaSuccess || !p) return MOE_ERR_CUDA;
+        cache[dev] = static_cast<int32_t*>(p);
+    }
+    *out = cache[dev];
+    return MOE_OK;
+}
+
+}  // namespace moe
+
+extern "C" size_t moe_route_noalloc_max_scratch_bytes(void) { return moe::kRouteStaticBytes; }
+
+extern "C" int moe_route_topk_noalloc(const float* logits, int64_t T, int E, int k,
+                                      int32_t* topk_ids, float* topk_w, int32_t* expert_offsets,
+                                      int32_t* sorted_pairs, int32_t* row_of_pair,
+                                      moe_stream_t stream) {
+    using namespace moe;
+    int st = route_args_ok(T, E, k);
+    if (st != MOE_OK) return st;
+    if (!expert_offsets) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!logits || !topk_ids || !topk_w || !sorted_pairs || !row_of_pair))
+        return MOE_ERR_INVALID_ARG;
+    if (route_ws_bytes(T, E, k) > kRouteStaticBytes) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned(logits, 4) || !aligned(topk_ids, 4) || !aligned(topk_w, 4) ||
+        !aligned(expert_offsets, 4) || !aligned(sorted_pairs, 4) || !aligned(row_of_pair, 4))
+        return MOE_ERR_MISALIGNED;
+    int32_t* scratch = nullptr;
+    if ((st = route_static_scratch(&scratch)) != MOE_OK) return st;
+    if (T == 0) {
+        if (cudaMemsetAsync(expert_offsets, 0, (E + 1) * sizeof(int32_t), stream) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        return MOE_OK;
+    }
+    // every count the permutation reads is written earlier in the same call: nothing to clear
+    st = launch_topk(logits, T, E, k, topk_ids, topk_w, stream);
+    if (st != MOE_OK) return st;
+    return launch_permute(topk_ids, T, E, k, expert_offsets, sorted_pairs, row_of_pair, scratch, stream);
+}

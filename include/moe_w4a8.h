@@ -192,6 +192,24 @@ int moe_last_device_status(moe_stream_t stream);
  * without hanging a GPU. */
 int moe_selftest_bounded_wait(int64_t limit_ns, moe_stream_t stream);
 
+/* Allocation-free variant of moe_route_topk, for callers that cannot allocate device memory
+ * (an engine whose own allocator has reserved all of the GPU's memory up front, so a further
+ * allocation fails; a C caller with no device allocator to link).  There is no counterpart on
+ * the pages: it is moe_route_topk with the permutation scratch taken from a fixed array inside
+ * the library (moe_route_noalloc_max_scratch_bytes() bytes, held by every GPU that loads the
+ * library until the process exits) instead of a caller buffer; all outputs are still the
+ * caller's.  It supports shapes with moe_route_workspace_bytes(T, E, k) <= that size (for
+ * E = 256, up to 262,144 routed pairs) and returns MOE_ERR_UNSUPPORTED_SHAPE beyond it.
+ * The first call on a device looks up the array's device address (cudaGetSymbolAddress), so
+ * make that first call before any stream capture.  All calls share the one array: calls that
+ * overlap on the GPU (issued on streams with no ordering between them) race and must be
+ * serialised by the caller.  Every scratch word a call reads is written earlier in the same
+ * call, so stale contents from a previous call do not matter.  Never allocates or frees. */
+size_t moe_route_noalloc_max_scratch_bytes(void);
+int moe_route_topk_noalloc(const float* logits, int64_t T, int E, int k, int32_t* topk_ids,
+                           float* topk_w, int32_t* expert_offsets, int32_t* sorted_pairs,
+                           int32_t* row_of_pair, moe_stream_t stream);
+
 /* Static description of a status code. */
 const char* moe_status_string(int status);
 
