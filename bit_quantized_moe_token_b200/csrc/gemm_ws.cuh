@@ -6,8 +6,9 @@
 //              bytes in a 128-byte-swizzled A stage.  Four consecutive threads take the four
 //              16-byte chunks of a row, so shared-memory reads and the swizzled writes are both
 //              free of bank conflicts.  They never wait on the tensor core, only on free stages.
-//   promotion warps (4): thread i owns TMEM lane i = A row i.  Per K-group they fold the
-//              group's TMEM partial into an fp32 register accumulator with the group scale
+//   promotion warps (4 for narrow tiles, 8 for wide ones): a thread owns one TMEM lane = A row
+//              (and, with 8 warps, half of the tile's token columns).  Per K-group they fold
+//              the group's TMEM partial into an fp32 register accumulator with the group scale
 //              (acc += s[n,g] * partial), then run the tile's epilogue.
 //   TMA warp:  streams each group's packed weight tile into a ring of RW stages and the
 //              activation tile (BN rows x 128 B, landing pre-swizzled for the MMA) into a ring
@@ -88,9 +89,12 @@ __device__ __forceinline__ void prefetch_map(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
+// Named barrier 1 among the promotion / epilogue warps only.
+template <int kThreads = 128>
 __device__ __forceinline__ void named_sync_math() {
-    asm volatile("bar.sync 1, 128;" ::: "memory");
+    asm volatile("bar.sync 1, %0;" ::"n"(kThreads) : "memory");
 }
+
 
 // Bounded wait that gives up at once after an abort.
 __device__ __forceinline__ bool wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
@@ -131,9 +135,15 @@ struct WsCfg {
     static constexpr int kBytes = kOffMisc + 16;
     static constexpr int kAlloc = kBytes + 1024;
     static constexpr int kTmemCols = (kNT * BN < 32) ? 32 : kNT * BN;   // a power of two
+    // Warp roles.  Narrow: warps 0-7 widen, 8-11 promote, 12 TMA, 13 MMA.  Wide: warps 0-3
+    // widen, 4-11 promote (two warps per TMEM lane quadrant, each owning half of the token
+    // columns), 12 TMA, 13 MMA.  A promotion thread issues up to 32 columns of TMEM loads before
+    // each wait, so a 128-column group costs two load round trips.
     static constexpr int kNW = kNarrow ? 8 : 4;                 // widening warps
-    static constexpr int kNP = 4;                               // promotion / epilogue warps
+    static constexpr int kNP = kNarrow ? 4 : 8;                 // promotion / epilogue warps
+    static constexpr int kCPW = BN / (kNP / 4);                 // token columns per promotion thread
     static constexpr int kWarpTma = kNW + kNP, kWarpMma = kNW + kNP + 1;
+    static constexpr int kLd = kCPW < 32 ? kCPW : 32;          // TMEM columns per load wait
     static constexpr int kThreads = 32 * (kNW + kNP + 2);
 };
 
@@ -142,9 +152,10 @@ struct WsCfg {
 // contribution (counted with a device-scope atomic after a fence) does that work, reading the
 // other CTAs' outputs through L2.  The result does not depend on which CTA finishes last.
 __device__ __forceinline__ void requant_row(const float* __restrict__ h, int N, unsigned amax_bits,
-                                            uint8_t* __restrict__ hq, float* __restrict__ s_h, int tid) {
+                                            uint8_t* __restrict__ hq, float* __restrict__ s_h, int tid,
+                                            int nthreads) {
     const float s = __fdiv_rn(__uint_as_float(amax_bits), kFp8Max);
-    for (int c = tid; c < (N >> 3); c += 128) {
+    for (int c = tid; c < (N >> 3); c += nthreads) {
         uint2 codes = make_uint2(0u, 0u);
         if (s != 0.0f) {
             const float4 a = __ldcg(reinterpret_cast<const float4*>(h) + 2 * c);
@@ -342,10 +353,15 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
                 if (lane == 0) tc::mbar_arrive(&a_full[as]);
             }
         }
-    } else {
+    } else if (warp < C::kNW + C::kNP) {
         // ------------------------------------------------------------ promotion + epilogue warps
-        // Promotion warp i owns TMEM lanes 32*(i % 4) .. +31 (warp id % 4 selects the lanes).
-        const int pt = tid - 32 * C::kNW;                 // 0..127: TMEM lane = A row
+        // Promotion warp i owns TMEM lanes 32*(i % 4) .. +31 (warp id % 4 selects the lanes) and
+        // the token columns [ch*kCPW, (ch+1)*kCPW) of them.
+        constexpr int kCPW = C::kCPW;
+        constexpr int kNPT = 32 * C::kNP;
+        const int pt = tid - 32 * C::kNW;                 // 0 .. kNPT-1
+        const int ch = (warp - C::kNW) >> 2;              // column block of this warp
+        const int c_base = ch * kCPW;
         const uint32_t t_lane = static_cast<uint32_t>((warp & 3) * 32) << 16;
         uint32_t it = 0;
         for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
@@ -363,9 +379,9 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
             } else {
                 ssrc = a.s0 + ((int64_t)e * a.R0 + mt * 128 + lrow) * G;
             }
-            float acc[BN];
+            float acc[kCPW];
 #pragma unroll
-            for (int j = 0; j < BN; ++j) acc[j] = 0.0f;
+            for (int j = 0; j < kCPW; ++j) acc[j] = 0.0f;
             float sc_next = bf16_bits_to_f32(__ldg(ssrc));
             for (int g = 0; g < G; ++g, ++it) {
                 float sc = sc_next;
@@ -375,12 +391,15 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
                 ws::wait(&t_full[tb], (it / C::kNT) & 1, abort);
                 tc::tc_fence_after();
 #pragma unroll
-                for (int c0 = 0; c0 < BN; c0 += 16) {      // 16-column loads keep few registers live
-                    uint32_t v[16];
-                    tc::tmem_ld16(tmem + t_lane + tb * BN + c0, v);
+                for (int c1 = 0; c1 < kCPW; c1 += C::kLd) {    // kLd columns in flight per wait
+                    uint32_t v[C::kLd];
+#pragma unroll
+                    for (int c0 = 0; c0 < C::kLd; c0 += 16)
+                        tc::tmem_ld16(tmem + t_lane + tb * BN + c_base + c1 + c0,
+                                      *reinterpret_cast<uint32_t(*)[16]>(v + c0));
                     tc::tmem_wait_ld();
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) acc[c0 + j] = fmaf(sc, __uint_as_float(v[j]), acc[c0 + j]);
+                    for (int j = 0; j < C::kLd; ++j) acc[c1 + j] = fmaf(sc, __uint_as_float(v[j]), acc[c1 + j]);
                 }
                 tc::tc_fence_before();
                 __syncwarp();
@@ -391,50 +410,52 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
             if constexpr (kSwiGLU) {
                 if (lrow >= 64) {
 #pragma unroll
-                    for (int j = 0; j < BN; ++j) sUs[(lrow - 64) * C::kUsStride + j] = acc[j];
+                    for (int j = 0; j < kCPW; ++j) sUs[(lrow - 64) * C::kUsStride + c_base + j] = acc[j];
                 }
-                ws::named_sync_math();
+                ws::named_sync_math<kNPT>();
                 if (lrow < 64) {
                     const int n = mt * 64 + lrow;
 #pragma unroll
-                    for (int j = 0; j < BN; ++j) {
-                        if (j < nrows) {
-                            const float sr = kGather ? a.s_row[a.sorted[row0 + j] / a.k] : a.s_row[row0 + j];
-                            const float h = silu(acc[j] * sr) * (sUs[lrow * C::kUsStride + j] * sr);
-                            a.out[(row0 + j) * a.ldo + n] = h;
+                    for (int j = 0; j < kCPW; ++j) {
+                        if (c_base + j < nrows) {
+                            const int64_t r = row0 + c_base + j;
+                            const float sr = kGather ? a.s_row[a.sorted[r] / a.k] : a.s_row[r];
+                            const float h = silu(acc[j] * sr) * (sUs[lrow * C::kUsStride + c_base + j] * sr);
+                            a.out[r * a.ldo + n] = h;
                             const float m = warp_max(fabsf(h));
-                            if (lane == 0) atomicMax(a.amax + row0 + j, __float_as_uint(m));
+                            if (lane == 0) atomicMax(a.amax + r, __float_as_uint(m));
                         }
                     }
                 }
                 if constexpr (kFused) {
                     __threadfence();
-                    ws::named_sync_math();
+                    ws::named_sync_math<kNPT>();
                     if (pt < nrows) flag[pt] = atomicAdd(a.cnt + row0 + pt, 1u) == (unsigned)(m_tiles - 1);
-                    ws::named_sync_math();
+                    ws::named_sync_math<kNPT>();
                     for (int j = 0; j < nrows; ++j) {
                         if (flag[j]) {
                             __threadfence();
                             const int64_t r = row0 + j;
                             requant_row(a.out + r * a.ldo, a.ldo, __ldcg(a.amax + r), a.hq + r * a.ldo,
-                                        a.s_h + r, pt);
+                                        a.s_h + r, pt, kNPT);
                         }
                     }
                 }
-                ws::named_sync_math();
+                ws::named_sync_math<kNPT>();
             } else {
                 const int m = mt * 128 + lrow;
 #pragma unroll
-                for (int j = 0; j < BN; ++j)
-                    if (j < nrows) a.out[(row0 + j) * a.ldo + m] = acc[j] * a.s_row[row0 + j];
+                for (int j = 0; j < kCPW; ++j)
+                    if (c_base + j < nrows)
+                        a.out[(row0 + c_base + j) * a.ldo + m] = acc[j] * a.s_row[row0 + c_base + j];
                 if constexpr (kFused) {
                     __threadfence();
-                    ws::named_sync_math();
+                    ws::named_sync_math<kNPT>();
                     if (pt < nrows) {
                         const int t = a.sorted[row0 + pt] / a.k;
                         flag[pt] = atomicAdd(a.cnt + (int64_t)t * m_tiles + mt, 1u) == (unsigned)(a.k - 1) ? t : -1;
                     }
-                    ws::named_sync_math();
+                    ws::named_sync_math<kNPT>();
                     for (int j = 0; j < nrows; ++j) {
                         const int t = flag[j];
                         if (t >= 0) {
@@ -447,7 +468,7 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
                             a.out_bf16[(int64_t)t * a.ldo + m] = f32_to_bf16_bits(o);
                         }
                     }
-                    ws::named_sync_math();
+                    ws::named_sync_math<kNPT>();
                 }
             }
         }
