@@ -129,7 +129,8 @@ struct WsCfg {
     static constexpr int kOffUs = kOffW + kRW * kRaw;
     static constexpr int kOffPre = kOffUs + 64 * kUsStride * 4;
     static constexpr int kOffFlag = kOffPre + 1025 * 4;          // BN ints (fused epilogues)
-    static constexpr int kOffBar = ((kOffFlag + BN * 4 + 7) / 8) * 8;
+    static constexpr int kOffSr = kOffFlag + BN * 4;             // 2 x BN per-column scales
+    static constexpr int kOffBar = ((kOffSr + 2 * BN * 4 + 7) / 8) * 8;
     static constexpr int kNumBars = 2 * kRW + 2 * kRB + 2 * kAS + 2 * kNT;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;     // TMEM slot, abort flag
     static constexpr int kBytes = kOffMisc + 16;
@@ -184,6 +185,7 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
     float* sUs = reinterpret_cast<float*>(sm + C::kOffUs);
     int* pre = reinterpret_cast<int*>(sm + C::kOffPre);
     int* flag = reinterpret_cast<int*>(sm + C::kOffFlag);
+    float* sSr = reinterpret_cast<float*>(sm + C::kOffSr);
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + C::kOffBar);
     uint64_t* w_full = bar;                       // weight ring: TMA -> widening warps
     uint64_t* w_empty = w_full + C::kRW;          //              widening warps -> TMA
@@ -363,7 +365,7 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
         const int ch = (warp - C::kNW) >> 2;              // column block of this warp
         const int c_base = ch * kCPW;
         const uint32_t t_lane = static_cast<uint32_t>((warp & 3) * 32) << 16;
-        uint32_t it = 0;
+        uint32_t it = 0, tcount = 0;
         for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
             const int rt = static_cast<int>(tile / m_tiles), mt = static_cast<int>(tile % m_tiles);
             const int e = expert_of_tile(pre, a.E, rt);
@@ -372,6 +374,11 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
             const int nrows = min(BN, a.offsets[e + 1] - seg0 - r0);
             const int64_t row0 = seg0 + r0;
             const int lrow = (warp & 3) * 32 + lane;       // this thread's A row / TMEM lane
+            // token scale of column pt, fetched now and staged in shared memory for the epilogue
+            float my_sr = 0.0f;
+            if (pt < nrows) my_sr = kGather ? a.s_row[a.sorted[row0 + pt] / a.k] : a.s_row[row0 + pt];
+            float* sr_t = sSr + (tcount & 1) * BN;         // two buffers: tile parity
+            ++tcount;
             const uint16_t* ssrc;
             if (kSwiGLU) {
                 const int n = mt * 64 + (lrow & 63);
@@ -407,25 +414,36 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
             }
 
             // ---- epilogue (static indices keep acc[] in registers) ----
+            // The column scales come from shared memory, so no load waits behind the stores, and
+            // the per-column max|h| is one redux per warp.
+            if (pt < BN) sr_t[pt] = my_sr;
             if constexpr (kSwiGLU) {
-                if (lrow >= 64) {
+                // Gate warps (lrow < 64) finish the first half of the columns, up warps the second:
+                // each hands the other the half it does not finish through sUs.
+                constexpr int kHalf = kCPW / 2;
+                const bool gate = lrow < 64;
+                const int r64 = lrow & 63;
+                const int c_mine = c_base + (gate ? 0 : kHalf);
 #pragma unroll
-                    for (int j = 0; j < kCPW; ++j) sUs[(lrow - 64) * C::kUsStride + c_base + j] = acc[j];
-                }
+                for (int j = 0; j < kHalf; ++j)
+                    sUs[r64 * C::kUsStride + c_base + (gate ? kHalf : 0) + j] = gate ? acc[kHalf + j] : acc[j];
                 ws::named_sync_math<kNPT>();
-                if (lrow < 64) {
-                    const int n = mt * 64 + lrow;
+                const int n = mt * 64 + r64;
 #pragma unroll
-                    for (int j = 0; j < kCPW; ++j) {
-                        if (c_base + j < nrows) {
-                            const int64_t r = row0 + c_base + j;
-                            const float sr = kGather ? a.s_row[a.sorted[r] / a.k] : a.s_row[r];
-                            const float h = silu(acc[j] * sr) * (sUs[lrow * C::kUsStride + c_base + j] * sr);
-                            a.out[r * a.ldo + n] = h;
-                            const float m = warp_max(fabsf(h));
-                            if (lane == 0) atomicMax(a.amax + r, __float_as_uint(m));
-                        }
-                    }
+                for (int j = 0; j < kHalf; ++j) {
+                    const float sr = sr_t[c_mine + j];
+                    const float other = sUs[r64 * C::kUsStride + c_mine + j];
+                    const float gv = gate ? acc[j] : other;
+                    const float uv = gate ? other : acc[kHalf + j];
+                    acc[j] = silu(gv * sr) * (uv * sr);
+                }
+#pragma unroll
+                for (int j = 0; j < kHalf; ++j)
+                    if (c_mine + j < nrows) a.out[(row0 + c_mine + j) * a.ldo + n] = acc[j];
+#pragma unroll
+                for (int j = 0; j < kHalf; ++j) {
+                    const unsigned m = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(acc[j])));
+                    if (lane == 0 && c_mine + j < nrows) atomicMax(a.amax + row0 + c_mine + j, m);
                 }
                 if constexpr (kFused) {
                     __threadfence();
@@ -444,10 +462,10 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
                 ws::named_sync_math<kNPT>();
             } else {
                 const int m = mt * 128 + lrow;
+                ws::named_sync_math<kNPT>();
 #pragma unroll
                 for (int j = 0; j < kCPW; ++j)
-                    if (c_base + j < nrows)
-                        a.out[(row0 + c_base + j) * a.ldo + m] = acc[j] * a.s_row[row0 + c_base + j];
+                    if (c_base + j < nrows) a.out[(row0 + c_base + j) * a.ldo + m] = acc[j] * sr_t[c_base + j];
                 if constexpr (kFused) {
                     __threadfence();
                     ws::named_sync_math<kNPT>();
