@@ -116,16 +116,21 @@ struct WsCfg {
     static constexpr int kB = BN * 128;                         // activation tile, one group
     static constexpr int kBSlot = ((kB + 1023) / 1024) * 1024;
     static constexpr int kCtasPerSm = (BN <= 16) ? 2 : 1;       // BN = 16: two CTAs per SM
-    static constexpr int kRW = (BN <= 16) ? 5 : kNarrow ? 12 : (BN <= 64 ? 8 : 6);   // weight ring
-    static constexpr int kRB = (BN <= 16) ? 3 : kNarrow ? 4 : 3;                  // activation ring
-    static constexpr int kAS = (BN <= 16) ? 2 : 3;                                 // widened A stages
-    static constexpr int kNT = kNarrow ? 8 : 4;                 // TMEM partial buffers
-    static constexpr int kA = 128 * 128;
+    static constexpr int kRW = (BN <= 16) ? 10 : kNarrow ? 16 : (BN <= 64 ? 12 : 8);   // weight ring
+    static constexpr int kRB = (BN <= 16) ? 6 : kNarrow ? 8 : (BN <= 64 ? 6 : 5);     // activation ring
+    static constexpr int kAS = (BN <= 16) ? 3 : 4;                                 // widened A stages
+    static constexpr int kNT = kNarrow ? 8 : (BN <= 64 ? 4 : 3);                   // TMEM partials
+    // TMEM columns: partial buffers | widened A stages (32 columns = 128 E4M3 per row) | the
+    // constant -2^-6 tile of the unsigned widening.
+    static constexpr int kColA = kNT * BN;
+    static constexpr int kColConst = kColA + kAS * 32;
+    static constexpr int kTmemNeed = kColConst + (kUnsigned ? 32 : 0);
+    static constexpr int kTmemCols = kTmemNeed <= 32 ? 32 : kTmemNeed <= 64 ? 64 : kTmemNeed <= 128 ? 128
+                                   : kTmemNeed <= 256 ? 256 : 512;
+    static_assert(kTmemNeed <= 512 / kCtasPerSm, "TMEM budget");
     static constexpr int kUsStride = BN + 1;
     static constexpr int kOffB = 0;
-    static constexpr int kOffA = kOffB + kRB * kBSlot;
-    static constexpr int kOffConst = kOffA + kAS * kA;          // constant -2^-6 A tile (unsigned)
-    static constexpr int kOffW = kOffConst + (kUnsigned ? kA : 0);
+    static constexpr int kOffW = kOffB + kRB * kBSlot;
     static constexpr int kOffUs = kOffW + kRW * kRaw;
     static constexpr int kOffPre = kOffUs + 64 * kUsStride * 4;
     static constexpr int kOffFlag = kOffPre + 1025 * 4;          // BN ints (fused epilogues)
@@ -135,7 +140,6 @@ struct WsCfg {
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;     // TMEM slot, abort flag
     static constexpr int kBytes = kOffMisc + 16;
     static constexpr int kAlloc = kBytes + 1024;
-    static constexpr int kTmemCols = (kNT * BN < 32) ? 32 : kNT * BN;   // a power of two
     // Warp roles.  Narrow: warps 0-7 widen, 8-11 promote, 12 TMA, 13 MMA.  Wide: warps 0-3
     // widen, 4-11 promote (two warps per TMEM lane quadrant, each owning half of the token
     // columns), 12 TMA, 13 MMA.  A promotion thread issues up to 32 columns of TMEM loads before
@@ -180,8 +184,6 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* bring = sm + C::kOffB;
     uint8_t* wring = sm + C::kOffW;
-    uint8_t* sA = sm + C::kOffA;
-    uint8_t* sConst = sm + C::kOffConst;
     float* sUs = reinterpret_cast<float*>(sm + C::kOffUs);
     int* pre = reinterpret_cast<int*>(sm + C::kOffPre);
     int* flag = reinterpret_cast<int*>(sm + C::kOffFlag);
@@ -217,16 +219,22 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
         tc::tmem_alloc(tslot, C::kTmemCols);
         tc::tmem_relinquish();
     }
-    if (kUnsigned && warp < C::kNW) {   // constant A tile: every byte E4M3(-2^-6) = 0x88
-        uint4* c4 = reinterpret_cast<uint4*>(sConst);
-        for (int i = tid; i < C::kA / 16; i += 32 * C::kNW)
-            c4[i] = make_uint4(0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u);
-        tc::fence_proxy_async_smem();
-    }
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem = *tslot;
+    if constexpr (kUnsigned) {          // constant A tile: every byte E4M3(-2^-6) = 0x88
+        if (warp < 4) {
+            uint32_t cst[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) cst[i] = 0x88888888u;
+            tc::tmem_st32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + C::kColConst, cst);
+            tc::tmem_wait_st();
+        }
+        tc::tc_fence_before();
+        __syncthreads();
+        tc::tc_fence_after();
+    }
 
     if (warp == C::kWarpTma) {
         // ------------------------------------------------------------ TMA producer
@@ -298,18 +306,17 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
                     if (!ws::wait(&t_empty[tb], ((it / C::kNT) & 1) ^ 1, abort)) break;
                     tc::tc_fence_after();
                     const uint32_t b_addr = tc::smem_u32(bring + bs * C::kBSlot);
-                    const uint32_t a_addr = tc::smem_u32(sA + as * C::kA);
+                    const uint32_t a_col = tmem + C::kColA + as * 32;
                     const uint32_t d = tmem + tb * BN;
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        tc::mma_e4m3(d, tc::sdesc_sw128(a_addr + kk * 32), tc::sdesc_sw128(b_addr + kk * 32),
-                                     idesc, kk > 0 ? 1u : 0u);
+                        tc::mma_e4m3_ta(d, a_col + kk * 8, tc::sdesc_sw128(b_addr + kk * 32), idesc,
+                                        kk > 0 ? 1u : 0u);
                     if (kUnsigned) {
-                        const uint32_t c_addr = tc::smem_u32(sConst);
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)
-                            tc::mma_e4m3(d, tc::sdesc_sw128(c_addr + kk * 32),
-                                         tc::sdesc_sw128(b_addr + kk * 32), idesc, 1u);
+                            tc::mma_e4m3_ta(d, tmem + C::kColConst + kk * 8,
+                                            tc::sdesc_sw128(b_addr + kk * 32), idesc, 1u);
                     }
                     tc::mma_commit(&t_full[tb]);
                     tc::mma_commit(&a_empty[as]);
@@ -322,35 +329,46 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
         }
     } else if (warp < C::kNW) {
         // ------------------------------------------------------------ widening warps
-        // Four consecutive threads widen the four 16-byte chunks of one row: a quarter warp reads
-        // 128 contiguous bytes and writes two rows whose swizzled chunks all differ.
-        constexpr int kRowsPerThread = 128 * 4 / (32 * C::kNW);
-        const int q = tid & 3;
-        const int rbase = tid >> 2;
+        // A thread owns one A row = one TMEM lane (warp id % 4 selects the lane quadrant); on
+        // narrow tiles two warps split each row's K group.  The packed tile lands with the
+        // 64-byte TMA swizzle (16-byte chunk c of row r at chunk c ^ ((r >> 1) & 3)), so the 32
+        // rows a warp reads fall in distinct banks.
+        constexpr int kParts = C::kNW / 4;                 // warps per lane quadrant
+        constexpr int kChunks = 4 / kParts;                // 16-byte packed chunks per thread
+        const int quad = warp & 3, part = warp >> 2;
+        const int row = quad * 32 + lane;
+        const int swz = (row >> 1) & 3;
+        const uint32_t t_dst = tmem + (static_cast<uint32_t>(quad * 32) << 16) + C::kColA + part * 8 * kChunks;
         uint32_t it = 0;
         for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
             for (int g = 0; g < G; ++g, ++it) {
                 const int ws_ = it % C::kRW, as = it % C::kAS;
                 ws::wait(&w_full[ws_], (it / C::kRW) & 1, abort);
-                const uint8_t* raw = wring + ws_ * C::kRaw;
-                uint4 w[kRowsPerThread];
+                const uint8_t* raw = wring + ws_ * C::kRaw + row * 64;
+                uint4 w[kChunks];
 #pragma unroll
-                for (int p = 0; p < kRowsPerThread; ++p)
-                    w[p] = *reinterpret_cast<const uint4*>(raw + (rbase + p * (128 / kRowsPerThread)) * 64 + q * 16);
+                for (int p = 0; p < kChunks; ++p)
+                    w[p] = *reinterpret_cast<const uint4*>(raw + (((part * kChunks + p) ^ swz) << 4));
                 tc::fence_proxy_async_smem();              // order these reads before the next TMA write
                 __syncwarp();                              // this warp's reads of the slot are done
                 if (lane == 0) tc::mbar_arrive(&w_empty[ws_]);
                 ws::wait(&a_empty[as], ((it / C::kAS) & 1) ^ 1, abort);
-                uint8_t* a_st = sA + as * C::kA;
+                tc::tc_fence_after();
+                uint32_t o[8 * kChunks];
 #pragma unroll
-                for (int p = 0; p < kRowsPerThread; ++p) {
-                    const int row = rbase + p * (128 / kRowsPerThread);
-                    const uint2 w0 = widen8<kUnsigned>(w[p].x), w1 = widen8<kUnsigned>(w[p].y);
-                    const uint2 w2 = widen8<kUnsigned>(w[p].z), w3 = widen8<kUnsigned>(w[p].w);
-                    *reinterpret_cast<uint4*>(a_st + sw128_off(row, 2 * q)) = make_uint4(w0.x, w0.y, w1.x, w1.y);
-                    *reinterpret_cast<uint4*>(a_st + sw128_off(row, 2 * q + 1)) = make_uint4(w2.x, w2.y, w3.x, w3.y);
+                for (int p = 0; p < kChunks; ++p) {
+                    const uint32_t ww[4] = {w[p].x, w[p].y, w[p].z, w[p].w};
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const uint2 x = widen8<kUnsigned>(ww[q]);
+                        o[8 * p + 2 * q] = x.x;
+                        o[8 * p + 2 * q + 1] = x.y;
+                    }
                 }
-                tc::fence_proxy_async_smem();
+                if constexpr (kChunks == 2) tc::tmem_st16(t_dst + as * 32, o);
+                else tc::tmem_st32(t_dst + as * 32, o);
+                tc::tmem_wait_st();
+                tc::tc_fence_before();
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(&a_full[as]);
             }
@@ -523,7 +541,7 @@ inline PFN_encodeTiled encode_fn() {
 
 // 2D byte tensor [rows, row_bytes] (row-major) with a box of box_rows x box_bytes.
 inline bool make_map_u8(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t rows,
-                        uint32_t box_bytes, uint32_t box_rows, bool swizzle128) {
+                        uint32_t box_bytes, uint32_t box_rows, CUtensorMapSwizzle swizzle) {
     PFN_encodeTiled fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[2] = {row_bytes, rows};
@@ -531,8 +549,7 @@ inline bool make_map_u8(CUtensorMap* m, const void* base, uint64_t row_bytes, ui
     const cuuint32_t box[2] = {box_bytes, box_rows};
     const cuuint32_t estr[2] = {1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE,
-              swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -555,9 +572,11 @@ int launch_gemm_ws_inst(const WsGemmArgs& a, const void* act, const void* w0, co
     }
     CUtensorMap m0, m1, mact;
     const int rows_per_load = kSwiGLU ? 64 : 128;
-    if (!make_map_u8(&m0, w0, a.K / 2, (uint64_t)a.E * a.R0, 64, rows_per_load, false) ||
-        !make_map_u8(&m1, kSwiGLU ? w1 : w0, a.K / 2, (uint64_t)a.E * a.R0, 64, rows_per_load, false) ||
-        !make_map_u8(&mact, act, a.K, kGather ? (uint64_t)a.T : (uint64_t)a.P, 128, kGather ? 1 : BN, true))
+    if (!make_map_u8(&m0, w0, a.K / 2, (uint64_t)a.E * a.R0, 64, rows_per_load, CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !make_map_u8(&m1, kSwiGLU ? w1 : w0, a.K / 2, (uint64_t)a.E * a.R0, 64, rows_per_load,
+                     CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !make_map_u8(&mact, act, a.K, kGather ? (uint64_t)a.T : (uint64_t)a.P, 128, kGather ? 1 : BN,
+                     CU_TENSOR_MAP_SWIZZLE_128B))
         return MOE_ERR_CUDA;
     const int m_tiles = kSwiGLU ? a.R0 / 64 : a.R0 / 128;
     const int64_t grid = std::max<int64_t>(
