@@ -49,6 +49,30 @@ __device__ __forceinline__ float e4m3_to_f32(uint8_t c) {
     return __half2float(*reinterpret_cast<__half*>(&h));
 }
 
+// Sum of the eight E4M3 values in `codes` (byte 0 of .x first), each decoded exactly.
+__device__ __forceinline__ float e4m3x8_sum(uint2 codes) {
+    const uint32_t w[2] = {codes.x, codes.y};
+    float s = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+#pragma unroll
+        for (int hgh = 0; hgh < 2; ++hgh) {
+            const __half2_raw h2 = __nv_cvt_fp8x2_to_halfraw2(
+                static_cast<__nv_fp8x2_storage_t>((w[i] >> (16 * hgh)) & 0xFFFFu), __NV_E4M3);
+            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h2));
+            s += f.x + f.y;
+        }
+    }
+    return s;
+}
+
+// Sum over the 16 lanes of each half-warp (all 32 lanes take part).
+__device__ __forceinline__ float halfwarp_sum(float v) {
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));

@@ -75,7 +75,8 @@ __global__ void __launch_bounds__(256) k_quant_topk(const float* __restrict__ lo
                                                     int H, int32_t* __restrict__ ids,
                                                     float* __restrict__ gates,
                                                     uint8_t* __restrict__ xq,
-                                                    float* __restrict__ s_x) {
+                                                    float* __restrict__ s_x,
+                                                    float* __restrict__ qsum) {
     __shared__ float red[32];
     const int64_t t = blockIdx.x;
     if (threadIdx.x < 32) topk_row<EPL>(logits + t * E, E, k, ids + t * k, gates + t * k, threadIdx.x);
@@ -85,16 +86,25 @@ __global__ void __launch_bounds__(256) k_quant_topk(const float* __restrict__ lo
     for (int c = threadIdx.x; c < chunks; c += blockDim.x) a = fmaxf(a, amax8(__ldg(row + c)));
     a = block_max(a, red);
     const float s = __fdiv_rn(a, kFp8Max);
-    for (int c = threadIdx.x; c < chunks; c += blockDim.x)
-        reinterpret_cast<uint2*>(xq + t * H)[c] = quant8(__ldg(row + c), s);
+    // codes, and per K-group of 128 (16 chunks = one half-warp) the sum of the decoded values
+    const int G = H / kGroup;
+    for (int base = 0; base < chunks; base += blockDim.x) {
+        const int c = base + threadIdx.x;
+        const bool live = c < chunks;
+        const uint2 codes = live ? quant8(__ldg(row + c), s) : make_uint2(0u, 0u);
+        if (live) reinterpret_cast<uint2*>(xq + t * H)[c] = codes;
+        const float gs = halfwarp_sum(e4m3x8_sum(codes));
+        if (live && (threadIdx.x & 15) == 0) qsum[t * G + c / 16] = gs;
+    }
     if (threadIdx.x == 0) s_x[t] = s;
 }
 
 inline int launch_quant_topk(const float* logits, const uint16_t* x, int64_t T, int E, int k, int H,
-                             int32_t* ids, float* gates, uint8_t* xq, float* s_x, cudaStream_t stream) {
+                             int32_t* ids, float* gates, uint8_t* xq, float* s_x, float* qsum,
+                             cudaStream_t stream) {
     const int epl = (E + 31) / 32;
     const unsigned grid = static_cast<unsigned>(T);
-#define MOE_QT(N) k_quant_topk<N><<<grid, 256, 0, stream>>>(logits, x, E, k, H, ids, gates, xq, s_x)
+#define MOE_QT(N) k_quant_topk<N><<<grid, 256, 0, stream>>>(logits, x, E, k, H, ids, gates, xq, s_x, qsum)
     if (epl <= 1) MOE_QT(1);
     else if (epl <= 2) MOE_QT(2);
     else if (epl <= 4) MOE_QT(4);
@@ -111,6 +121,7 @@ inline int launch_quant_topk(const float* logits, const uint16_t* x, int64_t T, 
 struct WsPlan {
     size_t topk_ids, topk_w, offsets, sorted, rop, route_ws;
     size_t xq, s_x, x_sorted, s_x_sorted, h, zero, hq, s_h, y;
+    size_t qs_x, qs_h;   // per (activation row, K-group) sums of the FP8 values (narrow tiles)
     int64_t n_zero;   // u32 words at `zero`: max|h| per row [P], row counters [P], token counters
     size_t sh_a, sh_y;
     size_t total;
@@ -141,6 +152,8 @@ inline WsPlan plan_workspace(const moe_w4a8_layer& L, int64_t T, int k) {
     p.hq = take((size_t)P * L.N);
     p.s_h = take(P * 4);
     p.y = take((size_t)P * L.H * 4);
+    p.qs_x = take((size_t)T * (L.H / 128) * 4);
+    p.qs_h = take((size_t)P * (L.N / 128) * 4);
     if (L.n_shared > 0) {
         p.sh_a = take((size_t)T * L.n_shared * L.shared_N * 2);
         p.sh_y = take((size_t)T * L.H * 4);
@@ -267,6 +280,8 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const uint16_t* x_bf16,
     uint8_t* hq = (uint8_t*)at(p.hq);
     float* sh = (float*)at(p.s_h);
     float* y = (float*)at(p.y);
+    float* qs_x = (float*)at(p.qs_x);
+    float* qs_h = (float*)at(p.qs_h);
     // narrow token tiles (decode): codes written once per token and gathered by the GEMM, fused
     // requantization and combine; wide tiles (prefill): codes copied to expert-sorted rows.
     const bool fused = ws_narrow(tc_tile_rows(P, L.E));
@@ -274,7 +289,7 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const uint16_t* x_bf16,
     sm.mark(0, stream);
     if (fused) {
         // S1 + S2: per-token FP8 codes and top-k
-        if ((st = launch_quant_topk(router_logits, x_bf16, T, L.E, k, L.H, ids, gates, xq, sx, stream)))
+        if ((st = launch_quant_topk(router_logits, x_bf16, T, L.E, k, L.H, ids, gates, xq, sx, qs_x, stream)))
             return st;
         sm.launches += 1;
         sm.mark(1, stream);
@@ -313,7 +328,8 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const uint16_t* x_bf16,
     // S4 + SwiGLU (+ S5 when fused): h = silu(G) * U, max|h| per row
     {
         WsGemmArgs a{fused ? sx : sxs, L.gate_scales, L.up_scales, offsets, L.E, L.N, L.H, (int)P, h, L.N,
-                     amax, rowcnt, hq, sh, sorted, nullptr, nullptr, k, nullptr, nullptr, (int)T};
+                     amax, rowcnt, hq, sh, sorted, nullptr, nullptr, k, nullptr, nullptr, (int)T,
+                     fused ? qs_x : nullptr, fused ? qs_h : nullptr};
         if ((st = launch_gemm_ws<true>(a, fused ? (const void*)xq : (const void*)xs, L.gate_packed,
                                        L.up_packed, stream)))
             return st;
@@ -330,7 +346,8 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const uint16_t* x_bf16,
     // S6 (+ S7 when fused)
     {
         WsGemmArgs a{sh, L.down_scales, nullptr, offsets, L.E, L.H, L.N, (int)P, y, L.H, nullptr,
-                     tokcnt, nullptr, nullptr, sorted, rop, gates, k, shared, out_bf16, (int)T};
+                     tokcnt, nullptr, nullptr, sorted, rop, gates, k, shared, out_bf16, (int)T,
+                     fused ? qs_h : nullptr, nullptr};
         if ((st = launch_gemm_ws<false>(a, hq, L.down_packed, nullptr, stream))) return st;
         sm.launches += 1;
     }

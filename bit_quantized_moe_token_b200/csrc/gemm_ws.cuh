@@ -18,10 +18,11 @@
 //              promotion warps and release the ring / A stages; the warp also owns the TMEM.
 //
 // Widening (see tc_tiles.cuh for the arithmetic):
-//   kUnsigned (narrow token tiles, decode): byte = nibble = E4M3 of (code+8)*2^-9; four more
-//     MMAs per group with a constant A tile of -2^-6 (E4M3 0x88) against the same activation
-//     tile add -8*2^-9*sum_k q_k, so TMEM holds exactly 2^-9 * sum_k q_k*code_k and the
-//     promotion is one FMA with 512*scale.  The tensor core has ample headroom at decode sizes.
+//   kUnsigned (narrow token tiles, decode): byte = nibble = E4M3 of (code+8)*2^-9, so TMEM
+//     holds 2^-9 * sum_k q_k*(code_k + 8) and the promotion subtracts the offset term with the
+//     group's activation sum: acc += 512*s*partial - 8*s*sum_k q_k (one more FMA per element;
+//     a tcgen05.mma costs the same issue time at N = 16 as at N = 64, so the offset is cheaper
+//     in the promotion than as four more MMAs).
 //   signed (wide token tiles, prefill): byte = E4M3(code) by byte-permute lookup.
 //
 // Every mbarrier wait is bounded; a timeout sets a CTA-wide abort flag that turns all later
@@ -59,6 +60,10 @@ struct WsGemmArgs {
     const float* shared;    // plain: [T, ldo] shared-expert output or null
     uint16_t* out_bf16;     // plain: [T, ldo] layer output
     int T;                  // tokens (rows of the gathered activation tensor)
+    // unsigned widening: per (activation row, K-group) sums of the FP8 values the GEMM reads
+    // (per token when gathering, per sorted row otherwise), for the +8 offset correction
+    const float* qsum;
+    float* qsum_out;        // SwiGLU fused: the same sums of the requantized rows [P, R0/128]
 };
 
 namespace ws {
@@ -118,13 +123,11 @@ struct WsCfg {
     static constexpr int kCtasPerSm = (BN <= 16) ? 2 : 1;       // BN = 16: two CTAs per SM
     static constexpr int kRW = (BN <= 16) ? 10 : kNarrow ? 16 : (BN <= 64 ? 12 : 8);   // weight ring
     static constexpr int kRB = (BN <= 16) ? 6 : kNarrow ? 8 : (BN <= 64 ? 6 : 5);     // activation ring
-    static constexpr int kAS = (BN <= 16) ? 3 : 4;                                 // widened A stages
+    static constexpr int kAS = 4;                                                  // widened A stages
     static constexpr int kNT = kNarrow ? 8 : (BN <= 64 ? 4 : 3);                   // TMEM partials
-    // TMEM columns: partial buffers | widened A stages (32 columns = 128 E4M3 per row) | the
-    // constant -2^-6 tile of the unsigned widening.
+    // TMEM columns: partial buffers | widened A stages (32 columns = 128 E4M3 per row)
     static constexpr int kColA = kNT * BN;
-    static constexpr int kColConst = kColA + kAS * 32;
-    static constexpr int kTmemNeed = kColConst + (kUnsigned ? 32 : 0);
+    static constexpr int kTmemNeed = kColA + kAS * 32;
     static constexpr int kTmemCols = kTmemNeed <= 32 ? 32 : kTmemNeed <= 64 ? 64 : kTmemNeed <= 128 ? 128
                                    : kTmemNeed <= 256 ? 256 : 512;
     static_assert(kTmemNeed <= 512 / kCtasPerSm, "TMEM budget");
@@ -135,7 +138,9 @@ struct WsCfg {
     static constexpr int kOffPre = kOffUs + 64 * kUsStride * 4;
     static constexpr int kOffFlag = kOffPre + 1025 * 4;          // BN ints (fused epilogues)
     static constexpr int kOffSr = kOffFlag + BN * 4;             // 2 x BN per-column scales
-    static constexpr int kOffBar = ((kOffSr + 2 * BN * 4 + 7) / 8) * 8;
+    static constexpr int kMaxG = 128;                            // K <= 16384
+    static constexpr int kOffQs = kOffSr + 2 * BN * 4;           // unsigned: [G][BN] group sums
+    static constexpr int kOffBar = ((kOffQs + (kUnsigned ? kMaxG * BN * 4 : 0) + 7) / 8) * 8;
     static constexpr int kNumBars = 2 * kRW + 2 * kRB + 2 * kAS + 2 * kNT;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;     // TMEM slot, abort flag
     static constexpr int kBytes = kOffMisc + 16;
@@ -158,11 +163,13 @@ struct WsCfg {
 // other CTAs' outputs through L2.  The result does not depend on which CTA finishes last.
 __device__ __forceinline__ void requant_row(const float* __restrict__ h, int N, unsigned amax_bits,
                                             uint8_t* __restrict__ hq, float* __restrict__ s_h, int tid,
-                                            int nthreads) {
+                                            int nthreads, float* __restrict__ qs_row) {
     const float s = __fdiv_rn(__uint_as_float(amax_bits), kFp8Max);
-    for (int c = tid; c < (N >> 3); c += nthreads) {
+    for (int base = 0; base < (N >> 3); base += nthreads) {
+        const int c = base + tid;
+        const bool live = c < (N >> 3);
         uint2 codes = make_uint2(0u, 0u);
-        if (s != 0.0f) {
+        if (live && s != 0.0f) {
             const float4 a = __ldcg(reinterpret_cast<const float4*>(h) + 2 * c);
             const float4 b = __ldcg(reinterpret_cast<const float4*>(h) + 2 * c + 1);
             codes.x = static_cast<uint32_t>(f32x2_to_e4m3x2(__fdiv_rn(a.x, s), __fdiv_rn(a.y, s))) |
@@ -170,7 +177,11 @@ __device__ __forceinline__ void requant_row(const float* __restrict__ h, int N, 
             codes.y = static_cast<uint32_t>(f32x2_to_e4m3x2(__fdiv_rn(b.x, s), __fdiv_rn(b.y, s))) |
                       (static_cast<uint32_t>(f32x2_to_e4m3x2(__fdiv_rn(b.z, s), __fdiv_rn(b.w, s))) << 16);
         }
-        reinterpret_cast<uint2*>(hq)[c] = codes;
+        if (live) reinterpret_cast<uint2*>(hq)[c] = codes;
+        if (qs_row) {   // sums of the decoded codes per K-group of 128 (16 chunks = one half-warp)
+            const float gs = halfwarp_sum(e4m3x8_sum(codes));
+            if (live && (tid & 15) == 0) qs_row[c / 16] = gs;
+        }
     }
     if (tid == 0) *s_h = s;
 }
@@ -188,6 +199,7 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
     int* pre = reinterpret_cast<int*>(sm + C::kOffPre);
     int* flag = reinterpret_cast<int*>(sm + C::kOffFlag);
     float* sSr = reinterpret_cast<float*>(sm + C::kOffSr);
+    float* sQs = reinterpret_cast<float*>(sm + C::kOffQs);
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + C::kOffBar);
     uint64_t* w_full = bar;                       // weight ring: TMA -> widening warps
     uint64_t* w_empty = w_full + C::kRW;          //              widening warps -> TMA
@@ -223,18 +235,6 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem = *tslot;
-    if constexpr (kUnsigned) {          // constant A tile: every byte E4M3(-2^-6) = 0x88
-        if (warp < 4) {
-            uint32_t cst[32];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) cst[i] = 0x88888888u;
-            tc::tmem_st32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + C::kColConst, cst);
-            tc::tmem_wait_st();
-        }
-        tc::tc_fence_before();
-        __syncthreads();
-        tc::tc_fence_after();
-    }
 
     if (warp == C::kWarpTma) {
         // ------------------------------------------------------------ TMA producer
@@ -312,12 +312,6 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
                     for (int kk = 0; kk < 4; ++kk)
                         tc::mma_e4m3_ta(d, a_col + kk * 8, tc::sdesc_sw128(b_addr + kk * 32), idesc,
                                         kk > 0 ? 1u : 0u);
-                    if (kUnsigned) {
-#pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            tc::mma_e4m3_ta(d, tmem + C::kColConst + kk * 8,
-                                            tc::sdesc_sw128(b_addr + kk * 32), idesc, 1u);
-                    }
                     tc::mma_commit(&t_full[tb]);
                     tc::mma_commit(&a_empty[as]);
                     tc::mma_commit(&b_empty[bs]);
@@ -404,6 +398,18 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
             } else {
                 ssrc = a.s0 + ((int64_t)e * a.R0 + mt * 128 + lrow) * G;
             }
+            if constexpr (kUnsigned) {   // the tile's activation group sums, sQs[g * BN + j]
+                for (int i = pt; i < G * BN; i += kNPT) {
+                    const int j = i / G, g = i - j * G;
+                    float v = 0.0f;
+                    if (j < nrows) {
+                        const int64_t rr = kGather ? (int64_t)(a.sorted[row0 + j] / a.k) : row0 + j;
+                        v = a.qsum[rr * G + g];
+                    }
+                    sQs[g * BN + j] = v;
+                }
+                ws::named_sync_math<kNPT>();
+            }
             float acc[kCPW];
 #pragma unroll
             for (int j = 0; j < kCPW; ++j) acc[j] = 0.0f;
@@ -425,6 +431,12 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
                     tc::tmem_wait_ld();
 #pragma unroll
                     for (int j = 0; j < C::kLd; ++j) acc[c1 + j] = fmaf(sc, __uint_as_float(v[j]), acc[c1 + j]);
+                    if constexpr (kUnsigned) {   // minus 8 * s * (group sum of the column's q)
+                        const float scm = sc * (-1.0f / 64.0f);
+                        const float* qg = sQs + g * BN + c_base + c1;
+#pragma unroll
+                        for (int j = 0; j < C::kLd; ++j) acc[c1 + j] = fmaf(scm, qg[j], acc[c1 + j]);
+                    }
                 }
                 tc::tc_fence_before();
                 __syncwarp();
@@ -473,7 +485,8 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
                             __threadfence();
                             const int64_t r = row0 + j;
                             requant_row(a.out + r * a.ldo, a.ldo, __ldcg(a.amax + r), a.hq + r * a.ldo,
-                                        a.s_h + r, pt, kNPT);
+                                        a.s_h + r, pt, kNPT,
+                                        a.qsum_out ? a.qsum_out + r * (a.ldo / kGroup) : nullptr);
                         }
                     }
                 }
