@@ -122,18 +122,19 @@ struct WsCfg {
     static constexpr int kBSlot = ((kB + 1023) / 1024) * 1024;
     static constexpr int kCtasPerSm = (BN <= 16) ? 2 : 1;       // BN = 16: two CTAs per SM
     static constexpr int kRW = (BN <= 16) ? 10 : kNarrow ? 16 : (BN <= 64 ? 12 : 8);   // weight ring
-    static constexpr int kRB = (BN <= 16) ? 6 : kNarrow ? 8 : (BN <= 64 ? 6 : 5);     // activation ring
-    static constexpr int kAS = 4;                                                  // widened A stages
+    // Operand stages: an activation tile in shared memory plus the widened A tile in TMEM, with
+    // one "ready" barrier (widening warps + activation bytes) and one "free" barrier (MMA commit).
+    static constexpr int kS = (BN <= 16) ? 4 : (BN <= 64 ? 8 : 4);
     static constexpr int kNT = kNarrow ? 8 : (BN <= 64 ? 4 : 3);                   // TMEM partials
     // TMEM columns: partial buffers | widened A stages (32 columns = 128 E4M3 per row)
     static constexpr int kColA = kNT * BN;
-    static constexpr int kTmemNeed = kColA + kAS * 32;
+    static constexpr int kTmemNeed = kColA + kS * 32;
     static constexpr int kTmemCols = kTmemNeed <= 32 ? 32 : kTmemNeed <= 64 ? 64 : kTmemNeed <= 128 ? 128
                                    : kTmemNeed <= 256 ? 256 : 512;
     static_assert(kTmemNeed <= 512 / kCtasPerSm, "TMEM budget");
     static constexpr int kUsStride = BN + 1;
     static constexpr int kOffB = 0;
-    static constexpr int kOffW = kOffB + kRB * kBSlot;
+    static constexpr int kOffW = kOffB + kS * kBSlot;
     static constexpr int kOffUs = kOffW + kRW * kRaw;
     static constexpr int kOffPre = kOffUs + 64 * kUsStride * 4;
     static constexpr int kOffFlag = kOffPre + 1025 * 4;          // BN ints (fused epilogues)
@@ -141,7 +142,7 @@ struct WsCfg {
     static constexpr int kMaxG = 128;                            // K <= 16384
     static constexpr int kOffQs = kOffSr + 2 * BN * 4;           // unsigned: [G][BN] group sums
     static constexpr int kOffBar = ((kOffQs + (kUnsigned ? kMaxG * BN * 4 : 0) + 7) / 8) * 8;
-    static constexpr int kNumBars = 2 * kRW + 2 * kRB + 2 * kAS + 2 * kNT;
+    static constexpr int kNumBars = 2 * kRW + 2 * kS + 2 * kNT;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;     // TMEM slot, abort flag
     static constexpr int kBytes = kOffMisc + 16;
     static constexpr int kAlloc = kBytes + 1024;
@@ -203,11 +204,9 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + C::kOffBar);
     uint64_t* w_full = bar;                       // weight ring: TMA -> widening warps
     uint64_t* w_empty = w_full + C::kRW;          //              widening warps -> TMA
-    uint64_t* b_full = w_empty + C::kRW;          // activation ring: TMA -> MMA
-    uint64_t* b_empty = b_full + C::kRB;          //                  MMA commit -> TMA
-    uint64_t* a_full = b_empty + C::kRB;          // widened A: widening warps -> MMA
-    uint64_t* a_empty = a_full + C::kAS;          //            MMA commit -> widening warps
-    uint64_t* t_full = a_empty + C::kAS;          // TMEM partials: MMA commit -> promotion
+    uint64_t* s_ready = w_empty + C::kRW;         // operand stage: widening warps + TMA bytes -> MMA
+    uint64_t* s_free = s_ready + C::kS;           //                MMA commit -> widening warps, TMA
+    uint64_t* t_full = s_free + C::kS;            // TMEM partials: MMA commit -> promotion
     uint64_t* t_empty = t_full + C::kNT;          //                promotion -> MMA
     uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + C::kOffMisc);
     volatile int* abort = reinterpret_cast<volatile int*>(sm + C::kOffMisc + 4);
@@ -221,8 +220,7 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
 
     if (tid == 0) {
         for (int i = 0; i < C::kRW; ++i) { tc::mbar_init(&w_full[i], 1); tc::mbar_init(&w_empty[i], C::kNW); }
-        for (int i = 0; i < C::kRB; ++i) { tc::mbar_init(&b_full[i], 1); tc::mbar_init(&b_empty[i], 1); }
-        for (int i = 0; i < C::kAS; ++i) { tc::mbar_init(&a_full[i], C::kNW); tc::mbar_init(&a_empty[i], 1); }
+        for (int i = 0; i < C::kS; ++i) { tc::mbar_init(&s_ready[i], C::kNW + 1); tc::mbar_init(&s_free[i], 1); }
         for (int i = 0; i < C::kNT; ++i) { tc::mbar_init(&t_full[i], 1); tc::mbar_init(&t_empty[i], C::kNP); }
         *abort = 0;
         tc::fence_mbar_init();
@@ -262,7 +260,7 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
             const uint32_t b_bytes = kGather ? static_cast<uint32_t>(ngather) * 512u : C::kB;
             bool stop = false;
             for (int g = 0; g < G; ++g, ++it) {
-                const int ws_ = it % C::kRW, bs = it % C::kRB;
+                const int ws_ = it % C::kRW, bs = it % C::kS;
                 int ok = 1;
                 if (lane == 0) {
                     ok = ws::wait(&w_empty[ws_], ((it / C::kRW) & 1) ^ 1, abort);
@@ -276,8 +274,8 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
                         } else {
                             ws::tma_load_2d(wst, &tm_w0, g * 64, e * a.R0 + mt * 128, &w_full[ws_]);
                         }
-                        ok = ws::wait(&b_empty[bs], ((it / C::kRB) & 1) ^ 1, abort);
-                        if (ok) tc::mbar_arrive_expect_tx(&b_full[bs], b_bytes);
+                        ok = ws::wait(&s_free[bs], ((it / C::kS) & 1) ^ 1, abort);
+                        if (ok) tc::mbar_arrive_expect_tx(&s_ready[bs], b_bytes);
                     }
                 }
                 ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -286,9 +284,9 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
                 if (kGather) {
                     if (lane < ngather)
                         ws::tma_gather4(bst + lane * 512, &tm_act, g * kGroup, tok[0], tok[1], tok[2], tok[3],
-                                        &b_full[bs]);
+                                        &s_ready[bs]);
                 } else if (lane == 0) {
-                    ws::tma_load_2d(bst, &tm_act, g * kGroup, row0, &b_full[bs]);
+                    ws::tma_load_2d(bst, &tm_act, g * kGroup, row0, &s_ready[bs]);
                 }
             }
             if (stop) break;
@@ -300,26 +298,24 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
             uint32_t it = 0;
             for (int64_t tile = blockIdx.x; tile < n_tiles && !*abort; tile += gridDim.x) {
                 for (int g = 0; g < G; ++g, ++it) {
-                    const int bs = it % C::kRB, as = it % C::kAS, tb = it % C::kNT;
-                    if (!ws::wait(&b_full[bs], (it / C::kRB) & 1, abort)) break;
-                    if (!ws::wait(&a_full[as], (it / C::kAS) & 1, abort)) break;
+                    const int ss = it % C::kS, tb = it % C::kNT;
+                    if (!ws::wait(&s_ready[ss], (it / C::kS) & 1, abort)) break;
                     if (!ws::wait(&t_empty[tb], ((it / C::kNT) & 1) ^ 1, abort)) break;
                     tc::tc_fence_after();
-                    const uint32_t b_addr = tc::smem_u32(bring + bs * C::kBSlot);
-                    const uint32_t a_col = tmem + C::kColA + as * 32;
+                    const uint32_t b_addr = tc::smem_u32(bring + ss * C::kBSlot);
+                    const uint32_t a_col = tmem + C::kColA + ss * 32;
                     const uint32_t d = tmem + tb * BN;
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         tc::mma_e4m3_ta(d, a_col + kk * 8, tc::sdesc_sw128(b_addr + kk * 32), idesc,
                                         kk > 0 ? 1u : 0u);
                     tc::mma_commit(&t_full[tb]);
-                    tc::mma_commit(&a_empty[as]);
-                    tc::mma_commit(&b_empty[bs]);
+                    tc::mma_commit(&s_free[ss]);
                 }
             }
             // the commits complete in order: once the last one has arrived, no tensor-core
             // arrive on this CTA's barriers is still pending
-            if (it > 0) ws::wait(&b_empty[(it - 1) % C::kRB], ((it - 1) / C::kRB) & 1, abort);
+            if (it > 0) ws::wait(&s_free[(it - 1) % C::kS], ((it - 1) / C::kS) & 1, abort);
         }
     } else if (warp < C::kNW) {
         // ------------------------------------------------------------ widening warps
@@ -336,7 +332,7 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
         uint32_t it = 0;
         for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
             for (int g = 0; g < G; ++g, ++it) {
-                const int ws_ = it % C::kRW, as = it % C::kAS;
+                const int ws_ = it % C::kRW, as = it % C::kS;
                 ws::wait(&w_full[ws_], (it / C::kRW) & 1, abort);
                 const uint8_t* raw = wring + ws_ * C::kRaw + row * 64;
                 uint4 w[kChunks];
@@ -346,7 +342,7 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
                 tc::fence_proxy_async_smem();              // order these reads before the next TMA write
                 __syncwarp();                              // this warp's reads of the slot are done
                 if (lane == 0) tc::mbar_arrive(&w_empty[ws_]);
-                ws::wait(&a_empty[as], ((it / C::kAS) & 1) ^ 1, abort);
+                ws::wait(&s_free[as], ((it / C::kS) & 1) ^ 1, abort);
                 tc::tc_fence_after();
                 uint32_t o[8 * kChunks];
 #pragma unroll
@@ -364,7 +360,7 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
                 tc::tmem_wait_st();
                 tc::tc_fence_before();
                 __syncwarp();
-                if (lane == 0) tc::mbar_arrive(&a_full[as]);
+                if (lane == 0) tc::mbar_arrive(&s_ready[as]);
             }
         }
     } else if (warp < C::kNW + C::kNP) {
