@@ -47,6 +47,11 @@ def flops_per_pair(wl):
     return 2 * wl.H * 2 * wl.N + 2 * wl.N * wl.H
 
 
+def is_prefill(wl):
+    """Prefill shapes are scored against the FP8 tensor peak, decode shapes against HBM."""
+    return wl.T >= 1024
+
+
 def peaks():
     try:
         with open(PEAKS_FILE) as f:
@@ -279,13 +284,26 @@ def run_ours(args):
     gu_bytes, down_bytes = expert_bytes(wl)
     mean_touched = sum(touched[i % N_BATCHES] for i in range(args.steps)) / args.steps
     dom_bytes = mean_touched * gu_bytes
-    achieved = dom_bytes / (dom_ms / 1e3) / 1e9
-    roofline = {"bound": "hbm", "kernel": "grouped gate/up W4A8 GEMM (stage)",
-                "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
-                "frac": round(achieved / hbm, 4), "traffic": None,
-                "peak_source": f"{peak_kind} hbm_gbs",
-                "algorithmic_bytes_per_launch": int(dom_bytes),
-                "units": f"{mean_touched:.1f} touched experts x {gu_bytes} B (gate+up codes+scales)"}
+    if is_prefill(wl):
+        # compute-bound shape: gate/up FLOPs over the dense FP8 tensor peak (the measured bf16
+        # cuBLAS peak x 2, NVIDIA's nominal FP8 / BF16 ratio)
+        dom_flops = T * k * 2 * wl.H * 2 * wl.N
+        achieved = dom_flops / (dom_ms / 1e3) / 1e12
+        fp8 = 2.0 * bf16
+        roofline = {"bound": "tensor", "kernel": "grouped gate/up W4A8 GEMM (stage)",
+                    "achieved": round(achieved, 1), "peak": round(fp8, 1), "unit": "TFLOP/s",
+                    "frac": round(achieved / fp8, 4), "traffic": None,
+                    "peak_source": f"{peak_kind} bf16_tflops x 2 (nominal FP8/BF16 ratio)",
+                    "algorithmic_flops_per_launch": int(dom_flops),
+                    "units": f"{T * k} routed pairs x {2 * wl.H * 2 * wl.N} FLOP (gate+up)"}
+    else:
+        achieved = dom_bytes / (dom_ms / 1e3) / 1e9
+        roofline = {"bound": "hbm", "kernel": "grouped gate/up W4A8 GEMM (stage)",
+                    "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                    "frac": round(achieved / hbm, 4), "traffic": None,
+                    "peak_source": f"{peak_kind} hbm_gbs",
+                    "algorithmic_bytes_per_launch": int(dom_bytes),
+                    "units": f"{mean_touched:.1f} touched experts x {gu_bytes} B (gate+up codes+scales)"}
     layer_bytes = mean_touched * (gu_bytes + down_bytes)
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
