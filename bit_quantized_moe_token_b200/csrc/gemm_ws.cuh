@@ -117,24 +117,30 @@ struct WsCfg {
     // widening, 8 widening warps, and for BN = 16 two persistent CTAs per SM.  Wide tiles
     // (prefill) keep more smem for the activation tiles, one CTA per SM.
     static constexpr bool kNarrow = BN <= 32;
-    static constexpr int kRaw = 128 * 64;                       // packed codes, one group tile
+    // Every pipeline stage carries kGS K-groups: narrow tiles move two per stage, which halves
+    // the waits, commits and TMA issues per weight byte of the single-thread TMA and MMA roles.
+    static constexpr int kGS = kNarrow ? 2 : 1;
+    static constexpr int kRowB = 64 * kGS;                      // packed bytes per row per stage
+    static constexpr int kRaw = 128 * kRowB;                    // packed codes, one stage
     static constexpr int kB = BN * 128;                         // activation tile, one group
     static constexpr int kBSlot = ((kB + 1023) / 1024) * 1024;
     static constexpr int kCtasPerSm = (BN <= 16) ? 2 : 1;       // BN = 16: two CTAs per SM
-    static constexpr int kRW = (BN <= 16) ? 10 : kNarrow ? 16 : (BN <= 64 ? 12 : 8);   // weight ring
-    // Operand stages: an activation tile in shared memory plus the widened A tile in TMEM, with
-    // one "ready" barrier (widening warps + activation bytes) and one "free" barrier (MMA commit).
-    static constexpr int kS = (BN <= 16) ? 4 : (BN <= 64 ? 8 : 4);
+    static constexpr int kRW = (BN <= 16) ? 5 : kNarrow ? 8 : (BN <= 64 ? 12 : 8);     // weight ring
+    // Operand stages: kGS activation tiles in shared memory plus the widened A tiles in TMEM,
+    // with one "ready" barrier (widening warps + activation bytes) and one "free" barrier (MMA
+    // commit).
+    static constexpr int kS = (BN <= 16) ? 2 : (BN <= 32 ? 4 : (BN <= 64 ? 8 : 4));
     static constexpr int kNT = kNarrow ? 8 : (BN <= 64 ? 4 : 3);                   // TMEM partials
-    // TMEM columns: partial buffers | widened A stages (32 columns = 128 E4M3 per row)
+    static constexpr int kNTS = kNT / kGS;                       // partial stages (barrier pairs)
+    // TMEM columns: partial buffers | widened A tiles (32 columns = 128 E4M3 per row)
     static constexpr int kColA = kNT * BN;
-    static constexpr int kTmemNeed = kColA + kS * 32;
+    static constexpr int kTmemNeed = kColA + kS * kGS * 32;
     static constexpr int kTmemCols = kTmemNeed <= 32 ? 32 : kTmemNeed <= 64 ? 64 : kTmemNeed <= 128 ? 128
                                    : kTmemNeed <= 256 ? 256 : 512;
     static_assert(kTmemNeed <= 512 / kCtasPerSm, "TMEM budget");
     static constexpr int kUsStride = BN + 1;
     static constexpr int kOffB = 0;
-    static constexpr int kOffW = kOffB + kS * kBSlot;
+    static constexpr int kOffW = kOffB + kS * kGS * kBSlot;
     static constexpr int kOffUs = kOffW + kRW * kRaw;
     static constexpr int kOffPre = kOffUs + 64 * kUsStride * 4;
     static constexpr int kOffFlag = kOffPre + 1025 * 4;          // BN ints (fused epilogues)
@@ -142,7 +148,7 @@ struct WsCfg {
     static constexpr int kMaxG = 128;                            // K <= 16384
     static constexpr int kOffQs = kOffSr + 2 * BN * 4;           // unsigned: [G][BN] group sums
     static constexpr int kOffBar = ((kOffQs + (kUnsigned ? kMaxG * BN * 4 : 0) + 7) / 8) * 8;
-    static constexpr int kNumBars = 2 * kRW + 2 * kS + 2 * kNT;
+    static constexpr int kNumBars = 2 * kRW + 2 * kS + 2 * kNTS;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;     // TMEM slot, abort flag
     static constexpr int kBytes = kOffMisc + 16;
     static constexpr int kAlloc = kBytes + 1024;
@@ -207,12 +213,13 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
     uint64_t* s_ready = w_empty + C::kRW;         // operand stage: widening warps + TMA bytes -> MMA
     uint64_t* s_free = s_ready + C::kS;           //                MMA commit -> widening warps, TMA
     uint64_t* t_full = s_free + C::kS;            // TMEM partials: MMA commit -> promotion
-    uint64_t* t_empty = t_full + C::kNT;          //                promotion -> MMA
+    uint64_t* t_empty = t_full + C::kNTS;         //                promotion -> MMA
     uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + C::kOffMisc);
     volatile int* abort = reinterpret_cast<volatile int*>(sm + C::kOffMisc + 4);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int G = a.K / kGroup;
+    const int nst = (G + C::kGS - 1) / C::kGS;             // stages per tile
     const int m_tiles = kSwiGLU ? a.R0 / 64 : a.R0 / 128;
     const int row_tiles = row_tile_prefix(a.offsets, a.E, BN, pre);
     const int64_t n_tiles = (int64_t)row_tiles * m_tiles;
@@ -221,7 +228,7 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
     if (tid == 0) {
         for (int i = 0; i < C::kRW; ++i) { tc::mbar_init(&w_full[i], 1); tc::mbar_init(&w_empty[i], C::kNW); }
         for (int i = 0; i < C::kS; ++i) { tc::mbar_init(&s_ready[i], C::kNW + 1); tc::mbar_init(&s_free[i], 1); }
-        for (int i = 0; i < C::kNT; ++i) { tc::mbar_init(&t_full[i], 1); tc::mbar_init(&t_empty[i], C::kNP); }
+        for (int i = 0; i < C::kNTS; ++i) { tc::mbar_init(&t_full[i], 1); tc::mbar_init(&t_empty[i], C::kNP); }
         *abort = 0;
         tc::fence_mbar_init();
     }
@@ -259,34 +266,38 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
             }
             const uint32_t b_bytes = kGather ? static_cast<uint32_t>(ngather) * 512u : C::kB;
             bool stop = false;
-            for (int g = 0; g < G; ++g, ++it) {
+            for (int st = 0; st < nst; ++st, ++it) {
+                const int g0 = st * C::kGS, ng = min(C::kGS, G - g0);
                 const int ws_ = it % C::kRW, bs = it % C::kS;
                 int ok = 1;
                 if (lane == 0) {
                     ok = ws::wait(&w_empty[ws_], ((it / C::kRW) & 1) ^ 1, abort);
                     if (ok) {
+                        // a stage past K (odd group count) is filled with zeros by the TMA unit
                         uint8_t* wst = wring + ws_ * C::kRaw;
                         tc::mbar_arrive_expect_tx(&w_full[ws_], C::kRaw);
                         if (kSwiGLU) {
                             const int y = e * a.R0 + mt * 64;
-                            ws::tma_load_2d(wst, &tm_w0, g * 64, y, &w_full[ws_]);
-                            ws::tma_load_2d(wst + 64 * 64, &tm_w1, g * 64, y, &w_full[ws_]);
+                            ws::tma_load_2d(wst, &tm_w0, g0 * 64, y, &w_full[ws_]);
+                            ws::tma_load_2d(wst + 64 * C::kRowB, &tm_w1, g0 * 64, y, &w_full[ws_]);
                         } else {
-                            ws::tma_load_2d(wst, &tm_w0, g * 64, e * a.R0 + mt * 128, &w_full[ws_]);
+                            ws::tma_load_2d(wst, &tm_w0, g0 * 64, e * a.R0 + mt * 128, &w_full[ws_]);
                         }
                         ok = ws::wait(&s_free[bs], ((it / C::kS) & 1) ^ 1, abort);
-                        if (ok) tc::mbar_arrive_expect_tx(&s_ready[bs], b_bytes);
+                        if (ok) tc::mbar_arrive_expect_tx(&s_ready[bs], b_bytes * ng);
                     }
                 }
                 ok = __shfl_sync(0xffffffffu, ok, 0);
                 if (!ok) { stop = true; break; }
-                uint8_t* bst = bring + bs * C::kBSlot;
-                if (kGather) {
-                    if (lane < ngather)
-                        ws::tma_gather4(bst + lane * 512, &tm_act, g * kGroup, tok[0], tok[1], tok[2], tok[3],
-                                        &s_ready[bs]);
-                } else if (lane == 0) {
-                    ws::tma_load_2d(bst, &tm_act, g * kGroup, row0, &s_ready[bs]);
+                for (int h = 0; h < ng; ++h) {
+                    uint8_t* bst = bring + (bs * C::kGS + h) * C::kBSlot;
+                    if (kGather) {
+                        if (lane < ngather)
+                            ws::tma_gather4(bst + lane * 512, &tm_act, (g0 + h) * kGroup, tok[0], tok[1], tok[2],
+                                            tok[3], &s_ready[bs]);
+                    } else if (lane == 0) {
+                        ws::tma_load_2d(bst, &tm_act, (g0 + h) * kGroup, row0, &s_ready[bs]);
+                    }
                 }
             }
             if (stop) break;
@@ -297,19 +308,22 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
             constexpr uint32_t idesc = tc::idesc_e4m3_f32(128, BN);
             uint32_t it = 0;
             for (int64_t tile = blockIdx.x; tile < n_tiles && !*abort; tile += gridDim.x) {
-                for (int g = 0; g < G; ++g, ++it) {
-                    const int ss = it % C::kS, tb = it % C::kNT;
+                for (int st = 0; st < nst; ++st, ++it) {
+                    const int ng = min(C::kGS, G - st * C::kGS);
+                    const int ss = it % C::kS, ts = it % C::kNTS;
                     if (!ws::wait(&s_ready[ss], (it / C::kS) & 1, abort)) break;
-                    if (!ws::wait(&t_empty[tb], ((it / C::kNT) & 1) ^ 1, abort)) break;
+                    if (!ws::wait(&t_empty[ts], ((it / C::kNTS) & 1) ^ 1, abort)) break;
                     tc::tc_fence_after();
-                    const uint32_t b_addr = tc::smem_u32(bring + ss * C::kBSlot);
-                    const uint32_t a_col = tmem + C::kColA + ss * 32;
-                    const uint32_t d = tmem + tb * BN;
+                    for (int h = 0; h < ng; ++h) {
+                        const uint32_t b_addr = tc::smem_u32(bring + (ss * C::kGS + h) * C::kBSlot);
+                        const uint32_t a_col = tmem + C::kColA + (ss * C::kGS + h) * 32;
+                        const uint32_t d = tmem + (ts * C::kGS + h) * BN;
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        tc::mma_e4m3_ta(d, a_col + kk * 8, tc::sdesc_sw128(b_addr + kk * 32), idesc,
-                                        kk > 0 ? 1u : 0u);
-                    tc::mma_commit(&t_full[tb]);
+                        for (int kk = 0; kk < 4; ++kk)
+                            tc::mma_e4m3_ta(d, a_col + kk * 8, tc::sdesc_sw128(b_addr + kk * 32), idesc,
+                                            kk > 0 ? 1u : 0u);
+                    }
+                    tc::mma_commit(&t_full[ts]);
                     tc::mma_commit(&s_free[ss]);
                 }
             }
@@ -320,43 +334,50 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
     } else if (warp < C::kNW) {
         // ------------------------------------------------------------ widening warps
         // A thread owns one A row = one TMEM lane (warp id % 4 selects the lane quadrant); on
-        // narrow tiles two warps split each row's K group.  The packed tile lands with the
-        // 64-byte TMA swizzle (16-byte chunk c of row r at chunk c ^ ((r >> 1) & 3)), so the 32
-        // rows a warp reads fall in distinct banks.
+        // narrow tiles two warps split each row's K groups.  The packed stage lands with the
+        // 64-byte (one group per row) or 128-byte (two) TMA swizzle: 16-byte chunk c of row r sits
+        // at chunk c ^ ((r >> 1) & 3), resp. c ^ (r & 7), so the 32 rows a warp reads fall in
+        // distinct banks.
         constexpr int kParts = C::kNW / 4;                 // warps per lane quadrant
-        constexpr int kChunks = 4 / kParts;                // 16-byte packed chunks per thread
+        constexpr int kChunks = 4 / kParts;                // 16-byte packed chunks per thread per group
         const int quad = warp & 3, part = warp >> 2;
         const int row = quad * 32 + lane;
-        const int swz = (row >> 1) & 3;
+        const int swz = C::kGS == 1 ? (row >> 1) & 3 : row & 7;
         const uint32_t t_dst = tmem + (static_cast<uint32_t>(quad * 32) << 16) + C::kColA + part * 8 * kChunks;
         uint32_t it = 0;
         for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
-            for (int g = 0; g < G; ++g, ++it) {
+            for (int st = 0; st < nst; ++st, ++it) {
                 const int ws_ = it % C::kRW, as = it % C::kS;
                 ws::wait(&w_full[ws_], (it / C::kRW) & 1, abort);
-                const uint8_t* raw = wring + ws_ * C::kRaw + row * 64;
-                uint4 w[kChunks];
+                const uint8_t* raw = wring + ws_ * C::kRaw + row * C::kRowB;
+                uint4 w[C::kGS][kChunks];
 #pragma unroll
-                for (int p = 0; p < kChunks; ++p)
-                    w[p] = *reinterpret_cast<const uint4*>(raw + (((part * kChunks + p) ^ swz) << 4));
+                for (int h = 0; h < C::kGS; ++h)
+#pragma unroll
+                    for (int p = 0; p < kChunks; ++p)
+                        w[h][p] = *reinterpret_cast<const uint4*>(raw + (((4 * h + part * kChunks + p) ^ swz) << 4));
                 tc::fence_proxy_async_smem();              // order these reads before the next TMA write
                 __syncwarp();                              // this warp's reads of the slot are done
                 if (lane == 0) tc::mbar_arrive(&w_empty[ws_]);
                 ws::wait(&s_free[as], ((it / C::kS) & 1) ^ 1, abort);
                 tc::tc_fence_after();
-                uint32_t o[8 * kChunks];
 #pragma unroll
-                for (int p = 0; p < kChunks; ++p) {
-                    const uint32_t ww[4] = {w[p].x, w[p].y, w[p].z, w[p].w};
+                for (int h = 0; h < C::kGS; ++h) {
+                    uint32_t o[8 * kChunks];
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const uint2 x = widen8<kUnsigned>(ww[q]);
-                        o[8 * p + 2 * q] = x.x;
-                        o[8 * p + 2 * q + 1] = x.y;
+                    for (int p = 0; p < kChunks; ++p) {
+                        const uint32_t ww[4] = {w[h][p].x, w[h][p].y, w[h][p].z, w[h][p].w};
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const uint2 x = widen8<kUnsigned>(ww[q]);
+                            o[8 * p + 2 * q] = x.x;
+                            o[8 * p + 2 * q + 1] = x.y;
+                        }
                     }
+                    const uint32_t dst = t_dst + (as * C::kGS + h) * 32;
+                    if constexpr (kChunks == 2) tc::tmem_st16(dst, o);
+                    else tc::tmem_st32(dst, o);
                 }
-                if constexpr (kChunks == 2) tc::tmem_st16(t_dst + as * 32, o);
-                else tc::tmem_st32(t_dst + as * 32, o);
                 tc::tmem_wait_st();
                 tc::tc_fence_before();
                 __syncwarp();
@@ -409,34 +430,47 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
             float acc[kCPW];
 #pragma unroll
             for (int j = 0; j < kCPW; ++j) acc[j] = 0.0f;
-            float sc_next = bf16_bits_to_f32(__ldg(ssrc));
-            for (int g = 0; g < G; ++g, ++it) {
-                float sc = sc_next;
-                if (g + 1 < G) sc_next = bf16_bits_to_f32(__ldg(ssrc + g + 1));
-                if (kUnsigned) sc *= 512.0f;
-                const int tb = it % C::kNT;
-                ws::wait(&t_full[tb], (it / C::kNT) & 1, abort);
+            float sc_next[C::kGS];
+#pragma unroll
+            for (int h = 0; h < C::kGS; ++h) sc_next[h] = h < G ? bf16_bits_to_f32(__ldg(ssrc + h)) : 0.0f;
+            for (int st = 0; st < nst; ++st, ++it) {
+                const int g0 = st * C::kGS;
+                float scs[C::kGS];
+#pragma unroll
+                for (int h = 0; h < C::kGS; ++h) {
+                    scs[h] = sc_next[h];
+                    const int gn = g0 + C::kGS + h;
+                    if (gn < G) sc_next[h] = bf16_bits_to_f32(__ldg(ssrc + gn));
+                }
+                const int ts = it % C::kNTS;
+                ws::wait(&t_full[ts], (it / C::kNTS) & 1, abort);
                 tc::tc_fence_after();
 #pragma unroll
-                for (int c1 = 0; c1 < kCPW; c1 += C::kLd) {    // kLd columns in flight per wait
-                    uint32_t v[C::kLd];
+                for (int h = 0; h < C::kGS; ++h) {
+                    const int g = g0 + h;
+                    if (g >= G) break;
+                    const float sc = kUnsigned ? scs[h] * 512.0f : scs[h];
+                    const uint32_t tcol = tmem + t_lane + (ts * C::kGS + h) * BN + c_base;
 #pragma unroll
-                    for (int c0 = 0; c0 < C::kLd; c0 += 16)
-                        tc::tmem_ld16(tmem + t_lane + tb * BN + c_base + c1 + c0,
-                                      *reinterpret_cast<uint32_t(*)[16]>(v + c0));
-                    tc::tmem_wait_ld();
+                    for (int c1 = 0; c1 < kCPW; c1 += C::kLd) {    // kLd columns in flight per wait
+                        uint32_t v[C::kLd];
 #pragma unroll
-                    for (int j = 0; j < C::kLd; ++j) acc[c1 + j] = fmaf(sc, __uint_as_float(v[j]), acc[c1 + j]);
-                    if constexpr (kUnsigned) {   // minus 8 * s * (group sum of the column's q)
-                        const float scm = sc * (-1.0f / 64.0f);
-                        const float* qg = sQs + g * BN + c_base + c1;
+                        for (int c0 = 0; c0 < C::kLd; c0 += 16)
+                            tc::tmem_ld16(tcol + c1 + c0, *reinterpret_cast<uint32_t(*)[16]>(v + c0));
+                        tc::tmem_wait_ld();
 #pragma unroll
-                        for (int j = 0; j < C::kLd; ++j) acc[c1 + j] = fmaf(scm, qg[j], acc[c1 + j]);
+                        for (int j = 0; j < C::kLd; ++j) acc[c1 + j] = fmaf(sc, __uint_as_float(v[j]), acc[c1 + j]);
+                        if constexpr (kUnsigned) {   // minus 8 * s * (group sum of the column's q)
+                            const float scm = sc * (-1.0f / 64.0f);
+                            const float* qg = sQs + g * BN + c_base + c1;
+#pragma unroll
+                            for (int j = 0; j < C::kLd; ++j) acc[c1 + j] = fmaf(scm, qg[j], acc[c1 + j]);
+                        }
                     }
                 }
                 tc::tc_fence_before();
                 __syncwarp();
-                if (lane == 0) tc::mbar_arrive(&t_empty[tb]);
+                if (lane == 0) tc::mbar_arrive(&t_empty[ts]);
             }
 
             // ---- epilogue (static indices keep acc[] in registers) ----
@@ -581,9 +615,9 @@ int launch_gemm_ws_inst(const WsGemmArgs& a, const void* act, const void* w0, co
     }
     CUtensorMap m0, m1, mact;
     const int rows_per_load = kSwiGLU ? 64 : 128;
-    if (!make_map_u8(&m0, w0, a.K / 2, (uint64_t)a.E * a.R0, 64, rows_per_load, CU_TENSOR_MAP_SWIZZLE_64B) ||
-        !make_map_u8(&m1, kSwiGLU ? w1 : w0, a.K / 2, (uint64_t)a.E * a.R0, 64, rows_per_load,
-                     CU_TENSOR_MAP_SWIZZLE_64B) ||
+    const CUtensorMapSwizzle wsw = C::kGS == 1 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+    if (!make_map_u8(&m0, w0, a.K / 2, (uint64_t)a.E * a.R0, C::kRowB, rows_per_load, wsw) ||
+        !make_map_u8(&m1, kSwiGLU ? w1 : w0, a.K / 2, (uint64_t)a.E * a.R0, C::kRowB, rows_per_load, wsw) ||
         !make_map_u8(&mact, act, a.K, kGather ? (uint64_t)a.T : (uint64_t)a.P, 128, kGather ? 1 : BN,
                      CU_TENSOR_MAP_SWIZZLE_128B))
         return MOE_ERR_CUDA;
