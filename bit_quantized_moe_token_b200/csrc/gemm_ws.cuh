@@ -125,11 +125,17 @@ struct WsCfg {
     static constexpr int kB = BN * 128;                         // activation tile, one group
     static constexpr int kBSlot = ((kB + 1023) / 1024) * 1024;
     static constexpr int kCtasPerSm = (BN <= 16) ? 2 : 1;       // BN = 16: two CTAs per SM
-    static constexpr int kRW = (BN <= 16) ? 5 : kNarrow ? 8 : (BN <= 64 ? 12 : 8);     // weight ring
-    // Operand stages: kGS activation tiles in shared memory plus the widened A tiles in TMEM,
-    // with one "ready" barrier (widening warps + activation bytes) and one "free" barrier (MMA
-    // commit).
-    static constexpr int kS = (BN <= 16) ? 2 : (BN <= 32 ? 4 : (BN <= 64 ? 8 : 4));
+    // Three rings, in stages: packed weights (shared memory), widened A tiles (TMEM) and
+    // activation tiles (shared memory).  With kRB >= kRW + kS a free activation slot is always
+    // waiting once a weight slot is, so the one producer lane is paced by the weight ring alone
+    // and the activation tiles are fetched kRW stages ahead of their MMAs.
+    static constexpr int kRW = (BN <= 16) ? 4 : (BN <= 32 ? 6 : (BN <= 64 ? 12 : 8));  // weight ring
+    static constexpr int kS = (BN <= 16) ? 2 : (BN <= 32 ? 4 : (BN <= 64 ? 8 : 4));    // A stages
+    // Wide tiles instead share one ring between activation and A tiles (kRB = kS: one "ready"
+    // barrier counting the widening warps and the activation bytes, one "free" commit), which
+    // saves the MMA lane a wait and a commit per group.
+    static constexpr bool kSplitB = kNarrow;
+    static constexpr int kRB = kSplitB ? kRW + kS : kS;                                 // activation ring
     static constexpr int kNT = kNarrow ? 8 : (BN <= 64 ? 4 : 3);                   // TMEM partials
     static constexpr int kNTS = kNT / kGS;                       // partial stages (barrier pairs)
     // TMEM columns: partial buffers | widened A tiles (32 columns = 128 E4M3 per row)
@@ -140,7 +146,7 @@ struct WsCfg {
     static_assert(kTmemNeed <= 512 / kCtasPerSm, "TMEM budget");
     static constexpr int kUsStride = BN + 1;
     static constexpr int kOffB = 0;
-    static constexpr int kOffW = kOffB + kS * kGS * kBSlot;
+    static constexpr int kOffW = kOffB + kRB * kGS * kBSlot;
     static constexpr int kOffUs = kOffW + kRW * kRaw;
     static constexpr int kOffPre = kOffUs + 64 * kUsStride * 4;
     static constexpr int kOffFlag = kOffPre + 1025 * 4;          // BN ints (fused epilogues)
@@ -148,7 +154,7 @@ struct WsCfg {
     static constexpr int kMaxG = 128;                            // K <= 16384
     static constexpr int kOffQs = kOffSr + 2 * BN * 4;           // unsigned: [G][BN] group sums
     static constexpr int kOffBar = ((kOffQs + (kUnsigned ? kMaxG * BN * 4 : 0) + 7) / 8) * 8;
-    static constexpr int kNumBars = 2 * kRW + 2 * kS + 2 * kNTS;
+    static constexpr int kNumBars = 2 * kRW + (kSplitB ? 2 * kRB : 0) + 2 * kS + 2 * kNTS;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;     // TMEM slot, abort flag
     static constexpr int kBytes = kOffMisc + 16;
     static constexpr int kAlloc = kBytes + 1024;
@@ -210,9 +216,12 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + C::kOffBar);
     uint64_t* w_full = bar;                       // weight ring: TMA -> widening warps
     uint64_t* w_empty = w_full + C::kRW;          //              widening warps -> TMA
-    uint64_t* s_ready = w_empty + C::kRW;         // operand stage: widening warps + TMA bytes -> MMA
-    uint64_t* s_free = s_ready + C::kS;           //                MMA commit -> widening warps, TMA
-    uint64_t* t_full = s_free + C::kS;            // TMEM partials: MMA commit -> promotion
+    uint64_t* s_ready = w_empty + C::kRW;         // widened A stage: widening warps (+ TMA bytes) -> MMA
+    uint64_t* s_free = s_ready + C::kS;           //                  MMA commit -> widening warps
+    // activation ring (own barriers on narrow tiles; the A stage's otherwise)
+    uint64_t* b_full = C::kSplitB ? s_free + C::kS : s_ready;
+    uint64_t* b_empty = C::kSplitB ? b_full + C::kRB : s_free;
+    uint64_t* t_full = s_free + C::kS + (C::kSplitB ? 2 * C::kRB : 0);   // TMEM partials: MMA -> promotion
     uint64_t* t_empty = t_full + C::kNTS;         //                promotion -> MMA
     uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + C::kOffMisc);
     volatile int* abort = reinterpret_cast<volatile int*>(sm + C::kOffMisc + 4);
@@ -227,7 +236,12 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
 
     if (tid == 0) {
         for (int i = 0; i < C::kRW; ++i) { tc::mbar_init(&w_full[i], 1); tc::mbar_init(&w_empty[i], C::kNW); }
-        for (int i = 0; i < C::kS; ++i) { tc::mbar_init(&s_ready[i], C::kNW + 1); tc::mbar_init(&s_free[i], 1); }
+        if (C::kSplitB)
+            for (int i = 0; i < C::kRB; ++i) { tc::mbar_init(&b_full[i], 1); tc::mbar_init(&b_empty[i], 1); }
+        for (int i = 0; i < C::kS; ++i) {
+            tc::mbar_init(&s_ready[i], C::kNW + (C::kSplitB ? 0 : 1));
+            tc::mbar_init(&s_free[i], 1);
+        }
         for (int i = 0; i < C::kNTS; ++i) { tc::mbar_init(&t_full[i], 1); tc::mbar_init(&t_empty[i], C::kNP); }
         *abort = 0;
         tc::fence_mbar_init();
@@ -268,7 +282,7 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
             bool stop = false;
             for (int st = 0; st < nst; ++st, ++it) {
                 const int g0 = st * C::kGS, ng = min(C::kGS, G - g0);
-                const int ws_ = it % C::kRW, bs = it % C::kS;
+                const int ws_ = it % C::kRW, bs = it % C::kRB;
                 int ok = 1;
                 if (lane == 0) {
                     ok = ws::wait(&w_empty[ws_], ((it / C::kRW) & 1) ^ 1, abort);
@@ -283,8 +297,8 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
                         } else {
                             ws::tma_load_2d(wst, &tm_w0, g0 * 64, e * a.R0 + mt * 128, &w_full[ws_]);
                         }
-                        ok = ws::wait(&s_free[bs], ((it / C::kS) & 1) ^ 1, abort);
-                        if (ok) tc::mbar_arrive_expect_tx(&s_ready[bs], b_bytes * ng);
+                        ok = ws::wait(&b_empty[bs], ((it / C::kRB) & 1) ^ 1, abort);
+                        if (ok) tc::mbar_arrive_expect_tx(&b_full[bs], b_bytes * ng);
                     }
                 }
                 ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -294,9 +308,9 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
                     if (kGather) {
                         if (lane < ngather)
                             ws::tma_gather4(bst + lane * 512, &tm_act, (g0 + h) * kGroup, tok[0], tok[1], tok[2],
-                                            tok[3], &s_ready[bs]);
+                                            tok[3], &b_full[bs]);
                     } else if (lane == 0) {
-                        ws::tma_load_2d(bst, &tm_act, (g0 + h) * kGroup, row0, &s_ready[bs]);
+                        ws::tma_load_2d(bst, &tm_act, (g0 + h) * kGroup, row0, &b_full[bs]);
                     }
                 }
             }
@@ -310,12 +324,13 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
             for (int64_t tile = blockIdx.x; tile < n_tiles && !*abort; tile += gridDim.x) {
                 for (int st = 0; st < nst; ++st, ++it) {
                     const int ng = min(C::kGS, G - st * C::kGS);
-                    const int ss = it % C::kS, ts = it % C::kNTS;
+                    const int ss = it % C::kS, ts = it % C::kNTS, bs = it % C::kRB;
+                    if (C::kSplitB && !ws::wait(&b_full[bs], (it / C::kRB) & 1, abort)) break;
                     if (!ws::wait(&s_ready[ss], (it / C::kS) & 1, abort)) break;
                     if (!ws::wait(&t_empty[ts], ((it / C::kNTS) & 1) ^ 1, abort)) break;
                     tc::tc_fence_after();
                     for (int h = 0; h < ng; ++h) {
-                        const uint32_t b_addr = tc::smem_u32(bring + (ss * C::kGS + h) * C::kBSlot);
+                        const uint32_t b_addr = tc::smem_u32(bring + (bs * C::kGS + h) * C::kBSlot);
                         const uint32_t a_col = tmem + C::kColA + (ss * C::kGS + h) * 32;
                         const uint32_t d = tmem + (ts * C::kGS + h) * BN;
 #pragma unroll
@@ -325,11 +340,12 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
                     }
                     tc::mma_commit(&t_full[ts]);
                     tc::mma_commit(&s_free[ss]);
+                    if (C::kSplitB) tc::mma_commit(&b_empty[bs]);
                 }
             }
             // the commits complete in order: once the last one has arrived, no tensor-core
             // arrive on this CTA's barriers is still pending
-            if (it > 0) ws::wait(&s_free[(it - 1) % C::kS], ((it - 1) / C::kS) & 1, abort);
+            if (it > 0) ws::wait(&b_empty[(it - 1) % C::kRB], ((it - 1) / C::kRB) & 1, abort);
         }
     } else if (warp < C::kNW) {
         // ------------------------------------------------------------ widening warps
