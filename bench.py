@@ -14,7 +14,9 @@ own batches: weak scaling, no data-path collective.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
+import re
 import os
 import statistics
 import subprocess
@@ -50,6 +52,32 @@ def flops_per_pair(wl):
 def is_prefill(wl):
     """Prefill shapes are scored against the FP8 tensor peak, decode shapes against HBM."""
     return wl.T >= 1024
+
+
+KERNEL_SOURCES = ("gemm_ws.cuh", "tc_ptx.cuh", "tc_tiles.cuh", "common.cuh")
+PROFILE_FOR = {"decode_t8": "gemm_w4a8_ws_decode_t8.md",
+               "prefill_t2048_zipf": "gemm_w4a8_ws_prefill_t2048.md"}
+
+
+def ncu_traffic(workload):
+    """DRAM bytes per gate/up launch from the committed ncu summary of this workload, or None
+    when there is none or the GEMM sources changed since it was taken."""
+    name = PROFILE_FOR.get(workload)
+    if not name:
+        return None
+    try:
+        text = open(os.path.join(ROOT, "profiles", name)).read()
+        vals = dict(re.findall(r"^\s*(traffic_gateup_bytes_per_launch|sources_sha256):\s*(\S+)", text,
+                               flags=re.M))
+        h = hashlib.sha256()
+        for f in KERNEL_SOURCES:
+            with open(os.path.join(ROOT, "bit_quantized_moe_token_b200", "csrc", f), "rb") as fh:
+                h.update(fh.read())
+        if vals.get("sources_sha256") != h.hexdigest():
+            return None
+        return int(vals["traffic_gateup_bytes_per_launch"])
+    except (OSError, KeyError, ValueError):
+        return None
 
 
 def peaks():
@@ -292,7 +320,7 @@ def run_ours(args):
         fp8 = 2.0 * bf16
         roofline = {"bound": "tensor", "kernel": "grouped gate/up W4A8 GEMM (stage)",
                     "achieved": round(achieved, 1), "peak": round(fp8, 1), "unit": "TFLOP/s",
-                    "frac": round(achieved / fp8, 4), "traffic": None,
+                    "frac": round(achieved / fp8, 4), "traffic": ncu_traffic(wl.name),
                     "peak_source": f"{peak_kind} bf16_tflops x 2 (nominal FP8/BF16 ratio)",
                     "algorithmic_flops_per_launch": int(dom_flops),
                     "units": f"{T * k} routed pairs x {2 * wl.H * 2 * wl.N} FLOP (gate+up)"}
@@ -300,7 +328,7 @@ def run_ours(args):
         achieved = dom_bytes / (dom_ms / 1e3) / 1e9
         roofline = {"bound": "hbm", "kernel": "grouped gate/up W4A8 GEMM (stage)",
                     "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
-                    "frac": round(achieved / hbm, 4), "traffic": None,
+                    "frac": round(achieved / hbm, 4), "traffic": ncu_traffic(wl.name),
                     "peak_source": f"{peak_kind} hbm_gbs",
                     "algorithmic_bytes_per_launch": int(dom_bytes),
                     "units": f"{mean_touched:.1f} touched experts x {gu_bytes} B (gate+up codes+scales)"}
