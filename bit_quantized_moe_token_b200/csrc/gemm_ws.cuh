@@ -149,7 +149,8 @@ struct WsCfg {
     static constexpr int kOffW = kOffB + kRB * kGS * kBSlot;
     static constexpr int kOffUs = kOffW + kRW * kRaw;
     static constexpr int kOffPre = kOffUs + 64 * kUsStride * 4;
-    static constexpr int kOffFlag = kOffPre + 1025 * 4;          // BN ints (fused epilogues)
+    static constexpr int kOffSoff = kOffPre + 1025 * 4;          // segment offsets [0..E]
+    static constexpr int kOffFlag = kOffSoff + 1025 * 4;         // BN ints (fused epilogues)
     static constexpr int kOffSr = kOffFlag + BN * 4;             // 2 x BN per-column scales
     static constexpr int kMaxG = 128;                            // K <= 16384
     static constexpr int kOffQs = kOffSr + 2 * BN * 4;           // unsigned: [G][BN] group sums
@@ -163,10 +164,11 @@ struct WsCfg {
     // columns), 12 TMA, 13 MMA.  A promotion thread issues up to 32 columns of TMEM loads before
     // each wait, so a 128-column group costs two load round trips.
     static constexpr int kNW = kNarrow ? 8 : 4;                 // widening warps
-    static constexpr int kNP = kNarrow ? 4 : 8;                 // promotion / epilogue warps
+    static constexpr int kNP = kNarrow ? 4 : (BN >= 128 ? 16 : 8);   // promotion / epilogue warps
     static constexpr int kCPW = BN / (kNP / 4);                 // token columns per promotion thread
     static constexpr int kWarpTma = kNW + kNP, kWarpMma = kNW + kNP + 1;
-    static constexpr int kLd = kCPW < 32 ? kCPW : 32;          // TMEM columns per load wait
+    // TMEM columns per load wait (16 where 704 threads leave 88 registers per thread)
+    static constexpr int kLd = kNP > 8 ? 16 : (kCPW < 32 ? kCPW : 32);
     static constexpr int kThreads = 32 * (kNW + kNP + 2);
 };
 
@@ -210,6 +212,7 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
     uint8_t* wring = sm + C::kOffW;
     float* sUs = reinterpret_cast<float*>(sm + C::kOffUs);
     int* pre = reinterpret_cast<int*>(sm + C::kOffPre);
+    int* soff = reinterpret_cast<int*>(sm + C::kOffSoff);
     int* flag = reinterpret_cast<int*>(sm + C::kOffFlag);
     float* sSr = reinterpret_cast<float*>(sm + C::kOffSr);
     float* sQs = reinterpret_cast<float*>(sm + C::kOffQs);
@@ -230,7 +233,7 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
     const int G = a.K / kGroup;
     const int nst = (G + C::kGS - 1) / C::kGS;             // stages per tile
     const int m_tiles = kSwiGLU ? a.R0 / 64 : a.R0 / 128;
-    const int row_tiles = row_tile_prefix(a.offsets, a.E, BN, pre);
+    const int row_tiles = row_tile_prefix(a.offsets, a.E, BN, pre, soff);
     const int64_t n_tiles = (int64_t)row_tiles * m_tiles;
     if ((int64_t)blockIdx.x >= n_tiles) return;
 
@@ -270,8 +273,8 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
             if (__shfl_sync(0xffffffffu, *abort, 0)) break;
             const int rt = static_cast<int>(tile / m_tiles), mt = static_cast<int>(tile % m_tiles);
             const int e = expert_of_tile(pre, a.E, rt);
-            const int row0 = a.offsets[e] + (rt - pre[e]) * BN;
-            const int nrows = min(BN, a.offsets[e + 1] - row0);
+            const int row0 = soff[e] + (rt - pre[e]) * BN;
+            const int nrows = min(BN, soff[e + 1] - row0);
             const int ngather = (nrows + 3) / 4;
             int tok[4] = {0, 0, 0, 0};
             if (kGather && lane < ngather) {
@@ -414,9 +417,9 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
         for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
             const int rt = static_cast<int>(tile / m_tiles), mt = static_cast<int>(tile % m_tiles);
             const int e = expert_of_tile(pre, a.E, rt);
-            const int seg0 = a.offsets[e];
+            const int seg0 = soff[e];
             const int r0 = (rt - pre[e]) * BN;
-            const int nrows = min(BN, a.offsets[e + 1] - seg0 - r0);
+            const int nrows = min(BN, soff[e + 1] - seg0 - r0);
             const int64_t row0 = seg0 + r0;
             const int lrow = (warp & 3) * 32 + lane;       // this thread's A row / TMEM lane
             // token scale of column pt, fetched now and staged in shared memory for the epilogue

@@ -53,14 +53,18 @@ __device__ __forceinline__ uint32_t sw128_off(int r, int j) {
 // ---- tile map ------------------------------------------------------------------------------
 
 // Per-expert prefix of row tiles (ceil(len / BN)) into shared `pre[0..E]`; returns the total.
-__device__ int row_tile_prefix(const int32_t* __restrict__ offsets, int E, int BN, int* pre) {
+// With `soff` non-null the segment offsets [0..E] are copied there too.
+__device__ int row_tile_prefix(const int32_t* __restrict__ offsets, int E, int BN, int* pre,
+                               int* soff = nullptr) {
     __shared__ int s_total;
     if (threadIdx.x < 32) {
         const int lane = threadIdx.x;
         int run = 0;
         for (int e0 = 0; e0 < E; e0 += 32) {
             const int e = e0 + lane;
-            const int n = (e < E) ? (offsets[e + 1] - offsets[e] + BN - 1) / BN : 0;
+            const int o0 = (e < E) ? offsets[e] : 0, o1 = (e < E) ? offsets[e + 1] : 0;
+            if (soff && e < E) soff[e] = o0;
+            const int n = (e < E) ? (o1 - o0 + BN - 1) / BN : 0;
             int inc = n;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
@@ -70,7 +74,11 @@ __device__ int row_tile_prefix(const int32_t* __restrict__ offsets, int E, int B
             if (e < E) pre[e] = run + inc - n;
             run += __shfl_sync(0xffffffffu, inc, 31);
         }
-        if (lane == 0) { pre[E] = run; s_total = run; }
+        if (lane == 0) {
+            pre[E] = run;
+            s_total = run;
+            if (soff) soff[E] = offsets[E];
+        }
     }
     __syncthreads();
     return s_total;
