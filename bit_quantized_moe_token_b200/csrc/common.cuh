@@ -79,6 +79,12 @@ __device__ __forceinline__ float warp_max(float v) {
     return v;
 }
 
+// g * sigmoid(g) with the hardware exp2-based exponential and fast division: a few ulp from
+// the IEEE form below, orders of magnitude under the FP8 rounding step that follows it.
+__device__ __forceinline__ float silu_fast(float g) {
+    return __fdividef(g, 1.0f + __expf(-g));
+}
+
 __device__ __forceinline__ float silu(float g) {
     // g * sigmoid(g) with IEEE division; expf is CUDA's (max 2 ulp).
     return g * __fdiv_rn(1.0f, 1.0f + expf(-g));

@@ -413,6 +413,22 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
         const int ch = (warp - C::kNW) >> 2;              // column block of this warp
         const int c_base = ch * kCPW;
         const uint32_t t_lane = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const int lrow = (warp & 3) * 32 + lane;           // this thread's A row / TMEM lane
+        // group-scale row of this thread in a tile; the first scales of the next tile are fetched
+        // before the current tile's epilogue so that a tile never starts on a DRAM round trip
+        auto scale_row = [&](int64_t t) -> const uint16_t* {
+            const int rt_ = static_cast<int>(t / m_tiles), mt_ = static_cast<int>(t % m_tiles);
+            const int e_ = expert_of_tile(pre, a.E, rt_);
+            if (kSwiGLU)
+                return (lrow < 64 ? a.s0 : a.s1) + ((int64_t)e_ * a.R0 + mt_ * 64 + (lrow & 63)) * G;
+            return a.s0 + ((int64_t)e_ * a.R0 + mt_ * 128 + lrow) * G;
+        };
+        uint16_t first_raw[C::kGS];
+        if (kSwiGLU && !C::kNarrow) {
+            const uint16_t* s0 = scale_row(blockIdx.x);
+#pragma unroll
+            for (int h = 0; h < C::kGS; ++h) first_raw[h] = h < G ? __ldg(s0 + h) : uint16_t(0);
+        }
         uint32_t it = 0, tcount = 0;
         for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
             const int rt = static_cast<int>(tile / m_tiles), mt = static_cast<int>(tile % m_tiles);
@@ -421,19 +437,13 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
             const int r0 = (rt - pre[e]) * BN;
             const int nrows = min(BN, soff[e + 1] - seg0 - r0);
             const int64_t row0 = seg0 + r0;
-            const int lrow = (warp & 3) * 32 + lane;       // this thread's A row / TMEM lane
             // token scale of column pt, fetched now and staged in shared memory for the epilogue
             float my_sr = 0.0f;
             if (pt < nrows) my_sr = kGather ? a.s_row[a.sorted[row0 + pt] / a.k] : a.s_row[row0 + pt];
             float* sr_t = sSr + (tcount & 1) * BN;         // two buffers: tile parity
             ++tcount;
-            const uint16_t* ssrc;
-            if (kSwiGLU) {
-                const int n = mt * 64 + (lrow & 63);
-                ssrc = (lrow < 64 ? a.s0 : a.s1) + ((int64_t)e * a.R0 + n) * G;
-            } else {
-                ssrc = a.s0 + ((int64_t)e * a.R0 + mt * 128 + lrow) * G;
-            }
+            const uint16_t* ssrc = scale_row(tile);
+            (void)mt;
             if constexpr (kUnsigned) {   // the tile's activation group sums, sQs[g * BN + j]
                 for (int i = pt; i < G * BN; i += kNPT) {
                     const int j = i / G, g = i - j * G;
@@ -451,7 +461,9 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
             for (int j = 0; j < kCPW; ++j) acc[j] = 0.0f;
             float sc_next[C::kGS];
 #pragma unroll
-            for (int h = 0; h < C::kGS; ++h) sc_next[h] = h < G ? bf16_bits_to_f32(__ldg(ssrc + h)) : 0.0f;
+            for (int h = 0; h < C::kGS; ++h)
+                sc_next[h] = bf16_bits_to_f32((C::kNarrow || !kSwiGLU) ? (h < G ? __ldg(ssrc + h) : uint16_t(0))
+                                                                        : first_raw[h]);
             for (int st = 0; st < nst; ++st, ++it) {
                 const int g0 = st * C::kGS;
                 float scs[C::kGS];
@@ -492,6 +504,12 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
                 if (lane == 0) tc::mbar_arrive(&t_empty[ts]);
             }
 
+            if (kSwiGLU && !C::kNarrow && tile + gridDim.x < n_tiles) {   // wide gate/up tiles only
+                const uint16_t* sn = scale_row(tile + gridDim.x);
+#pragma unroll
+                for (int h = 0; h < C::kGS; ++h) first_raw[h] = h < G ? __ldg(sn + h) : uint16_t(0);
+            }
+
             // ---- epilogue (static indices keep acc[] in registers) ----
             // The column scales come from shared memory, so no load waits behind the stores, and
             // the per-column max|h| is one redux per warp.
@@ -514,7 +532,7 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
                     const float other = sUs[r64 * C::kUsStride + c_mine + j];
                     const float gv = gate ? acc[j] : other;
                     const float uv = gate ? other : acc[kHalf + j];
-                    acc[j] = silu(gv * sr) * (uv * sr);
+                    acc[j] = silu_fast(gv * sr) * (uv * sr);
                 }
 #pragma unroll
                 for (int j = 0; j < kHalf; ++j)
