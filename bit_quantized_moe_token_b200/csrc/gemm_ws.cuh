@@ -543,9 +543,13 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
                     if (lane == 0 && c_mine + j < nrows) atomicMax(a.amax + row0 + c_mine + j, m);
                 }
                 if constexpr (kFused) {
-                    __threadfence();
+                    // The barrier orders every thread's h stores before the counting threads'
+                    // fences, and a fence is cumulative, so one fence per counted row suffices.
                     ws::named_sync_math<kNPT>();
-                    if (pt < nrows) flag[pt] = atomicAdd(a.cnt + row0 + pt, 1u) == (unsigned)(m_tiles - 1);
+                    if (pt < nrows) {
+                        __threadfence();
+                        flag[pt] = atomicAdd(a.cnt + row0 + pt, 1u) == (unsigned)(m_tiles - 1);
+                    }
                     ws::named_sync_math<kNPT>();
                     for (int j = 0; j < nrows; ++j) {
                         if (flag[j]) {
@@ -565,9 +569,9 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
                 for (int j = 0; j < kCPW; ++j)
                     if (c_base + j < nrows) a.out[(row0 + c_base + j) * a.ldo + m] = acc[j] * sr_t[c_base + j];
                 if constexpr (kFused) {
-                    __threadfence();
-                    ws::named_sync_math<kNPT>();
+                    ws::named_sync_math<kNPT>();          // as above: one fence per counted row
                     if (pt < nrows) {
+                        __threadfence();
                         const int t = a.sorted[row0 + pt] / a.k;
                         flag[pt] = atomicAdd(a.cnt + (int64_t)t * m_tiles + mt, 1u) == (unsigned)(a.k - 1) ? t : -1;
                     }
