@@ -103,6 +103,7 @@ __device__ __forceinline__ void named_sync_math() {
 
 // Bounded wait that gives up at once after an abort.
 __device__ __forceinline__ bool wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+    if (tc::mbar_try_wait(bar, parity)) return true;      // completed phase: no flag read
     if (*abort) return false;
     if (tc::mbar_wait(bar, parity)) return true;
     *abort = 1;
@@ -333,13 +334,14 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
                     if (!ws::wait(&t_empty[ts], ((it / C::kNTS) & 1) ^ 1, abort)) break;
                     tc::tc_fence_after();
                     for (int h = 0; h < ng; ++h) {
-                        const uint32_t b_addr = tc::smem_u32(bring + (bs * C::kGS + h) * C::kBSlot);
+                        // K step of 32 bytes = +2 in the descriptor's start-address field (the
+                        // 1024-byte-aligned tiles keep it from carrying)
+                        const uint64_t bd = tc::sdesc_sw128(tc::smem_u32(bring + (bs * C::kGS + h) * C::kBSlot));
                         const uint32_t a_col = tmem + C::kColA + (ss * C::kGS + h) * 32;
                         const uint32_t d = tmem + (ts * C::kGS + h) * BN;
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)
-                            tc::mma_e4m3_ta(d, a_col + kk * 8, tc::sdesc_sw128(b_addr + kk * 32), idesc,
-                                            kk > 0 ? 1u : 0u);
+                            tc::mma_e4m3_ta(d, a_col + kk * 8, bd + 2 * kk, idesc, kk > 0 ? 1u : 0u);
                     }
                     tc::mma_commit(&t_full[ts]);
                     tc::mma_commit(&s_free[ss]);
