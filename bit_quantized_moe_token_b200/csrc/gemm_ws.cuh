@@ -101,6 +101,16 @@ __device__ __forceinline__ void named_sync_math() {
 }
 
 
+// Slot and phase parity of a ring of N stages, advanced once per stage (no division).
+template <int N>
+struct Ring {
+    int idx = 0;
+    uint32_t phase = 0;
+    __device__ __forceinline__ void next() {
+        if (++idx == N) { idx = 0; phase ^= 1u; }
+    }
+};
+
 // Bounded wait that gives up at once after an abort.
 __device__ __forceinline__ bool wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
     if (tc::mbar_try_wait(bar, parity)) return true;      // completed phase: no flag read
@@ -269,7 +279,8 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
             if (kSwiGLU) ws::prefetch_map(&tm_w1);
             ws::prefetch_map(&tm_act);
         }
-        uint32_t it = 0;
+        ws::Ring<C::kRW> rw;
+        ws::Ring<C::kRB> rb;
         for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
             if (__shfl_sync(0xffffffffu, *abort, 0)) break;
             const int rt = static_cast<int>(tile / m_tiles), mt = static_cast<int>(tile % m_tiles);
@@ -284,12 +295,12 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
             }
             const uint32_t b_bytes = kGather ? static_cast<uint32_t>(ngather) * 512u : C::kB;
             bool stop = false;
-            for (int st = 0; st < nst; ++st, ++it) {
+            for (int st = 0; st < nst; ++st, rw.next(), rb.next()) {
                 const int g0 = st * C::kGS, ng = min(C::kGS, G - g0);
-                const int ws_ = it % C::kRW, bs = it % C::kRB;
+                const int ws_ = rw.idx, bs = rb.idx;
                 int ok = 1;
                 if (lane == 0) {
-                    ok = ws::wait(&w_empty[ws_], ((it / C::kRW) & 1) ^ 1, abort);
+                    ok = ws::wait(&w_empty[ws_], rw.phase ^ 1u, abort);
                     if (ok) {
                         // a stage past K (odd group count) is filled with zeros by the TMA unit
                         uint8_t* wst = wring + ws_ * C::kRaw;
@@ -301,7 +312,7 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
                         } else {
                             ws::tma_load_2d(wst, &tm_w0, g0 * 64, e * a.R0 + mt * 128, &w_full[ws_]);
                         }
-                        ok = ws::wait(&b_empty[bs], ((it / C::kRB) & 1) ^ 1, abort);
+                        ok = ws::wait(&b_empty[bs], rb.phase ^ 1u, abort);
                         if (ok) tc::mbar_arrive_expect_tx(&b_full[bs], b_bytes * ng);
                     }
                 }
@@ -324,33 +335,43 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc = tc::idesc_e4m3_f32(128, BN);
-            uint32_t it = 0;
+            // descriptor of activation slot 0; slot i starts i * kBSlot / 16 later in the
+            // start-address field, and a K step of 32 bytes adds 2 (1024-byte-aligned tiles in
+            // the first 256 KB of shared memory keep the 14-bit field from carrying)
+            const uint64_t bd0 = tc::sdesc_sw128(tc::smem_u32(bring));
+            ws::Ring<C::kS> rs;
+            ws::Ring<C::kNTS> rt;
+            ws::Ring<C::kRB> rb;
+            int last_b = -1;
+            uint32_t last_bp = 0;
             for (int64_t tile = blockIdx.x; tile < n_tiles && !*abort; tile += gridDim.x) {
-                for (int st = 0; st < nst; ++st, ++it) {
-                    const int ng = min(C::kGS, G - st * C::kGS);
-                    const int ss = it % C::kS, ts = it % C::kNTS, bs = it % C::kRB;
-                    if (C::kSplitB && !ws::wait(&b_full[bs], (it / C::kRB) & 1, abort)) break;
-                    if (!ws::wait(&s_ready[ss], (it / C::kS) & 1, abort)) break;
-                    if (!ws::wait(&t_empty[ts], ((it / C::kNTS) & 1) ^ 1, abort)) break;
+                for (int st = 0; st < nst; ++st) {
+                    const int ng = C::kGS == 1 ? 1 : min(C::kGS, G - st * C::kGS);
+                    if (C::kSplitB && !ws::wait(&b_full[rb.idx], rb.phase, abort)) break;
+                    if (!ws::wait(&s_ready[rs.idx], rs.phase, abort)) break;
+                    if (!ws::wait(&t_empty[rt.idx], rt.phase ^ 1u, abort)) break;
                     tc::tc_fence_after();
                     for (int h = 0; h < ng; ++h) {
-                        // K step of 32 bytes = +2 in the descriptor's start-address field (the
-                        // 1024-byte-aligned tiles keep it from carrying)
-                        const uint64_t bd = tc::sdesc_sw128(tc::smem_u32(bring + (bs * C::kGS + h) * C::kBSlot));
-                        const uint32_t a_col = tmem + C::kColA + (ss * C::kGS + h) * 32;
-                        const uint32_t d = tmem + (ts * C::kGS + h) * BN;
+                        const uint64_t bd = bd0 + static_cast<uint64_t>((rb.idx * C::kGS + h) * (C::kBSlot >> 4));
+                        const uint32_t a_col = tmem + C::kColA + (rs.idx * C::kGS + h) * 32;
+                        const uint32_t d = tmem + (rt.idx * C::kGS + h) * BN;
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)
                             tc::mma_e4m3_ta(d, a_col + kk * 8, bd + 2 * kk, idesc, kk > 0 ? 1u : 0u);
                     }
-                    tc::mma_commit(&t_full[ts]);
-                    tc::mma_commit(&s_free[ss]);
-                    if (C::kSplitB) tc::mma_commit(&b_empty[bs]);
+                    tc::mma_commit(&t_full[rt.idx]);
+                    tc::mma_commit(&s_free[rs.idx]);
+                    if (C::kSplitB) tc::mma_commit(&b_empty[rb.idx]);
+                    last_b = rb.idx;
+                    last_bp = rb.phase;
+                    rs.next();
+                    rt.next();
+                    rb.next();
                 }
             }
             // the commits complete in order: once the last one has arrived, no tensor-core
             // arrive on this CTA's barriers is still pending
-            if (it > 0) ws::wait(&b_empty[(it - 1) % C::kRB], ((it - 1) / C::kRB) & 1, abort);
+            if (last_b >= 0) ws::wait(&b_empty[last_b], last_bp, abort);
         }
     } else if (warp < C::kNW) {
         // ------------------------------------------------------------ widening warps
@@ -365,11 +386,12 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
         const int row = quad * 32 + lane;
         const int swz = C::kGS == 1 ? (row >> 1) & 3 : row & 7;
         const uint32_t t_dst = tmem + (static_cast<uint32_t>(quad * 32) << 16) + C::kColA + part * 8 * kChunks;
-        uint32_t it = 0;
+        ws::Ring<C::kRW> rw;
+        ws::Ring<C::kS> ra;
         for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
-            for (int st = 0; st < nst; ++st, ++it) {
-                const int ws_ = it % C::kRW, as = it % C::kS;
-                ws::wait(&w_full[ws_], (it / C::kRW) & 1, abort);
+            for (int st = 0; st < nst; ++st, rw.next(), ra.next()) {
+                const int ws_ = rw.idx, as = ra.idx;
+                ws::wait(&w_full[ws_], rw.phase, abort);
                 const uint8_t* raw = wring + ws_ * C::kRaw + row * C::kRowB;
                 uint4 w[C::kGS][kChunks];
 #pragma unroll
@@ -380,7 +402,7 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
                 tc::fence_proxy_async_smem();              // order these reads before the next TMA write
                 __syncwarp();                              // this warp's reads of the slot are done
                 if (lane == 0) tc::mbar_arrive(&w_empty[ws_]);
-                ws::wait(&s_free[as], ((it / C::kS) & 1) ^ 1, abort);
+                ws::wait(&s_free[as], ra.phase ^ 1u, abort);
                 tc::tc_fence_after();
 #pragma unroll
                 for (int h = 0; h < C::kGS; ++h) {
@@ -431,7 +453,8 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
 #pragma unroll
             for (int h = 0; h < C::kGS; ++h) first_raw[h] = h < G ? __ldg(s0 + h) : uint16_t(0);
         }
-        uint32_t it = 0, tcount = 0;
+        uint32_t tcount = 0;
+        ws::Ring<C::kNTS> rq;
         for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
             const int rt = static_cast<int>(tile / m_tiles), mt = static_cast<int>(tile % m_tiles);
             const int e = expert_of_tile(pre, a.E, rt);
@@ -466,7 +489,7 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
             for (int h = 0; h < C::kGS; ++h)
                 sc_next[h] = bf16_bits_to_f32((C::kNarrow || !kSwiGLU) ? (h < G ? __ldg(ssrc + h) : uint16_t(0))
                                                                         : first_raw[h]);
-            for (int st = 0; st < nst; ++st, ++it) {
+            for (int st = 0; st < nst; ++st, rq.next()) {
                 const int g0 = st * C::kGS;
                 float scs[C::kGS];
 #pragma unroll
@@ -475,8 +498,8 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
                     const int gn = g0 + C::kGS + h;
                     if (gn < G) sc_next[h] = bf16_bits_to_f32(__ldg(ssrc + gn));
                 }
-                const int ts = it % C::kNTS;
-                ws::wait(&t_full[ts], (it / C::kNTS) & 1, abort);
+                const int ts = rq.idx;
+                ws::wait(&t_full[ts], rq.phase, abort);
                 tc::tc_fence_after();
 #pragma unroll
                 for (int h = 0; h < C::kGS; ++h) {
