@@ -329,7 +329,7 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const uint16_t* x_bf16,
     {
         WsGemmArgs a{fused ? sx : sxs, L.gate_scales, L.up_scales, offsets, L.E, L.N, L.H, (int)P, h, L.N,
                      amax, rowcnt, hq, sh, sorted, nullptr, nullptr, k, nullptr, nullptr, (int)T,
-                     fused ? qs_x : nullptr, fused ? qs_h : nullptr};
+                     fused ? qs_x : nullptr, nullptr};
         if ((st = launch_gemm_ws<true>(a, fused ? (const void*)xq : (const void*)xs, L.gate_packed,
                                        L.up_packed, stream)))
             return st;
@@ -347,7 +347,7 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const uint16_t* x_bf16,
     {
         WsGemmArgs a{sh, L.down_scales, nullptr, offsets, L.E, L.H, L.N, (int)P, y, L.H, nullptr,
                      tokcnt, nullptr, nullptr, sorted, rop, gates, k, shared, out_bf16, (int)T,
-                     fused ? qs_h : nullptr, nullptr};
+                     nullptr, nullptr};
         if ((st = launch_gemm_ws<false>(a, hq, L.down_packed, nullptr, stream))) return st;
         sm.launches += 1;
     }

@@ -18,12 +18,13 @@
 //              promotion warps and release the ring / A stages; the warp also owns the TMEM.
 //
 // Widening (see tc_tiles.cuh for the arithmetic):
-//   kUnsigned (narrow token tiles, decode): byte = nibble = E4M3 of (code+8)*2^-9, so TMEM
+//   kUnsigned (narrow gate/up tiles, decode): byte = nibble = E4M3 of (code+8)*2^-9, so TMEM
 //     holds 2^-9 * sum_k q_k*(code_k + 8) and the promotion subtracts the offset term with the
 //     group's activation sum: acc += 512*s*partial - 8*s*sum_k q_k (one more FMA per element;
 //     a tcgen05.mma costs the same issue time at N = 16 as at N = 64, so the offset is cheaper
 //     in the promotion than as four more MMAs).
-//   signed (wide token tiles, prefill): byte = E4M3(code) by byte-permute lookup.
+//   signed (the down GEMM and all wide token tiles): byte = E4M3(code) by byte-permute lookup;
+//     exact codes, so no offset term that would amplify the tensor core's accumulation error.
 //
 // Every mbarrier wait is bounded; a timeout sets a CTA-wide abort flag that turns all later
 // waits into no-ops (so the named barrier among the promotion warps stays uniform), records
@@ -704,8 +705,11 @@ int launch_gemm_ws(const WsGemmArgs& a, const void* act, const void* w0, const v
     const int BN = tc_tile_rows(a.P, a.E);
     const int64_t max_row_tiles = ((int64_t)a.P + BN - 1) / BN + a.E;
     switch (BN) {
-        case 16: return launch_gemm_ws_inst<16, true, kSwiGLU, true, kSwiGLU>(a, act, w0, w1, max_row_tiles, stream);
-        case 32: return launch_gemm_ws_inst<32, true, kSwiGLU, true, kSwiGLU>(a, act, w0, w1, max_row_tiles, stream);
+        // narrow gate/up tiles widen unsigned (the FP8 requantization after them absorbs the
+        // accumulation error of the +8 offset); the down GEMM, whose sums are the layer output,
+        // keeps the exact signed codes
+        case 16: return launch_gemm_ws_inst<16, kSwiGLU, kSwiGLU, true, kSwiGLU>(a, act, w0, w1, max_row_tiles, stream);
+        case 32: return launch_gemm_ws_inst<32, kSwiGLU, kSwiGLU, true, kSwiGLU>(a, act, w0, w1, max_row_tiles, stream);
         case 64: return launch_gemm_ws_inst<64, false, kSwiGLU, false, false>(a, act, w0, w1, max_row_tiles, stream);
         default: return launch_gemm_ws_inst<128, false, kSwiGLU, false, false>(a, act, w0, w1, max_row_tiles, stream);
     }
