@@ -68,6 +68,7 @@ def lib():
         L.or_quant_tokens.argtypes = [vp, i64, i64, vp, vp]
         L.or_quant_tokens.restype = None
         L.or_route_topk.argtypes = [vp, i64, i32, i32, vp, vp]
+        L.or_router_logits.argtypes = [vp, vp, i64, i64, i32, vp]
         L.or_route_topk.restype = None
         L.or_permute.argtypes = [vp, i64, i32, i32, vp, vp, vp]
         L.or_permute.restype = None
@@ -135,6 +136,18 @@ def quant_tokens(x_bf16: np.ndarray):
     s = np.zeros(T, np.float32)
     lib().or_quant_tokens(_p(x), T, H, _p(q), _p(s))
     return q, s
+
+
+def router_logits(x_bf16: np.ndarray, wr_bf16: np.ndarray) -> np.ndarray:
+    """[T, E] fp32 logits of bf16 tokens [T, H] against the bf16 router weight [E, H]."""
+    x = np.ascontiguousarray(x_bf16, np.uint16)
+    w = np.ascontiguousarray(wr_bf16, np.uint16)
+    T, H = x.shape
+    E = w.shape[0]
+    assert w.shape[1] == H
+    out = np.zeros((T, E), np.float32)
+    lib().or_router_logits(_p(x), _p(w), T, H, E, _p(out))
+    return out
 
 
 def route_topk(logits: np.ndarray, k: int):

@@ -35,7 +35,9 @@
  *   R5 group partial sums in increasing k, promoted with the group scale in
  *      increasing g, token scale applied last; combine sums the k routed
  *      outputs in selection order, adds the shared experts, rounds once to
- *      bf16.
+ *      bf16;
+ *   R6 router logits = x . wr over the bf16 router weight, no bias, fp32
+ *      accumulation in increasing k.
  */
 #include <math.h>
 #include <stdint.h>
@@ -188,6 +190,25 @@ void or_quant_tokens(const uint16_t* x, int64_t T, int64_t H, uint8_t* q, float*
         quant_row_f32(row, H, q + t * H, s + t);
         free(row);
     }
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* Router (the step upstream of S2): logits[t][e] = sum over k of x[t][k] * wr[e][k] with the  */
+/* router weight kept in its source bf16 precision ("Baekpica/Inkling-Small-Mixed-Quant-GGUF"  */
+/* card, "Precision differences": router tensors stay native; [P2] "Layout summary": the gate */
+/* is copied verbatim).  Reading R6: no bias, fp32 accumulation in increasing k; each product */
+/* of two bf16 values is exact in fp32, so only the running sum rounds.                       */
+/* ------------------------------------------------------------------------------------------ */
+
+void or_router_logits(const uint16_t* x, const uint16_t* wr, int64_t T, int64_t H, int E,
+                      float* logits) {
+    for (int64_t t = 0; t < T; ++t)
+        for (int e = 0; e < E; ++e) {
+            float acc = 0.0f;
+            for (int64_t k = 0; k < H; ++k)
+                acc += or_bf16_to_f32(x[t * H + k]) * or_bf16_to_f32(wr[(int64_t)e * H + k]);
+            logits[t * E + e] = acc;
+        }
 }
 
 /* ------------------------------------------------------------------------------------------ */

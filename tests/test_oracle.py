@@ -250,6 +250,64 @@ def test_routing_vs_sort_and_softmax():
             assert np.allclose(back, full, rtol=2e-6, atol=1e-7)
 
 
+# ------------------------------------------------------------------------------------------------
+# Router logits (the step upstream of top-k)
+# ------------------------------------------------------------------------------------------------
+
+def _bf16(a):
+    """fp32 array -> bf16 bits, round to nearest even (numpy, independent of the oracle)."""
+    u = np.asarray(a, np.float32).view(np.uint32).astype(np.uint64)
+    return ((u + 0x7FFF + ((u >> 16) & 1)) >> 16).astype(np.uint16)
+
+
+def _f32(b):
+    return (np.asarray(b, np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+def test_router_one_hot_rows_select_weight_columns():
+    """x = e_j picks column j of the router weight: catches a transposed or shifted operand."""
+    rng = np.random.default_rng(11)
+    E, H = 12, 256
+    wr = _bf16(rng.standard_normal((E, H)) / 16)
+    cols = [0, 1, 77, 128, 255]
+    x = np.zeros((len(cols), H), np.uint16)
+    for t, j in enumerate(cols):
+        x[t, j] = 0x3F80                                    # bf16 1.0
+    got = oracle.router_logits(x, wr)
+    assert np.array_equal(got, _f32(wr[:, cols]).T)
+
+
+def test_router_two_terms_round_once():
+    """Two non-zero inputs: each bf16 product is exact in fp32, the sum rounds once."""
+    rng = np.random.default_rng(12)
+    E, H = 9, 384
+    wr = _bf16(rng.standard_normal((E, H)))
+    x = np.zeros((20, H), np.uint16)
+    want = np.zeros((20, E), np.float32)
+    for t in range(20):
+        j1, j2 = sorted(rng.choice(H, 2, replace=False))
+        a, b = _bf16(rng.standard_normal(2) * 3)
+        x[t, j1], x[t, j2] = a, b
+        exact = (_f32(a).astype(np.float64) * _f32(wr[:, j1]).astype(np.float64)
+                 + _f32(b).astype(np.float64) * _f32(wr[:, j2]).astype(np.float64))
+        want[t] = exact.astype(np.float32)
+    assert np.array_equal(oracle.router_logits(x, wr), want)
+
+
+def test_router_within_sequential_fp32_bound():
+    """|fp32 sequential sum - exact| <= (H-1) * 2^-24 * sum |x_k w_k| (standard summation bound)."""
+    rng = np.random.default_rng(13)
+    T, E, H = 7, 40, 512
+    x = _bf16(rng.standard_normal((T, H)))
+    wr = _bf16(rng.standard_normal((E, H)) / math.sqrt(H))
+    got = oracle.router_logits(x, wr).astype(np.float64)
+    xf, wf = _f32(x).astype(np.float64), _f32(wr).astype(np.float64)
+    exact = xf @ wf.T
+    bound = (H - 1) * 2.0 ** -24 * (np.abs(xf) @ np.abs(wf).T)
+    assert np.all(np.abs(got - exact) <= bound)
+    assert np.abs(got - exact).max() > 0                   # it is a real fp32 sum, not fp64
+
+
 def test_permutation_vs_stable_sort():
     rng = np.random.default_rng(5)
     for T, k, E in ((50, 6, 256), (16, 2, 8), (1, 1, 1), (0, 2, 8), (333, 3, 17)):
