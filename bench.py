@@ -16,6 +16,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+import math
 import re
 import os
 import statistics
@@ -47,6 +48,22 @@ def expert_bytes(wl):
 
 def flops_per_pair(wl):
     return 2 * wl.H * 2 * wl.N + 2 * wl.N * wl.H
+
+
+def router_line(wl, T, ms, hbm, bf16, peak_kind):
+    """The router GEMM (moe_router_logits), timed apart from the layer step: HBM-bound at decode
+    (the bf16 router weight is read once), bf16-tensor-bound at prefill."""
+    if is_prefill(wl):
+        flops = 2.0 * T * wl.H * wl.E
+        ach = flops / (ms / 1e3) / 1e12
+        return {"ms": round(ms, 4), "bound": "tensor", "achieved": round(ach, 1), "peak": bf16,
+                "unit": "TFLOP/s", "frac": round(ach / bf16, 4),
+                "peak_source": f"{peak_kind} bf16_tflops"}
+    nbytes = wl.E * wl.H * 2 + T * wl.H * 2 + T * wl.E * 4
+    ach = nbytes / (ms / 1e3) / 1e9
+    return {"ms": round(ms, 4), "bound": "hbm", "achieved": round(ach, 1), "peak": hbm,
+            "unit": "GB/s", "frac": round(ach / hbm, 4), "peak_source": f"{peak_kind} hbm_gbs",
+            "algorithmic_bytes": int(nbytes)}
 
 
 def is_prefill(wl):
@@ -306,6 +323,22 @@ def run_ours(args):
         dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
     e2e_ms = float(e2e_ms.item())
 
+    # router logits (the step upstream of the layer's given logits), timed on its own
+    wr = torch.empty(wl.E, wl.H, dtype=torch.int16, device=dev)
+    synth.dev_weight(wl.seed, synth.ROUTER_STREAM, wr, sigma=1.0 / math.sqrt(wl.H))
+    wr = wr.view(torch.bfloat16)
+    rlog = torch.empty(T, wl.E, dtype=torch.float32, device=dev)
+    for i in range(3):
+        moe.moe_router_logits(batches[i % N_BATCHES][0], wr, rlog)
+    r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    r0.record(stream)
+    for i in range(args.steps):
+        moe.moe_router_logits(batches[i % N_BATCHES][0], wr, rlog)
+    r1.record(stream)
+    torch.cuda.synchronize()
+    r_ms = r0.elapsed_time(r1) / args.steps
+
     tokens = world * T * args.steps
     value = tokens / (total_ms / 1e3)
     hbm, bf16, peak_kind = peaks()
@@ -347,6 +380,7 @@ def run_ours(args):
         "roofline": roofline,
         "stages_ms": {s: round(v, 4) for s, v in stage_ms.items()},
         "gpu_launches": launches,
+        "router": router_line(wl, T, r_ms, hbm, bf16, peak_kind),
         "e2e": {"value": round(tokens / (e2e_ms / 1e3), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * wl.H * 2 + T * wl.E * 4,
                 "d2h_bytes_per_step": T * wl.H * 2},

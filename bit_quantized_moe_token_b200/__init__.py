@@ -5,6 +5,7 @@ The work happens in ``libmoe_w4a8.so`` (hand-written CUDA, C ABI in
 """
 from ._binding import (MOE_OK, Layer, MoeError, fp8_quant_tokens, layer_struct, lib,
                        moe_last_device_status, moe_route_topk, moe_route_workspace_bytes,
+                       moe_router_logits,
                        moe_status_string, moe_w4a8_forward, moe_w4a8_forward_profiled,
                        moe_w4a8_workspace_bytes, STAGES, N_STAGE_EVENTS,
                        moe_w4a8_workspace_layout, w4a8_pack_weights,
@@ -13,6 +14,7 @@ from .layer import alloc_workspace, forward, make_layer, pack_expert_weights
 
 __all__ = ["MOE_OK", "Layer", "MoeError", "fp8_quant_tokens", "layer_struct", "lib",
            "moe_last_device_status", "moe_route_topk", "moe_route_workspace_bytes",
+           "moe_router_logits",
            "moe_status_string", "moe_w4a8_forward", "moe_w4a8_forward_profiled", "STAGES",
            "N_STAGE_EVENTS", "moe_w4a8_workspace_bytes",
            "moe_w4a8_workspace_layout", "w4a8_pack_weights", "alloc_workspace", "forward",

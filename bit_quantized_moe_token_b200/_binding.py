@@ -64,6 +64,7 @@ def lib() -> ctypes.CDLL:
         L.moe_route_workspace_bytes.argtypes = [i64, i32, i32]
         L.moe_route_workspace_bytes.restype = sz
         L.moe_route_topk.argtypes = [vp, i64, i32, i32, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.moe_router_logits.argtypes = [vp, vp, i64, i32, i32, vp, vp]
         L.moe_w4a8_workspace_bytes.argtypes = [ctypes.POINTER(_CLayer), i64, i32]
         L.moe_w4a8_workspace_bytes.restype = sz
         L.moe_w4a8_workspace_layout.argtypes = [ctypes.POINTER(_CLayer), i64, i32,
@@ -75,7 +76,7 @@ def lib() -> ctypes.CDLL:
         L.moe_selftest_bounded_wait.argtypes = [i64, vp]
         L.moe_status_string.argtypes = [i32]
         L.moe_status_string.restype = ctypes.c_char_p
-        for f in (L.w4a8_pack_weights, L.fp8_quant_tokens, L.moe_route_topk,
+        for f in (L.w4a8_pack_weights, L.fp8_quant_tokens, L.moe_route_topk, L.moe_router_logits,
                   L.moe_w4a8_workspace_layout, L.moe_w4a8_forward, L.moe_w4a8_forward_profiled,
                   L.moe_last_device_status, L.moe_selftest_bounded_wait):
             f.restype = i32
@@ -131,6 +132,14 @@ def fp8_quant_tokens(x, q, scale, stream=None) -> None:
     T, H = x.shape
     _check(lib().fp8_quant_tokens(_ptr(x), T, H, _ptr(q), _ptr(scale), _stream(stream)),
            "fp8_quant_tokens")
+
+
+def moe_router_logits(x, wr, logits, stream=None) -> None:
+    """x bf16 [T, H], router weight wr bf16 [E, H] -> logits fp32 [T, E]."""
+    T, H = x.shape
+    E = wr.shape[0]
+    _check(lib().moe_router_logits(_ptr(x), _ptr(wr), T, H, E, _ptr(logits), _stream(stream)),
+           "moe_router_logits")
 
 
 def moe_route_workspace_bytes(T: int, E: int, k: int) -> int:

@@ -16,6 +16,7 @@ __device__ int g_device_status = 0;
 #include "quant.cuh"
 #include "route.cuh"
 #include "forward.cuh"
+#include "router.cuh"
 #include "tc_ptx.cuh"
 
 namespace moe {

@@ -86,6 +86,24 @@ int fp8_quant_tokens(const uint16_t* x_bf16, int64_t T, int64_t H, uint8_t* q_e4
                      float* scale, moe_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------
+ * Router logits: the step upstream of S2.
+ *
+ * logits[t][e] = sum over k of x[t][k] * wr[e][k], with the router weight kept in its source
+ * bf16 precision (the "Inkling-Small-Mixed-Quant-GGUF" card, "Precision differences": router
+ * tensors stay native; the "Inkling-512k-NVFP4-AQLM-hybrid" card, "Layout summary": the gate
+ * is copied verbatim).  Products of two bf16 values are exact in fp32; the sum is fp32 in an
+ * order of the kernel's choosing (so not bit-identical to a sequential sum); no bias.
+ *
+ *   x_bf16   [T, H] bf16, 16-byte aligned;  H a positive multiple of 8, at most 16384
+ *   wr_bf16  [E, H] bf16, 16-byte aligned;  E in [1, 1024]
+ *   logits   [T, E] fp32 output, 4-byte aligned (feeds moe_route_topk / moe_w4a8_forward)
+ * T == 0 is a no-op.  Small T runs on the CUDA cores (each weight row read once); T >= 256
+ * with E a multiple of 128 and H of 64 runs on the tensor cores.
+ * --------------------------------------------------------------------------------------- */
+int moe_router_logits(const uint16_t* x_bf16, const uint16_t* wr_bf16, int64_t T, int H, int E,
+                      float* logits, moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------
  * S2 + S3. Top-k routing and the stable token permutation.
  *
  * Top-k of each row of the router logits (the Inkling-512k card's opening paragraph: 256

@@ -256,6 +256,17 @@ def shared_weight(wl: Workload, s: int, proj: str) -> np.ndarray:
     return out
 
 
+ROUTER_STREAM = 2_000_000
+
+
+def router_weight(wl: Workload) -> np.ndarray:
+    """bf16 router weight [E, H] ~ N(0, 1/sqrt(H)): with N(0,1) tokens the logits are ~N(0,1),
+    the spread the workloads' given logits have."""
+    out = np.zeros((wl.E, wl.H), np.uint16)
+    host_lib().syn_fill_normal_bf16(wl.seed, ROUTER_STREAM, 0, out.size, 1.0 / np.sqrt(wl.H), _p(out))
+    return out
+
+
 def normal_f32(seed: int, stream: int, n: int, sigma: float = 1.0, start: int = 0) -> np.ndarray:
     out = np.zeros(n, np.float32)
     host_lib().syn_fill_normal_f32(seed, stream, start, n, sigma, _p(out))

@@ -27,6 +27,7 @@ def _declared_functions():
 def test_header_declares_the_boundary():
     names = _declared_functions()
     for n in ("w4a8_pack_weights", "fp8_quant_tokens", "moe_route_topk", "moe_w4a8_forward",
+              "moe_router_logits",
               "moe_w4a8_workspace_bytes", "moe_last_device_status", "moe_status_string"):
         assert n in names
 
@@ -87,6 +88,18 @@ def test_route_rejects_bad_args():
     assert L.moe_route_topk(p, 64, 256, 6, p, p, p, p, p, None, ws, None) == -4
     assert L.moe_route_topk(p, 64, 256, 6, p, p, p, p, p, ctypes.c_void_p(4096 + 16), ws, None) == -3
     assert L.moe_route_topk(None, 64, 256, 6, p, p, p, p, p, p, ws, None) == -1
+
+
+def test_router_rejects_bad_args():
+    L = _L()
+    p = ctypes.c_void_p(4096)
+    assert L.moe_router_logits(p, p, 4, 100, 8, p, None) == -2          # H % 8
+    assert L.moe_router_logits(p, p, 4, 256, 2000, p, None) == -2       # E > 1024
+    assert L.moe_router_logits(p, p, 4, 32768, 8, p, None) == -2        # H > 16384
+    assert L.moe_router_logits(p, p, -1, 256, 8, p, None) == -1
+    assert L.moe_router_logits(None, p, 4, 256, 8, p, None) == -1
+    assert L.moe_router_logits(ctypes.c_void_p(4104), p, 4, 256, 8, p, None) == -3
+    assert L.moe_router_logits(p, p, 0, 256, 8, p, None) == 0            # no-op
 
 
 def test_forward_workspace_and_layout():

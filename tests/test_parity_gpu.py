@@ -255,6 +255,43 @@ def test_forward_zero_tokens_and_zero_rows():
     moe.moe_w4a8_forward(dl, xd, ld, 2, out, torch.empty(256, dtype=torch.uint8, device="cuda"))
 
 
+# ---- router logits (the step upstream of top-k) ---------------------------------------------------
+
+@pytest.mark.parametrize("T,E,H", [(1, 256, 4096), (8, 256, 4096), (37, 20, 1000), (300, 256, 1024),
+                                   (2048, 256, 4096)])
+def test_router_logits_vs_oracle(T, E, H):
+    """CUDA-core path for small T, tensor-core path for T >= 256: logits within the fp32
+    summation bound of the oracle's, top-k selection equal wherever the oracle's margin at the
+    k-th place exceeds that bound."""
+    x = synth.normal_bf16(6, 990 + T, T * H).reshape(T, H)
+    wr = synth.normal_bf16(6, 991 + E, E * H, 1.0 / np.sqrt(H)).reshape(E, H)
+    ref = oracle.router_logits(x, wr).astype(np.float64)
+    got = torch.empty(T, E, dtype=torch.float32, device="cuda")
+    moe.moe_router_logits(to_dev_bf16(x), to_dev_bf16(wr), got)
+    torch.cuda.synchronize()
+    g = got.cpu().numpy().astype(np.float64)
+    xa = np.abs(bf16_to_f32(x).astype(np.float64))
+    wa = np.abs(bf16_to_f32(wr).astype(np.float64))
+    bound = 2 * H * 2.0 ** -24 * (xa @ wa.T) + 1e-30     # both sums within H*2^-24*sum|xw| of exact
+    assert np.all(np.abs(g - ref) <= bound)
+    # the selection is unique wherever the oracle's gap at the k-th place exceeds twice the
+    # largest logit difference seen; there the ids must agree
+    k = min(6, E)
+    ids_ref, _ = oracle.route_topk(ref.astype(np.float32), k)
+    ids_got, _ = oracle.route_topk(g.astype(np.float32), k)
+    srt = -np.sort(-ref, axis=1)
+    margin = srt[:, k - 1] - (srt[:, k] if k < E else -np.inf)
+    clear = margin > 2 * np.abs(g - ref).max() + 1e-12
+    assert clear.sum() >= 0.8 * T
+    assert np.array_equal(ids_got[clear], ids_ref[clear])
+
+
+def test_router_logits_zero_tokens():
+    wr = torch.zeros(8, 64, dtype=torch.bfloat16, device="cuda")
+    moe.moe_router_logits(torch.empty(0, 64, dtype=torch.bfloat16, device="cuda"), wr,
+                          torch.empty(0, 8, dtype=torch.float32, device="cuda"))
+
+
 # ---- the layer at full size: sampled tokens -----------------------------------------------------
 
 FULL = ["decode_t8", "decode_t64", "prefill_t2048_zipf", "prefill_t16384_shared"]
