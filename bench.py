@@ -188,6 +188,27 @@ class ClockSampler:
                 "samples": len(sm), "window_s": round(self.t1 - self.t0, 4)}
 
 
+def replica_token_offset(rank, batch, T):
+    """First token of batch `batch` on replica `rank`: the ranks draw disjoint stretches of the
+    workload's token stream (weak scaling: every rank does a full batch per step)."""
+    return (rank * N_BATCHES + batch) * T
+
+
+def max_over_ranks(ms, device, world):
+    """The slowest rank's device time (a single rank returns its own)."""
+    import torch
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(world, T, steps, ms):
+    """Tokens per second of all ranks together over `steps` steps of the slowest rank's `ms`."""
+    return world * T * steps / (ms / 1e3)
+
+
 def dist_setup():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -219,7 +240,7 @@ def run_ours(args):
     T, k = wl.T, wl.k
     batches = []
     for b in range(N_BATCHES):
-        t0 = (rank * N_BATCHES + b) * T
+        t0 = replica_token_offset(rank, b, T)
         batches.append(device_inputs(wl, device=dev, t0=t0, T=T))
     out = torch.empty(T, wl.H, dtype=torch.bfloat16, device=dev)
     ws = moe.alloc_workspace(layer, T, k, dev)
@@ -289,10 +310,7 @@ def run_ours(args):
     if moe.moe_last_device_status() != 0:
         raise RuntimeError("device status: timeout in the timed region")
     dom_ms = sum(ev[i][DOM_A].elapsed_time(ev[i][DOM_B]) for i in range(args.steps)) / args.steps
-    t_max = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
-    total_ms = float(t_max.item())
+    total_ms = max_over_ranks(total_ms, dev, world)
 
     # ---- end to end through the public API with host buffers ----
     hx = [b[0].cpu().pin_memory() for b in batches]
@@ -318,10 +336,7 @@ def run_ours(args):
         hout.copy_(out, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
-    e2e_ms = float(e2e_ms.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev, world)
 
     # router logits (the step upstream of the layer's given logits), timed on its own
     wr = torch.empty(wl.E, wl.H, dtype=torch.int16, device=dev)
@@ -337,10 +352,10 @@ def run_ours(args):
         moe.moe_router_logits(batches[i % N_BATCHES][0], wr, rlog)
     r1.record(stream)
     torch.cuda.synchronize()
-    r_ms = r0.elapsed_time(r1) / args.steps
+    r_ms = max_over_ranks(r0.elapsed_time(r1), dev, world) / args.steps
 
     tokens = world * T * args.steps
-    value = tokens / (total_ms / 1e3)
+    value = whole_job_rate(world, T, args.steps, total_ms)
     hbm, bf16, peak_kind = peaks()
     gu_bytes, down_bytes = expert_bytes(wl)
     mean_touched = sum(touched[i % N_BATCHES] for i in range(args.steps)) / args.steps
