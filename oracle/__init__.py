@@ -41,7 +41,15 @@ class _Layer(ctypes.Structure):
                 ("down_scales", ctypes.c_void_p),
                 ("n_shared", ctypes.c_int), ("shared_N", ctypes.c_int),
                 ("sh_gate", ctypes.c_void_p), ("sh_up", ctypes.c_void_p),
-                ("sh_down", ctypes.c_void_p)]
+                ("sh_down", ctypes.c_void_p),
+                ("fmt", ctypes.c_int),
+                ("gate_w8", ctypes.c_void_p), ("up_w8", ctypes.c_void_p),
+                ("down_w8", ctypes.c_void_p),
+                ("gate_rs", ctypes.c_void_p), ("up_rs", ctypes.c_void_p),
+                ("down_rs", ctypes.c_void_p)]
+
+FMT_W4A8 = 0
+FMT_W8A8 = 1
 
 
 _lib = None
@@ -67,6 +75,8 @@ def lib():
         L.or_unpack.restype = None
         L.or_quant_tokens.argtypes = [vp, i64, i64, vp, vp]
         L.or_quant_tokens.restype = None
+        L.or_quant_rows.argtypes = [vp, i64, i64, vp, vp]
+        L.or_quant_rows.restype = None
         L.or_route_topk.argtypes = [vp, i64, i32, i32, vp, vp]
         L.or_router_logits.argtypes = [vp, vp, i64, i64, i32, vp]
         L.or_route_topk.restype = None
@@ -138,6 +148,16 @@ def quant_tokens(x_bf16: np.ndarray):
     return q, s
 
 
+def quant_rows(w_bf16: np.ndarray):
+    """Row-scaled FP8 weights: bf16 bits [rows, K] -> (E4M3 codes [rows, K], fp32 scale [rows])."""
+    w = np.ascontiguousarray(w_bf16, np.uint16)
+    rows, K = w.shape
+    q = np.zeros((rows, K), np.uint8)
+    s = np.zeros(rows, np.float32)
+    lib().or_quant_rows(_p(w), rows, K, _p(q), _p(s))
+    return q, s
+
+
 def router_logits(x_bf16: np.ndarray, wr_bf16: np.ndarray) -> np.ndarray:
     """[T, E] fp32 logits of bf16 tokens [T, H] against the bf16 router weight [E, H]."""
     x = np.ascontiguousarray(x_bf16, np.uint16)
@@ -173,29 +193,54 @@ def permute(ids: np.ndarray, E: int):
 # ---- the layer ------------------------------------------------------------------------------
 
 class Layer:
-    """Host copy of one layer's packed weights (numpy), laid out like the C ABI's layer."""
+    """Host copy of one layer's packed weights (numpy), laid out like the C ABI's layer.
+
+    The default format is W4A8 (packed INT4 + bf16 group scales); ``Layer.w8a8`` builds the
+    row-scaled FP8 format (E4M3 codes + one fp32 scale per output row)."""
 
     def __init__(self, E, H, N, gate_packed, up_packed, down_packed, gate_scales, up_scales,
                  down_scales, group=128, sh_gate=None, sh_up=None, sh_down=None):
         self.E, self.H, self.N, self.group = E, H, N, group
-        self.gate_packed = np.ascontiguousarray(gate_packed, np.int32)
-        self.up_packed = np.ascontiguousarray(up_packed, np.int32)
-        self.down_packed = np.ascontiguousarray(down_packed, np.int32)
-        self.gate_scales = np.ascontiguousarray(gate_scales, np.uint16)
-        self.up_scales = np.ascontiguousarray(up_scales, np.uint16)
-        self.down_scales = np.ascontiguousarray(down_scales, np.uint16)
+        self.fmt = FMT_W4A8
+        self.gate_packed = None if gate_packed is None else np.ascontiguousarray(gate_packed, np.int32)
+        self.up_packed = None if up_packed is None else np.ascontiguousarray(up_packed, np.int32)
+        self.down_packed = None if down_packed is None else np.ascontiguousarray(down_packed, np.int32)
+        self.gate_scales = None if gate_scales is None else np.ascontiguousarray(gate_scales, np.uint16)
+        self.up_scales = None if up_scales is None else np.ascontiguousarray(up_scales, np.uint16)
+        self.down_scales = None if down_scales is None else np.ascontiguousarray(down_scales, np.uint16)
+        self.gate_w8 = self.up_w8 = self.down_w8 = None
+        self.gate_rs = self.up_rs = self.down_rs = None
         self.sh_gate = None if sh_gate is None else np.ascontiguousarray(sh_gate, np.uint16)
         self.sh_up = None if sh_up is None else np.ascontiguousarray(sh_up, np.uint16)
         self.sh_down = None if sh_down is None else np.ascontiguousarray(sh_down, np.uint16)
         self.n_shared = 0 if sh_gate is None else sh_gate.shape[0]
         self.shared_N = 0 if sh_gate is None else sh_gate.shape[1]
 
+    @classmethod
+    def w8a8(cls, E, H, N, gate_w8, up_w8, down_w8, gate_rs, up_rs, down_rs, group=128,
+             sh_gate=None, sh_up=None, sh_down=None):
+        """Row-scaled FP8 layer: codes [E,N,H], [E,N,H], [E,H,N]; scales [E,N], [E,N], [E,H]."""
+        L = cls(E, H, N, None, None, None, None, None, None, group=group, sh_gate=sh_gate,
+                sh_up=sh_up, sh_down=sh_down)
+        L.fmt = FMT_W8A8
+        L.gate_w8 = np.ascontiguousarray(gate_w8, np.uint8)
+        L.up_w8 = np.ascontiguousarray(up_w8, np.uint8)
+        L.down_w8 = np.ascontiguousarray(down_w8, np.uint8)
+        L.gate_rs = np.ascontiguousarray(gate_rs, np.float32)
+        L.up_rs = np.ascontiguousarray(up_rs, np.float32)
+        L.down_rs = np.ascontiguousarray(down_rs, np.float32)
+        assert L.gate_w8.shape == (E, N, H) and L.down_w8.shape == (E, H, N)
+        assert L.gate_rs.shape == (E, N) and L.down_rs.shape == (E, H)
+        return L
+
     def _c(self):
         return _Layer(self.E, self.H, self.N, self.group,
                       _p(self.gate_packed), _p(self.up_packed), _p(self.down_packed),
                       _p(self.gate_scales), _p(self.up_scales), _p(self.down_scales),
                       self.n_shared, self.shared_N,
-                      _p(self.sh_gate), _p(self.sh_up), _p(self.sh_down))
+                      _p(self.sh_gate), _p(self.sh_up), _p(self.sh_down),
+                      self.fmt, _p(self.gate_w8), _p(self.up_w8), _p(self.down_w8),
+                      _p(self.gate_rs), _p(self.up_rs), _p(self.down_rs))
 
 
 def moe_forward(layer: Layer, x_bf16: np.ndarray, logits: np.ndarray, k: int):
@@ -261,3 +306,26 @@ def pack_workload_layer(wl, experts=None, with_shared=True):
                   sh_up=np.stack([synth.shared_weight(wl, s, "up") for s in range(wl.n_shared)]),
                   sh_down=np.stack([synth.shared_weight(wl, s, "down") for s in range(wl.n_shared)]))
     return Layer(E, H, N, gp, up, dp, gs, us, ds, group=g, **sh)
+
+
+def quant_workload_layer_w8a8(wl, experts=None, with_shared=True):
+    """Row-quantize (oracle side) the seeded weights of workload `wl` to the row-scaled FP8
+    format; experts outside `experts` stay zero, as in ``pack_workload_layer``."""
+    import synth
+    E, H, N = wl.E, wl.H, wl.N
+    gq = np.zeros((E, N, H), np.uint8)
+    uq = np.zeros((E, N, H), np.uint8)
+    dq = np.zeros((E, H, N), np.uint8)
+    gs = np.zeros((E, N), np.float32)
+    us = np.zeros((E, N), np.float32)
+    ds = np.zeros((E, H), np.float32)
+    for e in (range(E) if experts is None else experts):
+        gq[e], gs[e] = quant_rows(synth.expert_weight(wl, e, "gate"))
+        uq[e], us[e] = quant_rows(synth.expert_weight(wl, e, "up"))
+        dq[e], ds[e] = quant_rows(synth.expert_weight(wl, e, "down"))
+    sh = {}
+    if with_shared and wl.n_shared:
+        sh = dict(sh_gate=np.stack([synth.shared_weight(wl, s, "gate") for s in range(wl.n_shared)]),
+                  sh_up=np.stack([synth.shared_weight(wl, s, "up") for s in range(wl.n_shared)]),
+                  sh_down=np.stack([synth.shared_weight(wl, s, "down") for s in range(wl.n_shared)]))
+    return Layer.w8a8(E, H, N, gq, uq, dq, gs, us, ds, group=wl.group, **sh)

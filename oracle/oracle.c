@@ -24,6 +24,9 @@
  *       little-endian I32, first code in the least significant nibble.
  *  [P2] "Inkling-512k-NVFP4-AQLM-hybrid" model card: 256 routed experts, 6
  *       active; "On-disk tensor format" — w13 = fused gate|up, w2 = down.
+ *  [P5] "Inkling 2 Small FP8 for AMD MI300X", "Precision and files": expert
+ *       projections in FP8 with one fp32 scale per expert output channel,
+ *       scale = max|row| / (largest FP8 value), per-token FP8 activations.
  *  Readings where the pages are silent (listed with each function):
  *   R1 symmetric RTN scale = amax/7 stored as BF16 (round to nearest even),
  *      codes = clamp(rint(w/scale), -8, 7), all-zero group -> scale 0, codes 0;
@@ -37,7 +40,11 @@
  *      outputs in selection order, adds the shared experts, rounds once to
  *      bf16;
  *   R6 router logits = x . wr over the bf16 router weight, no bias, fp32
- *      accumulation in increasing k.
+ *      accumulation in increasing k;
+ *   R7 row-scaled FP8 experts ([P5]) use the OCP E4M3FN format of R2, so the
+ *      row scale is amax/448 (the page's 240 is the largest E4M3FNUZ value),
+ *      codes = E4M3(w/scale) exactly as R2 does for a token row; a projection
+ *      output is (sum_k dec(q_k) dec(w_k), k increasing) * s_w[n] * s_x.
  */
 #include <math.h>
 #include <stdint.h>
@@ -192,6 +199,11 @@ void or_quant_tokens(const uint16_t* x, int64_t T, int64_t H, uint8_t* q, float*
     }
 }
 
+/* Row-scaled FP8 weights ([P5], reading R7): one scale per row, same rule as a token row. */
+void or_quant_rows(const uint16_t* w, int64_t rows, int64_t K, uint8_t* q, float* s) {
+    or_quant_tokens(w, rows, K, q, s);
+}
+
 /* ------------------------------------------------------------------------------------------ */
 /* Router (the step upstream of S2): logits[t][e] = sum over k of x[t][k] * wr[e][k] with the  */
 /* router weight kept in its source bf16 precision ("Baekpica/Inkling-Small-Mixed-Quant-GGUF"  */
@@ -272,6 +284,10 @@ typedef struct {
     const uint16_t *gate_scales, *up_scales, *down_scales;  /* bf16 [E,N,H/g], [E,N,H/g], [E,H,N/g] */
     int n_shared, shared_N;
     const uint16_t *sh_gate, *sh_up, *sh_down;              /* bf16 [S,Ns,H], [S,Ns,H], [S,H,Ns] */
+    /* fmt 1 = row-scaled FP8 experts (reading R7): E4M3 codes and one fp32 scale per output row */
+    int fmt;
+    const uint8_t *gate_w8, *up_w8, *down_w8;               /* [E,N,H], [E,N,H], [E,H,N] */
+    const float *gate_rs, *up_rs, *down_rs;                  /* [E,N], [E,N], [E,H] */
 } or_layer;
 
 /* Unpacked codes of one projection as floats, transposed to [K][rows] so that the
@@ -305,6 +321,25 @@ static void w4a8_proj(const uint8_t* q, float s_x, const float* cT, const uint16
     for (int64_t n = 0; n < rows; ++n) out[n] = acc[n] * s_x;
 }
 
+/* Decoded E4M3 codes of one projection, transposed to [K][rows]. */
+static void w8_T(const uint8_t* codes, int64_t rows, int64_t K, float* cT) {
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t kk = 0; kk < K; ++kk) cT[kk * rows + r] = or_e4m3_decode(codes[r * K + kk]);
+}
+
+/* Row-scaled FP8 projection of one FP8 row (reading R7): for every output n,
+ *   acc_n = sum_k dec(q_k) * dec(w[n,k])  (k increasing),   out_n = acc_n * s_w[n] * s_x. */
+static void w8a8_proj(const uint8_t* q, float s_x, const float* cT, const float* rs, int64_t rows,
+                      int64_t K, float* out, float* acc) {
+    for (int64_t n = 0; n < rows; ++n) acc[n] = 0.0f;
+    for (int64_t kk = 0; kk < K; ++kk) {
+        float a = or_e4m3_decode(q[kk]);
+        const float* c = cT + kk * rows;
+        for (int64_t n = 0; n < rows; ++n) acc[n] += a * c[n];
+    }
+    for (int64_t n = 0; n < rows; ++n) out[n] = acc[n] * rs[n] * s_x;
+}
+
 static float silu_f32(float g) { return g * (1.0f / (1.0f + expf(-g))); }
 
 /*
@@ -325,6 +360,21 @@ static void expert_row(const uint8_t* q, float s_x, const float* cg, const float
     for (int64_t n = 0; n < N; ++n) h[n] = silu_f32(G[n]) * U[n];
     quant_row_f32(h, N, hq, s_h);
     w4a8_proj(hq, *s_h, cd, sd, H, N, group, y, part, acc);
+}
+
+/* expert_row for row-scaled FP8 experts (same steps, w8a8_proj for the three projections). */
+static void expert_row_w8(const uint8_t* q, float s_x, const float* cg, const float* cu,
+                          const float* cd, const float* rg, const float* ru, const float* rd,
+                          int64_t H, int64_t N, uint8_t* hq, float* s_h, float* y, float* scratch) {
+    float* G = scratch;
+    float* U = G + N;
+    float* h = U + N;
+    float* acc = h + N;
+    w8a8_proj(q, s_x, cg, rg, N, H, G, acc);
+    w8a8_proj(q, s_x, cu, ru, N, H, U, acc);
+    for (int64_t n = 0; n < N; ++n) h[n] = silu_f32(G[n]) * U[n];
+    quant_row_f32(h, N, hq, s_h);
+    w8a8_proj(hq, *s_h, cd, rd, H, N, y, acc);
 }
 
 /* Shared expert in bf16 weights / fp32 arithmetic on the unquantized token row:
@@ -389,14 +439,25 @@ int or_moe_forward(const or_layer* L, const uint16_t* x, const float* logits, in
         float* cu = (float*)malloc((size_t)N * H * 4);
         float* cd = (float*)malloc((size_t)H * N * 4);
         float* scratch = (float*)malloc((size_t)(3 * N + 2 * (H > N ? H : N)) * 4);
-        codes_T(L->gate_packed + e * N * (H / 8), N, H, cg);
-        codes_T(L->up_packed + e * N * (H / 8), N, H, cu);
-        codes_T(L->down_packed + e * H * (N / 8), H, N, cd);
+        if (L->fmt == 1) {
+            w8_T(L->gate_w8 + e * N * H, N, H, cg);
+            w8_T(L->up_w8 + e * N * H, N, H, cu);
+            w8_T(L->down_w8 + e * H * N, H, N, cd);
+        } else {
+            codes_T(L->gate_packed + e * N * (H / 8), N, H, cg);
+            codes_T(L->up_packed + e * N * (H / 8), N, H, cu);
+            codes_T(L->down_packed + e * H * (N / 8), H, N, cd);
+        }
         for (int32_t r = r0; r < r1; ++r) {
             int64_t t = sorted[r] / k;
-            expert_row(xq + t * H, sx[t], cg, cu, cd, L->gate_scales + e * N * G_h,
-                       L->up_scales + e * N * G_h, L->down_scales + e * H * G_n, H, N, group,
-                       hq + (int64_t)r * N, sh + r, y + (int64_t)r * H, scratch);
+            if (L->fmt == 1)
+                expert_row_w8(xq + t * H, sx[t], cg, cu, cd, L->gate_rs + e * N, L->up_rs + e * N,
+                              L->down_rs + e * H, H, N, hq + (int64_t)r * N, sh + r,
+                              y + (int64_t)r * H, scratch);
+            else
+                expert_row(xq + t * H, sx[t], cg, cu, cd, L->gate_scales + e * N * G_h,
+                           L->up_scales + e * N * G_h, L->down_scales + e * H * G_n, H, N, group,
+                           hq + (int64_t)r * N, sh + r, y + (int64_t)r * H, scratch);
         }
         free(cg); free(cu); free(cd); free(scratch);
     }
@@ -474,14 +535,26 @@ int or_moe_forward_dense(const or_layer* L, const uint16_t* x, const float* logi
     float* cd = (float*)malloc((size_t)H * N * 4);
     float* scratch = (float*)malloc((size_t)(3 * N + 2 * (H > N ? H : N)) * 4);
     for (int64_t e = 0; e < E; ++e) {
-        codes_T(L->gate_packed + e * N * (H / 8), N, H, cg);
-        codes_T(L->up_packed + e * N * (H / 8), N, H, cu);
-        codes_T(L->down_packed + e * H * (N / 8), H, N, cd);
-        for (int64_t t = 0; t < T; ++t)
-            expert_row(xq + t * H, sx[t], cg, cu, cd, L->gate_scales + e * N * G_h,
-                       L->up_scales + e * N * G_h, L->down_scales + e * H * G_n, H, N, group,
-                       hq_dense + (t * E + e) * N, sh_dense + t * E + e, y_dense + (t * E + e) * H,
-                       scratch);
+        if (L->fmt == 1) {
+            w8_T(L->gate_w8 + e * N * H, N, H, cg);
+            w8_T(L->up_w8 + e * N * H, N, H, cu);
+            w8_T(L->down_w8 + e * H * N, H, N, cd);
+        } else {
+            codes_T(L->gate_packed + e * N * (H / 8), N, H, cg);
+            codes_T(L->up_packed + e * N * (H / 8), N, H, cu);
+            codes_T(L->down_packed + e * H * (N / 8), H, N, cd);
+        }
+        for (int64_t t = 0; t < T; ++t) {
+            if (L->fmt == 1)
+                expert_row_w8(xq + t * H, sx[t], cg, cu, cd, L->gate_rs + e * N, L->up_rs + e * N,
+                              L->down_rs + e * H, H, N, hq_dense + (t * E + e) * N,
+                              sh_dense + t * E + e, y_dense + (t * E + e) * H, scratch);
+            else
+                expert_row(xq + t * H, sx[t], cg, cu, cd, L->gate_scales + e * N * G_h,
+                           L->up_scales + e * N * G_h, L->down_scales + e * H * G_n, H, N, group,
+                           hq_dense + (t * E + e) * N, sh_dense + t * E + e,
+                           y_dense + (t * E + e) * H, scratch);
+        }
     }
     float* dense_gate = (float*)malloc((size_t)E * 4);
     for (int64_t t = 0; t < T; ++t) {

@@ -418,6 +418,133 @@ def test_layer_empty_batch():
 
 
 # ------------------------------------------------------------------------------------------------
+# row-scaled FP8 (W8A8) experts
+# ------------------------------------------------------------------------------------------------
+
+def test_row_quant_closed_form():
+    w = np.zeros((4, 128), np.float32)
+    w[0, :] = 0.02734375          # 7 * 2^-8: scale = 2^-14 exactly, every code E4M3(448) = 0x7e
+    w[1, 0] = -1.0                # scale = fp32(1/448); -448 -> 0xfe
+    w[1, 1] = 0.25                # 112 = 1.75 * 2^6 -> 0x6e
+    w[3, 5] = 0.875               # scale 2^-9; the other entries 0 -> code 0
+    q, s = oracle.quant_rows(_f32_to_bf16_bits(w))
+    assert s[0] == 2.0 ** -14 and np.all(q[0] == 0x7E)
+    assert s[1] == np.float32(1.0) / np.float32(448.0)
+    assert list(q[1, :3]) == [0xFE, 0x6E, 0x00]
+    assert s[2] == 0.0 and not q[2].any()
+    assert s[3] == 2.0 ** -9 and q[3, 5] == 0x7E and int(q[3].astype(np.int64).sum()) == 0x7E
+
+
+def _w8_layer_from_f32(Wg, Wu, Wd):
+    """Row-quantize fp32 expert weights [E,N,H],[E,N,H],[E,H,N] (rounded to bf16 first)."""
+    E, N, H = Wg.shape
+    def rq(W):
+        qs = [oracle.quant_rows(_f32_to_bf16_bits(W[e])) for e in range(E)]
+        return np.stack([a for a, _ in qs]), np.stack([b for _, b in qs])
+    (gq, gs), (uq, us), (dq, ds) = rq(Wg), rq(Wu), rq(Wd)
+    return oracle.Layer.w8a8(E, H, N, gq, uq, dq, gs, us, ds), (gq, gs, uq, us, dq, ds)
+
+
+def test_w8a8_constant_closed_form():
+    want = {}
+    for line in golden_lines("constant_layer.txt"):
+        t, o, hq = line.split()
+        want[int(t)] = (float(o), int(hq, 16))
+    T, H, N, E, k = 4, 128, 128, 2, 1
+    w0 = 0.02734375
+    sgn = np.array([1.0, -1.0], np.float32)[:, None, None]
+    Wg = np.broadcast_to(sgn * w0, (E, N, H)).astype(np.float32)
+    Wd = np.broadcast_to(sgn * w0, (E, H, N)).astype(np.float32)
+    layer, (gq, gs, _, _, dq, ds) = _w8_layer_from_f32(Wg, Wg, Wd)
+    assert np.all(gs == 2.0 ** -14) and np.all(ds == 2.0 ** -14)
+    assert np.all(gq[0] == 0x7E) and np.all(gq[1] == 0xFE)
+    x = _f32_to_bf16_bits(np.full((T, H), 0.875, np.float32))
+    lg = np.array([[1, 0], [0, 1], [1, 0], [0, 1]], np.float32)
+    r = oracle.moe_forward(layer, x, lg, k)
+    out = oracle.bf16_to_f32(r["out"])
+    sig = lambda v: 1.0 / (1.0 + math.exp(-v))
+    for t in range(T):
+        assert np.all(out[t] == want[t][0]), (t, out[t, :4])
+        assert np.all(r["hq"][r["row_of_pair"][t]] == want[t][1])
+        s = 1.0 if t % 2 == 0 else -1.0
+        assert np.allclose(r["out_f32"][t], s * 3.5 * 9.37890625 * sig(s * 3.0625), rtol=1e-6)
+
+
+def test_w8a8_down_projection_within_fp32_bound():
+    """y[r, m] = (sum_n dec(hq[r,n]) dec(wd[e,m,n])) * s_wd[e,m] * s_h[r], checked row by row
+    against an fp64 sum of the same codes within the sequential-fp32 error bound.  Rows of the
+    weights are scaled over 2^-3..2^3 so that a scale applied per column, or a transposed
+    weight, is far outside the bound."""
+    rng = np.random.default_rng(11)
+    T, H, N, E, k = 12, 256, 128, 4, 2
+    rs_g = 2.0 ** rng.uniform(-3, 3, (E, N, 1))
+    rs_d = 2.0 ** rng.uniform(-3, 3, (E, H, 1))
+    Wg = (rng.standard_normal((E, N, H)) * 0.02 * rs_g).astype(np.float32)
+    Wu = (rng.standard_normal((E, N, H)) * 0.02 * rs_g[:, ::-1]).astype(np.float32)
+    Wd = (rng.standard_normal((E, H, N)) * 0.02 * rs_d).astype(np.float32)
+    layer, (_, _, _, _, dq, ds) = _w8_layer_from_f32(Wg, Wu, Wd)
+    x = _f32_to_bf16_bits(rng.standard_normal((T, H)).astype(np.float32))
+    lg = rng.standard_normal((T, E)).astype(np.float32)
+    r = oracle.moe_forward(layer, x, lg, k)
+    dec = oracle.e4m3_decode_table().astype(np.float64)
+    for e in range(E):
+        for row in range(r["offsets"][e], r["offsets"][e + 1]):
+            terms = dec[r["hq"][row]][None, :] * dec[dq[e]]          # [H, N]
+            exact = terms.sum(axis=1)
+            bound = N * 2.0 ** -24 * np.abs(terms).sum(axis=1)
+            acc = r["y"][row].astype(np.float64) / (ds[e].astype(np.float64) * r["s_h"][row])
+            # the two final fp32 multiplies add at most 2 ulp of the result each
+            slack = 4 * 2.0 ** -24 * np.abs(exact)
+            assert np.all(np.abs(acc - exact) <= bound + slack + 1e-30), (e, row)
+
+
+def test_w8a8_single_expert_vs_fp64_mlp():
+    """E = 1, k = 1: a row-scaled FP8 SwiGLU MLP against a textbook fp64 MLP on the dequantized
+    FP8 weights and the unquantized input: the gap is the FP8 activation rounding only."""
+    rng = np.random.default_rng(12)
+    T, H, N = 24, 512, 256
+    Wg = (rng.standard_normal((1, N, H)) * 0.02 * 2.0 ** rng.uniform(-3, 3, (1, N, 1))).astype(np.float32)
+    Wu = (rng.standard_normal((1, N, H)) * 0.02 * 2.0 ** rng.uniform(-3, 3, (1, N, 1))).astype(np.float32)
+    Wd = (rng.standard_normal((1, H, N)) * 0.02 * 2.0 ** rng.uniform(-3, 3, (1, H, 1))).astype(np.float32)
+    layer, (gq, gs, uq, us, dq, ds) = _w8_layer_from_f32(Wg, Wu, Wd)
+    x = _f32_to_bf16_bits(rng.standard_normal((T, H)).astype(np.float32))
+    r = oracle.moe_forward(layer, x, np.zeros((T, 1), np.float32), 1)
+    dec = oracle.e4m3_decode_table().astype(np.float64)
+    Dg = dec[gq[0]] * gs[0][:, None]
+    Du = dec[uq[0]] * us[0][:, None]
+    Dd = dec[dq[0]] * ds[0][:, None]
+    xf = oracle.bf16_to_f32(x).astype(np.float64)
+    g, u = xf @ Dg.T, xf @ Du.T
+    ref = (g / (1 + np.exp(-g)) * u) @ Dd.T
+    got = r["out_f32"].astype(np.float64)
+    rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
+    assert rel < 0.05, rel
+    assert np.corrcoef(got.ravel(), ref.ravel())[0, 1] > 0.998
+
+
+def test_w8a8_dense_brute_force_matches_permuted():
+    wl = synth.WORKLOADS["tiny"]
+    layer = oracle.quant_workload_layer_w8a8(wl)
+    assert layer.fmt == oracle.FMT_W8A8
+    x, lg = synth.tokens(wl), synth.logits(wl)
+    r = oracle.moe_forward(layer, x, lg, wl.k)
+    d = oracle.moe_forward_dense(layer, x, lg, wl.k)
+    assert np.array_equal(r["out"], d["out"])
+    for p in range(wl.P):
+        t, j = divmod(p, wl.k)
+        e = r["ids"][t, j]
+        row = r["row_of_pair"][p]
+        assert np.array_equal(r["hq"][row], d["hq"][t, e])
+        assert np.array_equal(r["y"][row], d["y"][t, e])
+    # the two formats agree to the INT4 weight-rounding gap (a step of amax/7 per weight,
+    # through three projections), not bit for bit
+    w4 = oracle.moe_forward(_tiny_layer(wl), x, lg, wl.k)
+    a, b = r["out_f32"].astype(np.float64), w4["out_f32"].astype(np.float64)
+    assert np.linalg.norm(a - b) / np.linalg.norm(a) < 0.35
+    assert not np.array_equal(r["out"], w4["out"])
+
+
+# ------------------------------------------------------------------------------------------------
 # the generator (input recipe)
 # ------------------------------------------------------------------------------------------------
 
