@@ -1,10 +1,12 @@
 """Throughput of the W4A8-FP8 routed MoE layer on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+                    [--experts w4a8|w8a8]
 
 One step = one moe_w4a8_forward over a T-token batch (routing, FP8 quantization, grouped
 gate/up GEMM, SwiGLU requantization, grouped down GEMM, shared experts if any, combine), with
-inputs already in HBM.  Batches rotate over 8 distinct seeded token sets, so the experts a
+inputs already in HBM.  `--experts w8a8` runs the same layer with row-scaled FP8 experts
+(moe_w8a8_forward) instead.  Batches rotate over 8 distinct seeded token sets, so the experts a
 step touches change from step to step; the touched expert weights of one step (~0.57 GB at
 T=8) already exceed the 126 MB L2.  Ranks (torchrun) are independent replicas, each with its
 own batches: weak scaling, no data-path collective.
@@ -39,10 +41,15 @@ FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 
 
-def expert_bytes(wl):
-    """Algorithmic bytes of one routed expert: packed INT4 codes + bf16 group scales."""
-    gate = wl.N * wl.H // 2 + wl.N * (wl.H // wl.group) * 2
-    down = wl.H * wl.N // 2 + wl.H * (wl.N // wl.group) * 2
+def expert_bytes(wl, fmt="w4a8"):
+    """Algorithmic bytes of one routed expert: packed INT4 codes + bf16 group scales (W4A8), or
+    E4M3 codes + fp32 row scales (W8A8)."""
+    if fmt == "w8a8":
+        gate = wl.N * wl.H + wl.N * 4
+        down = wl.H * wl.N + wl.H * 4
+    else:
+        gate = wl.N * wl.H // 2 + wl.N * (wl.H // wl.group) * 2
+        down = wl.H * wl.N // 2 + wl.H * (wl.N // wl.group) * 2
     return 2 * gate, down            # (gate+up, down)
 
 
@@ -71,15 +78,18 @@ def is_prefill(wl):
     return wl.T >= 1024
 
 
-KERNEL_SOURCES = ("gemm_ws.cuh", "tc_ptx.cuh", "tc_tiles.cuh", "common.cuh")
-PROFILE_FOR = {"decode_t8": "gemm_w4a8_ws_decode_t8.md",
-               "prefill_t2048_zipf": "gemm_w4a8_ws_prefill_t2048.md"}
+KERNEL_SOURCES = {"w4a8": ("gemm_ws.cuh", "tc_ptx.cuh", "tc_tiles.cuh", "common.cuh"),
+                  "w8a8": ("gemm_w8a8.cuh", "gemm_ws.cuh", "tc_ptx.cuh", "tc_tiles.cuh", "common.cuh")}
+PROFILE_FOR = {("w4a8", "decode_t8"): "gemm_w4a8_ws_decode_t8.md",
+               ("w4a8", "prefill_t2048_zipf"): "gemm_w4a8_ws_prefill_t2048.md",
+               ("w8a8", "decode_t8"): "gemm_w8a8_decode_t8.md",
+               ("w8a8", "prefill_t2048_zipf"): "gemm_w8a8_prefill_t2048.md"}
 
 
-def ncu_traffic(workload):
+def ncu_traffic(workload, fmt="w4a8"):
     """DRAM bytes per gate/up launch from the committed ncu summary of this workload, or None
     when there is none or the GEMM sources changed since it was taken."""
-    name = PROFILE_FOR.get(workload)
+    name = PROFILE_FOR.get((fmt, workload))
     if not name:
         return None
     try:
@@ -87,7 +97,7 @@ def ncu_traffic(workload):
         vals = dict(re.findall(r"^\s*(traffic_gateup_bytes_per_launch|sources_sha256):\s*(\S+)", text,
                                flags=re.M))
         h = hashlib.sha256()
-        for f in KERNEL_SOURCES:
+        for f in KERNEL_SOURCES[fmt]:
             with open(os.path.join(ROOT, "bit_quantized_moe_token_b200", "csrc", f), "rb") as fh:
                 h.update(fh.read())
         if vals.get("sources_sha256") != h.hexdigest():
@@ -224,7 +234,7 @@ def run_ours(args):
     import torch
     import torch.distributed as dist
     import bit_quantized_moe_token_b200 as moe
-    from bit_quantized_moe_token_b200.synthetic import device_inputs, device_layer
+    from bit_quantized_moe_token_b200.synthetic import device_inputs, device_layer, device_layer_w8a8
 
     world, rank, local = dist_setup()
     torch.cuda.set_device(local)
@@ -234,7 +244,11 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
 
     wl = synth.WORKLOADS[args.workload]
-    layer = device_layer(wl, device=dev)
+    w8 = args.experts == "w8a8"
+    layer = (device_layer_w8a8 if w8 else device_layer)(wl, device=dev)
+    fwd = moe.moe_w8a8_forward if w8 else moe.moe_w4a8_forward
+    fwd_profiled = moe.moe_w8a8_forward_profiled if w8 else moe.moe_w4a8_forward_profiled
+    layout = moe.moe_w8a8_workspace_layout if w8 else moe.moe_w4a8_workspace_layout
     if not wl.n_shared:
         layer.sh_gate = layer.sh_up = layer.sh_down = None
     T, k = wl.T, wl.k
@@ -247,7 +261,7 @@ def run_ours(args):
     stream = torch.cuda.current_stream(dev)
 
     # touched experts per batch (for the algorithmic byte count), from the routing outputs
-    lay = moe.moe_w4a8_workspace_layout(layer, T, k)
+    lay = layout(layer, T, k)
     touched = []
     for x, lg in batches:
         moe.forward(layer, x, lg, k, out=out, ws=ws)
@@ -275,7 +289,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     for i in range(N_BATCHES):
         x, lg = batches[i]
-        moe.moe_w4a8_forward_profiled(layer, x, lg, k, out, ws, full[i])
+        fwd_profiled(layer, x, lg, k, out, ws, full[i])
     torch.cuda.synchronize()
     stage_ms = {s: 0.0 for s in moe.STAGES}
     for i in range(N_BATCHES):
@@ -299,7 +313,7 @@ def run_ours(args):
     start.record(stream)
     for i in range(args.steps):
         x, lg = batches[i % N_BATCHES]
-        launches += moe.moe_w4a8_forward_profiled(layer, x, lg, k, out, ws, ev[i])
+        launches += fwd_profiled(layer, x, lg, k, out, ws, ev[i])
     end.record(stream)
     torch.cuda.synchronize()
     clk.mark_end()
@@ -321,7 +335,7 @@ def run_ours(args):
     for i in range(2):
         dx.copy_(hx[i], non_blocking=True)
         dl.copy_(hl[i], non_blocking=True)
-        moe.moe_w4a8_forward(layer, dx, dl, k, out, ws)
+        fwd(layer, dx, dl, k, out, ws)
         hout.copy_(out, non_blocking=True)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -332,7 +346,7 @@ def run_ours(args):
     for i in range(args.steps):
         dx.copy_(hx[i % N_BATCHES], non_blocking=True)
         dl.copy_(hl[i % N_BATCHES], non_blocking=True)
-        moe.moe_w4a8_forward(layer, dx, dl, k, out, ws)
+        fwd(layer, dx, dl, k, out, ws)
         hout.copy_(out, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
@@ -357,7 +371,9 @@ def run_ours(args):
     tokens = world * T * args.steps
     value = whole_job_rate(world, T, args.steps, total_ms)
     hbm, bf16, peak_kind = peaks()
-    gu_bytes, down_bytes = expert_bytes(wl)
+    fmt = args.experts
+    kname = "W8A8" if w8 else "W4A8"
+    gu_bytes, down_bytes = expert_bytes(wl, fmt)
     mean_touched = sum(touched[i % N_BATCHES] for i in range(args.steps)) / args.steps
     dom_bytes = mean_touched * gu_bytes
     if is_prefill(wl):
@@ -366,27 +382,29 @@ def run_ours(args):
         dom_flops = T * k * 2 * wl.H * 2 * wl.N
         achieved = dom_flops / (dom_ms / 1e3) / 1e12
         fp8 = 2.0 * bf16
-        roofline = {"bound": "tensor", "kernel": "grouped gate/up W4A8 GEMM (stage)",
+        roofline = {"bound": "tensor", "kernel": f"grouped gate/up {kname} GEMM (stage)",
                     "achieved": round(achieved, 1), "peak": round(fp8, 1), "unit": "TFLOP/s",
-                    "frac": round(achieved / fp8, 4), "traffic": ncu_traffic(wl.name),
+                    "frac": round(achieved / fp8, 4), "traffic": ncu_traffic(wl.name, fmt),
                     "peak_source": f"{peak_kind} bf16_tflops x 2 (nominal FP8/BF16 ratio)",
                     "algorithmic_flops_per_launch": int(dom_flops),
                     "units": f"{T * k} routed pairs x {2 * wl.H * 2 * wl.N} FLOP (gate+up)"}
     else:
         achieved = dom_bytes / (dom_ms / 1e3) / 1e9
-        roofline = {"bound": "hbm", "kernel": "grouped gate/up W4A8 GEMM (stage)",
+        roofline = {"bound": "hbm", "kernel": f"grouped gate/up {kname} GEMM (stage)",
                     "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
-                    "frac": round(achieved / hbm, 4), "traffic": ncu_traffic(wl.name),
+                    "frac": round(achieved / hbm, 4), "traffic": ncu_traffic(wl.name, fmt),
                     "peak_source": f"{peak_kind} hbm_gbs",
                     "algorithmic_bytes_per_launch": int(dom_bytes),
                     "units": f"{mean_touched:.1f} touched experts x {gu_bytes} B (gate+up codes+scales)"}
+    if w8:
+        roofline["units"] = roofline["units"].replace("(gate+up)", "(gate+up, W8A8)")
     layer_bytes = mean_touched * (gu_bytes + down_bytes)
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "e4m3 x int4 -> f32", "data": "synthetic",
-        "config": {"workload": wl.name, "T": T, "H": wl.H, "N": wl.N, "E": wl.E, "k": k,
+        "dtype": "e4m3 x e4m3 -> f32" if w8 else "e4m3 x int4 -> f32", "data": "synthetic",
+        "config": {"workload": wl.name, "experts": fmt, "T": T, "H": wl.H, "N": wl.N, "E": wl.E, "k": k,
                    "routing": wl.routing, "n_shared": wl.n_shared, "seed": wl.seed,
                    "batches": N_BATCHES, "parallelism": f"replicas x{world}",
                    "l2": "inputs larger than L2: touched expert weights per step "
@@ -402,7 +420,7 @@ def run_ours(args):
         "clocks": clk.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = cpu_baseline(wl, batches_t0=0)
+        result["cpu_baseline"] = cpu_baseline(wl, batches_t0=0, fmt=fmt)
     if world > 1:
         dist.destroy_process_group()
     if rank == 0:
@@ -413,7 +431,7 @@ def run_ours(args):
 # the CPU oracle
 # ------------------------------------------------------------------------------------------------
 
-def oracle_sample(wl, t0, max_tokens):
+def oracle_sample(wl, t0, max_tokens, fmt="w4a8"):
     """A bounded sample of the workload for the CPU oracle: the first tokens of one batch,
     with the experts they route to packed (untimed setup)."""
     import oracle
@@ -421,7 +439,11 @@ def oracle_sample(wl, t0, max_tokens):
     x = synth.tokens(wl, t0, n)
     lg = synth.logits(wl, t0, n)
     ids, _ = oracle.route_topk(lg, wl.k)
-    layer = oracle.pack_workload_layer(wl, experts=sorted(set(ids.reshape(-1).tolist())))
+    used = sorted(set(ids.reshape(-1).tolist()))
+    if fmt == "w8a8":
+        layer = oracle.quant_workload_layer_w8a8(wl, experts=used)
+    else:
+        layer = oracle.pack_workload_layer(wl, experts=used)
     return layer, x, lg, n
 
 
@@ -432,9 +454,9 @@ def cores_used():
         return os.cpu_count() or 1
 
 
-def cpu_baseline(wl, batches_t0=0, max_tokens=8):
+def cpu_baseline(wl, batches_t0=0, max_tokens=8, fmt="w4a8"):
     import oracle
-    layer, x, lg, n = oracle_sample(wl, batches_t0, max_tokens)
+    layer, x, lg, n = oracle_sample(wl, batches_t0, max_tokens, fmt)
     t = time.perf_counter()
     oracle.moe_forward(layer, x, lg, wl.k)
     dt = time.perf_counter() - t
@@ -449,7 +471,7 @@ def run_reference(args):
         return
     import oracle
     wl = synth.WORKLOADS[args.workload]
-    layer, x, lg, n = oracle_sample(wl, 0, args.ref_tokens)
+    layer, x, lg, n = oracle_sample(wl, 0, args.ref_tokens, args.experts)
     for _ in range(args.warmup):
         oracle.moe_forward(layer, x, lg, wl.k)
     t = time.perf_counter()
@@ -462,9 +484,9 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic", "impl": "reference",
-        "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "N": wl.N, "E": wl.E, "k": wl.k,
-                   "routing": wl.routing, "n_shared": wl.n_shared, "seed": wl.seed,
-                   "parallelism": "host cores"},
+        "config": {"workload": wl.name, "experts": args.experts, "T": wl.T, "H": wl.H, "N": wl.N,
+                   "E": wl.E, "k": wl.k, "routing": wl.routing, "n_shared": wl.n_shared,
+                   "seed": wl.seed, "parallelism": "host cores"},
         "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": cores_used(),
                          "kind": "oracle",
                          "sample": f"{n} tokens of {wl.name} per step (C oracle, fp32)"},
@@ -482,6 +504,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ref-tokens", type=int, default=8)
+    ap.add_argument("--experts", default="w4a8", choices=["w4a8", "w8a8"],
+                    help="routed-expert weight format (default: W4A8 INT4 x FP8)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:

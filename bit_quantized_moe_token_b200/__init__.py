@@ -9,8 +9,11 @@ from ._binding import (MOE_OK, Layer, MoeError, fp8_quant_tokens, layer_struct, 
                        moe_status_string, moe_w4a8_forward, moe_w4a8_forward_profiled,
                        moe_w4a8_workspace_bytes, STAGES, N_STAGE_EVENTS,
                        moe_w4a8_workspace_layout, w4a8_pack_weights,
-                       moe_selftest_bounded_wait)
-from .layer import alloc_workspace, forward, make_layer, pack_expert_weights
+                       moe_selftest_bounded_wait, Layer8, layer8_struct, w8a8_quant_weights,
+                       moe_w8a8_workspace_bytes, moe_w8a8_workspace_layout, moe_w8a8_forward,
+                       moe_w8a8_forward_profiled)
+from .layer import (alloc_workspace, forward, make_layer, make_layer_w8a8, pack_expert_weights,
+                    quant_expert_weights_w8a8)
 
 __all__ = ["MOE_OK", "Layer", "MoeError", "fp8_quant_tokens", "layer_struct", "lib",
            "moe_last_device_status", "moe_route_topk", "moe_route_workspace_bytes",
@@ -18,4 +21,7 @@ __all__ = ["MOE_OK", "Layer", "MoeError", "fp8_quant_tokens", "layer_struct", "l
            "moe_status_string", "moe_w4a8_forward", "moe_w4a8_forward_profiled", "STAGES",
            "N_STAGE_EVENTS", "moe_w4a8_workspace_bytes",
            "moe_w4a8_workspace_layout", "w4a8_pack_weights", "alloc_workspace", "forward",
-           "make_layer", "pack_expert_weights", "moe_selftest_bounded_wait"]
+           "make_layer", "pack_expert_weights", "moe_selftest_bounded_wait",
+           "Layer8", "layer8_struct", "w8a8_quant_weights", "moe_w8a8_workspace_bytes",
+           "moe_w8a8_workspace_layout", "moe_w8a8_forward", "moe_w8a8_forward_profiled",
+           "make_layer_w8a8", "quant_expert_weights_w8a8"]

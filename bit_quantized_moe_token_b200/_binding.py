@@ -37,6 +37,17 @@ class _CLayer(ctypes.Structure):
                 ("sh_down", ctypes.c_void_p)]
 
 
+class _CLayer8(ctypes.Structure):
+    _fields_ = [("E", ctypes.c_int), ("H", ctypes.c_int), ("N", ctypes.c_int),
+                ("gate_w8", ctypes.c_void_p), ("up_w8", ctypes.c_void_p),
+                ("down_w8", ctypes.c_void_p),
+                ("gate_rs", ctypes.c_void_p), ("up_rs", ctypes.c_void_p),
+                ("down_rs", ctypes.c_void_p),
+                ("n_shared", ctypes.c_int), ("shared_N", ctypes.c_int),
+                ("sh_gate", ctypes.c_void_p), ("sh_up", ctypes.c_void_p),
+                ("sh_down", ctypes.c_void_p)]
+
+
 class _CLayout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in
                 ("topk_ids", "topk_w", "expert_offsets", "sorted_pairs", "row_of_pair",
@@ -72,6 +83,14 @@ def lib() -> ctypes.CDLL:
         L.moe_w4a8_forward.argtypes = [ctypes.POINTER(_CLayer), vp, vp, i64, i32, vp, vp, sz, vp]
         L.moe_w4a8_forward_profiled.argtypes = [ctypes.POINTER(_CLayer), vp, vp, i64, i32, vp, vp,
                                                 sz, vp, vp, i32, ctypes.POINTER(ctypes.c_int)]
+        L.w8a8_quant_weights.argtypes = [vp, i64, i64, vp, vp, vp]
+        L.moe_w8a8_workspace_bytes.argtypes = [ctypes.POINTER(_CLayer8), i64, i32]
+        L.moe_w8a8_workspace_bytes.restype = sz
+        L.moe_w8a8_workspace_layout.argtypes = [ctypes.POINTER(_CLayer8), i64, i32,
+                                                ctypes.POINTER(_CLayout)]
+        L.moe_w8a8_forward.argtypes = [ctypes.POINTER(_CLayer8), vp, vp, i64, i32, vp, vp, sz, vp]
+        L.moe_w8a8_forward_profiled.argtypes = [ctypes.POINTER(_CLayer8), vp, vp, i64, i32, vp, vp,
+                                                sz, vp, vp, i32, vp]
         L.moe_last_device_status.argtypes = [vp]
         L.moe_selftest_bounded_wait.argtypes = [i64, vp]
         L.moe_status_string.argtypes = [i32]
@@ -246,3 +265,89 @@ def moe_last_device_status(stream=None) -> int:
 def moe_selftest_bounded_wait(limit_ns: int, stream=None) -> None:
     _check(lib().moe_selftest_bounded_wait(int(limit_ns), _stream(stream)),
            "moe_selftest_bounded_wait")
+
+
+# ---- row-scaled FP8 (W8A8) experts -------------------------------------------------------------
+
+def w8a8_quant_weights(w, q, row_scale, stream=None) -> None:
+    """w bf16 [..., rows, K] -> q uint8 (E4M3 codes) [..., rows, K], row_scale fp32 [..., rows]."""
+    K = w.shape[-1]
+    rows = w.numel() // K
+    _check(lib().w8a8_quant_weights(_ptr(w), rows, K, _ptr(q), _ptr(row_scale), _stream(stream)),
+           "w8a8_quant_weights")
+
+
+@dataclass
+class Layer8:
+    """Device tensors of one layer with row-scaled FP8 experts (moe_w8a8_layer)."""
+    E: int
+    H: int
+    N: int
+    gate_w8: object
+    up_w8: object
+    down_w8: object
+    gate_rs: object
+    up_rs: object
+    down_rs: object
+    sh_gate: object = None
+    sh_up: object = None
+    sh_down: object = None
+
+    @property
+    def n_shared(self) -> int:
+        return 0 if self.sh_gate is None else int(self.sh_gate.shape[0])
+
+    @property
+    def shared_N(self) -> int:
+        return 0 if self.sh_gate is None else int(self.sh_gate.shape[1])
+
+    def c_struct(self) -> _CLayer8:
+        return _CLayer8(self.E, self.H, self.N,
+                        _ptr(self.gate_w8), _ptr(self.up_w8), _ptr(self.down_w8),
+                        _ptr(self.gate_rs), _ptr(self.up_rs), _ptr(self.down_rs),
+                        self.n_shared, self.shared_N,
+                        _ptr(self.sh_gate), _ptr(self.sh_up), _ptr(self.sh_down))
+
+    def shape_struct(self) -> _CLayer8:
+        return _CLayer8(self.E, self.H, self.N, None, None, None, None, None, None,
+                        self.n_shared, self.shared_N, None, None, None)
+
+
+def layer8_struct(E, H, N, n_shared=0, shared_N=0) -> _CLayer8:
+    return _CLayer8(E, H, N, None, None, None, None, None, None, n_shared, shared_N,
+                    None, None, None)
+
+
+def moe_w8a8_workspace_bytes(layer, T: int, k: int) -> int:
+    s = layer if isinstance(layer, _CLayer8) else layer.shape_struct()
+    return int(lib().moe_w8a8_workspace_bytes(ctypes.byref(s), T, k))
+
+
+def moe_w8a8_workspace_layout(layer, T: int, k: int) -> dict:
+    s = layer if isinstance(layer, _CLayer8) else layer.shape_struct()
+    out = _CLayout()
+    _check(lib().moe_w8a8_workspace_layout(ctypes.byref(s), T, k, ctypes.byref(out)),
+           "moe_w8a8_workspace_layout")
+    return {n: int(getattr(out, n)) for n, _ in _CLayout._fields_}
+
+
+def moe_w8a8_forward(layer: Layer8, x, logits, k: int, out, ws, stream=None) -> None:
+    """out bf16 [T, H] = the routed MoE layer with row-scaled FP8 experts applied to x."""
+    T = x.shape[0]
+    s = layer.c_struct()
+    nbytes = ws.numel() * ws.element_size() if ws is not None else 0
+    _check(lib().moe_w8a8_forward(ctypes.byref(s), _ptr(x), _ptr(logits), T, k, _ptr(out),
+                                  _ptr(ws), nbytes, _stream(stream)), "moe_w8a8_forward")
+
+
+def moe_w8a8_forward_profiled(layer: Layer8, x, logits, k: int, out, ws, events, stream=None) -> int:
+    T = x.shape[0]
+    s = layer.c_struct()
+    nbytes = ws.numel() * ws.element_size() if ws is not None else 0
+    arr = (ctypes.c_void_p * len(events))(
+        *[ctypes.c_void_p(e.cuda_event if e is not None else 0) for e in events])
+    n = ctypes.c_int(0)
+    _check(lib().moe_w8a8_forward_profiled(ctypes.byref(s), _ptr(x), _ptr(logits), T, k, _ptr(out),
+                                           _ptr(ws), nbytes, _stream(stream), arr, len(events),
+                                           ctypes.byref(n)), "moe_w8a8_forward_profiled")
+    return int(n.value)

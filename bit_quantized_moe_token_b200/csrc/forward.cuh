@@ -1,10 +1,11 @@
 // forward.cuh — S5 SwiGLU + per-row FP8 requantization, S7 combine, the workspace plan and
-// moe_w4a8_forward.
+// the layer entry points (moe_w4a8_forward, and moe_w8a8_forward for row-scaled FP8 experts).
 #pragma once
 #include "common.cuh"
 #include "quant.cuh"
 #include "route.cuh"
 #include "gemm_ws.cuh"
+#include "gemm_w8a8.cuh"
 #include "gemm_bf16_tc.cuh"
 
 namespace moe {
@@ -94,7 +95,7 @@ __global__ void __launch_bounds__(256) k_quant_topk(const float* __restrict__ lo
         const uint2 codes = live ? quant8(__ldg(row + c), s) : make_uint2(0u, 0u);
         if (live) reinterpret_cast<uint2*>(xq + t * H)[c] = codes;
         const float gs = halfwarp_sum(e4m3x8_sum(codes));
-        if (live && (threadIdx.x & 15) == 0) qsum[t * G + c / 16] = gs;
+        if (qsum && live && (threadIdx.x & 15) == 0) qsum[t * G + c / 16] = gs;
     }
     if (threadIdx.x == 0) s_x[t] = s;
 }
@@ -202,6 +203,18 @@ extern "C" int moe_w4a8_workspace_layout(const moe_w4a8_layer* layer, int64_t T,
 
 namespace moe {
 
+// Routed-expert weights of one layer in either format.
+struct ExpertSet {
+    bool w8;                              // row-scaled FP8 (true) or W4A8 (false)
+    const void *gate, *up, *down;         // W4A8: int32 [E,R,K/8]; W8A8: E4M3 [E,R,K]
+    const void *gate_s, *up_s, *down_s;   // W4A8: bf16 [E,R,K/128]; W8A8: fp32 [E,R]
+};
+
+inline ExpertSet experts_of(const moe_w4a8_layer& L) {
+    return ExpertSet{false, L.gate_packed, L.up_packed, L.down_packed, L.gate_scales, L.up_scales,
+                     L.down_scales};
+}
+
 // Records stage-boundary events when profiling; counts kernel launches.
 struct StageMarks {
     void* const* ev;
@@ -212,9 +225,10 @@ struct StageMarks {
     }
 };
 
-int forward_impl(const moe_w4a8_layer* layer, const uint16_t* x_bf16, const float* router_logits,
-                 int64_t T, int k, uint16_t* out_bf16, void* ws, size_t ws_bytes,
-                 cudaStream_t stream, StageMarks& sm);
+// `layer` gives the shapes and the shared experts; `xs` the routed experts' weights.
+int forward_impl(const moe_w4a8_layer* layer, const ExpertSet& xs, const uint16_t* x_bf16,
+                 const float* router_logits, int64_t T, int k, uint16_t* out_bf16, void* ws,
+                 size_t ws_bytes, cudaStream_t stream, StageMarks& sm);
 
 }  // namespace moe
 
@@ -222,7 +236,9 @@ extern "C" int moe_w4a8_forward(const moe_w4a8_layer* layer, const uint16_t* x_b
                                 const float* router_logits, int64_t T, int k, uint16_t* out_bf16,
                                 void* ws, size_t ws_bytes, moe_stream_t stream) {
     moe::StageMarks sm{nullptr, 0, 0};
-    return moe::forward_impl(layer, x_bf16, router_logits, T, k, out_bf16, ws, ws_bytes, stream, sm);
+    if (!layer) return MOE_ERR_INVALID_ARG;
+    return moe::forward_impl(layer, moe::experts_of(*layer), x_bf16, router_logits, T, k, out_bf16, ws,
+                             ws_bytes, stream, sm);
 }
 
 extern "C" int moe_w4a8_forward_profiled(const moe_w4a8_layer* layer, const uint16_t* x_bf16,
@@ -232,13 +248,14 @@ extern "C" int moe_w4a8_forward_profiled(const moe_w4a8_layer* layer, const uint
                                          int* n_launches) {
     if (events && n_events < MOE_W4A8_N_STAGE_EVENTS) return MOE_ERR_INVALID_ARG;
     moe::StageMarks sm{events, n_events, 0};
-    const int st =
-        moe::forward_impl(layer, x_bf16, router_logits, T, k, out_bf16, ws, ws_bytes, stream, sm);
+    if (!layer) return MOE_ERR_INVALID_ARG;
+    const int st = moe::forward_impl(layer, moe::experts_of(*layer), x_bf16, router_logits, T, k,
+                                     out_bf16, ws, ws_bytes, stream, sm);
     if (n_launches) *n_launches = sm.launches;
     return st;
 }
 
-int moe::forward_impl(const moe_w4a8_layer* layer, const uint16_t* x_bf16,
+int moe::forward_impl(const moe_w4a8_layer* layer, const ExpertSet& xw, const uint16_t* x_bf16,
                       const float* router_logits, int64_t T, int k, uint16_t* out_bf16, void* ws,
                       size_t ws_bytes, cudaStream_t stream, StageMarks& sm) {
     using namespace moe;
@@ -246,18 +263,19 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const uint16_t* x_bf16,
     if (st != MOE_OK) return st;
     const moe_w4a8_layer& L = *layer;
     if (T == 0) return MOE_OK;
-    if (!x_bf16 || !router_logits || !out_bf16 || !L.gate_packed || !L.up_packed ||
-        !L.down_packed || !L.gate_scales || !L.up_scales || !L.down_scales)
+    if (!x_bf16 || !router_logits || !out_bf16 || !xw.gate || !xw.up || !xw.down || !xw.gate_s ||
+        !xw.up_s || !xw.down_s)
         return MOE_ERR_INVALID_ARG;
     if (L.n_shared > 0 && (!L.sh_gate || !L.sh_up || !L.sh_down)) return MOE_ERR_INVALID_ARG;
     if (L.n_shared > 0 && (!aligned(L.sh_gate, 16) || !aligned(L.sh_up, 16) || !aligned(L.sh_down, 16)))
         return MOE_ERR_MISALIGNED;
     const WsPlan p = plan_workspace(L, T, k);
     if (!ws || ws_bytes < p.total) return MOE_ERR_WORKSPACE;
+    const size_t s_al = xw.w8 ? 4 : 2;   // fp32 row scales / bf16 group scales
     if (!aligned(ws, 256) || !aligned(x_bf16, 16) || !aligned(out_bf16, 16) ||
-        !aligned(router_logits, 4) || !aligned(L.gate_packed, 16) || !aligned(L.up_packed, 16) ||
-        !aligned(L.down_packed, 16) || !aligned(L.gate_scales, 2) || !aligned(L.up_scales, 2) ||
-        !aligned(L.down_scales, 2))
+        !aligned(router_logits, 4) || !aligned(xw.gate, 16) || !aligned(xw.up, 16) ||
+        !aligned(xw.down, 16) || !aligned(xw.gate_s, s_al) || !aligned(xw.up_s, s_al) ||
+        !aligned(xw.down_s, s_al))
         return MOE_ERR_MISALIGNED;
 
     const int64_t P = T * k;
@@ -289,7 +307,8 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const uint16_t* x_bf16,
     sm.mark(0, stream);
     if (fused) {
         // S1 + S2: per-token FP8 codes and top-k
-        if ((st = launch_quant_topk(router_logits, x_bf16, T, L.E, k, L.H, ids, gates, xq, sx, qs_x, stream)))
+        if ((st = launch_quant_topk(router_logits, x_bf16, T, L.E, k, L.H, ids, gates, xq, sx,
+                                    xw.w8 ? nullptr : qs_x, stream)))
             return st;
         sm.launches += 1;
         sm.mark(1, stream);
@@ -326,12 +345,20 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const uint16_t* x_bf16,
     }
     sm.mark(3, stream);
     // S4 + SwiGLU (+ S5 when fused): h = silu(G) * U, max|h| per row
-    {
-        WsGemmArgs a{fused ? sx : sxs, L.gate_scales, L.up_scales, offsets, L.E, L.N, L.H, (int)P, h, L.N,
-                     amax, rowcnt, hq, sh, sorted, nullptr, nullptr, k, nullptr, nullptr, (int)T,
-                     fused ? qs_x : nullptr, nullptr};
-        if ((st = launch_gemm_ws<true>(a, fused ? (const void*)xq : (const void*)xs, L.gate_packed,
-                                       L.up_packed, stream)))
+    if (xw.w8) {
+        W8GemmArgs a{fused ? sx : sxs, (const float*)xw.gate_s, (const float*)xw.up_s, offsets, L.E, L.N,
+                     L.H, (int)P, h, L.N, amax, rowcnt, hq, sh, sorted, nullptr, nullptr, k, nullptr,
+                     nullptr, (int)T};
+        if ((st = launch_gemm_w8a8<true>(a, fused ? (const void*)xq : (const void*)xs, xw.gate, xw.up,
+                                         stream)))
+            return st;
+        sm.launches += 1;
+    } else {
+        WsGemmArgs a{fused ? sx : sxs, (const uint16_t*)xw.gate_s, (const uint16_t*)xw.up_s, offsets, L.E,
+                     L.N, L.H, (int)P, h, L.N, amax, rowcnt, hq, sh, sorted, nullptr, nullptr, k, nullptr,
+                     nullptr, (int)T, fused ? qs_x : nullptr, nullptr};
+        if ((st = launch_gemm_ws<true>(a, fused ? (const void*)xq : (const void*)xs, xw.gate, xw.up,
+                                       stream)))
             return st;
         sm.launches += 1;
     }
@@ -344,11 +371,16 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const uint16_t* x_bf16,
     }
     sm.mark(5, stream);
     // S6 (+ S7 when fused)
-    {
-        WsGemmArgs a{sh, L.down_scales, nullptr, offsets, L.E, L.H, L.N, (int)P, y, L.H, nullptr,
-                     tokcnt, nullptr, nullptr, sorted, rop, gates, k, shared, out_bf16, (int)T,
+    if (xw.w8) {
+        W8GemmArgs a{sh, (const float*)xw.down_s, nullptr, offsets, L.E, L.H, L.N, (int)P, y, L.H, nullptr,
+                     tokcnt, nullptr, nullptr, sorted, rop, gates, k, shared, out_bf16, (int)T};
+        if ((st = launch_gemm_w8a8<false>(a, hq, xw.down, nullptr, stream))) return st;
+        sm.launches += 1;
+    } else {
+        WsGemmArgs a{sh, (const uint16_t*)xw.down_s, nullptr, offsets, L.E, L.H, L.N, (int)P, y, L.H,
+                     nullptr, tokcnt, nullptr, nullptr, sorted, rop, gates, k, shared, out_bf16, (int)T,
                      nullptr, nullptr};
-        if ((st = launch_gemm_ws<false>(a, hq, L.down_packed, nullptr, stream))) return st;
+        if ((st = launch_gemm_ws<false>(a, hq, xw.down, nullptr, stream))) return st;
         sm.launches += 1;
     }
     sm.mark(6, stream);
@@ -362,4 +394,55 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const uint16_t* x_bf16,
     }
     sm.mark(7, stream);
     return MOE_OK;
+}
+
+// ---- row-scaled FP8 experts ------------------------------------------------------------------
+
+namespace moe {
+// The shape / shared-expert view of a W8A8 layer (group 128: the GEMM's K step).
+inline moe_w4a8_layer shape_of(const moe_w8a8_layer& L) {
+    return moe_w4a8_layer{L.E, L.H, L.N, kGroup, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
+                          L.n_shared, L.shared_N, L.sh_gate, L.sh_up, L.sh_down};
+}
+inline ExpertSet experts_of(const moe_w8a8_layer& L) {
+    return ExpertSet{true, L.gate_w8, L.up_w8, L.down_w8, L.gate_rs, L.up_rs, L.down_rs};
+}
+}  // namespace moe
+
+extern "C" size_t moe_w8a8_workspace_bytes(const moe_w8a8_layer* layer, int64_t T, int k) {
+    if (!layer) return 0;
+    const moe_w4a8_layer s = moe::shape_of(*layer);
+    return moe_w4a8_workspace_bytes(&s, T, k);
+}
+
+extern "C" int moe_w8a8_workspace_layout(const moe_w8a8_layer* layer, int64_t T, int k,
+                                         moe_w4a8_ws_layout* out) {
+    if (!layer) return MOE_ERR_INVALID_ARG;
+    const moe_w4a8_layer s = moe::shape_of(*layer);
+    return moe_w4a8_workspace_layout(&s, T, k, out);
+}
+
+extern "C" int moe_w8a8_forward(const moe_w8a8_layer* layer, const uint16_t* x_bf16,
+                                const float* router_logits, int64_t T, int k, uint16_t* out_bf16,
+                                void* ws, size_t ws_bytes, moe_stream_t stream) {
+    if (!layer) return MOE_ERR_INVALID_ARG;
+    moe::StageMarks sm{nullptr, 0, 0};
+    const moe_w4a8_layer s = moe::shape_of(*layer);
+    return moe::forward_impl(&s, moe::experts_of(*layer), x_bf16, router_logits, T, k, out_bf16, ws,
+                             ws_bytes, stream, sm);
+}
+
+extern "C" int moe_w8a8_forward_profiled(const moe_w8a8_layer* layer, const uint16_t* x_bf16,
+                                         const float* router_logits, int64_t T, int k,
+                                         uint16_t* out_bf16, void* ws, size_t ws_bytes,
+                                         moe_stream_t stream, void* const* events, int n_events,
+                                         int* n_launches) {
+    if (!layer) return MOE_ERR_INVALID_ARG;
+    if (events && n_events < MOE_W4A8_N_STAGE_EVENTS) return MOE_ERR_INVALID_ARG;
+    moe::StageMarks sm{events, n_events, 0};
+    const moe_w4a8_layer s = moe::shape_of(*layer);
+    const int st = moe::forward_impl(&s, moe::experts_of(*layer), x_bf16, router_logits, T, k,
+                                     out_bf16, ws, ws_bytes, stream, sm);
+    if (n_launches) *n_launches = sm.launches;
+    return st;
 }

@@ -100,3 +100,11 @@ extern "C" int fp8_quant_tokens(const uint16_t* x_bf16, int64_t T, int64_t H, ui
     if (T > 0x7FFFFFFF) return MOE_ERR_UNSUPPORTED_SHAPE;
     return launch_quant_tokens(x_bf16, T, H, q_e4m3, scale, nullptr, 1, stream);
 }
+
+// Row-scaled FP8 weights ("Inkling 2 Small FP8 for AMD MI300X" card, "Precision and files": one
+// fp32 scale per output channel, the row's max |w| over the largest FP8 value): the per-token
+// rule above applied to weight rows.
+extern "C" int w8a8_quant_weights(const uint16_t* w_bf16, int64_t rows, int64_t K, uint8_t* q_e4m3,
+                                  float* row_scale, moe_stream_t stream) {
+    return fp8_quant_tokens(w_bf16, rows, K, q_e4m3, row_scale, stream);
+}

@@ -1,7 +1,8 @@
 """Convenience wrappers: torch allocation around the C entry points."""
 from __future__ import annotations
 
-from ._binding import (Layer, moe_w4a8_forward, moe_w4a8_workspace_bytes, w4a8_pack_weights)
+from ._binding import (Layer, Layer8, moe_w4a8_forward, moe_w4a8_workspace_bytes, moe_w8a8_forward,
+                       moe_w8a8_workspace_bytes, w4a8_pack_weights, w8a8_quant_weights)
 
 
 def pack_expert_weights(w, group: int = 128, stream=None):
@@ -25,20 +26,46 @@ def make_layer(gate_w, up_w, down_w, sh_gate=None, sh_up=None, sh_down=None,
     return Layer(E, H, N, gp, up, dp, gs, us, ds, sh_gate=sh_gate, sh_up=sh_up, sh_down=sh_down)
 
 
-def alloc_workspace(layer: Layer, T: int, k: int, device=None):
+def quant_expert_weights_w8a8(w, stream=None):
+    """bf16 weights [..., rows, K] on the GPU -> (E4M3 codes uint8 [..., rows, K],
+    fp32 row scales [..., rows])."""
     import torch
-    n = moe_w4a8_workspace_bytes(layer, T, k)
+    *lead, rows, K = w.shape
+    q = torch.empty(*lead, rows, K, dtype=torch.uint8, device=w.device)
+    s = torch.empty(*lead, rows, dtype=torch.float32, device=w.device)
+    w8a8_quant_weights(w.contiguous(), q, s, stream=stream)
+    return q, s
+
+
+def make_layer_w8a8(gate_w, up_w, down_w, sh_gate=None, sh_up=None, sh_down=None,
+                    stream=None) -> Layer8:
+    """Row-quantize bf16 expert weights gate/up [E, N, H], down [E, H, N] to FP8."""
+    E, N, H = gate_w.shape
+    gq, gs = quant_expert_weights_w8a8(gate_w, stream=stream)
+    uq, us = quant_expert_weights_w8a8(up_w, stream=stream)
+    dq, ds = quant_expert_weights_w8a8(down_w, stream=stream)
+    return Layer8(E, H, N, gq, uq, dq, gs, us, ds, sh_gate=sh_gate, sh_up=sh_up, sh_down=sh_down)
+
+
+def alloc_workspace(layer, T: int, k: int, device=None):
+    import torch
+    w8 = isinstance(layer, Layer8)
+    n = (moe_w8a8_workspace_bytes if w8 else moe_w4a8_workspace_bytes)(layer, T, k)
     if n == 0 and T > 0:
-        raise ValueError("unsupported layer shape for moe_w4a8_forward")
-    dev = device if device is not None else layer.gate_packed.device
+        raise ValueError("unsupported layer shape for the MoE forward")
+    dev = device if device is not None else (layer.gate_w8 if w8 else layer.gate_packed).device
     return torch.empty(max(n, 256), dtype=torch.uint8, device=dev)
 
 
-def forward(layer: Layer, x, logits, k: int, out=None, ws=None, stream=None):
+def forward(layer, x, logits, k: int, out=None, ws=None, stream=None):
+    """The layer on x for either expert format (Layer: W4A8, Layer8: row-scaled FP8)."""
     import torch
     if out is None:
         out = torch.empty_like(x)
     if ws is None:
         ws = alloc_workspace(layer, x.shape[0], k, x.device)
-    moe_w4a8_forward(layer, x, logits, k, out, ws, stream=stream)
+    if isinstance(layer, Layer8):
+        moe_w8a8_forward(layer, x, logits, k, out, ws, stream=stream)
+    else:
+        moe_w4a8_forward(layer, x, logits, k, out, ws, stream=stream)
     return out

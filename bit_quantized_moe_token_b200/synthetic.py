@@ -1,35 +1,44 @@
 """Seeded synthetic layers and batches in HBM (for tests, smoke and the benchmark).
 
 Weights are drawn on the GPU by the seeded generator (``synth``), bit-identical to the host
-draws the CPU oracle makes, then quantized and packed by ``w4a8_pack_weights``.
+draws the CPU oracle makes, then quantized and packed by ``w4a8_pack_weights`` (or, for the
+row-scaled FP8 format, quantized by ``w8a8_quant_weights``).
 """
 from __future__ import annotations
 
 import synth
 
-from ._binding import Layer
-from .layer import pack_expert_weights
+from ._binding import Layer, Layer8
+from .layer import pack_expert_weights, quant_expert_weights_w8a8
 
 
-def device_layer(wl: synth.Workload, device="cuda", experts_per_chunk: int = 32) -> Layer:
-    """The packed routed experts (and bf16 shared experts) of workload `wl` on `device`."""
+def _expert_tensors(wl, device, experts_per_chunk, w8):
     import torch
-    E, H, N = wl.E, wl.H, wl.N
-    packed = {}
+    E = wl.E
+    out = {}
     for proj in ("gate", "up", "down"):
         rows, K = synth.weight_shape(wl, proj)
-        p = torch.empty(E, rows, K // 8, dtype=torch.int32, device=device)
-        s = torch.empty(E, rows, K // wl.group, dtype=torch.bfloat16, device=device)
+        if w8:
+            p = torch.empty(E, rows, K, dtype=torch.uint8, device=device)
+            s = torch.empty(E, rows, dtype=torch.float32, device=device)
+        else:
+            p = torch.empty(E, rows, K // 8, dtype=torch.int32, device=device)
+            s = torch.empty(E, rows, K // wl.group, dtype=torch.bfloat16, device=device)
         buf = torch.empty(min(E, experts_per_chunk), rows, K, dtype=torch.bfloat16, device=device)
         for e0 in range(0, E, experts_per_chunk):
             n = min(experts_per_chunk, E - e0)
             for i in range(n):
                 synth.dev_weight(wl.seed, synth.weight_stream(e0 + i, proj), buf[i])
-            pp, ss = pack_expert_weights(buf[:n])
+            pp, ss = (quant_expert_weights_w8a8 if w8 else pack_expert_weights)(buf[:n])
             p[e0:e0 + n].copy_(pp)
             s[e0:e0 + n].copy_(ss)
-        packed[proj] = (p, s)
+        out[proj] = (p, s)
         del buf
+    return out
+
+
+def _shared_tensors(wl, device):
+    import torch
     sh = {}
     if wl.n_shared:
         for proj, key in (("gate", "sh_gate"), ("up", "sh_up"), ("down", "sh_down")):
@@ -38,9 +47,27 @@ def device_layer(wl: synth.Workload, device="cuda", experts_per_chunk: int = 32)
             for s_ in range(wl.n_shared):
                 synth.dev_weight(wl.seed, synth.shared_stream(s_, proj), t[s_])
             sh[key] = t
+    return sh
+
+
+def device_layer(wl: synth.Workload, device="cuda", experts_per_chunk: int = 32) -> Layer:
+    """The packed routed experts (and bf16 shared experts) of workload `wl` on `device`."""
+    import torch
+    packed = _expert_tensors(wl, device, experts_per_chunk, w8=False)
+    sh = _shared_tensors(wl, device)
     torch.cuda.synchronize()
-    return Layer(E, H, N, packed["gate"][0], packed["up"][0], packed["down"][0],
+    return Layer(wl.E, wl.H, wl.N, packed["gate"][0], packed["up"][0], packed["down"][0],
                  packed["gate"][1], packed["up"][1], packed["down"][1], group=wl.group, **sh)
+
+
+def device_layer_w8a8(wl: synth.Workload, device="cuda", experts_per_chunk: int = 32) -> Layer8:
+    """The same seeded experts of workload `wl` in the row-scaled FP8 format."""
+    import torch
+    q = _expert_tensors(wl, device, experts_per_chunk, w8=True)
+    sh = _shared_tensors(wl, device)
+    torch.cuda.synchronize()
+    return Layer8(wl.E, wl.H, wl.N, q["gate"][0], q["up"][0], q["down"][0],
+                  q["gate"][1], q["up"][1], q["down"][1], **sh)
 
 
 def device_inputs(wl: synth.Workload, device="cuda", t0: int = 0, T: int | None = None):

@@ -196,6 +196,61 @@ int moe_w4a8_forward_profiled(const moe_w4a8_layer* layer, const uint16_t* x_bf1
                               void* ws, size_t ws_bytes, moe_stream_t stream,
                               void* const* events, int n_events, int* n_launches);
 
+/* ---------------------------------------------------------------------------------------
+ * Row-scaled FP8 (W8A8) experts: a second weight format on the same layer.
+ *
+ * The "Inkling 2 Small FP8 for AMD MI300X" card ("Precision and files") stores the expert
+ * projections as FP8 with one fp32 scale per expert output channel, computed as the row's
+ * max |w| over the largest FP8 value, and runs them on per-token FP8 activations.  The card's
+ * FP8 is AMD's E4M3FNUZ (largest value 240); this library keeps the one FP8 format it uses
+ * everywhere, OCP E4M3FN (448), so a weight row is quantized exactly like a token row of
+ * fp8_quant_tokens:
+ *     scale[r] = max_k |w[r,k]| / 448,   q[r,k] = e4m3_rn_satfinite(w[r,k] / scale[r])
+ *
+ *   w_bf16     [rows, K] bf16 weights, 16-byte aligned;  K a positive multiple of 8, <= 65536
+ *   q_e4m3     [rows, K] E4M3 output, 16-byte aligned
+ *   row_scale  [rows] fp32 output
+ * rows == 0 is a no-op.
+ * --------------------------------------------------------------------------------------- */
+int w8a8_quant_weights(const uint16_t* w_bf16, int64_t rows, int64_t K, uint8_t* q_e4m3,
+                       float* row_scale, moe_stream_t stream);
+
+/* The layer with row-scaled FP8 routed experts, gate and up as separate projections:
+ *   gate_w8, up_w8  [E, N, H] E4M3      gate_rs, up_rs  [E, N] fp32 row scales
+ *   down_w8         [E, H, N] E4M3      down_rs         [E, H] fp32 row scales
+ * (E4M3 pointers 16-byte aligned, scales 4-byte aligned); shared experts as in moe_w4a8_layer. */
+typedef struct {
+    int E, H, N;
+    const uint8_t *gate_w8, *up_w8, *down_w8;
+    const float *gate_rs, *up_rs, *down_rs;
+    int n_shared, shared_N;
+    const uint16_t *sh_gate, *sh_up, *sh_down;
+} moe_w8a8_layer;
+
+/* Workspace size and layout of moe_w8a8_forward: the same plan (and the same offsets) as the
+ * W4A8 layer of equal shape. */
+size_t moe_w8a8_workspace_bytes(const moe_w8a8_layer* layer, int64_t T, int k);
+int moe_w8a8_workspace_layout(const moe_w8a8_layer* layer, int64_t T, int k,
+                              moe_w4a8_ws_layout* out);
+
+/*
+ * The layer of moe_w4a8_forward with each projection computed on row-scaled FP8 weights:
+ *   G[n] = (sum_k Xq[t,k] * Wgate[e,n,k]) * s_gate[e,n] * s_x[t]      (likewise U)
+ *   h    = silu(G) * U;   s_h = max|h| / 448;   Hq = e4m3(h / s_h)
+ *   Y[m] = (sum_n Hq[n] * Wdown[e,m,n]) * s_down[e,m] * s_h
+ * with the same routing, permutation, requantization, shared experts and combine.  Same
+ * shape limits and return codes as moe_w4a8_forward.
+ */
+int moe_w8a8_forward(const moe_w8a8_layer* layer, const uint16_t* x_bf16,
+                     const float* router_logits, int64_t T, int k, uint16_t* out_bf16, void* ws,
+                     size_t ws_bytes, moe_stream_t stream);
+
+/* Profiling variant of moe_w8a8_forward, with the stage events of moe_w4a8_forward_profiled. */
+int moe_w8a8_forward_profiled(const moe_w8a8_layer* layer, const uint16_t* x_bf16,
+                              const float* router_logits, int64_t T, int k, uint16_t* out_bf16,
+                              void* ws, size_t ws_bytes, moe_stream_t stream,
+                              void* const* events, int n_events, int* n_launches);
+
 /* Waits for `stream`, then returns and clears the library's sticky device-status word for
  * the current device: MOE_OK, or MOE_ERR_TIMEOUT when a bounded device-side wait gave up
  * (its kernel then skipped the rest of its work and returned), or MOE_ERR_CUDA when the

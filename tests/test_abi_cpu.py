@@ -27,7 +27,8 @@ def _declared_functions():
 def test_header_declares_the_boundary():
     names = _declared_functions()
     for n in ("w4a8_pack_weights", "fp8_quant_tokens", "moe_route_topk", "moe_w4a8_forward",
-              "moe_router_logits",
+              "moe_router_logits", "w8a8_quant_weights", "moe_w8a8_forward",
+              "moe_w8a8_workspace_bytes", "moe_w8a8_forward_profiled",
               "moe_w4a8_workspace_bytes", "moe_last_device_status", "moe_status_string"):
         assert n in names
 
@@ -133,6 +134,28 @@ def test_forward_rejects_bad_args():
     assert L.moe_w4a8_forward(ctypes.byref(full), p, p, 4, 0, p, p, need, None) == -1
     assert L.moe_w4a8_forward(ctypes.byref(full), p, p, 0, 2, p, p, need, None) == 0
     assert L.moe_w4a8_forward(None, p, p, 4, 2, p, p, need, None) == -1
+
+
+def test_w8a8_rejects_bad_args():
+    L = _L()
+    p = ctypes.c_void_p(4096)
+    assert L.w8a8_quant_weights(p, 4, 12, p, p, None) == -2              # K % 8
+    assert L.w8a8_quant_weights(None, 4, 16, p, p, None) == -1
+    assert L.w8a8_quant_weights(p, 0, 16, p, p, None) == 0
+    s8 = moe.layer8_struct(256, 4096, 2048)
+    s4 = moe.layer_struct(256, 4096, 2048)
+    assert moe.moe_w8a8_workspace_bytes(s8, 8, 6) == moe.moe_w4a8_workspace_bytes(s4, 8, 6) > 0
+    assert moe.moe_w8a8_workspace_layout(s8, 8, 6) == moe.moe_w4a8_workspace_layout(s4, 8, 6)
+    assert moe.moe_w8a8_workspace_bytes(moe.layer8_struct(256, 4000, 2048), 8, 6) == 0
+    assert L.moe_w8a8_forward(ctypes.byref(s8), p, p, 4, 2, p, p, 1 << 24, None) == -1   # null weights
+    full = moe._binding._CLayer8(8, 256, 128, p, p, p, p, p, p, 0, 0, None, None, None)
+    need = moe.moe_w8a8_workspace_bytes(full, 4, 2)
+    assert L.moe_w8a8_forward(ctypes.byref(full), p, p, 4, 2, p, p, need - 1, None) == -4
+    odd = moe._binding._CLayer8(8, 256, 128, p, p, p, ctypes.c_void_p(4098), p, p, 0, 0, None, None,
+                                None)                                     # fp32 scales need 4 bytes
+    assert L.moe_w8a8_forward(ctypes.byref(odd), p, p, 4, 2, p, p, need, None) == -3
+    assert L.moe_w8a8_forward(ctypes.byref(full), p, p, 0, 2, p, p, need, None) == 0
+    assert L.moe_w8a8_forward(None, p, p, 4, 2, p, p, need, None) == -1
 
 
 def test_binding_has_no_fallback():

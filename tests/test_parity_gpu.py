@@ -13,7 +13,7 @@ pytestmark = pytest.mark.gpu
 if cuda_ok():
     import torch
     import bit_quantized_moe_token_b200 as moe
-    from bit_quantized_moe_token_b200.synthetic import device_inputs, device_layer
+    from bit_quantized_moe_token_b200.synthetic import device_inputs, device_layer, device_layer_w8a8
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -34,7 +34,8 @@ def bits(t):
 
 
 def ws_views(layer, ws, T, k):
-    lay = moe.moe_w4a8_workspace_layout(layer, T, k)
+    layout = moe.moe_w8a8_workspace_layout if isinstance(layer, moe.Layer8) else moe.moe_w4a8_workspace_layout
+    lay = layout(layer, T, k)
     P = T * k
     b = ws.cpu().numpy()
     def arr(off, dtype, n):
@@ -372,3 +373,125 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     hl = oracle.pack_workload_layer(wl)
     dl = device_layer(wl)
     _run_and_compare(hl, dl, synth.tokens(wl), synth.logits(wl), wl.k)
+
+
+# ---- row-scaled FP8 (W8A8) experts ---------------------------------------------------------------
+
+def test_w8a8_quant_weights_bitexact():
+    rng = np.random.default_rng(21)
+    w = (rng.standard_normal((300, 512)) * 0.02 * 2.0 ** rng.uniform(-6, 6, (300, 1))).astype(np.float32)
+    w[5] = 0.0                                         # zero row: scale 0, codes 0
+    w[6, 7] = 1e30                                     # huge outlier: every other code flushes to 0
+    w[7, :] = -3.0e-38                                 # subnormal-scale row
+    wb = _f32_to_bf16_bits(w)
+    q_ref, s_ref = oracle.quant_rows(wb)
+    q = torch.empty(300, 512, dtype=torch.uint8, device="cuda")
+    sc = torch.empty(300, dtype=torch.float32, device="cuda")
+    moe.w8a8_quant_weights(to_dev_bf16(wb), q, sc)
+    torch.cuda.synchronize()
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+    assert np.array_equal(sc.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+
+
+def _host_layer_and_dev_w8a8(E, H, N, seed, n_shared=0, shared_N=0):
+    """Seeded random layer, rows scaled over 2^-3..2^3: row-quantized on the host by the oracle
+    and on the GPU by the library."""
+    rng_stream = 60_000 + seed * 10
+    def w(stream, rows, K):
+        a = synth.normal_f32(seed, stream, E * rows * K, 0.02).reshape(E, rows, K)
+        scale = 2.0 ** np.round(synth.normal_f32(seed, stream + 5, E * rows).reshape(E, rows, 1) * 1.5)
+        return _f32_to_bf16_bits((a * scale).astype(np.float32))
+    gw, uw, dw = w(rng_stream, N, H), w(rng_stream + 1, N, H), w(rng_stream + 2, H, N)
+    def rq(W):
+        qs = [oracle.quant_rows(W[e]) for e in range(E)]
+        return np.stack([a for a, _ in qs]), np.stack([b for _, b in qs])
+    (gq, gs), (uq, us), (dq, ds) = rq(gw), rq(uw), rq(dw)
+    sh, shd = {}, {}
+    if n_shared:
+        for i, key in enumerate(("sh_gate", "sh_up", "sh_down")):
+            shape = (n_shared, shared_N, H) if i < 2 else (n_shared, H, shared_N)
+            a = synth.normal_bf16(seed, rng_stream + 3 + i, int(np.prod(shape)), 0.02).reshape(shape)
+            sh[key] = a
+            shd[key] = to_dev_bf16(a)
+    hl = oracle.Layer.w8a8(E, H, N, gq, uq, dq, gs, us, ds, **sh)
+    dl = moe.make_layer_w8a8(to_dev_bf16(gw), to_dev_bf16(uw), to_dev_bf16(dw), **shd)
+    torch.cuda.synchronize()
+    assert np.array_equal(dl.gate_w8.cpu().numpy(), gq)
+    assert np.array_equal(dl.down_w8.cpu().numpy(), dq)
+    assert np.array_equal(dl.up_rs.cpu().numpy(), us)
+    return hl, dl
+
+
+def test_w8a8_forward_tiny_workload():
+    wl = synth.WORKLOADS["tiny"]
+    hl = oracle.quant_workload_layer_w8a8(wl)
+    dl = device_layer_w8a8(wl)
+    assert np.array_equal(dl.up_w8.cpu().numpy(), hl.up_w8)
+    assert np.array_equal(dl.down_rs.cpu().numpy(), hl.down_rs)
+    r1 = _run_and_compare(hl, dl, synth.tokens(wl), synth.logits(wl), wl.k)
+    r2 = _run_and_compare(hl, dl, synth.tokens(wl), synth.logits(wl), wl.k)
+    assert np.array_equal(r1["out"], r2["out"])        # deterministic
+
+
+# token-tile widths chosen by rows per expert: 16 (decode, fused), 32 (fused), 64, 128 (prefill)
+@pytest.mark.parametrize("E,H,N,k,T", [(5, 384, 256, 3, 37), (1, 256, 128, 1, 9), (8, 256, 128, 2, 1),
+                                       (8, 256, 256, 2, 200), (16, 512, 384, 8, 130),
+                                       (3, 1024, 128, 2, 700), (64, 1024, 1024, 6, 16)])
+def test_w8a8_forward_ragged_shapes(E, H, N, k, T):
+    hl, dl = _host_layer_and_dev_w8a8(E, H, N, seed=E * 7 + T)
+    x = synth.normal_bf16(3, 777 + T, T * H).reshape(T, H)
+    logits = synth.normal_f32(3, 778 + T, T * E).reshape(T, E)
+    _run_and_compare(hl, dl, x, logits, k)
+
+
+def test_w8a8_forward_shared_experts_and_zero_rows():
+    hl, dl = _host_layer_and_dev_w8a8(4, 256, 128, seed=5, n_shared=2, shared_N=256)
+    T = 21
+    x = synth.normal_bf16(4, 901, T * 256).reshape(T, 256)
+    x[3, :] = 0
+    logits = synth.normal_f32(4, 902, T * 4).reshape(T, 4)
+    r = _run_and_compare(hl, dl, x, logits, 2)
+    ref = oracle.moe_forward(hl, x, logits, 2)
+    assert np.array_equal(r["out"][3], ref["out"][3])  # shared experts of a zero row: exactly 0
+    xd = torch.empty(0, 256, dtype=torch.bfloat16, device="cuda")
+    ld = torch.empty(0, 4, dtype=torch.float32, device="cuda")
+    out = torch.empty(0, 256, dtype=torch.bfloat16, device="cuda")
+    moe.moe_w8a8_forward(dl, xd, ld, 2, out, torch.empty(256, dtype=torch.uint8, device="cuda"))
+
+
+@pytest.fixture(scope="module")
+def full_layer_w8a8():
+    return device_layer_w8a8(synth.WORKLOADS["prefill_t16384_shared"])
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_w8a8_forward_full_size_sampled(name, full_layer_w8a8):
+    wl = synth.WORKLOADS[name]
+    dl = full_layer_w8a8
+    if not wl.n_shared:
+        dl = moe.Layer8(dl.E, dl.H, dl.N, dl.gate_w8, dl.up_w8, dl.down_w8, dl.gate_rs, dl.up_rs,
+                        dl.down_rs)
+    x, lg = device_inputs(wl)
+    ws = moe.alloc_workspace(dl, wl.T, wl.k)
+    out = moe.forward(dl, x, lg, wl.k, ws=ws)
+    torch.cuda.synchronize()
+    assert moe.moe_last_device_status() == 0
+    v = ws_views(dl, ws, wl.T, wl.k)
+    outb = bits(out)
+    assert np.isfinite(bf16_to_f32(outb)).all()
+    toks = _sample_tokens(wl)
+    xs = np.stack([synth.tokens(wl, t, 1)[0] for t in toks])
+    ls = np.stack([synth.logits(wl, t, 1)[0] for t in toks])
+    ids_ref, _ = oracle.route_topk(ls, wl.k)
+    experts = sorted(set(ids_ref.reshape(-1).tolist()))
+    hl = oracle.quant_workload_layer_w8a8(wl, experts=experts)
+    for e in experts[:3]:
+        assert np.array_equal(dl.gate_w8[e].cpu().numpy(), hl.gate_w8[e])
+        assert np.array_equal(dl.down_rs[e].cpu().numpy(), hl.down_rs[e])
+    ref = oracle.moe_forward(hl, xs, ls, wl.k)
+    assert np.array_equal(v["ids"][toks], ref["ids"])
+    gpu_rows = v["row_of_pair"].reshape(wl.T, wl.k)[toks].reshape(-1)
+    assert np.array_equal(v["xq"][toks], ref["xq"])
+    check_fp8_codes(v["hq"][gpu_rows], ref["hq"][ref["row_of_pair"]])
+    np.testing.assert_allclose(v["s_h"][gpu_rows], ref["s_h"][ref["row_of_pair"]], rtol=2e-5)
+    check_output(outb[toks], ref["out"])
