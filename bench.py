@@ -74,7 +74,8 @@ def router_line(wl, T, ms, hbm, bf16, peak_kind):
 
 
 def is_prefill(wl):
-    """Prefill shapes are scored against the FP8 tensor peak, decode shapes against HBM."""
+    """Prefill-sized batches: the router GEMM runs on the tensor cores from T >= 256 and is
+    scored against the bf16 peak here."""
     return wl.T >= 1024
 
 
@@ -86,23 +87,29 @@ PROFILE_FOR = {("w4a8", "decode_t8"): "gemm_w4a8_ws_decode_t8.md",
                ("w8a8", "prefill_t2048_zipf"): "gemm_w8a8_prefill_t2048.md"}
 
 
-def ncu_traffic(workload, fmt="w4a8"):
+def ncu_traffic(workload, fmt="w4a8", algorithmic_bytes=None):
     """DRAM bytes per gate/up launch from the committed ncu summary of this workload, or None
-    when there is none or the GEMM sources changed since it was taken."""
+    when there is none or the GEMM sources changed since it was taken.  A summary taken on a
+    reduced-expert case of the same shape gives DRAM bytes per algorithmic byte instead, scaled
+    here to this launch's algorithmic bytes (the traffic grows with the touched experts)."""
     name = PROFILE_FOR.get((fmt, workload))
     if not name:
         return None
     try:
         text = open(os.path.join(ROOT, "profiles", name)).read()
-        vals = dict(re.findall(r"^\s*(traffic_gateup_bytes_per_launch|sources_sha256):\s*(\S+)", text,
-                               flags=re.M))
+        vals = dict(re.findall(r"^\s*(traffic_gateup_bytes_per_launch|traffic_gateup_per_algorithmic_byte|"
+                               r"sources_sha256):\s*(\S+)", text, flags=re.M))
         h = hashlib.sha256()
         for f in KERNEL_SOURCES[fmt]:
             with open(os.path.join(ROOT, "bit_quantized_moe_token_b200", "csrc", f), "rb") as fh:
                 h.update(fh.read())
         if vals.get("sources_sha256") != h.hexdigest():
             return None
-        return int(vals["traffic_gateup_bytes_per_launch"])
+        if "traffic_gateup_bytes_per_launch" in vals:
+            return int(vals["traffic_gateup_bytes_per_launch"])
+        if algorithmic_bytes is not None and "traffic_gateup_per_algorithmic_byte" in vals:
+            return int(float(vals["traffic_gateup_per_algorithmic_byte"]) * algorithmic_bytes)
+        return None
     except (OSError, KeyError, ValueError):
         return None
 
@@ -376,28 +383,32 @@ def run_ours(args):
     gu_bytes, down_bytes = expert_bytes(wl, fmt)
     mean_touched = sum(touched[i % N_BATCHES] for i in range(args.steps)) / args.steps
     dom_bytes = mean_touched * gu_bytes
-    if is_prefill(wl):
-        # compute-bound shape: gate/up FLOPs over the dense FP8 tensor peak (the measured bf16
-        # cuBLAS peak x 2, NVIDIA's nominal FP8 / BF16 ratio)
-        dom_flops = T * k * 2 * wl.H * 2 * wl.N
-        achieved = dom_flops / (dom_ms / 1e3) / 1e12
-        fp8 = 2.0 * bf16
-        roofline = {"bound": "tensor", "kernel": f"grouped gate/up {kname} GEMM (stage)",
-                    "achieved": round(achieved, 1), "peak": round(fp8, 1), "unit": "TFLOP/s",
-                    "frac": round(achieved / fp8, 4), "traffic": ncu_traffic(wl.name, fmt),
-                    "peak_source": f"{peak_kind} bf16_tflops x 2 (nominal FP8/BF16 ratio)",
-                    "algorithmic_flops_per_launch": int(dom_flops),
-                    "units": f"{T * k} routed pairs x {2 * wl.H * 2 * wl.N} FLOP (gate+up)"}
-    else:
-        achieved = dom_bytes / (dom_ms / 1e3) / 1e9
-        roofline = {"bound": "hbm", "kernel": f"grouped gate/up {kname} GEMM (stage)",
-                    "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
-                    "frac": round(achieved / hbm, 4), "traffic": ncu_traffic(wl.name, fmt),
-                    "peak_source": f"{peak_kind} hbm_gbs",
-                    "algorithmic_bytes_per_launch": int(dom_bytes),
-                    "units": f"{mean_touched:.1f} touched experts x {gu_bytes} B (gate+up codes+scales)"}
-    if w8:
-        roofline["units"] = roofline["units"].replace("(gate+up)", "(gate+up, W8A8)")
+    # Both bounds of the gate/up GEMM: its algorithmic bytes (touched experts' gate+up weights)
+    # over the measured HBM bandwidth, and its FLOPs over the dense FP8 tensor peak (the measured
+    # bf16 cuBLAS peak x 2, NVIDIA's nominal FP8 / BF16 ratio).  The reported bound is the one
+    # with the longer ideal time (the binding one); the other is reported beside it.
+    dom_flops = T * k * 2 * wl.H * 2 * wl.N
+    fp8 = 2.0 * bf16
+    t_hbm = dom_bytes / (hbm * 1e9)
+    t_tc = dom_flops / (fp8 * 1e12)
+    ach_gbs = dom_bytes / (dom_ms / 1e3) / 1e9
+    ach_tf = dom_flops / (dom_ms / 1e3) / 1e12
+    hbm_side = {"bound": "hbm", "achieved": round(ach_gbs, 1), "peak": hbm, "unit": "GB/s",
+                "frac": round(ach_gbs / hbm, 4), "peak_source": f"{peak_kind} hbm_gbs",
+                "algorithmic_bytes_per_launch": int(dom_bytes),
+                "units": f"{mean_touched:.1f} touched experts x {gu_bytes} B (gate+up codes+scales)"}
+    tc_side = {"bound": "tensor", "achieved": round(ach_tf, 1), "peak": round(fp8, 1),
+               "unit": "TFLOP/s", "frac": round(ach_tf / fp8, 4),
+               "peak_source": f"{peak_kind} bf16_tflops x 2 (nominal FP8/BF16 ratio)",
+               "algorithmic_flops_per_launch": int(dom_flops),
+               "units": f"{T * k} routed pairs x {2 * wl.H * 2 * wl.N} FLOP (gate+up)"}
+    main, other = (tc_side, hbm_side) if t_tc >= t_hbm else (hbm_side, tc_side)
+    roofline = {"bound": main["bound"], "kernel": f"grouped gate/up {kname} GEMM (stage)",
+                "achieved": main["achieved"], "peak": main["peak"], "unit": main["unit"],
+                "frac": main["frac"], "traffic": ncu_traffic(wl.name, fmt, dom_bytes)}
+    roofline.update({k_: v for k_, v in main.items() if k_ not in roofline})
+    roofline["other_bound"] = {k_: v for k_, v in other.items() if k_ != "units"}
+    roofline["ideal_us"] = {"hbm": round(t_hbm * 1e6, 1), "tensor": round(t_tc * 1e6, 1)}
     layer_bytes = mean_touched * (gu_bytes + down_bytes)
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,

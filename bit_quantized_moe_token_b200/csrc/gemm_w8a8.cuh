@@ -15,7 +15,9 @@
 //              swizzle the MMA reads.
 //   warp 5     MMA: one lane issues four tcgen05.mma.kind::f8f6f4 (K = 32 each) per stage,
 //              commits the stage back to the TMA warp and, after a tile's last stage, the
-//              accumulator to the epilogue warps; the warp owns the TMEM.
+//              accumulator to the epilogue warps; the warp owns the TMEM.  The MMA's N is the
+//              tile's live rows rounded up to 16 (a runtime field of the instruction
+//              descriptor), so a segment's last, partly filled tile costs only what it holds.
 // Swap AB as in the W4A8 GEMM: MMA M = 128 weight rows (gate/up: 64 gate rows and the same 64
 // up rows), N = BN tokens of one expert's segment.  The epilogues are the W4A8 GEMM's: SwiGLU
 // with max|h| per row (narrow tiles: the requantization fused behind a row counter), or the
@@ -61,7 +63,7 @@ struct W8Cfg {
     static constexpr int kStage = kA + kB;                  // a multiple of 1024
     static_assert(kStage % 1024 == 0, "stage alignment");
     // ring depth: about 190 KB of stages in flight per SM
-    static constexpr int kRS = BN <= 32 ? 10 : (BN <= 64 ? 8 : 6);
+    static constexpr int kRS = BN <= 32 ? 10 : (BN <= 64 ? 8 : (BN <= 128 ? 6 : 4));
     static constexpr int kChunk = BN < 32 ? BN : 32;        // TMEM columns per epilogue load
     static constexpr int kXStride = kChunk + 1;             // SwiGLU exchange: 64 x kChunk (+1)
     static constexpr int kOffX = kRS * kStage;
@@ -176,7 +178,7 @@ __global__ void __launch_bounds__(W8Cfg<BN>::kThreads, 1)
     } else if (warp == C::kWarpMma) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idesc = tc::idesc_e4m3_f32(128, BN);
+            const uint32_t idesc_full = tc::idesc_e4m3_f32(128, BN);
             // descriptors of stage 0; stage i starts i * kStage / 16 later in the start-address
             // field and a K step of 32 bytes adds 2 (1024-byte-aligned tiles in the first 256 KB
             // of shared memory keep the 14-bit field from carrying)
@@ -188,6 +190,11 @@ __global__ void __launch_bounds__(W8Cfg<BN>::kThreads, 1)
             uint32_t last_phase = 0;
             for (int64_t tile = blockIdx.x; tile < n_tiles && !*abort; tile += gridDim.x, ++tcount) {
                 const int tb = tcount & 1;
+                const int rt = static_cast<int>(tile / m_tiles);
+                const int e = expert_of_tile(pre, a.E, rt);
+                const int nrows = min(BN, soff[e + 1] - soff[e] - (rt - pre[e]) * BN);
+                const int n_mma = min(BN, (nrows + 15) & ~15);
+                const uint32_t idesc = n_mma == BN ? idesc_full : tc::idesc_e4m3_f32(128, n_mma);
                 if (!ws::wait(&t_empty[tb], ((tcount >> 1) & 1) ^ 1u, abort)) break;
                 tc::tc_fence_after();
                 const uint32_t d = tmem + tb * BN;
@@ -223,10 +230,10 @@ __global__ void __launch_bounds__(W8Cfg<BN>::kThreads, 1)
             const int64_t row0 = soff[e] + (rt - pre[e]) * BN;
             const int nrows = min(BN, soff[e + 1] - static_cast<int>(row0));
             float* sr_t = sSr + (tcount & 1) * BN;         // two buffers: tile parity
-            if (tid < BN) {
+            for (int c = tid; c < BN; c += kNPT) {
                 float v = 0.0f;
-                if (tid < nrows) v = kGather ? a.s_row[a.sorted[row0 + tid] / a.k] : a.s_row[row0 + tid];
-                sr_t[tid] = v;
+                if (c < nrows) v = kGather ? a.s_row[a.sorted[row0 + c] / a.k] : a.s_row[row0 + c];
+                sr_t[c] = v;
             }
             const float rs = kSwiGLU
                 ? __ldg((lrow < 64 ? a.rs0 : a.rs1) + (int64_t)e * a.R0 + mt * 64 + (lrow & 63))
@@ -237,7 +244,7 @@ __global__ void __launch_bounds__(W8Cfg<BN>::kThreads, 1)
             ws::named_sync_math<kNPT>();                   // column scales visible
             const uint32_t tcol = tmem + t_lane + tb * BN;
 #pragma unroll 1
-            for (int c0 = 0; c0 < BN; c0 += kCh) {
+            for (int c0 = 0; c0 < nrows; c0 += kCh) {       // only the columns the MMA wrote
                 uint32_t v[kCh];
                 if constexpr (kCh == 32) tc::tmem_ld32(tcol + c0, *reinterpret_cast<uint32_t(*)[32]>(v));
                 else tc::tmem_ld16(tcol + c0, *reinterpret_cast<uint32_t(*)[16]>(v));
@@ -369,18 +376,26 @@ int launch_gemm_w8a8_inst(const W8GemmArgs& a, const void* act, const void* w0, 
     return launch_status();
 }
 
-// Token-tile width as for the W4A8 GEMM; narrow tiles (decode) gather their gate/up activation
-// rows by token and fuse the requantization / combine into the epilogues.
+// Token-tile width for the expected rows per expert: as for the W4A8 GEMM, plus 256-row tiles
+// for long segments (a weight stage then feeds twice the tokens, halving the weight bytes moved
+// per FLOP).  Narrow tiles (decode) gather their gate/up activation rows by token and fuse the
+// requantization / combine into the epilogues.
+inline int w8_tile_rows(int64_t P, int E) {
+    const int64_t avg = (P + E - 1) / E;
+    return avg > 160 ? 256 : tc_tile_rows(P, E);
+}
+
 template <bool kSwiGLU>
 int launch_gemm_w8a8(const W8GemmArgs& a, const void* act, const void* w0, const void* w1,
                      cudaStream_t stream) {
-    const int BN = tc_tile_rows(a.P, a.E);
+    const int BN = w8_tile_rows(a.P, a.E);
     const int64_t max_row_tiles = ((int64_t)a.P + BN - 1) / BN + a.E;
     switch (BN) {
         case 16: return launch_gemm_w8a8_inst<16, kSwiGLU, true, kSwiGLU>(a, act, w0, w1, max_row_tiles, stream);
         case 32: return launch_gemm_w8a8_inst<32, kSwiGLU, true, kSwiGLU>(a, act, w0, w1, max_row_tiles, stream);
         case 64: return launch_gemm_w8a8_inst<64, kSwiGLU, false, false>(a, act, w0, w1, max_row_tiles, stream);
-        default: return launch_gemm_w8a8_inst<128, kSwiGLU, false, false>(a, act, w0, w1, max_row_tiles, stream);
+        case 128: return launch_gemm_w8a8_inst<128, kSwiGLU, false, false>(a, act, w0, w1, max_row_tiles, stream);
+        default: return launch_gemm_w8a8_inst<256, kSwiGLU, false, false>(a, act, w0, w1, max_row_tiles, stream);
     }
 }
 

@@ -80,6 +80,12 @@ WORKLOADS = {
     "prefill_t16384_shared": Workload("prefill_t16384_shared", T=16384, H=4096, N=2048, E=256,
                                       k=6, outliers=False, routing="uniform", n_shared=2,
                                       shared_N=2048),
+    # The same layer shape with 64 experts: profiler captures that replay each launch many times
+    # stay within a few GB of device memory (the full 256-expert row-scaled FP8 layer is 6.4 GB).
+    "decode_t8_e64": Workload("decode_t8_e64", T=8, H=4096, N=2048, E=64, k=6, outliers=True,
+                              routing="uniform"),
+    "prefill_t512_e64_zipf": Workload("prefill_t512_e64_zipf", T=512, H=4096, N=2048, E=64, k=6,
+                                      outliers=True, routing="zipf"),
 }
 
 

@@ -433,10 +433,11 @@ def test_w8a8_forward_tiny_workload():
     assert np.array_equal(r1["out"], r2["out"])        # deterministic
 
 
-# token-tile widths chosen by rows per expert: 16 (decode, fused), 32 (fused), 64, 128 (prefill)
+# token-tile widths chosen by rows per expert: 16 (decode, fused), 32 (fused), 64, 128, 256
 @pytest.mark.parametrize("E,H,N,k,T", [(5, 384, 256, 3, 37), (1, 256, 128, 1, 9), (8, 256, 128, 2, 1),
                                        (8, 256, 256, 2, 200), (16, 512, 384, 8, 130),
-                                       (3, 1024, 128, 2, 700), (64, 1024, 1024, 6, 16)])
+                                       (8, 256, 256, 2, 600), (3, 1024, 128, 2, 700),
+                                       (2, 512, 256, 1, 1000), (64, 1024, 1024, 6, 16)])
 def test_w8a8_forward_ragged_shapes(E, H, N, k, T):
     hl, dl = _host_layer_and_dev_w8a8(E, H, N, seed=E * 7 + T)
     x = synth.normal_bf16(3, 777 + T, T * H).reshape(T, H)
