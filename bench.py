@@ -73,6 +73,38 @@ def router_line(wl, T, ms, hbm, bf16, peak_kind):
             "algorithmic_bytes": int(nbytes)}
 
 
+def graph_time(call, n, stream):
+    """Mean device time (ms) of call(0..n-1), the n calls captured in one CUDA graph and replayed
+    once between CUDA events; falls back to an eager loop if capture fails.  Returns (ms, graph?)."""
+    import torch
+    for i in range(3):
+        call(i)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    try:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(n):
+                call(i)
+        g.replay()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / n
+        del g
+        return ms, True
+    except Exception:
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for i in range(n):
+            call(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / n, False
+
+
 def is_prefill(wl):
     """Prefill-sized batches: the router GEMM runs on the tensor cores from T >= 256 and is
     scored against the bf16 peak here."""
@@ -359,21 +391,36 @@ def run_ours(args):
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev, world)
 
-    # router logits (the step upstream of the layer's given logits), timed on its own
+    # router logits (the step upstream of the layer's given logits), timed on its own: `steps`
+    # calls captured in one CUDA graph, so that the host-side cost of a Python call per tiny
+    # launch is not what is measured (an eager loop is the fallback if capture fails)
     wr = torch.empty(wl.E, wl.H, dtype=torch.int16, device=dev)
     synth.dev_weight(wl.seed, synth.ROUTER_STREAM, wr, sigma=1.0 / math.sqrt(wl.H))
     wr = wr.view(torch.bfloat16)
     rlog = torch.empty(T, wl.E, dtype=torch.float32, device=dev)
+    rids = torch.empty(T, k, dtype=torch.int32, device=dev)
+    rgw = torch.empty(T, k, dtype=torch.float32, device=dev)
+    rws = torch.empty(max(256, moe.moe_router_topk_workspace_bytes(T, wl.E, k)), dtype=torch.uint8, device=dev)
+    r_ms, r_graph = graph_time(lambda i: moe.moe_router_logits(batches[i % N_BATCHES][0], wr, rlog),
+                               args.steps, stream)
+    rt_ms, _ = graph_time(lambda i: moe.moe_router_topk(batches[i % N_BATCHES][0], wr, k, rlog, rids, rgw, rws),
+                          args.steps, stream)
+    r_ms = max_over_ranks(r_ms, dev, world)
+    rt_ms = max_over_ranks(rt_ms, dev, world)
+    # the whole layer fed by the router weight (router, S1, S2 fused at decode)
+    fwd_router = moe.moe_w8a8_forward_router if w8 else moe.moe_w4a8_forward_router
     for i in range(3):
-        moe.moe_router_logits(batches[i % N_BATCHES][0], wr, rlog)
-    r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        fwd_router(layer, batches[i % N_BATCHES][0], wr, k, out, ws)
+    q0, q1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
-    r0.record(stream)
+    q0.record(stream)
     for i in range(args.steps):
-        moe.moe_router_logits(batches[i % N_BATCHES][0], wr, rlog)
-    r1.record(stream)
+        fwd_router(layer, batches[i % N_BATCHES][0], wr, k, out, ws)
+    q1.record(stream)
     torch.cuda.synchronize()
-    r_ms = max_over_ranks(r0.elapsed_time(r1), dev, world) / args.steps
+    lr_ms = max_over_ranks(q0.elapsed_time(q1), dev, world) / args.steps
+    if moe.moe_last_device_status() != 0:
+        raise RuntimeError("device status: timeout in the router timing")
 
     tokens = world * T * args.steps
     value = whole_job_rate(world, T, args.steps, total_ms)
@@ -424,7 +471,11 @@ def run_ours(args):
         "roofline": roofline,
         "stages_ms": {s: round(v, 4) for s, v in stage_ms.items()},
         "gpu_launches": launches,
-        "router": router_line(wl, T, r_ms, hbm, bf16, peak_kind),
+        "router": dict(router_line(wl, T, r_ms, hbm, bf16, peak_kind),
+                       topk_fused_ms=round(rt_ms, 4), cuda_graph=r_graph),
+        "layer_with_router": {"ms_per_step": round(lr_ms, 4),
+                              "value": round(world * T / (lr_ms / 1e3), 1), "unit": "tokens/s",
+                              "note": "moe_*_forward_router: router logits + the layer per step"},
         "e2e": {"value": round(tokens / (e2e_ms / 1e3), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * wl.H * 2 + T * wl.E * 4,
                 "d2h_bytes_per_step": T * wl.H * 2},

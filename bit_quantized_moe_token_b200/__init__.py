@@ -11,7 +11,8 @@ from ._binding import (MOE_OK, Layer, MoeError, fp8_quant_tokens, layer_struct, 
                        moe_w4a8_workspace_layout, w4a8_pack_weights,
                        moe_selftest_bounded_wait, Layer8, layer8_struct, w8a8_quant_weights,
                        moe_w8a8_workspace_bytes, moe_w8a8_workspace_layout, moe_w8a8_forward,
-                       moe_w8a8_forward_profiled)
+                       moe_w8a8_forward_profiled, moe_router_topk, moe_router_topk_workspace_bytes,
+                       moe_w4a8_forward_router, moe_w8a8_forward_router)
 from .layer import (alloc_workspace, forward, make_layer, make_layer_w8a8, pack_expert_weights,
                     quant_expert_weights_w8a8)
 
@@ -24,4 +25,5 @@ __all__ = ["MOE_OK", "Layer", "MoeError", "fp8_quant_tokens", "layer_struct", "l
            "make_layer", "pack_expert_weights", "moe_selftest_bounded_wait",
            "Layer8", "layer8_struct", "w8a8_quant_weights", "moe_w8a8_workspace_bytes",
            "moe_w8a8_workspace_layout", "moe_w8a8_forward", "moe_w8a8_forward_profiled",
-           "make_layer_w8a8", "quant_expert_weights_w8a8"]
+           "make_layer_w8a8", "quant_expert_weights_w8a8", "moe_router_topk",
+           "moe_router_topk_workspace_bytes", "moe_w4a8_forward_router", "moe_w8a8_forward_router"]

@@ -91,6 +91,11 @@ def lib() -> ctypes.CDLL:
         L.moe_w8a8_forward.argtypes = [ctypes.POINTER(_CLayer8), vp, vp, i64, i32, vp, vp, sz, vp]
         L.moe_w8a8_forward_profiled.argtypes = [ctypes.POINTER(_CLayer8), vp, vp, i64, i32, vp, vp,
                                                 sz, vp, vp, i32, vp]
+        L.moe_router_topk_workspace_bytes.argtypes = [i64, i32, i32]
+        L.moe_router_topk_workspace_bytes.restype = sz
+        L.moe_router_topk.argtypes = [vp, vp, i64, i32, i32, i32, vp, vp, vp, vp, sz, vp]
+        L.moe_w4a8_forward_router.argtypes = [ctypes.POINTER(_CLayer), vp, vp, i64, i32, vp, vp, sz, vp]
+        L.moe_w8a8_forward_router.argtypes = [ctypes.POINTER(_CLayer8), vp, vp, i64, i32, vp, vp, sz, vp]
         L.moe_last_device_status.argtypes = [vp]
         L.moe_selftest_bounded_wait.argtypes = [i64, vp]
         L.moe_status_string.argtypes = [i32]
@@ -159,6 +164,20 @@ def moe_router_logits(x, wr, logits, stream=None) -> None:
     E = wr.shape[0]
     _check(lib().moe_router_logits(_ptr(x), _ptr(wr), T, H, E, _ptr(logits), _stream(stream)),
            "moe_router_logits")
+
+
+def moe_router_topk_workspace_bytes(T: int, E: int, k: int) -> int:
+    return int(lib().moe_router_topk_workspace_bytes(T, E, k))
+
+
+def moe_router_topk(x, wr, k: int, logits, topk_ids, topk_w, ws, stream=None) -> None:
+    """x bf16 [T, H], router weight wr bf16 [E, H] -> logits fp32 [T, E], top-k ids int32 [T, k]
+    and gates fp32 [T, k] (router and top-k fused)."""
+    T, H = x.shape
+    E = wr.shape[0]
+    nbytes = ws.numel() * ws.element_size() if ws is not None else 0
+    _check(lib().moe_router_topk(_ptr(x), _ptr(wr), T, H, E, k, _ptr(logits), _ptr(topk_ids),
+                                 _ptr(topk_w), _ptr(ws), nbytes, _stream(stream)), "moe_router_topk")
 
 
 def moe_route_workspace_bytes(T: int, E: int, k: int) -> int:
@@ -351,3 +370,21 @@ def moe_w8a8_forward_profiled(layer: Layer8, x, logits, k: int, out, ws, events,
                                            _ptr(ws), nbytes, _stream(stream), arr, len(events),
                                            ctypes.byref(n)), "moe_w8a8_forward_profiled")
     return int(n.value)
+
+
+def moe_w4a8_forward_router(layer: Layer, x, wr, k: int, out, ws, stream=None) -> None:
+    """The W4A8 layer fed by the router weight wr bf16 [E, H] (logits computed inside)."""
+    T = x.shape[0]
+    s = layer.c_struct()
+    nbytes = ws.numel() * ws.element_size() if ws is not None else 0
+    _check(lib().moe_w4a8_forward_router(ctypes.byref(s), _ptr(x), _ptr(wr), T, k, _ptr(out), _ptr(ws),
+                                         nbytes, _stream(stream)), "moe_w4a8_forward_router")
+
+
+def moe_w8a8_forward_router(layer: Layer8, x, wr, k: int, out, ws, stream=None) -> None:
+    """The row-scaled FP8 layer fed by the router weight wr bf16 [E, H]."""
+    T = x.shape[0]
+    s = layer.c_struct()
+    nbytes = ws.numel() * ws.element_size() if ws is not None else 0
+    _check(lib().moe_w8a8_forward_router(ctypes.byref(s), _ptr(x), _ptr(wr), T, k, _ptr(out), _ptr(ws),
+                                         nbytes, _stream(stream)), "moe_w8a8_forward_router")

@@ -7,6 +7,7 @@
 #include "gemm_ws.cuh"
 #include "gemm_w8a8.cuh"
 #include "gemm_bf16_tc.cuh"
+#include "router.cuh"
 
 namespace moe {
 
@@ -69,8 +70,9 @@ __global__ void __launch_bounds__(256) k_combine(const float* __restrict__ Y,
 // S1 + S2 for one token per CTA: warp 0 ranks the token's router logits (top-k, softmax
 // gate) while all threads quantize its hidden state to FP8 (amax, scale, codes), written once
 // per token; the grouped GEMM gathers the rows it needs by token index.  Same arithmetic as
-// k_topk and k_quant_tokens.
-template <int EPL>
+// k_topk and k_quant_tokens.  kTopk = false: quantization only (the routing came from the
+// fused router front).
+template <int EPL, bool kTopk = true>
 __global__ void __launch_bounds__(256) k_quant_topk(const float* __restrict__ logits,
                                                     const uint16_t* __restrict__ x, int E, int k,
                                                     int H, int32_t* __restrict__ ids,
@@ -80,31 +82,19 @@ __global__ void __launch_bounds__(256) k_quant_topk(const float* __restrict__ lo
                                                     float* __restrict__ qsum) {
     __shared__ float red[32];
     const int64_t t = blockIdx.x;
-    if (threadIdx.x < 32) topk_row<EPL>(logits + t * E, E, k, ids + t * k, gates + t * k, threadIdx.x);
-    const uint4* row = reinterpret_cast<const uint4*>(x + t * H);
-    const int chunks = H >> 3;
-    float a = 0.0f;
-    for (int c = threadIdx.x; c < chunks; c += blockDim.x) a = fmaxf(a, amax8(__ldg(row + c)));
-    a = block_max(a, red);
-    const float s = __fdiv_rn(a, kFp8Max);
-    // codes, and per K-group of 128 (16 chunks = one half-warp) the sum of the decoded values
-    const int G = H / kGroup;
-    for (int base = 0; base < chunks; base += blockDim.x) {
-        const int c = base + threadIdx.x;
-        const bool live = c < chunks;
-        const uint2 codes = live ? quant8(__ldg(row + c), s) : make_uint2(0u, 0u);
-        if (live) reinterpret_cast<uint2*>(xq + t * H)[c] = codes;
-        const float gs = halfwarp_sum(e4m3x8_sum(codes));
-        if (qsum && live && (threadIdx.x & 15) == 0) qsum[t * G + c / 16] = gs;
-    }
-    if (threadIdx.x == 0) s_x[t] = s;
+    if (kTopk && threadIdx.x < 32) topk_row<EPL>(logits + t * E, E, k, ids + t * k, gates + t * k, threadIdx.x);
+    quant_token_cta(x, t, H, xq, s_x, qsum, red);
 }
 
 inline int launch_quant_topk(const float* logits, const uint16_t* x, int64_t T, int E, int k, int H,
                              int32_t* ids, float* gates, uint8_t* xq, float* s_x, float* qsum,
-                             cudaStream_t stream) {
+                             cudaStream_t stream, bool topk = true) {
     const int epl = (E + 31) / 32;
     const unsigned grid = static_cast<unsigned>(T);
+    if (!topk) {
+        k_quant_topk<1, false><<<grid, 256, 0, stream>>>(logits, x, E, k, H, ids, gates, xq, s_x, qsum);
+        return launch_status();
+    }
 #define MOE_QT(N) k_quant_topk<N><<<grid, 256, 0, stream>>>(logits, x, E, k, H, ids, gates, xq, s_x, qsum)
     if (epl <= 1) MOE_QT(1);
     else if (epl <= 2) MOE_QT(2);
@@ -123,6 +113,7 @@ struct WsPlan {
     size_t topk_ids, topk_w, offsets, sorted, rop, route_ws;
     size_t xq, s_x, x_sorted, s_x_sorted, h, zero, hq, s_h, y;
     size_t qs_x, qs_h;   // per (activation row, K-group) sums of the FP8 values (narrow tiles)
+    size_t logits, rcnt; // router logits [T, E] and the fused router's counters (router entry points)
     int64_t n_zero;   // u32 words at `zero`: max|h| per row [P], row counters [P], token counters
     size_t sh_a, sh_y;
     size_t total;
@@ -155,6 +146,8 @@ inline WsPlan plan_workspace(const moe_w4a8_layer& L, int64_t T, int k) {
     p.y = take((size_t)P * L.H * 4);
     p.qs_x = take((size_t)T * (L.H / 128) * 4);
     p.qs_h = take((size_t)P * (L.N / 128) * 4);
+    p.logits = take((size_t)T * L.E * 4);
+    p.rcnt = take((size_t)router_counter_words(T) * 4);
     if (L.n_shared > 0) {
         p.sh_a = take((size_t)T * L.n_shared * L.shared_N * 2);
         p.sh_y = take((size_t)T * L.H * 4);
@@ -225,10 +218,13 @@ struct StageMarks {
     }
 };
 
-// `layer` gives the shapes and the shared experts; `xs` the routed experts' weights.
+// `layer` gives the shapes and the shared experts; `xs` the routed experts' weights.  With
+// `router_w` non-null the router logits are computed from it (into the workspace) and
+// `router_logits` is ignored.
 int forward_impl(const moe_w4a8_layer* layer, const ExpertSet& xs, const uint16_t* x_bf16,
                  const float* router_logits, int64_t T, int k, uint16_t* out_bf16, void* ws,
-                 size_t ws_bytes, cudaStream_t stream, StageMarks& sm);
+                 size_t ws_bytes, cudaStream_t stream, StageMarks& sm,
+                 const uint16_t* router_w = nullptr);
 
 }  // namespace moe
 
@@ -257,15 +253,16 @@ extern "C" int moe_w4a8_forward_profiled(const moe_w4a8_layer* layer, const uint
 
 int moe::forward_impl(const moe_w4a8_layer* layer, const ExpertSet& xw, const uint16_t* x_bf16,
                       const float* router_logits, int64_t T, int k, uint16_t* out_bf16, void* ws,
-                      size_t ws_bytes, cudaStream_t stream, StageMarks& sm) {
+                      size_t ws_bytes, cudaStream_t stream, StageMarks& sm, const uint16_t* router_w) {
     using namespace moe;
     int st = layer_args_ok(layer, T, k);
     if (st != MOE_OK) return st;
     const moe_w4a8_layer& L = *layer;
     if (T == 0) return MOE_OK;
-    if (!x_bf16 || !router_logits || !out_bf16 || !xw.gate || !xw.up || !xw.down || !xw.gate_s ||
-        !xw.up_s || !xw.down_s)
+    if (!x_bf16 || (!router_logits && !router_w) || !out_bf16 || !xw.gate || !xw.up || !xw.down ||
+        !xw.gate_s || !xw.up_s || !xw.down_s)
         return MOE_ERR_INVALID_ARG;
+    if (router_w && !aligned(router_w, 16)) return MOE_ERR_MISALIGNED;
     if (L.n_shared > 0 && (!L.sh_gate || !L.sh_up || !L.sh_down)) return MOE_ERR_INVALID_ARG;
     if (L.n_shared > 0 && (!aligned(L.sh_gate, 16) || !aligned(L.sh_up, 16) || !aligned(L.sh_down, 16)))
         return MOE_ERR_MISALIGNED;
@@ -303,12 +300,44 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const ExpertSet& xw, const ui
     // narrow token tiles (decode): codes written once per token and gathered by the GEMM, fused
     // requantization and combine; wide tiles (prefill): codes copied to expert-sorted rows.
     const bool fused = ws_narrow(tc_tile_rows(P, L.E));
+    float* qsum_x = xw.w8 ? nullptr : qs_x;       // group sums serve the unsigned widening only
 
     sm.mark(0, stream);
-    if (fused) {
+    if (router_w) {
+        // router logits + S2 (+ S1 at decode) from the router weight
+        float* lg = (float*)at(p.logits);
+        unsigned* rc = (unsigned*)at(p.rcnt);
+        if (cudaMemsetAsync(rc, 0, router_counter_words(T) * 4, stream) != cudaSuccess) return MOE_ERR_CUDA;
+        const bool front_quant = fused && T <= 16;
+        int nl = 0;
+        if ((st = launch_router_topk(x_bf16, router_w, T, L.H, L.E, k, lg, ids, gates, rc,
+                                     front_quant ? xq : nullptr, sx, qsum_x, stream, &nl)))
+            return st;
+        sm.launches += nl;
+        sm.mark(1, stream);
+        if (fused) {
+            if (!front_quant) {
+                if ((st = launch_quant_topk(nullptr, x_bf16, T, L.E, k, L.H, ids, gates, xq, sx, qsum_x,
+                                            stream, false)))
+                    return st;
+                sm.launches += 1;
+            }
+            if ((st = launch_permute(ids, T, L.E, k, offsets, sorted, rop, (int32_t*)at(p.route_ws), stream,
+                                     zero, p.n_zero)))
+                return st;
+            sm.launches += (P <= kSinglePassMaxP ? 1 : 3);
+        } else {
+            if ((st = launch_permute(ids, T, L.E, k, offsets, sorted, rop, (int32_t*)at(p.route_ws), stream,
+                                     zero, p.n_zero)))
+                return st;
+            if ((st = launch_quant_tokens(x_bf16, T, L.H, xs, sxs, rop, k, stream, xq, sx))) return st;
+            sm.launches += (P <= kSinglePassMaxP ? 1 : 3) + 1;
+        }
+        sm.mark(2, stream);
+    } else if (fused) {
         // S1 + S2: per-token FP8 codes and top-k
-        if ((st = launch_quant_topk(router_logits, x_bf16, T, L.E, k, L.H, ids, gates, xq, sx,
-                                    xw.w8 ? nullptr : qs_x, stream)))
+        if ((st = launch_quant_topk(router_logits, x_bf16, T, L.E, k, L.H, ids, gates, xq, sx, qsum_x,
+                                    stream)))
             return st;
         sm.launches += 1;
         sm.mark(1, stream);
@@ -445,4 +474,29 @@ extern "C" int moe_w8a8_forward_profiled(const moe_w8a8_layer* layer, const uint
                                      out_bf16, ws, ws_bytes, stream, sm);
     if (n_launches) *n_launches = sm.launches;
     return st;
+}
+
+// ---- the layer from the router weight ----------------------------------------------------------
+
+extern "C" int moe_w4a8_forward_router(const moe_w4a8_layer* layer, const uint16_t* x_bf16,
+                                       const uint16_t* router_w_bf16, int64_t T, int k,
+                                       uint16_t* out_bf16, void* ws, size_t ws_bytes,
+                                       moe_stream_t stream) {
+    if (!layer) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && !router_w_bf16) return MOE_ERR_INVALID_ARG;
+    moe::StageMarks sm{nullptr, 0, 0};
+    return moe::forward_impl(layer, moe::experts_of(*layer), x_bf16, nullptr, T, k, out_bf16, ws, ws_bytes,
+                             stream, sm, router_w_bf16);
+}
+
+extern "C" int moe_w8a8_forward_router(const moe_w8a8_layer* layer, const uint16_t* x_bf16,
+                                       const uint16_t* router_w_bf16, int64_t T, int k,
+                                       uint16_t* out_bf16, void* ws, size_t ws_bytes,
+                                       moe_stream_t stream) {
+    if (!layer) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && !router_w_bf16) return MOE_ERR_INVALID_ARG;
+    moe::StageMarks sm{nullptr, 0, 0};
+    const moe_w4a8_layer s = moe::shape_of(*layer);
+    return moe::forward_impl(&s, moe::experts_of(*layer), x_bf16, nullptr, T, k, out_bf16, ws, ws_bytes,
+                             stream, sm, router_w_bf16);
 }

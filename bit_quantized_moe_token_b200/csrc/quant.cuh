@@ -78,6 +78,30 @@ __global__ void __launch_bounds__(256) k_quant_tokens(const uint16_t* __restrict
     }
 }
 
+// S1 for token t by the whole CTA: amax, scale = amax / 448, the FP8 codes written once per
+// token, and (qsum non-null) per K-group of 128 (16 chunks = one half-warp) the sum of the
+// decoded codes.  Same arithmetic as k_quant_tokens.
+__device__ __forceinline__ void quant_token_cta(const uint16_t* __restrict__ x, int64_t t, int H,
+                                                uint8_t* __restrict__ xq, float* __restrict__ s_x,
+                                                float* __restrict__ qsum, float* red) {
+    const uint4* row = reinterpret_cast<const uint4*>(x + t * H);
+    const int chunks = H >> 3;
+    float a = 0.0f;
+    for (int c = threadIdx.x; c < chunks; c += blockDim.x) a = fmaxf(a, amax8(__ldg(row + c)));
+    a = block_max(a, red);
+    const float s = __fdiv_rn(a, kFp8Max);
+    const int G = H / kGroup;
+    for (int base = 0; base < chunks; base += blockDim.x) {
+        const int c = base + threadIdx.x;
+        const bool live = c < chunks;
+        const uint2 codes = live ? quant8(__ldg(row + c), s) : make_uint2(0u, 0u);
+        if (live) reinterpret_cast<uint2*>(xq + t * H)[c] = codes;
+        const float gs = halfwarp_sum(e4m3x8_sum(codes));
+        if (qsum && live && (threadIdx.x & 15) == 0) qsum[t * G + c / 16] = gs;
+    }
+    if (threadIdx.x == 0) s_x[t] = s;
+}
+
 inline int launch_quant_tokens(const uint16_t* x, int64_t T, int64_t H, uint8_t* q, float* s,
                                const int32_t* row_of_pair, int k, cudaStream_t stream,
                                uint8_t* q_tok = nullptr, float* s_tok = nullptr) {

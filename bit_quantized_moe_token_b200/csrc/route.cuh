@@ -15,7 +15,8 @@ constexpr int kSinglePassMaxP = 4096; // above this the permutation runs on one 
 // ------------------------------------------------------------------------------------------
 // top-k: one warp per token; lane l holds experts l, l+32, ..., (EPL slots)
 // ------------------------------------------------------------------------------------------
-template <int EPL>
+// kCoherent: read the logits through L2 (they were written by other CTAs of the same kernel).
+template <int EPL, bool kCoherent = false>
 __device__ __forceinline__ void topk_row(const float* __restrict__ l, int E, int k,
                                          int32_t* __restrict__ ids, float* __restrict__ gates,
                                          int lane) {
@@ -24,7 +25,7 @@ __device__ __forceinline__ void topk_row(const float* __restrict__ l, int E, int
 #pragma unroll
     for (int s = 0; s < EPL; ++s) {
         const int e = lane + 32 * s;
-        float x = (e < E) ? __ldg(l + e) : -INFINITY;
+        float x = (e < E) ? (kCoherent ? __ldcg(l + e) : __ldg(l + e)) : -INFINITY;
         v[s] = isnan(x) ? -INFINITY : x;
         if (e >= E) taken |= 1u << s;
     }

@@ -104,6 +104,27 @@ int moe_router_logits(const uint16_t* x_bf16, const uint16_t* wr_bf16, int64_t T
                       float* logits, moe_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------
+ * Router logits fused with S2 (top-k and softmax gate).
+ *
+ * logits as moe_router_logits, and from them topk_ids / topk_w exactly as moe_route_topk's S2
+ * (ranking by logit descending then index ascending, softmax over the selected logits).  For
+ * T < 256 (or E not a multiple of 128) the top-k runs inside the router kernel: the CTA that
+ * completes a block of tokens ranks those tokens' logits, so routing is one launch; for larger
+ * T the tensor-core router is followed by the top-k kernel.
+ *
+ *   x_bf16, wr_bf16, T, H, E   as moe_router_logits;  k in [1, min(E, 8)]
+ *   logits     [T, E] fp32 output (the logits the top-k ranked)
+ *   topk_ids   [T, k] int32 out      topk_w [T, k] fp32 out
+ *   ws, ws_bytes   device scratch of at least moe_router_topk_workspace_bytes(T, E, k) bytes,
+ *                  256-byte aligned (completion counters; contents on entry are ignored)
+ * T == 0 is a no-op.
+ * --------------------------------------------------------------------------------------- */
+size_t moe_router_topk_workspace_bytes(int64_t T, int E, int k);
+int moe_router_topk(const uint16_t* x_bf16, const uint16_t* wr_bf16, int64_t T, int H, int E, int k,
+                    float* logits, int32_t* topk_ids, float* topk_w, void* ws, size_t ws_bytes,
+                    moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------
  * S2 + S3. Top-k routing and the stable token permutation.
  *
  * Top-k of each row of the router logits (the Inkling-512k card's opening paragraph: 256
@@ -250,6 +271,19 @@ int moe_w8a8_forward_profiled(const moe_w8a8_layer* layer, const uint16_t* x_bf1
                               const float* router_logits, int64_t T, int k, uint16_t* out_bf16,
                               void* ws, size_t ws_bytes, moe_stream_t stream,
                               void* const* events, int n_events, int* n_launches);
+
+/* The layer fed by the router weight instead of precomputed logits: the router logits
+ * (moe_router_logits' definition, written into the workspace), then the layer of
+ * moe_w4a8_forward / moe_w8a8_forward on them.  At decode sizes (T <= 16) the router, the
+ * per-token FP8 quantization (S1) and the top-k (S2) are one kernel.
+ *   wr_bf16   [E, H] bf16 router weight, 16-byte aligned
+ * Everything else as moe_w4a8_forward / moe_w8a8_forward (same workspace size). */
+int moe_w4a8_forward_router(const moe_w4a8_layer* layer, const uint16_t* x_bf16,
+                            const uint16_t* wr_bf16, int64_t T, int k, uint16_t* out_bf16,
+                            void* ws, size_t ws_bytes, moe_stream_t stream);
+int moe_w8a8_forward_router(const moe_w8a8_layer* layer, const uint16_t* x_bf16,
+                            const uint16_t* wr_bf16, int64_t T, int k, uint16_t* out_bf16,
+                            void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /* Waits for `stream`, then returns and clears the library's sticky device-status word for
  * the current device: MOE_OK, or MOE_ERR_TIMEOUT when a bounded device-side wait gave up

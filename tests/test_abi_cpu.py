@@ -28,7 +28,8 @@ def test_header_declares_the_boundary():
     names = _declared_functions()
     for n in ("w4a8_pack_weights", "fp8_quant_tokens", "moe_route_topk", "moe_w4a8_forward",
               "moe_router_logits", "w8a8_quant_weights", "moe_w8a8_forward",
-              "moe_w8a8_workspace_bytes", "moe_w8a8_forward_profiled",
+              "moe_w8a8_workspace_bytes", "moe_w8a8_forward_profiled", "moe_router_topk",
+              "moe_router_topk_workspace_bytes", "moe_w4a8_forward_router", "moe_w8a8_forward_router",
               "moe_w4a8_workspace_bytes", "moe_last_device_status", "moe_status_string"):
         assert n in names
 
@@ -134,6 +135,26 @@ def test_forward_rejects_bad_args():
     assert L.moe_w4a8_forward(ctypes.byref(full), p, p, 4, 0, p, p, need, None) == -1
     assert L.moe_w4a8_forward(ctypes.byref(full), p, p, 0, 2, p, p, need, None) == 0
     assert L.moe_w4a8_forward(None, p, p, 4, 2, p, p, need, None) == -1
+
+
+def test_router_topk_rejects_bad_args():
+    L = _L()
+    p = ctypes.c_void_p(4096)
+    ws = moe.moe_router_topk_workspace_bytes(8, 256, 6)
+    assert ws >= 256 and ws % 256 == 0
+    assert moe.moe_router_topk_workspace_bytes(8, 256, 9) == 0          # k > 8
+    assert L.moe_router_topk(p, p, 8, 100, 256, 6, p, p, p, p, ws, None) == -2     # H % 8
+    assert L.moe_router_topk(p, p, 8, 256, 4, 6, p, p, p, p, ws, None) == -2       # k > E
+    assert L.moe_router_topk(p, p, 8, 256, 256, 6, p, p, p, p, ws - 1, None) == -4
+    assert L.moe_router_topk(p, p, 8, 256, 256, 6, None, p, p, p, ws, None) == -1
+    assert L.moe_router_topk(p, p, 8, 256, 256, 6, p, p, p, ctypes.c_void_p(4096 + 64), ws, None) == -3
+    assert L.moe_router_topk(p, p, 0, 256, 256, 6, p, p, p, p, ws, None) == 0
+    full = moe._binding._CLayer(8, 256, 128, 128, p, p, p, p, p, p, 0, 0, None, None, None)
+    need = moe.moe_w4a8_workspace_bytes(full, 4, 2)
+    assert L.moe_w4a8_forward_router(ctypes.byref(full), p, None, 4, 2, p, p, need, None) == -1
+    assert L.moe_w4a8_forward_router(ctypes.byref(full), p, ctypes.c_void_p(4098), 4, 2, p, p, need,
+                                     None) == -3
+    assert L.moe_w4a8_forward_router(ctypes.byref(full), p, p, 4, 2, p, p, need - 1, None) == -4
 
 
 def test_w8a8_rejects_bad_args():

@@ -287,6 +287,65 @@ def test_router_logits_vs_oracle(T, E, H):
     assert np.array_equal(ids_got[clear], ids_ref[clear])
 
 
+@pytest.mark.parametrize("T,E,H,k", [(1, 256, 4096, 6), (8, 256, 4096, 6), (16, 64, 512, 8),
+                                     (37, 20, 1000, 3), (300, 256, 1024, 6), (2048, 256, 4096, 6),
+                                     (70, 1000, 256, 2)])
+def test_router_topk_fused(T, E, H, k):
+    """Router + top-k in one call: the logits equal moe_router_logits' bit for bit (same kernels,
+    same summation order), and the ids / gates are the oracle's top-k of those logits (ids exact;
+    gates to the last bits of expf)."""
+    x = synth.normal_bf16(7, 880 + T, T * H).reshape(T, H)
+    wr = synth.normal_bf16(7, 881 + E, E * H, 1.0 / np.sqrt(H)).reshape(E, H)
+    xd, wd = to_dev_bf16(x), to_dev_bf16(wr)
+    lg = torch.empty(T, E, dtype=torch.float32, device="cuda")
+    ids = torch.empty(T, k, dtype=torch.int32, device="cuda")
+    gw = torch.empty(T, k, dtype=torch.float32, device="cuda")
+    ws = torch.full((moe.moe_router_topk_workspace_bytes(T, E, k),), 0xAB, dtype=torch.uint8, device="cuda")
+    for _ in range(2):                                 # the counters are reused by the second call
+        moe.moe_router_topk(xd, wd, k, lg, ids, gw, ws)
+    lg2 = torch.empty(T, E, dtype=torch.float32, device="cuda")
+    moe.moe_router_logits(xd, wd, lg2)
+    torch.cuda.synchronize()
+    assert moe.moe_last_device_status() == 0
+    g = lg.cpu().numpy()
+    assert np.array_equal(g.view(np.uint32), lg2.cpu().numpy().view(np.uint32))
+    ids_ref, gates_ref = oracle.route_topk(g, k)
+    assert np.array_equal(ids.cpu().numpy(), ids_ref)
+    np.testing.assert_allclose(gw.cpu().numpy(), gates_ref, rtol=1e-6)
+    ref = oracle.router_logits(x, wr).astype(np.float64)
+    bound = 2 * H * 2.0 ** -24 * (np.abs(bf16_to_f32(x).astype(np.float64)) @
+                                  np.abs(bf16_to_f32(wr).astype(np.float64)).T) + 1e-30
+    assert np.all(np.abs(g.astype(np.float64) - ref) <= bound)
+
+
+@pytest.mark.parametrize("w8", [False, True])
+@pytest.mark.parametrize("E,H,N,k,T", [(16, 256, 128, 2, 8), (16, 256, 128, 2, 40),
+                                       (16, 256, 128, 2, 300), (128, 256, 128, 2, 300)])
+def test_forward_router_matches_logits_path(w8, E, H, N, k, T):
+    """The layer fed by the router weight equals, bit for bit, the layer fed by the logits that
+    moe_router_logits computes (decode front: router + quantization + top-k in one kernel;
+    16 < T: fused router + top-k, then quantization; E = 128, T = 300: tensor-core router)."""
+    hl, dl = (_host_layer_and_dev_w8a8 if w8 else _host_layer_and_dev)(E, H, N, seed=30 + E + T)
+    x = synth.normal_bf16(8, 870 + T, T * H).reshape(T, H)
+    wr = synth.normal_bf16(8, 871 + E, E * H, 1.0 / np.sqrt(H)).reshape(E, H)
+    xd, wd = to_dev_bf16(x), to_dev_bf16(wr)
+    lg = torch.empty(T, E, dtype=torch.float32, device="cuda")
+    moe.moe_router_logits(xd, wd, lg)
+    ws_a, ws_b = moe.alloc_workspace(dl, T, k), moe.alloc_workspace(dl, T, k)
+    out_a = moe.forward(dl, xd, lg, k, ws=ws_a)
+    out_b = torch.empty_like(out_a)
+    (moe.moe_w8a8_forward_router if w8 else moe.moe_w4a8_forward_router)(dl, xd, wd, k, out_b, ws_b)
+    torch.cuda.synchronize()
+    assert moe.moe_last_device_status() == 0
+    assert np.array_equal(bits(out_a), bits(out_b))
+    va, vb = ws_views(dl, ws_a, T, k), ws_views(dl, ws_b, T, k)
+    for key in ("ids", "offsets", "sorted_pairs", "xq", "s_x", "hq", "s_h"):
+        assert np.array_equal(va[key], vb[key]), key
+    # and the routing is the oracle's top-k of those logits
+    ids_ref, _ = oracle.route_topk(lg.cpu().numpy(), k)
+    assert np.array_equal(vb["ids"], ids_ref)
+
+
 def test_router_logits_zero_tokens():
     wr = torch.zeros(8, 64, dtype=torch.bfloat16, device="cuda")
     moe.moe_router_logits(torch.empty(0, 64, dtype=torch.bfloat16, device="cuda"), wr,
