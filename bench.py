@@ -111,8 +111,8 @@ def is_prefill(wl):
     return wl.T >= 1024
 
 
-KERNEL_SOURCES = {"w4a8": ("gemm_ws.cuh", "tc_ptx.cuh", "tc_tiles.cuh", "common.cuh"),
-                  "w8a8": ("gemm_w8a8.cuh", "gemm_ws.cuh", "tc_ptx.cuh", "tc_tiles.cuh", "common.cuh")}
+KERNEL_SOURCES = {"w4a8": ("gemm_ws.cuh", "tc_pipe.cuh", "tc_ptx.cuh", "tc_tiles.cuh", "common.cuh"),
+                  "w8a8": ("gemm_w8a8.cuh", "tc_pipe.cuh", "tc_ptx.cuh", "tc_tiles.cuh", "common.cuh")}
 PROFILE_FOR = {("w4a8", "decode_t8"): "gemm_w4a8_ws_decode_t8.md",
                ("w4a8", "prefill_t2048_zipf"): "gemm_w4a8_ws_prefill_t2048.md",
                ("w8a8", "decode_t8"): "gemm_w8a8_decode_t8.md",

@@ -17,7 +17,7 @@
 #include <cuda.h>
 #include "common.cuh"
 #include "tc_ptx.cuh"
-#include "gemm_ws.cuh"
+#include "tc_pipe.cuh"
 
 namespace moe {
 

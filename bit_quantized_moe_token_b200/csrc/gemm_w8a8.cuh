@@ -30,7 +30,7 @@
 #include "common.cuh"
 #include "tc_ptx.cuh"
 #include "tc_tiles.cuh"
-#include "gemm_ws.cuh"
+#include "tc_pipe.cuh"
 
 namespace moe {
 

@@ -34,6 +34,7 @@
 #include "common.cuh"
 #include "tc_ptx.cuh"
 #include "tc_tiles.cuh"
+#include "tc_pipe.cuh"
 
 namespace moe {
 
@@ -67,61 +68,6 @@ struct WsGemmArgs {
     float* qsum_out;        // SwiGLU fused: the same sums of the requantized rows [P, R0/128]
 };
 
-namespace ws {
-
-// Four rows (r0..r3) of a 2-D tensor, `box_w` wide from column x, into four consecutive
-// box rows at dst (the tensor map's box is one row high).
-__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, int x, int r0, int r1,
-                                            int r2, int r3, uint64_t* bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];"
-        ::"r"(tc::smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(tc::smem_u32(bar)),
-          "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
-        : "memory");
-}
-
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
-                                            uint64_t* bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4}], [%2];"
-        ::"r"(tc::smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(tc::smem_u32(bar)),
-          "r"(x), "r"(y)
-        : "memory");
-}
-
-__device__ __forceinline__ void prefetch_map(const CUtensorMap* map) {
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
-}
-
-// Named barrier 1 among the promotion / epilogue warps only.
-template <int kThreads = 128>
-__device__ __forceinline__ void named_sync_math() {
-    asm volatile("bar.sync 1, %0;" ::"n"(kThreads) : "memory");
-}
-
-
-// Slot and phase parity of a ring of N stages, advanced once per stage (no division).
-template <int N>
-struct Ring {
-    int idx = 0;
-    uint32_t phase = 0;
-    __device__ __forceinline__ void next() {
-        if (++idx == N) { idx = 0; phase ^= 1u; }
-    }
-};
-
-// Bounded wait that gives up at once after an abort.
-__device__ __forceinline__ bool wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
-    if (tc::mbar_try_wait(bar, parity)) return true;      // completed phase: no flag read
-    if (*abort) return false;
-    if (tc::mbar_wait(bar, parity)) return true;
-    *abort = 1;
-    return false;
-}
-
-}  // namespace ws
 
 template <int BN, bool kUnsigned>
 struct WsCfg {
@@ -183,35 +129,6 @@ struct WsCfg {
     static constexpr int kLd = kNP > 8 ? 16 : (kCPW < 32 ? kCPW : 32);
     static constexpr int kThreads = 32 * (kNW + kNP + 2);
 };
-
-// Fused decode epilogues.  Requantization (S5) of a row needs max|h| over all of its M tiles,
-// and the combine (S7) of a token needs all k routed rows: the CTA that finishes the last
-// contribution (counted with a device-scope atomic after a fence) does that work, reading the
-// other CTAs' outputs through L2.  The result does not depend on which CTA finishes last.
-__device__ __forceinline__ void requant_row(const float* __restrict__ h, int N, unsigned amax_bits,
-                                            uint8_t* __restrict__ hq, float* __restrict__ s_h, int tid,
-                                            int nthreads, float* __restrict__ qs_row) {
-    const float s = __fdiv_rn(__uint_as_float(amax_bits), kFp8Max);
-    for (int base = 0; base < (N >> 3); base += nthreads) {
-        const int c = base + tid;
-        const bool live = c < (N >> 3);
-        uint2 codes = make_uint2(0u, 0u);
-        if (live && s != 0.0f) {
-            const float4 a = __ldcg(reinterpret_cast<const float4*>(h) + 2 * c);
-            const float4 b = __ldcg(reinterpret_cast<const float4*>(h) + 2 * c + 1);
-            codes.x = static_cast<uint32_t>(f32x2_to_e4m3x2(__fdiv_rn(a.x, s), __fdiv_rn(a.y, s))) |
-                      (static_cast<uint32_t>(f32x2_to_e4m3x2(__fdiv_rn(a.z, s), __fdiv_rn(a.w, s))) << 16);
-            codes.y = static_cast<uint32_t>(f32x2_to_e4m3x2(__fdiv_rn(b.x, s), __fdiv_rn(b.y, s))) |
-                      (static_cast<uint32_t>(f32x2_to_e4m3x2(__fdiv_rn(b.z, s), __fdiv_rn(b.w, s))) << 16);
-        }
-        if (live) reinterpret_cast<uint2*>(hq)[c] = codes;
-        if (qs_row) {   // sums of the decoded codes per K-group of 128 (16 chunks = one half-warp)
-            const float gs = halfwarp_sum(e4m3x8_sum(codes));
-            if (live && (tid & 15) == 0) qs_row[c / 16] = gs;
-        }
-    }
-    if (tid == 0) *s_h = s;
-}
 
 template <int BN, bool kUnsigned, bool kSwiGLU, bool kFused, bool kGather>
 __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUnsigned>::kCtasPerSm)
@@ -343,7 +260,7 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
             ws::Ring<C::kS> rs;
             ws::Ring<C::kNTS> rt;
             ws::Ring<C::kRB> rb;
-            int last_b = -1;
+            uint64_t* last_bar = nullptr;                  // the barrier of the last commit
             uint32_t last_bp = 0;
             for (int64_t tile = blockIdx.x; tile < n_tiles && !*abort; tile += gridDim.x) {
                 for (int st = 0; st < nst; ++st) {
@@ -361,10 +278,16 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
                             tc::mma_e4m3_ta(d, a_col + kk * 8, bd + 2 * kk, idesc, kk > 0 ? 1u : 0u);
                     }
                     tc::mma_commit(&t_full[rt.idx]);
-                    tc::mma_commit(&s_free[rs.idx]);
-                    if (C::kSplitB) tc::mma_commit(&b_empty[rb.idx]);
-                    last_b = rb.idx;
-                    last_bp = rb.phase;
+                    if (C::kSplitB) {
+                        // one commit per stage: the widening warps free the A stage and the
+                        // activation slot from the partial's completion (see below)
+                        last_bar = &t_full[rt.idx];
+                        last_bp = rt.phase;
+                    } else {
+                        tc::mma_commit(&s_free[rs.idx]);   // = b_empty: A stage + activation slot
+                        last_bar = &s_free[rs.idx];
+                        last_bp = rs.phase;
+                    }
                     rs.next();
                     rt.next();
                     rb.next();
@@ -372,7 +295,7 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
             }
             // the commits complete in order: once the last one has arrived, no tensor-core
             // arrive on this CTA's barriers is still pending
-            if (last_b >= 0) ws::wait(&b_empty[last_b], last_bp, abort);
+            if (last_bar) ws::wait(last_bar, last_bp, abort);
         }
     } else if (warp < C::kNW) {
         // ------------------------------------------------------------ widening warps
@@ -389,8 +312,9 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
         const uint32_t t_dst = tmem + (static_cast<uint32_t>(quad * 32) << 16) + C::kColA + part * 8 * kChunks;
         ws::Ring<C::kRW> rw;
         ws::Ring<C::kS> ra;
+        uint32_t g = 0;                                    // stages so far, in the MMA's order
         for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
-            for (int st = 0; st < nst; ++st, rw.next(), ra.next()) {
+            for (int st = 0; st < nst; ++st, rw.next(), ra.next(), ++g) {
                 const int ws_ = rw.idx, as = ra.idx;
                 ws::wait(&w_full[ws_], rw.phase, abort);
                 const uint8_t* raw = wring + ws_ * C::kRaw + row * C::kRowB;
@@ -403,7 +327,20 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
                 tc::fence_proxy_async_smem();              // order these reads before the next TMA write
                 __syncwarp();                              // this warp's reads of the slot are done
                 if (lane == 0) tc::mbar_arrive(&w_empty[ws_]);
-                ws::wait(&s_free[as], ra.phase ^ 1u, abort);
+                if constexpr (C::kSplitB) {
+                    // A stage `as` was last read by the MMAs of stage g - kS, whose completion is
+                    // the commit on that stage's partial buffer.  kNTS >= kS, so that buffer's
+                    // barrier cannot have completed a later phase yet and its parity is unambiguous.
+                    // The same completion frees the activation slot of stage g - kS.
+                    static_assert(C::kNTS >= C::kS, "partial ring shorter than the A ring");
+                    if (g >= static_cast<uint32_t>(C::kS)) {
+                        const uint32_t gp = g - C::kS;
+                        ws::wait(&t_full[gp % C::kNTS], (gp / C::kNTS) & 1u, abort);
+                        if (warp == 0 && lane == 0) tc::mbar_arrive(&b_empty[gp % C::kRB]);
+                    }
+                } else {
+                    ws::wait(&s_free[as], ra.phase ^ 1u, abort);
+                }
                 tc::tc_fence_after();
 #pragma unroll
                 for (int h = 0; h < C::kGS; ++h) {
@@ -630,38 +567,6 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
 }
 
 // ---- host side --------------------------------------------------------------------------------
-
-using PFN_encodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                     const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                     const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                     CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-inline PFN_encodeTiled encode_fn() {
-    static PFN_encodeTiled fn = nullptr;
-    if (!fn) {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
-            q != cudaDriverEntryPointSuccess)
-            return nullptr;
-        fn = reinterpret_cast<PFN_encodeTiled>(p);
-    }
-    return fn;
-}
-
-// 2D byte tensor [rows, row_bytes] (row-major) with a box of box_rows x box_bytes.
-inline bool make_map_u8(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t rows,
-                        uint32_t box_bytes, uint32_t box_rows, CUtensorMapSwizzle swizzle) {
-    PFN_encodeTiled fn = encode_fn();
-    if (!fn) return false;
-    const cuuint64_t dims[2] = {row_bytes, rows};
-    const cuuint64_t strides[1] = {row_bytes};
-    const cuuint32_t box[2] = {box_bytes, box_rows};
-    const cuuint32_t estr[2] = {1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
 
 template <int BN, bool kUnsigned, bool kSwiGLU, bool kFused, bool kGather>
 int launch_gemm_ws_inst(const WsGemmArgs& a, const void* act, const void* w0, const void* w1,

@@ -1,0 +1,130 @@
+// tc_pipe.cuh — pieces shared by the warp-specialised tcgen05 GEMMs (gemm_ws.cuh, gemm_w8a8.cuh,
+// gemm_bf16_tc.cuh): TMA issue helpers, ring counters, the bounded barrier wait, the fused
+// requantization of one row, and the host-side tensor-map encoders.
+#pragma once
+#include <cuda.h>
+#include "common.cuh"
+#include "tc_ptx.cuh"
+
+namespace moe {
+
+namespace ws {
+
+// Four rows (r0..r3) of a 2-D tensor, `box_w` wide from column x, into four consecutive
+// box rows at dst (the tensor map's box is one row high).
+__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, int x, int r0, int r1,
+                                            int r2, int r3, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];"
+        ::"r"(tc::smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(tc::smem_u32(bar)),
+          "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
+                                            uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];"
+        ::"r"(tc::smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(tc::smem_u32(bar)),
+          "r"(x), "r"(y)
+        : "memory");
+}
+
+__device__ __forceinline__ void prefetch_map(const CUtensorMap* map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// Named barrier 1 among the promotion / epilogue warps only.
+template <int kThreads = 128>
+__device__ __forceinline__ void named_sync_math() {
+    asm volatile("bar.sync 1, %0;" ::"n"(kThreads) : "memory");
+}
+
+
+// Slot and phase parity of a ring of N stages, advanced once per stage (no division).
+template <int N>
+struct Ring {
+    int idx = 0;
+    uint32_t phase = 0;
+    __device__ __forceinline__ void next() {
+        if (++idx == N) { idx = 0; phase ^= 1u; }
+    }
+};
+
+// Bounded wait that gives up at once after an abort.
+__device__ __forceinline__ bool wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+    if (tc::mbar_try_wait(bar, parity)) return true;      // completed phase: no flag read
+    if (*abort) return false;
+    if (tc::mbar_wait(bar, parity)) return true;
+    *abort = 1;
+    return false;
+}
+
+}  // namespace ws
+
+// Fused decode epilogues.  Requantization (S5) of a row needs max|h| over all of its M tiles,
+// and the combine (S7) of a token needs all k routed rows: the CTA that finishes the last
+// contribution (counted with a device-scope atomic after a fence) does that work, reading the
+// other CTAs' outputs through L2.  The result does not depend on which CTA finishes last.
+__device__ __forceinline__ void requant_row(const float* __restrict__ h, int N, unsigned amax_bits,
+                                            uint8_t* __restrict__ hq, float* __restrict__ s_h, int tid,
+                                            int nthreads, float* __restrict__ qs_row) {
+    const float s = __fdiv_rn(__uint_as_float(amax_bits), kFp8Max);
+    for (int base = 0; base < (N >> 3); base += nthreads) {
+        const int c = base + tid;
+        const bool live = c < (N >> 3);
+        uint2 codes = make_uint2(0u, 0u);
+        if (live && s != 0.0f) {
+            const float4 a = __ldcg(reinterpret_cast<const float4*>(h) + 2 * c);
+            const float4 b = __ldcg(reinterpret_cast<const float4*>(h) + 2 * c + 1);
+            codes.x = static_cast<uint32_t>(f32x2_to_e4m3x2(__fdiv_rn(a.x, s), __fdiv_rn(a.y, s))) |
+                      (static_cast<uint32_t>(f32x2_to_e4m3x2(__fdiv_rn(a.z, s), __fdiv_rn(a.w, s))) << 16);
+            codes.y = static_cast<uint32_t>(f32x2_to_e4m3x2(__fdiv_rn(b.x, s), __fdiv_rn(b.y, s))) |
+                      (static_cast<uint32_t>(f32x2_to_e4m3x2(__fdiv_rn(b.z, s), __fdiv_rn(b.w, s))) << 16);
+        }
+        if (live) reinterpret_cast<uint2*>(hq)[c] = codes;
+        if (qs_row) {   // sums of the decoded codes per K-group of 128 (16 chunks = one half-warp)
+            const float gs = halfwarp_sum(e4m3x8_sum(codes));
+            if (live && (tid & 15) == 0) qs_row[c / 16] = gs;
+        }
+    }
+    if (tid == 0) *s_h = s;
+}
+
+// ---- host side --------------------------------------------------------------------------------
+
+using PFN_encodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                     const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                     const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                     CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+inline PFN_encodeTiled encode_fn() {
+    static PFN_encodeTiled fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        fn = reinterpret_cast<PFN_encodeTiled>(p);
+    }
+    return fn;
+}
+
+// 2D byte tensor [rows, row_bytes] (row-major) with a box of box_rows x box_bytes.
+inline bool make_map_u8(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t rows,
+                        uint32_t box_bytes, uint32_t box_rows, CUtensorMapSwizzle swizzle) {
+    PFN_encodeTiled fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {row_bytes, rows};
+    const cuuint64_t strides[1] = {row_bytes};
+    const cuuint32_t box[2] = {box_bytes, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace moe
