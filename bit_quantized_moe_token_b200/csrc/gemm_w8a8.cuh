@@ -376,13 +376,15 @@ int launch_gemm_w8a8_inst(const W8GemmArgs& a, const void* act, const void* w0, 
     return launch_status();
 }
 
-// Token-tile width for the expected rows per expert: as for the W4A8 GEMM, plus 256-row tiles
-// for long segments (a weight stage then feeds twice the tokens, halving the weight bytes moved
-// per FLOP).  Narrow tiles (decode) gather their gate/up activation rows by token and fuse the
-// requantization / combine into the epilogues.
+// Token-tile width for the expected rows per expert: the narrow decode widths of the W4A8 GEMM
+// (16 / 32 rows), else 256 rows.  A wide tile's MMA N follows its live rows, so short segments
+// cost little more than in a narrower tile, while long ones re-read each weight stage for 256
+// tokens instead of 64 or 128 (measured: the Zipf T = 2048 gate/up GEMM 0.67 -> 0.46 ms, T =
+// 16384 36 -> 50 % of the FP8 peak).  Narrow tiles gather their gate/up activation rows by
+// token and fuse the requantization / combine into the epilogues.
 inline int w8_tile_rows(int64_t P, int E) {
-    const int64_t avg = (P + E - 1) / E;
-    return avg > 160 ? 256 : tc_tile_rows(P, E);
+    const int BN = tc_tile_rows(P, E);
+    return BN <= 32 ? BN : 256;
 }
 
 template <bool kSwiGLU>
@@ -393,8 +395,6 @@ int launch_gemm_w8a8(const W8GemmArgs& a, const void* act, const void* w0, const
     switch (BN) {
         case 16: return launch_gemm_w8a8_inst<16, kSwiGLU, true, kSwiGLU>(a, act, w0, w1, max_row_tiles, stream);
         case 32: return launch_gemm_w8a8_inst<32, kSwiGLU, true, kSwiGLU>(a, act, w0, w1, max_row_tiles, stream);
-        case 64: return launch_gemm_w8a8_inst<64, kSwiGLU, false, false>(a, act, w0, w1, max_row_tiles, stream);
-        case 128: return launch_gemm_w8a8_inst<128, kSwiGLU, false, false>(a, act, w0, w1, max_row_tiles, stream);
         default: return launch_gemm_w8a8_inst<256, kSwiGLU, false, false>(a, act, w0, w1, max_row_tiles, stream);
     }
 }

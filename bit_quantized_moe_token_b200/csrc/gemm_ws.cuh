@@ -615,7 +615,6 @@ int launch_gemm_ws(const WsGemmArgs& a, const void* act, const void* w0, const v
         // keeps the exact signed codes
         case 16: return launch_gemm_ws_inst<16, kSwiGLU, kSwiGLU, true, kSwiGLU>(a, act, w0, w1, max_row_tiles, stream);
         case 32: return launch_gemm_ws_inst<32, kSwiGLU, kSwiGLU, true, kSwiGLU>(a, act, w0, w1, max_row_tiles, stream);
-        case 64: return launch_gemm_ws_inst<64, false, kSwiGLU, false, false>(a, act, w0, w1, max_row_tiles, stream);
         default: return launch_gemm_ws_inst<128, false, kSwiGLU, false, false>(a, act, w0, w1, max_row_tiles, stream);
     }
 }
