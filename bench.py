@@ -475,7 +475,9 @@ def run_ours(args):
                        topk_fused_ms=round(rt_ms, 4), cuda_graph=r_graph),
         "layer_with_router": {"ms_per_step": round(lr_ms, 4),
                               "value": round(world * T / (lr_ms / 1e3), 1), "unit": "tokens/s",
-                              "note": "moe_*_forward_router: router logits + the layer per step"},
+                              "note": "moe_*_forward_router: router logits + the layer per step; "
+                                      "routing follows the synthetic N(0, 1/H) router weight (near "
+                                      "uniform), not the workload's given (e.g. Zipf) logits"},
         "e2e": {"value": round(tokens / (e2e_ms / 1e3), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * wl.H * 2 + T * wl.E * 4,
                 "d2h_bytes_per_step": T * wl.H * 2},
