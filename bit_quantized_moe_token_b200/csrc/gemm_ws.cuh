@@ -452,13 +452,26 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
                         for (int c0 = 0; c0 < C::kLd; c0 += 16)
                             tc::tmem_ld16(tcol + c1 + c0, *reinterpret_cast<uint32_t(*)[16]>(v + c0));
                         tc::tmem_wait_ld();
+                        // two columns per packed fp32 FMA (same rounding as two fmaf)
+                        const float2 sc2 = make_float2(sc, sc);
 #pragma unroll
-                        for (int j = 0; j < C::kLd; ++j) acc[c1 + j] = fmaf(sc, __uint_as_float(v[j]), acc[c1 + j]);
+                        for (int j = 0; j < C::kLd; j += 2) {
+                            const float2 r = __ffma2_rn(sc2, make_float2(__uint_as_float(v[j]), __uint_as_float(v[j + 1])),
+                                                        make_float2(acc[c1 + j], acc[c1 + j + 1]));
+                            acc[c1 + j] = r.x;
+                            acc[c1 + j + 1] = r.y;
+                        }
                         if constexpr (kUnsigned) {   // minus 8 * s * (group sum of the column's q)
                             const float scm = sc * (-1.0f / 64.0f);
+                            const float2 scm2 = make_float2(scm, scm);
                             const float* qg = sQs + g * BN + c_base + c1;
 #pragma unroll
-                            for (int j = 0; j < C::kLd; ++j) acc[c1 + j] = fmaf(scm, qg[j], acc[c1 + j]);
+                            for (int j = 0; j < C::kLd; j += 2) {
+                                const float2 r = __ffma2_rn(scm2, make_float2(qg[j], qg[j + 1]),
+                                                            make_float2(acc[c1 + j], acc[c1 + j + 1]));
+                                acc[c1 + j] = r.x;
+                                acc[c1 + j + 1] = r.y;
+                            }
                         }
                     }
                 }
