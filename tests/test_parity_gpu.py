@@ -235,6 +235,42 @@ def test_forward_ragged_shapes(E, H, N, k, T):
     _run_and_compare(hl, dl, x, logits, k)
 
 
+# the largest supported dimensions: H = 16384 (128 K-groups), N = 8192, E = 1024 with top-8
+@pytest.mark.parametrize("w8", [False, True])
+@pytest.mark.parametrize("E,H,N,k,T", [(2, 16384, 256, 1, 5), (2, 256, 8192, 2, 3), (1024, 256, 128, 8, 40)])
+def test_forward_max_shapes(w8, E, H, N, k, T):
+    hl, dl = (_host_layer_and_dev_w8a8 if w8 else _host_layer_and_dev)(E, H, N, seed=E + H + N)
+    x = synth.normal_bf16(9, 860 + T, T * H).reshape(T, H)
+    logits = synth.normal_f32(9, 861 + T, T * E).reshape(T, E)
+    _run_and_compare(hl, dl, x, logits, k)
+
+
+def test_forward_nan_logits_route_to_valid_experts():
+    """NaN logits are outside the input domain; the GPU ranks them as -inf, so every selected
+    id is a valid expert, and a NaN expert is never chosen while a finite one is left."""
+    hl, dl = _host_layer_and_dev(8, 256, 128, seed=77)
+    T, k = 6, 2
+    x = synth.normal_bf16(10, 850, T * 256).reshape(T, 256)
+    logits = synth.normal_f32(10, 851, T * 8).reshape(T, 8)
+    logits[0, :] = np.nan                               # all NaN: still k valid ids
+    logits[1, 3] = np.nan
+    logits[2, :7] = np.nan                              # one finite expert: it is chosen first
+    xd, ld = to_dev_bf16(x), torch.from_numpy(logits).cuda()
+    ws = moe.alloc_workspace(dl, T, k)
+    out = moe.forward(dl, xd, ld, k, ws=ws)
+    torch.cuda.synchronize()
+    assert moe.moe_last_device_status() == 0
+    ids = ws_views(dl, ws, T, k)["ids"]
+    assert ((ids >= 0) & (ids < 8)).all()
+    assert all(len(set(r)) == k for r in ids.tolist())
+    assert 3 not in ids[1].tolist()
+    assert ids[2, 0] == 7
+    finite = ~np.isnan(logits).any(axis=1)
+    ref_ids, _ = oracle.route_topk(np.where(np.isnan(logits), -np.inf, logits).astype(np.float32), k)
+    assert np.array_equal(ids[finite], ref_ids[finite])
+    assert np.isfinite(bf16_to_f32(bits(out))[finite]).all()
+
+
 def test_forward_shared_experts_small():
     hl, dl = _host_layer_and_dev(4, 256, 128, seed=5, n_shared=2, shared_N=256)
     T = 21
