@@ -46,10 +46,17 @@ class _Layer(ctypes.Structure):
                 ("gate_w8", ctypes.c_void_p), ("up_w8", ctypes.c_void_p),
                 ("down_w8", ctypes.c_void_p),
                 ("gate_rs", ctypes.c_void_p), ("up_rs", ctypes.c_void_p),
-                ("down_rs", ctypes.c_void_p)]
+                ("down_rs", ctypes.c_void_p),
+                ("gate_f4", ctypes.c_void_p), ("up_f4", ctypes.c_void_p),
+                ("down_f4", ctypes.c_void_p),
+                ("gate_bs", ctypes.c_void_p), ("up_bs", ctypes.c_void_p),
+                ("down_bs", ctypes.c_void_p),
+                ("gate_s2", ctypes.c_void_p), ("up_s2", ctypes.c_void_p),
+                ("down_s2", ctypes.c_void_p)]
 
 FMT_W4A8 = 0
 FMT_W8A8 = 1
+FMT_NVFP4 = 2
 
 
 _lib = None
@@ -77,6 +84,12 @@ def lib():
         L.or_quant_tokens.restype = None
         L.or_quant_rows.argtypes = [vp, i64, i64, vp, vp]
         L.or_quant_rows.restype = None
+        L.or_e2m1_decode.argtypes = [ctypes.c_uint8]
+        L.or_e2m1_decode.restype = ctypes.c_float
+        L.or_e2m1_encode.argtypes = [ctypes.c_float]
+        L.or_e2m1_encode.restype = ctypes.c_uint8
+        L.or_nvfp4_quant.argtypes = [vp, i64, i64, vp, vp, vp]
+        L.or_nvfp4_quant.restype = i32
         L.or_route_topk.argtypes = [vp, i64, i32, i32, vp, vp]
         L.or_router_logits.argtypes = [vp, vp, i64, i64, i32, vp]
         L.or_route_topk.restype = None
@@ -158,6 +171,27 @@ def quant_rows(w_bf16: np.ndarray):
     return q, s
 
 
+def e2m1_decode(c: int) -> float:
+    return float(lib().or_e2m1_decode(int(c)))
+
+
+def e2m1_encode(x: float) -> int:
+    return int(lib().or_e2m1_encode(float(x)))
+
+
+def nvfp4_quant(w_bf16: np.ndarray):
+    """NVFP4 of one projection: bf16 bits [rows, K] -> (codes uint8 [rows, K/2], E4M3 block
+    scales uint8 [rows, K/16], fp32 scale2)."""
+    w = np.ascontiguousarray(w_bf16, np.uint16)
+    rows, K = w.shape
+    codes = np.zeros((rows, K // 2), np.uint8)
+    scales = np.zeros((rows, K // 16), np.uint8)
+    s2 = ctypes.c_float(0.0)
+    if lib().or_nvfp4_quant(_p(w), rows, K, _p(codes), _p(scales), ctypes.byref(s2)) != 0:
+        raise ValueError("or_nvfp4_quant: K must be a multiple of 16")
+    return codes, scales, np.float32(s2.value)
+
+
 def router_logits(x_bf16: np.ndarray, wr_bf16: np.ndarray) -> np.ndarray:
     """[T, E] fp32 logits of bf16 tokens [T, H] against the bf16 router weight [E, H]."""
     x = np.ascontiguousarray(x_bf16, np.uint16)
@@ -210,6 +244,9 @@ class Layer:
         self.down_scales = None if down_scales is None else np.ascontiguousarray(down_scales, np.uint16)
         self.gate_w8 = self.up_w8 = self.down_w8 = None
         self.gate_rs = self.up_rs = self.down_rs = None
+        self.gate_f4 = self.up_f4 = self.down_f4 = None
+        self.gate_bs = self.up_bs = self.down_bs = None
+        self.gate_s2 = self.up_s2 = self.down_s2 = None
         self.sh_gate = None if sh_gate is None else np.ascontiguousarray(sh_gate, np.uint16)
         self.sh_up = None if sh_up is None else np.ascontiguousarray(sh_up, np.uint16)
         self.sh_down = None if sh_down is None else np.ascontiguousarray(sh_down, np.uint16)
@@ -233,6 +270,22 @@ class Layer:
         assert L.gate_rs.shape == (E, N) and L.down_rs.shape == (E, H)
         return L
 
+    @classmethod
+    def nvfp4(cls, E, H, N, gate_f4, up_f4, down_f4, gate_bs, up_bs, down_bs, gate_s2, up_s2,
+              down_s2, group=128, sh_gate=None, sh_up=None, sh_down=None):
+        """NVFP4 layer: codes [E,N,H/2], [E,N,H/2], [E,H,N/2]; E4M3 block scales [E,N,H/16],
+        [E,N,H/16], [E,H,N/16]; fp32 scale2 [E] per projection."""
+        L = cls(E, H, N, None, None, None, None, None, None, group=group, sh_gate=sh_gate,
+                sh_up=sh_up, sh_down=sh_down)
+        L.fmt = FMT_NVFP4
+        L.gate_f4, L.up_f4, L.down_f4 = (np.ascontiguousarray(a, np.uint8) for a in (gate_f4, up_f4, down_f4))
+        L.gate_bs, L.up_bs, L.down_bs = (np.ascontiguousarray(a, np.uint8) for a in (gate_bs, up_bs, down_bs))
+        L.gate_s2, L.up_s2, L.down_s2 = (np.ascontiguousarray(a, np.float32) for a in (gate_s2, up_s2, down_s2))
+        assert L.gate_f4.shape == (E, N, H // 2) and L.down_f4.shape == (E, H, N // 2)
+        assert L.gate_bs.shape == (E, N, H // 16) and L.down_bs.shape == (E, H, N // 16)
+        assert L.gate_s2.shape == (E,)
+        return L
+
     def _c(self):
         return _Layer(self.E, self.H, self.N, self.group,
                       _p(self.gate_packed), _p(self.up_packed), _p(self.down_packed),
@@ -240,7 +293,10 @@ class Layer:
                       self.n_shared, self.shared_N,
                       _p(self.sh_gate), _p(self.sh_up), _p(self.sh_down),
                       self.fmt, _p(self.gate_w8), _p(self.up_w8), _p(self.down_w8),
-                      _p(self.gate_rs), _p(self.up_rs), _p(self.down_rs))
+                      _p(self.gate_rs), _p(self.up_rs), _p(self.down_rs),
+                      _p(self.gate_f4), _p(self.up_f4), _p(self.down_f4),
+                      _p(self.gate_bs), _p(self.up_bs), _p(self.down_bs),
+                      _p(self.gate_s2), _p(self.up_s2), _p(self.down_s2))
 
 
 def moe_forward(layer: Layer, x_bf16: np.ndarray, logits: np.ndarray, k: int):
@@ -329,3 +385,25 @@ def quant_workload_layer_w8a8(wl, experts=None, with_shared=True):
                   sh_up=np.stack([synth.shared_weight(wl, s, "up") for s in range(wl.n_shared)]),
                   sh_down=np.stack([synth.shared_weight(wl, s, "down") for s in range(wl.n_shared)]))
     return Layer.w8a8(E, H, N, gq, uq, dq, gs, us, ds, group=wl.group, **sh)
+
+
+def quant_workload_layer_nvfp4(wl, experts=None, with_shared=True):
+    """NVFP4-quantize (oracle side) the seeded weights of workload `wl`; experts outside
+    `experts` stay zero, as in ``pack_workload_layer``."""
+    import synth
+    E, H, N = wl.E, wl.H, wl.N
+    c = {p: np.zeros((E, *synth.weight_shape(wl, p)[:1], synth.weight_shape(wl, p)[1] // 2), np.uint8)
+         for p in ("gate", "up", "down")}
+    b = {p: np.zeros((E, *synth.weight_shape(wl, p)[:1], synth.weight_shape(wl, p)[1] // 16), np.uint8)
+         for p in ("gate", "up", "down")}
+    s2 = {p: np.zeros(E, np.float32) for p in ("gate", "up", "down")}
+    for e in (range(E) if experts is None else experts):
+        for p in ("gate", "up", "down"):
+            c[p][e], b[p][e], s2[p][e] = nvfp4_quant(synth.expert_weight(wl, e, p))
+    sh = {}
+    if with_shared and wl.n_shared:
+        sh = dict(sh_gate=np.stack([synth.shared_weight(wl, s, "gate") for s in range(wl.n_shared)]),
+                  sh_up=np.stack([synth.shared_weight(wl, s, "up") for s in range(wl.n_shared)]),
+                  sh_down=np.stack([synth.shared_weight(wl, s, "down") for s in range(wl.n_shared)]))
+    return Layer.nvfp4(E, H, N, c["gate"], c["up"], c["down"], b["gate"], b["up"], b["down"],
+                       s2["gate"], s2["up"], s2["down"], group=wl.group, **sh)

@@ -27,6 +27,10 @@
  *  [P5] "Inkling 2 Small FP8 for AMD MI300X", "Precision and files": expert
  *       projections in FP8 with one fp32 scale per expert output channel,
  *       scale = max|row| / (largest FP8 value), per-token FP8 activations.
+ *  [P2] also, "On-disk tensor format" / "Dequant math": NVFP4 hot experts —
+ *       two E2M1 codes per byte (low nibble first), one E4M3 scale per block of
+ *       16 input weights, one fp32 scale2 per expert; W = LUT[code] * scale *
+ *       scale2 with LUT = 0 .5 1 1.5 2 3 4 6 and their negatives (codes 8..15).
  *  Readings where the pages are silent (listed with each function):
  *   R1 symmetric RTN scale = amax/7 stored as BF16 (round to nearest even),
  *      codes = clamp(rint(w/scale), -8, 7), all-zero group -> scale 0, codes 0;
@@ -45,6 +49,14 @@
  *      row scale is amax/448 (the page's 240 is the largest E4M3FNUZ value),
  *      codes = E4M3(w/scale) exactly as R2 does for a token row; a projection
  *      output is (sum_k dec(q_k) dec(w_k), k increasing) * s_w[n] * s_x.
+ *   R8 NVFP4 quantization (the page's hot slabs come from an NVFP4 base this
+ *      build does not have): per expert projection scale2 = amax / (6*448);
+ *      per block of 16 scale = E4M3(amax_block / (6*scale2)) as in R2; code =
+ *      nearest E2M1 value of w / (dec(scale)*scale2), ties to the even code,
+ *      saturating at +-6, sign kept (-0 -> code 8); a zero scale gives codes 0.
+ *   R9 NVFP4 experts run on the same per-token FP8 activations (S1): a
+ *      projection output is (sum_k dec(q_k) * W[n,k], k increasing) * s_x with
+ *      W dequantized by the page's formula in fp32.
  */
 #include <math.h>
 #include <stdint.h>
@@ -199,6 +211,63 @@ void or_quant_tokens(const uint16_t* x, int64_t T, int64_t H, uint8_t* q, float*
     }
 }
 
+/* ------------------------------------------------------------------------------------------ */
+/* NVFP4 ([P2] "Dequant math", reading R8)                                                      */
+/* ------------------------------------------------------------------------------------------ */
+
+static const float kE2M1[16] = {0.0f,  0.5f,  1.0f,  1.5f,  2.0f,  3.0f,  4.0f,  6.0f,
+                                -0.0f, -0.5f, -1.0f, -1.5f, -2.0f, -3.0f, -4.0f, -6.0f};
+
+float or_e2m1_decode(uint8_t c) { return kE2M1[c & 15]; }
+
+/* Nearest E2M1 value by exhaustive comparison with the eight magnitudes; on a tie the even
+ * code (lower code bit clear); above 6 the largest; the sign goes to code bit 3. */
+uint8_t or_e2m1_encode(float x) {
+    uint8_t sign = signbit(x) ? 8 : 0;
+    float a = fabsf(x);
+    int best = 0;
+    for (int i = 1; i < 8; ++i) {
+        float di = fabsf(a - kE2M1[i]), db = fabsf(a - kE2M1[best]);
+        if (di < db || (di == db && (i & 1) == 0)) best = i;
+    }
+    return (uint8_t)(sign | best);
+}
+
+/* NVFP4 quantization of one projection [rows, K] (reading R8): codes [rows, K/2] (element 2j
+ * in the low nibble of byte j), E4M3 block scales [rows, K/16], fp32 scale2.  -1 on K % 16. */
+int or_nvfp4_quant(const uint16_t* w, int64_t rows, int64_t K, uint8_t* codes, uint8_t* scales,
+                   float* scale2) {
+    if (K % 16) return -1;
+    float amax = 0.0f;
+    for (int64_t i = 0; i < rows * K; ++i) {
+        float a = fabsf(or_bf16_to_f32(w[i]));
+        if (a > amax) amax = a;
+    }
+    const float s2 = amax / 2688.0f;    /* 6 * 448 */
+    *scale2 = s2;
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t b = 0; b < K / 16; ++b) {
+            const uint16_t* wb = w + r * K + b * 16;
+            float ab = 0.0f;
+            for (int i = 0; i < 16; ++i) {
+                float a = fabsf(or_bf16_to_f32(wb[i]));
+                if (a > ab) ab = a;
+            }
+            uint8_t sc = (s2 == 0.0f) ? 0 : or_e4m3_encode(ab / (6.0f * s2));
+            scales[r * (K / 16) + b] = sc;
+            float d = or_e4m3_decode(sc) * s2;
+            for (int i = 0; i < 16; ++i) {
+                uint8_t c = (d == 0.0f) ? 0 : or_e2m1_encode(or_bf16_to_f32(wb[i]) / d);
+                int64_t k = b * 16 + i;
+                uint8_t* byte = codes + r * (K / 2) + k / 2;
+                if ((k & 1) == 0) *byte = c;
+                else *byte = (uint8_t)(*byte | (c << 4));
+            }
+        }
+    }
+    return 0;
+}
+
 /* Row-scaled FP8 weights ([P5], reading R7): one scale per row, same rule as a token row. */
 void or_quant_rows(const uint16_t* w, int64_t rows, int64_t K, uint8_t* q, float* s) {
     or_quant_tokens(w, rows, K, q, s);
@@ -288,6 +357,10 @@ typedef struct {
     int fmt;
     const uint8_t *gate_w8, *up_w8, *down_w8;               /* [E,N,H], [E,N,H], [E,H,N] */
     const float *gate_rs, *up_rs, *down_rs;                  /* [E,N], [E,N], [E,H] */
+    /* fmt 2 = NVFP4 experts (readings R8, R9) */
+    const uint8_t *gate_f4, *up_f4, *down_f4;               /* [E,N,H/2], [E,N,H/2], [E,H,N/2] */
+    const uint8_t *gate_bs, *up_bs, *down_bs;               /* [E,N,H/16], [E,N,H/16], [E,H,N/16] */
+    const float *gate_s2, *up_s2, *down_s2;                  /* [E] */
 } or_layer;
 
 /* Unpacked codes of one projection as floats, transposed to [K][rows] so that the
@@ -340,6 +413,30 @@ static void w8a8_proj(const uint8_t* q, float s_x, const float* cT, const float*
     for (int64_t n = 0; n < rows; ++n) out[n] = acc[n] * rs[n] * s_x;
 }
 
+/* NVFP4 weights dequantized by the page's formula ([P2] "Dequant math"), transposed to [K][rows]:
+ * W[r,k] = LUT[code] * dec(scale[r, k/16]) * scale2. */
+static void f4_T(const uint8_t* codes, const uint8_t* scales, float s2, int64_t rows, int64_t K,
+                 float* cT) {
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t kk = 0; kk < K; ++kk) {
+            uint8_t c = (codes[r * (K / 2) + kk / 2] >> (4 * (kk & 1))) & 15;
+            cT[kk * rows + r] = kE2M1[c] * or_e4m3_decode(scales[r * (K / 16) + kk / 16]) * s2;
+        }
+}
+
+/* Projection of one FP8 row on dequantized weights (reading R9): for every output n,
+ *   acc_n = sum_k dec(q_k) * W[n,k]  (k increasing),   out_n = acc_n * s_x. */
+static void f4_proj(const uint8_t* q, float s_x, const float* cT, int64_t rows, int64_t K,
+                    float* out, float* acc) {
+    for (int64_t n = 0; n < rows; ++n) acc[n] = 0.0f;
+    for (int64_t kk = 0; kk < K; ++kk) {
+        float a = or_e4m3_decode(q[kk]);
+        const float* c = cT + kk * rows;
+        for (int64_t n = 0; n < rows; ++n) acc[n] += a * c[n];
+    }
+    for (int64_t n = 0; n < rows; ++n) out[n] = acc[n] * s_x;
+}
+
 static float silu_f32(float g) { return g * (1.0f / (1.0f + expf(-g))); }
 
 /*
@@ -375,6 +472,21 @@ static void expert_row_w8(const uint8_t* q, float s_x, const float* cg, const fl
     for (int64_t n = 0; n < N; ++n) h[n] = silu_f32(G[n]) * U[n];
     quant_row_f32(h, N, hq, s_h);
     w8a8_proj(hq, *s_h, cd, rd, H, N, y, acc);
+}
+
+/* expert_row for NVFP4 experts (same steps, f4_proj for the three projections). */
+static void expert_row_f4(const uint8_t* q, float s_x, const float* cg, const float* cu,
+                          const float* cd, int64_t H, int64_t N, uint8_t* hq, float* s_h, float* y,
+                          float* scratch) {
+    float* G = scratch;
+    float* U = G + N;
+    float* h = U + N;
+    float* acc = h + N;
+    f4_proj(q, s_x, cg, N, H, G, acc);
+    f4_proj(q, s_x, cu, N, H, U, acc);
+    for (int64_t n = 0; n < N; ++n) h[n] = silu_f32(G[n]) * U[n];
+    quant_row_f32(h, N, hq, s_h);
+    f4_proj(hq, *s_h, cd, H, N, y, acc);
 }
 
 /* Shared expert in bf16 weights / fp32 arithmetic on the unquantized token row:
@@ -443,6 +555,10 @@ int or_moe_forward(const or_layer* L, const uint16_t* x, const float* logits, in
             w8_T(L->gate_w8 + e * N * H, N, H, cg);
             w8_T(L->up_w8 + e * N * H, N, H, cu);
             w8_T(L->down_w8 + e * H * N, H, N, cd);
+        } else if (L->fmt == 2) {
+            f4_T(L->gate_f4 + e * N * (H / 2), L->gate_bs + e * N * (H / 16), L->gate_s2[e], N, H, cg);
+            f4_T(L->up_f4 + e * N * (H / 2), L->up_bs + e * N * (H / 16), L->up_s2[e], N, H, cu);
+            f4_T(L->down_f4 + e * H * (N / 2), L->down_bs + e * H * (N / 16), L->down_s2[e], H, N, cd);
         } else {
             codes_T(L->gate_packed + e * N * (H / 8), N, H, cg);
             codes_T(L->up_packed + e * N * (H / 8), N, H, cu);
@@ -453,6 +569,9 @@ int or_moe_forward(const or_layer* L, const uint16_t* x, const float* logits, in
             if (L->fmt == 1)
                 expert_row_w8(xq + t * H, sx[t], cg, cu, cd, L->gate_rs + e * N, L->up_rs + e * N,
                               L->down_rs + e * H, H, N, hq + (int64_t)r * N, sh + r,
+                              y + (int64_t)r * H, scratch);
+            else if (L->fmt == 2)
+                expert_row_f4(xq + t * H, sx[t], cg, cu, cd, H, N, hq + (int64_t)r * N, sh + r,
                               y + (int64_t)r * H, scratch);
             else
                 expert_row(xq + t * H, sx[t], cg, cu, cd, L->gate_scales + e * N * G_h,
@@ -539,6 +658,10 @@ int or_moe_forward_dense(const or_layer* L, const uint16_t* x, const float* logi
             w8_T(L->gate_w8 + e * N * H, N, H, cg);
             w8_T(L->up_w8 + e * N * H, N, H, cu);
             w8_T(L->down_w8 + e * H * N, H, N, cd);
+        } else if (L->fmt == 2) {
+            f4_T(L->gate_f4 + e * N * (H / 2), L->gate_bs + e * N * (H / 16), L->gate_s2[e], N, H, cg);
+            f4_T(L->up_f4 + e * N * (H / 2), L->up_bs + e * N * (H / 16), L->up_s2[e], N, H, cu);
+            f4_T(L->down_f4 + e * H * (N / 2), L->down_bs + e * H * (N / 16), L->down_s2[e], H, N, cd);
         } else {
             codes_T(L->gate_packed + e * N * (H / 8), N, H, cg);
             codes_T(L->up_packed + e * N * (H / 8), N, H, cu);
@@ -548,6 +671,9 @@ int or_moe_forward_dense(const or_layer* L, const uint16_t* x, const float* logi
             if (L->fmt == 1)
                 expert_row_w8(xq + t * H, sx[t], cg, cu, cd, L->gate_rs + e * N, L->up_rs + e * N,
                               L->down_rs + e * H, H, N, hq_dense + (t * E + e) * N,
+                              sh_dense + t * E + e, y_dense + (t * E + e) * H, scratch);
+            else if (L->fmt == 2)
+                expert_row_f4(xq + t * H, sx[t], cg, cu, cd, H, N, hq_dense + (t * E + e) * N,
                               sh_dense + t * E + e, y_dense + (t * E + e) * H, scratch);
             else
                 expert_row(xq + t * H, sx[t], cg, cu, cd, L->gate_scales + e * N * G_h,

@@ -545,6 +545,156 @@ def test_w8a8_dense_brute_force_matches_permuted():
 
 
 # ------------------------------------------------------------------------------------------------
+# NVFP4 experts
+# ------------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("line", list(golden_lines("e2m1_lut.txt")))
+def test_e2m1_lut_golden(line):
+    c, v = line.split()
+    got = oracle.e2m1_decode(int(c))
+    assert got == float(v) and math.copysign(1.0, got) == math.copysign(1.0, float(v))
+
+
+def _e2m1_nearest_numpy(x):
+    """Nearest of the 16 E2M1 values by sorting distances (ties: the even code), sign kept."""
+    grid = np.array([0, .5, 1, 1.5, 2, 3, 4, 6], np.float64)
+    out = []
+    for v in np.asarray(x, np.float64):
+        d = np.abs(abs(v) - grid)
+        cand = np.flatnonzero(d == d.min())
+        i = int(cand[0]) if len(cand) == 1 else int(cand[cand % 2 == 0][0])
+        out.append(i | (8 if math.copysign(1.0, v) < 0 else 0))
+    return np.array(out)
+
+
+def test_e2m1_encode_vs_brute_force():
+    rng = np.random.default_rng(31)
+    mids = np.array([.25, .75, 1.25, 1.75, 2.5, 3.5, 5.0])
+    xs = np.concatenate([rng.uniform(-8, 8, 3000), mids, -mids, np.nextafter(mids, 0), np.nextafter(mids, 9),
+                         [0.0, -0.0, 6.0, 7.9, 100.0, -100.0]]).astype(np.float32)
+    got = np.array([oracle.e2m1_encode(float(v)) for v in xs])
+    assert np.array_equal(got, _e2m1_nearest_numpy(xs))
+
+
+def test_nvfp4_worked_row():
+    want = {}
+    for line in golden_lines("nvfp4_worked.txt"):
+        kind, i, v = line.split()
+        want[(kind, int(i))] = int(v, 16)
+    b0 = np.array([6, 3, 1.25, -0.75, 0.25, -6, 0, 2.5, 5, -1.75, 0.5, 4, -3.5, 1, 0, 0], np.float32) * 2.0 ** -4
+    b1 = np.zeros(16, np.float32)
+    b1[0] = 1.5 * 2.0 ** -6
+    codes, scales, s2 = oracle.nvfp4_quant(_f32_to_bf16_bits(np.concatenate([b0, b1])[None, :]))
+    assert s2 == np.float32(0.375) / np.float32(2688)
+    for (kind, i), v in want.items():
+        assert (scales[0, i] if kind == "scale" else codes[0, i]) == v, (kind, i)
+
+
+def _nvfp4_dequant(codes, scales, s2):
+    """The page's dequant math in fp64: LUT[code] * scale[block] * scale2, low nibble first."""
+    lut = np.array([oracle.e2m1_decode(c) for c in range(16)])
+    e4 = oracle.e4m3_decode_table().astype(np.float64)
+    rows, half = codes.shape
+    c = np.empty((rows, 2 * half), np.int64)
+    c[:, 0::2] = codes & 15
+    c[:, 1::2] = codes >> 4
+    return lut[c] * np.repeat(e4[scales], 16, axis=1) * float(s2)
+
+
+def test_nvfp4_roundtrip_error_bound():
+    """Every weight is within half an E2M1 step (relative 1/4 of the block's spacing; the
+    grid's widest gap is 2 at the top) of its dequantized value, block by block, and the
+    row maximum maps to +-6 * scale * scale2 of its block."""
+    rng = np.random.default_rng(32)
+    w = (rng.standard_normal((64, 256)) * 0.02 * 2.0 ** rng.uniform(-4, 4, (64, 1))).astype(np.float32)
+    w[3, 16:32] = 0.0                                  # an all-zero block: scale 0, codes 0
+    wb = _f32_to_bf16_bits(w)
+    codes, scales, s2 = oracle.nvfp4_quant(wb)
+    wf = oracle.bf16_to_f32(wb).astype(np.float64)
+    deq = _nvfp4_dequant(codes, scales, s2)
+    assert scales[3, 1] == 0 and not codes[3, 8:16].any()
+    e4 = oracle.e4m3_decode_table().astype(np.float64)
+    d = np.repeat(e4[scales], 16, axis=1) * float(s2)           # the block's unit
+    assert np.all(np.abs(deq - wf) <= d * 1.0 + 1e-30)         # half of the widest gap (2) of the grid
+    # relative error of the grid: at most half a step of 2^-1 relative spacing above 1
+    big = np.abs(wf) >= d
+    assert np.all(np.abs(deq - wf)[big] <= 0.25 * np.abs(wf)[big] + 1e-12)
+    # the largest weight of the tensor saturates the top code exactly
+    r, c = np.unravel_index(np.argmax(np.abs(wf)), wf.shape)
+    assert (codes[r, c // 2] >> (4 * (c % 2))) & 7 == 7
+
+
+def _f4_layer_from_f32(Wg, Wu, Wd):
+    E = Wg.shape[0]
+    def qp(W):
+        r = [oracle.nvfp4_quant(_f32_to_bf16_bits(W[e])) for e in range(E)]
+        return (np.stack([a for a, _, _ in r]), np.stack([b for _, b, _ in r]),
+                np.array([c for _, _, c in r], np.float32))
+    g, u, d = qp(Wg), qp(Wu), qp(Wd)
+    N, H = Wg.shape[1], Wg.shape[2]
+    return oracle.Layer.nvfp4(E, H, N, g[0], u[0], d[0], g[1], u[1], d[1], g[2], u[2], d[2]), (g, u, d)
+
+
+def test_nvfp4_constant_closed_form():
+    """The constant layer of tests/golden/constant_layer.txt in NVFP4: every weight is 6 x
+    block scale 448 x scale2 (= w0 / 2688) = w0 up to scale2's rounding, so the outputs match
+    the same golden values."""
+    want = {}
+    for line in golden_lines("constant_layer.txt"):
+        t, o, hq = line.split()
+        want[int(t)] = (float(o), int(hq, 16))
+    T, H, N, E, k = 4, 128, 128, 2, 1
+    w0 = 0.02734375
+    sgn = np.array([1.0, -1.0], np.float32)[:, None, None]
+    Wg = np.broadcast_to(sgn * w0, (E, N, H)).astype(np.float32)
+    Wd = np.broadcast_to(sgn * w0, (E, H, N)).astype(np.float32)
+    layer, (g, _, _) = _f4_layer_from_f32(Wg, Wg, Wd)
+    assert np.all(g[0][0] == 0x77) and np.all(g[0][1] == 0xFF) and np.all(g[1] == 0x7E)
+    x = _f32_to_bf16_bits(np.full((T, H), 0.875, np.float32))
+    lg = np.array([[1, 0], [0, 1], [1, 0], [0, 1]], np.float32)
+    r = oracle.moe_forward(layer, x, lg, k)
+    out = oracle.bf16_to_f32(r["out"])
+    for t in range(T):
+        assert np.all(out[t] == want[t][0]), (t, out[t, :4])
+        assert np.all(r["hq"][r["row_of_pair"][t]] == want[t][1])
+
+
+def test_nvfp4_single_expert_vs_fp64_mlp():
+    """E = 1, k = 1: the NVFP4 layer against a textbook fp64 SwiGLU MLP on the weights
+    dequantized by the page's formula and the unquantized input."""
+    rng = np.random.default_rng(33)
+    T, H, N = 24, 512, 256
+    def w(rows, K):
+        return (rng.standard_normal((1, rows, K)) * 0.02 * 2.0 ** rng.uniform(-3, 3, (1, rows, 1))).astype(np.float32)
+    layer, (g, u, d) = _f4_layer_from_f32(w(N, H), w(N, H), w(H, N))
+    x = _f32_to_bf16_bits(rng.standard_normal((T, H)).astype(np.float32))
+    r = oracle.moe_forward(layer, x, np.zeros((T, 1), np.float32), 1)
+    Dg, Du, Dd = (_nvfp4_dequant(p[0][0], p[1][0], p[2][0]) for p in (g, u, d))
+    xf = oracle.bf16_to_f32(x).astype(np.float64)
+    gg, uu = xf @ Dg.T, xf @ Du.T
+    ref = (gg / (1 + np.exp(-gg)) * uu) @ Dd.T
+    got = r["out_f32"].astype(np.float64)
+    assert np.linalg.norm(got - ref) / np.linalg.norm(ref) < 0.05
+    assert np.corrcoef(got.ravel(), ref.ravel())[0, 1] > 0.998
+
+
+def test_nvfp4_dense_brute_force_matches_permuted():
+    wl = synth.WORKLOADS["tiny"]
+    layer = oracle.quant_workload_layer_nvfp4(wl)
+    assert layer.fmt == oracle.FMT_NVFP4
+    x, lg = synth.tokens(wl), synth.logits(wl)
+    r = oracle.moe_forward(layer, x, lg, wl.k)
+    d = oracle.moe_forward_dense(layer, x, lg, wl.k)
+    assert np.array_equal(r["out"], d["out"])
+    for p in range(wl.P):
+        t, j = divmod(p, wl.k)
+        e = r["ids"][t, j]
+        row = r["row_of_pair"][p]
+        assert np.array_equal(r["hq"][row], d["hq"][t, e])
+        assert np.array_equal(r["y"][row], d["y"][t, e])
+
+
+# ------------------------------------------------------------------------------------------------
 # the generator (input recipe)
 # ------------------------------------------------------------------------------------------------
 
