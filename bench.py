@@ -47,6 +47,9 @@ def expert_bytes(wl, fmt="w4a8"):
     if fmt == "w8a8":
         gate = wl.N * wl.H + wl.N * 4
         down = wl.H * wl.N + wl.H * 4
+    elif fmt == "nvfp4":             # E2M1 codes + E4M3 block-16 scales + fp32 scale2
+        gate = wl.N * wl.H // 2 + wl.N * wl.H // 16 + 4
+        down = wl.H * wl.N // 2 + wl.H * wl.N // 16 + 4
     else:
         gate = wl.N * wl.H // 2 + wl.N * (wl.H // wl.group) * 2
         down = wl.H * wl.N // 2 + wl.H * (wl.N // wl.group) * 2
@@ -112,7 +115,9 @@ def is_prefill(wl):
 
 
 KERNEL_SOURCES = {"w4a8": ("gemm_ws.cuh", "tc_pipe.cuh", "tc_ptx.cuh", "tc_tiles.cuh", "common.cuh"),
-                  "w8a8": ("gemm_w8a8.cuh", "tc_pipe.cuh", "tc_ptx.cuh", "tc_tiles.cuh", "common.cuh")}
+                  "w8a8": ("gemm_w8a8.cuh", "tc_pipe.cuh", "tc_ptx.cuh", "tc_tiles.cuh", "common.cuh"),
+                  "nvfp4": ("gemm_nvfp4.cuh", "gemm_w8a8.cuh", "tc_pipe.cuh", "tc_ptx.cuh", "tc_tiles.cuh",
+                            "common.cuh")}
 PROFILE_FOR = {("w4a8", "decode_t8"): "gemm_w4a8_ws_decode_t8.md",
                ("w4a8", "prefill_t2048_zipf"): "gemm_w4a8_ws_prefill_t2048.md",
                ("w8a8", "decode_t8"): "gemm_w8a8_decode_t8.md",
@@ -273,7 +278,8 @@ def run_ours(args):
     import torch
     import torch.distributed as dist
     import bit_quantized_moe_token_b200 as moe
-    from bit_quantized_moe_token_b200.synthetic import device_inputs, device_layer, device_layer_w8a8
+    from bit_quantized_moe_token_b200.synthetic import (device_inputs, device_layer, device_layer_nvfp4,
+                                                        device_layer_w8a8)
 
     world, rank, local = dist_setup()
     torch.cuda.set_device(local)
@@ -284,10 +290,13 @@ def run_ours(args):
 
     wl = synth.WORKLOADS[args.workload]
     w8 = args.experts == "w8a8"
-    layer = (device_layer_w8a8 if w8 else device_layer)(wl, device=dev)
-    fwd = moe.moe_w8a8_forward if w8 else moe.moe_w4a8_forward
-    fwd_profiled = moe.moe_w8a8_forward_profiled if w8 else moe.moe_w4a8_forward_profiled
-    layout = moe.moe_w8a8_workspace_layout if w8 else moe.moe_w4a8_workspace_layout
+    f4 = args.experts == "nvfp4"
+    layer = (device_layer_w8a8 if w8 else device_layer_nvfp4 if f4 else device_layer)(wl, device=dev)
+    fwd = moe.moe_w8a8_forward if w8 else moe.moe_nvfp4_forward if f4 else moe.moe_w4a8_forward
+    fwd_profiled = (moe.moe_w8a8_forward_profiled if w8 else moe.moe_nvfp4_forward_profiled if f4
+                    else moe.moe_w4a8_forward_profiled)
+    layout = (moe.moe_w8a8_workspace_layout if w8 else moe.moe_nvfp4_workspace_layout if f4
+              else moe.moe_w4a8_workspace_layout)
     if not wl.n_shared:
         layer.sh_gate = layer.sh_up = layer.sh_down = None
     T, k = wl.T, wl.k
@@ -408,7 +417,8 @@ def run_ours(args):
     r_ms = max_over_ranks(r_ms, dev, world)
     rt_ms = max_over_ranks(rt_ms, dev, world)
     # the whole layer fed by the router weight (router, S1, S2 fused at decode)
-    fwd_router = moe.moe_w8a8_forward_router if w8 else moe.moe_w4a8_forward_router
+    fwd_router = (moe.moe_w8a8_forward_router if w8 else moe.moe_nvfp4_forward_router if f4
+                  else moe.moe_w4a8_forward_router)
     for i in range(3):
         fwd_router(layer, batches[i % N_BATCHES][0], wr, k, out, ws)
     q0, q1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -426,7 +436,7 @@ def run_ours(args):
     value = whole_job_rate(world, T, args.steps, total_ms)
     hbm, bf16, peak_kind = peaks()
     fmt = args.experts
-    kname = "W8A8" if w8 else "W4A8"
+    kname = "W8A8" if w8 else "NVFP4" if f4 else "W4A8"
     gu_bytes, down_bytes = expert_bytes(wl, fmt)
     mean_touched = sum(touched[i % N_BATCHES] for i in range(args.steps)) / args.steps
     dom_bytes = mean_touched * gu_bytes
@@ -461,7 +471,8 @@ def run_ours(args):
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "e4m3 x e4m3 -> f32" if w8 else "e4m3 x int4 -> f32", "data": "synthetic",
+        "dtype": ("e4m3 x e4m3 -> f32" if w8 else "f16(e2m1 x e4m3 scale) x f16(e4m3) -> f32" if f4
+                  else "e4m3 x int4 -> f32"), "data": "synthetic",
         "config": {"workload": wl.name, "experts": fmt, "T": T, "H": wl.H, "N": wl.N, "E": wl.E, "k": k,
                    "routing": wl.routing, "n_shared": wl.n_shared, "seed": wl.seed,
                    "batches": N_BATCHES, "parallelism": f"replicas x{world}",
@@ -506,6 +517,8 @@ def oracle_sample(wl, t0, max_tokens, fmt="w4a8"):
     used = sorted(set(ids.reshape(-1).tolist()))
     if fmt == "w8a8":
         layer = oracle.quant_workload_layer_w8a8(wl, experts=used)
+    elif fmt == "nvfp4":
+        layer = oracle.quant_workload_layer_nvfp4(wl, experts=used)
     else:
         layer = oracle.pack_workload_layer(wl, experts=used)
     return layer, x, lg, n
@@ -568,7 +581,7 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ref-tokens", type=int, default=8)
-    ap.add_argument("--experts", default="w4a8", choices=["w4a8", "w8a8"],
+    ap.add_argument("--experts", default="w4a8", choices=["w4a8", "w8a8", "nvfp4"],
                     help="routed-expert weight format (default: W4A8 INT4 x FP8)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

@@ -48,6 +48,16 @@ class _CLayer8(ctypes.Structure):
                 ("sh_down", ctypes.c_void_p)]
 
 
+class _CLayer4(ctypes.Structure):
+    _fields_ = [("E", ctypes.c_int), ("H", ctypes.c_int), ("N", ctypes.c_int),
+                ("gate_f4", ctypes.c_void_p), ("up_f4", ctypes.c_void_p), ("down_f4", ctypes.c_void_p),
+                ("gate_bs", ctypes.c_void_p), ("up_bs", ctypes.c_void_p), ("down_bs", ctypes.c_void_p),
+                ("gate_s2", ctypes.c_void_p), ("up_s2", ctypes.c_void_p), ("down_s2", ctypes.c_void_p),
+                ("n_shared", ctypes.c_int), ("shared_N", ctypes.c_int),
+                ("sh_gate", ctypes.c_void_p), ("sh_up", ctypes.c_void_p),
+                ("sh_down", ctypes.c_void_p)]
+
+
 class _CLayout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in
                 ("topk_ids", "topk_w", "expert_offsets", "sorted_pairs", "row_of_pair",
@@ -91,11 +101,20 @@ def lib() -> ctypes.CDLL:
         L.moe_w8a8_forward.argtypes = [ctypes.POINTER(_CLayer8), vp, vp, i64, i32, vp, vp, sz, vp]
         L.moe_w8a8_forward_profiled.argtypes = [ctypes.POINTER(_CLayer8), vp, vp, i64, i32, vp, vp,
                                                 sz, vp, vp, i32, vp]
+        L.nvfp4_quant_weights.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp]
+        L.moe_nvfp4_workspace_bytes.argtypes = [ctypes.POINTER(_CLayer4), i64, i32]
+        L.moe_nvfp4_workspace_bytes.restype = sz
+        L.moe_nvfp4_workspace_layout.argtypes = [ctypes.POINTER(_CLayer4), i64, i32,
+                                                 ctypes.POINTER(_CLayout)]
+        L.moe_nvfp4_forward.argtypes = [ctypes.POINTER(_CLayer4), vp, vp, i64, i32, vp, vp, sz, vp]
+        L.moe_nvfp4_forward_profiled.argtypes = [ctypes.POINTER(_CLayer4), vp, vp, i64, i32, vp, vp,
+                                                 sz, vp, vp, i32, vp]
         L.moe_router_topk_workspace_bytes.argtypes = [i64, i32, i32]
         L.moe_router_topk_workspace_bytes.restype = sz
         L.moe_router_topk.argtypes = [vp, vp, i64, i32, i32, i32, vp, vp, vp, vp, sz, vp]
         L.moe_w4a8_forward_router.argtypes = [ctypes.POINTER(_CLayer), vp, vp, i64, i32, vp, vp, sz, vp]
         L.moe_w8a8_forward_router.argtypes = [ctypes.POINTER(_CLayer8), vp, vp, i64, i32, vp, vp, sz, vp]
+        L.moe_nvfp4_forward_router.argtypes = [ctypes.POINTER(_CLayer4), vp, vp, i64, i32, vp, vp, sz, vp]
         L.moe_last_device_status.argtypes = [vp]
         L.moe_selftest_bounded_wait.argtypes = [i64, vp]
         L.moe_status_string.argtypes = [i32]
@@ -388,3 +407,101 @@ def moe_w8a8_forward_router(layer: Layer8, x, wr, k: int, out, ws, stream=None) 
     nbytes = ws.numel() * ws.element_size() if ws is not None else 0
     _check(lib().moe_w8a8_forward_router(ctypes.byref(s), _ptr(x), _ptr(wr), T, k, _ptr(out), _ptr(ws),
                                          nbytes, _stream(stream)), "moe_w8a8_forward_router")
+
+
+# ---- NVFP4 experts ------------------------------------------------------------------------------
+
+def nvfp4_quant_weights(w, codes, scales, scale2, stream=None) -> None:
+    """w bf16 [experts, rows, K] -> codes uint8 [experts, rows, K/2], E4M3 block scales uint8
+    [experts, rows, K/16], fp32 scale2 [experts]."""
+    E, rows, K = w.shape
+    _check(lib().nvfp4_quant_weights(_ptr(w), E, rows, K, _ptr(codes), _ptr(scales), _ptr(scale2),
+                                     _stream(stream)), "nvfp4_quant_weights")
+
+
+@dataclass
+class Layer4:
+    """Device tensors of one layer with NVFP4 experts (moe_nvfp4_layer)."""
+    E: int
+    H: int
+    N: int
+    gate_f4: object
+    up_f4: object
+    down_f4: object
+    gate_bs: object
+    up_bs: object
+    down_bs: object
+    gate_s2: object
+    up_s2: object
+    down_s2: object
+    sh_gate: object = None
+    sh_up: object = None
+    sh_down: object = None
+
+    @property
+    def n_shared(self) -> int:
+        return 0 if self.sh_gate is None else int(self.sh_gate.shape[0])
+
+    @property
+    def shared_N(self) -> int:
+        return 0 if self.sh_gate is None else int(self.sh_gate.shape[1])
+
+    def c_struct(self) -> _CLayer4:
+        return _CLayer4(self.E, self.H, self.N, _ptr(self.gate_f4), _ptr(self.up_f4), _ptr(self.down_f4),
+                        _ptr(self.gate_bs), _ptr(self.up_bs), _ptr(self.down_bs),
+                        _ptr(self.gate_s2), _ptr(self.up_s2), _ptr(self.down_s2),
+                        self.n_shared, self.shared_N, _ptr(self.sh_gate), _ptr(self.sh_up),
+                        _ptr(self.sh_down))
+
+    def shape_struct(self) -> _CLayer4:
+        return _CLayer4(self.E, self.H, self.N, None, None, None, None, None, None, None, None, None,
+                        self.n_shared, self.shared_N, None, None, None)
+
+
+def layer4_struct(E, H, N, n_shared=0, shared_N=0) -> _CLayer4:
+    return _CLayer4(E, H, N, None, None, None, None, None, None, None, None, None, n_shared, shared_N,
+                    None, None, None)
+
+
+def moe_nvfp4_workspace_bytes(layer, T: int, k: int) -> int:
+    s = layer if isinstance(layer, _CLayer4) else layer.shape_struct()
+    return int(lib().moe_nvfp4_workspace_bytes(ctypes.byref(s), T, k))
+
+
+def moe_nvfp4_workspace_layout(layer, T: int, k: int) -> dict:
+    s = layer if isinstance(layer, _CLayer4) else layer.shape_struct()
+    out = _CLayout()
+    _check(lib().moe_nvfp4_workspace_layout(ctypes.byref(s), T, k, ctypes.byref(out)),
+           "moe_nvfp4_workspace_layout")
+    return {n: int(getattr(out, n)) for n, _ in _CLayout._fields_}
+
+
+def moe_nvfp4_forward(layer: Layer4, x, logits, k: int, out, ws, stream=None) -> None:
+    """out bf16 [T, H] = the routed MoE layer with NVFP4 experts applied to x."""
+    T = x.shape[0]
+    s = layer.c_struct()
+    nbytes = ws.numel() * ws.element_size() if ws is not None else 0
+    _check(lib().moe_nvfp4_forward(ctypes.byref(s), _ptr(x), _ptr(logits), T, k, _ptr(out),
+                                   _ptr(ws), nbytes, _stream(stream)), "moe_nvfp4_forward")
+
+
+def moe_nvfp4_forward_profiled(layer: Layer4, x, logits, k: int, out, ws, events, stream=None) -> int:
+    T = x.shape[0]
+    s = layer.c_struct()
+    nbytes = ws.numel() * ws.element_size() if ws is not None else 0
+    arr = (ctypes.c_void_p * len(events))(
+        *[ctypes.c_void_p(e.cuda_event if e is not None else 0) for e in events])
+    n = ctypes.c_int(0)
+    _check(lib().moe_nvfp4_forward_profiled(ctypes.byref(s), _ptr(x), _ptr(logits), T, k, _ptr(out),
+                                            _ptr(ws), nbytes, _stream(stream), arr, len(events),
+                                            ctypes.byref(n)), "moe_nvfp4_forward_profiled")
+    return int(n.value)
+
+
+def moe_nvfp4_forward_router(layer: Layer4, x, wr, k: int, out, ws, stream=None) -> None:
+    """The NVFP4 layer fed by the router weight wr bf16 [E, H]."""
+    T = x.shape[0]
+    s = layer.c_struct()
+    nbytes = ws.numel() * ws.element_size() if ws is not None else 0
+    _check(lib().moe_nvfp4_forward_router(ctypes.byref(s), _ptr(x), _ptr(wr), T, k, _ptr(out), _ptr(ws),
+                                          nbytes, _stream(stream)), "moe_nvfp4_forward_router")

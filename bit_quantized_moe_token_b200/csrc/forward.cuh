@@ -6,6 +6,8 @@
 #include "route.cuh"
 #include "gemm_ws.cuh"
 #include "gemm_w8a8.cuh"
+#include "gemm_nvfp4.cuh"
+#include "nvfp4.cuh"
 #include "gemm_bf16_tc.cuh"
 #include "router.cuh"
 
@@ -114,12 +116,14 @@ struct WsPlan {
     size_t xq, s_x, x_sorted, s_x_sorted, h, zero, hq, s_h, y;
     size_t qs_x, qs_h;   // per (activation row, K-group) sums of the FP8 values (narrow tiles)
     size_t logits, rcnt; // router logits [T, E] and the fused router's counters (router entry points)
+    size_t act16;        // NVFP4 experts: f16 copies of the GEMM inputs (max of [T|P, H] and [P, N])
     int64_t n_zero;   // u32 words at `zero`: max|h| per row [P], row counters [P], token counters
     size_t sh_a, sh_y;
     size_t total;
 };
 
-inline WsPlan plan_workspace(const moe_w4a8_layer& L, int64_t T, int k) {
+// fmt: 0 W4A8, 1 row-scaled FP8, 2 NVFP4 (the last needs the f16 activation copies).
+inline WsPlan plan_workspace(const moe_w4a8_layer& L, int64_t T, int k, int fmt = 0) {
     WsPlan p{};
     const int64_t P = T * k;
     size_t off = 0;
@@ -148,6 +152,7 @@ inline WsPlan plan_workspace(const moe_w4a8_layer& L, int64_t T, int k) {
     p.qs_h = take((size_t)P * (L.N / 128) * 4);
     p.logits = take((size_t)T * L.E * 4);
     p.rcnt = take((size_t)router_counter_words(T) * 4);
+    p.act16 = fmt == 2 ? take((size_t)P * (L.H > L.N ? L.H : L.N) * 2) : 0;
     if (L.n_shared > 0) {
         p.sh_a = take((size_t)T * L.n_shared * L.shared_N * 2);
         p.sh_y = take((size_t)T * L.H * 4);
@@ -196,15 +201,17 @@ extern "C" int moe_w4a8_workspace_layout(const moe_w4a8_layer* layer, int64_t T,
 
 namespace moe {
 
-// Routed-expert weights of one layer in either format.
+// Routed-expert weights of one layer in any of the three formats.
+enum ExpertFmt { kFmtW4A8 = 0, kFmtW8A8 = 1, kFmtNvfp4 = 2 };
 struct ExpertSet {
-    bool w8;                              // row-scaled FP8 (true) or W4A8 (false)
-    const void *gate, *up, *down;         // W4A8: int32 [E,R,K/8]; W8A8: E4M3 [E,R,K]
-    const void *gate_s, *up_s, *down_s;   // W4A8: bf16 [E,R,K/128]; W8A8: fp32 [E,R]
+    int fmt;
+    const void *gate, *up, *down;         // W4A8: int32 [E,R,K/8]; W8A8: E4M3 [E,R,K]; NVFP4: [E,R,K/2]
+    const void *gate_s, *up_s, *down_s;   // W4A8: bf16 [E,R,K/128]; W8A8: fp32 [E,R]; NVFP4: E4M3 [E,R,K/16]
+    const float *gate_s2 = nullptr, *up_s2 = nullptr, *down_s2 = nullptr;   // NVFP4: fp32 [E]
 };
 
 inline ExpertSet experts_of(const moe_w4a8_layer& L) {
-    return ExpertSet{false, L.gate_packed, L.up_packed, L.down_packed, L.gate_scales, L.up_scales,
+    return ExpertSet{kFmtW4A8, L.gate_packed, L.up_packed, L.down_packed, L.gate_scales, L.up_scales,
                      L.down_scales};
 }
 
@@ -266,9 +273,10 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const ExpertSet& xw, const ui
     if (L.n_shared > 0 && (!L.sh_gate || !L.sh_up || !L.sh_down)) return MOE_ERR_INVALID_ARG;
     if (L.n_shared > 0 && (!aligned(L.sh_gate, 16) || !aligned(L.sh_up, 16) || !aligned(L.sh_down, 16)))
         return MOE_ERR_MISALIGNED;
-    const WsPlan p = plan_workspace(L, T, k);
+    const WsPlan p = plan_workspace(L, T, k, xw.fmt);
     if (!ws || ws_bytes < p.total) return MOE_ERR_WORKSPACE;
-    const size_t s_al = xw.w8 ? 4 : 2;   // fp32 row scales / bf16 group scales
+    const size_t s_al = xw.fmt == kFmtW8A8 ? 4 : xw.fmt == kFmtNvfp4 ? 8 : 2;   // scale alignment
+    if (xw.fmt == kFmtNvfp4 && (!xw.gate_s2 || !xw.up_s2 || !xw.down_s2)) return MOE_ERR_INVALID_ARG;
     if (!aligned(ws, 256) || !aligned(x_bf16, 16) || !aligned(out_bf16, 16) ||
         !aligned(router_logits, 4) || !aligned(xw.gate, 16) || !aligned(xw.up, 16) ||
         !aligned(xw.down, 16) || !aligned(xw.gate_s, s_al) || !aligned(xw.up_s, s_al) ||
@@ -300,7 +308,8 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const ExpertSet& xw, const ui
     // narrow token tiles (decode): codes written once per token and gathered by the GEMM, fused
     // requantization and combine; wide tiles (prefill): codes copied to expert-sorted rows.
     const bool fused = ws_narrow(tc_tile_rows(P, L.E));
-    float* qsum_x = xw.w8 ? nullptr : qs_x;       // group sums serve the unsigned widening only
+    float* qsum_x = xw.fmt == kFmtW4A8 ? qs_x : nullptr;   // group sums: the unsigned widening only
+    uint16_t* act16 = xw.fmt == kFmtNvfp4 ? (uint16_t*)at(p.act16) : nullptr;
 
     sm.mark(0, stream);
     if (router_w) {
@@ -374,7 +383,15 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const ExpertSet& xw, const ui
     }
     sm.mark(3, stream);
     // S4 + SwiGLU (+ S5 when fused): h = silu(G) * U, max|h| per row
-    if (xw.w8) {
+    if (xw.fmt == kFmtNvfp4) {
+        // f16 copy of the FP8 activations (exact), then the f16 tensor-core GEMM
+        if ((st = launch_e4m3_to_f16(fused ? xq : xs, (fused ? T : P) * L.H, act16, stream))) return st;
+        F4GemmArgs f{W8GemmArgs{fused ? sx : sxs, nullptr, nullptr, offsets, L.E, L.N, L.H, (int)P, h, L.N,
+                                amax, rowcnt, hq, sh, sorted, nullptr, nullptr, k, nullptr, nullptr, (int)T},
+                     (const uint8_t*)xw.gate_s, (const uint8_t*)xw.up_s, xw.gate_s2, xw.up_s2};
+        if ((st = launch_gemm_nvfp4<true>(f, act16, xw.gate, xw.up, stream))) return st;
+        sm.launches += 2;
+    } else if (xw.fmt == kFmtW8A8) {
         W8GemmArgs a{fused ? sx : sxs, (const float*)xw.gate_s, (const float*)xw.up_s, offsets, L.E, L.N,
                      L.H, (int)P, h, L.N, amax, rowcnt, hq, sh, sorted, nullptr, nullptr, k, nullptr,
                      nullptr, (int)T};
@@ -400,7 +417,14 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const ExpertSet& xw, const ui
     }
     sm.mark(5, stream);
     // S6 (+ S7 when fused)
-    if (xw.w8) {
+    if (xw.fmt == kFmtNvfp4) {
+        if ((st = launch_e4m3_to_f16(hq, P * L.N, act16, stream))) return st;
+        F4GemmArgs f{W8GemmArgs{sh, nullptr, nullptr, offsets, L.E, L.H, L.N, (int)P, y, L.H, nullptr, tokcnt,
+                                nullptr, nullptr, sorted, rop, gates, k, shared, out_bf16, (int)T},
+                     (const uint8_t*)xw.down_s, nullptr, xw.down_s2, nullptr};
+        if ((st = launch_gemm_nvfp4<false>(f, act16, xw.down, nullptr, stream))) return st;
+        sm.launches += 2;
+    } else if (xw.fmt == kFmtW8A8) {
         W8GemmArgs a{sh, (const float*)xw.down_s, nullptr, offsets, L.E, L.H, L.N, (int)P, y, L.H, nullptr,
                      tokcnt, nullptr, nullptr, sorted, rop, gates, k, shared, out_bf16, (int)T};
         if ((st = launch_gemm_w8a8<false>(a, hq, xw.down, nullptr, stream))) return st;
@@ -434,7 +458,7 @@ inline moe_w4a8_layer shape_of(const moe_w8a8_layer& L) {
                           L.n_shared, L.shared_N, L.sh_gate, L.sh_up, L.sh_down};
 }
 inline ExpertSet experts_of(const moe_w8a8_layer& L) {
-    return ExpertSet{true, L.gate_w8, L.up_w8, L.down_w8, L.gate_rs, L.up_rs, L.down_rs};
+    return ExpertSet{kFmtW8A8, L.gate_w8, L.up_w8, L.down_w8, L.gate_rs, L.up_rs, L.down_rs};
 }
 }  // namespace moe
 
@@ -493,6 +517,69 @@ extern "C" int moe_w8a8_forward_router(const moe_w8a8_layer* layer, const uint16
                                        const uint16_t* router_w_bf16, int64_t T, int k,
                                        uint16_t* out_bf16, void* ws, size_t ws_bytes,
                                        moe_stream_t stream) {
+    if (!layer) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && !router_w_bf16) return MOE_ERR_INVALID_ARG;
+    moe::StageMarks sm{nullptr, 0, 0};
+    const moe_w4a8_layer s = moe::shape_of(*layer);
+    return moe::forward_impl(&s, moe::experts_of(*layer), x_bf16, nullptr, T, k, out_bf16, ws, ws_bytes,
+                             stream, sm, router_w_bf16);
+}
+
+// ---- NVFP4 experts ----------------------------------------------------------------------------
+
+namespace moe {
+inline moe_w4a8_layer shape_of(const moe_nvfp4_layer& L) {
+    return moe_w4a8_layer{L.E, L.H, L.N, kGroup, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
+                          L.n_shared, L.shared_N, L.sh_gate, L.sh_up, L.sh_down};
+}
+inline ExpertSet experts_of(const moe_nvfp4_layer& L) {
+    return ExpertSet{kFmtNvfp4, L.gate_f4, L.up_f4, L.down_f4, L.gate_bs, L.up_bs, L.down_bs,
+                     L.gate_s2, L.up_s2, L.down_s2};
+}
+}  // namespace moe
+
+extern "C" size_t moe_nvfp4_workspace_bytes(const moe_nvfp4_layer* layer, int64_t T, int k) {
+    if (!layer) return 0;
+    const moe_w4a8_layer s = moe::shape_of(*layer);
+    if (moe::layer_args_ok(&s, T, k) != MOE_OK) return 0;
+    return moe::plan_workspace(s, T, k, moe::kFmtNvfp4).total;
+}
+
+extern "C" int moe_nvfp4_workspace_layout(const moe_nvfp4_layer* layer, int64_t T, int k,
+                                          moe_w4a8_ws_layout* out) {
+    if (!layer) return MOE_ERR_INVALID_ARG;
+    const moe_w4a8_layer s = moe::shape_of(*layer);
+    int st = moe_w4a8_workspace_layout(&s, T, k, out);
+    if (st == MOE_OK) out->total = moe::plan_workspace(s, T, k, moe::kFmtNvfp4).total;
+    return st;
+}
+
+extern "C" int moe_nvfp4_forward_profiled(const moe_nvfp4_layer* layer, const uint16_t* x_bf16,
+                                          const float* router_logits, int64_t T, int k,
+                                          uint16_t* out_bf16, void* ws, size_t ws_bytes,
+                                          moe_stream_t stream, void* const* events, int n_events,
+                                          int* n_launches) {
+    if (!layer) return MOE_ERR_INVALID_ARG;
+    if (events && n_events < MOE_W4A8_N_STAGE_EVENTS) return MOE_ERR_INVALID_ARG;
+    moe::StageMarks sm{events, n_events, 0};
+    const moe_w4a8_layer s = moe::shape_of(*layer);
+    const int st = moe::forward_impl(&s, moe::experts_of(*layer), x_bf16, router_logits, T, k,
+                                     out_bf16, ws, ws_bytes, stream, sm);
+    if (n_launches) *n_launches = sm.launches;
+    return st;
+}
+
+extern "C" int moe_nvfp4_forward(const moe_nvfp4_layer* layer, const uint16_t* x_bf16,
+                                 const float* router_logits, int64_t T, int k, uint16_t* out_bf16,
+                                 void* ws, size_t ws_bytes, moe_stream_t stream) {
+    return moe_nvfp4_forward_profiled(layer, x_bf16, router_logits, T, k, out_bf16, ws, ws_bytes, stream,
+                                      nullptr, 0, nullptr);
+}
+
+extern "C" int moe_nvfp4_forward_router(const moe_nvfp4_layer* layer, const uint16_t* x_bf16,
+                                        const uint16_t* router_w_bf16, int64_t T, int k,
+                                        uint16_t* out_bf16, void* ws, size_t ws_bytes,
+                                        moe_stream_t stream) {
     if (!layer) return MOE_ERR_INVALID_ARG;
     if (T > 0 && !router_w_bf16) return MOE_ERR_INVALID_ARG;
     moe::StageMarks sm{nullptr, 0, 0};

@@ -82,6 +82,133 @@ struct W8Cfg {
     static constexpr int kWarpTma = 4, kWarpMma = 5;
 };
 
+// The epilogue warps (threads 0..127, thread = TMEM lane = weight row): every tile's accumulator
+// times the tile's row scale rs_of(expert, m tile, row) and the column (token) scales, then the
+// SwiGLU epilogue (max|h| per row; narrow tiles: the requantization behind a row counter) or the
+// plain one (narrow tiles: the combine behind a token counter).  Shared by the FP8 and NVFP4
+// expert GEMMs, whose accumulators both hold the whole K.
+template <int BN, bool kSwiGLU, bool kFused, bool kGather, class RowScale>
+__device__ __forceinline__ void w8_epilogue_warps(const W8GemmArgs& a, int64_t n_tiles, int m_tiles,
+                                                  const int* pre, const int* soff, float* sSr, float* sX,
+                                                  int* flag, uint32_t tmem, uint64_t* t_full,
+                                                  uint64_t* t_empty, volatile int* abort, RowScale rs_of) {
+    constexpr int kXS = (BN < 32 ? BN : 32) + 1;         // SwiGLU exchange row stride
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    constexpr int kNPT = 128;
+    constexpr int kCh = BN < 32 ? BN : 32;            // TMEM columns per load
+    const uint32_t t_lane = static_cast<uint32_t>(warp * 32) << 16;
+    const int lrow = tid;                              // A row = TMEM lane
+    uint32_t tcount = 0;
+    for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++tcount) {
+        const int rt = static_cast<int>(tile / m_tiles), mt = static_cast<int>(tile % m_tiles);
+        const int e = expert_of_tile(pre, a.E, rt);
+        const int64_t row0 = soff[e] + (rt - pre[e]) * BN;
+        const int nrows = min(BN, soff[e + 1] - static_cast<int>(row0));
+        float* sr_t = sSr + (tcount & 1) * BN;         // two buffers: tile parity
+        for (int c = tid; c < BN; c += kNPT) {
+            float v = 0.0f;
+            if (c < nrows) v = kGather ? a.s_row[a.sorted[row0 + c] / a.k] : a.s_row[row0 + c];
+            sr_t[c] = v;
+        }
+        const float rs = rs_of(e, mt, lrow);
+        const int tb = tcount & 1;
+        ws::wait(&t_full[tb], (tcount >> 1) & 1, abort);
+        tc::tc_fence_after();
+        ws::named_sync_math<kNPT>();                   // column scales visible
+        const uint32_t tcol = tmem + t_lane + tb * BN;
+#pragma unroll 1
+        for (int c0 = 0; c0 < nrows; c0 += kCh) {       // only the columns the MMA wrote
+            uint32_t v[kCh];
+            if constexpr (kCh == 32) tc::tmem_ld32(tcol + c0, *reinterpret_cast<uint32_t(*)[32]>(v));
+            else tc::tmem_ld16(tcol + c0, *reinterpret_cast<uint32_t(*)[16]>(v));
+            tc::tmem_wait_ld();
+            float val[kCh];
+#pragma unroll
+            for (int j = 0; j < kCh; ++j) val[j] = __fmul_rn(__fmul_rn(__uint_as_float(v[j]), rs), sr_t[c0 + j]);
+            if constexpr (kSwiGLU) {
+                // gate rows finish the first half of the columns, up rows the second; each
+                // hands the other the half it does not finish
+                constexpr int kHalf = kCh / 2;
+                const bool gate = lrow < 64;
+                const int r64 = lrow & 63;
+#pragma unroll
+                for (int j = 0; j < kHalf; ++j)
+                    sX[r64 * kXS + (gate ? kHalf : 0) + j] = gate ? val[kHalf + j] : val[j];
+                ws::named_sync_math<kNPT>();
+                const int cm = c0 + (gate ? 0 : kHalf);
+                const int n = mt * 64 + r64;
+                float hv[kHalf];
+#pragma unroll
+                for (int j = 0; j < kHalf; ++j) {
+                    const float other = sX[r64 * kXS + (gate ? 0 : kHalf) + j];
+                    const float gv = gate ? val[j] : other;
+                    const float uv = gate ? other : val[kHalf + j];
+                    hv[j] = silu_fast(gv) * uv;
+                }
+#pragma unroll
+                for (int j = 0; j < kHalf; ++j)
+                    if (cm + j < nrows) a.out[(row0 + cm + j) * a.ldo + n] = hv[j];
+#pragma unroll
+                for (int j = 0; j < kHalf; ++j) {
+                    const unsigned m = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(hv[j])));
+                    if (lane == 0 && cm + j < nrows) atomicMax(a.amax + row0 + cm + j, m);
+                }
+                ws::named_sync_math<kNPT>();           // exchange buffer free again
+            } else {
+                const int m = mt * 128 + lrow;
+#pragma unroll
+                for (int j = 0; j < kCh; ++j)
+                    if (c0 + j < nrows) a.out[(row0 + c0 + j) * a.ldo + m] = val[j];
+            }
+        }
+        tc::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&t_empty[tb]);
+
+        if constexpr (kFused) {
+            // The barrier orders every thread's stores before the counting threads' fences,
+            // and a fence is cumulative, so one fence per counted row suffices.
+            ws::named_sync_math<kNPT>();
+            if constexpr (kSwiGLU) {
+                if (tid < nrows) {
+                    __threadfence();
+                    flag[tid] = atomicAdd(a.cnt + row0 + tid, 1u) == (unsigned)(m_tiles - 1);
+                }
+                ws::named_sync_math<kNPT>();
+                for (int j = 0; j < nrows; ++j) {
+                    if (flag[j]) {
+                        __threadfence();
+                        const int64_t r = row0 + j;
+                        requant_row(a.out + r * a.ldo, a.ldo, __ldcg(a.amax + r), a.hq + r * a.ldo,
+                                    a.s_h + r, tid, kNPT, nullptr);
+                    }
+                }
+            } else {
+                const int m = mt * 128 + lrow;
+                if (tid < nrows) {
+                    __threadfence();
+                    const int t = a.sorted[row0 + tid] / a.k;
+                    flag[tid] = atomicAdd(a.cnt + (int64_t)t * m_tiles + mt, 1u) == (unsigned)(a.k - 1) ? t : -1;
+                }
+                ws::named_sync_math<kNPT>();
+                for (int j = 0; j < nrows; ++j) {
+                    const int t = flag[j];
+                    if (t >= 0) {
+                        __threadfence();
+                        float o = 0.0f;
+                        for (int jj = 0; jj < a.k; ++jj)
+                            o = __fadd_rn(o, __fmul_rn(a.gates[t * a.k + jj],
+                                                       __ldcg(a.out + (int64_t)a.rop[t * a.k + jj] * a.ldo + m)));
+                        if (a.shared) o = __fadd_rn(o, a.shared[(int64_t)t * a.ldo + m]);
+                        a.out_bf16[(int64_t)t * a.ldo + m] = f32_to_bf16_bits(o);
+                    }
+                }
+            }
+            ws::named_sync_math<kNPT>();
+        }
+    }
+}
+
 template <int BN, bool kSwiGLU, bool kFused, bool kGather>
 __global__ void __launch_bounds__(W8Cfg<BN>::kThreads, 1)
     k_gemm_w8a8(const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__ CUtensorMap tm_w1,
@@ -219,121 +346,12 @@ __global__ void __launch_bounds__(W8Cfg<BN>::kThreads, 1)
         }
     } else {
         // ------------------------------------------------------------ epilogue warps 0-3
-        constexpr int kNPT = 128;
-        constexpr int kCh = C::kChunk;
-        const uint32_t t_lane = static_cast<uint32_t>(warp * 32) << 16;
-        const int lrow = tid;                              // A row = TMEM lane
-        uint32_t tcount = 0;
-        for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++tcount) {
-            const int rt = static_cast<int>(tile / m_tiles), mt = static_cast<int>(tile % m_tiles);
-            const int e = expert_of_tile(pre, a.E, rt);
-            const int64_t row0 = soff[e] + (rt - pre[e]) * BN;
-            const int nrows = min(BN, soff[e + 1] - static_cast<int>(row0));
-            float* sr_t = sSr + (tcount & 1) * BN;         // two buffers: tile parity
-            for (int c = tid; c < BN; c += kNPT) {
-                float v = 0.0f;
-                if (c < nrows) v = kGather ? a.s_row[a.sorted[row0 + c] / a.k] : a.s_row[row0 + c];
-                sr_t[c] = v;
-            }
-            const float rs = kSwiGLU
-                ? __ldg((lrow < 64 ? a.rs0 : a.rs1) + (int64_t)e * a.R0 + mt * 64 + (lrow & 63))
-                : __ldg(a.rs0 + (int64_t)e * a.R0 + mt * 128 + lrow);
-            const int tb = tcount & 1;
-            ws::wait(&t_full[tb], (tcount >> 1) & 1, abort);
-            tc::tc_fence_after();
-            ws::named_sync_math<kNPT>();                   // column scales visible
-            const uint32_t tcol = tmem + t_lane + tb * BN;
-#pragma unroll 1
-            for (int c0 = 0; c0 < nrows; c0 += kCh) {       // only the columns the MMA wrote
-                uint32_t v[kCh];
-                if constexpr (kCh == 32) tc::tmem_ld32(tcol + c0, *reinterpret_cast<uint32_t(*)[32]>(v));
-                else tc::tmem_ld16(tcol + c0, *reinterpret_cast<uint32_t(*)[16]>(v));
-                tc::tmem_wait_ld();
-                float val[kCh];
-#pragma unroll
-                for (int j = 0; j < kCh; ++j) val[j] = __fmul_rn(__fmul_rn(__uint_as_float(v[j]), rs), sr_t[c0 + j]);
-                if constexpr (kSwiGLU) {
-                    // gate rows finish the first half of the columns, up rows the second; each
-                    // hands the other the half it does not finish
-                    constexpr int kHalf = kCh / 2;
-                    const bool gate = lrow < 64;
-                    const int r64 = lrow & 63;
-#pragma unroll
-                    for (int j = 0; j < kHalf; ++j)
-                        sX[r64 * C::kXStride + (gate ? kHalf : 0) + j] = gate ? val[kHalf + j] : val[j];
-                    ws::named_sync_math<kNPT>();
-                    const int cm = c0 + (gate ? 0 : kHalf);
-                    const int n = mt * 64 + r64;
-                    float hv[kHalf];
-#pragma unroll
-                    for (int j = 0; j < kHalf; ++j) {
-                        const float other = sX[r64 * C::kXStride + (gate ? 0 : kHalf) + j];
-                        const float gv = gate ? val[j] : other;
-                        const float uv = gate ? other : val[kHalf + j];
-                        hv[j] = silu_fast(gv) * uv;
-                    }
-#pragma unroll
-                    for (int j = 0; j < kHalf; ++j)
-                        if (cm + j < nrows) a.out[(row0 + cm + j) * a.ldo + n] = hv[j];
-#pragma unroll
-                    for (int j = 0; j < kHalf; ++j) {
-                        const unsigned m = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(hv[j])));
-                        if (lane == 0 && cm + j < nrows) atomicMax(a.amax + row0 + cm + j, m);
-                    }
-                    ws::named_sync_math<kNPT>();           // exchange buffer free again
-                } else {
-                    const int m = mt * 128 + lrow;
-#pragma unroll
-                    for (int j = 0; j < kCh; ++j)
-                        if (c0 + j < nrows) a.out[(row0 + c0 + j) * a.ldo + m] = val[j];
-                }
-            }
-            tc::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&t_empty[tb]);
-
-            if constexpr (kFused) {
-                // The barrier orders every thread's stores before the counting threads' fences,
-                // and a fence is cumulative, so one fence per counted row suffices.
-                ws::named_sync_math<kNPT>();
-                if constexpr (kSwiGLU) {
-                    if (tid < nrows) {
-                        __threadfence();
-                        flag[tid] = atomicAdd(a.cnt + row0 + tid, 1u) == (unsigned)(m_tiles - 1);
-                    }
-                    ws::named_sync_math<kNPT>();
-                    for (int j = 0; j < nrows; ++j) {
-                        if (flag[j]) {
-                            __threadfence();
-                            const int64_t r = row0 + j;
-                            requant_row(a.out + r * a.ldo, a.ldo, __ldcg(a.amax + r), a.hq + r * a.ldo,
-                                        a.s_h + r, tid, kNPT, nullptr);
-                        }
-                    }
-                } else {
-                    const int m = mt * 128 + lrow;
-                    if (tid < nrows) {
-                        __threadfence();
-                        const int t = a.sorted[row0 + tid] / a.k;
-                        flag[tid] = atomicAdd(a.cnt + (int64_t)t * m_tiles + mt, 1u) == (unsigned)(a.k - 1) ? t : -1;
-                    }
-                    ws::named_sync_math<kNPT>();
-                    for (int j = 0; j < nrows; ++j) {
-                        const int t = flag[j];
-                        if (t >= 0) {
-                            __threadfence();
-                            float o = 0.0f;
-                            for (int jj = 0; jj < a.k; ++jj)
-                                o = __fadd_rn(o, __fmul_rn(a.gates[t * a.k + jj],
-                                                           __ldcg(a.out + (int64_t)a.rop[t * a.k + jj] * a.ldo + m)));
-                            if (a.shared) o = __fadd_rn(o, a.shared[(int64_t)t * a.ldo + m]);
-                            a.out_bf16[(int64_t)t * a.ldo + m] = f32_to_bf16_bits(o);
-                        }
-                    }
-                }
-                ws::named_sync_math<kNPT>();
-            }
-        }
+        w8_epilogue_warps<BN, kSwiGLU, kFused, kGather>(
+            a, n_tiles, m_tiles, pre, soff, sSr, sX, flag, tmem, t_full, t_empty, abort,
+            [&](int e, int mt, int lrow) {
+                return kSwiGLU ? __ldg((lrow < 64 ? a.rs0 : a.rs1) + (int64_t)e * a.R0 + mt * 64 + (lrow & 63))
+                               : __ldg(a.rs0 + (int64_t)e * a.R0 + mt * 128 + lrow);
+            });
     }
 
     __syncwarp();          // single-lane roles reconverge before the CTA-wide barrier

@@ -1,8 +1,10 @@
 """Convenience wrappers: torch allocation around the C entry points."""
 from __future__ import annotations
 
-from ._binding import (Layer, Layer8, moe_w4a8_forward, moe_w4a8_workspace_bytes, moe_w8a8_forward,
-                       moe_w8a8_workspace_bytes, w4a8_pack_weights, w8a8_quant_weights)
+from ._binding import (Layer, Layer4, Layer8, moe_nvfp4_forward, moe_nvfp4_workspace_bytes,
+                       moe_w4a8_forward, moe_w4a8_workspace_bytes, moe_w8a8_forward,
+                       moe_w8a8_workspace_bytes, nvfp4_quant_weights, w4a8_pack_weights,
+                       w8a8_quant_weights)
 
 
 def pack_expert_weights(w, group: int = 128, stream=None):
@@ -47,18 +49,45 @@ def make_layer_w8a8(gate_w, up_w, down_w, sh_gate=None, sh_up=None, sh_down=None
     return Layer8(E, H, N, gq, uq, dq, gs, us, ds, sh_gate=sh_gate, sh_up=sh_up, sh_down=sh_down)
 
 
+def quant_expert_weights_nvfp4(w, stream=None):
+    """bf16 weights [experts, rows, K] on the GPU -> (E2M1 codes uint8 [experts, rows, K/2],
+    E4M3 block scales uint8 [experts, rows, K/16], fp32 scale2 [experts])."""
+    import torch
+    E, rows, K = w.shape
+    codes = torch.empty(E, rows, K // 2, dtype=torch.uint8, device=w.device)
+    scales = torch.empty(E, rows, K // 16, dtype=torch.uint8, device=w.device)
+    s2 = torch.empty(E, dtype=torch.float32, device=w.device)
+    nvfp4_quant_weights(w.contiguous(), codes, scales, s2, stream=stream)
+    return codes, scales, s2
+
+
+def make_layer_nvfp4(gate_w, up_w, down_w, sh_gate=None, sh_up=None, sh_down=None,
+                     stream=None) -> Layer4:
+    """NVFP4-quantize bf16 expert weights gate/up [E, N, H], down [E, H, N]."""
+    E, N, H = gate_w.shape
+    g = quant_expert_weights_nvfp4(gate_w, stream=stream)
+    u = quant_expert_weights_nvfp4(up_w, stream=stream)
+    d = quant_expert_weights_nvfp4(down_w, stream=stream)
+    return Layer4(E, H, N, g[0], u[0], d[0], g[1], u[1], d[1], g[2], u[2], d[2],
+                  sh_gate=sh_gate, sh_up=sh_up, sh_down=sh_down)
+
+
 def alloc_workspace(layer, T: int, k: int, device=None):
     import torch
-    w8 = isinstance(layer, Layer8)
-    n = (moe_w8a8_workspace_bytes if w8 else moe_w4a8_workspace_bytes)(layer, T, k)
+    if isinstance(layer, Layer8):
+        n, ref = moe_w8a8_workspace_bytes(layer, T, k), layer.gate_w8
+    elif isinstance(layer, Layer4):
+        n, ref = moe_nvfp4_workspace_bytes(layer, T, k), layer.gate_f4
+    else:
+        n, ref = moe_w4a8_workspace_bytes(layer, T, k), layer.gate_packed
     if n == 0 and T > 0:
         raise ValueError("unsupported layer shape for the MoE forward")
-    dev = device if device is not None else (layer.gate_w8 if w8 else layer.gate_packed).device
+    dev = device if device is not None else ref.device
     return torch.empty(max(n, 256), dtype=torch.uint8, device=dev)
 
 
 def forward(layer, x, logits, k: int, out=None, ws=None, stream=None):
-    """The layer on x for either expert format (Layer: W4A8, Layer8: row-scaled FP8)."""
+    """The layer on x for any expert format (Layer: W4A8, Layer8: row-scaled FP8, Layer4: NVFP4)."""
     import torch
     if out is None:
         out = torch.empty_like(x)
@@ -66,6 +95,8 @@ def forward(layer, x, logits, k: int, out=None, ws=None, stream=None):
         ws = alloc_workspace(layer, x.shape[0], k, x.device)
     if isinstance(layer, Layer8):
         moe_w8a8_forward(layer, x, logits, k, out, ws, stream=stream)
+    elif isinstance(layer, Layer4):
+        moe_nvfp4_forward(layer, x, logits, k, out, ws, stream=stream)
     else:
         moe_w4a8_forward(layer, x, logits, k, out, ws, stream=stream)
     return out

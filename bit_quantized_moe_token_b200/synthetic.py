@@ -8,17 +8,21 @@ from __future__ import annotations
 
 import synth
 
-from ._binding import Layer, Layer8
-from .layer import pack_expert_weights, quant_expert_weights_w8a8
+from ._binding import Layer, Layer4, Layer8
+from .layer import pack_expert_weights, quant_expert_weights_nvfp4, quant_expert_weights_w8a8
 
 
-def _expert_tensors(wl, device, experts_per_chunk, w8):
+def _expert_tensors(wl, device, experts_per_chunk, w8=False, f4=False):
     import torch
     E = wl.E
     out = {}
     for proj in ("gate", "up", "down"):
         rows, K = synth.weight_shape(wl, proj)
-        if w8:
+        if f4:
+            p = torch.empty(E, rows, K // 2, dtype=torch.uint8, device=device)
+            s = torch.empty(E, rows, K // 16, dtype=torch.uint8, device=device)
+            s2 = torch.empty(E, dtype=torch.float32, device=device)
+        elif w8:
             p = torch.empty(E, rows, K, dtype=torch.uint8, device=device)
             s = torch.empty(E, rows, dtype=torch.float32, device=device)
         else:
@@ -29,10 +33,14 @@ def _expert_tensors(wl, device, experts_per_chunk, w8):
             n = min(experts_per_chunk, E - e0)
             for i in range(n):
                 synth.dev_weight(wl.seed, synth.weight_stream(e0 + i, proj), buf[i])
-            pp, ss = (quant_expert_weights_w8a8 if w8 else pack_expert_weights)(buf[:n])
+            if f4:
+                pp, ss, s22 = quant_expert_weights_nvfp4(buf[:n])
+                s2[e0:e0 + n].copy_(s22)
+            else:
+                pp, ss = (quant_expert_weights_w8a8 if w8 else pack_expert_weights)(buf[:n])
             p[e0:e0 + n].copy_(pp)
             s[e0:e0 + n].copy_(ss)
-        out[proj] = (p, s)
+        out[proj] = (p, s, s2) if f4 else (p, s)
         del buf
     return out
 
@@ -68,6 +76,16 @@ def device_layer_w8a8(wl: synth.Workload, device="cuda", experts_per_chunk: int 
     torch.cuda.synchronize()
     return Layer8(wl.E, wl.H, wl.N, q["gate"][0], q["up"][0], q["down"][0],
                   q["gate"][1], q["up"][1], q["down"][1], **sh)
+
+
+def device_layer_nvfp4(wl: synth.Workload, device="cuda", experts_per_chunk: int = 32) -> Layer4:
+    """The same seeded experts of workload `wl` in the NVFP4 format."""
+    import torch
+    q = _expert_tensors(wl, device, experts_per_chunk, f4=True)
+    sh = _shared_tensors(wl, device)
+    torch.cuda.synchronize()
+    return Layer4(wl.E, wl.H, wl.N, q["gate"][0], q["up"][0], q["down"][0], q["gate"][1], q["up"][1],
+                  q["down"][1], q["gate"][2], q["up"][2], q["down"][2], **sh)
 
 
 def device_inputs(wl: synth.Workload, device="cuda", t0: int = 0, T: int | None = None):

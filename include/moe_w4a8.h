@@ -272,6 +272,66 @@ int moe_w8a8_forward_profiled(const moe_w8a8_layer* layer, const uint16_t* x_bf1
                               void* ws, size_t ws_bytes, moe_stream_t stream,
                               void* const* events, int n_events, int* n_launches);
 
+/* ---------------------------------------------------------------------------------------
+ * NVFP4 experts: a third weight format on the same layer.
+ *
+ * Storage as the "Inkling-512k-NVFP4-AQLM-hybrid" card specifies for its hot experts ("On-disk
+ * tensor format", "Dequant math"): two E2M1 (FP4) codes per byte, the first weight of a pair in
+ * the low nibble; one E4M3 scale per block of 16 input weights; one fp32 scale2 per expert
+ * projection; W = LUT[code] * scale * scale2 with LUT = 0, .5, 1, 1.5, 2, 3, 4, 6 for codes
+ * 0..7 and their negatives for 8..15.
+ *
+ * nvfp4_quant_weights quantizes `experts` bf16 projections [experts, rows, K] (the card's slabs
+ * come from an NVFP4 base; this is the usual two-level recipe):
+ *     scale2[e] = max |w_e| / (6 * 448)
+ *     scale[e, r, b] = e4m3_rn_satfinite(max_{block b} |w| / (6 * scale2[e]))
+ *     code = nearest E2M1 value of w / (dec(scale) * scale2[e]), ties to the even code,
+ *            at most +-6, the sign kept (a zero scale gives codes 0)
+ *   codes    [experts, rows, K/2] uint8 out, 8-byte aligned
+ *   scales   [experts, rows, K/16] E4M3 out
+ *   scale2   [experts] fp32 out (also used as scratch during the call)
+ * K must be a multiple of 16.  Returns as w4a8_pack_weights.
+ * --------------------------------------------------------------------------------------- */
+int nvfp4_quant_weights(const uint16_t* w_bf16, int64_t experts, int64_t rows, int64_t K,
+                        uint8_t* codes, uint8_t* scales, float* scale2, moe_stream_t stream);
+
+/* The layer with NVFP4 routed experts (gate and up separate):
+ *   gate_f4, up_f4  [E, N, H/2]    gate_bs, up_bs  [E, N, H/16] E4M3    gate_s2, up_s2  [E] fp32
+ *   down_f4         [E, H, N/2]    down_bs         [E, H, N/16] E4M3    down_s2         [E] fp32
+ * (codes 16-byte aligned, block scales 8-byte aligned); shared experts as in moe_w4a8_layer. */
+typedef struct {
+    int E, H, N;
+    const uint8_t *gate_f4, *up_f4, *down_f4;
+    const uint8_t *gate_bs, *up_bs, *down_bs;
+    const float *gate_s2, *up_s2, *down_s2;
+    int n_shared, shared_N;
+    const uint16_t *sh_gate, *sh_up, *sh_down;
+} moe_nvfp4_layer;
+
+/* Workspace of moe_nvfp4_forward: the W4A8 plan plus f16 copies of the GEMM inputs
+ * (T*k * max(H, N) * 2 bytes); the layout offsets are the W4A8 layer's. */
+size_t moe_nvfp4_workspace_bytes(const moe_nvfp4_layer* layer, int64_t T, int k);
+int moe_nvfp4_workspace_layout(const moe_nvfp4_layer* layer, int64_t T, int k,
+                               moe_w4a8_ws_layout* out);
+
+/*
+ * The layer of moe_w4a8_forward with each projection on NVFP4 weights and the same per-token
+ * FP8 activations:
+ *   G[n] = (sum_k Xq[t,k] * W_gate[e,n,k]) * s_x[t]        (likewise U), W as dequantized above
+ *   h = silu(G) * U;   s_h = max|h| / 448;   Hq = e4m3(h / s_h)
+ *   Y[m] = (sum_n Hq[n] * W_down[e,m,n]) * s_h
+ * The GPU computes each sum as (sum_k f16(LUT[code] * scale) * f16(dec Xq)) * scale2 (exact
+ * products, fp32 accumulation in the tensor core's order).  Same shapes and return codes as
+ * moe_w4a8_forward; the profiled variant records the same stage events.
+ */
+int moe_nvfp4_forward(const moe_nvfp4_layer* layer, const uint16_t* x_bf16,
+                      const float* router_logits, int64_t T, int k, uint16_t* out_bf16, void* ws,
+                      size_t ws_bytes, moe_stream_t stream);
+int moe_nvfp4_forward_profiled(const moe_nvfp4_layer* layer, const uint16_t* x_bf16,
+                               const float* router_logits, int64_t T, int k, uint16_t* out_bf16,
+                               void* ws, size_t ws_bytes, moe_stream_t stream,
+                               void* const* events, int n_events, int* n_launches);
+
 /* The layer fed by the router weight instead of precomputed logits: the router logits
  * (moe_router_logits' definition, written into the workspace), then the layer of
  * moe_w4a8_forward / moe_w8a8_forward on them.  At decode sizes (T <= 16) the router, the
@@ -284,6 +344,9 @@ int moe_w4a8_forward_router(const moe_w4a8_layer* layer, const uint16_t* x_bf16,
 int moe_w8a8_forward_router(const moe_w8a8_layer* layer, const uint16_t* x_bf16,
                             const uint16_t* wr_bf16, int64_t T, int k, uint16_t* out_bf16,
                             void* ws, size_t ws_bytes, moe_stream_t stream);
+int moe_nvfp4_forward_router(const moe_nvfp4_layer* layer, const uint16_t* x_bf16,
+                             const uint16_t* wr_bf16, int64_t T, int k, uint16_t* out_bf16,
+                             void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /* Waits for `stream`, then returns and clears the library's sticky device-status word for
  * the current device: MOE_OK, or MOE_ERR_TIMEOUT when a bounded device-side wait gave up

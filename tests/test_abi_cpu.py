@@ -30,6 +30,8 @@ def test_header_declares_the_boundary():
               "moe_router_logits", "w8a8_quant_weights", "moe_w8a8_forward",
               "moe_w8a8_workspace_bytes", "moe_w8a8_forward_profiled", "moe_router_topk",
               "moe_router_topk_workspace_bytes", "moe_w4a8_forward_router", "moe_w8a8_forward_router",
+              "nvfp4_quant_weights", "moe_nvfp4_forward", "moe_nvfp4_workspace_bytes",
+              "moe_nvfp4_forward_profiled", "moe_nvfp4_forward_router",
               "moe_w4a8_workspace_bytes", "moe_last_device_status", "moe_status_string"):
         assert n in names
 
@@ -177,6 +179,28 @@ def test_w8a8_rejects_bad_args():
     assert L.moe_w8a8_forward(ctypes.byref(odd), p, p, 4, 2, p, p, need, None) == -3
     assert L.moe_w8a8_forward(ctypes.byref(full), p, p, 0, 2, p, p, need, None) == 0
     assert L.moe_w8a8_forward(None, p, p, 4, 2, p, p, need, None) == -1
+
+
+def test_nvfp4_rejects_bad_args():
+    L = _L()
+    p = ctypes.c_void_p(4096)
+    assert L.nvfp4_quant_weights(p, 2, 4, 24, p, p, p, None) == -2        # K % 16
+    assert L.nvfp4_quant_weights(None, 2, 4, 32, p, p, p, None) == -1
+    assert L.nvfp4_quant_weights(p, 0, 4, 32, p, p, p, None) == 0
+    assert L.nvfp4_quant_weights(p, 2, 4, 32, ctypes.c_void_p(4100), p, p, None) == -3
+    s4 = moe.layer4_struct(256, 4096, 2048)
+    n4 = moe.moe_nvfp4_workspace_bytes(s4, 64, 6)
+    assert n4 > moe.moe_w4a8_workspace_bytes(moe.layer_struct(256, 4096, 2048), 64, 6)
+    assert moe.moe_nvfp4_workspace_layout(s4, 64, 6)["total"] == n4
+    full = moe._binding._CLayer4(8, 256, 128, p, p, p, p, p, p, p, p, p, 0, 0, None, None, None)
+    need = moe.moe_nvfp4_workspace_bytes(full, 4, 2)
+    assert L.moe_nvfp4_forward(ctypes.byref(full), p, p, 4, 2, p, p, need - 1, None) == -4
+    odd = moe._binding._CLayer4(8, 256, 128, p, p, p, ctypes.c_void_p(4100), p, p, p, p, p, 0, 0, None,
+                                None, None)                           # block scales need 8 bytes
+    assert L.moe_nvfp4_forward(ctypes.byref(odd), p, p, 4, 2, p, p, need, None) == -3
+    nos2 = moe._binding._CLayer4(8, 256, 128, p, p, p, p, p, p, None, p, p, 0, 0, None, None, None)
+    assert L.moe_nvfp4_forward(ctypes.byref(nos2), p, p, 4, 2, p, p, need, None) == -1
+    assert L.moe_nvfp4_forward(ctypes.byref(full), p, p, 0, 2, p, p, need, None) == 0
 
 
 def test_binding_has_no_fallback():

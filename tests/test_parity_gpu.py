@@ -13,7 +13,8 @@ pytestmark = pytest.mark.gpu
 if cuda_ok():
     import torch
     import bit_quantized_moe_token_b200 as moe
-    from bit_quantized_moe_token_b200.synthetic import device_inputs, device_layer, device_layer_w8a8
+    from bit_quantized_moe_token_b200.synthetic import (device_inputs, device_layer, device_layer_nvfp4,
+                                                        device_layer_w8a8)
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -34,7 +35,8 @@ def bits(t):
 
 
 def ws_views(layer, ws, T, k):
-    layout = moe.moe_w8a8_workspace_layout if isinstance(layer, moe.Layer8) else moe.moe_w4a8_workspace_layout
+    layout = (moe.moe_w8a8_workspace_layout if isinstance(layer, moe.Layer8) else
+              moe.moe_nvfp4_workspace_layout if isinstance(layer, moe.Layer4) else moe.moe_w4a8_workspace_layout)
     lay = layout(layer, T, k)
     P = T * k
     b = ws.cpu().numpy()
@@ -354,14 +356,16 @@ def test_router_topk_fused(T, E, H, k):
     assert np.all(np.abs(g.astype(np.float64) - ref) <= bound)
 
 
-@pytest.mark.parametrize("w8", [False, True])
+@pytest.mark.parametrize("w8", [False, True, "nvfp4"])
 @pytest.mark.parametrize("E,H,N,k,T", [(16, 256, 128, 2, 8), (16, 256, 128, 2, 40),
                                        (16, 256, 128, 2, 300), (128, 256, 128, 2, 300)])
 def test_forward_router_matches_logits_path(w8, E, H, N, k, T):
     """The layer fed by the router weight equals, bit for bit, the layer fed by the logits that
     moe_router_logits computes (decode front: router + quantization + top-k in one kernel;
     16 < T: fused router + top-k, then quantization; E = 128, T = 300: tensor-core router)."""
-    hl, dl = (_host_layer_and_dev_w8a8 if w8 else _host_layer_and_dev)(E, H, N, seed=30 + E + T)
+    make = (_host_layer_and_dev_nvfp4 if w8 == "nvfp4" else _host_layer_and_dev_w8a8 if w8
+            else _host_layer_and_dev)
+    hl, dl = make(E, H, N, seed=30 + E + T)
     x = synth.normal_bf16(8, 870 + T, T * H).reshape(T, H)
     wr = synth.normal_bf16(8, 871 + E, E * H, 1.0 / np.sqrt(H)).reshape(E, H)
     xd, wd = to_dev_bf16(x), to_dev_bf16(wr)
@@ -370,7 +374,8 @@ def test_forward_router_matches_logits_path(w8, E, H, N, k, T):
     ws_a, ws_b = moe.alloc_workspace(dl, T, k), moe.alloc_workspace(dl, T, k)
     out_a = moe.forward(dl, xd, lg, k, ws=ws_a)
     out_b = torch.empty_like(out_a)
-    (moe.moe_w8a8_forward_router if w8 else moe.moe_w4a8_forward_router)(dl, xd, wd, k, out_b, ws_b)
+    (moe.moe_nvfp4_forward_router if w8 == "nvfp4" else moe.moe_w8a8_forward_router if w8
+     else moe.moe_w4a8_forward_router)(dl, xd, wd, k, out_b, ws_b)
     torch.cuda.synchronize()
     assert moe.moe_last_device_status() == 0
     assert np.array_equal(bits(out_a), bits(out_b))
@@ -585,6 +590,125 @@ def test_w8a8_forward_full_size_sampled(name, full_layer_w8a8):
     for e in experts[:3]:
         assert np.array_equal(dl.gate_w8[e].cpu().numpy(), hl.gate_w8[e])
         assert np.array_equal(dl.down_rs[e].cpu().numpy(), hl.down_rs[e])
+    ref = oracle.moe_forward(hl, xs, ls, wl.k)
+    assert np.array_equal(v["ids"][toks], ref["ids"])
+    gpu_rows = v["row_of_pair"].reshape(wl.T, wl.k)[toks].reshape(-1)
+    assert np.array_equal(v["xq"][toks], ref["xq"])
+    check_fp8_codes(v["hq"][gpu_rows], ref["hq"][ref["row_of_pair"]])
+    np.testing.assert_allclose(v["s_h"][gpu_rows], ref["s_h"][ref["row_of_pair"]], rtol=2e-5)
+    check_output(outb[toks], ref["out"])
+
+
+# ---- NVFP4 experts -------------------------------------------------------------------------------
+
+def test_nvfp4_quant_weights_bitexact():
+    rng = np.random.default_rng(41)
+    E, rows, K = 3, 100, 512
+    w = (rng.standard_normal((E, rows, K)) * 0.02 * 2.0 ** rng.uniform(-5, 5, (E, rows, 1))).astype(np.float32)
+    w[0, 4, 32:48] = 0.0                               # a zero block
+    w[1, 7, :16] = [6, 3, 1.25, -0.75, 0.25, -6, 0, 2.5, 5, -1.75, 0.5, 4, -3.5, 1, 0, 0]  # ties
+    w[2] = 0.0                                         # a zero expert: scale2 0, everything 0
+    wb = _f32_to_bf16_bits(w)
+    codes = torch.empty(E, rows, K // 2, dtype=torch.uint8, device="cuda")
+    scales = torch.empty(E, rows, K // 16, dtype=torch.uint8, device="cuda")
+    s2 = torch.empty(E, dtype=torch.float32, device="cuda")
+    moe.nvfp4_quant_weights(to_dev_bf16(wb), codes, scales, s2)
+    torch.cuda.synchronize()
+    for e in range(E):
+        c_ref, s_ref, s2_ref = oracle.nvfp4_quant(wb[e])
+        assert np.array_equal(codes[e].cpu().numpy(), c_ref), e
+        assert np.array_equal(scales[e].cpu().numpy(), s_ref), e
+        assert s2[e].item() == s2_ref, e
+
+
+def _host_layer_and_dev_nvfp4(E, H, N, seed, n_shared=0, shared_N=0):
+    """Seeded random layer, rows scaled over 2^-4..2^4: NVFP4-quantized on the host by the oracle
+    and on the GPU by the library."""
+    rng_stream = 70_000 + seed * 10
+    def w(stream, rows, K):
+        a = synth.normal_f32(seed, stream, E * rows * K, 0.02).reshape(E, rows, K)
+        scale = 2.0 ** np.round(synth.normal_f32(seed, stream + 5, E * rows).reshape(E, rows, 1) * 1.5)
+        return _f32_to_bf16_bits((a * scale).astype(np.float32))
+    gw, uw, dw = w(rng_stream, N, H), w(rng_stream + 1, N, H), w(rng_stream + 2, H, N)
+    def qp(W):
+        r = [oracle.nvfp4_quant(W[e]) for e in range(E)]
+        return (np.stack([a for a, _, _ in r]), np.stack([b for _, b, _ in r]),
+                np.array([c for _, _, c in r], np.float32))
+    g, u, d = qp(gw), qp(uw), qp(dw)
+    sh, shd = {}, {}
+    if n_shared:
+        for i, key in enumerate(("sh_gate", "sh_up", "sh_down")):
+            shape = (n_shared, shared_N, H) if i < 2 else (n_shared, H, shared_N)
+            a = synth.normal_bf16(seed, rng_stream + 3 + i, int(np.prod(shape)), 0.02).reshape(shape)
+            sh[key] = a
+            shd[key] = to_dev_bf16(a)
+    hl = oracle.Layer.nvfp4(E, H, N, g[0], u[0], d[0], g[1], u[1], d[1], g[2], u[2], d[2], **sh)
+    dl = moe.make_layer_nvfp4(to_dev_bf16(gw), to_dev_bf16(uw), to_dev_bf16(dw), **shd)
+    torch.cuda.synchronize()
+    assert np.array_equal(dl.gate_f4.cpu().numpy(), g[0])
+    assert np.array_equal(dl.down_bs.cpu().numpy(), d[1])
+    assert np.array_equal(dl.up_s2.cpu().numpy(), u[2])
+    return hl, dl
+
+
+def test_nvfp4_forward_tiny_workload():
+    wl = synth.WORKLOADS["tiny"]
+    hl = oracle.quant_workload_layer_nvfp4(wl)
+    dl = device_layer_nvfp4(wl)
+    assert np.array_equal(dl.up_f4.cpu().numpy(), hl.up_f4)
+    assert np.array_equal(dl.down_s2.cpu().numpy(), hl.down_s2)
+    r1 = _run_and_compare(hl, dl, synth.tokens(wl), synth.logits(wl), wl.k)
+    r2 = _run_and_compare(hl, dl, synth.tokens(wl), synth.logits(wl), wl.k)
+    assert np.array_equal(r1["out"], r2["out"])
+
+
+@pytest.mark.parametrize("E,H,N,k,T", [(5, 384, 256, 3, 37), (1, 256, 128, 1, 9), (8, 256, 128, 2, 1),
+                                       (8, 256, 256, 2, 200), (16, 512, 384, 8, 130),
+                                       (3, 1024, 128, 2, 700), (64, 1024, 1024, 6, 16)])
+def test_nvfp4_forward_ragged_shapes(E, H, N, k, T):
+    hl, dl = _host_layer_and_dev_nvfp4(E, H, N, seed=E * 7 + T)
+    x = synth.normal_bf16(3, 777 + T, T * H).reshape(T, H)
+    logits = synth.normal_f32(3, 778 + T, T * E).reshape(T, E)
+    _run_and_compare(hl, dl, x, logits, k)
+
+
+def test_nvfp4_forward_shared_experts():
+    hl, dl = _host_layer_and_dev_nvfp4(4, 256, 128, seed=5, n_shared=2, shared_N=256)
+    T = 21
+    x = synth.normal_bf16(4, 901, T * 256).reshape(T, 256)
+    logits = synth.normal_f32(4, 902, T * 4).reshape(T, 4)
+    _run_and_compare(hl, dl, x, logits, 2)
+
+
+@pytest.fixture(scope="module")
+def full_layer_nvfp4():
+    return device_layer_nvfp4(synth.WORKLOADS["prefill_t16384_shared"])
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_nvfp4_forward_full_size_sampled(name, full_layer_nvfp4):
+    wl = synth.WORKLOADS[name]
+    dl = full_layer_nvfp4
+    if not wl.n_shared:
+        dl = moe.Layer4(dl.E, dl.H, dl.N, dl.gate_f4, dl.up_f4, dl.down_f4, dl.gate_bs, dl.up_bs, dl.down_bs,
+                        dl.gate_s2, dl.up_s2, dl.down_s2)
+    x, lg = device_inputs(wl)
+    ws = moe.alloc_workspace(dl, wl.T, wl.k)
+    out = moe.forward(dl, x, lg, wl.k, ws=ws)
+    torch.cuda.synchronize()
+    assert moe.moe_last_device_status() == 0
+    v = ws_views(dl, ws, wl.T, wl.k)
+    outb = bits(out)
+    assert np.isfinite(bf16_to_f32(outb)).all()
+    toks = _sample_tokens(wl)
+    xs = np.stack([synth.tokens(wl, t, 1)[0] for t in toks])
+    ls = np.stack([synth.logits(wl, t, 1)[0] for t in toks])
+    ids_ref, _ = oracle.route_topk(ls, wl.k)
+    experts = sorted(set(ids_ref.reshape(-1).tolist()))
+    hl = oracle.quant_workload_layer_nvfp4(wl, experts=experts)
+    for e in experts[:3]:
+        assert np.array_equal(dl.gate_f4[e].cpu().numpy(), hl.gate_f4[e])
+        assert np.array_equal(dl.down_bs[e].cpu().numpy(), hl.down_bs[e])
     ref = oracle.moe_forward(hl, xs, ls, wl.k)
     assert np.array_equal(v["ids"][toks], ref["ids"])
     gpu_rows = v["row_of_pair"].reshape(wl.T, wl.k)[toks].reshape(-1)
