@@ -99,6 +99,8 @@ def lib():
         L.or_moe_forward.restype = i32
         L.or_moe_forward_dense.argtypes = [ctypes.POINTER(_Layer), vp, vp, i64, i32, vp, vp, vp,
                                            vp, vp]
+        L.or_moe_forward_given_h.argtypes = [ctypes.POINTER(_Layer), vp, vp, i64, i32, vp, vp, vp, vp]
+        L.or_moe_forward_given_h.restype = i32
         L.or_moe_forward_dense.restype = i32
         _lib = L
     return _lib
@@ -320,6 +322,24 @@ def moe_forward(layer: Layer, x_bf16: np.ndarray, logits: np.ndarray, k: int):
     if rc != 0:
         raise ValueError("or_moe_forward: bad shape")
     return r
+
+
+def moe_forward_given_h(layer: Layer, x_bf16: np.ndarray, logits: np.ndarray, k: int,
+                        hq_pairs: np.ndarray, sh_pairs: np.ndarray):
+    """The layer's output with the requantized SwiGLU activations given in pair order
+    (hq_pairs [T*k, N] E4M3, sh_pairs [T*k]): S6-S8 on them.  Returns (out bf16, out_f32)."""
+    x = np.ascontiguousarray(x_bf16, np.uint16)
+    l = np.ascontiguousarray(logits, np.float32)
+    hq = np.ascontiguousarray(hq_pairs, np.uint8)
+    sh = np.ascontiguousarray(sh_pairs, np.float32)
+    T, H = x.shape
+    out = np.zeros((T, H), np.uint16)
+    out_f32 = np.zeros((T, H), np.float32)
+    L = layer._c()
+    if lib().or_moe_forward_given_h(ctypes.byref(L), _p(x), _p(l), T, k, _p(hq), _p(sh), _p(out),
+                                    _p(out_f32)) != 0:
+        raise ValueError("or_moe_forward_given_h: bad shape")
+    return out, out_f32
 
 
 def moe_forward_dense(layer: Layer, x_bf16: np.ndarray, logits: np.ndarray, k: int):

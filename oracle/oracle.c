@@ -439,6 +439,10 @@ static void f4_proj(const uint8_t* q, float s_x, const float* cT, int64_t rows, 
 
 static float silu_f32(float g) { return g * (1.0f / (1.0f + expf(-g))); }
 
+/* Set only inside or_moe_forward_given_h: the expert rows take their requantized SwiGLU
+ * activations (S5) as given instead of computing them, and run the down projection on them. */
+static int g_given_h = 0;
+
 /*
  * One routed row: token row q/s_x through expert weights (already unpacked), giving the
  * FP8 SwiGLU activations (hq, s_h) and the down-projection output y[H].
@@ -452,10 +456,12 @@ static void expert_row(const uint8_t* q, float s_x, const float* cg, const float
     float* h = U + N;                 /* N */
     float* part = h + N;              /* max(N,H) */
     float* acc = part + (H > N ? H : N);
-    w4a8_proj(q, s_x, cg, sg, N, H, group, G, part, acc);
-    w4a8_proj(q, s_x, cu, su, N, H, group, U, part, acc);
-    for (int64_t n = 0; n < N; ++n) h[n] = silu_f32(G[n]) * U[n];
-    quant_row_f32(h, N, hq, s_h);
+    if (!g_given_h) {
+        w4a8_proj(q, s_x, cg, sg, N, H, group, G, part, acc);
+        w4a8_proj(q, s_x, cu, su, N, H, group, U, part, acc);
+        for (int64_t n = 0; n < N; ++n) h[n] = silu_f32(G[n]) * U[n];
+        quant_row_f32(h, N, hq, s_h);
+    }
     w4a8_proj(hq, *s_h, cd, sd, H, N, group, y, part, acc);
 }
 
@@ -467,10 +473,12 @@ static void expert_row_w8(const uint8_t* q, float s_x, const float* cg, const fl
     float* U = G + N;
     float* h = U + N;
     float* acc = h + N;
-    w8a8_proj(q, s_x, cg, rg, N, H, G, acc);
-    w8a8_proj(q, s_x, cu, ru, N, H, U, acc);
-    for (int64_t n = 0; n < N; ++n) h[n] = silu_f32(G[n]) * U[n];
-    quant_row_f32(h, N, hq, s_h);
+    if (!g_given_h) {
+        w8a8_proj(q, s_x, cg, rg, N, H, G, acc);
+        w8a8_proj(q, s_x, cu, ru, N, H, U, acc);
+        for (int64_t n = 0; n < N; ++n) h[n] = silu_f32(G[n]) * U[n];
+        quant_row_f32(h, N, hq, s_h);
+    }
     w8a8_proj(hq, *s_h, cd, rd, H, N, y, acc);
 }
 
@@ -482,10 +490,12 @@ static void expert_row_f4(const uint8_t* q, float s_x, const float* cg, const fl
     float* U = G + N;
     float* h = U + N;
     float* acc = h + N;
-    f4_proj(q, s_x, cg, N, H, G, acc);
-    f4_proj(q, s_x, cu, N, H, U, acc);
-    for (int64_t n = 0; n < N; ++n) h[n] = silu_f32(G[n]) * U[n];
-    quant_row_f32(h, N, hq, s_h);
+    if (!g_given_h) {
+        f4_proj(q, s_x, cg, N, H, G, acc);
+        f4_proj(q, s_x, cu, N, H, U, acc);
+        for (int64_t n = 0; n < N; ++n) h[n] = silu_f32(G[n]) * U[n];
+        quant_row_f32(h, N, hq, s_h);
+    }
     f4_proj(hq, *s_h, cd, H, N, y, acc);
 }
 
@@ -516,10 +526,42 @@ static void shared_expert_add(const float* x, const uint16_t* wg, const uint16_t
  *   hq [P,N], s_h [P], y [P,H] fp32, out_f32 [T,H] (sum before the bf16 rounding).
  * Returns 0, or -1 on a bad shape.
  */
+static int moe_forward_impl(const or_layer* L, const uint16_t* x, const float* logits, int64_t T,
+                            int k, uint16_t* out, int32_t* ids_o, float* gates_o, int32_t* offsets_o,
+                            int32_t* sorted_o, int32_t* rop_o, uint8_t* xq_o, float* sx_o,
+                            uint8_t* hq_o, float* sh_o, float* y_o, float* out_f32_o,
+                            const uint8_t* hq_pairs, const float* sh_pairs);
+
 int or_moe_forward(const or_layer* L, const uint16_t* x, const float* logits, int64_t T, int k,
                    uint16_t* out, int32_t* ids_o, float* gates_o, int32_t* offsets_o,
                    int32_t* sorted_o, int32_t* rop_o, uint8_t* xq_o, float* sx_o, uint8_t* hq_o,
                    float* sh_o, float* y_o, float* out_f32_o) {
+    return moe_forward_impl(L, x, logits, T, k, out, ids_o, gates_o, offsets_o, sorted_o, rop_o, xq_o,
+                            sx_o, hq_o, sh_o, y_o, out_f32_o, NULL, NULL);
+}
+
+/*
+ * The layer with the requantized SwiGLU activations given (test infrastructure for the parity
+ * rules): hq_pairs [T*k, N] and sh_pairs [T*k] in pair order p = t*k + j replace S5's result,
+ * and the down projection (S6) and combine (S7, S8) run on them.  Lets a test evaluate the
+ * oracle's output on another implementation's requantized codes, so that an output difference
+ * caused by a permitted FP8 code difference can be told from one that is not.
+ */
+int or_moe_forward_given_h(const or_layer* L, const uint16_t* x, const float* logits, int64_t T,
+                           int k, const uint8_t* hq_pairs, const float* sh_pairs, uint16_t* out,
+                           float* out_f32_o) {
+    g_given_h = 1;
+    int rc = moe_forward_impl(L, x, logits, T, k, out, NULL, NULL, NULL, NULL, NULL, NULL, NULL,
+                              NULL, NULL, NULL, out_f32_o, hq_pairs, sh_pairs);
+    g_given_h = 0;
+    return rc;
+}
+
+static int moe_forward_impl(const or_layer* L, const uint16_t* x, const float* logits, int64_t T,
+                            int k, uint16_t* out, int32_t* ids_o, float* gates_o, int32_t* offsets_o,
+                            int32_t* sorted_o, int32_t* rop_o, uint8_t* xq_o, float* sx_o,
+                            uint8_t* hq_o, float* sh_o, float* y_o, float* out_f32_o,
+                            const uint8_t* hq_pairs, const float* sh_pairs) {
     const int64_t H = L->H, N = L->N, E = L->E;
     const int group = L->group;
     if (H % group || N % group || k < 1 || k > E) return -1;
@@ -540,6 +582,12 @@ int or_moe_forward(const or_layer* L, const uint16_t* x, const float* logits, in
     or_quant_tokens(x, T, H, xq, sx);
     or_route_topk(logits, T, (int)E, k, ids, gates);
     or_permute(ids, T, k, (int)E, offsets, sorted, rop);
+    if (hq_pairs) {                      /* S5's result given, pair order -> sorted rows */
+        for (int64_t pp = 0; pp < P; ++pp) {
+            memcpy(hq + (int64_t)rop[pp] * N, hq_pairs + pp * N, (size_t)N);
+            sh[rop[pp]] = sh_pairs[pp];
+        }
+    }
 
     /* S4..S6, one expert segment at a time (experts are independent) */
     const int64_t G_h = H / group, G_n = N / group;

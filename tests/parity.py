@@ -7,7 +7,13 @@
 3. Each bf16 output element within 1e-2 * max(|ref|, rms(ref row)).
 
 Where fp32 arithmetic decides an integer (an FP8 code after a GPU sum with a different
-accumulation order than the oracle's), rule 2 is what allows the difference.
+accumulation order than the oracle's), rule 2 is what allows the difference.  Such a permitted
+code difference propagates into the outputs of its token (one E4M3 step of a large activation,
+through a short down projection, can move an output by more than rule 3's tolerance), so rule 3
+is applied with that allowance: an output outside the tolerance of the oracle's passes only if
+its token has a requantized code that differs from the oracle's and the output is within the
+tolerance of the oracle's layer evaluated on the GPU's requantized codes (the oracle's own down
+projection and combine, see oracle.moe_forward_given_h).
 """
 import numpy as np
 
@@ -45,3 +51,18 @@ def check_output(got_bf16: np.ndarray, ref_bf16: np.ndarray, rtol=OUT_RTOL):
     assert not bad.any(), (f"{int(bad.sum())} outputs out of tolerance; worst "
                            f"{float((err / np.maximum(tol, 1e-30)).max()):.3f}x tol")
     return float((err / np.maximum(np.maximum(np.abs(r), rms), 1e-30)).max())
+
+
+def check_output_explained(got_bf16, ref_bf16, alt_bf16, flipped_tokens, rtol=OUT_RTOL):
+    """Rule 3 with rule 2's allowance (module docstring).  alt_bf16: the oracle's output on the
+    GPU's requantized codes; flipped_tokens: bool [T], tokens with a differing code."""
+    g = bf16_to_f32(got_bf16).astype(np.float64)
+    out = []
+    for ref in (ref_bf16, alt_bf16):
+        r = bf16_to_f32(ref).astype(np.float64)
+        rms = np.sqrt((r ** 2).mean(axis=1, keepdims=True))
+        out.append(np.abs(g - r) <= rtol * np.maximum(np.abs(r), rms))
+    ok_ref, ok_alt = out
+    ok = ok_ref | (ok_alt & np.asarray(flipped_tokens, bool)[:, None])
+    assert ok.all(), f"{int((~ok).sum())} outputs out of tolerance (not explained by permitted code flips)"
+    return int((~ok_ref).sum())

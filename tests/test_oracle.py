@@ -695,6 +695,49 @@ def test_nvfp4_dense_brute_force_matches_permuted():
 
 
 # ------------------------------------------------------------------------------------------------
+# rule 3 with rule 2's allowance (tests/parity.py)
+# ------------------------------------------------------------------------------------------------
+
+def test_given_h_reproduces_the_forward():
+    wl = synth.WORKLOADS["tiny"]
+    for layer in (oracle.pack_workload_layer(wl), oracle.quant_workload_layer_nvfp4(wl)):
+        x, lg = synth.tokens(wl), synth.logits(wl)
+        r = oracle.moe_forward(layer, x, lg, wl.k)
+        out, out_f32 = oracle.moe_forward_given_h(layer, x, lg, wl.k, r["hq"][r["row_of_pair"]],
+                                                  r["s_h"][r["row_of_pair"]])
+        assert np.array_equal(out, r["out"]) and np.array_equal(out_f32, r["out_f32"])
+
+
+def test_planted_code_flip_is_local_and_only_explained_for_its_token():
+    from parity import check_output, check_output_explained
+    wl = synth.WORKLOADS["tiny"]
+    layer = oracle.pack_workload_layer(wl)
+    x, lg = synth.tokens(wl), synth.logits(wl)
+    r = oracle.moe_forward(layer, x, lg, wl.k)
+    hq = r["hq"][r["row_of_pair"]].copy()
+    sh = r["s_h"][r["row_of_pair"]].copy()
+    t = 5
+    p = t * wl.k
+    n = int(np.argmax(oracle.e4m3_decode_table()[hq[p]]))   # the largest code of the row
+    hq[p, n] += 1 if hq[p, n] & 0x7F < 0x7E else -1         # one E4M3 step
+    alt, _ = oracle.moe_forward_given_h(layer, x, lg, wl.k, hq, sh)
+    changed = (alt != r["out"]).any(axis=1)
+    assert changed[t] and changed.sum() == 1                  # only the token of the flipped row
+    flipped = np.zeros(wl.T, bool)
+    flipped[t] = True
+    check_output_explained(alt, r["out"], alt, flipped)       # explained by its own flip
+    # the same outputs with the allowance withheld: fail unless already within tolerance
+    within = True
+    try:
+        check_output(alt, r["out"])
+    except AssertionError:
+        within = False
+    if not within:
+        with pytest.raises(AssertionError):
+            check_output_explained(alt, r["out"], alt, np.zeros(wl.T, bool))
+
+
+# ------------------------------------------------------------------------------------------------
 # the generator (input recipe)
 # ------------------------------------------------------------------------------------------------
 

@@ -6,7 +6,7 @@ import pytest
 import oracle
 import synth
 from conftest import cuda_ok
-from parity import bf16_to_f32, check_fp8_codes, check_output
+from parity import bf16_to_f32, check_fp8_codes, check_output, check_output_explained
 
 pytestmark = pytest.mark.gpu
 
@@ -196,6 +196,20 @@ def _host_layer_and_dev(E, H, N, seed, n_shared=0, shared_N=0):
     return hl, dl
 
 
+def _check_output_rules(hl, x, logits, k, got_out, ref, gpu_hq_pairs, gpu_sh_pairs):
+    """Rule 3, with rule 2's allowance for outputs of tokens whose requantized codes differ
+    (tests/parity.py): returns the number of outputs that needed the allowance."""
+    try:
+        check_output(got_out, ref["out"])
+        return 0
+    except AssertionError:
+        T = x.shape[0]
+        ref_pairs = ref["hq"][ref["row_of_pair"]]
+        flipped = (gpu_hq_pairs != ref_pairs).reshape(T, -1).any(axis=1)
+        alt, _ = oracle.moe_forward_given_h(hl, x, logits, k, gpu_hq_pairs, gpu_sh_pairs)
+        return check_output_explained(got_out, ref["out"], alt, flipped)
+
+
 def _run_and_compare(hl, dl, x, logits, k, check_all=True):
     T = x.shape[0]
     ref = oracle.moe_forward(hl, x, logits, k)
@@ -213,8 +227,9 @@ def _run_and_compare(hl, dl, x, logits, k, check_all=True):
     assert np.array_equal(v["s_x"], ref["s_x"])
     n_diff, frac = check_fp8_codes(v["hq"], ref["hq"])
     np.testing.assert_allclose(v["s_h"], ref["s_h"], rtol=2e-5)
-    err = check_output(bits(out), ref["out"])
-    return dict(hq_diff=n_diff, hq_frac=frac, out_err=err, out=bits(out))
+    n_explained = _check_output_rules(hl, x, logits, k, bits(out), ref, v["hq"][v["row_of_pair"]],
+                                      v["s_h"][v["row_of_pair"]])
+    return dict(hq_diff=n_diff, hq_frac=frac, explained=n_explained, out=bits(out))
 
 
 def test_forward_tiny_workload():
@@ -459,7 +474,7 @@ def test_forward_full_size_sampled(name, full_layer):
     assert np.array_equal(v["s_x"][toks], ref["s_x"])
     check_fp8_codes(v["hq"][gpu_rows], ref["hq"][ref_rows])
     np.testing.assert_allclose(v["s_h"][gpu_rows], ref["s_h"][ref_rows], rtol=2e-5)
-    check_output(outb[toks], ref["out"])
+    _check_output_rules(hl, xs, ls, wl.k, outb[toks], ref, v["hq"][gpu_rows], v["s_h"][gpu_rows])
 
 
 # ---- failure detection: a bounded device wait that runs out -------------------------------------
@@ -596,7 +611,7 @@ def test_w8a8_forward_full_size_sampled(name, full_layer_w8a8):
     assert np.array_equal(v["xq"][toks], ref["xq"])
     check_fp8_codes(v["hq"][gpu_rows], ref["hq"][ref["row_of_pair"]])
     np.testing.assert_allclose(v["s_h"][gpu_rows], ref["s_h"][ref["row_of_pair"]], rtol=2e-5)
-    check_output(outb[toks], ref["out"])
+    _check_output_rules(hl, xs, ls, wl.k, outb[toks], ref, v["hq"][gpu_rows], v["s_h"][gpu_rows])
 
 
 # ---- NVFP4 experts -------------------------------------------------------------------------------
@@ -715,4 +730,4 @@ def test_nvfp4_forward_full_size_sampled(name, full_layer_nvfp4):
     assert np.array_equal(v["xq"][toks], ref["xq"])
     check_fp8_codes(v["hq"][gpu_rows], ref["hq"][ref["row_of_pair"]])
     np.testing.assert_allclose(v["s_h"][gpu_rows], ref["s_h"][ref["row_of_pair"]], rtol=2e-5)
-    check_output(outb[toks], ref["out"])
+    _check_output_rules(hl, xs, ls, wl.k, outb[toks], ref, v["hq"][gpu_rows], v["s_h"][gpu_rows])
