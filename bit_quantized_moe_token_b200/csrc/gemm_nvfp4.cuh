@@ -9,7 +9,7 @@
 //     out[t, n] = (sum_k f16(LUT[c] * scale)[n, k] * f16(dec q)[t, k]) * scale2 * s_x[t]
 // with every product exact in fp32.
 //
-// Roles (one persistent CTA per SM, 320 threads):
+// Roles (persistent CTAs of 320 threads; two per SM on 16-row tiles, else one):
 //   warps 0-3  epilogue (the FP8 GEMM's, with scale2 as the row scale)
 //   warps 4-7  widening: thread = weight row = TMEM lane; per 128-wide K step the row's 64 code
 //              bytes (from the TMA stage) and its 8 block scales (global, fetched a step ahead)
@@ -80,7 +80,10 @@ struct F4Cfg {
     static constexpr int kBBox = BN * 128;                  // one f16 box: BN rows x 64 K
     static constexpr int kStage = kW + 2 * kBBox;           // a multiple of 1024
     static_assert(kStage % 1024 == 0, "stage alignment");
-    static constexpr int kRS = kNarrow ? 12 : 4;            // ring stages
+    // ring stages; 16-row tiles run two CTAs per SM (each with half the ring): the single MMA
+    // lane is then shared by fewer bytes per cycle (measured: decode +29 %)
+    static constexpr int kRS = kNarrow ? (BN <= 16 ? 8 : 12) : 4;
+    static constexpr int kCtasPerSm = BN <= 16 ? 2 : 1;
     static constexpr int kS = kNarrow ? 2 : 4;              // TMEM A stages (64 columns each)
     static constexpr int kColA = 2 * BN;                    // TMEM: two accumulators | A stages
     static constexpr int kTmemNeed = kColA + kS * 64;
@@ -103,7 +106,7 @@ struct F4Cfg {
 };
 
 template <int BN, bool kSwiGLU, bool kFused, bool kGather>
-__global__ void __launch_bounds__(F4Cfg<BN>::kThreads, 1)
+__global__ void __launch_bounds__(F4Cfg<BN>::kThreads, F4Cfg<BN>::kCtasPerSm)
     k_gemm_nvfp4(const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__ CUtensorMap tm_w1,
                  const __grid_constant__ CUtensorMap tm_act, const F4GemmArgs f) {
     using C = F4Cfg<BN>;
@@ -352,7 +355,8 @@ int launch_gemm_nvfp4_inst(const F4GemmArgs& f, const void* act_f16, const void*
                      kGather ? 1 : BN, CU_TENSOR_MAP_SWIZZLE_128B))
         return MOE_ERR_CUDA;
     const int m_tiles = kSwiGLU ? a.R0 / 64 : a.R0 / 128;
-    const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(max_row_tiles * m_tiles, sms_cache[dev & 15]));
+    const int64_t grid = std::max<int64_t>(
+        1, std::min<int64_t>(max_row_tiles * m_tiles, (int64_t)sms_cache[dev & 15] * C::kCtasPerSm));
     kern<<<static_cast<unsigned>(grid), C::kThreads, C::kAlloc, stream>>>(m0, m1, mact, f);
     return launch_status();
 }
