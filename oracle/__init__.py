@@ -52,11 +52,14 @@ class _Layer(ctypes.Structure):
                 ("gate_bs", ctypes.c_void_p), ("up_bs", ctypes.c_void_p),
                 ("down_bs", ctypes.c_void_p),
                 ("gate_s2", ctypes.c_void_p), ("up_s2", ctypes.c_void_p),
-                ("down_s2", ctypes.c_void_p)]
+                ("down_s2", ctypes.c_void_p),
+                ("hot_ids", ctypes.c_void_p), ("cold_ids", ctypes.c_void_p),
+                ("n_hot", ctypes.c_int), ("n_cold", ctypes.c_int)]
 
 FMT_W4A8 = 0
 FMT_W8A8 = 1
 FMT_NVFP4 = 2
+FMT_HYBRID = 3
 
 
 _lib = None
@@ -249,6 +252,7 @@ class Layer:
         self.gate_f4 = self.up_f4 = self.down_f4 = None
         self.gate_bs = self.up_bs = self.down_bs = None
         self.gate_s2 = self.up_s2 = self.down_s2 = None
+        self.hot_ids = self.cold_ids = None
         self.sh_gate = None if sh_gate is None else np.ascontiguousarray(sh_gate, np.uint16)
         self.sh_up = None if sh_up is None else np.ascontiguousarray(sh_up, np.uint16)
         self.sh_down = None if sh_down is None else np.ascontiguousarray(sh_down, np.uint16)
@@ -288,6 +292,23 @@ class Layer:
         assert L.gate_s2.shape == (E,)
         return L
 
+    @classmethod
+    def hybrid(cls, cold: "Layer", hot: "Layer", hot_ids, cold_ids):
+        """Hot experts in NVFP4 (the slabs of `hot`, slab i = expert hot_ids[i]) and cold experts
+        in W4A8 (the slabs of `cold`, slab j = expert cold_ids[j]); the lists partition 0..E-1."""
+        hot_ids = np.ascontiguousarray(hot_ids, np.int32)
+        cold_ids = np.ascontiguousarray(cold_ids, np.int32)
+        E = len(hot_ids) + len(cold_ids)
+        assert np.array_equal(np.sort(np.concatenate([hot_ids, cold_ids])), np.arange(E))
+        L = cls(E, cold.H, cold.N, cold.gate_packed, cold.up_packed, cold.down_packed, cold.gate_scales,
+                cold.up_scales, cold.down_scales, group=cold.group, sh_gate=cold.sh_gate,
+                sh_up=cold.sh_up, sh_down=cold.sh_down)
+        L.fmt = FMT_HYBRID
+        for a in ("gate_f4", "up_f4", "down_f4", "gate_bs", "up_bs", "down_bs", "gate_s2", "up_s2", "down_s2"):
+            setattr(L, a, getattr(hot, a))
+        L.hot_ids, L.cold_ids = hot_ids, cold_ids
+        return L
+
     def _c(self):
         return _Layer(self.E, self.H, self.N, self.group,
                       _p(self.gate_packed), _p(self.up_packed), _p(self.down_packed),
@@ -298,7 +319,10 @@ class Layer:
                       _p(self.gate_rs), _p(self.up_rs), _p(self.down_rs),
                       _p(self.gate_f4), _p(self.up_f4), _p(self.down_f4),
                       _p(self.gate_bs), _p(self.up_bs), _p(self.down_bs),
-                      _p(self.gate_s2), _p(self.up_s2), _p(self.down_s2))
+                      _p(self.gate_s2), _p(self.up_s2), _p(self.down_s2),
+                      _p(self.hot_ids), _p(self.cold_ids),
+                      0 if self.hot_ids is None else len(self.hot_ids),
+                      0 if self.cold_ids is None else len(self.cold_ids))
 
 
 def moe_forward(layer: Layer, x_bf16: np.ndarray, logits: np.ndarray, k: int):

@@ -361,7 +361,26 @@ typedef struct {
     const uint8_t *gate_f4, *up_f4, *down_f4;               /* [E,N,H/2], [E,N,H/2], [E,H,N/2] */
     const uint8_t *gate_bs, *up_bs, *down_bs;               /* [E,N,H/16], [E,N,H/16], [E,H,N/16] */
     const float *gate_s2, *up_s2, *down_s2;                  /* [E] */
+    /* fmt 3 = hybrid ([P2] "On-disk tensor format": hot experts NVFP4, the rest another format;
+     * hot_ids / cold_ids give the routed expert of each slab and partition 0..E-1): hot slab i
+     * is NVFP4 slab i of the fmt-2 arrays, cold slab j is W4A8 slab j of the fmt-0 arrays. */
+    const int32_t *hot_ids, *cold_ids;
+    int n_hot, n_cold;
 } or_layer;
+
+/* Format and slab of routed expert e: the layer's format with slab e, or for a hybrid layer
+ * NVFP4 (2) with its hot slab or W4A8 (0) with its cold slab; -1 if e is in neither list. */
+static int expert_fmt(const or_layer* L, int64_t e, int64_t* slab) {
+    if (L->fmt != 3) {
+        *slab = e;
+        return L->fmt;
+    }
+    for (int i = 0; i < L->n_hot; ++i)
+        if (L->hot_ids[i] == e) { *slab = i; return 2; }
+    for (int j = 0; j < L->n_cold; ++j)
+        if (L->cold_ids[j] == e) { *slab = j; return 0; }
+    return -1;
+}
 
 /* Unpacked codes of one projection as floats, transposed to [K][rows] so that the
  * inner loop runs over independent outputs. */
@@ -565,6 +584,11 @@ static int moe_forward_impl(const or_layer* L, const uint16_t* x, const float* l
     const int64_t H = L->H, N = L->N, E = L->E;
     const int group = L->group;
     if (H % group || N % group || k < 1 || k > E) return -1;
+    if (L->fmt == 3)                     /* the hot and cold lists must cover every expert */
+        for (int64_t e = 0; e < E; ++e) {
+            int64_t b;
+            if (expert_fmt(L, e, &b) < 0) return -1;
+        }
     const int64_t P = T * k;
 
     int32_t* ids = (int32_t*)malloc((size_t)(P > 0 ? P : 1) * 4);
@@ -599,31 +623,33 @@ static int moe_forward_impl(const or_layer* L, const uint16_t* x, const float* l
         float* cu = (float*)malloc((size_t)N * H * 4);
         float* cd = (float*)malloc((size_t)H * N * 4);
         float* scratch = (float*)malloc((size_t)(3 * N + 2 * (H > N ? H : N)) * 4);
-        if (L->fmt == 1) {
-            w8_T(L->gate_w8 + e * N * H, N, H, cg);
-            w8_T(L->up_w8 + e * N * H, N, H, cu);
-            w8_T(L->down_w8 + e * H * N, H, N, cd);
-        } else if (L->fmt == 2) {
-            f4_T(L->gate_f4 + e * N * (H / 2), L->gate_bs + e * N * (H / 16), L->gate_s2[e], N, H, cg);
-            f4_T(L->up_f4 + e * N * (H / 2), L->up_bs + e * N * (H / 16), L->up_s2[e], N, H, cu);
-            f4_T(L->down_f4 + e * H * (N / 2), L->down_bs + e * H * (N / 16), L->down_s2[e], H, N, cd);
+        int64_t b;                       /* the expert's slab in its format's arrays */
+        const int f = expert_fmt(L, e, &b);
+        if (f == 1) {
+            w8_T(L->gate_w8 + b * N * H, N, H, cg);
+            w8_T(L->up_w8 + b * N * H, N, H, cu);
+            w8_T(L->down_w8 + b * H * N, H, N, cd);
+        } else if (f == 2) {
+            f4_T(L->gate_f4 + b * N * (H / 2), L->gate_bs + b * N * (H / 16), L->gate_s2[b], N, H, cg);
+            f4_T(L->up_f4 + b * N * (H / 2), L->up_bs + b * N * (H / 16), L->up_s2[b], N, H, cu);
+            f4_T(L->down_f4 + b * H * (N / 2), L->down_bs + b * H * (N / 16), L->down_s2[b], H, N, cd);
         } else {
-            codes_T(L->gate_packed + e * N * (H / 8), N, H, cg);
-            codes_T(L->up_packed + e * N * (H / 8), N, H, cu);
-            codes_T(L->down_packed + e * H * (N / 8), H, N, cd);
+            codes_T(L->gate_packed + b * N * (H / 8), N, H, cg);
+            codes_T(L->up_packed + b * N * (H / 8), N, H, cu);
+            codes_T(L->down_packed + b * H * (N / 8), H, N, cd);
         }
         for (int32_t r = r0; r < r1; ++r) {
             int64_t t = sorted[r] / k;
-            if (L->fmt == 1)
-                expert_row_w8(xq + t * H, sx[t], cg, cu, cd, L->gate_rs + e * N, L->up_rs + e * N,
-                              L->down_rs + e * H, H, N, hq + (int64_t)r * N, sh + r,
+            if (f == 1)
+                expert_row_w8(xq + t * H, sx[t], cg, cu, cd, L->gate_rs + b * N, L->up_rs + b * N,
+                              L->down_rs + b * H, H, N, hq + (int64_t)r * N, sh + r,
                               y + (int64_t)r * H, scratch);
-            else if (L->fmt == 2)
+            else if (f == 2)
                 expert_row_f4(xq + t * H, sx[t], cg, cu, cd, H, N, hq + (int64_t)r * N, sh + r,
                               y + (int64_t)r * H, scratch);
             else
-                expert_row(xq + t * H, sx[t], cg, cu, cd, L->gate_scales + e * N * G_h,
-                           L->up_scales + e * N * G_h, L->down_scales + e * H * G_n, H, N, group,
+                expert_row(xq + t * H, sx[t], cg, cu, cd, L->gate_scales + b * N * G_h,
+                           L->up_scales + b * N * G_h, L->down_scales + b * H * G_n, H, N, group,
                            hq + (int64_t)r * N, sh + r, y + (int64_t)r * H, scratch);
         }
         free(cg); free(cu); free(cd); free(scratch);
@@ -690,6 +716,11 @@ int or_moe_forward_dense(const or_layer* L, const uint16_t* x, const float* logi
     const int64_t H = L->H, N = L->N, E = L->E;
     const int group = L->group;
     if (H % group || N % group || k < 1 || k > E) return -1;
+    if (L->fmt == 3)                     /* the hot and cold lists must cover every expert */
+        for (int64_t e = 0; e < E; ++e) {
+            int64_t b;
+            if (expert_fmt(L, e, &b) < 0) return -1;
+        }
     uint8_t* xq = (uint8_t*)malloc((size_t)(T > 0 ? T : 1) * H);
     float* sx = (float*)malloc((size_t)(T > 0 ? T : 1) * 4);
     int32_t* ids = (int32_t*)malloc((size_t)(T * k > 0 ? T * k : 1) * 4);
@@ -702,30 +733,32 @@ int or_moe_forward_dense(const or_layer* L, const uint16_t* x, const float* logi
     float* cd = (float*)malloc((size_t)H * N * 4);
     float* scratch = (float*)malloc((size_t)(3 * N + 2 * (H > N ? H : N)) * 4);
     for (int64_t e = 0; e < E; ++e) {
-        if (L->fmt == 1) {
-            w8_T(L->gate_w8 + e * N * H, N, H, cg);
-            w8_T(L->up_w8 + e * N * H, N, H, cu);
-            w8_T(L->down_w8 + e * H * N, H, N, cd);
-        } else if (L->fmt == 2) {
-            f4_T(L->gate_f4 + e * N * (H / 2), L->gate_bs + e * N * (H / 16), L->gate_s2[e], N, H, cg);
-            f4_T(L->up_f4 + e * N * (H / 2), L->up_bs + e * N * (H / 16), L->up_s2[e], N, H, cu);
-            f4_T(L->down_f4 + e * H * (N / 2), L->down_bs + e * H * (N / 16), L->down_s2[e], H, N, cd);
+        int64_t b;                       /* the expert's slab in its format's arrays */
+        const int f = expert_fmt(L, e, &b);
+        if (f == 1) {
+            w8_T(L->gate_w8 + b * N * H, N, H, cg);
+            w8_T(L->up_w8 + b * N * H, N, H, cu);
+            w8_T(L->down_w8 + b * H * N, H, N, cd);
+        } else if (f == 2) {
+            f4_T(L->gate_f4 + b * N * (H / 2), L->gate_bs + b * N * (H / 16), L->gate_s2[b], N, H, cg);
+            f4_T(L->up_f4 + b * N * (H / 2), L->up_bs + b * N * (H / 16), L->up_s2[b], N, H, cu);
+            f4_T(L->down_f4 + b * H * (N / 2), L->down_bs + b * H * (N / 16), L->down_s2[b], H, N, cd);
         } else {
-            codes_T(L->gate_packed + e * N * (H / 8), N, H, cg);
-            codes_T(L->up_packed + e * N * (H / 8), N, H, cu);
-            codes_T(L->down_packed + e * H * (N / 8), H, N, cd);
+            codes_T(L->gate_packed + b * N * (H / 8), N, H, cg);
+            codes_T(L->up_packed + b * N * (H / 8), N, H, cu);
+            codes_T(L->down_packed + b * H * (N / 8), H, N, cd);
         }
         for (int64_t t = 0; t < T; ++t) {
-            if (L->fmt == 1)
-                expert_row_w8(xq + t * H, sx[t], cg, cu, cd, L->gate_rs + e * N, L->up_rs + e * N,
-                              L->down_rs + e * H, H, N, hq_dense + (t * E + e) * N,
+            if (f == 1)
+                expert_row_w8(xq + t * H, sx[t], cg, cu, cd, L->gate_rs + b * N, L->up_rs + b * N,
+                              L->down_rs + b * H, H, N, hq_dense + (t * E + e) * N,
                               sh_dense + t * E + e, y_dense + (t * E + e) * H, scratch);
-            else if (L->fmt == 2)
+            else if (f == 2)
                 expert_row_f4(xq + t * H, sx[t], cg, cu, cd, H, N, hq_dense + (t * E + e) * N,
                               sh_dense + t * E + e, y_dense + (t * E + e) * H, scratch);
             else
-                expert_row(xq + t * H, sx[t], cg, cu, cd, L->gate_scales + e * N * G_h,
-                           L->up_scales + e * N * G_h, L->down_scales + e * H * G_n, H, N, group,
+                expert_row(xq + t * H, sx[t], cg, cu, cd, L->gate_scales + b * N * G_h,
+                           L->up_scales + b * N * G_h, L->down_scales + b * H * G_n, H, N, group,
                            hq_dense + (t * E + e) * N, sh_dense + t * E + e,
                            y_dense + (t * E + e) * H, scratch);
         }

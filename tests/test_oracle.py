@@ -694,6 +694,50 @@ def test_nvfp4_dense_brute_force_matches_permuted():
         assert np.array_equal(r["y"][row], d["y"][t, e])
 
 
+def _hybrid_from(wl, hot_ids):
+    """A hybrid layer of workload `wl`: the NVFP4 slabs of the hot experts, the W4A8 slabs of the
+    others, both taken from the single-format layers of the same seeded weights."""
+    w4 = oracle.pack_workload_layer(wl)
+    f4 = oracle.quant_workload_layer_nvfp4(wl)
+    hot_ids = np.array(hot_ids, np.int32)
+    cold_ids = np.array([e for e in range(wl.E) if e not in set(hot_ids.tolist())], np.int32)
+    cold = oracle.Layer(wl.E - len(hot_ids), wl.H, wl.N, w4.gate_packed[cold_ids], w4.up_packed[cold_ids],
+                        w4.down_packed[cold_ids], w4.gate_scales[cold_ids], w4.up_scales[cold_ids],
+                        w4.down_scales[cold_ids])
+    hot = oracle.Layer.nvfp4(len(hot_ids), wl.H, wl.N, f4.gate_f4[hot_ids], f4.up_f4[hot_ids],
+                             f4.down_f4[hot_ids], f4.gate_bs[hot_ids], f4.up_bs[hot_ids], f4.down_bs[hot_ids],
+                             f4.gate_s2[hot_ids], f4.up_s2[hot_ids], f4.down_s2[hot_ids])
+    return oracle.Layer.hybrid(cold, hot, hot_ids, cold_ids), w4, f4
+
+
+def test_hybrid_dispatches_each_expert_to_its_format():
+    """Every routed pair of the hybrid layer computes exactly what the single-format layer of
+    its expert's format computes for it (hot experts: NVFP4, the rest: W4A8)."""
+    wl = synth.WORKLOADS["tiny"]
+    hot_ids = [6, 1, 3]                                 # slab order differs from expert order
+    hy, w4, f4 = _hybrid_from(wl, hot_ids)
+    x, lg = synth.tokens(wl), synth.logits(wl)
+    rh = oracle.moe_forward(hy, x, lg, wl.k)
+    r4 = oracle.moe_forward(w4, x, lg, wl.k)
+    rf = oracle.moe_forward(f4, x, lg, wl.k)
+    assert np.array_equal(rh["ids"], r4["ids"])
+    for p in range(wl.P):
+        t, j = divmod(p, wl.k)
+        ref = rf if rh["ids"][t, j] in hot_ids else r4
+        assert np.array_equal(rh["hq"][rh["row_of_pair"][p]], ref["hq"][ref["row_of_pair"][p]])
+        assert np.array_equal(rh["y"][rh["row_of_pair"][p]], ref["y"][ref["row_of_pair"][p]])
+    d = oracle.moe_forward_dense(hy, x, lg, wl.k)
+    assert np.array_equal(d["out"], rh["out"])
+
+
+def test_hybrid_rejects_lists_that_do_not_cover_every_expert():
+    wl = synth.WORKLOADS["tiny"]
+    hy, _, _ = _hybrid_from(wl, [6, 1, 3])
+    hy.cold_ids = hy.cold_ids[:-1].copy()               # an expert in neither list
+    with pytest.raises(ValueError):
+        oracle.moe_forward(hy, synth.tokens(wl), synth.logits(wl), wl.k)
+
+
 # ------------------------------------------------------------------------------------------------
 # rule 3 with rule 2's allowance (tests/parity.py)
 # ------------------------------------------------------------------------------------------------
