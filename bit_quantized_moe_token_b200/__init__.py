@@ -14,8 +14,10 @@ from ._binding import (MOE_OK, Layer, MoeError, fp8_quant_tokens, layer_struct, 
                        moe_w8a8_forward_profiled, moe_router_topk, moe_router_topk_workspace_bytes,
                        moe_w4a8_forward_router, moe_w8a8_forward_router, Layer4, layer4_struct,
                        nvfp4_quant_weights, moe_nvfp4_workspace_bytes, moe_nvfp4_workspace_layout,
-                       moe_nvfp4_forward, moe_nvfp4_forward_profiled, moe_nvfp4_forward_router)
-from .layer import (alloc_workspace, forward, make_layer, make_layer_nvfp4, make_layer_w8a8,
+                       moe_nvfp4_forward, moe_nvfp4_forward_profiled, moe_nvfp4_forward_router,
+                       LayerH, moe_hybrid_workspace_bytes, moe_hybrid_workspace_layout,
+                       moe_hybrid_forward, moe_hybrid_forward_profiled)
+from .layer import (alloc_workspace, forward, hybrid_from, make_layer, make_layer_nvfp4, make_layer_w8a8,
                     pack_expert_weights, quant_expert_weights_nvfp4, quant_expert_weights_w8a8)
 
 __all__ = ["MOE_OK", "Layer", "MoeError", "fp8_quant_tokens", "layer_struct", "lib",
@@ -31,4 +33,6 @@ __all__ = ["MOE_OK", "Layer", "MoeError", "fp8_quant_tokens", "layer_struct", "l
            "moe_router_topk_workspace_bytes", "moe_w4a8_forward_router", "moe_w8a8_forward_router",
            "Layer4", "layer4_struct", "nvfp4_quant_weights", "moe_nvfp4_workspace_bytes",
            "moe_nvfp4_workspace_layout", "moe_nvfp4_forward", "moe_nvfp4_forward_profiled",
-           "make_layer_nvfp4", "quant_expert_weights_nvfp4", "moe_nvfp4_forward_router"]
+           "make_layer_nvfp4", "quant_expert_weights_nvfp4", "moe_nvfp4_forward_router",
+           "LayerH", "moe_hybrid_workspace_bytes", "moe_hybrid_workspace_layout", "moe_hybrid_forward",
+           "moe_hybrid_forward_profiled", "hybrid_from"]

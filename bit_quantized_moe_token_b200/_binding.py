@@ -58,6 +58,22 @@ class _CLayer4(ctypes.Structure):
                 ("sh_down", ctypes.c_void_p)]
 
 
+class _CLayerH(ctypes.Structure):
+    _fields_ = [("E", ctypes.c_int), ("H", ctypes.c_int), ("N", ctypes.c_int),
+                ("n_hot", ctypes.c_int), ("n_cold", ctypes.c_int),
+                ("hot_ids", ctypes.c_void_p), ("cold_ids", ctypes.c_void_p),
+                ("hot_gate_f4", ctypes.c_void_p), ("hot_up_f4", ctypes.c_void_p), ("hot_down_f4", ctypes.c_void_p),
+                ("hot_gate_bs", ctypes.c_void_p), ("hot_up_bs", ctypes.c_void_p), ("hot_down_bs", ctypes.c_void_p),
+                ("hot_gate_s2", ctypes.c_void_p), ("hot_up_s2", ctypes.c_void_p), ("hot_down_s2", ctypes.c_void_p),
+                ("cold_gate_packed", ctypes.c_void_p), ("cold_up_packed", ctypes.c_void_p),
+                ("cold_down_packed", ctypes.c_void_p),
+                ("cold_gate_scales", ctypes.c_void_p), ("cold_up_scales", ctypes.c_void_p),
+                ("cold_down_scales", ctypes.c_void_p),
+                ("n_shared", ctypes.c_int), ("shared_N", ctypes.c_int),
+                ("sh_gate", ctypes.c_void_p), ("sh_up", ctypes.c_void_p),
+                ("sh_down", ctypes.c_void_p)]
+
+
 class _CLayout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in
                 ("topk_ids", "topk_w", "expert_offsets", "sorted_pairs", "row_of_pair",
@@ -109,6 +125,13 @@ def lib() -> ctypes.CDLL:
         L.moe_nvfp4_forward.argtypes = [ctypes.POINTER(_CLayer4), vp, vp, i64, i32, vp, vp, sz, vp]
         L.moe_nvfp4_forward_profiled.argtypes = [ctypes.POINTER(_CLayer4), vp, vp, i64, i32, vp, vp,
                                                  sz, vp, vp, i32, vp]
+        L.moe_hybrid_workspace_bytes.argtypes = [ctypes.POINTER(_CLayerH), i64, i32]
+        L.moe_hybrid_workspace_bytes.restype = sz
+        L.moe_hybrid_workspace_layout.argtypes = [ctypes.POINTER(_CLayerH), i64, i32,
+                                                  ctypes.POINTER(_CLayout)]
+        L.moe_hybrid_forward.argtypes = [ctypes.POINTER(_CLayerH), vp, vp, i64, i32, vp, vp, sz, vp]
+        L.moe_hybrid_forward_profiled.argtypes = [ctypes.POINTER(_CLayerH), vp, vp, i64, i32, vp, vp,
+                                                  sz, vp, vp, i32, vp]
         L.moe_router_topk_workspace_bytes.argtypes = [i64, i32, i32]
         L.moe_router_topk_workspace_bytes.restype = sz
         L.moe_router_topk.argtypes = [vp, vp, i64, i32, i32, i32, vp, vp, vp, vp, sz, vp]
@@ -505,3 +528,74 @@ def moe_nvfp4_forward_router(layer: Layer4, x, wr, k: int, out, ws, stream=None)
     nbytes = ws.numel() * ws.element_size() if ws is not None else 0
     _check(lib().moe_nvfp4_forward_router(ctypes.byref(s), _ptr(x), _ptr(wr), T, k, _ptr(out), _ptr(ws),
                                           nbytes, _stream(stream)), "moe_nvfp4_forward_router")
+
+
+# ---- hybrid layers: NVFP4 hot experts, W4A8 cold experts ---------------------------------------
+
+@dataclass
+class LayerH:
+    """Device tensors of a hybrid layer (moe_hybrid_layer): `hot` (a Layer4 of the hot slabs),
+    `cold` (a Layer of the cold slabs), and the int32 slab -> expert lists."""
+    E: int
+    hot: Layer4
+    cold: Layer
+    hot_ids: object
+    cold_ids: object
+
+    @property
+    def H(self) -> int:
+        return self.cold.H
+
+    @property
+    def N(self) -> int:
+        return self.cold.N
+
+    def c_struct(self) -> _CLayerH:
+        h, c = self.hot, self.cold
+        return _CLayerH(self.E, c.H, c.N, int(self.hot_ids.numel()), int(self.cold_ids.numel()),
+                        _ptr(self.hot_ids), _ptr(self.cold_ids),
+                        _ptr(h.gate_f4), _ptr(h.up_f4), _ptr(h.down_f4), _ptr(h.gate_bs), _ptr(h.up_bs),
+                        _ptr(h.down_bs), _ptr(h.gate_s2), _ptr(h.up_s2), _ptr(h.down_s2),
+                        _ptr(c.gate_packed), _ptr(c.up_packed), _ptr(c.down_packed), _ptr(c.gate_scales),
+                        _ptr(c.up_scales), _ptr(c.down_scales), c.n_shared, c.shared_N,
+                        _ptr(c.sh_gate), _ptr(c.sh_up), _ptr(c.sh_down))
+
+    def shape_struct(self) -> _CLayerH:
+        c = self.cold
+        return _CLayerH(self.E, c.H, c.N, 0, 0, None, None, None, None, None, None, None, None, None, None,
+                        None, None, None, None, None, None, None, c.n_shared, c.shared_N, None, None, None)
+
+
+def moe_hybrid_workspace_bytes(layer, T: int, k: int) -> int:
+    s = layer if isinstance(layer, _CLayerH) else layer.shape_struct()
+    return int(lib().moe_hybrid_workspace_bytes(ctypes.byref(s), T, k))
+
+
+def moe_hybrid_workspace_layout(layer, T: int, k: int) -> dict:
+    s = layer if isinstance(layer, _CLayerH) else layer.shape_struct()
+    out = _CLayout()
+    _check(lib().moe_hybrid_workspace_layout(ctypes.byref(s), T, k, ctypes.byref(out)),
+           "moe_hybrid_workspace_layout")
+    return {n: int(getattr(out, n)) for n, _ in _CLayout._fields_}
+
+
+def moe_hybrid_forward(layer: LayerH, x, logits, k: int, out, ws, stream=None) -> None:
+    """out bf16 [T, H] = the routed MoE layer with NVFP4 hot and W4A8 cold experts."""
+    T = x.shape[0]
+    s = layer.c_struct()
+    nbytes = ws.numel() * ws.element_size() if ws is not None else 0
+    _check(lib().moe_hybrid_forward(ctypes.byref(s), _ptr(x), _ptr(logits), T, k, _ptr(out),
+                                    _ptr(ws), nbytes, _stream(stream)), "moe_hybrid_forward")
+
+
+def moe_hybrid_forward_profiled(layer: LayerH, x, logits, k: int, out, ws, events, stream=None) -> int:
+    T = x.shape[0]
+    s = layer.c_struct()
+    nbytes = ws.numel() * ws.element_size() if ws is not None else 0
+    arr = (ctypes.c_void_p * len(events))(
+        *[ctypes.c_void_p(e.cuda_event if e is not None else 0) for e in events])
+    n = ctypes.c_int(0)
+    _check(lib().moe_hybrid_forward_profiled(ctypes.byref(s), _ptr(x), _ptr(logits), T, k, _ptr(out),
+                                             _ptr(ws), nbytes, _stream(stream), arr, len(events),
+                                             ctypes.byref(n)), "moe_hybrid_forward_profiled")
+    return int(n.value)

@@ -117,12 +117,13 @@ struct WsPlan {
     size_t qs_x, qs_h;   // per (activation row, K-group) sums of the FP8 values (narrow tiles)
     size_t logits, rcnt; // router logits [T, E] and the fused router's counters (router entry points)
     size_t act16;        // NVFP4 experts: f16 copies of the GEMM inputs (max of [T|P, H] and [P, N])
+    size_t slot_of;      // hybrid layers: expert -> slab map [E]
     int64_t n_zero;   // u32 words at `zero`: max|h| per row [P], row counters [P], token counters
     size_t sh_a, sh_y;
     size_t total;
 };
 
-// fmt: 0 W4A8, 1 row-scaled FP8, 2 NVFP4 (the last needs the f16 activation copies).
+// fmt: 0 W4A8, 1 row-scaled FP8, 2 NVFP4, 3 hybrid (2 and 3 need the f16 activation copies).
 inline WsPlan plan_workspace(const moe_w4a8_layer& L, int64_t T, int k, int fmt = 0) {
     WsPlan p{};
     const int64_t P = T * k;
@@ -152,7 +153,8 @@ inline WsPlan plan_workspace(const moe_w4a8_layer& L, int64_t T, int k, int fmt 
     p.qs_h = take((size_t)P * (L.N / 128) * 4);
     p.logits = take((size_t)T * L.E * 4);
     p.rcnt = take((size_t)router_counter_words(T) * 4);
-    p.act16 = fmt == 2 ? take((size_t)P * (L.H > L.N ? L.H : L.N) * 2) : 0;
+    p.act16 = fmt >= 2 ? take((size_t)P * (L.H > L.N ? L.H : L.N) * 2) : 0;
+    p.slot_of = fmt == 3 ? take((size_t)L.E * 4) : 0;
     if (L.n_shared > 0) {
         p.sh_a = take((size_t)T * L.n_shared * L.shared_N * 2);
         p.sh_y = take((size_t)T * L.H * 4);
@@ -202,13 +204,35 @@ extern "C" int moe_w4a8_workspace_layout(const moe_w4a8_layer* layer, int64_t T,
 namespace moe {
 
 // Routed-expert weights of one layer in any of the three formats.
-enum ExpertFmt { kFmtW4A8 = 0, kFmtW8A8 = 1, kFmtNvfp4 = 2 };
+enum ExpertFmt { kFmtW4A8 = 0, kFmtW8A8 = 1, kFmtNvfp4 = 2, kFmtHybrid = 3 };
 struct ExpertSet {
     int fmt;
-    const void *gate, *up, *down;         // W4A8: int32 [E,R,K/8]; W8A8: E4M3 [E,R,K]; NVFP4: [E,R,K/2]
-    const void *gate_s, *up_s, *down_s;   // W4A8: bf16 [E,R,K/128]; W8A8: fp32 [E,R]; NVFP4: E4M3 [E,R,K/16]
+    // W4A8: int32 [E,R,K/8]; W8A8: E4M3 [E,R,K]; NVFP4: [E,R,K/2]; hybrid: the cold W4A8 slabs
+    const void *gate, *up, *down;
+    // W4A8: bf16 [E,R,K/128]; W8A8: fp32 [E,R]; NVFP4: E4M3 [E,R,K/16]; hybrid: the cold scales
+    const void *gate_s, *up_s, *down_s;
     const float *gate_s2 = nullptr, *up_s2 = nullptr, *down_s2 = nullptr;   // NVFP4: fp32 [E]
+    // hybrid: the hot NVFP4 slabs and the slab lists
+    const void *h_gate = nullptr, *h_up = nullptr, *h_down = nullptr;
+    const void *h_gate_s = nullptr, *h_up_s = nullptr, *h_down_s = nullptr;
+    const float *h_gate_s2 = nullptr, *h_up_s2 = nullptr, *h_down_s2 = nullptr;
+    const int32_t *hot_ids = nullptr, *cold_ids = nullptr;
+    int n_hot = 0, n_cold = 0;
 };
+
+// Hybrid layers: slot_of[e] = i for the expert of hot slab i, -(j + 1) for that of cold slab j,
+// kSlotNone for an expert in neither list (ids outside [0, E) are ignored).
+__global__ void __launch_bounds__(1024) k_slot_map(const int32_t* __restrict__ hot_ids, int n_hot,
+                                                   const int32_t* __restrict__ cold_ids, int n_cold, int E,
+                                                   int32_t* __restrict__ slot_of) {
+    for (int e = threadIdx.x; e < E; e += blockDim.x) slot_of[e] = kSlotNone;
+    __syncthreads();
+    for (int i = threadIdx.x; i < n_hot + n_cold; i += blockDim.x) {
+        const int hot = i < n_hot;
+        const int32_t e = hot ? hot_ids[i] : cold_ids[i - n_hot];
+        if (e >= 0 && e < E) slot_of[e] = hot ? i : -(i - n_hot) - 1;
+    }
+}
 
 inline ExpertSet experts_of(const moe_w4a8_layer& L) {
     return ExpertSet{kFmtW4A8, L.gate_packed, L.up_packed, L.down_packed, L.gate_scales, L.up_scales,
@@ -266,8 +290,9 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const ExpertSet& xw, const ui
     if (st != MOE_OK) return st;
     const moe_w4a8_layer& L = *layer;
     if (T == 0) return MOE_OK;
-    if (!x_bf16 || (!router_logits && !router_w) || !out_bf16 || !xw.gate || !xw.up || !xw.down ||
-        !xw.gate_s || !xw.up_s || !xw.down_s)
+    const bool need_base = xw.fmt != kFmtHybrid || xw.n_cold > 0;   // a hybrid may have no cold slab
+    if (!x_bf16 || (!router_logits && !router_w) || !out_bf16 ||
+        (need_base && (!xw.gate || !xw.up || !xw.down || !xw.gate_s || !xw.up_s || !xw.down_s)))
         return MOE_ERR_INVALID_ARG;
     if (router_w && !aligned(router_w, 16)) return MOE_ERR_MISALIGNED;
     if (L.n_shared > 0 && (!L.sh_gate || !L.sh_up || !L.sh_down)) return MOE_ERR_INVALID_ARG;
@@ -277,11 +302,21 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const ExpertSet& xw, const ui
     if (!ws || ws_bytes < p.total) return MOE_ERR_WORKSPACE;
     const size_t s_al = xw.fmt == kFmtW8A8 ? 4 : xw.fmt == kFmtNvfp4 ? 8 : 2;   // scale alignment
     if (xw.fmt == kFmtNvfp4 && (!xw.gate_s2 || !xw.up_s2 || !xw.down_s2)) return MOE_ERR_INVALID_ARG;
+    if (xw.fmt == kFmtHybrid) {
+        if (xw.n_hot < 0 || xw.n_cold < 0 || (xw.n_hot > 0 && !xw.hot_ids) || (xw.n_cold > 0 && !xw.cold_ids))
+            return MOE_ERR_INVALID_ARG;
+        if (xw.n_hot > 0 && (!xw.h_gate || !xw.h_up || !xw.h_down || !xw.h_gate_s || !xw.h_up_s ||
+                             !xw.h_down_s || !xw.h_gate_s2 || !xw.h_up_s2 || !xw.h_down_s2))
+            return MOE_ERR_INVALID_ARG;
+        if (xw.n_hot > 0 && (!aligned(xw.h_gate, 16) || !aligned(xw.h_up, 16) || !aligned(xw.h_down, 16) ||
+                             !aligned(xw.h_gate_s, 8) || !aligned(xw.h_up_s, 8) || !aligned(xw.h_down_s, 8)))
+            return MOE_ERR_MISALIGNED;
+    }
     if (!aligned(ws, 256) || !aligned(x_bf16, 16) || !aligned(out_bf16, 16) ||
         !aligned(router_logits, 4) || !aligned(xw.gate, 16) || !aligned(xw.up, 16) ||
         !aligned(xw.down, 16) || !aligned(xw.gate_s, s_al) || !aligned(xw.up_s, s_al) ||
         !aligned(xw.down_s, s_al))
-        return MOE_ERR_MISALIGNED;
+        return MOE_ERR_MISALIGNED;      // (null pointers count as aligned)
 
     const int64_t P = T * k;
     char* w = static_cast<char*>(ws);
@@ -308,8 +343,27 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const ExpertSet& xw, const ui
     // narrow token tiles (decode): codes written once per token and gathered by the GEMM, fused
     // requantization and combine; wide tiles (prefill): codes copied to expert-sorted rows.
     const bool fused = ws_narrow(tc_tile_rows(P, L.E));
-    float* qsum_x = xw.fmt == kFmtW4A8 ? qs_x : nullptr;   // group sums: the unsigned widening only
-    uint16_t* act16 = xw.fmt == kFmtNvfp4 ? (uint16_t*)at(p.act16) : nullptr;
+    const bool hybrid = xw.fmt == kFmtHybrid;
+    float* qsum_x = (xw.fmt == kFmtW4A8 || hybrid) ? qs_x : nullptr;   // the unsigned widening only
+    uint16_t* act16 = xw.fmt >= kFmtNvfp4 ? (uint16_t*)at(p.act16) : nullptr;
+    int32_t* slot_of = hybrid ? (int32_t*)at(p.slot_of) : nullptr;
+    // the two launches of a hybrid layer's GEMM: W4A8 on the cold experts, NVFP4 on the hot ones
+    const bool run_w4 = xw.fmt == kFmtW4A8 || (hybrid && xw.n_cold > 0);
+    const bool run_f4 = xw.fmt == kFmtNvfp4 || (hybrid && xw.n_hot > 0);
+    const void* f4_gate = hybrid ? xw.h_gate : xw.gate;
+    const void* f4_up = hybrid ? xw.h_up : xw.up;
+    const void* f4_down = hybrid ? xw.h_down : xw.down;
+    const uint8_t* f4_gs = (const uint8_t*)(hybrid ? xw.h_gate_s : xw.gate_s);
+    const uint8_t* f4_us = (const uint8_t*)(hybrid ? xw.h_up_s : xw.up_s);
+    const uint8_t* f4_ds = (const uint8_t*)(hybrid ? xw.h_down_s : xw.down_s);
+    const float* f4_g2 = hybrid ? xw.h_gate_s2 : xw.gate_s2;
+    const float* f4_u2 = hybrid ? xw.h_up_s2 : xw.up_s2;
+    const float* f4_d2 = hybrid ? xw.h_down_s2 : xw.down_s2;
+    if (hybrid) {
+        k_slot_map<<<1, 1024, 0, stream>>>(xw.hot_ids, xw.n_hot, xw.cold_ids, xw.n_cold, L.E, slot_of);
+        if ((st = launch_status())) return st;
+        sm.launches += 1;
+    }
 
     sm.mark(0, stream);
     if (router_w) {
@@ -383,15 +437,16 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const ExpertSet& xw, const ui
     }
     sm.mark(3, stream);
     // S4 + SwiGLU (+ S5 when fused): h = silu(G) * U, max|h| per row
-    if (xw.fmt == kFmtNvfp4) {
+    if (run_f4) {
         // f16 copy of the FP8 activations (exact), then the f16 tensor-core GEMM
         if ((st = launch_e4m3_to_f16(fused ? xq : xs, (fused ? T : P) * L.H, act16, stream))) return st;
         F4GemmArgs f{W8GemmArgs{fused ? sx : sxs, nullptr, nullptr, offsets, L.E, L.N, L.H, (int)P, h, L.N,
                                 amax, rowcnt, hq, sh, sorted, nullptr, nullptr, k, nullptr, nullptr, (int)T},
-                     (const uint8_t*)xw.gate_s, (const uint8_t*)xw.up_s, xw.gate_s2, xw.up_s2};
-        if ((st = launch_gemm_nvfp4<true>(f, act16, xw.gate, xw.up, stream))) return st;
+                     f4_gs, f4_us, f4_g2, f4_u2, slot_of, hybrid ? kSlotHot : kSlotAll};
+        if ((st = launch_gemm_nvfp4<true>(f, act16, f4_gate, f4_up, stream))) return st;
         sm.launches += 2;
-    } else if (xw.fmt == kFmtW8A8) {
+    }
+    if (xw.fmt == kFmtW8A8) {
         W8GemmArgs a{fused ? sx : sxs, (const float*)xw.gate_s, (const float*)xw.up_s, offsets, L.E, L.N,
                      L.H, (int)P, h, L.N, amax, rowcnt, hq, sh, sorted, nullptr, nullptr, k, nullptr,
                      nullptr, (int)T};
@@ -399,10 +454,10 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const ExpertSet& xw, const ui
                                          stream)))
             return st;
         sm.launches += 1;
-    } else {
+    } else if (run_w4) {
         WsGemmArgs a{fused ? sx : sxs, (const uint16_t*)xw.gate_s, (const uint16_t*)xw.up_s, offsets, L.E,
                      L.N, L.H, (int)P, h, L.N, amax, rowcnt, hq, sh, sorted, nullptr, nullptr, k, nullptr,
-                     nullptr, (int)T, fused ? qs_x : nullptr, nullptr};
+                     nullptr, (int)T, fused ? qs_x : nullptr, nullptr, slot_of, hybrid ? kSlotCold : kSlotAll};
         if ((st = launch_gemm_ws<true>(a, fused ? (const void*)xq : (const void*)xs, xw.gate, xw.up,
                                        stream)))
             return st;
@@ -417,22 +472,23 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const ExpertSet& xw, const ui
     }
     sm.mark(5, stream);
     // S6 (+ S7 when fused)
-    if (xw.fmt == kFmtNvfp4) {
+    if (run_f4) {
         if ((st = launch_e4m3_to_f16(hq, P * L.N, act16, stream))) return st;
         F4GemmArgs f{W8GemmArgs{sh, nullptr, nullptr, offsets, L.E, L.H, L.N, (int)P, y, L.H, nullptr, tokcnt,
                                 nullptr, nullptr, sorted, rop, gates, k, shared, out_bf16, (int)T},
-                     (const uint8_t*)xw.down_s, nullptr, xw.down_s2, nullptr};
-        if ((st = launch_gemm_nvfp4<false>(f, act16, xw.down, nullptr, stream))) return st;
+                     f4_ds, nullptr, f4_d2, nullptr, slot_of, hybrid ? kSlotHot : kSlotAll};
+        if ((st = launch_gemm_nvfp4<false>(f, act16, f4_down, nullptr, stream))) return st;
         sm.launches += 2;
-    } else if (xw.fmt == kFmtW8A8) {
+    }
+    if (xw.fmt == kFmtW8A8) {
         W8GemmArgs a{sh, (const float*)xw.down_s, nullptr, offsets, L.E, L.H, L.N, (int)P, y, L.H, nullptr,
                      tokcnt, nullptr, nullptr, sorted, rop, gates, k, shared, out_bf16, (int)T};
         if ((st = launch_gemm_w8a8<false>(a, hq, xw.down, nullptr, stream))) return st;
         sm.launches += 1;
-    } else {
+    } else if (run_w4) {
         WsGemmArgs a{sh, (const uint16_t*)xw.down_s, nullptr, offsets, L.E, L.H, L.N, (int)P, y, L.H,
                      nullptr, tokcnt, nullptr, nullptr, sorted, rop, gates, k, shared, out_bf16, (int)T,
-                     nullptr, nullptr};
+                     nullptr, nullptr, slot_of, hybrid ? kSlotCold : kSlotAll};
         if ((st = launch_gemm_ws<false>(a, hq, xw.down, nullptr, stream))) return st;
         sm.launches += 1;
     }
@@ -586,4 +642,69 @@ extern "C" int moe_nvfp4_forward_router(const moe_nvfp4_layer* layer, const uint
     const moe_w4a8_layer s = moe::shape_of(*layer);
     return moe::forward_impl(&s, moe::experts_of(*layer), x_bf16, nullptr, T, k, out_bf16, ws, ws_bytes,
                              stream, sm, router_w_bf16);
+}
+
+// ---- hybrid layers: NVFP4 hot experts, W4A8 cold experts -------------------------------------
+
+namespace moe {
+inline moe_w4a8_layer shape_of(const moe_hybrid_layer& L) {
+    return moe_w4a8_layer{L.E, L.H, L.N, kGroup, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
+                          L.n_shared, L.shared_N, L.sh_gate, L.sh_up, L.sh_down};
+}
+inline ExpertSet experts_of(const moe_hybrid_layer& L) {
+    ExpertSet x{kFmtHybrid, L.cold_gate_packed, L.cold_up_packed, L.cold_down_packed, L.cold_gate_scales,
+                L.cold_up_scales, L.cold_down_scales};
+    x.h_gate = L.hot_gate_f4;
+    x.h_up = L.hot_up_f4;
+    x.h_down = L.hot_down_f4;
+    x.h_gate_s = L.hot_gate_bs;
+    x.h_up_s = L.hot_up_bs;
+    x.h_down_s = L.hot_down_bs;
+    x.h_gate_s2 = L.hot_gate_s2;
+    x.h_up_s2 = L.hot_up_s2;
+    x.h_down_s2 = L.hot_down_s2;
+    x.hot_ids = L.hot_ids;
+    x.cold_ids = L.cold_ids;
+    x.n_hot = L.n_hot;
+    x.n_cold = L.n_cold;
+    return x;
+}
+}  // namespace moe
+
+extern "C" size_t moe_hybrid_workspace_bytes(const moe_hybrid_layer* layer, int64_t T, int k) {
+    if (!layer) return 0;
+    const moe_w4a8_layer s = moe::shape_of(*layer);
+    if (moe::layer_args_ok(&s, T, k) != MOE_OK) return 0;
+    return moe::plan_workspace(s, T, k, moe::kFmtHybrid).total;
+}
+
+extern "C" int moe_hybrid_workspace_layout(const moe_hybrid_layer* layer, int64_t T, int k,
+                                           moe_w4a8_ws_layout* out) {
+    if (!layer) return MOE_ERR_INVALID_ARG;
+    const moe_w4a8_layer s = moe::shape_of(*layer);
+    int st = moe_w4a8_workspace_layout(&s, T, k, out);
+    if (st == MOE_OK) out->total = moe::plan_workspace(s, T, k, moe::kFmtHybrid).total;
+    return st;
+}
+
+extern "C" int moe_hybrid_forward_profiled(const moe_hybrid_layer* layer, const uint16_t* x_bf16,
+                                           const float* router_logits, int64_t T, int k,
+                                           uint16_t* out_bf16, void* ws, size_t ws_bytes,
+                                           moe_stream_t stream, void* const* events, int n_events,
+                                           int* n_launches) {
+    if (!layer) return MOE_ERR_INVALID_ARG;
+    if (events && n_events < MOE_W4A8_N_STAGE_EVENTS) return MOE_ERR_INVALID_ARG;
+    moe::StageMarks sm{events, n_events, 0};
+    const moe_w4a8_layer s = moe::shape_of(*layer);
+    const int st = moe::forward_impl(&s, moe::experts_of(*layer), x_bf16, router_logits, T, k,
+                                     out_bf16, ws, ws_bytes, stream, sm);
+    if (n_launches) *n_launches = sm.launches;
+    return st;
+}
+
+extern "C" int moe_hybrid_forward(const moe_hybrid_layer* layer, const uint16_t* x_bf16,
+                                  const float* router_logits, int64_t T, int k, uint16_t* out_bf16,
+                                  void* ws, size_t ws_bytes, moe_stream_t stream) {
+    return moe_hybrid_forward_profiled(layer, x_bf16, router_logits, T, k, out_bf16, ws, ws_bytes, stream,
+                                       nullptr, 0, nullptr);
 }

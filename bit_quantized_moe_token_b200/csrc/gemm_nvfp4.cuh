@@ -36,6 +36,9 @@ struct F4GemmArgs {
     const uint8_t* bs1;       // up block scales (SwiGLU instance)
     const float* s2_0;        // [E] scale2 of w0
     const float* s2_1;        // [E] scale2 of w1
+    // hybrid layers: expert -> slab map (null: slab = expert) and the experts this launch takes
+    const int32_t* slot_of = nullptr;
+    int slot_want = 0;
 };
 
 namespace tc {
@@ -132,7 +135,7 @@ __global__ void __launch_bounds__(F4Cfg<BN>::kThreads, F4Cfg<BN>::kCtasPerSm)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int steps = a.K / 128;
     const int m_tiles = kSwiGLU ? a.R0 / 64 : a.R0 / 128;
-    const int row_tiles = row_tile_prefix(a.offsets, a.E, BN, pre, soff);
+    const int row_tiles = row_tile_prefix(a.offsets, a.E, BN, pre, soff, f.slot_of, f.slot_want);
     const int64_t n_tiles = (int64_t)row_tiles * m_tiles;
     if ((int64_t)blockIdx.x >= n_tiles) return;
 
@@ -181,12 +184,13 @@ __global__ void __launch_bounds__(F4Cfg<BN>::kThreads, F4Cfg<BN>::kCtasPerSm)
                     ok = ws::wait(&empty[r.idx], r.phase ^ 1u, abort);
                     if (ok) {
                         tc::mbar_arrive_expect_tx(&full[r.idx], C::kW + b_bytes);
+                        const int wb = weight_slab(f.slot_of, e);
                         if (kSwiGLU) {
-                            const int y = e * a.R0 + mt * 64;
+                            const int y = wb * a.R0 + mt * 64;
                             ws::tma_load_2d(st, &tm_w0, s * 64, y, &full[r.idx]);
                             ws::tma_load_2d(st + 64 * 64, &tm_w1, s * 64, y, &full[r.idx]);
                         } else {
-                            ws::tma_load_2d(st, &tm_w0, s * 64, e * a.R0 + mt * 128, &full[r.idx]);
+                            ws::tma_load_2d(st, &tm_w0, s * 64, wb * a.R0 + mt * 128, &full[r.idx]);
                         }
                     }
                 }
@@ -262,10 +266,10 @@ __global__ void __launch_bounds__(F4Cfg<BN>::kThreads, F4Cfg<BN>::kCtasPerSm)
         ws::Ring<C::kS> ra;
         for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
             const int rt = static_cast<int>(tile / m_tiles), mt = static_cast<int>(tile % m_tiles);
-            const int e = expert_of_tile(pre, a.E, rt);
+            const int wb = weight_slab(f.slot_of, expert_of_tile(pre, a.E, rt));
             const uint8_t* srow = kSwiGLU
-                ? (row < 64 ? f.bs0 : f.bs1) + ((int64_t)e * a.R0 + mt * 64 + (row & 63)) * kb
-                : f.bs0 + ((int64_t)e * a.R0 + mt * 128 + row) * kb;
+                ? (row < 64 ? f.bs0 : f.bs1) + ((int64_t)wb * a.R0 + mt * 64 + (row & 63)) * kb
+                : f.bs0 + ((int64_t)wb * a.R0 + mt * 128 + row) * kb;
             uint2 sc_next = __ldg(reinterpret_cast<const uint2*>(srow));
             for (int s = 0; s < steps; ++s, r.next(), ra.next()) {
                 const uint2 sc = sc_next;
@@ -316,7 +320,10 @@ __global__ void __launch_bounds__(F4Cfg<BN>::kThreads, F4Cfg<BN>::kCtasPerSm)
         // ------------------------------------------------------------ epilogue warps 0-3
         w8_epilogue_warps<BN, kSwiGLU, kFused, kGather>(
             a, n_tiles, m_tiles, pre, soff, sSr, sX, flag, tmem, t_full, t_empty, abort,
-            [&](int e, int, int lrow) { return kSwiGLU ? (lrow < 64 ? f.s2_0[e] : f.s2_1[e]) : f.s2_0[e]; });
+            [&](int e, int, int lrow) {
+                const int wb = weight_slab(f.slot_of, e);
+                return kSwiGLU ? (lrow < 64 ? f.s2_0[wb] : f.s2_1[wb]) : f.s2_0[wb];
+            });
     }
 
     __syncwarp();

@@ -66,6 +66,9 @@ struct WsGemmArgs {
     // (per token when gathering, per sorted row otherwise), for the +8 offset correction
     const float* qsum;
     float* qsum_out;        // SwiGLU fused: the same sums of the requantized rows [P, R0/128]
+    // hybrid layers: expert -> slab map (null: slab = expert) and the experts this launch takes
+    const int32_t* slot_of = nullptr;
+    int slot_want = 0;
 };
 
 
@@ -162,7 +165,7 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
     const int G = a.K / kGroup;
     const int nst = (G + C::kGS - 1) / C::kGS;             // stages per tile
     const int m_tiles = kSwiGLU ? a.R0 / 64 : a.R0 / 128;
-    const int row_tiles = row_tile_prefix(a.offsets, a.E, BN, pre, soff);
+    const int row_tiles = row_tile_prefix(a.offsets, a.E, BN, pre, soff, a.slot_of, a.slot_want);
     const int64_t n_tiles = (int64_t)row_tiles * m_tiles;
     if ((int64_t)blockIdx.x >= n_tiles) return;
 
@@ -223,12 +226,13 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
                         // a stage past K (odd group count) is filled with zeros by the TMA unit
                         uint8_t* wst = wring + ws_ * C::kRaw;
                         tc::mbar_arrive_expect_tx(&w_full[ws_], C::kRaw);
+                        const int wb = weight_slab(a.slot_of, e);
                         if (kSwiGLU) {
-                            const int y = e * a.R0 + mt * 64;
+                            const int y = wb * a.R0 + mt * 64;
                             ws::tma_load_2d(wst, &tm_w0, g0 * 64, y, &w_full[ws_]);
                             ws::tma_load_2d(wst + 64 * C::kRowB, &tm_w1, g0 * 64, y, &w_full[ws_]);
                         } else {
-                            ws::tma_load_2d(wst, &tm_w0, g0 * 64, e * a.R0 + mt * 128, &w_full[ws_]);
+                            ws::tma_load_2d(wst, &tm_w0, g0 * 64, wb * a.R0 + mt * 128, &w_full[ws_]);
                         }
                         ok = ws::wait(&b_empty[bs], rb.phase ^ 1u, abort);
                         if (ok) tc::mbar_arrive_expect_tx(&b_full[bs], b_bytes * ng);
@@ -380,10 +384,10 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
         // before the current tile's epilogue so that a tile never starts on a DRAM round trip
         auto scale_row = [&](int64_t t) -> const uint16_t* {
             const int rt_ = static_cast<int>(t / m_tiles), mt_ = static_cast<int>(t % m_tiles);
-            const int e_ = expert_of_tile(pre, a.E, rt_);
+            const int b_ = weight_slab(a.slot_of, expert_of_tile(pre, a.E, rt_));
             if (kSwiGLU)
-                return (lrow < 64 ? a.s0 : a.s1) + ((int64_t)e_ * a.R0 + mt_ * 64 + (lrow & 63)) * G;
-            return a.s0 + ((int64_t)e_ * a.R0 + mt_ * 128 + lrow) * G;
+                return (lrow < 64 ? a.s0 : a.s1) + ((int64_t)b_ * a.R0 + mt_ * 64 + (lrow & 63)) * G;
+            return a.s0 + ((int64_t)b_ * a.R0 + mt_ * 128 + lrow) * G;
         };
         uint16_t first_raw[C::kGS];
         if (kSwiGLU && !C::kNarrow) {

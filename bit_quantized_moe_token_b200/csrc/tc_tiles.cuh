@@ -52,10 +52,30 @@ __device__ __forceinline__ uint32_t sw128_off(int r, int j) {
 
 // ---- tile map ------------------------------------------------------------------------------
 
+// Slab map of a hybrid layer (hot NVFP4 / cold W4A8 experts): slot_of[e] = i for hot slab i,
+// -(j + 1) for cold slab j, kSlotNone for an expert in neither list.
+constexpr int32_t kSlotNone = INT32_MIN;
+enum SlotWant { kSlotAll = 0, kSlotCold = 1, kSlotHot = 2 };
+
+__device__ __forceinline__ bool slot_kept(const int32_t* slot_of, int want, int e) {
+    if (!slot_of || want == kSlotAll) return true;
+    const int32_t s = slot_of[e];
+    return want == kSlotHot ? s >= 0 : (s < 0 && s != kSlotNone);
+}
+
+// Weight slab of expert e (e itself for a single-format layer).
+__device__ __forceinline__ int weight_slab(const int32_t* slot_of, int e) {
+    if (!slot_of) return e;
+    const int32_t s = slot_of[e];
+    return s >= 0 ? s : -s - 1;
+}
+
 // Per-expert prefix of row tiles (ceil(len / BN)) into shared `pre[0..E]`; returns the total.
-// With `soff` non-null the segment offsets [0..E] are copied there too.
+// With `soff` non-null the segment offsets [0..E] are copied there too.  With `slot_of`, experts
+// of the other format get no tiles (`want`: kSlotCold or kSlotHot).
 __device__ int row_tile_prefix(const int32_t* __restrict__ offsets, int E, int BN, int* pre,
-                               int* soff = nullptr) {
+                               int* soff = nullptr, const int32_t* slot_of = nullptr,
+                               int want = kSlotAll) {
     __shared__ int s_total;
     if (threadIdx.x < 32) {
         const int lane = threadIdx.x;
@@ -64,7 +84,7 @@ __device__ int row_tile_prefix(const int32_t* __restrict__ offsets, int E, int B
             const int e = e0 + lane;
             const int o0 = (e < E) ? offsets[e] : 0, o1 = (e < E) ? offsets[e + 1] : 0;
             if (soff && e < E) soff[e] = o0;
-            const int n = (e < E) ? (o1 - o0 + BN - 1) / BN : 0;
+            const int n = (e < E && slot_kept(slot_of, want, e)) ? (o1 - o0 + BN - 1) / BN : 0;
             int inc = n;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {

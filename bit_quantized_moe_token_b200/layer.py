@@ -1,7 +1,8 @@
 """Convenience wrappers: torch allocation around the C entry points."""
 from __future__ import annotations
 
-from ._binding import (Layer, Layer4, Layer8, moe_nvfp4_forward, moe_nvfp4_workspace_bytes,
+from ._binding import (Layer, Layer4, Layer8, LayerH, moe_hybrid_forward, moe_hybrid_workspace_bytes,
+                       moe_nvfp4_forward, moe_nvfp4_workspace_bytes,
                        moe_w4a8_forward, moe_w4a8_workspace_bytes, moe_w8a8_forward,
                        moe_w8a8_workspace_bytes, nvfp4_quant_weights, w4a8_pack_weights,
                        w8a8_quant_weights)
@@ -72,9 +73,32 @@ def make_layer_nvfp4(gate_w, up_w, down_w, sh_gate=None, sh_up=None, sh_down=Non
                   sh_gate=sh_gate, sh_up=sh_up, sh_down=sh_down)
 
 
+def hybrid_from(w4: Layer, f4: Layer4, hot_ids) -> LayerH:
+    """A hybrid layer from a W4A8 layer and an NVFP4 layer of the same experts: the hot experts
+    (hot_ids, in slab order) take their NVFP4 slabs, the others their W4A8 slabs."""
+    import torch
+    dev = w4.gate_packed.device
+    hot = torch.as_tensor(hot_ids, dtype=torch.int32).to(dev)
+    mask = torch.ones(w4.E, dtype=torch.bool, device=dev)
+    mask[hot.long()] = False
+    cold = torch.arange(w4.E, dtype=torch.int32, device=dev)[mask]
+    hi, ci = hot.long(), cold.long()
+    h = Layer4(len(hot_ids), f4.H, f4.N, f4.gate_f4[hi].contiguous(), f4.up_f4[hi].contiguous(),
+               f4.down_f4[hi].contiguous(), f4.gate_bs[hi].contiguous(), f4.up_bs[hi].contiguous(),
+               f4.down_bs[hi].contiguous(), f4.gate_s2[hi].contiguous(), f4.up_s2[hi].contiguous(),
+               f4.down_s2[hi].contiguous())
+    c = Layer(int(cold.numel()), w4.H, w4.N, w4.gate_packed[ci].contiguous(), w4.up_packed[ci].contiguous(),
+              w4.down_packed[ci].contiguous(), w4.gate_scales[ci].contiguous(), w4.up_scales[ci].contiguous(),
+              w4.down_scales[ci].contiguous(), group=w4.group, sh_gate=w4.sh_gate, sh_up=w4.sh_up,
+              sh_down=w4.sh_down)
+    return LayerH(w4.E, h, c, hot.contiguous(), cold.contiguous())
+
+
 def alloc_workspace(layer, T: int, k: int, device=None):
     import torch
-    if isinstance(layer, Layer8):
+    if isinstance(layer, LayerH):
+        n, ref = moe_hybrid_workspace_bytes(layer, T, k), layer.hot_ids
+    elif isinstance(layer, Layer8):
         n, ref = moe_w8a8_workspace_bytes(layer, T, k), layer.gate_w8
     elif isinstance(layer, Layer4):
         n, ref = moe_nvfp4_workspace_bytes(layer, T, k), layer.gate_f4
@@ -93,7 +117,9 @@ def forward(layer, x, logits, k: int, out=None, ws=None, stream=None):
         out = torch.empty_like(x)
     if ws is None:
         ws = alloc_workspace(layer, x.shape[0], k, x.device)
-    if isinstance(layer, Layer8):
+    if isinstance(layer, LayerH):
+        moe_hybrid_forward(layer, x, logits, k, out, ws, stream=stream)
+    elif isinstance(layer, Layer8):
         moe_w8a8_forward(layer, x, logits, k, out, ws, stream=stream)
     elif isinstance(layer, Layer4):
         moe_nvfp4_forward(layer, x, logits, k, out, ws, stream=stream)

@@ -332,6 +332,45 @@ int moe_nvfp4_forward_profiled(const moe_nvfp4_layer* layer, const uint16_t* x_b
                                void* ws, size_t ws_bytes, moe_stream_t stream,
                                void* const* events, int n_events, int* n_launches);
 
+/* ---------------------------------------------------------------------------------------
+ * Hybrid layers: hot experts in NVFP4, the others in W4A8, dispatched by expert.
+ *
+ * The "Inkling-512k-NVFP4-AQLM-hybrid" card ("On-disk tensor format") splits each layer's routed
+ * experts into a small hot set kept in NVFP4 and a cold set in another format, with hot_ids /
+ * cold_ids giving the routed expert of each slab (together a partition of 0..E-1).  Here the
+ * cold format is W4A8.  Each routed pair runs the projections of its expert's format; the two
+ * formats' grouped GEMMs share the routing, the permutation, the requantization, the combine
+ * and (at decode sizes) the fused epilogues' counters.
+ *   hot_ids  [n_hot] int32, cold_ids [n_cold] int32: must partition 0..E-1 (ids outside [0, E)
+ *            are ignored; an expert in neither list contributes nothing)
+ *   hot_*    NVFP4 slabs as in moe_nvfp4_layer with n_hot slabs
+ *   cold_*   W4A8 slabs as in moe_w4a8_layer with n_cold slabs
+ * Workspace, shapes and return codes as moe_nvfp4_forward.
+ * --------------------------------------------------------------------------------------- */
+typedef struct {
+    int E, H, N;
+    int n_hot, n_cold;
+    const int32_t *hot_ids, *cold_ids;
+    const uint8_t *hot_gate_f4, *hot_up_f4, *hot_down_f4;
+    const uint8_t *hot_gate_bs, *hot_up_bs, *hot_down_bs;
+    const float *hot_gate_s2, *hot_up_s2, *hot_down_s2;
+    const int32_t *cold_gate_packed, *cold_up_packed, *cold_down_packed;
+    const uint16_t *cold_gate_scales, *cold_up_scales, *cold_down_scales;
+    int n_shared, shared_N;
+    const uint16_t *sh_gate, *sh_up, *sh_down;
+} moe_hybrid_layer;
+
+size_t moe_hybrid_workspace_bytes(const moe_hybrid_layer* layer, int64_t T, int k);
+int moe_hybrid_workspace_layout(const moe_hybrid_layer* layer, int64_t T, int k,
+                                moe_w4a8_ws_layout* out);
+int moe_hybrid_forward(const moe_hybrid_layer* layer, const uint16_t* x_bf16,
+                       const float* router_logits, int64_t T, int k, uint16_t* out_bf16, void* ws,
+                       size_t ws_bytes, moe_stream_t stream);
+int moe_hybrid_forward_profiled(const moe_hybrid_layer* layer, const uint16_t* x_bf16,
+                                const float* router_logits, int64_t T, int k, uint16_t* out_bf16,
+                                void* ws, size_t ws_bytes, moe_stream_t stream,
+                                void* const* events, int n_events, int* n_launches);
+
 /* The layer fed by the router weight instead of precomputed logits: the router logits
  * (moe_router_logits' definition, written into the workspace), then the layer of
  * moe_w4a8_forward / moe_w8a8_forward on them.  At decode sizes (T <= 16) the router, the

@@ -31,7 +31,8 @@ def test_header_declares_the_boundary():
               "moe_w8a8_workspace_bytes", "moe_w8a8_forward_profiled", "moe_router_topk",
               "moe_router_topk_workspace_bytes", "moe_w4a8_forward_router", "moe_w8a8_forward_router",
               "nvfp4_quant_weights", "moe_nvfp4_forward", "moe_nvfp4_workspace_bytes",
-              "moe_nvfp4_forward_profiled", "moe_nvfp4_forward_router",
+              "moe_nvfp4_forward_profiled", "moe_nvfp4_forward_router", "moe_hybrid_forward",
+              "moe_hybrid_workspace_bytes", "moe_hybrid_forward_profiled",
               "moe_w4a8_workspace_bytes", "moe_last_device_status", "moe_status_string"):
         assert n in names
 
@@ -201,6 +202,23 @@ def test_nvfp4_rejects_bad_args():
     nos2 = moe._binding._CLayer4(8, 256, 128, p, p, p, p, p, p, None, p, p, 0, 0, None, None, None)
     assert L.moe_nvfp4_forward(ctypes.byref(nos2), p, p, 4, 2, p, p, need, None) == -1
     assert L.moe_nvfp4_forward(ctypes.byref(full), p, p, 0, 2, p, p, need, None) == 0
+
+
+def test_hybrid_rejects_bad_args():
+    L = _L()
+    p = ctypes.c_void_p(4096)
+    H = moe._binding._CLayerH
+    full = H(8, 256, 128, 2, 6, p, p, *([p] * 15), 0, 0, None, None, None)
+    need = moe.moe_hybrid_workspace_bytes(full, 4, 2)
+    assert need > 0
+    assert L.moe_hybrid_forward(ctypes.byref(full), p, p, 4, 2, p, p, need - 1, None) == -4
+    no_ids = H(8, 256, 128, 2, 6, None, p, *([p] * 15), 0, 0, None, None, None)
+    assert L.moe_hybrid_forward(ctypes.byref(no_ids), p, p, 4, 2, p, p, need, None) == -1
+    all_hot = H(8, 256, 128, 8, 0, p, None, *([p] * 9), *([None] * 6), 0, 0, None, None, None)
+    assert L.moe_hybrid_forward(ctypes.byref(all_hot), p, p, 0, 2, p, p, need, None) == 0
+    odd = H(8, 256, 128, 2, 6, p, p, *([p] * 3), ctypes.c_void_p(4100), p, p, *([p] * 9), 0, 0, None,
+            None, None)                                               # hot block scales need 8 bytes
+    assert L.moe_hybrid_forward(ctypes.byref(odd), p, p, 4, 2, p, p, need, None) == -3
 
 
 def test_binding_has_no_fallback():

@@ -36,7 +36,8 @@ def bits(t):
 
 def ws_views(layer, ws, T, k):
     layout = (moe.moe_w8a8_workspace_layout if isinstance(layer, moe.Layer8) else
-              moe.moe_nvfp4_workspace_layout if isinstance(layer, moe.Layer4) else moe.moe_w4a8_workspace_layout)
+              moe.moe_nvfp4_workspace_layout if isinstance(layer, moe.Layer4) else
+              moe.moe_hybrid_workspace_layout if isinstance(layer, moe.LayerH) else moe.moe_w4a8_workspace_layout)
     lay = layout(layer, T, k)
     P = T * k
     b = ws.cpu().numpy()
@@ -731,3 +732,76 @@ def test_nvfp4_forward_full_size_sampled(name, full_layer_nvfp4):
     check_fp8_codes(v["hq"][gpu_rows], ref["hq"][ref["row_of_pair"]])
     np.testing.assert_allclose(v["s_h"][gpu_rows], ref["s_h"][ref["row_of_pair"]], rtol=2e-5)
     _check_output_rules(hl, xs, ls, wl.k, outb[toks], ref, v["hq"][gpu_rows], v["s_h"][gpu_rows])
+
+
+# ---- hybrid layers: NVFP4 hot experts, W4A8 cold experts -------------------------------------------
+
+def _host_hybrid(w4: "oracle.Layer", f4: "oracle.Layer", hot_ids):
+    hot_ids = np.array(hot_ids, np.int32)
+    cold_ids = np.array([e for e in range(w4.E) if e not in set(hot_ids.tolist())], np.int32)
+    cold = oracle.Layer(len(cold_ids), w4.H, w4.N, w4.gate_packed[cold_ids], w4.up_packed[cold_ids],
+                        w4.down_packed[cold_ids], w4.gate_scales[cold_ids], w4.up_scales[cold_ids],
+                        w4.down_scales[cold_ids], sh_gate=w4.sh_gate, sh_up=w4.sh_up, sh_down=w4.sh_down)
+    hot = oracle.Layer.nvfp4(len(hot_ids), w4.H, w4.N, f4.gate_f4[hot_ids], f4.up_f4[hot_ids],
+                             f4.down_f4[hot_ids], f4.gate_bs[hot_ids], f4.up_bs[hot_ids], f4.down_bs[hot_ids],
+                             f4.gate_s2[hot_ids], f4.up_s2[hot_ids], f4.down_s2[hot_ids])
+    return oracle.Layer.hybrid(cold, hot, hot_ids, cold_ids)
+
+
+def _host_layer_and_dev_hybrid(E, H, N, seed, hot_ids):
+    """One set of seeded weights, W4A8-packed and NVFP4-quantized on both sides; the hybrid takes
+    the NVFP4 slabs of the hot experts and the W4A8 slabs of the rest."""
+    rng_stream = 80_000 + seed * 10
+    gw = synth.normal_bf16(seed, rng_stream + 0, E * N * H, 0.02).reshape(E, N, H)
+    uw = synth.normal_bf16(seed, rng_stream + 1, E * N * H, 0.02).reshape(E, N, H)
+    dw = synth.normal_bf16(seed, rng_stream + 2, E * H * N, 0.02).reshape(E, H, N)
+    gp, gs = zip(*[oracle.rtn_pack(gw[e])[:2] for e in range(E)])
+    up, us = zip(*[oracle.rtn_pack(uw[e])[:2] for e in range(E)])
+    dp, ds = zip(*[oracle.rtn_pack(dw[e])[:2] for e in range(E)])
+    w4 = oracle.Layer(E, H, N, np.stack(gp), np.stack(up), np.stack(dp), np.stack(gs), np.stack(us), np.stack(ds))
+    def qp(W):
+        r = [oracle.nvfp4_quant(W[e]) for e in range(E)]
+        return (np.stack([a for a, _, _ in r]), np.stack([b for _, b, _ in r]),
+                np.array([c for _, _, c in r], np.float32))
+    g, u, d = qp(gw), qp(uw), qp(dw)
+    f4 = oracle.Layer.nvfp4(E, H, N, g[0], u[0], d[0], g[1], u[1], d[1], g[2], u[2], d[2])
+    hl = _host_hybrid(w4, f4, hot_ids)
+    dgw, duw, ddw = to_dev_bf16(gw), to_dev_bf16(uw), to_dev_bf16(dw)
+    dl = moe.hybrid_from(moe.make_layer(dgw, duw, ddw), moe.make_layer_nvfp4(dgw, duw, ddw), hot_ids)
+    torch.cuda.synchronize()
+    return hl, dl
+
+
+@pytest.mark.parametrize("E,H,N,k,T,hot", [(16, 256, 128, 2, 8, [0, 5, 9]), (16, 256, 128, 2, 40, [3]),
+                                           (8, 256, 256, 2, 600, [2, 7]), (4, 256, 128, 2, 21, [0, 1, 2, 3]),
+                                           (4, 256, 128, 2, 21, []), (64, 1024, 1024, 6, 16, list(range(0, 64, 7)))])
+def test_hybrid_forward(E, H, N, k, T, hot):
+    """Hot experts on the NVFP4 GEMM, cold ones on the W4A8 GEMM, in one layer (decode: fused
+    epilogues counting both GEMMs' contributions; prefill; all hot; all cold)."""
+    hl, dl = _host_layer_and_dev_hybrid(E, H, N, seed=E + T + len(hot), hot_ids=hot)
+    x = synth.normal_bf16(11, 840 + T, T * H).reshape(T, H)
+    logits = synth.normal_f32(11, 841 + T, T * E).reshape(T, E)
+    _run_and_compare(hl, dl, x, logits, k)
+
+
+def test_hybrid_full_size_decode_sampled():
+    """decode_t8 with 15 % of the experts hot (the page's 512k tier keeps 14.8 % in NVFP4)."""
+    wl = synth.WORKLOADS["decode_t8"]
+    hot = [int(e) for e in np.random.default_rng(5).choice(wl.E, 38, replace=False)]
+    dl = moe.hybrid_from(device_layer(wl), device_layer_nvfp4(wl), hot)
+    x, lg = device_inputs(wl)
+    ws = moe.alloc_workspace(dl, wl.T, wl.k)
+    out = moe.forward(dl, x, lg, wl.k, ws=ws)
+    torch.cuda.synchronize()
+    assert moe.moe_last_device_status() == 0
+    v = ws_views(dl, ws, wl.T, wl.k)
+    ids_ref, _ = oracle.route_topk(synth.logits(wl), wl.k)
+    experts = sorted(set(ids_ref.reshape(-1).tolist()))
+    assert any(e in hot for e in experts) and any(e not in hot for e in experts)
+    hl = _host_hybrid(oracle.pack_workload_layer(wl, experts=experts),
+                      oracle.quant_workload_layer_nvfp4(wl, experts=experts), hot)
+    xs, ls = synth.tokens(wl), synth.logits(wl)
+    ref = oracle.moe_forward(hl, xs, ls, wl.k)
+    assert np.array_equal(v["ids"], ref["ids"])
+    check_fp8_codes(v["hq"][v["row_of_pair"]], ref["hq"][ref["row_of_pair"]])
+    _check_output_rules(hl, xs, ls, wl.k, bits(out), ref, v["hq"][v["row_of_pair"]], v["s_h"][v["row_of_pair"]])
