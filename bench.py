@@ -293,14 +293,23 @@ def run_ours(args):
     wl = synth.WORKLOADS[args.workload]
     w8 = args.experts == "w8a8"
     f4 = args.experts == "nvfp4"
-    layer = (device_layer_w8a8 if w8 else device_layer_nvfp4 if f4 else device_layer)(wl, device=dev)
-    fwd = moe.moe_w8a8_forward if w8 else moe.moe_nvfp4_forward if f4 else moe.moe_w4a8_forward
+    hy = args.experts == "hybrid"
+    hot_set = set(synth.hot_experts(wl).tolist()) if hy else set()
+    if hy:
+        layer = moe.hybrid_from(device_layer(wl, device=dev), device_layer_nvfp4(wl, device=dev),
+                                synth.hot_experts(wl))
+        torch.cuda.empty_cache()
+    else:
+        layer = (device_layer_w8a8 if w8 else device_layer_nvfp4 if f4 else device_layer)(wl, device=dev)
+    fwd = (moe.moe_w8a8_forward if w8 else moe.moe_nvfp4_forward if f4 else moe.moe_hybrid_forward if hy
+           else moe.moe_w4a8_forward)
     fwd_profiled = (moe.moe_w8a8_forward_profiled if w8 else moe.moe_nvfp4_forward_profiled if f4
-                    else moe.moe_w4a8_forward_profiled)
+                    else moe.moe_hybrid_forward_profiled if hy else moe.moe_w4a8_forward_profiled)
     layout = (moe.moe_w8a8_workspace_layout if w8 else moe.moe_nvfp4_workspace_layout if f4
-              else moe.moe_w4a8_workspace_layout)
+              else moe.moe_hybrid_workspace_layout if hy else moe.moe_w4a8_workspace_layout)
     if not wl.n_shared:
-        layer.sh_gate = layer.sh_up = layer.sh_down = None
+        tgt = layer.cold if hy else layer
+        tgt.sh_gate = tgt.sh_up = tgt.sh_down = None
     T, k = wl.T, wl.k
     batches = []
     for b in range(N_BATCHES):
@@ -312,11 +321,13 @@ def run_ours(args):
 
     # touched experts per batch (for the algorithmic byte count), from the routing outputs
     lay = layout(layer, T, k)
-    touched = []
+    touched, touched_hot = [], []
     for x, lg in batches:
         moe.forward(layer, x, lg, k, out=out, ws=ws)
         offs = ws[lay["expert_offsets"]:lay["expert_offsets"] + 4 * (wl.E + 1)].view(torch.int32)
-        touched.append(int((offs[1:] - offs[:-1] > 0).sum().item()))
+        used = torch.nonzero(offs[1:] - offs[:-1] > 0).flatten().tolist()
+        touched.append(len(used))
+        touched_hot.append(sum(1 for e in used if e in hot_set))
     torch.cuda.synchronize()
     if moe.moe_last_device_status() != 0:
         raise RuntimeError("device status: timeout during warm-up")
@@ -420,17 +431,20 @@ def run_ours(args):
     rt_ms = max_over_ranks(rt_ms, dev, world)
     # the whole layer fed by the router weight (router, S1, S2 fused at decode)
     fwd_router = (moe.moe_w8a8_forward_router if w8 else moe.moe_nvfp4_forward_router if f4
-                  else moe.moe_w4a8_forward_router)
-    for i in range(3):
-        fwd_router(layer, batches[i % N_BATCHES][0], wr, k, out, ws)
-    q0, q1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    torch.cuda.synchronize()
-    q0.record(stream)
-    for i in range(args.steps):
-        fwd_router(layer, batches[i % N_BATCHES][0], wr, k, out, ws)
-    q1.record(stream)
-    torch.cuda.synchronize()
-    lr_ms = max_over_ranks(q0.elapsed_time(q1), dev, world) / args.steps
+                  else None if hy else moe.moe_w4a8_forward_router)
+    lr_ms = None
+    if fwd_router is not None:
+        for i in range(3):
+            fwd_router(layer, batches[i % N_BATCHES][0], wr, k, out, ws)
+        q0, q1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        q0.record(stream)
+        for i in range(args.steps):
+            fwd_router(layer, batches[i % N_BATCHES][0], wr, k, out, ws)
+        q1.record(stream)
+        torch.cuda.synchronize()
+        lr_ms = q0.elapsed_time(q1) / args.steps
+    lr_ms = max_over_ranks(lr_ms if lr_ms is not None else 0.0, dev, world)
     if moe.moe_last_device_status() != 0:
         raise RuntimeError("device status: timeout in the router timing")
 
@@ -438,9 +452,17 @@ def run_ours(args):
     value = whole_job_rate(world, T, args.steps, total_ms)
     hbm, bf16, peak_kind = peaks()
     fmt = args.experts
-    kname = "W8A8" if w8 else "NVFP4" if f4 else "W4A8"
-    gu_bytes, down_bytes = expert_bytes(wl, fmt)
-    mean_touched = sum(touched[i % N_BATCHES] for i in range(args.steps)) / args.steps
+    kname = "W8A8" if w8 else "NVFP4" if f4 else "NVFP4-hot + W4A8-cold" if hy else "W4A8"
+    if hy:   # touched hot experts at NVFP4 bytes, the others at W4A8 bytes
+        gu4, dn4 = expert_bytes(wl, "w4a8")
+        guf, dnf = expert_bytes(wl, "nvfp4")
+        mean_hot = sum(touched_hot[i % N_BATCHES] for i in range(args.steps)) / args.steps
+        mean_touched = sum(touched[i % N_BATCHES] for i in range(args.steps)) / args.steps
+        gu_bytes = (mean_hot * guf + (mean_touched - mean_hot) * gu4) / max(mean_touched, 1e-9)
+        down_bytes = (mean_hot * dnf + (mean_touched - mean_hot) * dn4) / max(mean_touched, 1e-9)
+    else:
+        gu_bytes, down_bytes = expert_bytes(wl, fmt)
+        mean_touched = sum(touched[i % N_BATCHES] for i in range(args.steps)) / args.steps
     dom_bytes = mean_touched * gu_bytes
     # Both bounds of the gate/up GEMM: its algorithmic bytes (touched experts' gate+up weights)
     # over the measured HBM bandwidth, and its FLOPs over the dense FP8 tensor peak (the measured
@@ -455,7 +477,7 @@ def run_ours(args):
     hbm_side = {"bound": "hbm", "achieved": round(ach_gbs, 1), "peak": hbm, "unit": "GB/s",
                 "frac": round(ach_gbs / hbm, 4), "peak_source": f"{peak_kind} hbm_gbs",
                 "algorithmic_bytes_per_launch": int(dom_bytes),
-                "units": f"{mean_touched:.1f} touched experts x {gu_bytes} B (gate+up codes+scales)"}
+                "units": f"{mean_touched:.1f} touched experts x {gu_bytes:.0f} B (gate+up codes+scales)"}
     tc_side = {"bound": "tensor", "achieved": round(ach_tf, 1), "peak": round(fp8, 1),
                "unit": "TFLOP/s", "frac": round(ach_tf / fp8, 4),
                "peak_source": f"{peak_kind} bf16_tflops x 2 (nominal FP8/BF16 ratio)",
@@ -474,6 +496,7 @@ def run_ours(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": ("e4m3 x e4m3 -> f32" if w8 else "f16(e2m1 x e4m3 scale) x f16(e4m3) -> f32" if f4
+                  else "hot: f16(e2m1 x e4m3 scale) x f16(e4m3); cold: e4m3 x int4 -> f32" if hy
                   else "e4m3 x int4 -> f32"), "data": "synthetic",
         "config": {"workload": wl.name, "experts": fmt, "T": T, "H": wl.H, "N": wl.N, "E": wl.E, "k": k,
                    "routing": wl.routing, "n_shared": wl.n_shared, "seed": wl.seed,
@@ -486,7 +509,7 @@ def run_ours(args):
         "gpu_launches": launches,
         "router": dict(router_line(wl, T, r_ms, hbm, bf16, peak_kind),
                        topk_fused_ms=round(rt_ms, 4), cuda_graph=r_graph),
-        "layer_with_router": {"ms_per_step": round(lr_ms, 4),
+        "layer_with_router": None if lr_ms <= 0 else {"ms_per_step": round(lr_ms, 4),
                               "value": round(world * T / (lr_ms / 1e3), 1), "unit": "tokens/s",
                               "note": "moe_*_forward_router: router logits + the layer per step; "
                                       "routing follows the synthetic N(0, 1/H) router weight (near "
@@ -521,6 +544,19 @@ def oracle_sample(wl, t0, max_tokens, fmt="w4a8"):
         layer = oracle.quant_workload_layer_w8a8(wl, experts=used)
     elif fmt == "nvfp4":
         layer = oracle.quant_workload_layer_nvfp4(wl, experts=used)
+    elif fmt == "hybrid":
+        hot = synth.hot_experts(wl)
+        cold_ids = np.array([e for e in range(wl.E) if e not in set(hot.tolist())], np.int32)
+        w4 = oracle.pack_workload_layer(wl, experts=used)
+        f4 = oracle.quant_workload_layer_nvfp4(wl, experts=used, with_shared=False)
+        cold = oracle.Layer(len(cold_ids), wl.H, wl.N, w4.gate_packed[cold_ids], w4.up_packed[cold_ids],
+                            w4.down_packed[cold_ids], w4.gate_scales[cold_ids], w4.up_scales[cold_ids],
+                            w4.down_scales[cold_ids], group=wl.group, sh_gate=w4.sh_gate, sh_up=w4.sh_up,
+                            sh_down=w4.sh_down)
+        hotl = oracle.Layer.nvfp4(len(hot), wl.H, wl.N, f4.gate_f4[hot], f4.up_f4[hot], f4.down_f4[hot],
+                                  f4.gate_bs[hot], f4.up_bs[hot], f4.down_bs[hot], f4.gate_s2[hot],
+                                  f4.up_s2[hot], f4.down_s2[hot])
+        layer = oracle.Layer.hybrid(cold, hotl, hot, cold_ids)
     else:
         layer = oracle.pack_workload_layer(wl, experts=used)
     return layer, x, lg, n
@@ -583,7 +619,7 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ref-tokens", type=int, default=8)
-    ap.add_argument("--experts", default="w4a8", choices=["w4a8", "w8a8", "nvfp4"],
+    ap.add_argument("--experts", default="w4a8", choices=["w4a8", "w8a8", "nvfp4", "hybrid"],
                     help="routed-expert weight format (default: W4A8 INT4 x FP8)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

@@ -209,6 +209,18 @@ def expert_ranks(wl: Workload) -> np.ndarray:
     return (permutation(wl.seed, S_RANKS, wl.E) + 1).astype(np.int32)
 
 
+HOT_FRACTION = 0.148   # the NVFP4 share of expert slots in the hybrid card's 512k tier
+
+
+def hot_experts(wl: Workload) -> np.ndarray:
+    """int32[round(0.148 * E)]: the hot (NVFP4) experts of a hybrid layer of workload `wl`, in
+    slab order: the most popular experts under Zipf routing, a seeded choice otherwise."""
+    n = int(round(HOT_FRACTION * wl.E))
+    if wl.routing == "zipf":
+        return np.argsort(expert_ranks(wl), kind="stable")[:n].astype(np.int32)
+    return np.sort(permutation(wl.seed, S_RANKS + 1, wl.E)[:n]).astype(np.int32)
+
+
 def logit_bias(wl: Workload) -> np.ndarray | None:
     """float64[E]: -1.1*ln(rank_e) for zipf routing, else None."""
     if wl.routing != "zipf":
