@@ -1,21 +1,22 @@
-// gemm_ws.cuh — S4/S6: warp-specialised grouped W4A8 GEMM on tcgen05 with a TMA ring.
+// gemm_ws.cuh — S4/S6: warp-specialised grouped W4A8 GEMM on tcgen05 with TMA rings.
 //
-// Roles (one or two persistent CTAs per SM):
-//   widening warps (8 for narrow token tiles, 4 for wide ones): per K-group they turn the
-//              tile's packed INT4 codes (128 rows x 64 B, from the TMA ring) into 128 x 128 E4M3
-//              bytes in a 128-byte-swizzled A stage.  Four consecutive threads take the four
-//              16-byte chunks of a row, so shared-memory reads and the swizzled writes are both
-//              free of bank conflicts.  They never wait on the tensor core, only on free stages.
-//   promotion warps (4 for narrow tiles, 8 for wide ones): a thread owns one TMEM lane = A row
-//              (and, with 8 warps, half of the tile's token columns).  Per K-group they fold
-//              the group's TMEM partial into an fp32 register accumulator with the group scale
-//              (acc += s[n,g] * partial), then run the tile's epilogue.
-//   TMA warp:  streams each group's packed weight tile into a ring of RW stages and the
-//              activation tile (BN rows x 128 B, landing pre-swizzled for the MMA) into a ring
-//              of RB stages; narrow gate/up tiles gather their live rows four at a time.
-//   MMA warp:  one lane issues four (or eight) tcgen05.mma.kind::f8f6f4 per group into one of
-//              two TMEM partial buffers and commits to the barriers that hand the buffer to the
-//              promotion warps and release the ring / A stages; the warp also owns the TMEM.
+// Roles (persistent CTAs; two per SM on 16-row token tiles, else one):
+//   widening warps (8 on narrow token tiles, 4 on wide ones): a thread owns one weight row = one
+//              TMEM lane.  Per stage (two K-groups on narrow tiles, one on wide ones) it reads the
+//              row's packed INT4 codes from the TMA stage (the 64- or 128-byte TMA swizzle spreads
+//              the 32 rows of a warp over distinct banks), widens them to E4M3 and writes them
+//              into a TMEM A stage with tcgen05.st; the MMA takes A from TMEM.
+//   promotion warps (4 on narrow tiles, 16 on 128-row tiles, each owning a lane quadrant and a
+//              slice of the token columns): per K-group they fold the group's TMEM partial into
+//              fp32 register accumulators with the group scale (acc += s[n,g] * partial, two
+//              columns per packed FMA), then run the tile's epilogue.
+//   TMA warp:  streams the packed weight tiles into a weight ring and the activation tiles
+//              (BN rows x 128 B per group, landing pre-swizzled for the MMA) into an activation
+//              ring; narrow gate/up tiles gather their live token rows four at a time.
+//   MMA warp:  one lane issues four tcgen05.mma.kind::f8f6f4 per K-group into one of kNT TMEM
+//              partial buffers.  Narrow tiles commit once per stage (the partial's barrier; the
+//              widening warps free the A stage and the activation slot from that completion);
+//              wide tiles also commit the shared A / activation stage.  The warp owns the TMEM.
 //
 // Widening (see tc_tiles.cuh for the arithmetic):
 //   kUnsigned (narrow gate/up tiles, decode): byte = nibble = E4M3 of (code+8)*2^-9, so TMEM
@@ -25,6 +26,9 @@
 //     in the promotion than as four more MMAs).
 //   signed (the down GEMM and all wide token tiles): byte = E4M3(code) by byte-permute lookup;
 //     exact codes, so no offset term that would amplify the tensor core's accumulation error.
+//
+// Hybrid layers pass an expert -> slab map: the launch then takes only its format's experts and
+// reads each one's weights from its slab.
 //
 // Every mbarrier wait is bounded; a timeout sets a CTA-wide abort flag that turns all later
 // waits into no-ops (so the named barrier among the promotion warps stays uniform), records
