@@ -101,7 +101,7 @@ struct WsCfg {
     // saves the MMA lane a wait and a commit per group.
     static constexpr bool kSplitB = kNarrow;
     static constexpr int kRB = kSplitB ? kRW + kS : kS;                                 // activation ring
-    static constexpr int kNT = kNarrow ? 8 : (BN <= 64 ? 4 : 3);                   // TMEM partials
+    static constexpr int kNT = kNarrow ? 8 : (BN <= 64 ? 4 : (BN <= 128 ? 3 : 2));  // TMEM partials
     static constexpr int kNTS = kNT / kGS;                       // partial stages (barrier pairs)
     // TMEM columns: partial buffers | widened A tiles (32 columns = 128 E4M3 per row)
     static constexpr int kColA = kNT * BN;
@@ -628,7 +628,7 @@ inline bool ws_narrow(int BN) { return BN <= 32; }
 template <bool kSwiGLU>
 int launch_gemm_ws(const WsGemmArgs& a, const void* act, const void* w0, const void* w1,
                    cudaStream_t stream) {
-    const int BN = tc_tile_rows(a.P, a.E);
+    const int BN = ws_tile_rows(a.P, a.E);
     const int64_t max_row_tiles = ((int64_t)a.P + BN - 1) / BN + a.E;
     switch (BN) {
         // narrow gate/up tiles widen unsigned (the FP8 requantization after them absorbs the
@@ -636,7 +636,8 @@ int launch_gemm_ws(const WsGemmArgs& a, const void* act, const void* w0, const v
         // keeps the exact signed codes
         case 16: return launch_gemm_ws_inst<16, kSwiGLU, kSwiGLU, true, kSwiGLU>(a, act, w0, w1, max_row_tiles, stream);
         case 32: return launch_gemm_ws_inst<32, kSwiGLU, kSwiGLU, true, kSwiGLU>(a, act, w0, w1, max_row_tiles, stream);
-        default: return launch_gemm_ws_inst<128, false, kSwiGLU, false, false>(a, act, w0, w1, max_row_tiles, stream);
+        case 128: return launch_gemm_ws_inst<128, false, kSwiGLU, false, false>(a, act, w0, w1, max_row_tiles, stream);
+        default: return launch_gemm_ws_inst<192, false, kSwiGLU, false, false>(a, act, w0, w1, max_row_tiles, stream);
     }
 }
 

@@ -125,10 +125,19 @@ struct TcLaunchShape {
 // T = 2048 (48 rows per expert on average) the popular experts' long segments dominate the
 // work, and 128-row tiles re-read each of their weight tiles half as often as 64-row ones
 // (measured: W4A8 gate/up 1.14 -> 0.94 ms).
+constexpr int64_t kWsWideAvg = 160;
 inline int tc_tile_rows(int64_t P, int E) {
     const int64_t avg = (P + E - 1) / E;
     return avg <= 8 ? 16 : avg <= 24 ? 32 : 128;
 }
 inline bool tc_unsigned(int BN) { return BN <= 32; }
+
+// The W4A8 GEMM widens each weight stage once per token tile, so long segments want the widest
+// tile whose partial buffers still leave TMEM room for the widened A stages: 192 rows (two
+// 192-column partials + four 32-column A stages = 512 columns).
+inline int ws_tile_rows(int64_t P, int E) {
+    const int bn = tc_tile_rows(P, E);
+    return bn == 128 && (P + E - 1) / E >= kWsWideAvg ? 192 : bn;
+}
 
 }  // namespace moe

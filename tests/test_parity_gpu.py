@@ -245,7 +245,7 @@ def test_forward_tiny_workload():
 
 @pytest.mark.parametrize("E,H,N,k,T", [(5, 384, 256, 3, 37), (1, 256, 128, 1, 9), (8, 256, 128, 2, 1),
                                        (16, 512, 384, 8, 130), (3, 1024, 128, 2, 700),
-                                       (64, 1024, 1024, 6, 16)])
+                                       (64, 1024, 1024, 6, 16), (4, 512, 256, 2, 500)])
 def test_forward_ragged_shapes(E, H, N, k, T):
     hl, dl = _host_layer_and_dev(E, H, N, seed=E * 7 + T)
     x = synth.normal_bf16(3, 777 + T, T * H).reshape(T, H)
