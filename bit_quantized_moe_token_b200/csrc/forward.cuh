@@ -36,7 +36,8 @@ __global__ void __launch_bounds__(256) k_requant(const float* __restrict__ h, in
 }
 
 // out[t, m] = bf16( sum_j gate[t,j] * Y[row(t,j), m]  (+ shared[t, m]) ), j in selection
-// order.  One thread per (token, 4 consecutive m): float4 loads of the k routed rows.
+// order.  One thread per (token, 4 consecutive m): the k row indices and gates first, then the k
+// float4 loads of the routed rows all in flight at once, then the sum in order.
 __global__ void __launch_bounds__(256) k_combine(const float* __restrict__ Y,
                                                  const float* __restrict__ gates,
                                                  const int32_t* __restrict__ rop, int k, int H,
@@ -47,14 +48,26 @@ __global__ void __launch_bounds__(256) k_combine(const float* __restrict__ Y,
     if (i >= T * q) return;
     const int64_t t = i / q;
     const int m4 = static_cast<int>(i % q);
+    int row[kMaxK];
+    float g[kMaxK];
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) {
+        row[j] = j < k ? rop[t * k + j] : 0;
+        g[j] = j < k ? gates[t * k + j] : 0.0f;
+    }
+    float4 y[kMaxK];
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j)
+        if (j < k) y[j] = reinterpret_cast<const float4*>(Y + (int64_t)row[j] * H)[m4];
     float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int j = 0; j < k; ++j) {
-        const float g = gates[t * k + j];
-        const float4 y = reinterpret_cast<const float4*>(Y + (int64_t)rop[t * k + j] * H)[m4];
-        o.x = __fadd_rn(o.x, __fmul_rn(g, y.x));
-        o.y = __fadd_rn(o.y, __fmul_rn(g, y.y));
-        o.z = __fadd_rn(o.z, __fmul_rn(g, y.z));
-        o.w = __fadd_rn(o.w, __fmul_rn(g, y.w));
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) {
+        if (j < k) {
+            o.x = __fadd_rn(o.x, __fmul_rn(g[j], y[j].x));
+            o.y = __fadd_rn(o.y, __fmul_rn(g[j], y[j].y));
+            o.z = __fadd_rn(o.z, __fmul_rn(g[j], y[j].z));
+            o.w = __fadd_rn(o.w, __fmul_rn(g[j], y[j].w));
+        }
     }
     if (shared) {
         const float4 sh = reinterpret_cast<const float4*>(shared + t * H)[m4];
@@ -114,11 +127,11 @@ inline int launch_quant_topk(const float* logits, const uint16_t* x, int64_t T, 
 struct WsPlan {
     size_t topk_ids, topk_w, offsets, sorted, rop, route_ws;
     size_t xq, s_x, x_sorted, s_x_sorted, h, zero, hq, s_h, y;
-    size_t qs_x, qs_h;   // per (activation row, K-group) sums of the FP8 values (narrow tiles)
+    size_t qs_x;         // per (token, K-group) sums of the FP8 values (narrow W4A8 tiles)
     size_t logits, rcnt; // router logits [T, E] and the fused router's counters (router entry points)
     size_t act16;        // NVFP4 experts: f16 copies of the GEMM inputs (max of [T|P, H] and [P, N])
     size_t slot_of;      // hybrid layers: expert -> slab map [E]
-    int64_t n_zero;   // u32 words at `zero`: max|h| per row [P], row counters [P], token counters
+    int64_t n_zero;   // u32 words at `zero`: max|h| per row [P]
     size_t sh_a, sh_y;
     size_t total;
 };
@@ -144,13 +157,12 @@ inline WsPlan plan_workspace(const moe_w4a8_layer& L, int64_t T, int k, int fmt 
     p.x_sorted = take((size_t)P * L.H);
     p.s_x_sorted = take(P * 4);
     p.h = take((size_t)P * L.N * 4);
-    p.n_zero = 2 * P + T * (L.H / 128);
+    p.n_zero = P;
     p.zero = take((size_t)p.n_zero * 4);
     p.hq = take((size_t)P * L.N);
     p.s_h = take(P * 4);
     p.y = take((size_t)P * L.H * 4);
     p.qs_x = take((size_t)T * (L.H / 128) * 4);
-    p.qs_h = take((size_t)P * (L.N / 128) * 4);
     p.logits = take((size_t)T * L.E * 4);
     p.rcnt = take((size_t)router_counter_words(T) * 4);
     p.act16 = fmt >= 2 ? take((size_t)P * (L.H > L.N ? L.H : L.N) * 2) : 0;
@@ -333,16 +345,16 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const ExpertSet& xw, const ui
     float* h = (float*)at(p.h);
     unsigned* zero = (unsigned*)at(p.zero);
     unsigned* amax = zero;
-    unsigned* rowcnt = zero + P;
-    unsigned* tokcnt = zero + 2 * P;
     uint8_t* hq = (uint8_t*)at(p.hq);
     float* sh = (float*)at(p.s_h);
     float* y = (float*)at(p.y);
     float* qs_x = (float*)at(p.qs_x);
-    float* qs_h = (float*)at(p.qs_h);
-    // narrow token tiles (decode): codes written once per token and gathered by the GEMM, fused
-    // requantization and combine; wide tiles (prefill): codes copied to expert-sorted rows.
-    const bool fused = ws_narrow(tc_tile_rows(P, L.E));
+    // narrow token tiles (decode): codes written once per token and gathered by the GEMM; wide
+    // tiles (prefill): codes copied to expert-sorted rows.  Either way the requantization (S5)
+    // and the combine (S7) run as their own passes: fused into the GEMM epilogues behind
+    // device-scope counters they cost every tile a fence and an atomic round trip while the
+    // tensor core waited (measured: 7-26 % slower decode layers).
+    const bool gather = ws_narrow(tc_tile_rows(P, L.E));
     const bool hybrid = xw.fmt == kFmtHybrid;
     float* qsum_x = (xw.fmt == kFmtW4A8 || hybrid) ? qs_x : nullptr;   // the unsigned widening only
     uint16_t* act16 = xw.fmt >= kFmtNvfp4 ? (uint16_t*)at(p.act16) : nullptr;
@@ -371,14 +383,14 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const ExpertSet& xw, const ui
         float* lg = (float*)at(p.logits);
         unsigned* rc = (unsigned*)at(p.rcnt);
         if (cudaMemsetAsync(rc, 0, router_counter_words(T) * 4, stream) != cudaSuccess) return MOE_ERR_CUDA;
-        const bool front_quant = fused && T <= 16;
+        const bool front_quant = gather && T <= 16;
         int nl = 0;
         if ((st = launch_router_topk(x_bf16, router_w, T, L.H, L.E, k, lg, ids, gates, rc,
                                      front_quant ? xq : nullptr, sx, qsum_x, stream, &nl)))
             return st;
         sm.launches += nl;
         sm.mark(1, stream);
-        if (fused) {
+        if (gather) {
             if (!front_quant) {
                 if ((st = launch_quant_topk(nullptr, x_bf16, T, L.E, k, L.H, ids, gates, xq, sx, qsum_x,
                                             stream, false)))
@@ -397,14 +409,14 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const ExpertSet& xw, const ui
             sm.launches += (P <= kSinglePassMaxP ? 1 : 3) + 1;
         }
         sm.mark(2, stream);
-    } else if (fused) {
+    } else if (gather) {
         // S1 + S2: per-token FP8 codes and top-k
         if ((st = launch_quant_topk(router_logits, x_bf16, T, L.E, k, L.H, ids, gates, xq, sx, qsum_x,
                                     stream)))
             return st;
         sm.launches += 1;
         sm.mark(1, stream);
-        // S3 (+ zeroing of the per-row maxima and the fused epilogues' counters)
+        // S3 (+ zeroing of the per-row maxima)
         if ((st = launch_permute(ids, T, L.E, k, offsets, sorted, rop, (int32_t*)at(p.route_ws), stream,
                                  zero, p.n_zero)))
             return st;
@@ -436,65 +448,61 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const ExpertSet& xw, const ui
         sm.launches += 2;
     }
     sm.mark(3, stream);
-    // S4 + SwiGLU (+ S5 when fused): h = silu(G) * U, max|h| per row
+    // S4 + SwiGLU: h = silu(G) * U, max|h| per row
     if (run_f4) {
         // f16 copy of the FP8 activations (exact), then the f16 tensor-core GEMM
-        if ((st = launch_e4m3_to_f16(fused ? xq : xs, (fused ? T : P) * L.H, act16, stream))) return st;
-        F4GemmArgs f{W8GemmArgs{fused ? sx : sxs, nullptr, nullptr, offsets, L.E, L.N, L.H, (int)P, h, L.N,
-                                amax, rowcnt, hq, sh, sorted, nullptr, nullptr, k, nullptr, nullptr, (int)T},
+        if ((st = launch_e4m3_to_f16(gather ? xq : xs, (gather ? T : P) * L.H, act16, stream))) return st;
+        F4GemmArgs f{W8GemmArgs{gather ? sx : sxs, nullptr, nullptr, offsets, L.E, L.N, L.H, (int)P, h, L.N,
+                                amax, sorted, k, (int)T},
                      f4_gs, f4_us, f4_g2, f4_u2, slot_of, hybrid ? kSlotHot : kSlotAll};
         if ((st = launch_gemm_nvfp4<true>(f, act16, f4_gate, f4_up, stream))) return st;
         sm.launches += 2;
     }
     if (xw.fmt == kFmtW8A8) {
-        W8GemmArgs a{fused ? sx : sxs, (const float*)xw.gate_s, (const float*)xw.up_s, offsets, L.E, L.N,
-                     L.H, (int)P, h, L.N, amax, rowcnt, hq, sh, sorted, nullptr, nullptr, k, nullptr,
-                     nullptr, (int)T};
-        if ((st = launch_gemm_w8a8<true>(a, fused ? (const void*)xq : (const void*)xs, xw.gate, xw.up,
+        W8GemmArgs a{gather ? sx : sxs, (const float*)xw.gate_s, (const float*)xw.up_s, offsets, L.E, L.N,
+                     L.H, (int)P, h, L.N, amax, sorted, k, (int)T};
+        if ((st = launch_gemm_w8a8<true>(a, gather ? (const void*)xq : (const void*)xs, xw.gate, xw.up,
                                          stream)))
             return st;
         sm.launches += 1;
     } else if (run_w4) {
-        WsGemmArgs a{fused ? sx : sxs, (const uint16_t*)xw.gate_s, (const uint16_t*)xw.up_s, offsets, L.E,
-                     L.N, L.H, (int)P, h, L.N, amax, rowcnt, hq, sh, sorted, nullptr, nullptr, k, nullptr,
-                     nullptr, (int)T, fused ? qs_x : nullptr, nullptr, slot_of, hybrid ? kSlotCold : kSlotAll};
-        if ((st = launch_gemm_ws<true>(a, fused ? (const void*)xq : (const void*)xs, xw.gate, xw.up,
+        WsGemmArgs a{gather ? sx : sxs, (const uint16_t*)xw.gate_s, (const uint16_t*)xw.up_s, offsets, L.E,
+                     L.N, L.H, (int)P, h, L.N, amax, sorted, k, (int)T, gather ? qs_x : nullptr, slot_of,
+                     hybrid ? kSlotCold : kSlotAll};
+        if ((st = launch_gemm_ws<true>(a, gather ? (const void*)xq : (const void*)xs, xw.gate, xw.up,
                                        stream)))
             return st;
         sm.launches += 1;
     }
     sm.mark(4, stream);
     // S5
-    if (!fused) {
-        k_requant<<<static_cast<unsigned>(P), 256, 0, stream>>>(h, L.N, amax, hq, sh);
-        if ((st = launch_status())) return st;
-        sm.launches += 1;
-    }
+    k_requant<<<static_cast<unsigned>(P), 256, 0, stream>>>(h, L.N, amax, hq, sh);
+    if ((st = launch_status())) return st;
+    sm.launches += 1;
     sm.mark(5, stream);
-    // S6 (+ S7 when fused)
+    // S6
     if (run_f4) {
         if ((st = launch_e4m3_to_f16(hq, P * L.N, act16, stream))) return st;
-        F4GemmArgs f{W8GemmArgs{sh, nullptr, nullptr, offsets, L.E, L.H, L.N, (int)P, y, L.H, nullptr, tokcnt,
-                                nullptr, nullptr, sorted, rop, gates, k, shared, out_bf16, (int)T},
+        F4GemmArgs f{W8GemmArgs{sh, nullptr, nullptr, offsets, L.E, L.H, L.N, (int)P, y, L.H, nullptr, sorted,
+                                k, (int)T},
                      f4_ds, nullptr, f4_d2, nullptr, slot_of, hybrid ? kSlotHot : kSlotAll};
         if ((st = launch_gemm_nvfp4<false>(f, act16, f4_down, nullptr, stream))) return st;
         sm.launches += 2;
     }
     if (xw.fmt == kFmtW8A8) {
         W8GemmArgs a{sh, (const float*)xw.down_s, nullptr, offsets, L.E, L.H, L.N, (int)P, y, L.H, nullptr,
-                     tokcnt, nullptr, nullptr, sorted, rop, gates, k, shared, out_bf16, (int)T};
+                     sorted, k, (int)T};
         if ((st = launch_gemm_w8a8<false>(a, hq, xw.down, nullptr, stream))) return st;
         sm.launches += 1;
     } else if (run_w4) {
         WsGemmArgs a{sh, (const uint16_t*)xw.down_s, nullptr, offsets, L.E, L.H, L.N, (int)P, y, L.H,
-                     nullptr, tokcnt, nullptr, nullptr, sorted, rop, gates, k, shared, out_bf16, (int)T,
-                     nullptr, nullptr, slot_of, hybrid ? kSlotCold : kSlotAll};
+                     nullptr, sorted, k, (int)T, nullptr, slot_of, hybrid ? kSlotCold : kSlotAll};
         if ((st = launch_gemm_ws<false>(a, hq, xw.down, nullptr, stream))) return st;
         sm.launches += 1;
     }
     sm.mark(6, stream);
     // S7
-    if (!fused) {
+    {
         const int64_t n = T * (L.H / 4);
         k_combine<<<static_cast<unsigned>((n + 255) / 256), 256, 0, stream>>>(y, gates, rop, k, L.H, T,
                                                                             shared, out_bf16);

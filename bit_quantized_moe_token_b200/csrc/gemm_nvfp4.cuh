@@ -96,8 +96,7 @@ struct F4Cfg {
     static constexpr int kOffX = kRS * kStage;
     static constexpr int kOffPre = kOffX + 64 * kXStride * 4;
     static constexpr int kOffSoff = kOffPre + 1025 * 4;
-    static constexpr int kOffFlag = kOffSoff + 1025 * 4;
-    static constexpr int kOffSr = kOffFlag + BN * 4;
+    static constexpr int kOffSr = kOffSoff + 1025 * 4;
     static constexpr int kOffBar = ((kOffSr + 2 * BN * 4 + 7) / 8) * 8;
     static constexpr int kNumBars = 2 * kRS + 2 * kS + 4;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
@@ -108,7 +107,7 @@ struct F4Cfg {
     static constexpr int kWarpWiden = 4, kWarpTma = 8, kWarpMma = 9;
 };
 
-template <int BN, bool kSwiGLU, bool kFused, bool kGather>
+template <int BN, bool kSwiGLU, bool kGather>
 __global__ void __launch_bounds__(F4Cfg<BN>::kThreads, F4Cfg<BN>::kCtasPerSm)
     k_gemm_nvfp4(const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__ CUtensorMap tm_w1,
                  const __grid_constant__ CUtensorMap tm_act, const F4GemmArgs f) {
@@ -120,7 +119,6 @@ __global__ void __launch_bounds__(F4Cfg<BN>::kThreads, F4Cfg<BN>::kCtasPerSm)
     float* sX = reinterpret_cast<float*>(sm + C::kOffX);
     int* pre = reinterpret_cast<int*>(sm + C::kOffPre);
     int* soff = reinterpret_cast<int*>(sm + C::kOffSoff);
-    int* flag = reinterpret_cast<int*>(sm + C::kOffFlag);
     float* sSr = reinterpret_cast<float*>(sm + C::kOffSr);
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + C::kOffBar);
     uint64_t* full = bar;                  // stage filled: TMA bytes -> widening + MMA
@@ -318,8 +316,8 @@ __global__ void __launch_bounds__(F4Cfg<BN>::kThreads, F4Cfg<BN>::kCtasPerSm)
         }
     } else {
         // ------------------------------------------------------------ epilogue warps 0-3
-        w8_epilogue_warps<BN, kSwiGLU, kFused, kGather>(
-            a, n_tiles, m_tiles, pre, soff, sSr, sX, flag, tmem, t_full, t_empty, abort,
+        w8_epilogue_warps<BN, kSwiGLU, kGather>(
+            a, n_tiles, m_tiles, pre, soff, sSr, sX, tmem, t_full, t_empty, abort,
             [&](int e, int, int lrow) {
                 const int wb = weight_slab(f.slot_of, e);
                 return kSwiGLU ? (lrow < 64 ? f.s2_0[wb] : f.s2_1[wb]) : f.s2_0[wb];
@@ -337,7 +335,7 @@ __global__ void __launch_bounds__(F4Cfg<BN>::kThreads, F4Cfg<BN>::kCtasPerSm)
 
 // ---- host side --------------------------------------------------------------------------------
 
-template <int BN, bool kSwiGLU, bool kFused, bool kGather>
+template <int BN, bool kSwiGLU, bool kGather>
 int launch_gemm_nvfp4_inst(const F4GemmArgs& f, const void* act_f16, const void* w0, const void* w1,
                            int64_t max_row_tiles, cudaStream_t stream) {
     using C = F4Cfg<BN>;
@@ -345,7 +343,7 @@ int launch_gemm_nvfp4_inst(const F4GemmArgs& f, const void* act_f16, const void*
     static int sms_cache[16] = {0};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
-    auto kern = k_gemm_nvfp4<BN, kSwiGLU, kFused, kGather>;
+    auto kern = k_gemm_nvfp4<BN, kSwiGLU, kGather>;
     if (sms_cache[dev & 15] == 0) {
         int sms = 0;
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kAlloc) != cudaSuccess ||
@@ -375,9 +373,9 @@ int launch_gemm_nvfp4(const F4GemmArgs& f, const void* act_f16, const void* w0, 
     const int BN = tc_tile_rows(a.P, a.E);
     const int64_t max_row_tiles = ((int64_t)a.P + BN - 1) / BN + a.E;
     switch (BN) {
-        case 16: return launch_gemm_nvfp4_inst<16, kSwiGLU, true, kSwiGLU>(f, act_f16, w0, w1, max_row_tiles, stream);
-        case 32: return launch_gemm_nvfp4_inst<32, kSwiGLU, true, kSwiGLU>(f, act_f16, w0, w1, max_row_tiles, stream);
-        default: return launch_gemm_nvfp4_inst<128, kSwiGLU, false, false>(f, act_f16, w0, w1, max_row_tiles, stream);
+        case 16: return launch_gemm_nvfp4_inst<16, kSwiGLU, kSwiGLU>(f, act_f16, w0, w1, max_row_tiles, stream);
+        case 32: return launch_gemm_nvfp4_inst<32, kSwiGLU, kSwiGLU>(f, act_f16, w0, w1, max_row_tiles, stream);
+        default: return launch_gemm_nvfp4_inst<128, kSwiGLU, false>(f, act_f16, w0, w1, max_row_tiles, stream);
     }
 }
 

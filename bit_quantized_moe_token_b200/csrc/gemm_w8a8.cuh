@@ -20,8 +20,8 @@
 //              descriptor), so a segment's last, partly filled tile costs only what it holds.
 // Swap AB as in the W4A8 GEMM: MMA M = 128 weight rows (gate/up: 64 gate rows and the same 64
 // up rows), N = BN tokens of one expert's segment.  The epilogues are the W4A8 GEMM's: SwiGLU
-// with max|h| per row (narrow tiles: the requantization fused behind a row counter), or the
-// plain projection (narrow tiles: the combine fused behind a token counter).
+// with max|h| per row, or the plain projection; the requantization and the combine run as
+// their own passes after the GEMMs.
 //
 // Every mbarrier wait is bounded; a timeout sets the CTA's abort flag, later waits give up at
 // once, the device status is recorded and the CTA frees its TMEM and exits.
@@ -43,15 +43,8 @@ struct W8GemmArgs {
     float* out;             // SwiGLU: h [P, R0]; plain: Y [P, ldo]
     int ldo;
     unsigned* amax;         // SwiGLU: [P] float bits of max|h| per row
-    unsigned* cnt;          // fused epilogues: SwiGLU [P] row counters; plain [T * m_tiles]
-    uint8_t* hq;            // SwiGLU fused: [P, R0] requantized activations
-    float* s_h;             // SwiGLU fused: [P]
-    const int32_t* sorted;  // [P] pair of each sorted row
-    const int32_t* rop;     // plain fused: [P] sorted row of each pair
-    const float* gates;     // plain fused: [T, k]
+    const int32_t* sorted;  // [P] pair of each sorted row (gathering: token = pair / k)
     int k;
-    const float* shared;    // plain fused: [T, ldo] shared-expert output or null
-    uint16_t* out_bf16;     // plain fused: [T, ldo] layer output
     int T;                  // tokens (rows of the gathered activation tensor)
 };
 
@@ -69,8 +62,7 @@ struct W8Cfg {
     static constexpr int kOffX = kRS * kStage;
     static constexpr int kOffPre = kOffX + 64 * kXStride * 4;
     static constexpr int kOffSoff = kOffPre + 1025 * 4;     // segment offsets [0..E]
-    static constexpr int kOffFlag = kOffSoff + 1025 * 4;    // BN ints (fused epilogues)
-    static constexpr int kOffSr = kOffFlag + BN * 4;        // 2 x BN column scales
+    static constexpr int kOffSr = kOffSoff + 1025 * 4;      // 2 x BN column scales
     static constexpr int kOffBar = ((kOffSr + 2 * BN * 4 + 7) / 8) * 8;
     static constexpr int kNumBars = 2 * kRS + 4;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8; // TMEM slot, abort flag
@@ -84,13 +76,12 @@ struct W8Cfg {
 
 // The epilogue warps (threads 0..127, thread = TMEM lane = weight row): every tile's accumulator
 // times the tile's row scale rs_of(expert, m tile, row) and the column (token) scales, then the
-// SwiGLU epilogue (max|h| per row; narrow tiles: the requantization behind a row counter) or the
-// plain one (narrow tiles: the combine behind a token counter).  Shared by the FP8 and NVFP4
+// SwiGLU epilogue (h and max|h| per row) or the plain one (Y rows).  Shared by the FP8 and NVFP4
 // expert GEMMs, whose accumulators both hold the whole K.
-template <int BN, bool kSwiGLU, bool kFused, bool kGather, class RowScale>
+template <int BN, bool kSwiGLU, bool kGather, class RowScale>
 __device__ __forceinline__ void w8_epilogue_warps(const W8GemmArgs& a, int64_t n_tiles, int m_tiles,
                                                   const int* pre, const int* soff, float* sSr, float* sX,
-                                                  int* flag, uint32_t tmem, uint64_t* t_full,
+                                                  uint32_t tmem, uint64_t* t_full,
                                                   uint64_t* t_empty, volatile int* abort, RowScale rs_of) {
     constexpr int kXS = (BN < 32 ? BN : 32) + 1;         // SwiGLU exchange row stride
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -164,52 +155,10 @@ __device__ __forceinline__ void w8_epilogue_warps(const W8GemmArgs& a, int64_t n
         tc::tc_fence_before();
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(&t_empty[tb]);
-
-        if constexpr (kFused) {
-            // The barrier orders every thread's stores before the counting threads' fences,
-            // and a fence is cumulative, so one fence per counted row suffices.
-            ws::named_sync_math<kNPT>();
-            if constexpr (kSwiGLU) {
-                if (tid < nrows) {
-                    __threadfence();
-                    flag[tid] = atomicAdd(a.cnt + row0 + tid, 1u) == (unsigned)(m_tiles - 1);
-                }
-                ws::named_sync_math<kNPT>();
-                for (int j = 0; j < nrows; ++j) {
-                    if (flag[j]) {
-                        __threadfence();
-                        const int64_t r = row0 + j;
-                        requant_row(a.out + r * a.ldo, a.ldo, __ldcg(a.amax + r), a.hq + r * a.ldo,
-                                    a.s_h + r, tid, kNPT, nullptr);
-                    }
-                }
-            } else {
-                const int m = mt * 128 + lrow;
-                if (tid < nrows) {
-                    __threadfence();
-                    const int t = a.sorted[row0 + tid] / a.k;
-                    flag[tid] = atomicAdd(a.cnt + (int64_t)t * m_tiles + mt, 1u) == (unsigned)(a.k - 1) ? t : -1;
-                }
-                ws::named_sync_math<kNPT>();
-                for (int j = 0; j < nrows; ++j) {
-                    const int t = flag[j];
-                    if (t >= 0) {
-                        __threadfence();
-                        float o = 0.0f;
-                        for (int jj = 0; jj < a.k; ++jj)
-                            o = __fadd_rn(o, __fmul_rn(a.gates[t * a.k + jj],
-                                                       __ldcg(a.out + (int64_t)a.rop[t * a.k + jj] * a.ldo + m)));
-                        if (a.shared) o = __fadd_rn(o, a.shared[(int64_t)t * a.ldo + m]);
-                        a.out_bf16[(int64_t)t * a.ldo + m] = f32_to_bf16_bits(o);
-                    }
-                }
-            }
-            ws::named_sync_math<kNPT>();
-        }
     }
 }
 
-template <int BN, bool kSwiGLU, bool kFused, bool kGather>
+template <int BN, bool kSwiGLU, bool kGather>
 __global__ void __launch_bounds__(W8Cfg<BN>::kThreads, 1)
     k_gemm_w8a8(const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__ CUtensorMap tm_w1,
                 const __grid_constant__ CUtensorMap tm_act, const W8GemmArgs a) {
@@ -220,7 +169,6 @@ __global__ void __launch_bounds__(W8Cfg<BN>::kThreads, 1)
     float* sX = reinterpret_cast<float*>(sm + C::kOffX);
     int* pre = reinterpret_cast<int*>(sm + C::kOffPre);
     int* soff = reinterpret_cast<int*>(sm + C::kOffSoff);
-    int* flag = reinterpret_cast<int*>(sm + C::kOffFlag);
     float* sSr = reinterpret_cast<float*>(sm + C::kOffSr);
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + C::kOffBar);
     uint64_t* full = bar;                  // stage filled: TMA bytes -> MMA
@@ -346,8 +294,8 @@ __global__ void __launch_bounds__(W8Cfg<BN>::kThreads, 1)
         }
     } else {
         // ------------------------------------------------------------ epilogue warps 0-3
-        w8_epilogue_warps<BN, kSwiGLU, kFused, kGather>(
-            a, n_tiles, m_tiles, pre, soff, sSr, sX, flag, tmem, t_full, t_empty, abort,
+        w8_epilogue_warps<BN, kSwiGLU, kGather>(
+            a, n_tiles, m_tiles, pre, soff, sSr, sX, tmem, t_full, t_empty, abort,
             [&](int e, int mt, int lrow) {
                 return kSwiGLU ? __ldg((lrow < 64 ? a.rs0 : a.rs1) + (int64_t)e * a.R0 + mt * 64 + (lrow & 63))
                                : __ldg(a.rs0 + (int64_t)e * a.R0 + mt * 128 + lrow);
@@ -365,14 +313,14 @@ __global__ void __launch_bounds__(W8Cfg<BN>::kThreads, 1)
 
 // ---- host side --------------------------------------------------------------------------------
 
-template <int BN, bool kSwiGLU, bool kFused, bool kGather>
+template <int BN, bool kSwiGLU, bool kGather>
 int launch_gemm_w8a8_inst(const W8GemmArgs& a, const void* act, const void* w0, const void* w1,
                           int64_t max_row_tiles, cudaStream_t stream) {
     using C = W8Cfg<BN>;
     static int sms_cache[16] = {0};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
-    auto kern = k_gemm_w8a8<BN, kSwiGLU, kFused, kGather>;
+    auto kern = k_gemm_w8a8<BN, kSwiGLU, kGather>;
     if (sms_cache[dev & 15] == 0) {
         int sms = 0;
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kAlloc) != cudaSuccess ||
@@ -399,7 +347,7 @@ int launch_gemm_w8a8_inst(const W8GemmArgs& a, const void* act, const void* w0, 
 // cost little more than in a narrower tile, while long ones re-read each weight stage for 256
 // tokens instead of 64 or 128 (measured: the Zipf T = 2048 gate/up GEMM 0.67 -> 0.46 ms, T =
 // 16384 36 -> 50 % of the FP8 peak).  Narrow tiles gather their gate/up activation rows by
-// token and fuse the requantization / combine into the epilogues.
+// token.
 inline int w8_tile_rows(int64_t P, int E) {
     const int BN = tc_tile_rows(P, E);
     return BN <= 32 ? BN : 256;
@@ -411,9 +359,9 @@ int launch_gemm_w8a8(const W8GemmArgs& a, const void* act, const void* w0, const
     const int BN = w8_tile_rows(a.P, a.E);
     const int64_t max_row_tiles = ((int64_t)a.P + BN - 1) / BN + a.E;
     switch (BN) {
-        case 16: return launch_gemm_w8a8_inst<16, kSwiGLU, true, kSwiGLU>(a, act, w0, w1, max_row_tiles, stream);
-        case 32: return launch_gemm_w8a8_inst<32, kSwiGLU, true, kSwiGLU>(a, act, w0, w1, max_row_tiles, stream);
-        default: return launch_gemm_w8a8_inst<256, kSwiGLU, false, false>(a, act, w0, w1, max_row_tiles, stream);
+        case 16: return launch_gemm_w8a8_inst<16, kSwiGLU, kSwiGLU>(a, act, w0, w1, max_row_tiles, stream);
+        case 32: return launch_gemm_w8a8_inst<32, kSwiGLU, kSwiGLU>(a, act, w0, w1, max_row_tiles, stream);
+        default: return launch_gemm_w8a8_inst<256, kSwiGLU, false>(a, act, w0, w1, max_row_tiles, stream);
     }
 }
 

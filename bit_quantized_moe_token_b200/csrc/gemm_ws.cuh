@@ -55,21 +55,12 @@ struct WsGemmArgs {
     float* out;             // SwiGLU: h [P, R0]; plain: Y [P, ldo]
     int ldo;
     unsigned* amax;         // SwiGLU: [P] float bits of max|h| per row
-    // fused epilogues (narrow tiles): counters zeroed by the front kernel
-    unsigned* cnt;          // SwiGLU: [P] finished M tiles per row; plain: [T * m_tiles] per token
-    uint8_t* hq;            // SwiGLU: [P, R0] requantized activations
-    float* s_h;             // SwiGLU: [P]
-    const int32_t* sorted;  // [P] pair of each sorted row
-    const int32_t* rop;     // plain: [P] sorted row of each pair
-    const float* gates;     // plain: [T, k]
+    const int32_t* sorted;  // [P] pair of each sorted row (gathering: token = pair / k)
     int k;
-    const float* shared;    // plain: [T, ldo] shared-expert output or null
-    uint16_t* out_bf16;     // plain: [T, ldo] layer output
     int T;                  // tokens (rows of the gathered activation tensor)
     // unsigned widening: per (activation row, K-group) sums of the FP8 values the GEMM reads
     // (per token when gathering, per sorted row otherwise), for the +8 offset correction
     const float* qsum;
-    float* qsum_out;        // SwiGLU fused: the same sums of the requantized rows [P, R0/128]
     // hybrid layers: expert -> slab map (null: slab = expert) and the experts this launch takes
     const int32_t* slot_of = nullptr;
     int slot_want = 0;
@@ -115,8 +106,7 @@ struct WsCfg {
     static constexpr int kOffUs = kOffW + kRW * kRaw;
     static constexpr int kOffPre = kOffUs + 64 * kUsStride * 4;
     static constexpr int kOffSoff = kOffPre + 1025 * 4;          // segment offsets [0..E]
-    static constexpr int kOffFlag = kOffSoff + 1025 * 4;         // BN ints (fused epilogues)
-    static constexpr int kOffSr = kOffFlag + BN * 4;             // 2 x BN per-column scales
+    static constexpr int kOffSr = kOffSoff + 1025 * 4;           // 2 x BN per-column scales
     static constexpr int kMaxG = 128;                            // K <= 16384
     static constexpr int kOffQs = kOffSr + 2 * BN * 4;           // unsigned: [G][BN] group sums
     static constexpr int kOffBar = ((kOffQs + (kUnsigned ? kMaxG * BN * 4 : 0) + 7) / 8) * 8;
@@ -137,7 +127,7 @@ struct WsCfg {
     static constexpr int kThreads = 32 * (kNW + kNP + 2);
 };
 
-template <int BN, bool kUnsigned, bool kSwiGLU, bool kFused, bool kGather>
+template <int BN, bool kUnsigned, bool kSwiGLU, bool kGather>
 __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUnsigned>::kCtasPerSm)
     k_gemm_w4a8_ws(const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__ CUtensorMap tm_w1,
                    const __grid_constant__ CUtensorMap tm_act, const WsGemmArgs a) {
@@ -149,7 +139,6 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
     float* sUs = reinterpret_cast<float*>(sm + C::kOffUs);
     int* pre = reinterpret_cast<int*>(sm + C::kOffPre);
     int* soff = reinterpret_cast<int*>(sm + C::kOffSoff);
-    int* flag = reinterpret_cast<int*>(sm + C::kOffFlag);
     float* sSr = reinterpret_cast<float*>(sm + C::kOffSr);
     float* sQs = reinterpret_cast<float*>(sm + C::kOffQs);
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + C::kOffBar);
@@ -526,54 +515,13 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
                     const unsigned m = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(acc[j])));
                     if (lane == 0 && c_mine + j < nrows) atomicMax(a.amax + row0 + c_mine + j, m);
                 }
-                if constexpr (kFused) {
-                    // The barrier orders every thread's h stores before the counting threads'
-                    // fences, and a fence is cumulative, so one fence per counted row suffices.
-                    ws::named_sync_math<kNPT>();
-                    if (pt < nrows) {
-                        __threadfence();
-                        flag[pt] = atomicAdd(a.cnt + row0 + pt, 1u) == (unsigned)(m_tiles - 1);
-                    }
-                    ws::named_sync_math<kNPT>();
-                    for (int j = 0; j < nrows; ++j) {
-                        if (flag[j]) {
-                            __threadfence();
-                            const int64_t r = row0 + j;
-                            requant_row(a.out + r * a.ldo, a.ldo, __ldcg(a.amax + r), a.hq + r * a.ldo,
-                                        a.s_h + r, pt, kNPT,
-                                        a.qsum_out ? a.qsum_out + r * (a.ldo / kGroup) : nullptr);
-                        }
-                    }
-                }
-                ws::named_sync_math<kNPT>();
+                ws::named_sync_math<kNPT>();                  // exchange buffer free again
             } else {
                 const int m = mt * 128 + lrow;
                 ws::named_sync_math<kNPT>();
 #pragma unroll
                 for (int j = 0; j < kCPW; ++j)
                     if (c_base + j < nrows) a.out[(row0 + c_base + j) * a.ldo + m] = acc[j] * sr_t[c_base + j];
-                if constexpr (kFused) {
-                    ws::named_sync_math<kNPT>();          // as above: one fence per counted row
-                    if (pt < nrows) {
-                        __threadfence();
-                        const int t = a.sorted[row0 + pt] / a.k;
-                        flag[pt] = atomicAdd(a.cnt + (int64_t)t * m_tiles + mt, 1u) == (unsigned)(a.k - 1) ? t : -1;
-                    }
-                    ws::named_sync_math<kNPT>();
-                    for (int j = 0; j < nrows; ++j) {
-                        const int t = flag[j];
-                        if (t >= 0) {
-                            __threadfence();
-                            float o = 0.0f;
-                            for (int jj = 0; jj < a.k; ++jj)
-                                o = __fadd_rn(o, __fmul_rn(a.gates[t * a.k + jj],
-                                                           __ldcg(a.out + (int64_t)a.rop[t * a.k + jj] * a.ldo + m)));
-                            if (a.shared) o = __fadd_rn(o, a.shared[(int64_t)t * a.ldo + m]);
-                            a.out_bf16[(int64_t)t * a.ldo + m] = f32_to_bf16_bits(o);
-                        }
-                    }
-                    ws::named_sync_math<kNPT>();
-                }
             }
         }
     }
@@ -589,14 +537,14 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
 
 // ---- host side --------------------------------------------------------------------------------
 
-template <int BN, bool kUnsigned, bool kSwiGLU, bool kFused, bool kGather>
+template <int BN, bool kUnsigned, bool kSwiGLU, bool kGather>
 int launch_gemm_ws_inst(const WsGemmArgs& a, const void* act, const void* w0, const void* w1,
                         int64_t max_row_tiles, cudaStream_t stream) {
     using C = WsCfg<BN, kUnsigned>;
     static TcLaunchShape cache[16];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
-    auto kern = k_gemm_w4a8_ws<BN, kUnsigned, kSwiGLU, kFused, kGather>;
+    auto kern = k_gemm_w4a8_ws<BN, kUnsigned, kSwiGLU, kGather>;
     TcLaunchShape& c = cache[dev & 15];
     if (c.sms == 0) {
         int sms = 0;
@@ -621,8 +569,8 @@ int launch_gemm_ws_inst(const WsGemmArgs& a, const void* act, const void* w0, co
     return launch_status();
 }
 
-// Narrow token tiles (decode) fuse the requantization / combine into the GEMM epilogues, and
-// their gate/up instance gathers activation rows by token from the per-token FP8 array.
+// Narrow token tiles (decode): the gate/up instance gathers its activation rows by token from the
+// per-token FP8 array instead of an expert-sorted copy.
 inline bool ws_narrow(int BN) { return BN <= 32; }
 
 template <bool kSwiGLU>
@@ -634,10 +582,10 @@ int launch_gemm_ws(const WsGemmArgs& a, const void* act, const void* w0, const v
         // narrow gate/up tiles widen unsigned (the FP8 requantization after them absorbs the
         // accumulation error of the +8 offset); the down GEMM, whose sums are the layer output,
         // keeps the exact signed codes
-        case 16: return launch_gemm_ws_inst<16, kSwiGLU, kSwiGLU, true, kSwiGLU>(a, act, w0, w1, max_row_tiles, stream);
-        case 32: return launch_gemm_ws_inst<32, kSwiGLU, kSwiGLU, true, kSwiGLU>(a, act, w0, w1, max_row_tiles, stream);
-        case 128: return launch_gemm_ws_inst<128, false, kSwiGLU, false, false>(a, act, w0, w1, max_row_tiles, stream);
-        default: return launch_gemm_ws_inst<192, false, kSwiGLU, false, false>(a, act, w0, w1, max_row_tiles, stream);
+        case 16: return launch_gemm_ws_inst<16, kSwiGLU, kSwiGLU, kSwiGLU>(a, act, w0, w1, max_row_tiles, stream);
+        case 32: return launch_gemm_ws_inst<32, kSwiGLU, kSwiGLU, kSwiGLU>(a, act, w0, w1, max_row_tiles, stream);
+        case 128: return launch_gemm_ws_inst<128, false, kSwiGLU, false>(a, act, w0, w1, max_row_tiles, stream);
+        default: return launch_gemm_ws_inst<192, false, kSwiGLU, false>(a, act, w0, w1, max_row_tiles, stream);
     }
 }
 

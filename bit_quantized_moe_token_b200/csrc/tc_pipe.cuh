@@ -64,35 +64,6 @@ __device__ __forceinline__ bool wait(uint64_t* bar, uint32_t parity, volatile in
 
 }  // namespace ws
 
-// Fused decode epilogues.  Requantization (S5) of a row needs max|h| over all of its M tiles,
-// and the combine (S7) of a token needs all k routed rows: the CTA that finishes the last
-// contribution (counted with a device-scope atomic after a fence) does that work, reading the
-// other CTAs' outputs through L2.  The result does not depend on which CTA finishes last.
-__device__ __forceinline__ void requant_row(const float* __restrict__ h, int N, unsigned amax_bits,
-                                            uint8_t* __restrict__ hq, float* __restrict__ s_h, int tid,
-                                            int nthreads, float* __restrict__ qs_row) {
-    const float s = __fdiv_rn(__uint_as_float(amax_bits), kFp8Max);
-    for (int base = 0; base < (N >> 3); base += nthreads) {
-        const int c = base + tid;
-        const bool live = c < (N >> 3);
-        uint2 codes = make_uint2(0u, 0u);
-        if (live && s != 0.0f) {
-            const float4 a = __ldcg(reinterpret_cast<const float4*>(h) + 2 * c);
-            const float4 b = __ldcg(reinterpret_cast<const float4*>(h) + 2 * c + 1);
-            codes.x = static_cast<uint32_t>(f32x2_to_e4m3x2(__fdiv_rn(a.x, s), __fdiv_rn(a.y, s))) |
-                      (static_cast<uint32_t>(f32x2_to_e4m3x2(__fdiv_rn(a.z, s), __fdiv_rn(a.w, s))) << 16);
-            codes.y = static_cast<uint32_t>(f32x2_to_e4m3x2(__fdiv_rn(b.x, s), __fdiv_rn(b.y, s))) |
-                      (static_cast<uint32_t>(f32x2_to_e4m3x2(__fdiv_rn(b.z, s), __fdiv_rn(b.w, s))) << 16);
-        }
-        if (live) reinterpret_cast<uint2*>(hq)[c] = codes;
-        if (qs_row) {   // sums of the decoded codes per K-group of 128 (16 chunks = one half-warp)
-            const float gs = halfwarp_sum(e4m3x8_sum(codes));
-            if (live && (tid & 15) == 0) qs_row[c / 16] = gs;
-        }
-    }
-    if (tid == 0) *s_h = s;
-}
-
 // ---- host side --------------------------------------------------------------------------------
 
 using PFN_encodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,

@@ -120,8 +120,8 @@ struct TcLaunchShape {
 };
 
 // Token-tile width for the expected rows per expert: 16 / 32 rows at decode (narrow tiles: the
-// unsigned widening and the fused epilogues), else 128 rows.  Wide tiles are as wide as TMEM
-// allows whatever the average, because routed segments are skewed: with Zipf routing at
+// unsigned widening and the gathered activation rows), else 128 rows.  Wide tiles are as wide
+// as TMEM allows whatever the average, because routed segments are skewed: with Zipf routing at
 // T = 2048 (48 rows per expert on average) the popular experts' long segments dominate the
 // work, and 128-row tiles re-read each of their weight tiles half as often as 64-row ones
 // (measured: W4A8 gate/up 1.14 -> 0.94 ms).

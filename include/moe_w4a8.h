@@ -339,8 +339,8 @@ int moe_nvfp4_forward_profiled(const moe_nvfp4_layer* layer, const uint16_t* x_b
  * experts into a small hot set kept in NVFP4 and a cold set in another format, with hot_ids /
  * cold_ids giving the routed expert of each slab (together a partition of 0..E-1).  Here the
  * cold format is W4A8.  Each routed pair runs the projections of its expert's format; the two
- * formats' grouped GEMMs share the routing, the permutation, the requantization, the combine
- * and (at decode sizes) the fused epilogues' counters.
+ * formats' grouped GEMMs share the routing, the permutation, the requantization and the
+ * combine.
  *   hot_ids  [n_hot] int32, cold_ids [n_cold] int32: must partition 0..E-1 (ids outside [0, E)
  *            are ignored; an expert in neither list contributes nothing)
  *   hot_*    NVFP4 slabs as in moe_nvfp4_layer with n_hot slabs
