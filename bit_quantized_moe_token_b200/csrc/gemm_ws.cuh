@@ -6,10 +6,12 @@
 //              row's packed INT4 codes from the TMA stage (the 64- or 128-byte TMA swizzle spreads
 //              the 32 rows of a warp over distinct banks), widens them to E4M3 and writes them
 //              into a TMEM A stage with tcgen05.st; the MMA takes A from TMEM.
-//   promotion warps (4 on narrow tiles, 16 on 128-row tiles, each owning a lane quadrant and a
-//              slice of the token columns): per K-group they fold the group's TMEM partial into
-//              fp32 register accumulators with the group scale (acc += s[n,g] * partial, two
-//              columns per packed FMA), then run the tile's epilogue.
+//   promotion warps (4 on narrow tiles, 16 on 128- and 192-row tiles, each owning a lane
+//              quadrant and a slice of the token columns): per K-group they fold the group's TMEM
+//              partial into fp32 register accumulators with the group scale (acc += s[n,g] *
+//              partial, two columns per packed FMA), then run the tile's epilogue: SwiGLU, h rows
+//              and max|h| per row (gate/up), or Y rows (down).  Requantization and combine are
+//              separate passes after the GEMMs.
 //   TMA warp:  streams the packed weight tiles into a weight ring and the activation tiles
 //              (BN rows x 128 B per group, landing pre-swizzled for the MMA) into an activation
 //              ring; narrow gate/up tiles gather their live token rows four at a time.

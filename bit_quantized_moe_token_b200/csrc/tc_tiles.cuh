@@ -130,7 +130,6 @@ inline int tc_tile_rows(int64_t P, int E) {
     const int64_t avg = (P + E - 1) / E;
     return avg <= 8 ? 16 : avg <= 24 ? 32 : 128;
 }
-inline bool tc_unsigned(int BN) { return BN <= 32; }
 
 // The W4A8 GEMM widens each weight stage once per token tile, so long segments want the widest
 // tile whose partial buffers still leave TMEM room for the widened A stages: 192 rows (two
