@@ -208,9 +208,8 @@ int moe_w4a8_forward(const moe_w4a8_layer* layer, const uint16_t* x_bf16,
  * boundaries below, and the number of kernels the call launched in *n_launches (may be NULL).
  *   0 start  1 routed (top-k + permutation)  2 tokens quantized  3 shared experts done
  *   4 gate/up GEMM done  5 SwiGLU requant done  6 down GEMM done  7 combined (end).
- * Stages that a call fuses into a neighbour (the decode path fuses routing with
- * quantization, the requantization into the gate/up GEMM and the combine into the down GEMM)
- * show as zero-length intervals. */
+ * Stages that a call fuses into a neighbour (the decode path quantizes the tokens in the
+ * routing kernel) show as zero-length intervals. */
 #define MOE_W4A8_N_STAGE_EVENTS 8
 int moe_w4a8_forward_profiled(const moe_w4a8_layer* layer, const uint16_t* x_bf16,
                               const float* router_logits, int64_t T, int k, uint16_t* out_bf16,
