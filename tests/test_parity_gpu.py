@@ -549,7 +549,7 @@ def test_w8a8_forward_tiny_workload():
     assert np.array_equal(r1["out"], r2["out"])        # deterministic
 
 
-# token tiles of 16 (decode, fused), 32 (fused) and 256 rows (with the MMA's N following the
+# token tiles of 16 (decode, gathered rows), 32 (gathered) and 256 rows (with the MMA's N following the
 # live rows: segments of every length from 1 to several hundred rows)
 @pytest.mark.parametrize("E,H,N,k,T", [(5, 384, 256, 3, 37), (1, 256, 128, 1, 9), (8, 256, 128, 2, 1),
                                        (8, 256, 256, 2, 200), (16, 512, 384, 8, 130),
@@ -776,8 +776,9 @@ def _host_layer_and_dev_hybrid(E, H, N, seed, hot_ids):
                                            (8, 256, 256, 2, 600, [2, 7]), (4, 256, 128, 2, 21, [0, 1, 2, 3]),
                                            (4, 256, 128, 2, 21, []), (64, 1024, 1024, 6, 16, list(range(0, 64, 7)))])
 def test_hybrid_forward(E, H, N, k, T, hot):
-    """Hot experts on the NVFP4 GEMM, cold ones on the W4A8 GEMM, in one layer (decode: fused
-    epilogues counting both GEMMs' contributions; prefill; all hot; all cold)."""
+    """Hot experts on the NVFP4 GEMM, cold ones on the W4A8 GEMM, in one layer (decode: both
+    GEMMs write their rows of h and Y before the shared requantization and combine; prefill;
+    all hot; all cold)."""
     hl, dl = _host_layer_and_dev_hybrid(E, H, N, seed=E + T + len(hot), hot_ids=hot)
     x = synth.normal_bf16(11, 840 + T, T * H).reshape(T, H)
     logits = synth.normal_f32(11, 841 + T, T * E).reshape(T, E)
