@@ -549,8 +549,8 @@ def test_w8a8_forward_tiny_workload():
     assert np.array_equal(r1["out"], r2["out"])        # deterministic
 
 
-# token tiles of 16 (decode, gathered rows), 32 (gathered) and 256 rows (with the MMA's N following the
-# live rows: segments of every length from 1 to several hundred rows)
+# token tiles of 16 (decode, gathered rows), 32 (gathered) and 256 rows (with the MMA's N
+# following the live rows: segments of every length from 1 to several hundred rows)
 @pytest.mark.parametrize("E,H,N,k,T", [(5, 384, 256, 3, 37), (1, 256, 128, 1, 9), (8, 256, 128, 2, 1),
                                        (8, 256, 256, 2, 200), (16, 512, 384, 8, 130),
                                        (8, 256, 256, 2, 600), (3, 1024, 128, 2, 700),
