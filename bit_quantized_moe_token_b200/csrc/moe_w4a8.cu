@@ -3,6 +3,7 @@
 // Every kernel of the library is compiled here so that the device-status word below is one
 // symbol without relocatable device code.
 #include <algorithm>
+#include <atomic>
 
 #include "common.cuh"
 
@@ -76,19 +77,25 @@ namespace moe {
 constexpr size_t kRouteStaticBytes = 256 * 1024;
 static __device__ __align__(256) int32_t g_route_static_scratch[kRouteStaticBytes / sizeof(int32_t)];
 
-// Device address of the array on the current device, looked up once per device.  Host code may
-// not pass `g_route_static_scratch` itself to a kernel: on the host that name is only a stand-in.
+// Device address of the array on the current device, looked up on the first call made with that
+// device current and kept per device.  Host code may not pass `g_route_static_scratch` itself to a
+// kernel: on the host that name is only a stand-in.  The slots are atomics, so host threads making
+// their first calls at the same time only repeat the lookup (each stores the same address).  A
+// cudaDeviceReset() unloads the library's module on that device; the cached address is then
+// stale, and a process that resets a device must not call this entry point on it again.
 static int route_static_scratch(int32_t** out) {
-    static int32_t* cache[64] = {};
+    static std::atomic<int32_t*> cache[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
     if (dev < 0 || dev >= 64) return MOE_ERR_UNSUPPORTED_SHAPE;
-    if (!cache[dev]) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_route_static_scratch) != cudaSuccess || !p) return MOE_ERR_CUDA;
-        cache[dev] = static_cast<int32_t*>(p);
+    int32_t* p = cache[dev].load(std::memory_order_acquire);
+    if (!p) {
+        void* q = nullptr;
+        if (cudaGetSymbolAddress(&q, g_route_static_scratch) != cudaSuccess || !q) return MOE_ERR_CUDA;
+        p = static_cast<int32_t*>(q);
+        cache[dev].store(p, std::memory_order_release);
     }
-    *out = cache[dev];
+    *out = p;
     return MOE_OK;
 }
 

@@ -409,7 +409,9 @@ int moe_selftest_bounded_wait(int64_t limit_ns, moe_stream_t stream);
  * caller's.  It supports shapes with moe_route_workspace_bytes(T, E, k) <= that size (for
  * E = 256, up to 262,144 routed pairs) and returns MOE_ERR_UNSUPPORTED_SHAPE beyond it.
  * The first call on a device looks up the array's device address (cudaGetSymbolAddress), so
- * make that first call before any stream capture.  All calls share the one array: calls that
+ * make that first call before any stream capture; the address is kept per device (safe when
+ * several host threads make their first calls at once) and does not survive a cudaDeviceReset()
+ * of that device.  All calls share the one array: calls that
  * overlap on the GPU (issued on streams with no ordering between them) race and must be
  * serialised by the caller.  Every scratch word a call reads is written earlier in the same
  * call, so stale contents from a previous call do not matter.  Never allocates or frees. */

@@ -105,8 +105,21 @@ def lib():
         L.or_moe_forward_given_h.argtypes = [ctypes.POINTER(_Layer), vp, vp, i64, i32, vp, vp, vp, vp]
         L.or_moe_forward_given_h.restype = i32
         L.or_moe_forward_dense.restype = i32
+        L.or_set_threads.argtypes = [i32]
+        L.or_set_threads.restype = None
+        L.or_max_threads.argtypes = []
+        L.or_max_threads.restype = i32
         _lib = L
     return _lib
+
+
+def set_threads(n: int) -> None:
+    """Threads the oracle's OpenMP loops use from now on (timing only: results do not change)."""
+    lib().or_set_threads(int(n))
+
+
+def max_threads() -> int:
+    return int(lib().or_max_threads())
 
 
 def _p(a):
@@ -382,24 +395,46 @@ def moe_forward_dense(layer: Layer, x_bf16: np.ndarray, logits: np.ndarray, k: i
     return r
 
 
-def pack_workload_layer(wl, experts=None, with_shared=True):
+def _each_expert(fn, experts):
+    """fn(e) for every expert, on a pool of host threads (the C routines release the GIL; each
+    expert writes only its own slabs, so the result does not depend on the order)."""
+    from concurrent.futures import ThreadPoolExecutor
+    experts = list(experts)
+    n = min(len(experts), os.cpu_count() or 1)
+    if n <= 1:
+        for e in experts:
+            fn(e)
+        return
+    with ThreadPoolExecutor(n) as ex:
+        list(ex.map(fn, experts))
+
+
+def pack_workload_layer(wl, experts=None, with_shared=True, into=None):
     """Pack (RTN, oracle side) the seeded weights of workload `wl`.
 
     Only experts in `experts` (default: all) are drawn and packed; the others stay zero,
-    which is enough when the caller knows which experts its tokens route to.
+    which is enough when the caller knows which experts its tokens route to.  With `into` (a
+    Layer of this workload's shapes) the experts are packed into its arrays and it is returned.
     """
     import synth
     E, H, N, g = wl.E, wl.H, wl.N, wl.group
-    gp = np.zeros((E, N, H // 8), np.int32)
-    up = np.zeros((E, N, H // 8), np.int32)
-    dp = np.zeros((E, H, N // 8), np.int32)
-    gs = np.zeros((E, N, H // g), np.uint16)
-    us = np.zeros((E, N, H // g), np.uint16)
-    ds = np.zeros((E, H, N // g), np.uint16)
-    for e in (range(E) if experts is None else experts):
+    if into is not None:
+        gp, up, dp = into.gate_packed, into.up_packed, into.down_packed
+        gs, us, ds = into.gate_scales, into.up_scales, into.down_scales
+    else:
+        gp = np.zeros((E, N, H // 8), np.int32)
+        up = np.zeros((E, N, H // 8), np.int32)
+        dp = np.zeros((E, H, N // 8), np.int32)
+        gs = np.zeros((E, N, H // g), np.uint16)
+        us = np.zeros((E, N, H // g), np.uint16)
+        ds = np.zeros((E, H, N // g), np.uint16)
+    def one(e):
         gp[e], gs[e], _ = rtn_pack(synth.expert_weight(wl, e, "gate"), g)
         up[e], us[e], _ = rtn_pack(synth.expert_weight(wl, e, "up"), g)
         dp[e], ds[e], _ = rtn_pack(synth.expert_weight(wl, e, "down"), g)
+    _each_expert(one, range(E) if experts is None else experts)
+    if into is not None:
+        return into
     sh = {}
     if with_shared and wl.n_shared:
         sh = dict(sh_gate=np.stack([synth.shared_weight(wl, s, "gate") for s in range(wl.n_shared)]),
@@ -408,21 +443,28 @@ def pack_workload_layer(wl, experts=None, with_shared=True):
     return Layer(E, H, N, gp, up, dp, gs, us, ds, group=g, **sh)
 
 
-def quant_workload_layer_w8a8(wl, experts=None, with_shared=True):
+def quant_workload_layer_w8a8(wl, experts=None, with_shared=True, into=None):
     """Row-quantize (oracle side) the seeded weights of workload `wl` to the row-scaled FP8
-    format; experts outside `experts` stay zero, as in ``pack_workload_layer``."""
+    format; experts outside `experts` stay zero, and `into` fills a given layer, as in
+    ``pack_workload_layer``."""
     import synth
     E, H, N = wl.E, wl.H, wl.N
-    gq = np.zeros((E, N, H), np.uint8)
-    uq = np.zeros((E, N, H), np.uint8)
-    dq = np.zeros((E, H, N), np.uint8)
-    gs = np.zeros((E, N), np.float32)
-    us = np.zeros((E, N), np.float32)
-    ds = np.zeros((E, H), np.float32)
-    for e in (range(E) if experts is None else experts):
+    if into is not None:
+        gq, uq, dq, gs, us, ds = into.gate_w8, into.up_w8, into.down_w8, into.gate_rs, into.up_rs, into.down_rs
+    else:
+        gq = np.zeros((E, N, H), np.uint8)
+        uq = np.zeros((E, N, H), np.uint8)
+        dq = np.zeros((E, H, N), np.uint8)
+        gs = np.zeros((E, N), np.float32)
+        us = np.zeros((E, N), np.float32)
+        ds = np.zeros((E, H), np.float32)
+    def one(e):
         gq[e], gs[e] = quant_rows(synth.expert_weight(wl, e, "gate"))
         uq[e], us[e] = quant_rows(synth.expert_weight(wl, e, "up"))
         dq[e], ds[e] = quant_rows(synth.expert_weight(wl, e, "down"))
+    _each_expert(one, range(E) if experts is None else experts)
+    if into is not None:
+        return into
     sh = {}
     if with_shared and wl.n_shared:
         sh = dict(sh_gate=np.stack([synth.shared_weight(wl, s, "gate") for s in range(wl.n_shared)]),
@@ -431,19 +473,27 @@ def quant_workload_layer_w8a8(wl, experts=None, with_shared=True):
     return Layer.w8a8(E, H, N, gq, uq, dq, gs, us, ds, group=wl.group, **sh)
 
 
-def quant_workload_layer_nvfp4(wl, experts=None, with_shared=True):
+def quant_workload_layer_nvfp4(wl, experts=None, with_shared=True, into=None):
     """NVFP4-quantize (oracle side) the seeded weights of workload `wl`; experts outside
-    `experts` stay zero, as in ``pack_workload_layer``."""
+    `experts` stay zero, and `into` fills a given layer, as in ``pack_workload_layer``."""
     import synth
     E, H, N = wl.E, wl.H, wl.N
-    c = {p: np.zeros((E, *synth.weight_shape(wl, p)[:1], synth.weight_shape(wl, p)[1] // 2), np.uint8)
-         for p in ("gate", "up", "down")}
-    b = {p: np.zeros((E, *synth.weight_shape(wl, p)[:1], synth.weight_shape(wl, p)[1] // 16), np.uint8)
-         for p in ("gate", "up", "down")}
-    s2 = {p: np.zeros(E, np.float32) for p in ("gate", "up", "down")}
-    for e in (range(E) if experts is None else experts):
+    if into is not None:
+        c = {"gate": into.gate_f4, "up": into.up_f4, "down": into.down_f4}
+        b = {"gate": into.gate_bs, "up": into.up_bs, "down": into.down_bs}
+        s2 = {"gate": into.gate_s2, "up": into.up_s2, "down": into.down_s2}
+    else:
+        c = {p: np.zeros((E, *synth.weight_shape(wl, p)[:1], synth.weight_shape(wl, p)[1] // 2), np.uint8)
+             for p in ("gate", "up", "down")}
+        b = {p: np.zeros((E, *synth.weight_shape(wl, p)[:1], synth.weight_shape(wl, p)[1] // 16), np.uint8)
+             for p in ("gate", "up", "down")}
+        s2 = {p: np.zeros(E, np.float32) for p in ("gate", "up", "down")}
+    def one(e):
         for p in ("gate", "up", "down"):
             c[p][e], b[p][e], s2[p][e] = nvfp4_quant(synth.expert_weight(wl, e, p))
+    _each_expert(one, range(E) if experts is None else experts)
+    if into is not None:
+        return into
     sh = {}
     if with_shared and wl.n_shared:
         sh = dict(sh_gate=np.stack([synth.shared_weight(wl, s, "gate") for s in range(wl.n_shared)]),

@@ -62,6 +62,12 @@
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
+#include <omp.h>
+
+/* Threads of the OpenMP loops below, for timing the oracle at a chosen core count; results never
+ * depend on it (every parallel loop runs over independent experts or tokens). */
+void or_set_threads(int n) { omp_set_num_threads(n > 0 ? n : 1); }
+int or_max_threads(void) { return omp_get_max_threads(); }
 
 /* ------------------------------------------------------------------------------------------ */
 /* bf16                                                                                        */
@@ -458,24 +464,22 @@ static void f4_proj(const uint8_t* q, float s_x, const float* cT, int64_t rows, 
 
 static float silu_f32(float g) { return g * (1.0f / (1.0f + expf(-g))); }
 
-/* Set only inside or_moe_forward_given_h: the expert rows take their requantized SwiGLU
- * activations (S5) as given instead of computing them, and run the down projection on them. */
-static int g_given_h = 0;
-
 /*
  * One routed row: token row q/s_x through expert weights (already unpacked), giving the
- * FP8 SwiGLU activations (hq, s_h) and the down-projection output y[H].
+ * FP8 SwiGLU activations (hq, s_h) and the down-projection output y[H].  With given_h set
+ * (or_moe_forward_given_h only) hq/s_h already hold the row's requantized SwiGLU activations
+ * and only the down projection runs.
  */
 static void expert_row(const uint8_t* q, float s_x, const float* cg, const float* cu,
                        const float* cd, const uint16_t* sg, const uint16_t* su, const uint16_t* sd,
                        int64_t H, int64_t N, int group, uint8_t* hq, float* s_h, float* y,
-                       float* scratch) {
+                       float* scratch, int given_h) {
     float* G = scratch;               /* N */
     float* U = G + N;                 /* N */
     float* h = U + N;                 /* N */
     float* part = h + N;              /* max(N,H) */
     float* acc = part + (H > N ? H : N);
-    if (!g_given_h) {
+    if (!given_h) {
         w4a8_proj(q, s_x, cg, sg, N, H, group, G, part, acc);
         w4a8_proj(q, s_x, cu, su, N, H, group, U, part, acc);
         for (int64_t n = 0; n < N; ++n) h[n] = silu_f32(G[n]) * U[n];
@@ -487,12 +491,13 @@ static void expert_row(const uint8_t* q, float s_x, const float* cg, const float
 /* expert_row for row-scaled FP8 experts (same steps, w8a8_proj for the three projections). */
 static void expert_row_w8(const uint8_t* q, float s_x, const float* cg, const float* cu,
                           const float* cd, const float* rg, const float* ru, const float* rd,
-                          int64_t H, int64_t N, uint8_t* hq, float* s_h, float* y, float* scratch) {
+                          int64_t H, int64_t N, uint8_t* hq, float* s_h, float* y, float* scratch,
+                          int given_h) {
     float* G = scratch;
     float* U = G + N;
     float* h = U + N;
     float* acc = h + N;
-    if (!g_given_h) {
+    if (!given_h) {
         w8a8_proj(q, s_x, cg, rg, N, H, G, acc);
         w8a8_proj(q, s_x, cu, ru, N, H, U, acc);
         for (int64_t n = 0; n < N; ++n) h[n] = silu_f32(G[n]) * U[n];
@@ -504,12 +509,12 @@ static void expert_row_w8(const uint8_t* q, float s_x, const float* cg, const fl
 /* expert_row for NVFP4 experts (same steps, f4_proj for the three projections). */
 static void expert_row_f4(const uint8_t* q, float s_x, const float* cg, const float* cu,
                           const float* cd, int64_t H, int64_t N, uint8_t* hq, float* s_h, float* y,
-                          float* scratch) {
+                          float* scratch, int given_h) {
     float* G = scratch;
     float* U = G + N;
     float* h = U + N;
     float* acc = h + N;
-    if (!g_given_h) {
+    if (!given_h) {
         f4_proj(q, s_x, cg, N, H, G, acc);
         f4_proj(q, s_x, cu, N, H, U, acc);
         for (int64_t n = 0; n < N; ++n) h[n] = silu_f32(G[n]) * U[n];
@@ -569,11 +574,9 @@ int or_moe_forward(const or_layer* L, const uint16_t* x, const float* logits, in
 int or_moe_forward_given_h(const or_layer* L, const uint16_t* x, const float* logits, int64_t T,
                            int k, const uint8_t* hq_pairs, const float* sh_pairs, uint16_t* out,
                            float* out_f32_o) {
-    g_given_h = 1;
-    int rc = moe_forward_impl(L, x, logits, T, k, out, NULL, NULL, NULL, NULL, NULL, NULL, NULL,
-                              NULL, NULL, NULL, out_f32_o, hq_pairs, sh_pairs);
-    g_given_h = 0;
-    return rc;
+    if (!hq_pairs || !sh_pairs) return -1;
+    return moe_forward_impl(L, x, logits, T, k, out, NULL, NULL, NULL, NULL, NULL, NULL, NULL,
+                            NULL, NULL, NULL, out_f32_o, hq_pairs, sh_pairs);
 }
 
 static int moe_forward_impl(const or_layer* L, const uint16_t* x, const float* logits, int64_t T,
@@ -590,6 +593,7 @@ static int moe_forward_impl(const or_layer* L, const uint16_t* x, const float* l
             if (expert_fmt(L, e, &b) < 0) return -1;
         }
     const int64_t P = T * k;
+    const int given_h = hq_pairs != NULL;   /* S5's results given: only S6..S8 run */
 
     int32_t* ids = (int32_t*)malloc((size_t)(P > 0 ? P : 1) * 4);
     float* gates = (float*)malloc((size_t)(P > 0 ? P : 1) * 4);
@@ -643,14 +647,14 @@ static int moe_forward_impl(const or_layer* L, const uint16_t* x, const float* l
             if (f == 1)
                 expert_row_w8(xq + t * H, sx[t], cg, cu, cd, L->gate_rs + b * N, L->up_rs + b * N,
                               L->down_rs + b * H, H, N, hq + (int64_t)r * N, sh + r,
-                              y + (int64_t)r * H, scratch);
+                              y + (int64_t)r * H, scratch, given_h);
             else if (f == 2)
                 expert_row_f4(xq + t * H, sx[t], cg, cu, cd, H, N, hq + (int64_t)r * N, sh + r,
-                              y + (int64_t)r * H, scratch);
+                              y + (int64_t)r * H, scratch, given_h);
             else
                 expert_row(xq + t * H, sx[t], cg, cu, cd, L->gate_scales + b * N * G_h,
                            L->up_scales + b * N * G_h, L->down_scales + b * H * G_n, H, N, group,
-                           hq + (int64_t)r * N, sh + r, y + (int64_t)r * H, scratch);
+                           hq + (int64_t)r * N, sh + r, y + (int64_t)r * H, scratch, given_h);
         }
         free(cg); free(cu); free(cd); free(scratch);
     }
@@ -752,15 +756,15 @@ int or_moe_forward_dense(const or_layer* L, const uint16_t* x, const float* logi
             if (f == 1)
                 expert_row_w8(xq + t * H, sx[t], cg, cu, cd, L->gate_rs + b * N, L->up_rs + b * N,
                               L->down_rs + b * H, H, N, hq_dense + (t * E + e) * N,
-                              sh_dense + t * E + e, y_dense + (t * E + e) * H, scratch);
+                              sh_dense + t * E + e, y_dense + (t * E + e) * H, scratch, 0);
             else if (f == 2)
                 expert_row_f4(xq + t * H, sx[t], cg, cu, cd, H, N, hq_dense + (t * E + e) * N,
-                              sh_dense + t * E + e, y_dense + (t * E + e) * H, scratch);
+                              sh_dense + t * E + e, y_dense + (t * E + e) * H, scratch, 0);
             else
                 expert_row(xq + t * H, sx[t], cg, cu, cd, L->gate_scales + b * N * G_h,
                            L->up_scales + b * N * G_h, L->down_scales + b * H * G_n, H, N, group,
                            hq_dense + (t * E + e) * N, sh_dense + t * E + e,
-                           y_dense + (t * E + e) * H, scratch);
+                           y_dense + (t * E + e) * H, scratch, 0);
         }
     }
     float* dense_gate = (float*)malloc((size_t)E * 4);

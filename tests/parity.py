@@ -4,16 +4,18 @@
    bit-exact.
 2. Intermediate FP8 codes (the requantized SwiGLU activations): at most 0.1% differ, and
    those by at most one E4M3 step.
-3. Each bf16 output element within 1e-2 * max(|ref|, rms(ref row)).
+3. Each bf16 output element within 1e-2 * max(|ref|, rms(ref row)) of the oracle's.
 
-Where fp32 arithmetic decides an integer (an FP8 code after a GPU sum with a different
-accumulation order than the oracle's), rule 2 is what allows the difference.  Such a permitted
-code difference propagates into the outputs of its token (one E4M3 step of a large activation,
-through a short down projection, can move an output by more than rule 3's tolerance), so rule 3
-is applied with that allowance: an output outside the tolerance of the oracle's passes only if
-its token has a requantized code that differs from the oracle's and the output is within the
+Rule 3 is checked against the oracle alone.  One allowance exists, and only a test that names
+the expert format and the seeded case needing it may use it: where fp32 arithmetic decides an
+integer (an FP8 code after a GPU sum in another accumulation order than the oracle's), rule 2
+permits the difference, and such a code difference propagates into the outputs of its token
+(one E4M3 step of a large activation, through a short down projection, can move an output by
+more than rule 3's tolerance).  Under the allowance an output outside the tolerance passes only
+if its token has a requantized code that differs from the oracle's, the output is within the
 tolerance of the oracle's layer evaluated on the GPU's requantized codes (the oracle's own down
-projection and combine, see oracle.moe_forward_given_h).
+projection and combine, see oracle.moe_forward_given_h), and at most a capped number of outputs
+need it.
 """
 import numpy as np
 
@@ -41,21 +43,29 @@ def bf16_to_f32(h: np.ndarray) -> np.ndarray:
     return (np.asarray(h, np.uint16).astype(np.uint32) << 16).view(np.float32)
 
 
-def check_output(got_bf16: np.ndarray, ref_bf16: np.ndarray, rtol=OUT_RTOL):
+def output_errors(got_bf16: np.ndarray, ref_bf16: np.ndarray, rtol=OUT_RTOL):
+    """Per-output error as a fraction of rule 3's tolerance (> 1: out of tolerance)."""
     g = bf16_to_f32(got_bf16).astype(np.float64)
     r = bf16_to_f32(ref_bf16).astype(np.float64)
     rms = np.sqrt((r ** 2).mean(axis=1, keepdims=True))
     tol = rtol * np.maximum(np.abs(r), rms)
-    err = np.abs(g - r)
-    bad = err > tol
+    return np.abs(g - r) / np.maximum(tol, 1e-30)
+
+
+def check_output(got_bf16: np.ndarray, ref_bf16: np.ndarray, rtol=OUT_RTOL):
+    """Rule 3 against the oracle alone; returns the worst error as a fraction of the tolerance."""
+    ratio = output_errors(got_bf16, ref_bf16, rtol)
+    bad = ratio > 1.0
     assert not bad.any(), (f"{int(bad.sum())} outputs out of tolerance; worst "
-                           f"{float((err / np.maximum(tol, 1e-30)).max()):.3f}x tol")
-    return float((err / np.maximum(np.maximum(np.abs(r), rms), 1e-30)).max())
+                           f"{float(ratio.max()):.3f}x tol")
+    return float(ratio.max(initial=0.0))
 
 
-def check_output_explained(got_bf16, ref_bf16, alt_bf16, flipped_tokens, rtol=OUT_RTOL):
+def check_output_explained(got_bf16, ref_bf16, alt_bf16, flipped_tokens, rtol=OUT_RTOL,
+                           max_explained=None):
     """Rule 3 with rule 2's allowance (module docstring).  alt_bf16: the oracle's output on the
-    GPU's requantized codes; flipped_tokens: bool [T], tokens with a differing code."""
+    GPU's requantized codes; flipped_tokens: bool [T], tokens with a differing code;
+    max_explained: the most outputs the allowance may excuse (None: no cap)."""
     g = bf16_to_f32(got_bf16).astype(np.float64)
     out = []
     for ref in (ref_bf16, alt_bf16):
@@ -65,4 +75,7 @@ def check_output_explained(got_bf16, ref_bf16, alt_bf16, flipped_tokens, rtol=OU
     ok_ref, ok_alt = out
     ok = ok_ref | (ok_alt & np.asarray(flipped_tokens, bool)[:, None])
     assert ok.all(), f"{int((~ok).sum())} outputs out of tolerance (not explained by permitted code flips)"
-    return int((~ok_ref).sum())
+    n = int((~ok_ref).sum())
+    assert max_explained is None or n <= max_explained, \
+        f"{n} outputs need the code-flip allowance (cap {max_explained})"
+    return n

@@ -408,6 +408,91 @@ def test_layer_single_expert_vs_fp64_mlp():
     assert r["gates"].min() == 1.0
 
 
+def _shared_layer(H, Ns, sh_gate, sh_up, sh_down, E=2):
+    """A layer whose routed experts are all zero (scale 0, codes 0: routed output exactly 0), so
+    that out_f32 is the shared experts' sum alone."""
+    z = lambda rows, K: np.zeros((E, rows, K), np.int32)
+    zs = lambda rows, K: np.zeros((E, rows, K // 128), np.uint16)
+    return oracle.Layer(E, H, 128, z(128, H // 8), z(128, H // 8), z(H, 128 // 8), zs(128, H),
+                        zs(128, H), zs(H, 128), sh_gate=sh_gate, sh_up=sh_up, sh_down=sh_down)
+
+
+def test_shared_experts_constant_closed_form():
+    """Two shared experts with constant weights (tests/golden/shared_constant.txt): the output is
+    2 * 1.75 * silu(0.875) - 0.875 * silu(1.75), rounded once to bf16."""
+    (want_f32, want_bf16), = [tuple(map(float, l.split())) for l in golden_lines("shared_constant.txt")]
+    H, Ns, T = 128, 256, 2
+    c = lambda v, shape: np.full(shape, _f32_to_bf16_bits(np.float32(v)), np.uint16)
+    sg = np.stack([c(2.0 ** -7, (Ns, H)), c(2.0 ** -6, (Ns, H))])
+    su = np.stack([c(2.0 ** -6, (Ns, H)), c(-(2.0 ** -7), (Ns, H))])
+    sd = np.stack([c(2.0 ** -7, (H, Ns)), c(2.0 ** -8, (H, Ns))])
+    layer = _shared_layer(H, Ns, sg, su, sd)
+    x = _f32_to_bf16_bits(np.full((T, H), 0.875, np.float32))
+    r = oracle.moe_forward(layer, x, np.array([[1, 0], [0, 1]], np.float32), 1)
+    silu = lambda v: v / (1.0 + math.exp(-v))
+    closed = 2 * 1.75 * silu(0.875) - 0.875 * silu(1.75)
+    assert abs(closed - want_f32) < 1e-6
+    # fp32 sums of exact terms, two expf calls and a handful of roundings: a few ulp of 2.2
+    np.testing.assert_allclose(r["out_f32"], closed, rtol=0, atol=4e-6)
+    assert np.all(oracle.bf16_to_f32(r["out"]) == want_bf16)
+
+
+def test_shared_experts_vs_fp64_swiglu():
+    """Two random bf16 shared experts (H != Ns, so a transposed down weight reads other values)
+    against a textbook fp64 SwiGLU MLP per shared expert, summed.  The oracle's fp32 result lies
+    within the sequential-fp32 error bound of the fp64 value; swapped gate/up, a missing silu or a
+    transposed down projection fall far outside it."""
+    rng = np.random.default_rng(19)
+    H, Ns, S, T = 256, 384, 2, 7
+    def w(shape):
+        return _f32_to_bf16_bits((rng.standard_normal(shape) * 0.05).astype(np.float32))
+    sg, su, sd = w((S, Ns, H)), w((S, Ns, H)), w((S, H, Ns))
+    x = _f32_to_bf16_bits(rng.standard_normal((T, H)).astype(np.float32))
+    layer = _shared_layer(H, Ns, sg, su, sd)
+    r = oracle.moe_forward(layer, x, rng.standard_normal((T, 2)).astype(np.float32), 1)
+    got = r["out_f32"].astype(np.float64)
+    xf = oracle.bf16_to_f32(x).astype(np.float64)
+    Wg, Wu, Wd = (oracle.bf16_to_f32(a).astype(np.float64) for a in (sg, su, sd))
+    eps = 2.0 ** -24
+
+    def seq_dot(a, b):
+        """fp64 value of sum_i a[..., i] * b[..., i] and the error bound of evaluating it in fp32
+        in increasing i: every product and every partial sum s_i rounds once, so the error is at
+        most eps * (sum |p_i| + sum_{i>=2} |s_i|) (partial sums taken in fp64, 1 % margin)."""
+        prod = a[..., None, :] * b[None, ...]
+        part = np.cumsum(prod, axis=-1)
+        bnd = eps * (np.abs(prod).sum(-1) + np.abs(part[..., 1:]).sum(-1)) * 1.01
+        return part[..., -1], bnd
+
+    def mlp(gate_first=True, with_silu=True, down_T=False):
+        y = np.zeros((T, H))
+        bound = np.zeros((T, H))
+        for s in range(S):
+            (g, dg), (u, du) = seq_dot(xf, Wg[s]), seq_dot(xf, Wu[s])
+            if not gate_first:
+                g, u, dg, du = u, g, du, dg
+            sig = 1.0 / (1.0 + np.exp(-g))
+            a = (g * sig if with_silu else g) * u
+            # g and u errors carried through silu(g) * u (|d silu / dg| < 1.1), plus expf's ulps
+            # and the four roundings of g / (1 + e) * u on a itself
+            da = 1.1 * dg * np.abs(u) + np.abs(g * sig) * du + 8 * eps * np.abs(a)
+            D = Wd[s].reshape(Ns, H).T if down_T else Wd[s]
+            ys, dy = seq_dot(a, D)
+            y += ys
+            bound += da @ np.abs(D).T + dy
+        return y, bound + 4 * eps * np.abs(y)          # the two shared outputs summed, then added
+
+    ref, bound = mlp()
+    assert np.all(np.abs(got - ref) <= bound)
+    rms = np.sqrt((ref ** 2).mean())
+    assert bound.max() < 1e-3 * rms                     # the bound is tight enough to mean something
+    for wrong in (dict(gate_first=False), dict(with_silu=False), dict(down_T=True)):
+        alt, _ = mlp(**wrong)
+        assert np.abs(alt - ref).max() > 100 * bound.max(), wrong
+    # and the bf16 output is the single rounding of that fp32 sum
+    assert np.array_equal(r["out"], _f32_to_bf16_bits(r["out_f32"]))
+
+
 def test_layer_empty_batch():
     wl = synth.WORKLOADS["tiny"]
     layer = _tiny_layer(wl)

@@ -1,12 +1,15 @@
 """GPU parity: every entry point of libmoe_w4a8 (called through the C ABI) against the CPU
 oracle on the same seeded inputs, under the layer's three rules (tests/parity.py)."""
+import json
+import os
+
 import numpy as np
 import pytest
 
 import oracle
 import synth
 from conftest import cuda_ok
-from parity import bf16_to_f32, check_fp8_codes, check_output, check_output_explained
+from parity import bf16_to_f32, check_fp8_codes, check_output_explained, output_errors
 
 pytestmark = pytest.mark.gpu
 
@@ -197,21 +200,37 @@ def _host_layer_and_dev(E, H, N, seed, n_shared=0, shared_N=0):
     return hl, dl
 
 
-def _check_output_rules(hl, x, logits, k, got_out, ref, gpu_hq_pairs, gpu_sh_pairs):
-    """Rule 3, with rule 2's allowance for outputs of tokens whose requantized codes differ
-    (tests/parity.py): returns the number of outputs that needed the allowance."""
-    try:
-        check_output(got_out, ref["out"])
+def _report(**kv):
+    """One JSON line per parity check (the test, worst output error as a fraction of rule 3's
+    tolerance, FP8 code differences) appended to $MOE_PARITY_REPORT when it is set."""
+    path = os.environ.get("MOE_PARITY_REPORT")
+    if path:
+        kv["test"] = os.environ.get("PYTEST_CURRENT_TEST", "").split(" ")[0]
+        with open(path, "a") as f:
+            f.write(json.dumps(kv) + "\n")
+
+
+def _check_output_rules(hl, x, logits, k, got_out, ref, gpu_hq_pairs, gpu_sh_pairs, allow=None):
+    """Rule 3 against the oracle alone.  `allow` = (format and seeded case, cap): only a test
+    that names the case needing it gets rule 2's allowance for outputs of tokens whose
+    requantized codes differ (tests/parity.py), and for at most `cap` outputs.  Returns the
+    number of outputs that needed the allowance."""
+    ratio = output_errors(got_out, ref["out"])
+    worst = float(ratio.max(initial=0.0))
+    n_bad = int((ratio > 1.0).sum())
+    _report(worst_out_err_over_tol=round(worst, 4), outputs=int(ratio.size), out_of_tol=n_bad,
+            allowance=None if allow is None else allow[0])
+    if n_bad == 0:
         return 0
-    except AssertionError:
-        T = x.shape[0]
-        ref_pairs = ref["hq"][ref["row_of_pair"]]
-        flipped = (gpu_hq_pairs != ref_pairs).reshape(T, -1).any(axis=1)
-        alt, _ = oracle.moe_forward_given_h(hl, x, logits, k, gpu_hq_pairs, gpu_sh_pairs)
-        return check_output_explained(got_out, ref["out"], alt, flipped)
+    assert allow is not None, f"{n_bad} outputs out of tolerance; worst {worst:.3f}x tol"
+    T = x.shape[0]
+    ref_pairs = ref["hq"][ref["row_of_pair"]]
+    flipped = (gpu_hq_pairs != ref_pairs).reshape(T, -1).any(axis=1)
+    alt, _ = oracle.moe_forward_given_h(hl, x, logits, k, gpu_hq_pairs, gpu_sh_pairs)
+    return check_output_explained(got_out, ref["out"], alt, flipped, max_explained=allow[1])
 
 
-def _run_and_compare(hl, dl, x, logits, k, check_all=True):
+def _run_and_compare(hl, dl, x, logits, k, allow=None):
     T = x.shape[0]
     ref = oracle.moe_forward(hl, x, logits, k)
     xd, ld = to_dev_bf16(x), torch.from_numpy(logits).cuda()
@@ -227,9 +246,10 @@ def _run_and_compare(hl, dl, x, logits, k, check_all=True):
     assert np.array_equal(v["xq"], ref["xq"])
     assert np.array_equal(v["s_x"], ref["s_x"])
     n_diff, frac = check_fp8_codes(v["hq"], ref["hq"])
+    _report(hq_codes=int(v["hq"].size), hq_diff=n_diff)
     np.testing.assert_allclose(v["s_h"], ref["s_h"], rtol=2e-5)
     n_explained = _check_output_rules(hl, x, logits, k, bits(out), ref, v["hq"][v["row_of_pair"]],
-                                      v["s_h"][v["row_of_pair"]])
+                                      v["s_h"][v["row_of_pair"]], allow)
     return dict(hq_diff=n_diff, hq_frac=frac, explained=n_explained, out=bits(out))
 
 
@@ -250,6 +270,43 @@ def test_forward_ragged_shapes(E, H, N, k, T):
     hl, dl = _host_layer_and_dev(E, H, N, seed=E * 7 + T)
     x = synth.normal_bf16(3, 777 + T, T * H).reshape(T, H)
     logits = synth.normal_f32(3, 778 + T, T * E).reshape(T, E)
+    _run_and_compare(hl, dl, x, logits, k)
+
+
+def _random_nibble_layer(E, H, N, seed):
+    """Packed words of uniformly random nibbles (so code -8, nibble 0, is as common as any other
+    code: pack-quantized storage allows it although RTN never writes it) and random bf16 group
+    scales, built directly as words and given unchanged to the oracle and the GPU.  A few rows
+    are set to all -8, all +7 and alternating -8 / +7 codes."""
+    rng = np.random.default_rng(seed)
+    def words(rows, K):
+        w = rng.integers(0, 2 ** 32, size=(E, rows, K // 8), dtype=np.uint64).astype(np.uint32)
+        w[:, 0, :] = 0x00000000                        # every code -8
+        w[:, 1, : K // 16] = 0xFFFFFFFF                # +7 in the first half of the row
+        w[:, 2, :] = 0xF0F0F0F0                        # -8, +7, -8, +7, ...
+        return w.view(np.int32)
+    def scales(rows, K):
+        return _f32_to_bf16_bits(rng.uniform(0.003, 0.012, size=(E, rows, K // 128)))
+    gp, up, dp = words(N, H), words(N, H), words(H, N)
+    gs, us, ds = scales(N, H), scales(N, H), scales(H, N)
+    hl = oracle.Layer(E, H, N, gp, up, dp, gs, us, ds)
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    dl = moe.Layer(E, H, N, dev(gp), dev(up), dev(dp), dev(gs.view(np.int16)).view(torch.bfloat16),
+                   dev(us.view(np.int16)).view(torch.bfloat16), dev(ds.view(np.int16)).view(torch.bfloat16))
+    return hl, dl
+
+
+# token tiles of 16 and 32 rows (decode: unsigned widening of gate/up, gathered rows) and of 128
+# and 192 rows (prefill: signed widening), each on packed words in which nibble 0 (code -8) is
+# as frequent as every other nibble
+@pytest.mark.parametrize("E,H,N,k,T", [(64, 512, 256, 6, 8), (64, 512, 256, 6, 64), (16, 512, 256, 6, 40),
+                                       (4, 512, 256, 2, 100), (2, 512, 256, 1, 400)])
+def test_forward_code_minus8(E, H, N, k, T):
+    hl, dl = _random_nibble_layer(E, H, N, seed=E + T)
+    assert (oracle.unpack(hl.gate_packed[0], H) == -8).mean() > 0.05
+    x = synth.normal_bf16(12, 700 + T, T * H).reshape(T, H)
+    logits = synth.normal_f32(12, 701 + T, T * E).reshape(T, E)
+    logits[:, :3] += 4.0                               # the all -8 / +7 rows' experts are routed
     _run_and_compare(hl, dl, x, logits, k)
 
 
@@ -409,73 +466,152 @@ def test_router_logits_zero_tokens():
                           torch.empty(0, 8, dtype=torch.float32, device="cuda"))
 
 
-# ---- the layer at full size: sampled tokens -----------------------------------------------------
+# ---- the layer at full size: every token at decode, hundreds at prefill ----------------------------
 
 FULL = ["decode_t8", "decode_t64", "prefill_t2048_zipf", "prefill_t16384_shared"]
+FULL_WL = "prefill_t16384_shared"          # the full-size configs share its routed-expert weights
+
+
+def _boundary_tokens(v, T, k, n_min, tile_rows, rng):
+    """Tokens of a batch whose routed rows sit where token tiles start and end: the first and
+    last rows of the six longest expert segments and the rows on both sides of each tile
+    boundary inside them, the first and last rows of the last (partly filled) tile of 48 other
+    segments, every token routed to a one-row segment; then random tokens up to n_min."""
+    off, sp = v["offsets"], v["sorted_pairs"]
+    lens = np.diff(off)
+    rows = set()
+    for e in np.argsort(-lens, kind="stable")[:6]:
+        r0, r1 = int(off[e]), int(off[e + 1])
+        if r1 > r0:
+            rows |= {r0, r1 - 1}
+            for bn in tile_rows:
+                for b in range(r0 + bn, r1, bn):
+                    rows |= {b - 1, b}
+    live = np.flatnonzero(lens > 0)
+    for e in rng.permutation(live)[:48]:
+        r0, r1 = int(off[e]), int(off[e + 1])
+        rows.add(r1 - 1)
+        for bn in tile_rows:
+            rows.add(r0 + (r1 - r0 - 1) // bn * bn)
+    for e in np.flatnonzero(lens == 1):
+        rows.add(int(off[e]))
+    toks = {int(sp[r]) // k for r in rows}
+    while len(toks) < min(n_min, T):
+        toks.add(int(rng.integers(0, T)))
+    return sorted(toks)
+
+
+class _HostLayers:
+    """The oracle's copies of the full-size weights, packed expert by expert as tests need them
+    (one per format; the routed weights of every full-size config are the same draws)."""
+
+    def __init__(self):
+        self.layers, self.done = {}, {}
+
+    def get(self, fmt, experts, wl):
+        build = {"w4a8": oracle.pack_workload_layer, "w8a8": oracle.quant_workload_layer_w8a8,
+                 "nvfp4": oracle.quant_workload_layer_nvfp4}[fmt]
+        full = synth.WORKLOADS[FULL_WL]
+        if fmt not in self.layers:
+            self.layers[fmt] = build(full, experts=[])
+            self.done[fmt] = set()
+        todo = sorted(set(experts) - self.done[fmt])
+        if todo:
+            build(full, experts=todo, into=self.layers[fmt])
+            self.done[fmt] |= set(todo)
+        L = self.layers[fmt]
+        if not wl.n_shared:                            # the same routed weights, no shared experts
+            import copy
+            L = copy.copy(L)
+            L.sh_gate = L.sh_up = L.sh_down = None
+            L.n_shared = L.shared_N = 0
+        return L
+
+
+@pytest.fixture(scope="module")
+def host_layers():
+    return _HostLayers()
+
+
+def _full_size_check(name, dl, fmt, host_layers, n_batches=1, n_prefill_tokens=256, tile_rows=(128, 192)):
+    """The layer at full size on the GPU; every token of `n_batches` batches at decode (T <= 64),
+    at prefill at least `n_prefill_tokens` tokens chosen at token-tile boundaries, compared with
+    the oracle on those tokens (tokens are independent, so the oracle's sub-batch gives the same
+    rows) under the three rules; routing properties on the whole batch."""
+    wl = synth.WORKLOADS[name]
+    rng = np.random.default_rng(wl.T)
+    picks = []                                         # (first token of the batch, tokens, views, out)
+    for b in range(n_batches):
+        t0 = b * wl.T
+        x, lg = device_inputs(wl, t0=t0, T=wl.T)
+        ws = moe.alloc_workspace(dl, wl.T, wl.k)
+        out = moe.forward(dl, x, lg, wl.k, ws=ws)
+        torch.cuda.synchronize()
+        assert moe.moe_last_device_status() == 0
+        v = ws_views(dl, ws, wl.T, wl.k)
+        P = wl.P
+        off = v["offsets"]
+        assert off[0] == 0 and off[-1] == P and np.all(np.diff(off) >= 0)
+        assert np.array_equal(np.sort(v["sorted_pairs"]), np.arange(P))
+        assert np.array_equal(v["row_of_pair"][v["sorted_pairs"]], np.arange(P))
+        seg = np.repeat(np.arange(wl.E), np.diff(off))
+        assert np.array_equal(v["ids"].reshape(-1)[v["sorted_pairs"]], seg)
+        for e in range(wl.E):
+            s_ = v["sorted_pairs"][off[e]:off[e + 1]]
+            assert np.all(np.diff(s_) > 0)
+        outb = bits(out)
+        assert np.isfinite(bf16_to_f32(outb)).all()
+        toks = (list(range(wl.T)) if wl.T <= 64 else
+                _boundary_tokens(v, wl.T, wl.k, n_prefill_tokens, tile_rows, rng))
+        picks.append((t0, toks, v, outb))
+        del ws, out
+    xs = np.concatenate([synth.tokens(wl, t0 + t, 1) for t0, toks, _, _ in picks for t in toks])
+    ls = np.concatenate([synth.logits(wl, t0 + t, 1) for t0, toks, _, _ in picks for t in toks])
+    ids = np.concatenate([v["ids"][toks] for _, toks, v, _ in picks])
+    hl = host_layers.get(fmt, sorted(set(ids.reshape(-1).tolist())), wl)
+    ref = oracle.moe_forward(hl, xs, ls, wl.k)
+    assert np.array_equal(ids, ref["ids"])
+    np.testing.assert_allclose(np.concatenate([v["gates"][toks] for _, toks, v, _ in picks]), ref["gates"],
+                               rtol=1e-6)
+    assert np.array_equal(np.concatenate([v["xq"][toks] for _, toks, v, _ in picks]), ref["xq"])
+    assert np.array_equal(np.concatenate([v["s_x"][toks] for _, toks, v, _ in picks]), ref["s_x"])
+    rows = [v["row_of_pair"].reshape(wl.T, wl.k)[toks].reshape(-1) for _, toks, v, _ in picks]
+    hq = np.concatenate([v["hq"][r] for (_, _, v, _), r in zip(picks, rows)])
+    s_h = np.concatenate([v["s_h"][r] for (_, _, v, _), r in zip(picks, rows)])
+    n_diff, _ = check_fp8_codes(hq, ref["hq"][ref["row_of_pair"]])
+    _report(hq_codes=int(hq.size), hq_diff=n_diff, tokens=int(xs.shape[0]))
+    np.testing.assert_allclose(s_h, ref["s_h"][ref["row_of_pair"]], rtol=2e-5)
+    outb = np.concatenate([o[toks] for _, toks, _, o in picks])
+    _check_output_rules(hl, xs, ls, wl.k, outb, ref, hq, s_h)
+    return int(hq.size)
 
 
 @pytest.fixture(scope="module")
 def full_layer():
-    wl = synth.WORKLOADS["prefill_t16384_shared"]     # same weights for all full-size configs
-    return device_layer(wl)
+    return device_layer(synth.WORKLOADS[FULL_WL])     # same weights for all full-size configs
 
 
-def _sample_tokens(wl, n=4):
-    rng = np.random.default_rng(wl.T)
-    picks = {0, wl.T - 1}
-    while len(picks) < min(n, wl.T):
-        picks.add(int(rng.integers(0, wl.T)))
-    return sorted(picks)
+def _no_shared(dl):
+    cls = type(dl)
+    if cls is moe.Layer:
+        return moe.Layer(dl.E, dl.H, dl.N, dl.gate_packed, dl.up_packed, dl.down_packed,
+                         dl.gate_scales, dl.up_scales, dl.down_scales)
+    if cls is moe.Layer8:
+        return moe.Layer8(dl.E, dl.H, dl.N, dl.gate_w8, dl.up_w8, dl.down_w8, dl.gate_rs, dl.up_rs,
+                          dl.down_rs)
+    return moe.Layer4(dl.E, dl.H, dl.N, dl.gate_f4, dl.up_f4, dl.down_f4, dl.gate_bs, dl.up_bs, dl.down_bs,
+                      dl.gate_s2, dl.up_s2, dl.down_s2)
 
 
 @pytest.mark.parametrize("name", FULL)
-def test_forward_full_size_sampled(name, full_layer):
+def test_forward_full_size(name, full_layer, host_layers):
+    """W4A8 at full size: decode_t8 over all eight benchmark batches (64 tokens), decode_t64 all
+    64 tokens, the prefill configs at >= 256 tokens at tile boundaries; >= 0.5 M requantized codes
+    each under rule 2."""
     wl = synth.WORKLOADS[name]
-    dl = full_layer
-    if not wl.n_shared:
-        dl = moe.Layer(dl.E, dl.H, dl.N, dl.gate_packed, dl.up_packed, dl.down_packed,
-                       dl.gate_scales, dl.up_scales, dl.down_scales)
-    x, lg = device_inputs(wl)
-    ws = moe.alloc_workspace(dl, wl.T, wl.k)
-    out = moe.forward(dl, x, lg, wl.k, ws=ws)
-    torch.cuda.synchronize()
-    assert moe.moe_last_device_status() == 0
-    v = ws_views(dl, ws, wl.T, wl.k)
-    P = wl.P
-    # properties at full size
-    off = v["offsets"]
-    assert off[0] == 0 and off[-1] == P and np.all(np.diff(off) >= 0)
-    assert np.array_equal(np.sort(v["sorted_pairs"]), np.arange(P))
-    assert np.array_equal(v["row_of_pair"][v["sorted_pairs"]], np.arange(P))
-    seg = np.repeat(np.arange(wl.E), np.diff(off))
-    assert np.array_equal(v["ids"].reshape(-1)[v["sorted_pairs"]], seg)
-    for e in range(wl.E):
-        s = v["sorted_pairs"][off[e]:off[e + 1]]
-        assert np.all(np.diff(s) > 0)
-    outb = bits(out)
-    assert np.isfinite(bf16_to_f32(outb)).all()
-
-    # the oracle on sampled tokens (tokens are independent, so a sub-batch gives the same rows)
-    toks = _sample_tokens(wl)
-    xs = np.stack([synth.tokens(wl, t, 1)[0] for t in toks])
-    ls = np.stack([synth.logits(wl, t, 1)[0] for t in toks])
-    ids_ref, _ = oracle.route_topk(ls, wl.k)
-    experts = sorted(set(ids_ref.reshape(-1).tolist()))
-    hl = oracle.pack_workload_layer(wl, experts=experts)
-    # S0 parity on the experts the sample touches
-    for e in experts[:3]:
-        assert np.array_equal(dl.gate_packed[e].cpu().numpy(), hl.gate_packed[e])
-        assert np.array_equal(bits(dl.down_scales[e]), hl.down_scales[e])
-    ref = oracle.moe_forward(hl, xs, ls, wl.k)
-    assert np.array_equal(v["ids"][toks], ref["ids"])
-    np.testing.assert_allclose(v["gates"][toks], ref["gates"], rtol=1e-6)
-    gpu_rows = v["row_of_pair"].reshape(wl.T, wl.k)[toks].reshape(-1)
-    ref_rows = ref["row_of_pair"]
-    assert np.array_equal(v["xq"][toks], ref["xq"])
-    assert np.array_equal(v["s_x"][toks], ref["s_x"])
-    check_fp8_codes(v["hq"][gpu_rows], ref["hq"][ref_rows])
-    np.testing.assert_allclose(v["s_h"][gpu_rows], ref["s_h"][ref_rows], rtol=2e-5)
-    _check_output_rules(hl, xs, ls, wl.k, outb[toks], ref, v["hq"][gpu_rows], v["s_h"][gpu_rows])
+    dl = full_layer if wl.n_shared else _no_shared(full_layer)
+    n = _full_size_check(name, dl, "w4a8", host_layers, n_batches=8 if name == "decode_t8" else 1)
+    assert n >= 500_000
 
 
 # ---- failure detection: a bounded device wait that runs out -------------------------------------
@@ -579,40 +715,16 @@ def test_w8a8_forward_shared_experts_and_zero_rows():
 
 @pytest.fixture(scope="module")
 def full_layer_w8a8():
-    return device_layer_w8a8(synth.WORKLOADS["prefill_t16384_shared"])
+    return device_layer_w8a8(synth.WORKLOADS[FULL_WL])
 
 
 @pytest.mark.parametrize("name", FULL)
-def test_w8a8_forward_full_size_sampled(name, full_layer_w8a8):
+def test_w8a8_forward_full_size(name, full_layer_w8a8, host_layers):
+    """Row-scaled FP8 experts at full size: every token of one batch at decode, >= 64 tokens at
+    tile boundaries (128/192/256 rows) at prefill."""
     wl = synth.WORKLOADS[name]
-    dl = full_layer_w8a8
-    if not wl.n_shared:
-        dl = moe.Layer8(dl.E, dl.H, dl.N, dl.gate_w8, dl.up_w8, dl.down_w8, dl.gate_rs, dl.up_rs,
-                        dl.down_rs)
-    x, lg = device_inputs(wl)
-    ws = moe.alloc_workspace(dl, wl.T, wl.k)
-    out = moe.forward(dl, x, lg, wl.k, ws=ws)
-    torch.cuda.synchronize()
-    assert moe.moe_last_device_status() == 0
-    v = ws_views(dl, ws, wl.T, wl.k)
-    outb = bits(out)
-    assert np.isfinite(bf16_to_f32(outb)).all()
-    toks = _sample_tokens(wl)
-    xs = np.stack([synth.tokens(wl, t, 1)[0] for t in toks])
-    ls = np.stack([synth.logits(wl, t, 1)[0] for t in toks])
-    ids_ref, _ = oracle.route_topk(ls, wl.k)
-    experts = sorted(set(ids_ref.reshape(-1).tolist()))
-    hl = oracle.quant_workload_layer_w8a8(wl, experts=experts)
-    for e in experts[:3]:
-        assert np.array_equal(dl.gate_w8[e].cpu().numpy(), hl.gate_w8[e])
-        assert np.array_equal(dl.down_rs[e].cpu().numpy(), hl.down_rs[e])
-    ref = oracle.moe_forward(hl, xs, ls, wl.k)
-    assert np.array_equal(v["ids"][toks], ref["ids"])
-    gpu_rows = v["row_of_pair"].reshape(wl.T, wl.k)[toks].reshape(-1)
-    assert np.array_equal(v["xq"][toks], ref["xq"])
-    check_fp8_codes(v["hq"][gpu_rows], ref["hq"][ref["row_of_pair"]])
-    np.testing.assert_allclose(v["s_h"][gpu_rows], ref["s_h"][ref["row_of_pair"]], rtol=2e-5)
-    _check_output_rules(hl, xs, ls, wl.k, outb[toks], ref, v["hq"][gpu_rows], v["s_h"][gpu_rows])
+    dl = full_layer_w8a8 if wl.n_shared else _no_shared(full_layer_w8a8)
+    _full_size_check(name, dl, "w8a8", host_layers, n_prefill_tokens=64, tile_rows=(128, 256))
 
 
 # ---- NVFP4 experts -------------------------------------------------------------------------------
@@ -698,40 +810,16 @@ def test_nvfp4_forward_shared_experts():
 
 @pytest.fixture(scope="module")
 def full_layer_nvfp4():
-    return device_layer_nvfp4(synth.WORKLOADS["prefill_t16384_shared"])
+    return device_layer_nvfp4(synth.WORKLOADS[FULL_WL])
 
 
 @pytest.mark.parametrize("name", FULL)
-def test_nvfp4_forward_full_size_sampled(name, full_layer_nvfp4):
+def test_nvfp4_forward_full_size(name, full_layer_nvfp4, host_layers):
+    """NVFP4 experts at full size: every token of one batch at decode, >= 64 tokens at tile
+    boundaries at prefill."""
     wl = synth.WORKLOADS[name]
-    dl = full_layer_nvfp4
-    if not wl.n_shared:
-        dl = moe.Layer4(dl.E, dl.H, dl.N, dl.gate_f4, dl.up_f4, dl.down_f4, dl.gate_bs, dl.up_bs, dl.down_bs,
-                        dl.gate_s2, dl.up_s2, dl.down_s2)
-    x, lg = device_inputs(wl)
-    ws = moe.alloc_workspace(dl, wl.T, wl.k)
-    out = moe.forward(dl, x, lg, wl.k, ws=ws)
-    torch.cuda.synchronize()
-    assert moe.moe_last_device_status() == 0
-    v = ws_views(dl, ws, wl.T, wl.k)
-    outb = bits(out)
-    assert np.isfinite(bf16_to_f32(outb)).all()
-    toks = _sample_tokens(wl)
-    xs = np.stack([synth.tokens(wl, t, 1)[0] for t in toks])
-    ls = np.stack([synth.logits(wl, t, 1)[0] for t in toks])
-    ids_ref, _ = oracle.route_topk(ls, wl.k)
-    experts = sorted(set(ids_ref.reshape(-1).tolist()))
-    hl = oracle.quant_workload_layer_nvfp4(wl, experts=experts)
-    for e in experts[:3]:
-        assert np.array_equal(dl.gate_f4[e].cpu().numpy(), hl.gate_f4[e])
-        assert np.array_equal(dl.down_bs[e].cpu().numpy(), hl.down_bs[e])
-    ref = oracle.moe_forward(hl, xs, ls, wl.k)
-    assert np.array_equal(v["ids"][toks], ref["ids"])
-    gpu_rows = v["row_of_pair"].reshape(wl.T, wl.k)[toks].reshape(-1)
-    assert np.array_equal(v["xq"][toks], ref["xq"])
-    check_fp8_codes(v["hq"][gpu_rows], ref["hq"][ref["row_of_pair"]])
-    np.testing.assert_allclose(v["s_h"][gpu_rows], ref["s_h"][ref["row_of_pair"]], rtol=2e-5)
-    _check_output_rules(hl, xs, ls, wl.k, outb[toks], ref, v["hq"][gpu_rows], v["s_h"][gpu_rows])
+    dl = full_layer_nvfp4 if wl.n_shared else _no_shared(full_layer_nvfp4)
+    _full_size_check(name, dl, "nvfp4", host_layers, n_prefill_tokens=64, tile_rows=(128, 256))
 
 
 # ---- hybrid layers: NVFP4 hot experts, W4A8 cold experts -------------------------------------------
