@@ -168,7 +168,7 @@ inline WsPlan plan_workspace(const moe_w4a8_layer& L, int64_t T, int k, int fmt 
     p.act16 = fmt >= 2 ? take((size_t)P * (L.H > L.N ? L.H : L.N) * 2) : 0;
     p.slot_of = fmt == 3 ? take((size_t)L.E * 4) : 0;
     if (L.n_shared > 0) {
-        p.sh_a = take((size_t)T * L.n_shared * L.shared_N * 2);
+        p.sh_a = take((size_t)T * L.n_shared * L.shared_N * 2 * 2);   // bf16 hi | lo halves
         p.sh_y = take((size_t)T * L.H * 4);
     }
     p.total = off;
@@ -441,10 +441,11 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const ExpertSet& xw, const ui
         const int Wsh = L.n_shared * L.shared_N;
         uint16_t* sa = (uint16_t*)at(p.sh_a);
         shared = (float*)at(p.sh_y);
-        Bf16GemmArgs g{Wsh, (int)T, L.H, 0, sa, Wsh};
-        if ((st = launch_gemm_bf16_ws<true>(g, x_bf16, L.sh_gate, L.sh_up, L.n_shared, stream))) return st;
-        Bf16GemmArgs d{L.H, (int)T, Wsh, L.shared_N, shared, L.H};
-        if ((st = launch_gemm_bf16_ws<false>(d, sa, L.sh_down, nullptr, L.n_shared, stream))) return st;
+        // the SwiGLU activation as bf16 hi and lo halves [T, 2 Wsh]; the down GEMM reduces over both
+        Bf16GemmArgs g{Wsh, (int)T, L.H, 0, sa, 2 * Wsh, 0};
+        if ((st = launch_gemm_bf16_ws<true>(g, x_bf16, L.sh_gate, L.sh_up, stream))) return st;
+        Bf16GemmArgs d{L.H, (int)T, 2 * Wsh, L.shared_N, shared, L.H, Wsh};
+        if ((st = launch_gemm_bf16_ws<false>(d, sa, L.sh_down, nullptr, stream))) return st;
         sm.launches += 2;
     }
     sm.mark(3, stream);

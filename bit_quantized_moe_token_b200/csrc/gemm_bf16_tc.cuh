@@ -11,8 +11,11 @@
 // of two TMEM accumulators (2 x BN columns), and warps 0-3 drain a finished accumulator while
 // the tensor core fills the other.  Swap AB again: MMA M = 128 weight rows, N = BN tokens.
 //   SwiGLU instance: M tile = 64 gate rows + the same 64 up rows; the epilogue writes
-//     a = silu(gate . x) * (up . x), rounded to bf16 (the down GEMM's operand type).
-//   plain instance: Y[t, m] fp32.
+//     a = silu(gate . x) * (up . x) as two bf16 halves, hi = bf16(a) in columns [0, M) and
+//     lo = bf16(a - hi) in columns [M, 2M) (hi + lo carries a to ~2^-18 relative: the layer
+//     keeps this activation in fp32, and bf16 alone would move outputs by up to ~1 %).
+//   plain instance: Y[t, m] fp32; for the shared down projection its K runs over both halves
+//     (K = 2 Kw), and the weights of K index k are those of k mod Kw.
 #pragma once
 #include <cuda.h>
 #include "common.cuh"
@@ -24,10 +27,11 @@ namespace moe {
 struct Bf16GemmArgs {
     int M;       // output rows of one projection (SwiGLU: n_shared*Ns; plain: H)
     int T;       // tokens
-    int K;       // reduction length (SwiGLU: H; plain: n_shared*Ns)
+    int K;       // reduction length of the activations (SwiGLU: H; plain: 2 * n_shared*Ns)
     int Ks;      // plain: K extent per shared expert (Ns); the 3-D weight map's inner dim
-    void* out;   // SwiGLU: bf16 [T, ldo]; plain: fp32 [T, ldo]
+    void* out;   // SwiGLU: bf16 [T, ldo] (hi | lo halves, ldo >= 2M); plain: fp32 [T, ldo]
     int ldo;
+    int Kw;      // plain: K extent of the weights (n_shared*Ns); activation column k uses k mod Kw
 };
 
 namespace tc {
@@ -131,7 +135,7 @@ __global__ void __launch_bounds__(192, 1)
                         ws::tma_load_2d(st, &tm_w0, c * 64, mt * 64, &full[s]);
                         ws::tma_load_2d(st + 64 * 128, &tm_w1, c * 64, mt * 64, &full[s]);
                     } else {
-                        const int k0 = c * 64;
+                        const int k0 = (c * 64) % a.Kw;
                         ws::tma_load_3d(st, &tm_w0, k0 % a.Ks, mt * 128, k0 / a.Ks, &full[s]);
                     }
                 }
@@ -189,7 +193,9 @@ __global__ void __launch_bounds__(192, 1)
                             const int t = n0 + c0 + j;
                             if (t < a.T) {
                                 const float h = silu(__uint_as_float(v[j])) * sX[tid * C::kXStride + j];
-                                out[(int64_t)t * a.ldo + n] = f32_to_bf16_bits(h);
+                                const uint16_t hi = f32_to_bf16_bits(h);
+                                out[(int64_t)t * a.ldo + n] = hi;
+                                out[(int64_t)t * a.ldo + a.M + n] = f32_to_bf16_bits(h - bf16_bits_to_f32(hi));
                             }
                         }
                     }
@@ -222,36 +228,30 @@ __global__ void __launch_bounds__(192, 1)
 
 inline bool make_map_bf16_2d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows,
                              uint32_t box_cols, uint32_t box_rows) {
-    PFN_encodeTiled fn = encode_fn();
-    if (!fn) return false;
     const cuuint64_t dims[2] = {cols, rows};
     const cuuint64_t strides[1] = {cols * 2};
     const cuuint32_t box[2] = {box_cols, box_rows};
-    const cuuint32_t estr[2] = {1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return encode_tiled(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 // [d2, d1, d0] bf16 tensor (d0 innermost) with a box of 1 x box1 x box0.
 inline bool make_map_bf16_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
                              uint32_t box0, uint32_t box1) {
-    PFN_encodeTiled fn = encode_fn();
-    if (!fn) return false;
     const cuuint64_t dims[3] = {d0, d1, d2};
     const cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
     const cuuint32_t box[3] = {box0, box1, 1};
-    const cuuint32_t estr[3] = {1, 1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return encode_tiled(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 template <bool kSwiGLU>
 int launch_gemm_bf16_ws(const Bf16GemmArgs& a, const void* act, const void* w0, const void* w1,
-                        int n_shared, cudaStream_t stream) {
+                        cudaStream_t stream) {
     constexpr int BN = 256;
     using C = Bf16Cfg<BN>;
+    // plain instance: the weights' K extent Kw is a whole number of Ks-wide slices, and the
+    // activations' K a whole number of Kw (the shared down projection: two halves)
+    if (!kSwiGLU && (a.Ks <= 0 || a.Kw <= 0 || a.Kw % a.Ks || a.K % a.Kw || a.Kw % 64))
+        return MOE_ERR_INVALID_ARG;
     static int sms_cache[16] = {0};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
@@ -268,7 +268,7 @@ int launch_gemm_bf16_ws(const Bf16GemmArgs& a, const void* act, const void* w0, 
     if (kSwiGLU) {
         ok = make_map_bf16_2d(&m0, w0, a.K, a.M, 64, 64) && make_map_bf16_2d(&m1, w1, a.K, a.M, 64, 64);
     } else {
-        ok = make_map_bf16_3d(&m0, w0, a.Ks, a.M, n_shared, 64, 128);
+        ok = make_map_bf16_3d(&m0, w0, a.Ks, a.M, a.Kw / a.Ks, 64, 128);
         m1 = m0;
     }
     ok = ok && make_map_bf16_2d(&mact, act, a.K, a.T, 64, BN);

@@ -214,8 +214,8 @@ inline int launch_router_topk(const uint16_t* x, const uint16_t* wr, int64_t T, 
     const int epl = (E + 31) / 32;
     *launches = 0;
     if (router_uses_tensor_cores(T, H, E)) {
-        Bf16GemmArgs a{E, static_cast<int>(T), H, H, logits, E};
-        int st = launch_gemm_bf16_ws<false>(a, x, wr, nullptr, 1, stream);
+        Bf16GemmArgs a{E, static_cast<int>(T), H, H, logits, E, H};
+        int st = launch_gemm_bf16_ws<false>(a, x, wr, nullptr, stream);
         if (st != MOE_OK) return st;
         *launches = 2;
         return launch_topk(logits, T, E, k, ids, gates, stream);
@@ -260,8 +260,8 @@ extern "C" int moe_router_logits(const uint16_t* x_bf16, const uint16_t* wr_bf16
     if (!x_bf16 || !wr_bf16 || !logits) return MOE_ERR_INVALID_ARG;
     if (!aligned(x_bf16, 16) || !aligned(wr_bf16, 16) || !aligned(logits, 4)) return MOE_ERR_MISALIGNED;
     if (router_uses_tensor_cores(T, H, E)) {
-        Bf16GemmArgs a{E, static_cast<int>(T), H, H, logits, E};
-        return launch_gemm_bf16_ws<false>(a, x_bf16, wr_bf16, nullptr, 1, stream);
+        Bf16GemmArgs a{E, static_cast<int>(T), H, H, logits, E, H};
+        return launch_gemm_bf16_ws<false>(a, x_bf16, wr_bf16, nullptr, stream);
     }
     if (T <= 16) {
         k_router_rows<16><<<static_cast<unsigned>(E), 256, 0, stream>>>(
