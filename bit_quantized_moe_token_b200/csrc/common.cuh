@@ -24,6 +24,41 @@ inline int launch_status() {
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// ---- programmatic dependent launch ------------------------------------------------------------
+//
+// The layer's kernels follow one rule: a grid waits for the grid launched before it on the
+// stream (its completion and memory visibility, griddepcontrol.wait) before it touches any
+// buffer that grid writes or reads, and lets the next grid launch only after that wait.  A
+// grid that has started therefore knows that every grid two or more launches back has
+// completed, and a grid may read data written that far back (expert offsets, weights) before
+// its own wait.  The overlap gained: a grid's launch, prologue (barriers, TMEM allocation,
+// descriptor prefetch) and any such early reads run under its predecessor's tail.  Both
+// instructions are no-ops for a grid launched without the programmatic-serialization attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_enter() {
+    pdl_wait();
+    pdl_trigger();
+}
+
+// Launches `kern` on `stream` with programmatic stream serialization (the kernel must follow the
+// rule above).
+template <typename... KArgs, typename... Args>
+inline int launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                      Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
 // ---- conversions -------------------------------------------------------------------------------
 
 __device__ __forceinline__ float bf16_bits_to_f32(uint16_t h) {

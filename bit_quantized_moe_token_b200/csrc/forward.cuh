@@ -15,13 +15,18 @@ namespace moe {
 
 // S5 requantization of the SwiGLU activations h (fp32, one expert-sorted row per CTA, written
 // by the gate/up GEMM together with max|h| per row): s_h = max|h| / 448, Hq = e4m3(h / s_h).
+// With qsum non-null it also writes each row's per-128-column sums of the FP8 values (the down
+// GEMM's unsigned widening removes its +8 offset with them): a half-warp covers one group.
 __global__ void __launch_bounds__(256) k_requant(const float* __restrict__ h, int N,
                                                  const unsigned* __restrict__ amax,
-                                                 uint8_t* __restrict__ hq, float* __restrict__ s_h) {
+                                                 uint8_t* __restrict__ hq, float* __restrict__ s_h,
+                                                 float* __restrict__ qsum) {
+    pdl_enter();
     const int64_t r = blockIdx.x;
     const float s = __fdiv_rn(__uint_as_float(amax[r]), kFp8Max);
     const float4* src = reinterpret_cast<const float4*>(h + r * N);
-    for (int c = threadIdx.x; c < (N >> 3); c += blockDim.x) {
+    const int G = N / kGroup;
+    for (int c = threadIdx.x; c < (N >> 3); c += blockDim.x) {   // blockDim = 256: whole half-warps
         uint2 codes = make_uint2(0u, 0u);
         if (s != 0.0f) {
             const float4 a = src[2 * c], b = src[2 * c + 1];
@@ -31,6 +36,10 @@ __global__ void __launch_bounds__(256) k_requant(const float* __restrict__ h, in
                       (static_cast<uint32_t>(f32x2_to_e4m3x2(__fdiv_rn(b.z, s), __fdiv_rn(b.w, s))) << 16);
         }
         reinterpret_cast<uint2*>(hq + r * N)[c] = codes;
+        if (qsum) {
+            const float gs = halfwarp_sum(e4m3x8_sum(codes));
+            if ((threadIdx.x & 15) == 0) qsum[r * G + c / 16] = gs;
+        }
     }
     if (threadIdx.x == 0) s_h[r] = s;
 }
@@ -43,6 +52,7 @@ __global__ void __launch_bounds__(256) k_combine(const float* __restrict__ Y,
                                                  const int32_t* __restrict__ rop, int k, int H,
                                                  int64_t T, const float* __restrict__ shared,
                                                  uint16_t* __restrict__ out) {
+    pdl_enter();
     const int q = H >> 2;
     const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
     if (i >= T * q) return;
@@ -95,6 +105,7 @@ __global__ void __launch_bounds__(256) k_quant_topk(const float* __restrict__ lo
                                                     uint8_t* __restrict__ xq,
                                                     float* __restrict__ s_x,
                                                     float* __restrict__ qsum) {
+    pdl_enter();
     __shared__ float red[32];
     const int64_t t = blockIdx.x;
     if (kTopk && threadIdx.x < 32) topk_row<EPL>(logits + t * E, E, k, ids + t * k, gates + t * k, threadIdx.x);
@@ -106,19 +117,18 @@ inline int launch_quant_topk(const float* logits, const uint16_t* x, int64_t T, 
                              cudaStream_t stream, bool topk = true) {
     const int epl = (E + 31) / 32;
     const unsigned grid = static_cast<unsigned>(T);
-    if (!topk) {
-        k_quant_topk<1, false><<<grid, 256, 0, stream>>>(logits, x, E, k, H, ids, gates, xq, s_x, qsum);
-        return launch_status();
-    }
-#define MOE_QT(N) k_quant_topk<N><<<grid, 256, 0, stream>>>(logits, x, E, k, H, ids, gates, xq, s_x, qsum)
-    if (epl <= 1) MOE_QT(1);
-    else if (epl <= 2) MOE_QT(2);
-    else if (epl <= 4) MOE_QT(4);
-    else if (epl <= 8) MOE_QT(8);
-    else if (epl <= 16) MOE_QT(16);
-    else MOE_QT(32);
+    if (!topk)
+        return launch_pdl(k_quant_topk<1, false>, dim3(grid), dim3(256), 0, stream, logits, x, E, k, H, ids, gates,
+                          xq, s_x, qsum);
+#define MOE_QT(N) launch_pdl(k_quant_topk<N>, dim3(grid), dim3(256), 0, stream, logits, x, E, k, H, ids, gates, xq, \
+                             s_x, qsum)
+    if (epl <= 1) return MOE_QT(1);
+    if (epl <= 2) return MOE_QT(2);
+    if (epl <= 4) return MOE_QT(4);
+    if (epl <= 8) return MOE_QT(8);
+    if (epl <= 16) return MOE_QT(16);
+    return MOE_QT(32);
 #undef MOE_QT
-    return launch_status();
 }
 
 // ------------------------------------------------------------------------------------------
@@ -128,6 +138,7 @@ struct WsPlan {
     size_t topk_ids, topk_w, offsets, sorted, rop, route_ws;
     size_t xq, s_x, x_sorted, s_x_sorted, h, zero, hq, s_h, y;
     size_t qs_x;         // per (token, K-group) sums of the FP8 values (narrow W4A8 tiles)
+    size_t qs_h;         // per (sorted row, N-group) sums of the requantized values (W4A8 down GEMM)
     size_t logits, rcnt; // router logits [T, E] and the fused router's counters (router entry points)
     size_t act16;        // NVFP4 experts: f16 copies of the GEMM inputs (max of [T|P, H] and [P, N])
     size_t slot_of;      // hybrid layers: expert -> slab map [E]
@@ -163,6 +174,7 @@ inline WsPlan plan_workspace(const moe_w4a8_layer& L, int64_t T, int k, int fmt 
     p.s_h = take(P * 4);
     p.y = take((size_t)P * L.H * 4);
     p.qs_x = take((size_t)T * (L.H / 128) * 4);
+    p.qs_h = take((size_t)P * (L.N / 128) * 4);
     p.logits = take((size_t)T * L.E * 4);
     p.rcnt = take((size_t)router_counter_words(T) * 4);
     p.act16 = fmt >= 2 ? take((size_t)P * (L.H > L.N ? L.H : L.N) * 2) : 0;
@@ -237,6 +249,7 @@ struct ExpertSet {
 __global__ void __launch_bounds__(1024) k_slot_map(const int32_t* __restrict__ hot_ids, int n_hot,
                                                    const int32_t* __restrict__ cold_ids, int n_cold, int E,
                                                    int32_t* __restrict__ slot_of) {
+    pdl_enter();
     for (int e = threadIdx.x; e < E; e += blockDim.x) slot_of[e] = kSlotNone;
     __syncthreads();
     for (int i = threadIdx.x; i < n_hot + n_cold; i += blockDim.x) {
@@ -349,6 +362,7 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const ExpertSet& xw, const ui
     float* sh = (float*)at(p.s_h);
     float* y = (float*)at(p.y);
     float* qs_x = (float*)at(p.qs_x);
+    float* qs_h = (float*)at(p.qs_h);
     // narrow token tiles (decode): codes written once per token and gathered by the GEMM; wide
     // tiles (prefill): codes copied to expert-sorted rows.  Either way the requantization (S5)
     // and the combine (S7) run as their own passes: fused into the GEMM epilogues behind
@@ -372,8 +386,9 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const ExpertSet& xw, const ui
     const float* f4_u2 = hybrid ? xw.h_up_s2 : xw.up_s2;
     const float* f4_d2 = hybrid ? xw.h_down_s2 : xw.down_s2;
     if (hybrid) {
-        k_slot_map<<<1, 1024, 0, stream>>>(xw.hot_ids, xw.n_hot, xw.cold_ids, xw.n_cold, L.E, slot_of);
-        if ((st = launch_status())) return st;
+        if ((st = launch_pdl(k_slot_map, dim3(1), dim3(1024), 0, stream, xw.hot_ids, xw.n_hot, xw.cold_ids,
+                             xw.n_cold, L.E, slot_of)))
+            return st;
         sm.launches += 1;
     }
 
@@ -477,8 +492,11 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const ExpertSet& xw, const ui
     }
     sm.mark(4, stream);
     // S5
-    k_requant<<<static_cast<unsigned>(P), 256, 0, stream>>>(h, L.N, amax, hq, sh);
-    if ((st = launch_status())) return st;
+    // the W4A8 down GEMM widens its narrow tiles unsigned and needs the requantized rows' group sums
+    const bool down_sums = run_w4 && ws_narrow(ws_tile_rows(P, L.E));
+    if ((st = launch_pdl(k_requant, dim3(static_cast<unsigned>(P)), dim3(256), 0, stream, h, L.N, amax, hq, sh,
+                         down_sums ? qs_h : nullptr)))
+        return st;
     sm.launches += 1;
     sm.mark(5, stream);
     // S6
@@ -497,7 +515,7 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const ExpertSet& xw, const ui
         sm.launches += 1;
     } else if (run_w4) {
         WsGemmArgs a{sh, (const uint16_t*)xw.down_s, nullptr, offsets, L.E, L.H, L.N, (int)P, y, L.H,
-                     nullptr, sorted, k, (int)T, nullptr, slot_of, hybrid ? kSlotCold : kSlotAll};
+                     nullptr, sorted, k, (int)T, down_sums ? qs_h : nullptr, slot_of, hybrid ? kSlotCold : kSlotAll};
         if ((st = launch_gemm_ws<false>(a, hq, xw.down, nullptr, stream))) return st;
         sm.launches += 1;
     }
@@ -505,9 +523,9 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const ExpertSet& xw, const ui
     // S7
     {
         const int64_t n = T * (L.H / 4);
-        k_combine<<<static_cast<unsigned>((n + 255) / 256), 256, 0, stream>>>(y, gates, rop, k, L.H, T,
-                                                                            shared, out_bf16);
-        if ((st = launch_status())) return st;
+        if ((st = launch_pdl(k_combine, dim3(static_cast<unsigned>((n + 255) / 256)), dim3(256), 0, stream, y,
+                             gates, rop, k, L.H, T, shared, out_bf16)))
+            return st;
         sm.launches += 1;
     }
     sm.mark(7, stream);

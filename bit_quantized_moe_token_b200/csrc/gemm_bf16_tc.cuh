@@ -82,6 +82,7 @@ template <int BN, bool kSwiGLU>
 __global__ void __launch_bounds__(192, 1)
     k_gemm_bf16_ws(const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__ CUtensorMap tm_w1,
                    const __grid_constant__ CUtensorMap tm_act, const Bf16GemmArgs a) {
+    pdl_enter();
     using C = Bf16Cfg<BN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -276,8 +277,7 @@ int launch_gemm_bf16_ws(const Bf16GemmArgs& a, const void* act, const void* w0, 
     const int m_tiles = kSwiGLU ? a.M / 64 : a.M / 128;
     const int64_t tiles = (int64_t)m_tiles * ((a.T + BN - 1) / BN);
     const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(tiles, sms_cache[dev & 15]));
-    kern<<<static_cast<unsigned>(grid), 192, C::kAlloc, stream>>>(m0, m1, mact, a);
-    return launch_status();
+    return launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(192), C::kAlloc, stream, m0, m1, mact, a);
 }
 
 }  // namespace moe

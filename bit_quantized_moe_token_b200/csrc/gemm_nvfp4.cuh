@@ -111,6 +111,7 @@ template <int BN, bool kSwiGLU, bool kGather>
 __global__ void __launch_bounds__(F4Cfg<BN>::kThreads, F4Cfg<BN>::kCtasPerSm)
     k_gemm_nvfp4(const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__ CUtensorMap tm_w1,
                  const __grid_constant__ CUtensorMap tm_act, const F4GemmArgs f) {
+    pdl_enter();
     using C = F4Cfg<BN>;
     const W8GemmArgs& a = f.b;
     extern __shared__ uint8_t smem_raw[];
@@ -362,8 +363,8 @@ int launch_gemm_nvfp4_inst(const F4GemmArgs& f, const void* act_f16, const void*
     const int m_tiles = kSwiGLU ? a.R0 / 64 : a.R0 / 128;
     const int64_t grid = std::max<int64_t>(
         1, std::min<int64_t>(max_row_tiles * m_tiles, (int64_t)sms_cache[dev & 15] * C::kCtasPerSm));
-    kern<<<static_cast<unsigned>(grid), C::kThreads, C::kAlloc, stream>>>(m0, m1, mact, f);
-    return launch_status();
+    return launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(C::kThreads), C::kAlloc, stream, m0, m1, mact,
+                      f);
 }
 
 template <bool kSwiGLU>

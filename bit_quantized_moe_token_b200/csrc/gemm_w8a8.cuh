@@ -162,6 +162,7 @@ template <int BN, bool kSwiGLU, bool kGather>
 __global__ void __launch_bounds__(W8Cfg<BN>::kThreads, 1)
     k_gemm_w8a8(const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__ CUtensorMap tm_w1,
                 const __grid_constant__ CUtensorMap tm_act, const W8GemmArgs a) {
+    pdl_enter();
     using C = W8Cfg<BN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -338,8 +339,8 @@ int launch_gemm_w8a8_inst(const W8GemmArgs& a, const void* act, const void* w0, 
         return MOE_ERR_CUDA;
     const int m_tiles = kSwiGLU ? a.R0 / 64 : a.R0 / 128;
     const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(max_row_tiles * m_tiles, sms_cache[dev & 15]));
-    kern<<<static_cast<unsigned>(grid), C::kThreads, C::kAlloc, stream>>>(m0, m1, mact, a);
-    return launch_status();
+    return launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(C::kThreads), C::kAlloc, stream, m0, m1, mact,
+                      a);
 }
 
 // Token-tile width for the expected rows per expert: the narrow decode widths of the W4A8 GEMM

@@ -21,13 +21,14 @@
 //              wide tiles also commit the shared A / activation stage.  The warp owns the TMEM.
 //
 // Widening (see tc_tiles.cuh for the arithmetic):
-//   kUnsigned (narrow gate/up tiles, decode): byte = nibble = E4M3 of (code+8)*2^-9, so TMEM
+//   kUnsigned (narrow tiles, decode: gate/up and down): byte = nibble = E4M3 of (code+8)*2^-9, so TMEM
 //     holds 2^-9 * sum_k q_k*(code_k + 8) and the promotion subtracts the offset term with the
 //     group's activation sum: acc += 512*s*partial - 8*s*sum_k q_k (one more FMA per element;
 //     a tcgen05.mma costs the same issue time at N = 16 as at N = 64, so the offset is cheaper
 //     in the promotion than as four more MMAs).
-//   signed (the down GEMM and all wide token tiles): byte = E4M3(code) by byte-permute lookup;
-//     exact codes, so no offset term that would amplify the tensor core's accumulation error.
+//   signed (wide token tiles, prefill): byte = E4M3(code) by byte-permute lookup (12 integer ops
+//     per 8 codes against 2-5 unsigned; the unsigned form needs a [G][BN] group-sum table that
+//     wide tiles have no shared memory left for).
 //
 // Hybrid layers pass an expert -> slab map: the launch then takes only its format's experts and
 // reads each one's weights from its slab.
@@ -160,9 +161,18 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
     const int G = a.K / kGroup;
     const int nst = (G + C::kGS - 1) / C::kGS;             // stages per tile
     const int m_tiles = kSwiGLU ? a.R0 / 64 : a.R0 / 128;
+    // Programmatic dependent launch (common.cuh).  The gate/up instance reads the expert offsets
+    // of the grid just before it, so it waits first.  The down instance's offsets, weights and
+    // scales are older than the grid before it (the requantization), so it reads them and streams
+    // its first weight stages before waiting; only the activations and their scales wait.
+    if constexpr (kSwiGLU) pdl_enter();
+    else pdl_trigger();
     const int row_tiles = row_tile_prefix(a.offsets, a.E, BN, pre, soff, a.slot_of, a.slot_want);
     const int64_t n_tiles = (int64_t)row_tiles * m_tiles;
-    if ((int64_t)blockIdx.x >= n_tiles) return;
+    if ((int64_t)blockIdx.x >= n_tiles) {
+        pdl_wait();                                        // no CTA completes before its predecessor
+        return;
+    }
 
     if (tid == 0) {
         for (int i = 0; i < C::kRW; ++i) { tc::mbar_init(&w_full[i], 1); tc::mbar_init(&w_empty[i], C::kNW); }
@@ -197,6 +207,19 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
         }
         ws::Ring<C::kRW> rw;
         ws::Ring<C::kRB> rb;
+        int pre_w = 0;                        // weight stages of the first tile issued before the wait
+        if constexpr (!kSwiGLU) {
+            if (lane == 0) {
+                const int rt = static_cast<int>(blockIdx.x / m_tiles), mt = static_cast<int>(blockIdx.x % m_tiles);
+                const int wb = weight_slab(a.slot_of, expert_of_tile(pre, a.E, rt));
+                pre_w = min(nst, C::kRW);
+                for (int st = 0; st < pre_w; ++st) {   // a fresh ring: slots 0.. are free, phase 0
+                    tc::mbar_arrive_expect_tx(&w_full[st], C::kRaw);
+                    ws::tma_load_2d(wring + st * C::kRaw, &tm_w0, st * C::kGS * 64, wb * a.R0 + mt * 128, &w_full[st]);
+                }
+            }
+            pdl_wait();
+        }
         for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
             if (__shfl_sync(0xffffffffu, *abort, 0)) break;
             const int rt = static_cast<int>(tile / m_tiles), mt = static_cast<int>(tile % m_tiles);
@@ -215,20 +238,25 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
                 const int g0 = st * C::kGS, ng = min(C::kGS, G - g0);
                 const int ws_ = rw.idx, bs = rb.idx;
                 int ok = 1;
+                const bool w_issued = !kSwiGLU && tile == blockIdx.x && st < pre_w;
                 if (lane == 0) {
-                    ok = ws::wait(&w_empty[ws_], rw.phase ^ 1u, abort);
-                    if (ok) {
-                        // a stage past K (odd group count) is filled with zeros by the TMA unit
-                        uint8_t* wst = wring + ws_ * C::kRaw;
-                        tc::mbar_arrive_expect_tx(&w_full[ws_], C::kRaw);
-                        const int wb = weight_slab(a.slot_of, e);
-                        if (kSwiGLU) {
-                            const int y = wb * a.R0 + mt * 64;
-                            ws::tma_load_2d(wst, &tm_w0, g0 * 64, y, &w_full[ws_]);
-                            ws::tma_load_2d(wst + 64 * C::kRowB, &tm_w1, g0 * 64, y, &w_full[ws_]);
-                        } else {
-                            ws::tma_load_2d(wst, &tm_w0, g0 * 64, wb * a.R0 + mt * 128, &w_full[ws_]);
+                    if (!w_issued) {
+                        ok = ws::wait(&w_empty[ws_], rw.phase ^ 1u, abort);
+                        if (ok) {
+                            // a stage past K (odd group count) is filled with zeros by the TMA unit
+                            uint8_t* wst = wring + ws_ * C::kRaw;
+                            tc::mbar_arrive_expect_tx(&w_full[ws_], C::kRaw);
+                            const int wb = weight_slab(a.slot_of, e);
+                            if (kSwiGLU) {
+                                const int y = wb * a.R0 + mt * 64;
+                                ws::tma_load_2d(wst, &tm_w0, g0 * 64, y, &w_full[ws_]);
+                                ws::tma_load_2d(wst + 64 * C::kRowB, &tm_w1, g0 * 64, y, &w_full[ws_]);
+                            } else {
+                                ws::tma_load_2d(wst, &tm_w0, g0 * 64, wb * a.R0 + mt * 128, &w_full[ws_]);
+                            }
                         }
+                    }
+                    if (ok) {
                         ok = ws::wait(&b_empty[bs], rb.phase ^ 1u, abort);
                         if (ok) tc::mbar_arrive_expect_tx(&b_full[bs], b_bytes * ng);
                     }
@@ -366,6 +394,7 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
         }
     } else if (warp < C::kNW + C::kNP) {
         // ------------------------------------------------------------ promotion + epilogue warps
+        if constexpr (!kSwiGLU) pdl_wait();                // s_row: the requantization's scales
         // Promotion warp i owns TMEM lanes 32*(i % 4) .. +31 (warp id % 4 selects the lanes) and
         // the token columns [ch*kCPW, (ch+1)*kCPW) of them.
         constexpr int kCPW = C::kCPW;
@@ -529,6 +558,7 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
     }
 
     __syncwarp();          // single-lane roles reconverge before the CTA-wide barrier
+    if constexpr (!kSwiGLU) pdl_wait();   // (returns at once in the roles that waited already)
     __syncthreads();
     if (*abort && tid == 0) atomicExch(&g_device_status, 1);
     if (warp == C::kWarpMma) {
@@ -543,6 +573,7 @@ template <int BN, bool kUnsigned, bool kSwiGLU, bool kGather>
 int launch_gemm_ws_inst(const WsGemmArgs& a, const void* act, const void* w0, const void* w1,
                         int64_t max_row_tiles, cudaStream_t stream) {
     using C = WsCfg<BN, kUnsigned>;
+    if (kUnsigned && !a.qsum) return MOE_ERR_INVALID_ARG;   // the +8 offset needs the group sums
     static TcLaunchShape cache[16];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
@@ -567,8 +598,8 @@ int launch_gemm_ws_inst(const WsGemmArgs& a, const void* act, const void* w0, co
     const int m_tiles = kSwiGLU ? a.R0 / 64 : a.R0 / 128;
     const int64_t grid = std::max<int64_t>(
         1, std::min<int64_t>(max_row_tiles * m_tiles, (int64_t)c.sms * c.ctas_per_sm));
-    kern<<<static_cast<unsigned>(grid), C::kThreads, C::kAlloc, stream>>>(m0, m1, mact, a);
-    return launch_status();
+    return launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(C::kThreads), C::kAlloc, stream, m0, m1,
+                      mact, a);
 }
 
 // Narrow token tiles (decode): the gate/up instance gathers its activation rows by token from the
@@ -581,11 +612,12 @@ int launch_gemm_ws(const WsGemmArgs& a, const void* act, const void* w0, const v
     const int BN = ws_tile_rows(a.P, a.E);
     const int64_t max_row_tiles = ((int64_t)a.P + BN - 1) / BN + a.E;
     switch (BN) {
-        // narrow gate/up tiles widen unsigned (the FP8 requantization after them absorbs the
-        // accumulation error of the +8 offset); the down GEMM, whose sums are the layer output,
-        // keeps the exact signed codes
-        case 16: return launch_gemm_ws_inst<16, kSwiGLU, kSwiGLU, kSwiGLU>(a, act, w0, w1, max_row_tiles, stream);
-        case 32: return launch_gemm_ws_inst<32, kSwiGLU, kSwiGLU, kSwiGLU>(a, act, w0, w1, max_row_tiles, stream);
+        // narrow tiles (decode) widen unsigned: the tensor core sums the +8-offset products in fp32
+        // without loss (measured: exact, or 0.5 ulp, over 128-wide groups), and the promotion
+        // removes the offset with the activation rows' group sums (per token for the gathering
+        // gate/up instance, per sorted row for the down instance)
+        case 16: return launch_gemm_ws_inst<16, true, kSwiGLU, kSwiGLU>(a, act, w0, w1, max_row_tiles, stream);
+        case 32: return launch_gemm_ws_inst<32, true, kSwiGLU, kSwiGLU>(a, act, w0, w1, max_row_tiles, stream);
         case 128: return launch_gemm_ws_inst<128, false, kSwiGLU, false>(a, act, w0, w1, max_row_tiles, stream);
         default: return launch_gemm_ws_inst<192, false, kSwiGLU, false>(a, act, w0, w1, max_row_tiles, stream);
     }

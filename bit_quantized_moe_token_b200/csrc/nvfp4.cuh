@@ -30,6 +30,7 @@ __device__ __forceinline__ uint32_t e2m1_code(float x) {
 // amax over each expert projection (float bits, atomic max; the target words start at 0).
 __global__ void __launch_bounds__(256) k_nvfp4_amax(const uint4* __restrict__ w, int64_t chunks_per_expert,
                                                      unsigned* __restrict__ amax_bits) {
+    pdl_enter();
     const int64_t e = blockIdx.y;
     const uint4* we = w + e * chunks_per_expert;
     float a = 0.0f;
@@ -51,6 +52,7 @@ __global__ void __launch_bounds__(256) k_nvfp4_amax(const uint4* __restrict__ w,
 __global__ void __launch_bounds__(256) k_nvfp4_quant(const uint4* __restrict__ w, int64_t blocks_per_expert,
                                                       int64_t experts, const unsigned* __restrict__ amax_bits,
                                                       uint2* __restrict__ codes, uint8_t* __restrict__ scales) {
+    pdl_enter();
     const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
     if (i >= blocks_per_expert * experts) return;
     const int64_t e = i / blocks_per_expert;
@@ -78,6 +80,7 @@ __global__ void __launch_bounds__(256) k_nvfp4_quant(const uint4* __restrict__ w
 }
 
 __global__ void k_nvfp4_finish(unsigned* __restrict__ s2_bits, int64_t experts) {
+    pdl_enter();
     const int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
     if (e < experts) s2_bits[e] = __float_as_uint(__fdiv_rn(__uint_as_float(s2_bits[e]), 6.0f * kFp8Max));
 }
@@ -85,6 +88,7 @@ __global__ void k_nvfp4_finish(unsigned* __restrict__ s2_bits, int64_t experts) 
 // FP8 E4M3 codes -> f16 values (exact), eight per thread.
 __global__ void __launch_bounds__(256) k_e4m3_to_f16(const uint2* __restrict__ q, int64_t n8,
                                                      uint4* __restrict__ out) {
+    pdl_enter();
     const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
     if (i >= n8) return;
     const uint2 c = __ldg(q + i);
@@ -102,9 +106,8 @@ __global__ void __launch_bounds__(256) k_e4m3_to_f16(const uint2* __restrict__ q
 inline int launch_e4m3_to_f16(const uint8_t* q, int64_t n, uint16_t* out, cudaStream_t stream) {
     if (n == 0) return MOE_OK;
     const int64_t n8 = n / 8;
-    k_e4m3_to_f16<<<static_cast<unsigned>((n8 + 255) / 256), 256, 0, stream>>>(
-        reinterpret_cast<const uint2*>(q), n8, reinterpret_cast<uint4*>(out));
-    return launch_status();
+    return launch_pdl(k_e4m3_to_f16, dim3(static_cast<unsigned>((n8 + 255) / 256)), dim3(256), 0, stream,
+                      reinterpret_cast<const uint2*>(q), n8, reinterpret_cast<uint4*>(out));
 }
 
 }  // namespace moe

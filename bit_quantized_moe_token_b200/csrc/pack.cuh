@@ -15,6 +15,7 @@ __global__ void __launch_bounds__(256) k_pack_weights(const uint4* __restrict__ 
                                                       int64_t words_per_row,
                                                       int32_t* __restrict__ packed,
                                                       uint16_t* __restrict__ scales) {
+    pdl_enter();
     const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
     const bool live = i < words;
     const uint4 v = live ? __ldg(w + i) : make_uint4(0u, 0u, 0u, 0u);

@@ -55,6 +55,7 @@ __global__ void __launch_bounds__(256) k_quant_tokens(const uint16_t* __restrict
                                                       const int32_t* __restrict__ row_of_pair,
                                                       int k, uint8_t* __restrict__ q_tok,
                                                       float* __restrict__ s_tok) {
+    pdl_enter();
     __shared__ float red[32];
     const int64_t t = blockIdx.x;
     const uint4* row = reinterpret_cast<const uint4*>(x + t * H);
@@ -106,9 +107,8 @@ inline int launch_quant_tokens(const uint16_t* x, int64_t T, int64_t H, uint8_t*
                                const int32_t* row_of_pair, int k, cudaStream_t stream,
                                uint8_t* q_tok = nullptr, float* s_tok = nullptr) {
     if (T == 0) return MOE_OK;
-    k_quant_tokens<<<static_cast<unsigned>(T), 256, 0, stream>>>(x, static_cast<int>(H), q, s,
-                                                                 row_of_pair, k, q_tok, s_tok);
-    return launch_status();
+    return launch_pdl(k_quant_tokens, dim3(static_cast<unsigned>(T)), dim3(256), 0, stream, x, static_cast<int>(H),
+                      q, s, row_of_pair, k, q_tok, s_tok);
 }
 
 }  // namespace moe

@@ -75,6 +75,7 @@ template <int EPL>
 __global__ void __launch_bounds__(256) k_topk(const float* __restrict__ logits, int64_t T, int E,
                                               int k, int32_t* __restrict__ ids,
                                               float* __restrict__ gates) {
+    pdl_enter();
     const int64_t t = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
     if (t >= T) return;  // uniform per warp
     topk_row<EPL>(logits + t * E, E, k, ids + t * k, gates + t * k, threadIdx.x & 31);
@@ -85,13 +86,14 @@ inline int launch_topk(const float* logits, int64_t T, int E, int k, int32_t* id
     const int64_t warps = T;
     const unsigned blocks = static_cast<unsigned>((warps * 32 + 255) / 256);
     const int epl = (E + 31) / 32;
-    if (epl <= 1) k_topk<1><<<blocks, 256, 0, stream>>>(logits, T, E, k, ids, gates);
-    else if (epl <= 2) k_topk<2><<<blocks, 256, 0, stream>>>(logits, T, E, k, ids, gates);
-    else if (epl <= 4) k_topk<4><<<blocks, 256, 0, stream>>>(logits, T, E, k, ids, gates);
-    else if (epl <= 8) k_topk<8><<<blocks, 256, 0, stream>>>(logits, T, E, k, ids, gates);
-    else if (epl <= 16) k_topk<16><<<blocks, 256, 0, stream>>>(logits, T, E, k, ids, gates);
-    else k_topk<32><<<blocks, 256, 0, stream>>>(logits, T, E, k, ids, gates);
-    return launch_status();
+#define MOE_TK(N) launch_pdl(k_topk<N>, dim3(blocks), dim3(256), 0, stream, logits, T, E, k, ids, gates)
+    if (epl <= 1) return MOE_TK(1);
+    if (epl <= 2) return MOE_TK(2);
+    if (epl <= 4) return MOE_TK(4);
+    if (epl <= 8) return MOE_TK(8);
+    if (epl <= 16) return MOE_TK(16);
+    return MOE_TK(32);
+#undef MOE_TK
 }
 
 // ------------------------------------------------------------------------------------------
@@ -188,6 +190,7 @@ __global__ void __launch_bounds__(1024) k_permute_single(const int32_t* __restri
                                                          int32_t* __restrict__ sorted,
                                                          int32_t* __restrict__ rop,
                                                          unsigned* __restrict__ zero, int64_t n_zero) {
+    pdl_enter();
     extern __shared__ int sm[];
     for (int64_t i = threadIdx.x; i < n_zero; i += blockDim.x) zero[i] = 0u;
     permute_block(ids, P, E, offsets, sorted, rop, sm);
@@ -196,6 +199,7 @@ __global__ void __launch_bounds__(1024) k_permute_single(const int32_t* __restri
 // Large P, pass 1: per-chunk expert histogram -> counts[c][E].
 __global__ void __launch_bounds__(1024) k_chunk_hist(const int32_t* __restrict__ ids, int64_t P,
                                                      int E, int32_t* __restrict__ counts) {
+    pdl_enter();
     extern __shared__ int sm[];
     for (int i = threadIdx.x; i < E; i += blockDim.x) sm[i] = 0;
     __syncthreads();
@@ -209,6 +213,7 @@ __global__ void __launch_bounds__(1024) k_chunk_hist(const int32_t* __restrict__
 __global__ void __launch_bounds__(1024) k_chunk_scan(int32_t* __restrict__ counts, int64_t nchunks,
                                                      int64_t P, int E,
                                                      int32_t* __restrict__ offsets) {
+    pdl_enter();
     extern __shared__ int sm[];
     int* tot = sm;          // E
     int* base = tot + E;    // E
@@ -237,6 +242,7 @@ __global__ void __launch_bounds__(1024) k_chunk_scatter(const int32_t* __restric
                                                         int E, const int32_t* __restrict__ counts,
                                                         int32_t* __restrict__ sorted,
                                                         int32_t* __restrict__ rop) {
+    pdl_enter();
     extern __shared__ int sm[];
     int* base = sm;         // E
     int* wc = base + E;     // 32 * E
@@ -265,19 +271,23 @@ inline int launch_permute(const int32_t* ids, int64_t T, int E, int k, int32_t* 
     if (P <= kSinglePassMaxP) {
         const size_t smem = permute_block_smem(E);
         if (set_smem((const void*)k_permute_single, smem)) return MOE_ERR_CUDA;
-        k_permute_single<<<1, 1024, smem, stream>>>(ids, P, E, offsets, sorted, rop, zero, n_zero);
-        return launch_status();
+        return launch_pdl(k_permute_single, dim3(1), dim3(1024), smem, stream, ids, P, E, offsets, sorted, rop, zero,
+                          n_zero);
     }
     if (zero && cudaMemsetAsync(zero, 0, n_zero * sizeof(unsigned), stream) != cudaSuccess)
         return MOE_ERR_CUDA;
     const int64_t nchunks = (P + kChunk - 1) / kChunk;
-    k_chunk_hist<<<static_cast<unsigned>(nchunks), 1024, E * sizeof(int), stream>>>(ids, P, E, counts);
-    k_chunk_scan<<<1, 1024, (2 * E + 33) * sizeof(int), stream>>>(counts, nchunks, P, E, offsets);
+    int st = launch_pdl(k_chunk_hist, dim3(static_cast<unsigned>(nchunks)), dim3(1024), E * sizeof(int), stream, ids,
+                        P, E, counts);
+    if (st == MOE_OK)
+        st = launch_pdl(k_chunk_scan, dim3(1), dim3(1024), (2 * E + 33) * sizeof(int), stream, counts, nchunks, P, E,
+                        offsets);
     const size_t smem = (E + 32 * E) * sizeof(int);
-    if (set_smem((const void*)k_chunk_scatter, smem)) return MOE_ERR_CUDA;
-    k_chunk_scatter<<<static_cast<unsigned>(nchunks), 1024, smem, stream>>>(ids, P, E, counts, sorted,
-                                                                            rop);
-    return launch_status();
+    if (st == MOE_OK && set_smem((const void*)k_chunk_scatter, smem)) return MOE_ERR_CUDA;
+    if (st == MOE_OK)
+        st = launch_pdl(k_chunk_scatter, dim3(static_cast<unsigned>(nchunks)), dim3(1024), smem, stream, ids, P, E,
+                        counts, sorted, rop);
+    return st;
 }
 
 inline int route_args_ok(int64_t T, int E, int k) {

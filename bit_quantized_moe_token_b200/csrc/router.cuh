@@ -85,6 +85,7 @@ template <int kT>
 __global__ void __launch_bounds__(256) k_router_rows(const uint4* __restrict__ x,
                                                      const uint4* __restrict__ wr, int T, int HC,
                                                      int E, float* __restrict__ logits) {
+    pdl_enter();
     router_rows_cta<kT>(x, wr, T, HC, E, blockIdx.x, logits);
 }
 
@@ -113,6 +114,7 @@ __global__ void __launch_bounds__(256) k_router_front(const uint4* __restrict__ 
                                                       unsigned* __restrict__ counter,
                                                       uint8_t* __restrict__ xq, float* __restrict__ s_x,
                                                       float* __restrict__ qsum) {
+    pdl_enter();
     __shared__ float red[32];
     router_rows_cta<kT>(x, wr, T, HC, E, blockIdx.x, logits);
     if (xq && (int)blockIdx.x < T)
@@ -133,6 +135,7 @@ __global__ void __launch_bounds__(256) k_router_gemv(const uint4* __restrict__ x
                                                      int32_t* __restrict__ ids = nullptr,
                                                      float* __restrict__ gates = nullptr,
                                                      unsigned* __restrict__ counters = nullptr) {
+    pdl_enter();
     extern __shared__ uint4 sx[];                    // [kTB][HC]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int e = blockIdx.x * 8 + warp;
@@ -191,10 +194,9 @@ int launch_router_gemv(const uint16_t* x, const uint16_t* wr, int64_t T, int H, 
         smem_set[dev & 15] = static_cast<int>(smem);
     }
     const dim3 grid(static_cast<unsigned>((E + 7) / 8), static_cast<unsigned>((T + kTB - 1) / kTB));
-    kern<<<grid, 256, smem, stream>>>(
-        reinterpret_cast<const uint4*>(x), reinterpret_cast<const uint4*>(wr), static_cast<int>(T), H / 8, E,
-        logits, k, ids, gates, counters);
-    return launch_status();
+    return launch_pdl(kern, grid, dim3(256), smem, stream, reinterpret_cast<const uint4*>(x),
+                      reinterpret_cast<const uint4*>(wr), static_cast<int>(T), H / 8, E, logits, k, ids, gates,
+                      counters);
 }
 
 inline bool router_uses_tensor_cores(int64_t T, int H, int E) {
@@ -224,16 +226,15 @@ inline int launch_router_topk(const uint16_t* x, const uint16_t* wr, int64_t T, 
     const uint4* x4 = reinterpret_cast<const uint4*>(x);
     const uint4* w4 = reinterpret_cast<const uint4*>(wr);
     if (T <= 16) {
-#define MOE_RF(N) k_router_front<16, N><<<static_cast<unsigned>(E), 256, 0, stream>>>( \
-        x4, w4, static_cast<int>(T), H / 8, E, k, logits, ids, gates, counters, xq, s_x, qsum)
-        if (epl <= 1) MOE_RF(1);
-        else if (epl <= 2) MOE_RF(2);
-        else if (epl <= 4) MOE_RF(4);
-        else if (epl <= 8) MOE_RF(8);
-        else if (epl <= 16) MOE_RF(16);
-        else MOE_RF(32);
+#define MOE_RF(N) launch_pdl(k_router_front<16, N>, dim3(static_cast<unsigned>(E)), dim3(256), 0, stream, x4, w4, \
+                             static_cast<int>(T), H / 8, E, k, logits, ids, gates, counters, xq, s_x, qsum)
+        if (epl <= 1) return MOE_RF(1);
+        if (epl <= 2) return MOE_RF(2);
+        if (epl <= 4) return MOE_RF(4);
+        if (epl <= 8) return MOE_RF(8);
+        if (epl <= 16) return MOE_RF(16);
+        return MOE_RF(32);
 #undef MOE_RF
-        return launch_status();
     }
 #define MOE_RG(TB, N) launch_router_gemv<TB, true, N>(x, wr, T, H, E, logits, stream, k, ids, gates, counters)
 #define MOE_RG_E(TB) (epl <= 1 ? MOE_RG(TB, 1) : epl <= 2 ? MOE_RG(TB, 2) : epl <= 4 ? MOE_RG(TB, 4) \
@@ -264,10 +265,9 @@ extern "C" int moe_router_logits(const uint16_t* x_bf16, const uint16_t* wr_bf16
         return launch_gemm_bf16_ws<false>(a, x_bf16, wr_bf16, nullptr, stream);
     }
     if (T <= 16) {
-        k_router_rows<16><<<static_cast<unsigned>(E), 256, 0, stream>>>(
-            reinterpret_cast<const uint4*>(x_bf16), reinterpret_cast<const uint4*>(wr_bf16),
-            static_cast<int>(T), H / 8, E, logits);
-        return launch_status();
+        return launch_pdl(k_router_rows<16>, dim3(static_cast<unsigned>(E)), dim3(256), 0, stream,
+                          reinterpret_cast<const uint4*>(x_bf16), reinterpret_cast<const uint4*>(wr_bf16),
+                          static_cast<int>(T), H / 8, E, logits);
     }
     return H <= 4096 ? launch_router_gemv<16>(x_bf16, wr_bf16, T, H, E, logits, stream)
                      : launch_router_gemv<4>(x_bf16, wr_bf16, T, H, E, logits, stream);

@@ -86,6 +86,8 @@ WORKLOADS = {
                               routing="uniform"),
     "prefill_t512_e64_zipf": Workload("prefill_t512_e64_zipf", T=512, H=4096, N=2048, E=64, k=6,
                                       outliers=True, routing="zipf"),
+    "prefill_t4096_e64": Workload("prefill_t4096_e64", T=4096, H=4096, N=2048, E=64, k=6,
+                                  outliers=False, routing="uniform"),
 }
 
 
