@@ -77,7 +77,7 @@ class _CLayerH(ctypes.Structure):
 class _CLayout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in
                 ("topk_ids", "topk_w", "expert_offsets", "sorted_pairs", "row_of_pair",
-                 "xq", "s_x", "hq", "s_h", "total")]
+                 "xq", "s_x", "hq", "s_h", "total", "act_order")]
 
 
 _lib = None

@@ -101,6 +101,17 @@ __device__ __forceinline__ float e4m3x8_sum(uint2 codes) {
     return s;
 }
 
+// The K order of the FP8 activations that narrow W4A8 token tiles read: within each block of
+// 8 columns, columns 0,2,4,6,1,3,5,7 (the order in which the GEMM's unsigned widening splits a
+// packed word into its even and odd nibbles, so that it needs no byte interleave).  perm8 maps
+// eight codes in column order (byte i of .x/.y = column i / i+4) to that order; unperm8 inverts it.
+__device__ __forceinline__ uint2 perm8(uint2 c) {
+    return make_uint2(__byte_perm(c.x, c.y, 0x6420), __byte_perm(c.x, c.y, 0x7531));
+}
+__device__ __forceinline__ uint2 unperm8(uint2 c) {
+    return make_uint2(__byte_perm(c.x, c.y, 0x5140), __byte_perm(c.x, c.y, 0x7362));
+}
+
 // Sum over the 16 lanes of each half-warp (all 32 lanes take part).
 __device__ __forceinline__ float halfwarp_sum(float v) {
 #pragma unroll

@@ -16,11 +16,12 @@ namespace moe {
 // S5 requantization of the SwiGLU activations h (fp32, one expert-sorted row per CTA, written
 // by the gate/up GEMM together with max|h| per row): s_h = max|h| / 448, Hq = e4m3(h / s_h).
 // With qsum non-null it also writes each row's per-128-column sums of the FP8 values (the down
-// GEMM's unsigned widening removes its +8 offset with them): a half-warp covers one group.
+// GEMM's unsigned widening removes its +8 offset with them; a half-warp covers one group).  With
+// perm the codes are stored in the narrow W4A8 tiles' K order (perm8).
 __global__ void __launch_bounds__(256) k_requant(const float* __restrict__ h, int N,
                                                  const unsigned* __restrict__ amax,
                                                  uint8_t* __restrict__ hq, float* __restrict__ s_h,
-                                                 float* __restrict__ qsum) {
+                                                 float* __restrict__ qsum, bool perm) {
     pdl_enter();
     const int64_t r = blockIdx.x;
     const float s = __fdiv_rn(__uint_as_float(amax[r]), kFp8Max);
@@ -35,7 +36,7 @@ __global__ void __launch_bounds__(256) k_requant(const float* __restrict__ h, in
             codes.y = static_cast<uint32_t>(f32x2_to_e4m3x2(__fdiv_rn(b.x, s), __fdiv_rn(b.y, s))) |
                       (static_cast<uint32_t>(f32x2_to_e4m3x2(__fdiv_rn(b.z, s), __fdiv_rn(b.w, s))) << 16);
         }
-        reinterpret_cast<uint2*>(hq + r * N)[c] = codes;
+        reinterpret_cast<uint2*>(hq + r * N)[c] = perm ? perm8(codes) : codes;
         if (qsum) {
             const float gs = halfwarp_sum(e4m3x8_sum(codes));
             if ((threadIdx.x & 15) == 0) qsum[r * G + c / 16] = gs;
@@ -222,6 +223,7 @@ extern "C" int moe_w4a8_workspace_layout(const moe_w4a8_layer* layer, int64_t T,
     out->hq = p.hq;
     out->s_h = p.s_h;
     out->total = p.total;
+    out->act_order = moe::ws_narrow(moe::ws_tile_rows(T * k, layer->E)) ? 1 : 0;   // W4A8 layer: see the header
     return MOE_OK;
 }
 
@@ -371,6 +373,9 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const ExpertSet& xw, const ui
     const bool gather = ws_narrow(tc_tile_rows(P, L.E));
     const bool hybrid = xw.fmt == kFmtHybrid;
     float* qsum_x = (xw.fmt == kFmtW4A8 || hybrid) ? qs_x : nullptr;   // the unsigned widening only
+    // narrow W4A8 / hybrid layers store xq and hq in the unsigned widening's K order (perm8); the
+    // token quantization writes xq that way exactly when it is given the group sums
+    const bool act_perm = gather && qsum_x != nullptr;
     uint16_t* act16 = xw.fmt >= kFmtNvfp4 ? (uint16_t*)at(p.act16) : nullptr;
     int32_t* slot_of = hybrid ? (int32_t*)at(p.slot_of) : nullptr;
     // the two launches of a hybrid layer's GEMM: W4A8 on the cold experts, NVFP4 on the hot ones
@@ -467,7 +472,9 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const ExpertSet& xw, const ui
     // S4 + SwiGLU: h = silu(G) * U, max|h| per row
     if (run_f4) {
         // f16 copy of the FP8 activations (exact), then the f16 tensor-core GEMM
-        if ((st = launch_e4m3_to_f16(gather ? xq : xs, (gather ? T : P) * L.H, act16, stream))) return st;
+        // (in a narrow hybrid layer the per-token codes are in the W4A8 tiles' K order)
+        if ((st = launch_e4m3_to_f16(gather ? xq : xs, (gather ? T : P) * L.H, act16, stream, act_perm)))
+            return st;
         F4GemmArgs f{W8GemmArgs{gather ? sx : sxs, nullptr, nullptr, offsets, L.E, L.N, L.H, (int)P, h, L.N,
                                 amax, sorted, k, (int)T},
                      f4_gs, f4_us, f4_g2, f4_u2, slot_of, hybrid ? kSlotHot : kSlotAll};
@@ -492,16 +499,17 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const ExpertSet& xw, const ui
     }
     sm.mark(4, stream);
     // S5
-    // the W4A8 down GEMM widens its narrow tiles unsigned and needs the requantized rows' group sums
-    const bool down_sums = run_w4 && ws_narrow(ws_tile_rows(P, L.E));
+    // the W4A8 down GEMM widens its narrow tiles unsigned and needs the requantized rows' group sums;
+    // hq, like xq, is stored in those tiles' K order whenever a W4A8 or hybrid layer runs narrow
+    const bool down_sums = run_w4 && gather;
     if ((st = launch_pdl(k_requant, dim3(static_cast<unsigned>(P)), dim3(256), 0, stream, h, L.N, amax, hq, sh,
-                         down_sums ? qs_h : nullptr)))
+                         down_sums ? qs_h : nullptr, act_perm)))
         return st;
     sm.launches += 1;
     sm.mark(5, stream);
     // S6
     if (run_f4) {
-        if ((st = launch_e4m3_to_f16(hq, P * L.N, act16, stream))) return st;
+        if ((st = launch_e4m3_to_f16(hq, P * L.N, act16, stream, act_perm))) return st;
         F4GemmArgs f{W8GemmArgs{sh, nullptr, nullptr, offsets, L.E, L.H, L.N, (int)P, y, L.H, nullptr, sorted,
                                 k, (int)T},
                      f4_ds, nullptr, f4_d2, nullptr, slot_of, hybrid ? kSlotHot : kSlotAll};
@@ -555,7 +563,9 @@ extern "C" int moe_w8a8_workspace_layout(const moe_w8a8_layer* layer, int64_t T,
                                          moe_w4a8_ws_layout* out) {
     if (!layer) return MOE_ERR_INVALID_ARG;
     const moe_w4a8_layer s = moe::shape_of(*layer);
-    return moe_w4a8_workspace_layout(&s, T, k, out);
+    const int st = moe_w4a8_workspace_layout(&s, T, k, out);
+    if (st == MOE_OK) out->act_order = 0;          // row-scaled FP8 tiles read the codes in column order
+    return st;
 }
 
 extern "C" int moe_w8a8_forward(const moe_w8a8_layer* layer, const uint16_t* x_bf16,
@@ -633,7 +643,10 @@ extern "C" int moe_nvfp4_workspace_layout(const moe_nvfp4_layer* layer, int64_t 
     if (!layer) return MOE_ERR_INVALID_ARG;
     const moe_w4a8_layer s = moe::shape_of(*layer);
     int st = moe_w4a8_workspace_layout(&s, T, k, out);
-    if (st == MOE_OK) out->total = moe::plan_workspace(s, T, k, moe::kFmtNvfp4).total;
+    if (st == MOE_OK) {
+        out->total = moe::plan_workspace(s, T, k, moe::kFmtNvfp4).total;
+        out->act_order = 0;                        // NVFP4 layers keep the codes in column order
+    }
     return st;
 }
 

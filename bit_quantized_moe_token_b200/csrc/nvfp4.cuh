@@ -85,13 +85,14 @@ __global__ void k_nvfp4_finish(unsigned* __restrict__ s2_bits, int64_t experts) 
     if (e < experts) s2_bits[e] = __float_as_uint(__fdiv_rn(__uint_as_float(s2_bits[e]), 6.0f * kFp8Max));
 }
 
-// FP8 E4M3 codes -> f16 values (exact), eight per thread.
+// FP8 E4M3 codes -> f16 values (exact), eight per thread; with `unperm` the codes are in the
+// narrow W4A8 tiles' K order (perm8) and the f16 values come out in column order.
 __global__ void __launch_bounds__(256) k_e4m3_to_f16(const uint2* __restrict__ q, int64_t n8,
-                                                     uint4* __restrict__ out) {
+                                                     uint4* __restrict__ out, bool unperm) {
     pdl_enter();
     const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
     if (i >= n8) return;
-    const uint2 c = __ldg(q + i);
+    const uint2 c = unperm ? unperm8(__ldg(q + i)) : __ldg(q + i);
     const uint32_t w[2] = {c.x, c.y};
     uint32_t o[4];
 #pragma unroll
@@ -103,11 +104,12 @@ __global__ void __launch_bounds__(256) k_e4m3_to_f16(const uint2* __restrict__ q
     out[i] = make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-inline int launch_e4m3_to_f16(const uint8_t* q, int64_t n, uint16_t* out, cudaStream_t stream) {
+inline int launch_e4m3_to_f16(const uint8_t* q, int64_t n, uint16_t* out, cudaStream_t stream,
+                              bool unperm = false) {
     if (n == 0) return MOE_OK;
     const int64_t n8 = n / 8;
     return launch_pdl(k_e4m3_to_f16, dim3(static_cast<unsigned>((n8 + 255) / 256)), dim3(256), 0, stream,
-                      reinterpret_cast<const uint2*>(q), n8, reinterpret_cast<uint4*>(out));
+                      reinterpret_cast<const uint2*>(q), n8, reinterpret_cast<uint4*>(out), unperm);
 }
 
 }  // namespace moe

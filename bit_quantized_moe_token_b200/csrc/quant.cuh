@@ -81,7 +81,9 @@ __global__ void __launch_bounds__(256) k_quant_tokens(const uint16_t* __restrict
 
 // S1 for token t by the whole CTA: amax, scale = amax / 448, the FP8 codes written once per
 // token, and (qsum non-null) per K-group of 128 (16 chunks = one half-warp) the sum of the
-// decoded codes.  Same arithmetic as k_quant_tokens.
+// decoded codes.  Same arithmetic as k_quant_tokens.  The group sums serve the narrow W4A8
+// tiles' unsigned widening, which reads the codes in its own K order: with qsum non-null the
+// codes are stored in that order (perm8).
 __device__ __forceinline__ void quant_token_cta(const uint16_t* __restrict__ x, int64_t t, int H,
                                                 uint8_t* __restrict__ xq, float* __restrict__ s_x,
                                                 float* __restrict__ qsum, float* red) {
@@ -96,7 +98,7 @@ __device__ __forceinline__ void quant_token_cta(const uint16_t* __restrict__ x, 
         const int c = base + threadIdx.x;
         const bool live = c < chunks;
         const uint2 codes = live ? quant8(__ldg(row + c), s) : make_uint2(0u, 0u);
-        if (live) reinterpret_cast<uint2*>(xq + t * H)[c] = codes;
+        if (live) reinterpret_cast<uint2*>(xq + t * H)[c] = qsum ? perm8(codes) : codes;
         const float gs = halfwarp_sum(e4m3x8_sum(codes));
         if (qsum && live && (threadIdx.x & 15) == 0) qsum[t * G + c / 16] = gs;
     }

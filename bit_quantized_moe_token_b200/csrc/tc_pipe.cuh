@@ -83,56 +83,15 @@ inline PFN_encodeTiled encode_fn() {
     return fn;
 }
 
-// cuTensorMapEncodeTiled with a small per-host-thread memo: a descriptor is a pure function of
-// its arguments, and a layer's calls encode the same few (weights, workspace sections) every
-// time, so repeated calls copy the stored descriptor instead of encoding it again.
+// cuTensorMapEncodeTiled (element strides 1, no interleave, 256-byte L2 promotion, zero fill).
 inline bool encode_tiled(CUtensorMap* m, CUtensorMapDataType dtype, uint32_t rank, const void* base,
                          const cuuint64_t* dims, const cuuint64_t* strides, const cuuint32_t* box,
                          CUtensorMapSwizzle swizzle) {
-    struct Key {
-        const void* base;
-        uint64_t dims[3], strides[2];
-        uint32_t box[3], dtype, rank, swizzle;
-        bool operator==(const Key& o) const {
-            if (base != o.base || dtype != o.dtype || rank != o.rank || swizzle != o.swizzle) return false;
-            for (int i = 0; i < 3; ++i)
-                if (dims[i] != o.dims[i] || box[i] != o.box[i]) return false;
-            return strides[0] == o.strides[0] && strides[1] == o.strides[1];
-        }
-    };
-    struct Entry {
-        Key key;
-        CUtensorMap map;
-        bool used;
-    };
-    constexpr int kSlots = 32;
-    thread_local Entry memo[kSlots] = {};
-    thread_local int next = 0;
-    if (rank < 1 || rank > 3) return false;
-    Key k{};
-    k.base = base;
-    k.dtype = static_cast<uint32_t>(dtype);
-    k.rank = rank;
-    k.swizzle = static_cast<uint32_t>(swizzle);
-    for (uint32_t i = 0; i < rank; ++i) {
-        k.dims[i] = dims[i];
-        k.box[i] = box[i];
-        if (i + 1 < rank) k.strides[i] = strides[i];
-    }
-    for (int i = 0; i < kSlots; ++i)
-        if (memo[i].used && memo[i].key == k) {
-            *m = memo[i].map;
-            return true;
-        }
     PFN_encodeTiled fn = encode_fn();
     if (!fn) return false;
     const cuuint32_t estr[3] = {1, 1, 1};
-    if (fn(m, dtype, rank, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-           swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-        return false;
-    memo[next] = Entry{k, *m, true};
-    next = (next + 1) % kSlots;
-    return true;
+    return fn(m, dtype, rank, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // 2D byte tensor [rows, row_bytes] (row-major) with a box of box_rows x box_bytes.

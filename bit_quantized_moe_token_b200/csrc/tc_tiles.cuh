@@ -8,9 +8,11 @@
 //    8 codes); one FMA per element promotes the group.  Used for wide token tiles (prefill).
 //  * unsigned: byte = the stored nibble itself (code + 8).  Bytes 0x00..0x0F are the E4M3
 //    values 0..15 x 2^-9 (the subnormals and the first normal binade form one equally spaced
-//    ladder), so the MMA sees 2^-9 * (code + 8) with 2-5 integer ops per 8 codes; the GEMM
-//    removes the +8 offset exactly (see gemm_ws.cuh).  Used for narrow token tiles (decode),
-//    where the widening dominates the issue slots.
+//    ladder), so the MMA sees 2^-9 * (code + 8); the GEMM removes the +8 offset (see
+//    gemm_ws.cuh).  The even nibbles become bytes 0..3 and the odd ones bytes 4..7 (3 integer
+//    ops per 8 codes), i.e. K order 0,2,4,6,1,3,5,7 within each word; the activations of these
+//    tiles are stored in the same order (perm8 in common.cuh), and a K-permutation applied to
+//    both operands leaves every dot product unchanged.  Used for narrow token tiles (decode).
 #pragma once
 #include "common.cuh"
 
@@ -24,13 +26,13 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t c) {
     return d;
 }
 
-// Eight codes of one packed word -> eight E4M3 bytes in K order (lo = codes 0..3).
+// Eight codes of one packed word -> eight E4M3 bytes: signed in K order (lo = codes 0..3);
+// unsigned in K order 0,2,4,6 (lo) and 1,3,5,7 (hi).
 template <bool kUnsigned>
 __device__ __forceinline__ uint2 widen8(uint32_t w) {
     if constexpr (kUnsigned) {
-        const uint32_t e = w & 0x0F0F0F0Fu;          // nibbles 0, 2, 4, 6
-        const uint32_t o = (w >> 4) & 0x0F0F0F0Fu;   // nibbles 1, 3, 5, 7
-        return make_uint2(prmt(e, o, 0x5140u), prmt(e, o, 0x7362u));
+        return make_uint2(w & 0x0F0F0F0Fu,            // nibbles 0, 2, 4, 6
+                          (w >> 4) & 0x0F0F0F0Fu);    // nibbles 1, 3, 5, 7
     } else {
         // E4M3 of code = nibble - 8: nibbles 0..7 (negative codes) and 8..15 (0..7)
         constexpr uint32_t kNeg0 = 0xCACCCED0u, kNeg1 = 0xB8C0C4C8u;

@@ -176,11 +176,16 @@ size_t moe_w4a8_workspace_bytes(const moe_w4a8_layer* layer, int64_t T, int k);
  * after the forward completes (all in expert-sorted row order r, P = T*k rows):
  *   topk_ids [T,k] i32, topk_w [T,k] f32, expert_offsets [E+1] i32, sorted_pairs [P] i32,
  *   row_of_pair [P] i32, xq [T,H] e4m3 and s_x [T] f32 (the S1 codes and scales of every
- *   token), hq [P,N] e4m3 and s_h [P] f32 (requantized SwiGLU activations, sorted rows). */
+ *   token), hq [P,N] e4m3 and s_h [P] f32 (requantized SwiGLU activations, sorted rows).
+ * act_order: 0 when xq and hq hold their codes in column order; 1 when, within every block of
+ * 8 columns, they hold columns 0,2,4,6,1,3,5,7 (the order in which the W4A8 GEMM's 16- and
+ * 32-row token tiles split a packed word into its even and odd nibbles; used for W4A8 and
+ * hybrid layers whose tiles are that narrow). */
 typedef struct {
     size_t topk_ids, topk_w, expert_offsets, sorted_pairs, row_of_pair;
     size_t xq, s_x, hq, s_h;
     size_t total;
+    size_t act_order;
 } moe_w4a8_ws_layout;
 int moe_w4a8_workspace_layout(const moe_w4a8_layer* layer, int64_t T, int k,
                               moe_w4a8_ws_layout* out);

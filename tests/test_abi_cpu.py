@@ -169,7 +169,11 @@ def test_w8a8_rejects_bad_args():
     s8 = moe.layer8_struct(256, 4096, 2048)
     s4 = moe.layer_struct(256, 4096, 2048)
     assert moe.moe_w8a8_workspace_bytes(s8, 8, 6) == moe.moe_w4a8_workspace_bytes(s4, 8, 6) > 0
-    assert moe.moe_w8a8_workspace_layout(s8, 8, 6) == moe.moe_w4a8_workspace_layout(s4, 8, 6)
+    l8, l4 = moe.moe_w8a8_workspace_layout(s8, 8, 6), moe.moe_w4a8_workspace_layout(s4, 8, 6)
+    # the same plan; only the W4A8 layer's narrow (decode) tiles keep their codes in the
+    # even/odd-nibble K order
+    assert l8["act_order"] == 0 and l4["act_order"] == 1
+    assert {k: v for k, v in l8.items() if k != "act_order"} == {k: v for k, v in l4.items() if k != "act_order"}
     assert moe.moe_w8a8_workspace_bytes(moe.layer8_struct(256, 4000, 2048), 8, 6) == 0
     assert L.moe_w8a8_forward(ctypes.byref(s8), p, p, 4, 2, p, p, 1 << 24, None) == -1   # null weights
     full = moe._binding._CLayer8(8, 256, 128, p, p, p, p, p, p, 0, 0, None, None, None)

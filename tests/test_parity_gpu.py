@@ -37,6 +37,10 @@ def bits(t):
     return t.detach().contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
 
 
+# stored position p of an 8-column block holds column (0,2,4,6,1,3,5,7)[p]; this gathers them back
+_UNPERM8 = np.argsort(np.array([0, 2, 4, 6, 1, 3, 5, 7]))
+
+
 def ws_views(layer, ws, T, k):
     layout = (moe.moe_w8a8_workspace_layout if isinstance(layer, moe.Layer8) else
               moe.moe_nvfp4_workspace_layout if isinstance(layer, moe.Layer4) else
@@ -46,14 +50,19 @@ def ws_views(layer, ws, T, k):
     b = ws.cpu().numpy()
     def arr(off, dtype, n):
         return np.frombuffer(b[off:off + n * np.dtype(dtype).itemsize].tobytes(), dtype=dtype).copy()
+    def codes(off, rows, cols):
+        c = arr(off, np.uint8, rows * cols).reshape(rows, cols)
+        if lay["act_order"]:                  # columns 0,2,4,6,1,3,5,7 of every 8-column block
+            c = c.reshape(rows, cols // 8, 8)[:, :, _UNPERM8].reshape(rows, cols)
+        return c
     return dict(ids=arr(lay["topk_ids"], np.int32, P).reshape(T, k),
                 gates=arr(lay["topk_w"], np.float32, P).reshape(T, k),
                 offsets=arr(lay["expert_offsets"], np.int32, layer.E + 1),
                 sorted_pairs=arr(lay["sorted_pairs"], np.int32, P),
                 row_of_pair=arr(lay["row_of_pair"], np.int32, P),
-                xq=arr(lay["xq"], np.uint8, T * layer.H).reshape(T, layer.H),
+                xq=codes(lay["xq"], T, layer.H),
                 s_x=arr(lay["s_x"], np.float32, T),
-                hq=arr(lay["hq"], np.uint8, P * layer.N).reshape(P, layer.N),
+                hq=codes(lay["hq"], P, layer.N),
                 s_h=arr(lay["s_h"], np.float32, P))
 
 
