@@ -561,9 +561,11 @@ class LayerH:
                         _ptr(c.sh_gate), _ptr(c.sh_up), _ptr(c.sh_down))
 
     def shape_struct(self) -> _CLayerH:
+        """Shapes and slab counts, null pointers: enough for the size/layout queries."""
         c = self.cold
-        return _CLayerH(self.E, c.H, c.N, 0, 0, None, None, None, None, None, None, None, None, None, None,
-                        None, None, None, None, None, None, None, c.n_shared, c.shared_N, None, None, None)
+        return _CLayerH(self.E, c.H, c.N, int(self.hot_ids.numel()), int(self.cold_ids.numel()), None, None,
+                        None, None, None, None, None, None, None, None, None, None, None, None, None, None, None,
+                        c.n_shared, c.shared_N, None, None, None)
 
 
 def moe_hybrid_workspace_bytes(layer, T: int, k: int) -> int:

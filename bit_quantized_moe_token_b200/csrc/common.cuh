@@ -56,7 +56,9 @@ inline int launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    if (cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...) == cudaSuccess) return MOE_OK;
+    (void)cudaGetLastError();   // a rejected launch leaves no error behind for later calls
+    return MOE_ERR_CUDA;
 }
 
 // ---- conversions -------------------------------------------------------------------------------
