@@ -161,19 +161,6 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
     const int G = a.K / kGroup;
     const int nst = (G + C::kGS - 1) / C::kGS;             // stages per tile
     const int m_tiles = kSwiGLU ? a.R0 / 64 : a.R0 / 128;
-    // Programmatic dependent launch (common.cuh).  The gate/up instance reads the expert offsets
-    // of the grid just before it, so it waits first.  The down instance's offsets, weights and
-    // scales are older than the grid before it (the requantization), so it reads them and streams
-    // its first weight stages before waiting; only the activations and their scales wait.
-    if constexpr (kSwiGLU) pdl_enter();
-    else pdl_trigger();
-    const int row_tiles = row_tile_prefix(a.offsets, a.E, BN, pre, soff, a.slot_of, a.slot_want);
-    const int64_t n_tiles = (int64_t)row_tiles * m_tiles;
-    if ((int64_t)blockIdx.x >= n_tiles) {
-        pdl_wait();                                        // no CTA completes before its predecessor
-        return;
-    }
-
     if (tid == 0) {
         for (int i = 0; i < C::kRW; ++i) { tc::mbar_init(&w_full[i], 1); tc::mbar_init(&w_empty[i], C::kNW); }
         if (C::kSplitB)
@@ -194,6 +181,23 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem = *tslot;
+    // Programmatic dependent launch (common.cuh): the set-up above ran under the predecessor's
+    // tail.  The gate/up instance reads the expert offsets of the grid just before it, so it
+    // waits now.  The down instance's offsets, weights and scales are older than the grid before
+    // it (the requantization), so it reads them and streams its first weight stages before
+    // waiting; only the activations and their scales wait.
+    if constexpr (kSwiGLU) pdl_enter();
+    else pdl_trigger();
+    const int row_tiles = row_tile_prefix(a.offsets, a.E, BN, pre, soff, a.slot_of, a.slot_want);
+    const int64_t n_tiles = (int64_t)row_tiles * m_tiles;
+    if ((int64_t)blockIdx.x >= n_tiles) {
+        pdl_wait();                                        // no CTA completes before its predecessor
+        if (warp == C::kWarpMma) {
+            tc::tc_fence_after();
+            tc::tmem_dealloc(tmem, C::kTmemCols);
+        }
+        return;
+    }
 
     if (warp == C::kWarpTma) {
         // ------------------------------------------------------------ TMA producer
@@ -217,6 +221,9 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
                     tc::mbar_arrive_expect_tx(&w_full[st], C::kRaw);
                     ws::tma_load_2d(wring + st * C::kRaw, &tm_w0, st * C::kGS * 64, wb * a.R0 + mt * 128, &w_full[st]);
                 }
+                // and the rest of the first tile into L2, where its loads will find it
+                for (int st = pre_w; st < nst; ++st)
+                    ws::tma_prefetch_l2_2d(&tm_w0, st * C::kGS * 64, wb * a.R0 + mt * 128);
             }
             pdl_wait();
         }

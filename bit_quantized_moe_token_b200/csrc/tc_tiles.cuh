@@ -72,21 +72,24 @@ __device__ __forceinline__ int weight_slab(const int32_t* slot_of, int e) {
     return s >= 0 ? s : -s - 1;
 }
 
-// Per-expert prefix of row tiles (ceil(len / BN)) into shared `pre[0..E]`; returns the total.
-// With `soff` non-null the segment offsets [0..E] are copied there too.  With `slot_of`, experts
-// of the other format get no tiles (`want`: kSlotCold or kSlotHot).
-__device__ int row_tile_prefix(const int32_t* __restrict__ offsets, int E, int BN, int* pre,
-                               int* soff = nullptr, const int32_t* slot_of = nullptr,
-                               int want = kSlotAll) {
+// Per-expert prefix of row tiles (ceil(len / BN)) into shared `pre[0..E]` and the segment offsets
+// [0..E] into shared `soff`; returns the total.  Every thread loads its share of the offsets at
+// once (one global round trip), then one warp scans the tile counts in shared memory.  With
+// `slot_of`, experts of the other format get no tiles (`want`: kSlotCold or kSlotHot).
+__device__ int row_tile_prefix(const int32_t* __restrict__ offsets, int E, int BN, int* pre, int* soff,
+                               const int32_t* slot_of = nullptr, int want = kSlotAll) {
     __shared__ int s_total;
+    for (int e = threadIdx.x; e <= E; e += blockDim.x) soff[e] = offsets[e];
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x)
+        pre[e] = slot_kept(slot_of, want, e) ? (soff[e + 1] - soff[e] + BN - 1) / BN : 0;
+    __syncthreads();
     if (threadIdx.x < 32) {
         const int lane = threadIdx.x;
         int run = 0;
         for (int e0 = 0; e0 < E; e0 += 32) {
             const int e = e0 + lane;
-            const int o0 = (e < E) ? offsets[e] : 0, o1 = (e < E) ? offsets[e + 1] : 0;
-            if (soff && e < E) soff[e] = o0;
-            const int n = (e < E && slot_kept(slot_of, want, e)) ? (o1 - o0 + BN - 1) / BN : 0;
+            const int n = e < E ? pre[e] : 0;
             int inc = n;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
@@ -99,7 +102,6 @@ __device__ int row_tile_prefix(const int32_t* __restrict__ offsets, int E, int B
         if (lane == 0) {
             pre[E] = run;
             s_total = run;
-            if (soff) soff[E] = offsets[E];
         }
     }
     __syncthreads();
