@@ -105,6 +105,10 @@ def lib():
         L.or_moe_forward_given_h.argtypes = [ctypes.POINTER(_Layer), vp, vp, i64, i32, vp, vp, vp, vp]
         L.or_moe_forward_given_h.restype = i32
         L.or_moe_forward_dense.restype = i32
+        L.or_expert_rows.argtypes = [ctypes.POINTER(_Layer), vp, vp, vp, i64, vp]
+        L.or_expert_rows.restype = i32
+        L.or_combine.argtypes = [ctypes.POINTER(_Layer), vp, vp, vp, i64, i32, vp]
+        L.or_combine.restype = i32
         L.or_set_threads.argtypes = [i32]
         L.or_set_threads.restype = None
         L.or_max_threads.argtypes = []
@@ -393,6 +397,40 @@ def moe_forward_dense(layer: Layer, x_bf16: np.ndarray, logits: np.ndarray, k: i
     if rc != 0:
         raise ValueError("or_moe_forward_dense: bad shape")
     return r
+
+
+def expert_slice(layer: Layer, e0: int, e1: int) -> Layer:
+    """Experts e0..e1-1 of a W4A8 layer as a layer of their own (no shared experts)."""
+    assert layer.fmt == FMT_W4A8 and 0 <= e0 < e1 <= layer.E
+    return Layer(e1 - e0, layer.H, layer.N, layer.gate_packed[e0:e1], layer.up_packed[e0:e1],
+                 layer.down_packed[e0:e1], layer.gate_scales[e0:e1], layer.up_scales[e0:e1],
+                 layer.down_scales[e0:e1], group=layer.group)
+
+
+def expert_rows(layer: Layer, q: np.ndarray, s_x: np.ndarray, expert: np.ndarray) -> np.ndarray:
+    """S4-S6 for given FP8 rows: q [R,H] E4M3 codes, s_x [R], expert [R] -> y [R,H] fp32."""
+    q = np.ascontiguousarray(q, np.uint8)
+    s = np.ascontiguousarray(s_x, np.float32)
+    e = np.ascontiguousarray(expert, np.int32)
+    R = q.shape[0]
+    y = np.zeros((R, layer.H), np.float32)
+    L = layer._c()
+    if lib().or_expert_rows(ctypes.byref(L), _p(q), _p(s), _p(e), R, _p(y)) != 0:
+        raise ValueError("or_expert_rows: bad shape or expert index")
+    return y
+
+
+def combine(layer: Layer, x_bf16: np.ndarray, gates: np.ndarray, y_pairs: np.ndarray, k: int) -> np.ndarray:
+    """S7 (+ S8) alone: bf16 out [T,H] from routed rows y_pairs [T*k, H] in pair order."""
+    x = np.ascontiguousarray(x_bf16, np.uint16)
+    g = np.ascontiguousarray(gates, np.float32)
+    y = np.ascontiguousarray(y_pairs, np.float32)
+    T = g.shape[0]
+    out = np.zeros((T, layer.H), np.uint16)
+    L = layer._c()
+    if lib().or_combine(ctypes.byref(L), _p(x), _p(g), _p(y), T, k, _p(out)) != 0:
+        raise ValueError("or_combine: bad shape")
+    return out
 
 
 def _each_expert(fn, experts):

@@ -544,6 +544,87 @@ static void shared_expert_add(const float* x, const uint16_t* wg, const uint16_t
 }
 
 /*
+ * S4..S6 for n routed rows of expert e: row i reads the FP8 codes q[i] (H of them) with scale
+ * s_x[i], writes its requantized SwiGLU activations to hq[i N ..] / s_h[i] and its
+ * down-projection output to y[i][0 .. H).  With given_h, hq / s_h are inputs.
+ */
+static void expert_segment(const or_layer* L, int64_t e, int64_t n, const uint8_t* const* q,
+                           const float* s_x, uint8_t* hq, float* s_h, float* const* y, int given_h) {
+    const int64_t H = L->H, N = L->N;
+    const int group = L->group;
+    const int64_t G_h = H / group, G_n = N / group;
+    float* cg = (float*)malloc((size_t)N * H * 4);
+    float* cu = (float*)malloc((size_t)N * H * 4);
+    float* cd = (float*)malloc((size_t)H * N * 4);
+    float* scratch = (float*)malloc((size_t)(3 * N + 2 * (H > N ? H : N)) * 4);
+    int64_t b;                           /* the expert's slab in its format's arrays */
+    const int f = expert_fmt(L, e, &b);
+    if (f == 1) {
+        w8_T(L->gate_w8 + b * N * H, N, H, cg);
+        w8_T(L->up_w8 + b * N * H, N, H, cu);
+        w8_T(L->down_w8 + b * H * N, H, N, cd);
+    } else if (f == 2) {
+        f4_T(L->gate_f4 + b * N * (H / 2), L->gate_bs + b * N * (H / 16), L->gate_s2[b], N, H, cg);
+        f4_T(L->up_f4 + b * N * (H / 2), L->up_bs + b * N * (H / 16), L->up_s2[b], N, H, cu);
+        f4_T(L->down_f4 + b * H * (N / 2), L->down_bs + b * H * (N / 16), L->down_s2[b], H, N, cd);
+    } else {
+        codes_T(L->gate_packed + b * N * (H / 8), N, H, cg);
+        codes_T(L->up_packed + b * N * (H / 8), N, H, cu);
+        codes_T(L->down_packed + b * H * (N / 8), H, N, cd);
+    }
+    for (int64_t i = 0; i < n; ++i) {
+        if (f == 1)
+            expert_row_w8(q[i], s_x[i], cg, cu, cd, L->gate_rs + b * N, L->up_rs + b * N,
+                          L->down_rs + b * H, H, N, hq + i * N, s_h + i, y[i], scratch, given_h);
+        else if (f == 2)
+            expert_row_f4(q[i], s_x[i], cg, cu, cd, H, N, hq + i * N, s_h + i, y[i], scratch,
+                          given_h);
+        else
+            expert_row(q[i], s_x[i], cg, cu, cd, L->gate_scales + b * N * G_h,
+                       L->up_scales + b * N * G_h, L->down_scales + b * H * G_n, H, N, group,
+                       hq + i * N, s_h + i, y[i], scratch, given_h);
+    }
+    free(cg); free(cu); free(cd); free(scratch);
+}
+
+/*
+ * S7 (+ S8) for token t: out[t] = bf16( sum_j gate_j * y_j  +  sum_s shared_s(x_t) ), j in
+ * selection order, y_j = yr[j] the output row of the token's j-th routed pair, accumulated in
+ * fp32 in that order; the shared experts' sum is added last.
+ */
+static void combine_token(const or_layer* L, const uint16_t* x, int64_t t, int k,
+                          const float* gates_t, const float* const* yr, uint16_t* out,
+                          float* out_f32) {
+    const int64_t H = L->H;
+    float* o = (float*)malloc((size_t)H * 4);
+    for (int64_t m = 0; m < H; ++m) o[m] = 0.0f;
+    for (int j = 0; j < k; ++j) {
+        float gj = gates_t[j];
+        for (int64_t m = 0; m < H; ++m) o[m] += gj * yr[j][m];
+    }
+    if (L->n_shared > 0) {
+        int64_t Ns = L->shared_N;
+        float* xf = (float*)malloc((size_t)H * 4);
+        float* ys = (float*)malloc((size_t)H * 4);
+        float* a = (float*)malloc((size_t)Ns * 4);
+        float* shsum = (float*)calloc((size_t)H, 4);
+        for (int64_t i = 0; i < H; ++i) xf[i] = or_bf16_to_f32(x[t * H + i]);
+        for (int s = 0; s < L->n_shared; ++s) {
+            shared_expert_add(xf, L->sh_gate + s * Ns * H, L->sh_up + s * Ns * H,
+                              L->sh_down + s * H * Ns, H, Ns, ys, a);
+            for (int64_t m = 0; m < H; ++m) shsum[m] += ys[m];
+        }
+        for (int64_t m = 0; m < H; ++m) o[m] += shsum[m];
+        free(xf); free(ys); free(a); free(shsum);
+    }
+    for (int64_t m = 0; m < H; ++m) {
+        out[t * H + m] = or_f32_to_bf16(o[m]);
+        if (out_f32) out_f32[t * H + m] = o[m];
+    }
+    free(o);
+}
+
+/*
  * The layer.  x bf16 [T,H], logits fp32 [T,E] -> out bf16 [T,H].
  * Optional intermediates (NULL to skip), all in expert-sorted row order r:
  *   ids/gates [T,k], offsets [E+1], sorted_pairs/row_of_pair [P], xq [T,H], s_x [T],
@@ -577,6 +658,61 @@ int or_moe_forward_given_h(const or_layer* L, const uint16_t* x, const float* lo
     if (!hq_pairs || !sh_pairs) return -1;
     return moe_forward_impl(L, x, logits, T, k, out, NULL, NULL, NULL, NULL, NULL, NULL, NULL,
                             NULL, NULL, NULL, out_f32_o, hq_pairs, sh_pairs);
+}
+
+/*
+ * Expert parallelism, receive side: S4..S6 for R routed rows given as FP8 codes q [R,H] with
+ * scales s_x [R] and experts expert [R] (indices into L) -> y [R,H] fp32.  The per-row
+ * arithmetic of the layer (each expert is independent of the others), rows taken expert by
+ * expert in increasing row order.  Returns -1 on a bad shape or an expert outside [0, E).
+ */
+int or_expert_rows(const or_layer* L, const uint8_t* q, const float* s_x, const int32_t* expert,
+                   int64_t R, float* y) {
+    const int64_t H = L->H, N = L->N, E = L->E;
+    if (H % L->group || N % L->group) return -1;
+    for (int64_t i = 0; i < R; ++i)
+        if (expert[i] < 0 || expert[i] >= E) return -1;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t e = 0; e < E; ++e) {
+        int64_t n = 0;
+        for (int64_t i = 0; i < R; ++i) n += expert[i] == e;
+        if (n == 0) continue;
+        const uint8_t** qr = (const uint8_t**)malloc((size_t)n * sizeof(void*));
+        float* sr = (float*)malloc((size_t)n * 4);
+        float** yr = (float**)malloc((size_t)n * sizeof(void*));
+        uint8_t* hq = (uint8_t*)malloc((size_t)n * N);
+        float* sh = (float*)malloc((size_t)n * 4);
+        int64_t c = 0;
+        for (int64_t i = 0; i < R; ++i) {
+            if (expert[i] != e) continue;
+            qr[c] = q + i * H;
+            sr[c] = s_x[i];
+            yr[c] = y + i * H;
+            ++c;
+        }
+        expert_segment(L, e, n, qr, sr, hq, sh, yr, 0);
+        free(qr); free(sr); free(yr); free(hq); free(sh);
+    }
+    return 0;
+}
+
+/*
+ * S7 (+ S8) alone: out bf16 [T,H] from the routed rows y_pairs [T*k, H] fp32 in pair order
+ * p = t*k + j, the gates [T,k] and (for the shared experts) x bf16 [T,H].  Same arithmetic as
+ * the layer's combine.
+ */
+int or_combine(const or_layer* L, const uint16_t* x, const float* gates, const float* y_pairs,
+               int64_t T, int k, uint16_t* out) {
+    if (k < 1) return -1;
+    const int64_t H = L->H;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t t = 0; t < T; ++t) {
+        const float** yr = (const float**)malloc((size_t)k * sizeof(void*));
+        for (int j = 0; j < k; ++j) yr[j] = y_pairs + (t * k + j) * H;
+        combine_token(L, x, t, k, gates + t * k, yr, out, NULL);
+        free(yr);
+    }
+    return 0;
 }
 
 static int moe_forward_impl(const or_layer* L, const uint16_t* x, const float* logits, int64_t T,
@@ -618,77 +754,30 @@ static int moe_forward_impl(const or_layer* L, const uint16_t* x, const float* l
     }
 
     /* S4..S6, one expert segment at a time (experts are independent) */
-    const int64_t G_h = H / group, G_n = N / group;
 #pragma omp parallel for schedule(dynamic, 1)
     for (int64_t e = 0; e < E; ++e) {
         int32_t r0 = offsets[e], r1 = offsets[e + 1];
         if (r0 == r1) continue;
-        float* cg = (float*)malloc((size_t)N * H * 4);
-        float* cu = (float*)malloc((size_t)N * H * 4);
-        float* cd = (float*)malloc((size_t)H * N * 4);
-        float* scratch = (float*)malloc((size_t)(3 * N + 2 * (H > N ? H : N)) * 4);
-        int64_t b;                       /* the expert's slab in its format's arrays */
-        const int f = expert_fmt(L, e, &b);
-        if (f == 1) {
-            w8_T(L->gate_w8 + b * N * H, N, H, cg);
-            w8_T(L->up_w8 + b * N * H, N, H, cu);
-            w8_T(L->down_w8 + b * H * N, H, N, cd);
-        } else if (f == 2) {
-            f4_T(L->gate_f4 + b * N * (H / 2), L->gate_bs + b * N * (H / 16), L->gate_s2[b], N, H, cg);
-            f4_T(L->up_f4 + b * N * (H / 2), L->up_bs + b * N * (H / 16), L->up_s2[b], N, H, cu);
-            f4_T(L->down_f4 + b * H * (N / 2), L->down_bs + b * H * (N / 16), L->down_s2[b], H, N, cd);
-        } else {
-            codes_T(L->gate_packed + b * N * (H / 8), N, H, cg);
-            codes_T(L->up_packed + b * N * (H / 8), N, H, cu);
-            codes_T(L->down_packed + b * H * (N / 8), H, N, cd);
-        }
+        const uint8_t** qr = (const uint8_t**)malloc((size_t)(r1 - r0) * sizeof(void*));
+        float* sr = (float*)malloc((size_t)(r1 - r0) * 4);
+        float** yr = (float**)malloc((size_t)(r1 - r0) * sizeof(void*));
         for (int32_t r = r0; r < r1; ++r) {
             int64_t t = sorted[r] / k;
-            if (f == 1)
-                expert_row_w8(xq + t * H, sx[t], cg, cu, cd, L->gate_rs + b * N, L->up_rs + b * N,
-                              L->down_rs + b * H, H, N, hq + (int64_t)r * N, sh + r,
-                              y + (int64_t)r * H, scratch, given_h);
-            else if (f == 2)
-                expert_row_f4(xq + t * H, sx[t], cg, cu, cd, H, N, hq + (int64_t)r * N, sh + r,
-                              y + (int64_t)r * H, scratch, given_h);
-            else
-                expert_row(xq + t * H, sx[t], cg, cu, cd, L->gate_scales + b * N * G_h,
-                           L->up_scales + b * N * G_h, L->down_scales + b * H * G_n, H, N, group,
-                           hq + (int64_t)r * N, sh + r, y + (int64_t)r * H, scratch, given_h);
+            qr[r - r0] = xq + t * H;
+            sr[r - r0] = sx[t];
+            yr[r - r0] = y + (int64_t)r * H;
         }
-        free(cg); free(cu); free(cd); free(scratch);
+        expert_segment(L, e, r1 - r0, qr, sr, hq + (int64_t)r0 * N, sh + r0, yr, given_h);
+        free(qr); free(sr); free(yr);
     }
 
-    /* S7 (+ S8): out[t] = bf16( sum_j gate_j * y[row(t,j)]  +  sum_s shared_s(x_t) ) */
+    /* S7 (+ S8) */
 #pragma omp parallel for schedule(dynamic, 1)
     for (int64_t t = 0; t < T; ++t) {
-        float* o = (float*)malloc((size_t)H * 4);
-        for (int64_t m = 0; m < H; ++m) o[m] = 0.0f;
-        for (int j = 0; j < k; ++j) {
-            float gj = gates[t * k + j];
-            const float* yr = y + (int64_t)rop[t * k + j] * H;
-            for (int64_t m = 0; m < H; ++m) o[m] += gj * yr[m];
-        }
-        if (L->n_shared > 0) {
-            int64_t Ns = L->shared_N;
-            float* xf = (float*)malloc((size_t)H * 4);
-            float* ys = (float*)malloc((size_t)H * 4);
-            float* a = (float*)malloc((size_t)Ns * 4);
-            float* shsum = (float*)calloc((size_t)H, 4);
-            for (int64_t i = 0; i < H; ++i) xf[i] = or_bf16_to_f32(x[t * H + i]);
-            for (int s = 0; s < L->n_shared; ++s) {
-                shared_expert_add(xf, L->sh_gate + s * Ns * H, L->sh_up + s * Ns * H,
-                                  L->sh_down + s * H * Ns, H, Ns, ys, a);
-                for (int64_t m = 0; m < H; ++m) shsum[m] += ys[m];
-            }
-            for (int64_t m = 0; m < H; ++m) o[m] += shsum[m];
-            free(xf); free(ys); free(a); free(shsum);
-        }
-        for (int64_t m = 0; m < H; ++m) {
-            out[t * H + m] = or_f32_to_bf16(o[m]);
-            if (out_f32_o) out_f32_o[t * H + m] = o[m];
-        }
-        free(o);
+        const float** yr = (const float**)malloc((size_t)k * sizeof(void*));
+        for (int j = 0; j < k; ++j) yr[j] = y + (int64_t)rop[t * k + j] * H;
+        combine_token(L, x, t, k, gates + t * k, yr, out, out_f32_o);
+        free(yr);
     }
 
     if (ids_o) memcpy(ids_o, ids, (size_t)P * 4);

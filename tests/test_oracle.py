@@ -346,6 +346,50 @@ def test_layer_dense_brute_force_matches_permuted():
         assert np.array_equal(r["y"][row], d["y"][t, e])
 
 
+def test_expert_rows_match_dense_brute_force():
+    """The expert-parallel receive step (S4-S6 on given FP8 rows) against the dense brute force,
+    which runs every (token, expert) pair without any permutation: any (token, expert), routed
+    or not, in any row order, and through a slice of the experts."""
+    wl = synth.WORKLOADS["tiny"]
+    layer = _tiny_layer(wl)
+    x, lg = synth.tokens(wl), synth.logits(wl)
+    d = oracle.moe_forward_dense(layer, x, lg, wl.k)
+    xq, sx = oracle.quant_tokens(x)
+    rng = np.random.default_rng(5)
+    t = rng.integers(0, wl.T, 40)
+    e = rng.integers(0, wl.E, 40)
+    y = oracle.expert_rows(layer, xq[t], sx[t], e)
+    for i in range(40):
+        assert np.array_equal(y[i], d["y"][t[i], e[i]]), i
+    e0, e1 = 2, 6
+    sel = (e >= e0) & (e < e1)
+    ys = oracle.expert_rows(oracle.expert_slice(layer, e0, e1), xq[t[sel]], sx[t[sel]], e[sel] - e0)
+    assert np.array_equal(ys, y[sel])
+    with pytest.raises(ValueError):
+        oracle.expert_rows(layer, xq[:1], sx[:1], np.array([wl.E]))
+
+
+def test_combine_closed_form_and_forward_decomposition():
+    """S7 alone: constant rows give bf16(sum_j g_j c_j); and the layer's own routed rows, gates
+    and shared experts put back together give the layer's output bit for bit."""
+    T, H, N, E, k = 3, 128, 128, 4, 2
+    z = np.zeros((E, N, H // 8), np.int32)
+    layer = oracle.Layer(E, H, N, z, z, np.zeros((E, H, N // 8), np.int32),
+                         np.zeros((E, N, 1), np.uint16), np.zeros((E, N, 1), np.uint16),
+                         np.zeros((E, H, 1), np.uint16))
+    gates = np.array([[0.25, 0.75], [0.5, 0.5], [1.0, 0.0]], np.float32)
+    c = np.array([[3.0, -1.5], [1.0, 2.0], [-7.0, 100.0]], np.float32)
+    y = np.repeat(c.reshape(T * k, 1), H, axis=1).astype(np.float32)
+    out = oracle.bf16_to_f32(oracle.combine(layer, np.zeros((T, H), np.uint16), gates, y, k))
+    for t, want in enumerate((-0.375, 1.5, -7.0)):
+        assert np.all(out[t] == want), (t, out[t, :2])
+    wl = synth.WORKLOADS["tiny"]
+    full = oracle.pack_workload_layer(wl)
+    x, lg = synth.tokens(wl), synth.logits(wl)
+    r = oracle.moe_forward(full, x, lg, wl.k)
+    assert np.array_equal(oracle.combine(full, x, r["gates"], r["y"][r["row_of_pair"]], wl.k), r["out"])
+
+
 def test_layer_constant_closed_form():
     want = {}
     for line in golden_lines("constant_layer.txt"):
