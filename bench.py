@@ -43,6 +43,7 @@ DEFAULT_WORKLOAD = HEADLINE
 # the other configs of the benchmark, reported under "workloads" (the tiny config is parity-only)
 EXTRA_WORKLOADS = ("decode_t8", "decode_t64", "prefill_t2048_zipf")
 MIN_TIMED_MS = 200.0
+EP_WORKLOADS = ("decode_t8", "decode_t64", "prefill_t2048_zipf")   # timed on the expert-parallel path too
 N_BATCHES = 8
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_HBM_GBS = 6650.0
@@ -577,6 +578,42 @@ def router_timing(fx, wl, layer, batches, out, ws, steps, dev, stream, world, hb
                         "given (e.g. Zipf) logits"}}
 
 
+def ep_timing(fx, wl, steps, warmup, dev, stream, world, fused_ms):
+    """The expert-parallel path (bit_quantized_moe_token_b200/ep.py) on this workload: experts split
+    over the `world` ranks, each rank's own tokens dispatched to the owners and combined back.  With
+    one rank the exchanges are skipped and what is timed is the path's own cost (records packed and
+    unpacked, output rows put back in record order, the host read of the counts) against the fused
+    forward's `fused_ms`."""
+    import torch
+    from bit_quantized_moe_token_b200.ep import EpLayer, local_experts
+    layer = fx.layer_for(wl)
+    rank = torch.distributed.get_rank() if world > 1 else 0
+    ep = EpLayer(layer, local_experts(layer, rank, world))
+    batches = [synth_batch(wl, rank, b, dev) for b in range(N_BATCHES)]
+    out = torch.empty(wl.T, wl.H, dtype=torch.bfloat16, device=dev)
+    for i in range(max(warmup, 3)):
+        x, lg = batches[i % N_BATCHES]
+        ep.forward(x, lg, wl.k, out=out)
+    n = max(steps, 20)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for i in range(n):
+        x, lg = batches[i % N_BATCHES]
+        ep.forward(x, lg, wl.k, out=out)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if fx.moe.moe_last_device_status() != 0:
+        raise RuntimeError("device status: error in the expert-parallel path")
+    ms = max_over_ranks(e0.elapsed_time(e1) / n, dev, world)
+    return {"n_ranks": world, "steps": n, "ms_per_step": round(ms, 4),
+            "value": round(whole_job_rate(world, wl.T, n, ms * n), 1), "unit": "tokens/s",
+            "fused_forward_ms_per_step": round(fused_ms, 4),
+            "records_per_step": world * wl.T * wl.k}
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -607,6 +644,16 @@ def run_ours(args):
             extra[name] = measure(fx, xw, args.steps, args.warmup, dev, stream, clk, rank, world,
                                   min_timed_ms=MIN_TIMED_MS)
             del extra[name]["config"]["parallelism"]
+    ep = {}
+    if args.experts == "w4a8" and (world == 1 or args.ep):
+        # the expert-parallel path on the decode and mid-size configs (one rank: the exchanges
+        # are skipped; several ranks only on request, since they run NCCL all-to-all exchanges)
+        for name in EP_WORKLOADS:
+            ref = head if name == wl.name else extra.get(name)
+            if ref is None:
+                continue
+            ep[name] = ep_timing(fx, synth.WORKLOADS[name], args.steps, args.warmup, dev, stream, world,
+                                 ref["ms_per_step"])
     clk.stop()
     result = {
         "metric": METRIC, "value": head["value"], "unit": "tokens/s", "n_gpus": world,
@@ -622,6 +669,8 @@ def run_ours(args):
         result["workloads"] = extra
         result["workloads_note"] = (f"the other configs on the same layer (shared experts left out), "
                                     f"each timed over >= {MIN_TIMED_MS:.0f} ms of steps")
+    if ep:
+        result["expert_parallel"] = ep
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(wl, fmt=args.experts)
     if world > 1:
@@ -759,6 +808,8 @@ def main():
     ap.add_argument("--no-extra", action="store_true",
                     help="time only --workload (not the other configs under \"workloads\")")
     ap.add_argument("--no-router", action="store_true", help="skip the router timings")
+    ap.add_argument("--ep", action="store_true",
+                    help="with several ranks, also time the expert-parallel path (NCCL all-to-all)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -16,7 +16,9 @@ from ._binding import (MOE_OK, Layer, MoeError, fp8_quant_tokens, layer_struct, 
                        nvfp4_quant_weights, moe_nvfp4_workspace_bytes, moe_nvfp4_workspace_layout,
                        moe_nvfp4_forward, moe_nvfp4_forward_profiled, moe_nvfp4_forward_router,
                        LayerH, moe_hybrid_workspace_bytes, moe_hybrid_workspace_layout,
-                       moe_hybrid_forward, moe_hybrid_forward_profiled)
+                       moe_hybrid_forward, moe_hybrid_forward_profiled, ep_record_bytes,
+                       moe_ep_dispatch_workspace_bytes, moe_ep_dispatch, moe_ep_experts_workspace_bytes,
+                       moe_ep_experts_forward, moe_ep_combine)
 from .layer import (alloc_workspace, forward, hybrid_from, make_layer, make_layer_nvfp4, make_layer_w8a8,
                     pack_expert_weights, quant_expert_weights_nvfp4, quant_expert_weights_w8a8)
 
@@ -35,4 +37,6 @@ __all__ = ["MOE_OK", "Layer", "MoeError", "fp8_quant_tokens", "layer_struct", "l
            "moe_nvfp4_workspace_layout", "moe_nvfp4_forward", "moe_nvfp4_forward_profiled",
            "make_layer_nvfp4", "quant_expert_weights_nvfp4", "moe_nvfp4_forward_router",
            "LayerH", "moe_hybrid_workspace_bytes", "moe_hybrid_workspace_layout", "moe_hybrid_forward",
-           "moe_hybrid_forward_profiled", "hybrid_from"]
+           "moe_hybrid_forward_profiled", "hybrid_from", "ep_record_bytes",
+           "moe_ep_dispatch_workspace_bytes", "moe_ep_dispatch", "moe_ep_experts_workspace_bytes",
+           "moe_ep_experts_forward", "moe_ep_combine"]

@@ -138,13 +138,21 @@ def lib() -> ctypes.CDLL:
         L.moe_w4a8_forward_router.argtypes = [ctypes.POINTER(_CLayer), vp, vp, i64, i32, vp, vp, sz, vp]
         L.moe_w8a8_forward_router.argtypes = [ctypes.POINTER(_CLayer8), vp, vp, i64, i32, vp, vp, sz, vp]
         L.moe_nvfp4_forward_router.argtypes = [ctypes.POINTER(_CLayer4), vp, vp, i64, i32, vp, vp, sz, vp]
+        L.moe_ep_dispatch_workspace_bytes.argtypes = [ctypes.POINTER(_CLayer), i64, i32]
+        L.moe_ep_dispatch_workspace_bytes.restype = sz
+        L.moe_ep_dispatch.argtypes = [ctypes.POINTER(_CLayer), vp, vp, i64, i32, i32, vp, vp, vp, sz, vp]
+        L.moe_ep_experts_workspace_bytes.argtypes = [ctypes.POINTER(_CLayer), i64]
+        L.moe_ep_experts_workspace_bytes.restype = sz
+        L.moe_ep_experts_forward.argtypes = [ctypes.POINTER(_CLayer), vp, i64, vp, vp, sz, vp]
+        L.moe_ep_combine.argtypes = [ctypes.POINTER(_CLayer), vp, vp, i64, i32, vp, vp, sz, vp]
         L.moe_last_device_status.argtypes = [vp]
         L.moe_selftest_bounded_wait.argtypes = [i64, vp]
         L.moe_status_string.argtypes = [i32]
         L.moe_status_string.restype = ctypes.c_char_p
         for f in (L.w4a8_pack_weights, L.fp8_quant_tokens, L.moe_route_topk, L.moe_router_logits,
                   L.moe_w4a8_workspace_layout, L.moe_w4a8_forward, L.moe_w4a8_forward_profiled,
-                  L.moe_last_device_status, L.moe_selftest_bounded_wait):
+                  L.moe_last_device_status, L.moe_selftest_bounded_wait, L.moe_ep_dispatch,
+                  L.moe_ep_experts_forward, L.moe_ep_combine):
             f.restype = i32
         _lib = L
     return _lib
@@ -317,6 +325,58 @@ def moe_w4a8_forward_profiled(layer: Layer, x, logits, k: int, out, ws, events, 
                                            _ptr(ws), nbytes, _stream(stream), arr, len(events),
                                            ctypes.byref(n)), "moe_w4a8_forward_profiled")
     return int(n.value)
+
+
+# ---- expert parallelism ---------------------------------------------------------------------
+
+def ep_record_bytes(H: int) -> int:
+    """Bytes of one dispatch record (MOE_EP_RECORD_BYTES): H FP8 codes, scale, expert, padding."""
+    return int(H) + 16
+
+
+def _shape_or_struct(layer) -> _CLayer:
+    return layer if isinstance(layer, _CLayer) else layer.c_struct()
+
+
+def moe_ep_dispatch_workspace_bytes(layer, T: int, k: int) -> int:
+    s = layer if isinstance(layer, _CLayer) else layer.shape_struct()
+    return int(lib().moe_ep_dispatch_workspace_bytes(ctypes.byref(s), T, k))
+
+
+def moe_ep_dispatch(layer, x, logits, k: int, n_ranks: int, send_counts, send_records, ws,
+                    stream=None) -> None:
+    """x bf16 [T, H], logits fp32 [T, E] -> send_counts int32 [n_ranks], send_records uint8
+    [T*k, ep_record_bytes(H)] (owner-major); ws keeps what moe_ep_combine needs."""
+    T = x.shape[0]
+    s = _shape_or_struct(layer)
+    nbytes = ws.numel() * ws.element_size() if ws is not None else 0
+    _check(lib().moe_ep_dispatch(ctypes.byref(s), _ptr(x), _ptr(logits), T, k, n_ranks,
+                                 _ptr(send_counts), _ptr(send_records), _ptr(ws), nbytes,
+                                 _stream(stream)), "moe_ep_dispatch")
+
+
+def moe_ep_experts_workspace_bytes(local_layer, R: int) -> int:
+    s = local_layer if isinstance(local_layer, _CLayer) else local_layer.shape_struct()
+    return int(lib().moe_ep_experts_workspace_bytes(ctypes.byref(s), R))
+
+
+def moe_ep_experts_forward(local_layer: Layer, records, y_rows, ws, stream=None) -> None:
+    """records uint8 [R, ep_record_bytes(H)] received for this GPU's experts -> y_rows fp32 [R, H]."""
+    R = records.shape[0]
+    s = local_layer.c_struct()
+    nbytes = ws.numel() * ws.element_size() if ws is not None else 0
+    _check(lib().moe_ep_experts_forward(ctypes.byref(s), _ptr(records) if R else None, R,
+                                        _ptr(y_rows) if R else None, _ptr(ws), nbytes,
+                                        _stream(stream)), "moe_ep_experts_forward")
+
+
+def moe_ep_combine(layer, x, y_back, k: int, out, ws, stream=None) -> None:
+    """y_back fp32 [T*k, H] (rows returned for this GPU's records, record order) -> out bf16 [T, H]."""
+    T = x.shape[0]
+    s = _shape_or_struct(layer)
+    nbytes = ws.numel() * ws.element_size() if ws is not None else 0
+    _check(lib().moe_ep_combine(ctypes.byref(s), _ptr(x), _ptr(y_back), T, k, _ptr(out), _ptr(ws),
+                                nbytes, _stream(stream)), "moe_ep_combine")
 
 
 def moe_last_device_status(stream=None) -> int:

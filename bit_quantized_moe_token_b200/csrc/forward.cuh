@@ -313,6 +313,139 @@ extern "C" int moe_w4a8_forward_profiled(const moe_w4a8_layer* layer, const uint
     return st;
 }
 
+namespace moe {
+// S8: the shared experts, summed = one SwiGLU MLP of width n_shared * shared_N, into y fp32
+// [T, H] through sa (bf16 [T, 2 n_shared shared_N]); *shared = y, or null for a layer without
+// shared experts.
+inline int run_shared(const moe_w4a8_layer& L, uint16_t* sa, float* y, const uint16_t* x_bf16,
+                      int64_t T, cudaStream_t stream, StageMarks& sm, float** shared) {
+    *shared = nullptr;
+    if (L.n_shared <= 0) return MOE_OK;
+    const int Wsh = L.n_shared * L.shared_N;
+    // the SwiGLU activation as bf16 hi and lo halves [T, 2 Wsh]; the down GEMM reduces over both
+    Bf16GemmArgs g{Wsh, (int)T, L.H, 0, sa, 2 * Wsh, 0};
+    int st = launch_gemm_bf16_ws<true>(g, x_bf16, L.sh_gate, L.sh_up, stream);
+    if (st) return st;
+    Bf16GemmArgs d{L.H, (int)T, 2 * Wsh, L.shared_N, y, L.H, Wsh};
+    if ((st = launch_gemm_bf16_ws<false>(d, sa, L.sh_down, nullptr, stream))) return st;
+    sm.launches += 2;
+    *shared = y;
+    return MOE_OK;
+}
+
+// Where S4's routed rows are: narrow tiles (gather) read the per-token codes xq / sx (token =
+// pair / k) and, for the W4A8 unsigned widening, the group sums qs_x; wide tiles read the
+// expert-sorted copies xs / sxs.
+struct RoutedRows {
+    const int32_t *offsets, *sorted;
+    int64_t P, T;
+    int k;
+    bool gather, act_perm;
+    const uint8_t* xq;
+    const float* sx;
+    const uint8_t* xs;
+    const float* sxs;
+    float* qs_x;
+};
+
+// S4-S6 on routed rows: gate/up GEMM with the SwiGLU epilogue (h, max|h| per row), the
+// requantization, and the down GEMM into the workspace's y [P, H] fp32, expert-sorted rows.
+inline int run_experts(const moe_w4a8_layer& L, const ExpertSet& xw, const WsPlan& p, char* w,
+                       const RoutedRows& rr, const int32_t* slot_of, cudaStream_t stream, StageMarks& sm) {
+    auto at = [&](size_t off) { return static_cast<void*>(w + off); };
+    const int32_t* offsets = rr.offsets;
+    const int32_t* sorted = rr.sorted;
+    const int64_t P = rr.P, T = rr.T;
+    const int k = rr.k;
+    const bool gather = rr.gather, act_perm = rr.act_perm;
+    const uint8_t *xq = rr.xq, *xs = rr.xs;
+    const float *sx = rr.sx, *sxs = rr.sxs;
+    float* qs_x = rr.qs_x;
+    float* h = (float*)at(p.h);
+    unsigned* amax = (unsigned*)at(p.zero);
+    uint8_t* hq = (uint8_t*)at(p.hq);
+    float* sh = (float*)at(p.s_h);
+    float* y = (float*)at(p.y);
+    float* qs_h = (float*)at(p.qs_h);
+    uint16_t* act16 = xw.fmt >= kFmtNvfp4 ? (uint16_t*)at(p.act16) : nullptr;
+    const bool hybrid = xw.fmt == kFmtHybrid;
+    // the two launches of a hybrid layer's GEMM: W4A8 on the cold experts, NVFP4 on the hot ones
+    const bool run_w4 = xw.fmt == kFmtW4A8 || (hybrid && xw.n_cold > 0);
+    const bool run_f4 = xw.fmt == kFmtNvfp4 || (hybrid && xw.n_hot > 0);
+    const void* f4_gate = hybrid ? xw.h_gate : xw.gate;
+    const void* f4_up = hybrid ? xw.h_up : xw.up;
+    const void* f4_down = hybrid ? xw.h_down : xw.down;
+    const uint8_t* f4_gs = (const uint8_t*)(hybrid ? xw.h_gate_s : xw.gate_s);
+    const uint8_t* f4_us = (const uint8_t*)(hybrid ? xw.h_up_s : xw.up_s);
+    const uint8_t* f4_ds = (const uint8_t*)(hybrid ? xw.h_down_s : xw.down_s);
+    const float* f4_g2 = hybrid ? xw.h_gate_s2 : xw.gate_s2;
+    const float* f4_u2 = hybrid ? xw.h_up_s2 : xw.up_s2;
+    const float* f4_d2 = hybrid ? xw.h_down_s2 : xw.down_s2;
+    int st = MOE_OK;
+    // S4 + SwiGLU: h = silu(G) * U, max|h| per row
+    if (run_f4) {
+        // f16 copy of the FP8 activations (exact), then the f16 tensor-core GEMM
+        // (in a narrow hybrid layer the per-token codes are in the W4A8 tiles' K order)
+        if ((st = launch_e4m3_to_f16(gather ? xq : xs, (gather ? T : P) * L.H, act16, stream, act_perm)))
+            return st;
+        F4GemmArgs f{W8GemmArgs{gather ? sx : sxs, nullptr, nullptr, offsets, L.E, L.N, L.H, (int)P, h, L.N,
+                                amax, sorted, k, (int)T},
+                     f4_gs, f4_us, f4_g2, f4_u2, slot_of, hybrid ? kSlotHot : kSlotAll};
+        if ((st = launch_gemm_nvfp4<true>(f, act16, f4_gate, f4_up, stream))) return st;
+        sm.launches += 2;
+    }
+    if (xw.fmt == kFmtW8A8) {
+        W8GemmArgs a{gather ? sx : sxs, (const float*)xw.gate_s, (const float*)xw.up_s, offsets, L.E, L.N,
+                     L.H, (int)P, h, L.N, amax, sorted, k, (int)T};
+        if ((st = launch_gemm_w8a8<true>(a, gather ? (const void*)xq : (const void*)xs, xw.gate, xw.up,
+                                         stream)))
+            return st;
+        sm.launches += 1;
+    } else if (run_w4) {
+        WsGemmArgs a{gather ? sx : sxs, (const uint16_t*)xw.gate_s, (const uint16_t*)xw.up_s, offsets, L.E,
+                     L.N, L.H, (int)P, h, L.N, amax, sorted, k, (int)T, gather ? qs_x : nullptr, slot_of,
+                     hybrid ? kSlotCold : kSlotAll};
+        if ((st = launch_gemm_ws<true>(a, gather ? (const void*)xq : (const void*)xs, xw.gate, xw.up,
+                                       stream)))
+            return st;
+        sm.launches += 1;
+    }
+    sm.mark(4, stream);
+    // S5
+    // the W4A8 down GEMM widens its narrow tiles unsigned and needs the requantized rows' group sums;
+    // hq, like xq, is stored in those tiles' K order whenever a W4A8 or hybrid layer runs narrow
+    const bool down_sums = run_w4 && gather;
+    if ((st = launch_pdl(k_requant, dim3(static_cast<unsigned>(P)), dim3(256), 0, stream, h, L.N, amax, hq, sh,
+                         down_sums ? qs_h : nullptr, act_perm)))
+        return st;
+    sm.launches += 1;
+    sm.mark(5, stream);
+    // S6
+    if (run_f4) {
+        if ((st = launch_e4m3_to_f16(hq, P * L.N, act16, stream, act_perm))) return st;
+        F4GemmArgs f{W8GemmArgs{sh, nullptr, nullptr, offsets, L.E, L.H, L.N, (int)P, y, L.H, nullptr, sorted,
+                                k, (int)T},
+                     f4_ds, nullptr, f4_d2, nullptr, slot_of, hybrid ? kSlotHot : kSlotAll};
+        if ((st = launch_gemm_nvfp4<false>(f, act16, f4_down, nullptr, stream))) return st;
+        sm.launches += 2;
+    }
+    if (xw.fmt == kFmtW8A8) {
+        W8GemmArgs a{sh, (const float*)xw.down_s, nullptr, offsets, L.E, L.H, L.N, (int)P, y, L.H, nullptr,
+                     sorted, k, (int)T};
+        if ((st = launch_gemm_w8a8<false>(a, hq, xw.down, nullptr, stream))) return st;
+        sm.launches += 1;
+    } else if (run_w4) {
+        WsGemmArgs a{sh, (const uint16_t*)xw.down_s, nullptr, offsets, L.E, L.H, L.N, (int)P, y, L.H,
+                     nullptr, sorted, k, (int)T, down_sums ? qs_h : nullptr, slot_of, hybrid ? kSlotCold : kSlotAll};
+        if ((st = launch_gemm_ws<false>(a, hq, xw.down, nullptr, stream))) return st;
+        sm.launches += 1;
+    }
+    sm.mark(6, stream);
+    return MOE_OK;
+}
+
+}  // namespace moe
+
 int moe::forward_impl(const moe_w4a8_layer* layer, const ExpertSet& xw, const uint16_t* x_bf16,
                       const float* router_logits, int64_t T, int k, uint16_t* out_bf16, void* ws,
                       size_t ws_bytes, cudaStream_t stream, StageMarks& sm, const uint16_t* router_w) {
@@ -361,14 +494,9 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const ExpertSet& xw, const ui
     float* sx = (float*)at(p.s_x);
     uint8_t* xs = (uint8_t*)at(p.x_sorted);
     float* sxs = (float*)at(p.s_x_sorted);
-    float* h = (float*)at(p.h);
     unsigned* zero = (unsigned*)at(p.zero);
-    unsigned* amax = zero;
-    uint8_t* hq = (uint8_t*)at(p.hq);
-    float* sh = (float*)at(p.s_h);
     float* y = (float*)at(p.y);
     float* qs_x = (float*)at(p.qs_x);
-    float* qs_h = (float*)at(p.qs_h);
     // narrow token tiles (decode): codes written once per token and gathered by the GEMM; wide
     // tiles (prefill): codes copied to expert-sorted rows.  Either way the requantization (S5)
     // and the combine (S7) run as their own passes: fused into the GEMM epilogues behind
@@ -380,20 +508,7 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const ExpertSet& xw, const ui
     // narrow W4A8 / hybrid layers store xq and hq in the unsigned widening's K order (perm8); the
     // token quantization writes xq that way exactly when it is given the group sums
     const bool act_perm = gather && qsum_x != nullptr;
-    uint16_t* act16 = xw.fmt >= kFmtNvfp4 ? (uint16_t*)at(p.act16) : nullptr;
     int32_t* slot_of = hybrid ? (int32_t*)at(p.slot_of) : nullptr;
-    // the two launches of a hybrid layer's GEMM: W4A8 on the cold experts, NVFP4 on the hot ones
-    const bool run_w4 = xw.fmt == kFmtW4A8 || (hybrid && xw.n_cold > 0);
-    const bool run_f4 = xw.fmt == kFmtNvfp4 || (hybrid && xw.n_hot > 0);
-    const void* f4_gate = hybrid ? xw.h_gate : xw.gate;
-    const void* f4_up = hybrid ? xw.h_up : xw.up;
-    const void* f4_down = hybrid ? xw.h_down : xw.down;
-    const uint8_t* f4_gs = (const uint8_t*)(hybrid ? xw.h_gate_s : xw.gate_s);
-    const uint8_t* f4_us = (const uint8_t*)(hybrid ? xw.h_up_s : xw.up_s);
-    const uint8_t* f4_ds = (const uint8_t*)(hybrid ? xw.h_down_s : xw.down_s);
-    const float* f4_g2 = hybrid ? xw.h_gate_s2 : xw.gate_s2;
-    const float* f4_u2 = hybrid ? xw.h_up_s2 : xw.up_s2;
-    const float* f4_d2 = hybrid ? xw.h_down_s2 : xw.down_s2;
     if (hybrid) {
         if ((st = launch_pdl(k_slot_map, dim3(1), dim3(1024), 0, stream, xw.hot_ids, xw.n_hot, xw.cold_ids,
                              xw.n_cold, L.E, slot_of)))
@@ -459,79 +574,15 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const ExpertSet& xw, const ui
         sm.launches += 1;
         sm.mark(2, stream);
     }
-    // S8: shared experts, summed = one SwiGLU MLP of width n_shared * shared_N
+    // S8
     float* shared = nullptr;
-    if (L.n_shared > 0) {
-        const int Wsh = L.n_shared * L.shared_N;
-        uint16_t* sa = (uint16_t*)at(p.sh_a);
-        shared = (float*)at(p.sh_y);
-        // the SwiGLU activation as bf16 hi and lo halves [T, 2 Wsh]; the down GEMM reduces over both
-        Bf16GemmArgs g{Wsh, (int)T, L.H, 0, sa, 2 * Wsh, 0};
-        if ((st = launch_gemm_bf16_ws<true>(g, x_bf16, L.sh_gate, L.sh_up, stream))) return st;
-        Bf16GemmArgs d{L.H, (int)T, 2 * Wsh, L.shared_N, shared, L.H, Wsh};
-        if ((st = launch_gemm_bf16_ws<false>(d, sa, L.sh_down, nullptr, stream))) return st;
-        sm.launches += 2;
-    }
-    sm.mark(3, stream);
-    // S4 + SwiGLU: h = silu(G) * U, max|h| per row
-    if (run_f4) {
-        // f16 copy of the FP8 activations (exact), then the f16 tensor-core GEMM
-        // (in a narrow hybrid layer the per-token codes are in the W4A8 tiles' K order)
-        if ((st = launch_e4m3_to_f16(gather ? xq : xs, (gather ? T : P) * L.H, act16, stream, act_perm)))
-            return st;
-        F4GemmArgs f{W8GemmArgs{gather ? sx : sxs, nullptr, nullptr, offsets, L.E, L.N, L.H, (int)P, h, L.N,
-                                amax, sorted, k, (int)T},
-                     f4_gs, f4_us, f4_g2, f4_u2, slot_of, hybrid ? kSlotHot : kSlotAll};
-        if ((st = launch_gemm_nvfp4<true>(f, act16, f4_gate, f4_up, stream))) return st;
-        sm.launches += 2;
-    }
-    if (xw.fmt == kFmtW8A8) {
-        W8GemmArgs a{gather ? sx : sxs, (const float*)xw.gate_s, (const float*)xw.up_s, offsets, L.E, L.N,
-                     L.H, (int)P, h, L.N, amax, sorted, k, (int)T};
-        if ((st = launch_gemm_w8a8<true>(a, gather ? (const void*)xq : (const void*)xs, xw.gate, xw.up,
-                                         stream)))
-            return st;
-        sm.launches += 1;
-    } else if (run_w4) {
-        WsGemmArgs a{gather ? sx : sxs, (const uint16_t*)xw.gate_s, (const uint16_t*)xw.up_s, offsets, L.E,
-                     L.N, L.H, (int)P, h, L.N, amax, sorted, k, (int)T, gather ? qs_x : nullptr, slot_of,
-                     hybrid ? kSlotCold : kSlotAll};
-        if ((st = launch_gemm_ws<true>(a, gather ? (const void*)xq : (const void*)xs, xw.gate, xw.up,
-                                       stream)))
-            return st;
-        sm.launches += 1;
-    }
-    sm.mark(4, stream);
-    // S5
-    // the W4A8 down GEMM widens its narrow tiles unsigned and needs the requantized rows' group sums;
-    // hq, like xq, is stored in those tiles' K order whenever a W4A8 or hybrid layer runs narrow
-    const bool down_sums = run_w4 && gather;
-    if ((st = launch_pdl(k_requant, dim3(static_cast<unsigned>(P)), dim3(256), 0, stream, h, L.N, amax, hq, sh,
-                         down_sums ? qs_h : nullptr, act_perm)))
+    if ((st = run_shared(L, (uint16_t*)at(p.sh_a), (float*)at(p.sh_y), x_bf16, T, stream, sm, &shared)))
         return st;
-    sm.launches += 1;
-    sm.mark(5, stream);
-    // S6
-    if (run_f4) {
-        if ((st = launch_e4m3_to_f16(hq, P * L.N, act16, stream, act_perm))) return st;
-        F4GemmArgs f{W8GemmArgs{sh, nullptr, nullptr, offsets, L.E, L.H, L.N, (int)P, y, L.H, nullptr, sorted,
-                                k, (int)T},
-                     f4_ds, nullptr, f4_d2, nullptr, slot_of, hybrid ? kSlotHot : kSlotAll};
-        if ((st = launch_gemm_nvfp4<false>(f, act16, f4_down, nullptr, stream))) return st;
-        sm.launches += 2;
+    sm.mark(3, stream);
+    {
+        RoutedRows rr{offsets, sorted, P, T, k, gather, act_perm, xq, sx, xs, sxs, qs_x};
+        if ((st = run_experts(L, xw, p, w, rr, slot_of, stream, sm))) return st;
     }
-    if (xw.fmt == kFmtW8A8) {
-        W8GemmArgs a{sh, (const float*)xw.down_s, nullptr, offsets, L.E, L.H, L.N, (int)P, y, L.H, nullptr,
-                     sorted, k, (int)T};
-        if ((st = launch_gemm_w8a8<false>(a, hq, xw.down, nullptr, stream))) return st;
-        sm.launches += 1;
-    } else if (run_w4) {
-        WsGemmArgs a{sh, (const uint16_t*)xw.down_s, nullptr, offsets, L.E, L.H, L.N, (int)P, y, L.H,
-                     nullptr, sorted, k, (int)T, down_sums ? qs_h : nullptr, slot_of, hybrid ? kSlotCold : kSlotAll};
-        if ((st = launch_gemm_ws<false>(a, hq, xw.down, nullptr, stream))) return st;
-        sm.launches += 1;
-    }
-    sm.mark(6, stream);
     // S7
     {
         const int64_t n = T * (L.H / 4);

@@ -218,7 +218,7 @@ __global__ void __launch_bounds__(192, 1)
 
     __syncwarp();
     __syncthreads();
-    if (*abort && tid == 0) atomicExch(&g_device_status, 1);
+    if (*abort && tid == 0) atomicOr(&g_device_status, kStatusTimeout);
     if (warp == 5) {
         tc::tc_fence_after();
         tc::tmem_dealloc(tmem, C::kTmemCols);

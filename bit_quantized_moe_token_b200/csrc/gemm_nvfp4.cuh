@@ -327,7 +327,7 @@ __global__ void __launch_bounds__(F4Cfg<BN>::kThreads, F4Cfg<BN>::kCtasPerSm)
 
     __syncwarp();
     __syncthreads();
-    if (*abort && tid == 0) atomicExch(&g_device_status, 1);
+    if (*abort && tid == 0) atomicOr(&g_device_status, kStatusTimeout);
     if (warp == C::kWarpMma) {
         tc::tc_fence_after();
         tc::tmem_dealloc(tmem, C::kTmemCols);

@@ -305,7 +305,7 @@ __global__ void __launch_bounds__(W8Cfg<BN>::kThreads, 1)
 
     __syncwarp();          // single-lane roles reconverge before the CTA-wide barrier
     __syncthreads();
-    if (*abort && tid == 0) atomicExch(&g_device_status, 1);
+    if (*abort && tid == 0) atomicOr(&g_device_status, kStatusTimeout);
     if (warp == C::kWarpMma) {
         tc::tc_fence_after();
         tc::tmem_dealloc(tmem, C::kTmemCols);

@@ -567,7 +567,7 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
     __syncwarp();          // single-lane roles reconverge before the CTA-wide barrier
     if constexpr (!kSwiGLU) pdl_wait();   // (returns at once in the roles that waited already)
     __syncthreads();
-    if (*abort && tid == 0) atomicExch(&g_device_status, 1);
+    if (*abort && tid == 0) atomicOr(&g_device_status, kStatusTimeout);
     if (warp == C::kWarpMma) {
         tc::tc_fence_after();
         tc::tmem_dealloc(tmem, C::kTmemCols);

@@ -8,8 +8,12 @@
 #include "common.cuh"
 
 namespace moe {
-// The library's sticky device-status word (one per device, per loaded library): kernels
-// with bounded waits set it when a wait gives up; moe_last_device_status() reads and clears it.
+// The library's sticky device-status word (one per device, per loaded library), a set of
+// flags: kStatusTimeout from kernels with bounded waits when a wait gives up, kStatusBadRecord
+// from the expert-parallel receive path when a record names an expert outside the receiver's
+// range.  moe_last_device_status() reads and clears it.
+constexpr int kStatusTimeout = 1;
+constexpr int kStatusBadRecord = 2;
 __device__ int g_device_status = 0;
 }
 
@@ -17,6 +21,7 @@ __device__ int g_device_status = 0;
 #include "quant.cuh"
 #include "route.cuh"
 #include "forward.cuh"
+#include "ep.cuh"
 #include "router.cuh"
 #include "tc_ptx.cuh"
 
@@ -27,7 +32,7 @@ __global__ void k_selftest_bounded_wait(uint64_t limit_ns) {
     if (threadIdx.x == 0) {
         tc::mbar_init(&bar, 1);
         tc::fence_mbar_init();
-        if (!tc::mbar_wait(&bar, 0, limit_ns)) atomicExch(&g_device_status, 1);
+        if (!tc::mbar_wait(&bar, 0, limit_ns)) atomicOr(&g_device_status, kStatusTimeout);
     }
 }
 }  // namespace moe
@@ -46,7 +51,7 @@ extern "C" int moe_last_device_status(moe_stream_t stream) {
         const int zero = 0;
         if (cudaMemcpyToSymbol(moe::g_device_status, &zero, sizeof(int)) != cudaSuccess)
             return MOE_ERR_CUDA;
-        return MOE_ERR_TIMEOUT;
+        return (v & moe::kStatusTimeout) ? MOE_ERR_TIMEOUT : MOE_ERR_INVALID_ARG;
     }
     return MOE_OK;
 }

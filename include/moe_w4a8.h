@@ -392,9 +392,10 @@ int moe_nvfp4_forward_router(const moe_nvfp4_layer* layer, const uint16_t* x_bf1
                              void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /* Waits for `stream`, then returns and clears the library's sticky device-status word for
- * the current device: MOE_OK, or MOE_ERR_TIMEOUT when a bounded device-side wait gave up
- * (its kernel then skipped the rest of its work and returned), or MOE_ERR_CUDA when the
- * stream itself reports an error. */
+ * the current device: MOE_OK; MOE_ERR_TIMEOUT when a bounded device-side wait gave up (its
+ * kernel then skipped the rest of its work and returned); MOE_ERR_INVALID_ARG when
+ * moe_ep_experts_forward met a record naming an expert outside its range (that row was computed
+ * as zero); MOE_ERR_CUDA when the stream itself reports an error. */
 int moe_last_device_status(moe_stream_t stream);
 
 /* Diagnostic for the failure-detection path: launches one CTA that waits, with the same
@@ -424,6 +425,64 @@ size_t moe_route_noalloc_max_scratch_bytes(void);
 int moe_route_topk_noalloc(const float* logits, int64_t T, int E, int k, int32_t* topk_ids,
                            float* topk_w, int32_t* expert_offsets, int32_t* sorted_pairs,
                            int32_t* row_of_pair, moe_stream_t stream);
+
+/* ---- Expert parallelism ---------------------------------------------------------------------
+ * The layer's E routed experts held by n_ranks GPUs (E % n_ranks == 0), GPU r owning experts
+ * [r E_l, (r + 1) E_l), E_l = E / n_ranks, as a W4A8 layer of E_l experts (its expert e is
+ * the full layer's expert r E_l + e).  The pages serve the layer tensor-parallel (TP4 on the
+ * Inkling-512k-NVFP4-AQLM-hybrid card, "Serving"; TP8 in the Inkling 2 Small FP8 for AMD MI300X
+ * card's launch command); splitting the experts is the plainest multi-GPU form of the same
+ * layer, with FP8 rows on the wire.  Per layer, every GPU:
+ *   1. moe_ep_dispatch on its T tokens: records and the count for each owner;
+ *   2. sends counts[r] records to GPU r and receives R records in total (all-to-all);
+ *   3. moe_ep_experts_forward on the R received records: R fp32 rows;
+ *   4. returns each received row to its sender, in the order received (all-to-all), so that
+ *      it gets back T k rows in the order of its own records;
+ *   5. moe_ep_combine on its T tokens.
+ * The result equals moe_w4a8_forward of the full layer on the same tokens bit for bit when
+ * n_ranks = 1; with more GPUs each owner picks the forward's token tile for its own R rows
+ * over E_l experts, and the output keeps that forward's accuracy.
+ *
+ * Record: MOE_EP_RECORD_BYTES(H) bytes, 16-byte aligned in an array: the token's E4M3 codes
+ * [H] (S1, column order), its fp32 scale s_x, the int32 expert index within the owner's range,
+ * and 8 zero bytes. */
+#define MOE_EP_RECORD_BYTES(H) ((size_t)(H) + 16)
+
+/* Workspace of moe_ep_dispatch, which moe_ep_combine reads back (0 on invalid arguments). */
+size_t moe_ep_dispatch_workspace_bytes(const moe_w4a8_layer* layer, int64_t T, int k);
+
+/* S2 (top-k), S3 (stable permutation by expert, hence by owner) and S1 (per-token FP8) on this
+ * GPU's tokens.  layer: the full layer's shapes (E, H, N, group; its weight pointers are not
+ * read).  x_bf16 [T, H] and router_logits fp32 [T, E] as in moe_w4a8_forward.
+ *   send_counts   device int32 [n_ranks]: records for each owner
+ *   send_records  device [T k] records, those of owner 0 first, then owner 1, ...; within an
+ *                 owner by (expert, pair t k + j)
+ * ws (256-byte aligned, moe_ep_dispatch_workspace_bytes) keeps the gates and each pair's
+ * record slot for moe_ep_combine: leave it untouched in between.  T == 0 zeroes send_counts.
+ * Returns MOE_ERR_UNSUPPORTED_SHAPE when E % n_ranks != 0, MOE_ERR_INVALID_ARG when n_ranks is
+ * outside [1, E], else as moe_w4a8_forward. */
+int moe_ep_dispatch(const moe_w4a8_layer* layer, const uint16_t* x_bf16, const float* router_logits,
+                    int64_t T, int k, int n_ranks, int32_t* send_counts, uint8_t* send_records,
+                    void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Workspace of moe_ep_experts_forward for R records (0 on invalid arguments). */
+size_t moe_ep_experts_workspace_bytes(const moe_w4a8_layer* local_layer, int64_t R);
+
+/* S4-S6 on R received records: y_rows fp32 [R, H] (16-byte aligned), row i for record i.
+ * local_layer: this GPU's E_l experts (shared-expert fields are not read).  A record whose
+ * expert index is outside [0, E_l) gives a zero row and sets the device-status word
+ * (moe_last_device_status).  R == 0 is a no-op. */
+int moe_ep_experts_forward(const moe_w4a8_layer* local_layer, const uint8_t* records, int64_t R,
+                           float* y_rows, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* S8 and S7 on this GPU's tokens: out_bf16 [T, H] = bf16( sum_j gate[t,j] y_back[slot(t,j)]
+ * + shared experts(x_t) ), j in selection order, exactly the forward's combine.  y_back fp32
+ * [T k, H]: the rows returned for this GPU's records, in record order.  layer, x_bf16, T, k
+ * and ws as given to moe_ep_dispatch (layer's shared experts are used; x_bf16 may be null
+ * without them). */
+int moe_ep_combine(const moe_w4a8_layer* layer, const uint16_t* x_bf16, const float* y_back,
+                   int64_t T, int k, uint16_t* out_bf16, void* ws, size_t ws_bytes,
+                   moe_stream_t stream);
 
 /* Static description of a status code. */
 const char* moe_status_string(int status);

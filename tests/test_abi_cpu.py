@@ -230,3 +230,34 @@ def test_binding_has_no_fallback():
     assert "oracle" not in src and "numpy" not in src
     for f in glob.glob(os.path.join(ROOT, "bit_quantized_moe_token_b200", "*.py")):
         assert "import oracle" not in open(f).read(), f
+
+
+def test_ep_entry_points_reject_bad_args():
+    L = _L()
+    p = ctypes.c_void_p(4096)
+    full = moe._binding._CLayer(8, 256, 128, 128, p, p, p, p, p, p, 0, 0, None, None, None)
+    nd = moe.moe_ep_dispatch_workspace_bytes(full, 4, 2)
+    assert 0 < nd < moe.moe_w4a8_workspace_bytes(full, 4, 2)
+    assert moe.moe_ep_dispatch_workspace_bytes(full, 4, 9) == 0                    # k > E
+    assert moe.moe_ep_experts_workspace_bytes(full, 40) == moe.moe_w4a8_workspace_bytes(full, 40, 1)
+    assert moe.ep_record_bytes(256) == 272
+    d = L.moe_ep_dispatch
+    assert d(ctypes.byref(full), p, p, 4, 2, 3, p, p, p, nd, None) == -2            # 8 % 3 != 0
+    assert d(ctypes.byref(full), p, p, 4, 2, 0, p, p, p, nd, None) == -1            # no ranks
+    assert d(ctypes.byref(full), p, p, 4, 2, 16, p, p, p, nd, None) == -1           # more ranks than experts
+    assert d(ctypes.byref(full), p, p, 4, 2, 2, None, p, p, nd, None) == -1         # no counts
+    assert d(ctypes.byref(full), p, p, 4, 2, 2, p, None, p, nd, None) == -1         # no records
+    assert d(ctypes.byref(full), p, p, 4, 2, 2, p, p, p, nd - 1, None) == -4
+    assert d(ctypes.byref(full), p, p, 4, 2, 2, p, ctypes.c_void_p(4104), p, nd, None) == -3
+    f = L.moe_ep_experts_forward
+    ne = moe.moe_ep_experts_workspace_bytes(full, 40)
+    assert f(ctypes.byref(full), p, 0, p, p, ne, None) == 0                          # no records: no-op
+    assert f(ctypes.byref(full), None, 40, p, p, ne, None) == -1
+    assert f(ctypes.byref(full), p, 40, p, p, ne - 1, None) == -4
+    assert f(ctypes.byref(full), ctypes.c_void_p(4104), 40, p, p, ne, None) == -3   # records below 16 B
+    assert f(ctypes.byref(moe.layer_struct(8, 256, 128)), p, 40, p, p, ne, None) == -1   # no weights
+    c = L.moe_ep_combine
+    assert c(ctypes.byref(full), p, p, 0, 2, p, p, nd, None) == 0                    # no tokens: no-op
+    assert c(ctypes.byref(full), p, None, 4, 2, p, p, nd, None) == -1
+    assert c(ctypes.byref(full), p, p, 4, 2, p, p, nd - 1, None) == -4
+    assert c(ctypes.byref(full), p, p, 4, 2, ctypes.c_void_p(4104), p, nd, None) == -3
