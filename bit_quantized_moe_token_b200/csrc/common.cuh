@@ -32,11 +32,8 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // grid that has started therefore knows that every grid two or more launches back has
 // completed, and a grid may read data written that far back (expert offsets, weights) before
 // its own wait.  The overlap gained: a grid's launch, prologue (barriers, TMEM allocation,
-// descriptor prefetch) and any such early reads run under its predecessor's tail.  One grid
-// deviates: the SwiGLU requantization releases the down GEMM before it waits, because the down
-// GEMM reads nothing of it before its own wait and its early reads (offsets, weights) were made
-// final by the gate/up GEMM's wait.  Both instructions are no-ops for a grid launched without
-// the programmatic-serialization attribute.
+// descriptor prefetch) and any such early reads run under its predecessor's tail.  Both
+// instructions are no-ops for a grid launched without the programmatic-serialization attribute.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void pdl_enter() {

@@ -22,11 +22,7 @@ __global__ void __launch_bounds__(256) k_requant(const float* __restrict__ h, in
                                                  const unsigned* __restrict__ amax,
                                                  uint8_t* __restrict__ hq, float* __restrict__ s_h,
                                                  float* __restrict__ qsum, bool perm) {
-    // releases the down GEMM before waiting: the down GEMM reads nothing of this grid before its
-    // own wait, and what it reads early (expert offsets, weights) the gate/up GEMM's wait made
-    // final; so it can start on SMs the gate/up GEMM's last tiles leave free
-    pdl_trigger();
-    pdl_wait();
+    pdl_enter();
     const int64_t r = blockIdx.x;
     const float s = __fdiv_rn(__uint_as_float(amax[r]), kFp8Max);
     const float4* src = reinterpret_cast<const float4*>(h + r * N);

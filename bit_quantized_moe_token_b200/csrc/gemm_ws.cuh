@@ -221,9 +221,6 @@ __global__ void __launch_bounds__(WsCfg<BN, kUnsigned>::kThreads, WsCfg<BN, kUns
                     tc::mbar_arrive_expect_tx(&w_full[st], C::kRaw);
                     ws::tma_load_2d(wring + st * C::kRaw, &tm_w0, st * C::kGS * 64, wb * a.R0 + mt * 128, &w_full[st]);
                 }
-                // and the rest of the first tile into L2, where its loads will find it
-                for (int st = pre_w; st < nst; ++st)
-                    ws::tma_prefetch_l2_2d(&tm_w0, st * C::kGS * 64, wb * a.R0 + mt * 128);
             }
             pdl_wait();
         }
