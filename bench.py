@@ -129,6 +129,7 @@ KERNEL_SOURCES = {"w4a8": ("gemm_ws.cuh", "tc_pipe.cuh", "tc_ptx.cuh", "tc_tiles
                             "common.cuh")}
 PROFILE_FOR = {("w4a8", "decode_t8"): "gemm_w4a8_ws_decode_t8.md",
                ("w4a8", "prefill_t2048_zipf"): "gemm_w4a8_ws_prefill_t2048.md",
+               ("w4a8", "prefill_t16384_shared"): "gemm_w4a8_ws_prefill_t16384.md",
                ("w8a8", "decode_t8"): "gemm_w8a8_decode_t8.md",
                ("w8a8", "prefill_t2048_zipf"): "gemm_w8a8_prefill_t2048.md",
                ("nvfp4", "decode_t8"): "gemm_nvfp4_decode_t8.md",
