@@ -18,12 +18,25 @@ namespace moe {
 // With qsum non-null it also writes each row's per-128-column sums of the FP8 values (the down
 // GEMM's unsigned widening removes its +8 offset with them; a half-warp covers one group).  With
 // perm the codes are stored in the narrow W4A8 tiles' K order (perm8).
+// With `offsets` non-null (a layer whose short segments run on narrow tiles) the order and the
+// sums are per row instead: the rows of segments of at most kShortRows rows in the K order with
+// their sums, the others in column order without.
 __global__ void __launch_bounds__(256) k_requant(const float* __restrict__ h, int N,
                                                  const unsigned* __restrict__ amax,
                                                  uint8_t* __restrict__ hq, float* __restrict__ s_h,
-                                                 float* __restrict__ qsum, bool perm) {
+                                                 float* __restrict__ qsum, bool perm,
+                                                 const int32_t* __restrict__ offsets, int E) {
     pdl_enter();
     const int64_t r = blockIdx.x;
+    if (offsets) {   // the segment of row r: offsets[e] <= r < offsets[e + 1]
+        int lo = 0, hi = E - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (offsets[mid] <= r) lo = mid; else hi = mid - 1;
+        }
+        perm = offsets[lo + 1] - offsets[lo] <= kShortRows;
+        if (!perm) qsum = nullptr;
+    }
     const float s = __fdiv_rn(__uint_as_float(amax[r]), kFp8Max);
     const float4* src = reinterpret_cast<const float4*>(h + r * N);
     const int G = N / kGroup;
@@ -132,6 +145,62 @@ inline int launch_quant_topk(const float* logits, const uint16_t* x, int64_t T, 
 #undef MOE_QT
 }
 
+// S1 for token t (one CTA, the arithmetic of k_quant_tokens) written to its k expert-sorted rows
+// and to row t of q_tok / s_tok, for a layer whose short segments (at most kShortRows rows) run on
+// narrow tiles: rows of short segments get the codes in the narrow tiles' K order (perm8) and
+// their per-128-column sums in qsum_rows [P, H / 128], the other rows the codes in column order.
+__global__ void __launch_bounds__(256) k_quant_tokens_split(const uint16_t* __restrict__ x, int H, int k,
+                                                            const int32_t* __restrict__ ids,
+                                                            const int32_t* __restrict__ rop,
+                                                            const int32_t* __restrict__ offsets,
+                                                            uint8_t* __restrict__ q, float* __restrict__ scale,
+                                                            float* __restrict__ qsum_rows,
+                                                            uint8_t* __restrict__ q_tok,
+                                                            float* __restrict__ s_tok) {
+    pdl_enter();
+    __shared__ float red[32];
+    const int64_t t = blockIdx.x;
+    const uint4* row = reinterpret_cast<const uint4*>(x + t * H);
+    const int chunks = H >> 3;
+    float a = 0.0f;
+    for (int c = threadIdx.x; c < chunks; c += blockDim.x) a = fmaxf(a, amax8(__ldg(row + c)));
+    a = block_max(a, red);
+    const float s = __fdiv_rn(a, kFp8Max);
+    int32_t r_[kMaxK];
+    bool short_[kMaxK];
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) {
+        r_[j] = j < k ? rop[t * k + j] : 0;
+        const int e = j < k ? ids[t * k + j] : 0;
+        short_[j] = j < k && offsets[e + 1] - offsets[e] <= kShortRows;
+    }
+    const int G = H / kGroup;
+    for (int base = 0; base < chunks; base += blockDim.x) {   // blockDim = 256: whole half-warps
+        const int c = base + threadIdx.x;
+        const bool live = c < chunks;
+        const uint2 codes = live ? quant8(__ldg(row + c), s) : make_uint2(0u, 0u);
+        const uint2 pc = perm8(codes);
+        if (live) {
+#pragma unroll
+            for (int j = 0; j < kMaxK; ++j)
+                if (j < k) reinterpret_cast<uint2*>(q + (int64_t)r_[j] * H)[c] = short_[j] ? pc : codes;
+            reinterpret_cast<uint2*>(q_tok + t * H)[c] = codes;
+        }
+        const float gs = halfwarp_sum(e4m3x8_sum(codes));
+        if (live && (threadIdx.x & 15) == 0) {
+#pragma unroll
+            for (int j = 0; j < kMaxK; ++j)
+                if (j < k && short_[j]) qsum_rows[(int64_t)r_[j] * G + c / 16] = gs;
+        }
+    }
+    if (threadIdx.x == 0) {
+#pragma unroll
+        for (int j = 0; j < kMaxK; ++j)
+            if (j < k) scale[r_[j]] = s;
+        s_tok[t] = s;
+    }
+}
+
 // ------------------------------------------------------------------------------------------
 // workspace
 // ------------------------------------------------------------------------------------------
@@ -140,6 +209,7 @@ struct WsPlan {
     size_t xq, s_x, x_sorted, s_x_sorted, h, zero, hq, s_h, y;
     size_t qs_x;         // per (token, K-group) sums of the FP8 values (narrow W4A8 tiles)
     size_t qs_h;         // per (sorted row, N-group) sums of the requantized values (W4A8 down GEMM)
+    size_t qs_xr;        // per (sorted row, K-group) sums of the FP8 input rows (short segments, split layers)
     size_t logits, rcnt; // router logits [T, E] and the fused router's counters (router entry points)
     size_t act16;        // NVFP4 experts: f16 copies of the GEMM inputs (max of [T|P, H] and [P, N])
     size_t slot_of;      // hybrid layers: expert -> slab map [E]
@@ -176,6 +246,7 @@ inline WsPlan plan_workspace(const moe_w4a8_layer& L, int64_t T, int k, int fmt 
     p.y = take((size_t)P * L.H * 4);
     p.qs_x = take((size_t)T * (L.H / 128) * 4);
     p.qs_h = take((size_t)P * (L.N / 128) * 4);
+    p.qs_xr = take((size_t)P * (L.H / 128) * 4);
     p.logits = take((size_t)T * L.E * 4);
     p.rcnt = take((size_t)router_counter_words(T) * 4);
     p.act16 = fmt >= 2 ? take((size_t)P * (L.H > L.N ? L.H : L.N) * 2) : 0;
@@ -223,7 +294,8 @@ extern "C" int moe_w4a8_workspace_layout(const moe_w4a8_layer* layer, int64_t T,
     out->hq = p.hq;
     out->s_h = p.s_h;
     out->total = p.total;
-    out->act_order = moe::ws_narrow(moe::ws_tile_rows(T * k, layer->E)) ? 1 : 0;   // W4A8 layer: see the header
+    // W4A8 layer: see the header
+    out->act_order = moe::ws_narrow(moe::ws_tile_rows(T * k, layer->E)) ? 1 : moe::ws_split(T * k, layer->E) ? 2 : 0;
     return MOE_OK;
 }
 
@@ -342,6 +414,10 @@ struct RoutedRows {
     const uint8_t* xs;
     const float* sxs;
     float* qs_x;
+    // W4A8 layers on wide tiles: segments of at most kShortRows rows run on narrow tiles (their
+    // sorted rows in the narrow tiles' K order, with per-row group sums qs_xr)
+    bool split = false;
+    const float* qs_xr = nullptr;
 };
 
 // S4-S6 on routed rows: gate/up GEMM with the SwiGLU epilogue (h, max|h| per row), the
@@ -397,6 +473,15 @@ inline int run_experts(const moe_w4a8_layer& L, const ExpertSet& xw, const WsPla
                                          stream)))
             return st;
         sm.launches += 1;
+    } else if (run_w4 && rr.split) {
+        // the short segments on narrow tiles, then the others on wide tiles
+        WsGemmArgs a{sxs, (const uint16_t*)xw.gate_s, (const uint16_t*)xw.up_s, offsets, L.E, L.N, L.H, (int)P, h,
+                     L.N, amax, sorted, k, (int)T, rr.qs_xr, nullptr, kSlotShort};
+        if ((st = launch_gemm_ws<true>(a, xs, xw.gate, xw.up, stream, kShortRows, true))) return st;
+        a.qsum = nullptr;
+        a.slot_want = kSlotLong;
+        if ((st = launch_gemm_ws<true>(a, xs, xw.gate, xw.up, stream))) return st;
+        sm.launches += 2;
     } else if (run_w4) {
         WsGemmArgs a{gather ? sx : sxs, (const uint16_t*)xw.gate_s, (const uint16_t*)xw.up_s, offsets, L.E,
                      L.N, L.H, (int)P, h, L.N, amax, sorted, k, (int)T, gather ? qs_x : nullptr, slot_of,
@@ -412,7 +497,8 @@ inline int run_experts(const moe_w4a8_layer& L, const ExpertSet& xw, const WsPla
     // hq, like xq, is stored in those tiles' K order whenever a W4A8 or hybrid layer runs narrow
     const bool down_sums = run_w4 && gather;
     if ((st = launch_pdl(k_requant, dim3(static_cast<unsigned>(P)), dim3(256), 0, stream, h, L.N, amax, hq, sh,
-                         down_sums ? qs_h : nullptr, act_perm)))
+                         (down_sums || rr.split) ? qs_h : nullptr, act_perm,
+                         rr.split ? offsets : (const int32_t*)nullptr, L.E)))
         return st;
     sm.launches += 1;
     sm.mark(5, stream);
@@ -430,6 +516,14 @@ inline int run_experts(const moe_w4a8_layer& L, const ExpertSet& xw, const WsPla
                      sorted, k, (int)T};
         if ((st = launch_gemm_w8a8<false>(a, hq, xw.down, nullptr, stream))) return st;
         sm.launches += 1;
+    } else if (run_w4 && rr.split) {
+        WsGemmArgs a{sh, (const uint16_t*)xw.down_s, nullptr, offsets, L.E, L.H, L.N, (int)P, y, L.H, nullptr, sorted,
+                     k, (int)T, qs_h, nullptr, kSlotShort};
+        if ((st = launch_gemm_ws<false>(a, hq, xw.down, nullptr, stream, kShortRows))) return st;
+        a.qsum = nullptr;
+        a.slot_want = kSlotLong;
+        if ((st = launch_gemm_ws<false>(a, hq, xw.down, nullptr, stream))) return st;
+        sm.launches += 2;
     } else if (run_w4) {
         WsGemmArgs a{sh, (const uint16_t*)xw.down_s, nullptr, offsets, L.E, L.H, L.N, (int)P, y, L.H,
                      nullptr, sorted, k, (int)T, down_sums ? qs_h : nullptr, slot_of, hybrid ? kSlotCold : kSlotAll};
@@ -504,6 +598,17 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const ExpertSet& xw, const ui
     // narrow W4A8 / hybrid layers store xq and hq in the unsigned widening's K order (perm8); the
     // token quantization writes xq that way exactly when it is given the group sums
     const bool act_perm = gather && qsum_x != nullptr;
+    // a W4A8 layer on 128-row tiles runs its short segments on narrow tiles (ws_split)
+    const bool split = xw.fmt == kFmtW4A8 && ws_split(P, L.E);
+    float* qs_xr = (float*)at(p.qs_xr);
+    // S1 into the expert-sorted rows (wide tiles) and per token
+    auto quant_rows = [&]() -> int {
+        if (split)
+            return launch_pdl(k_quant_tokens_split, dim3(static_cast<unsigned>(T)), dim3(256), 0, stream, x_bf16,
+                              L.H, k, (const int32_t*)ids, (const int32_t*)rop, (const int32_t*)offsets, xs, sxs,
+                              qs_xr, xq, sx);
+        return launch_quant_tokens(x_bf16, T, L.H, xs, sxs, rop, k, stream, xq, sx);
+    };
     int32_t* slot_of = hybrid ? (int32_t*)at(p.slot_of) : nullptr;
     if (hybrid) {
         if ((st = launch_pdl(k_slot_map, dim3(1), dim3(1024), 0, stream, xw.hot_ids, xw.n_hot, xw.cold_ids,
@@ -540,7 +645,7 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const ExpertSet& xw, const ui
             if ((st = launch_permute(ids, T, L.E, k, offsets, sorted, rop, (int32_t*)at(p.route_ws), stream,
                                      zero, p.n_zero)))
                 return st;
-            if ((st = launch_quant_tokens(x_bf16, T, L.H, xs, sxs, rop, k, stream, xq, sx))) return st;
+            if ((st = quant_rows())) return st;
             sm.launches += (P <= kSinglePassMaxP ? 1 : 3) + 1;
         }
         sm.mark(2, stream);
@@ -566,7 +671,7 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const ExpertSet& xw, const ui
         sm.launches += 1 + (P <= kSinglePassMaxP ? 1 : 3);
         sm.mark(1, stream);
         // S1, written to the token's k expert-sorted rows and to its own row
-        if ((st = launch_quant_tokens(x_bf16, T, L.H, xs, sxs, rop, k, stream, xq, sx))) return st;
+        if ((st = quant_rows())) return st;
         sm.launches += 1;
         sm.mark(2, stream);
     }
@@ -576,7 +681,7 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const ExpertSet& xw, const ui
         return st;
     sm.mark(3, stream);
     {
-        RoutedRows rr{offsets, sorted, P, T, k, gather, act_perm, xq, sx, xs, sxs, qs_x};
+        RoutedRows rr{offsets, sorted, P, T, k, gather, act_perm, xq, sx, xs, sxs, qs_x, split, qs_xr};
         if ((st = run_experts(L, xw, p, w, rr, slot_of, stream, sm))) return st;
     }
     // S7
@@ -774,7 +879,10 @@ extern "C" int moe_hybrid_workspace_layout(const moe_hybrid_layer* layer, int64_
     if (!layer) return MOE_ERR_INVALID_ARG;
     const moe_w4a8_layer s = moe::shape_of(*layer);
     int st = moe_w4a8_workspace_layout(&s, T, k, out);
-    if (st == MOE_OK) out->total = moe::plan_workspace(s, T, k, moe::kFmtHybrid).total;
+    if (st == MOE_OK) {
+        out->total = moe::plan_workspace(s, T, k, moe::kFmtHybrid).total;
+        if (out->act_order == 2) out->act_order = 0;   // hybrid layers do not split by segment length
+    }
     return st;
 }
 

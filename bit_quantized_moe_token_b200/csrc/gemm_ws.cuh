@@ -610,18 +610,30 @@ int launch_gemm_ws_inst(const WsGemmArgs& a, const void* act, const void* w0, co
 // per-token FP8 array instead of an expert-sorted copy.
 inline bool ws_narrow(int BN) { return BN <= 32; }
 
+// A W4A8 layer on 128-row tiles (segments of 24 to 160 rows on average, typically skewed) runs
+// its segments of at most kShortRows rows on 32-row tiles, which widen unsigned and cost a
+// quarter of the integer work per weight: at T = 2048 with Zipf routing 84 of 184 128-row tiles
+// hold at most 32 rows (5 % of the rows).
+inline bool ws_split(int64_t P, int E) { return ws_tile_rows(P, E) == 128; }
+
+// bn: the token-tile width (0: chosen from the average segment length, ws_tile_rows);
+// rows_sorted: a narrow gate/up launch reads expert-sorted activation rows instead of gathering
+// them by token (the short segments of a layer whose other segments run on wide tiles).
 template <bool kSwiGLU>
 int launch_gemm_ws(const WsGemmArgs& a, const void* act, const void* w0, const void* w1,
-                   cudaStream_t stream) {
-    const int BN = ws_tile_rows(a.P, a.E);
+                   cudaStream_t stream, int bn = 0, bool rows_sorted = false) {
+    const int BN = bn ? bn : ws_tile_rows(a.P, a.E);
     const int64_t max_row_tiles = ((int64_t)a.P + BN - 1) / BN + a.E;
     switch (BN) {
         // narrow tiles (decode) widen unsigned: the tensor core sums the +8-offset products in fp32
         // without loss (measured: exact, or 0.5 ulp, over 128-wide groups), and the promotion
         // removes the offset with the activation rows' group sums (per token for the gathering
-        // gate/up instance, per sorted row for the down instance)
+        // gate/up instance, per sorted row otherwise)
         case 16: return launch_gemm_ws_inst<16, true, kSwiGLU, kSwiGLU>(a, act, w0, w1, max_row_tiles, stream);
-        case 32: return launch_gemm_ws_inst<32, true, kSwiGLU, kSwiGLU>(a, act, w0, w1, max_row_tiles, stream);
+        case 32:
+            if (kSwiGLU && rows_sorted)
+                return launch_gemm_ws_inst<32, true, kSwiGLU, false>(a, act, w0, w1, max_row_tiles, stream);
+            return launch_gemm_ws_inst<32, true, kSwiGLU, kSwiGLU>(a, act, w0, w1, max_row_tiles, stream);
         case 128: return launch_gemm_ws_inst<128, false, kSwiGLU, false>(a, act, w0, w1, max_row_tiles, stream);
         default: return launch_gemm_ws_inst<192, false, kSwiGLU, false>(a, act, w0, w1, max_row_tiles, stream);
     }

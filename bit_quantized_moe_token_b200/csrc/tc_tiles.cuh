@@ -57,7 +57,10 @@ __device__ __forceinline__ uint32_t sw128_off(int r, int j) {
 // Slab map of a hybrid layer (hot NVFP4 / cold W4A8 experts): slot_of[e] = i for hot slab i,
 // -(j + 1) for cold slab j, kSlotNone for an expert in neither list.
 constexpr int32_t kSlotNone = INT32_MIN;
-enum SlotWant { kSlotAll = 0, kSlotCold = 1, kSlotHot = 2 };
+// kSlotShort / kSlotLong select experts by segment length instead (at most kShortRows rows, or
+// more): a W4A8 layer of mostly long segments runs its short ones on narrow tiles.
+enum SlotWant { kSlotAll = 0, kSlotCold = 1, kSlotHot = 2, kSlotShort = 3, kSlotLong = 4 };
+constexpr int kShortRows = 32;
 
 __device__ __forceinline__ bool slot_kept(const int32_t* slot_of, int want, int e) {
     if (!slot_of || want == kSlotAll) return true;
@@ -75,14 +78,19 @@ __device__ __forceinline__ int weight_slab(const int32_t* slot_of, int e) {
 // Per-expert prefix of row tiles (ceil(len / BN)) into shared `pre[0..E]` and the segment offsets
 // [0..E] into shared `soff`; returns the total.  Every thread loads its share of the offsets at
 // once (one global round trip), then one warp scans the tile counts in shared memory.  With
-// `slot_of`, experts of the other format get no tiles (`want`: kSlotCold or kSlotHot).
+// `slot_of`, experts of the other format get no tiles (`want`: kSlotCold or kSlotHot); with
+// kSlotShort / kSlotLong, experts of the other segment-length class get none.
 __device__ int row_tile_prefix(const int32_t* __restrict__ offsets, int E, int BN, int* pre, int* soff,
                                const int32_t* slot_of = nullptr, int want = kSlotAll) {
     __shared__ int s_total;
     for (int e = threadIdx.x; e <= E; e += blockDim.x) soff[e] = offsets[e];
     __syncthreads();
-    for (int e = threadIdx.x; e < E; e += blockDim.x)
-        pre[e] = slot_kept(slot_of, want, e) ? (soff[e + 1] - soff[e] + BN - 1) / BN : 0;
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        const int len = soff[e + 1] - soff[e];
+        const bool kept = want >= kSlotShort ? ((len <= kShortRows) == (want == kSlotShort))
+                                             : slot_kept(slot_of, want, e);
+        pre[e] = kept ? (len + BN - 1) / BN : 0;
+    }
     __syncthreads();
     if (threadIdx.x < 32) {
         const int lane = threadIdx.x;

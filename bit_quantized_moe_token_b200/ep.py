@@ -66,7 +66,10 @@ class EpLayer:
         self.local = local
         self.group = group
         self.ops = ops
-        if dist.is_available() and dist.is_initialized():
+        # with a process group the exchanges go through it (at one rank too); without one the
+        # layer runs alone and the rows stay where they are
+        self.grouped = dist.is_available() and dist.is_initialized()
+        if self.grouped:
             self.rank = dist.get_rank(group)
             self.n_ranks = dist.get_world_size(group)
         else:
@@ -86,7 +89,7 @@ class EpLayer:
     def _exchange(self, inp, rows: int, out_splits=None, in_splits=None):
         """All-to-all of inp's rows (in_splits[r] of them to rank r); returns the `rows` rows
         received (out_splits[r] from rank r).  Alone, the rows stay where they are."""
-        if self.n_ranks == 1:
+        if not self.grouped:
             return inp
         out = torch.empty((rows,) + tuple(inp.shape[1:]), dtype=inp.dtype, device=inp.device)
         dist.all_to_all_single(out, inp, out_splits, in_splits, group=self.group)

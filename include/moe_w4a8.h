@@ -180,7 +180,9 @@ size_t moe_w4a8_workspace_bytes(const moe_w4a8_layer* layer, int64_t T, int k);
  * act_order: 0 when xq and hq hold their codes in column order; 1 when, within every block of
  * 8 columns, they hold columns 0,2,4,6,1,3,5,7 (the order in which the W4A8 GEMM's 16- and
  * 32-row token tiles split a packed word into its even and odd nibbles; used for W4A8 and
- * hybrid layers whose tiles are that narrow). */
+ * hybrid layers whose tiles are that narrow); 2 when xq is in column order and the hq rows of
+ * experts whose segment has at most 32 rows are in that K order, the other rows in column order
+ * (a W4A8 layer on 128-row tiles, which runs its short segments on 32-row tiles). */
 typedef struct {
     size_t topk_ids, topk_w, expert_offsets, sorted_pairs, row_of_pair;
     size_t xq, s_x, hq, s_h;

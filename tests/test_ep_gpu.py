@@ -185,3 +185,50 @@ def test_ep_empty_batches():
     torch.cuda.synchronize()
     assert counts.cpu().tolist() == [0, 0]
     assert moe.moe_last_device_status() == 0
+
+
+_NCCL_ONE_RANK = r'''
+import os, sys, numpy as np, torch, torch.distributed as dist
+from datetime import timedelta
+sys.path.insert(0, os.environ["MOE_ROOT"]); sys.path.insert(0, os.path.join(os.environ["MOE_ROOT"], "tests"))
+torch.cuda.set_device(0)
+dist.init_process_group("nccl", rank=0, world_size=1, timeout=timedelta(seconds=60), device_id=torch.device("cuda", 0))
+try:
+    import bit_quantized_moe_token_b200 as moe
+    from bit_quantized_moe_token_b200.ep import EpLayer, local_experts
+    from test_parity_gpu import _host_layer_and_dev, to_dev_bf16
+    from test_ep_gpu import _inputs
+    for (E, H, N, k, T) in ((8, 256, 128, 2, 37), (8, 512, 256, 2, 700)):
+        _, dl = _host_layer_and_dev(E, H, N, seed=25, n_shared=1, shared_N=128)
+        x, logits = _inputs(15, T, E, H)
+        xd, ld = to_dev_bf16(x), torch.from_numpy(logits).cuda()
+        want = moe.forward(dl, xd, ld, k)
+        ep = EpLayer(dl, local_experts(dl, 0, 1))
+        assert ep.grouped and ep.n_ranks == 1
+        got = ep.forward(xd, ld, k)
+        torch.cuda.synchronize()
+        assert moe.moe_last_device_status() == 0
+        assert torch.equal(got.view(torch.int16), want.view(torch.int16)), (E, H, N, k, T)
+    print("nccl one rank ok")
+finally:
+    dist.destroy_process_group()
+'''
+
+
+def test_ep_nccl_exchanges_one_rank():
+    """The NCCL all-to-all exchanges of EpLayer on one GPU (a process group of one rank: the
+    exchanges run, no rank waits on another): bit-exact against moe_w4a8_forward."""
+    import os
+    import socket
+    import subprocess
+    import sys
+    from conftest import ROOT
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    env = dict(os.environ, MOE_ROOT=ROOT, MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port),
+               NCCL_NVLS_ENABLE="0")
+    r = subprocess.run([sys.executable, "-c", _NCCL_ONE_RANK], env=env, capture_output=True, text=True,
+                       timeout=300)
+    assert r.returncode == 0, r.stdout[-2000:] + r.stderr[-4000:]
+    assert "nccl one rank ok" in r.stdout

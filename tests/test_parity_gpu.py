@@ -50,19 +50,28 @@ def ws_views(layer, ws, T, k):
     b = ws.cpu().numpy()
     def arr(off, dtype, n):
         return np.frombuffer(b[off:off + n * np.dtype(dtype).itemsize].tobytes(), dtype=dtype).copy()
-    def codes(off, rows, cols):
+    offsets = arr(lay["expert_offsets"], np.int32, layer.E + 1)
+    def codes(off, rows, cols, which):
         c = arr(off, np.uint8, rows * cols).reshape(rows, cols)
-        if lay["act_order"]:                  # columns 0,2,4,6,1,3,5,7 of every 8-column block
-            c = c.reshape(rows, cols // 8, 8)[:, :, _UNPERM8].reshape(rows, cols)
+        # which rows hold columns 0,2,4,6,1,3,5,7 of every 8-column block: all (act_order 1), or
+        # for hq the rows of segments of at most 32 rows (act_order 2)
+        if lay["act_order"] == 1:
+            sel = np.ones(rows, bool)
+        elif lay["act_order"] == 2 and which == "hq":
+            seg = np.diff(offsets)
+            sel = np.repeat(seg <= 32, seg)
+        else:
+            sel = np.zeros(rows, bool)
+        c[sel] = c[sel].reshape(-1, cols // 8, 8)[:, :, _UNPERM8].reshape(-1, cols)
         return c
     return dict(ids=arr(lay["topk_ids"], np.int32, P).reshape(T, k),
                 gates=arr(lay["topk_w"], np.float32, P).reshape(T, k),
-                offsets=arr(lay["expert_offsets"], np.int32, layer.E + 1),
+                offsets=offsets,
                 sorted_pairs=arr(lay["sorted_pairs"], np.int32, P),
                 row_of_pair=arr(lay["row_of_pair"], np.int32, P),
-                xq=codes(lay["xq"], T, layer.H),
+                xq=codes(lay["xq"], T, layer.H, "xq"),
                 s_x=arr(lay["s_x"], np.float32, T),
-                hq=codes(lay["hq"], P, layer.N),
+                hq=codes(lay["hq"], P, layer.N, "hq"),
                 s_h=arr(lay["s_h"], np.float32, P))
 
 
@@ -280,6 +289,26 @@ def test_forward_ragged_shapes(E, H, N, k, T):
     x = synth.normal_bf16(3, 777 + T, T * H).reshape(T, H)
     logits = synth.normal_f32(3, 778 + T, T * E).reshape(T, E)
     _run_and_compare(hl, dl, x, logits, k)
+
+
+@pytest.mark.parametrize("E,H,N,k,T,skew", [(16, 512, 256, 2, 400, 3.0), (32, 256, 128, 4, 600, 2.0),
+                                              (8, 256, 256, 2, 600, 0.0)])
+def test_forward_split_short_segments(E, H, N, k, T, skew):
+    """Layers on 128-row tiles run their segments of at most 32 rows on 32-row tiles (unsigned
+    widening, sorted rows in its K order) and the others on 128-row tiles: skewed routing gives
+    both kinds in one layer (the last case, uniform, leaves the narrow launch empty)."""
+    hl, dl = _host_layer_and_dev(E, H, N, seed=31 + E, n_shared=1, shared_N=128)
+    x = synth.normal_bf16(33, 73_000, T * H, 1.0).reshape(T, H)
+    logits = synth.normal_f32(33, 73_001, T * E, 1.0).reshape(T, E)
+    logits += (skew * np.linspace(1.0, 0.0, E)).astype(np.float32)   # early experts preferred
+    lay = moe.moe_w4a8_workspace_layout(dl, T, k)
+    assert lay["act_order"] == 2
+    r = _run_and_compare(hl, dl, x, logits, k)
+    seg = np.diff(oracle.moe_forward(hl, x, logits, k)["offsets"])
+    if skew > 0:
+        assert (seg[seg > 0] <= 32).any() and (seg > 32).any()
+    _report(short_segments=int(((seg > 0) & (seg <= 32)).sum()), long_segments=int((seg > 32).sum()))
+    return r
 
 
 def _random_nibble_layer(E, H, N, seed):
