@@ -308,7 +308,7 @@ def test_forward_split_short_segments(E, H, N, k, T, skew):
     if skew > 0:
         assert (seg[seg > 0] <= 32).any() and (seg > 32).any()
     _report(short_segments=int(((seg > 0) & (seg <= 32)).sum()), long_segments=int((seg > 32).sum()))
-    return r
+    assert r["hq_frac"] <= 1e-3
 
 
 def _random_nibble_layer(E, H, N, seed):
