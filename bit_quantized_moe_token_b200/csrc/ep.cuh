@@ -84,13 +84,15 @@ __global__ void __launch_bounds__(256) k_ep_ids(const uint8_t* __restrict__ rec,
 // One CTA per received record r: its codes to row dst of q_out (dst = r when rop is null, the
 // narrow tiles' per-row gather, in their K order when perm; else rop[r], the expert-sorted row),
 // its scale to s_out[dst], and with qsum non-null the per-128-column sums of the FP8 values the
-// unsigned widening needs.  With ids non-null the checked local expert goes to ids[r].  A record
-// with a bad expert index gives a zero row with scale 0 under expert 0.
+// unsigned widening needs.  With `offsets` non-null (expert-sorted rows of a layer that runs its
+// short segments on narrow tiles) perm and qsum apply only to rows of segments of at most
+// kShortRows rows.  With ids non-null the checked local expert goes to ids[r].  A record with a
+// bad expert index gives a zero row with scale 0 under expert 0.
 __global__ void __launch_bounds__(256) k_ep_unpack(const uint8_t* __restrict__ rec, int H, int E_local,
                                                    const int32_t* __restrict__ rop,
                                                    int32_t* __restrict__ ids, uint8_t* __restrict__ q_out,
                                                    float* __restrict__ s_out, float* __restrict__ qsum,
-                                                   bool perm) {
+                                                   bool perm, const int32_t* __restrict__ offsets) {
     pdl_enter();
     const int64_t r = blockIdx.x;
     const uint8_t* src = rec + r * ep_record_bytes(H);
@@ -98,6 +100,11 @@ __global__ void __launch_bounds__(256) k_ep_unpack(const uint8_t* __restrict__ r
     const int e = *reinterpret_cast<const int32_t*>(meta + 4);
     const bool bad = e < 0 || e >= E_local;
     const int64_t dst = rop ? rop[r] : r;
+    if (offsets) {   // uniform over the CTA
+        const int ee = bad ? 0 : e;
+        perm = offsets[ee + 1] - offsets[ee] <= kShortRows;
+        if (!perm) qsum = nullptr;
+    }
     const int chunks = H >> 3;
     const int G = H / kGroup;
     for (int base = 0; base < chunks; base += blockDim.x) {   // blockDim = 256: whole half-warps
@@ -132,7 +139,7 @@ __global__ void __launch_bounds__(256) k_ep_unsort(const float* __restrict__ y,
 
 // The dispatching GPU's workspace, kept from moe_ep_dispatch to moe_ep_combine.
 struct EpSendPlan {
-    size_t ids, gates, offsets, sorted, rop, route_ws, sh_a, sh_y, total;
+    size_t ids, gates, offsets, sorted, rop, route_ws, sh_a, sh_y, sh_wd, total;
 };
 
 inline EpSendPlan plan_ep_send(const moe_w4a8_layer& L, int64_t T, int k) {
@@ -151,8 +158,9 @@ inline EpSendPlan plan_ep_send(const moe_w4a8_layer& L, int64_t T, int k) {
     p.rop = take(P * 4);
     p.route_ws = take(route_ws_bytes(T, L.E, k));
     if (L.n_shared > 0) {
-        p.sh_a = take((size_t)T * L.n_shared * L.shared_N * 2 * 2);
+        p.sh_a = take((size_t)T * L.n_shared * L.shared_N * 2);
         p.sh_y = take((size_t)T * L.H * 4);
+        p.sh_wd = take((size_t)L.n_shared * L.H * L.shared_N * 2);
     }
     p.total = off;
     return p;
@@ -244,10 +252,12 @@ extern "C" int moe_ep_experts_forward(const moe_w4a8_layer* local_layer, const u
     // tiles gather the rows in their K order with their group sums, wide ones read expert-sorted
     // copies
     const bool gather = ws_narrow(tc_tile_rows(R, L.E));
+    const bool split = ws_split(R, L.E, L.H, L.N);
+    float* qs_xr = (float*)at(p.qs_xr);
     const unsigned grid = static_cast<unsigned>(R);
     if (gather) {
         if ((st = launch_pdl(k_ep_unpack, dim3(grid), dim3(256), 0, stream, records, L.H, L.E,
-                             (const int32_t*)nullptr, ids, xq, sx, qs_x, true)))
+                             (const int32_t*)nullptr, ids, xq, sx, qs_x, true, (const int32_t*)nullptr)))
             return st;
         if ((st = launch_permute(ids, R, L.E, 1, offsets, sorted, rop, (int32_t*)at(p.route_ws), stream, zero,
                                  p.n_zero)))
@@ -258,12 +268,15 @@ extern "C" int moe_ep_experts_forward(const moe_w4a8_layer* local_layer, const u
         if ((st = launch_permute(ids, R, L.E, 1, offsets, sorted, rop, (int32_t*)at(p.route_ws), stream, zero,
                                  p.n_zero)))
             return st;
+        // the forward's split of a layer on 128-row tiles: rows of short segments in the narrow
+        // tiles' K order with their group sums
         if ((st = launch_pdl(k_ep_unpack, dim3(grid), dim3(256), 0, stream, records, L.H, L.E, (const int32_t*)rop,
-                             (int32_t*)nullptr, xs, sxs, (float*)nullptr, false)))
+                             (int32_t*)nullptr, xs, sxs, split ? qs_xr : (float*)nullptr, false,
+                             split ? (const int32_t*)offsets : (const int32_t*)nullptr)))
             return st;
     }
     StageMarks sm{nullptr, 0, 0};
-    RoutedRows rr{offsets, sorted, R, R, 1, gather, gather, xq, sx, xs, sxs, qs_x};
+    RoutedRows rr{offsets, sorted, R, R, 1, gather, gather, xq, sx, xs, sxs, qs_x, split, qs_xr};
     if ((st = run_experts(L, experts_of(L), p, w, rr, nullptr, stream, sm))) return st;
     const int64_t n = R * (L.H / 4);
     return launch_pdl(k_ep_unsort, dim3(static_cast<unsigned>((n + 255) / 256)), dim3(256), 0, stream,
@@ -288,8 +301,8 @@ extern "C" int moe_ep_combine(const moe_w4a8_layer* layer, const uint16_t* x_bf1
     char* w = static_cast<char*>(ws);
     StageMarks sm{nullptr, 0, 0};
     float* shared = nullptr;
-    if ((st = run_shared(L, reinterpret_cast<uint16_t*>(w + p.sh_a), reinterpret_cast<float*>(w + p.sh_y), x_bf16,
-                         T, stream, sm, &shared)))
+    if ((st = run_shared(L, reinterpret_cast<uint16_t*>(w + p.sh_a), reinterpret_cast<uint16_t*>(w + p.sh_wd),
+                         reinterpret_cast<float*>(w + p.sh_y), x_bf16, T, stream, sm, &shared)))
         return st;
     const int64_t n = T * (L.H / 4);
     return launch_pdl(k_combine, dim3(static_cast<unsigned>((n + 255) / 256)), dim3(256), 0, stream, y_back,

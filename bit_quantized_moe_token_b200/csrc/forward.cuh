@@ -214,7 +214,7 @@ struct WsPlan {
     size_t act16;        // NVFP4 experts: f16 copies of the GEMM inputs (max of [T|P, H] and [P, N])
     size_t slot_of;      // hybrid layers: expert -> slab map [E]
     int64_t n_zero;   // u32 words at `zero`: max|h| per row [P]
-    size_t sh_a, sh_y;
+    size_t sh_a, sh_y, sh_wd;
     size_t total;
 };
 
@@ -252,8 +252,9 @@ inline WsPlan plan_workspace(const moe_w4a8_layer& L, int64_t T, int k, int fmt 
     p.act16 = fmt >= 2 ? take((size_t)P * (L.H > L.N ? L.H : L.N) * 2) : 0;
     p.slot_of = fmt == 3 ? take((size_t)L.E * 4) : 0;
     if (L.n_shared > 0) {
-        p.sh_a = take((size_t)T * L.n_shared * L.shared_N * 2 * 2);   // bf16 hi | lo halves
+        p.sh_a = take((size_t)T * L.n_shared * L.shared_N * 2);      // f16 SwiGLU activations
         p.sh_y = take((size_t)T * L.H * 4);
+        p.sh_wd = take((size_t)L.n_shared * L.H * L.shared_N * 2);   // f16 copy of the down weights
     }
     p.total = off;
     return p;
@@ -295,7 +296,7 @@ extern "C" int moe_w4a8_workspace_layout(const moe_w4a8_layer* layer, int64_t T,
     out->s_h = p.s_h;
     out->total = p.total;
     // W4A8 layer: see the header
-    out->act_order = moe::ws_narrow(moe::ws_tile_rows(T * k, layer->E)) ? 1 : moe::ws_split(T * k, layer->E) ? 2 : 0;
+    out->act_order = moe::ws_narrow(moe::ws_tile_rows(T * k, layer->E)) ? 1 : moe::ws_split(T * k, layer->E, layer->H, layer->N) ? 2 : 0;
     return MOE_OK;
 }
 
@@ -383,20 +384,24 @@ extern "C" int moe_w4a8_forward_profiled(const moe_w4a8_layer* layer, const uint
 
 namespace moe {
 // S8: the shared experts, summed = one SwiGLU MLP of width n_shared * shared_N, into y fp32
-// [T, H] through sa (bf16 [T, 2 n_shared shared_N]); *shared = y, or null for a layer without
-// shared experts.
-inline int run_shared(const moe_w4a8_layer& L, uint16_t* sa, float* y, const uint16_t* x_bf16,
+// [T, H] through sa (the SwiGLU activations as f16 [T, n_shared shared_N], prescaled by 2^-8)
+// and wd (an f16 copy of the down weights [n_shared, H, shared_N]); *shared = y, or null for a
+// layer without shared experts.
+inline int run_shared(const moe_w4a8_layer& L, uint16_t* sa, uint16_t* wd, float* y, const uint16_t* x_bf16,
                       int64_t T, cudaStream_t stream, StageMarks& sm, float** shared) {
     *shared = nullptr;
     if (L.n_shared <= 0) return MOE_OK;
     const int Wsh = L.n_shared * L.shared_N;
-    // the SwiGLU activation as bf16 hi and lo halves [T, 2 Wsh]; the down GEMM reduces over both
-    Bf16GemmArgs g{Wsh, (int)T, L.H, 0, sa, 2 * Wsh, 0};
+    Bf16GemmArgs g{Wsh, (int)T, L.H, 0, sa, Wsh, 0};
     int st = launch_gemm_bf16_ws<true>(g, x_bf16, L.sh_gate, L.sh_up, stream);
     if (st) return st;
-    Bf16GemmArgs d{L.H, (int)T, 2 * Wsh, L.shared_N, y, L.H, Wsh};
-    if ((st = launch_gemm_bf16_ws<false>(d, sa, L.sh_down, nullptr, stream))) return st;
-    sm.launches += 2;
+    const int64_t n8 = (int64_t)Wsh * L.H / 8;
+    if ((st = launch_pdl(k_bf16_to_f16, dim3(static_cast<unsigned>((n8 + 255) / 256)), dim3(256), 0, stream,
+                         reinterpret_cast<const uint4*>(L.sh_down), reinterpret_cast<uint4*>(wd), n8)))
+        return st;
+    Bf16GemmArgs d{L.H, (int)T, Wsh, L.shared_N, y, L.H, Wsh};
+    if ((st = launch_gemm_bf16_ws<false, true>(d, sa, wd, nullptr, stream))) return st;
+    sm.launches += 3;
     *shared = y;
     return MOE_OK;
 }
@@ -599,7 +604,7 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const ExpertSet& xw, const ui
     // token quantization writes xq that way exactly when it is given the group sums
     const bool act_perm = gather && qsum_x != nullptr;
     // a W4A8 layer on 128-row tiles runs its short segments on narrow tiles (ws_split)
-    const bool split = xw.fmt == kFmtW4A8 && ws_split(P, L.E);
+    const bool split = xw.fmt == kFmtW4A8 && ws_split(P, L.E, L.H, L.N);
     float* qs_xr = (float*)at(p.qs_xr);
     // S1 into the expert-sorted rows (wide tiles) and per token
     auto quant_rows = [&]() -> int {
@@ -677,7 +682,8 @@ int moe::forward_impl(const moe_w4a8_layer* layer, const ExpertSet& xw, const ui
     }
     // S8
     float* shared = nullptr;
-    if ((st = run_shared(L, (uint16_t*)at(p.sh_a), (float*)at(p.sh_y), x_bf16, T, stream, sm, &shared)))
+    if ((st = run_shared(L, (uint16_t*)at(p.sh_a), (uint16_t*)at(p.sh_wd), (float*)at(p.sh_y), x_bf16, T, stream,
+                         sm, &shared)))
         return st;
     sm.mark(3, stream);
     {

@@ -11,11 +11,14 @@
 // of two TMEM accumulators (2 x BN columns), and warps 0-3 drain a finished accumulator while
 // the tensor core fills the other.  Swap AB again: MMA M = 128 weight rows, N = BN tokens.
 //   SwiGLU instance: M tile = 64 gate rows + the same 64 up rows; the epilogue writes
-//     a = silu(gate . x) * (up . x) as two bf16 halves, hi = bf16(a) in columns [0, M) and
-//     lo = bf16(a - hi) in columns [M, 2M) (hi + lo carries a to ~2^-18 relative: the layer
-//     keeps this activation in fp32, and bf16 alone would move outputs by up to ~1 %).
-//   plain instance: Y[t, m] fp32; for the shared down projection its K runs over both halves
-//     (K = 2 Kw), and the weights of K index k are those of k mod Kw.
+//     a = silu(gate . x) * (up . x) as f16(a * 2^-8): the layer keeps this activation in fp32,
+//     bf16 would move outputs by up to ~1 % (its 8-bit significand), f16 carries 11 bits, and
+//     the 2^-8 prescale keeps |a| up to 2^24 inside its range (values below 2^-6 lose relative
+//     precision as f16 subnormals, never more than 2^-17 absolute).
+//   plain instance, kF16: the shared down projection as an f16 MMA over those activations and an
+//     f16 copy of the bf16 down weights (every bf16 weight of magnitude 2^-14 .. 65504 is exact
+//     in f16), Y[t, m] = 256 * acc in fp32; the weights of K index k are those of k mod Kw.
+//   plain instance, bf16: Y[t, m] fp32 (not used by the layer).
 #pragma once
 #include <cuda.h>
 #include "common.cuh"
@@ -27,9 +30,9 @@ namespace moe {
 struct Bf16GemmArgs {
     int M;       // output rows of one projection (SwiGLU: n_shared*Ns; plain: H)
     int T;       // tokens
-    int K;       // reduction length of the activations (SwiGLU: H; plain: 2 * n_shared*Ns)
+    int K;       // reduction length of the activations (SwiGLU: H; plain: n_shared*Ns)
     int Ks;      // plain: K extent per shared expert (Ns); the 3-D weight map's inner dim
-    void* out;   // SwiGLU: bf16 [T, ldo] (hi | lo halves, ldo >= 2M); plain: fp32 [T, ldo]
+    void* out;   // SwiGLU: f16 [T, ldo] (a * 2^-8, ldo >= M); plain: fp32 [T, ldo]
     int ldo;
     int Kw;      // plain: K extent of the weights (n_shared*Ns); activation column k uses k mod Kw
 };
@@ -39,6 +42,10 @@ namespace tc {
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
     return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
            (static_cast<uint32_t>(M >> 4) << 24);
+}
+// The same with A = B = F16.
+__host__ __device__ constexpr uint32_t idesc_h16_f32(int M, int N) {
+    return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                          uint32_t idesc, uint32_t accumulate) {
@@ -78,7 +85,7 @@ struct Bf16Cfg {
     static constexpr int kTmemCols = 2 * BN;
 };
 
-template <int BN, bool kSwiGLU>
+template <int BN, bool kSwiGLU, bool kF16 = false>
 __global__ void __launch_bounds__(192, 1)
     k_gemm_bf16_ws(const __grid_constant__ CUtensorMap tm_w0, const __grid_constant__ CUtensorMap tm_w1,
                    const __grid_constant__ CUtensorMap tm_act, const Bf16GemmArgs a) {
@@ -144,7 +151,8 @@ __global__ void __launch_bounds__(192, 1)
         }
     } else if (warp == 5) {
         if (lane == 0) {
-            constexpr uint32_t idesc = tc::idesc_bf16_f32(128, BN);
+            // the SwiGLU instance multiplies bf16 tokens and weights; the plain kF16 instance f16 ones
+            constexpr uint32_t idesc = (!kSwiGLU && kF16) ? tc::idesc_h16_f32(128, BN) : tc::idesc_bf16_f32(128, BN);
             uint32_t it = 0, tcount = 0;
             for (int64_t tile = blockIdx.x; tile < n_tiles && !*abort; tile += gridDim.x, ++tcount) {
                 const int tb = tcount & 1;
@@ -187,16 +195,14 @@ __global__ void __launch_bounds__(192, 1)
                     }
                     ws::named_sync_math();
                     if (tid < 64) {
-                        uint16_t* out = static_cast<uint16_t*>(a.out);
+                        __half* out = static_cast<__half*>(a.out);
                         const int n = mt * 64 + tid;
 #pragma unroll
                         for (int j = 0; j < 32; ++j) {
                             const int t = n0 + c0 + j;
                             if (t < a.T) {
                                 const float h = silu(__uint_as_float(v[j])) * sX[tid * C::kXStride + j];
-                                const uint16_t hi = f32_to_bf16_bits(h);
-                                out[(int64_t)t * a.ldo + n] = hi;
-                                out[(int64_t)t * a.ldo + a.M + n] = f32_to_bf16_bits(h - bf16_bits_to_f32(hi));
+                                out[(int64_t)t * a.ldo + n] = __float2half_rn(h * 0.00390625f);   // h * 2^-8
                             }
                         }
                     }
@@ -204,10 +210,11 @@ __global__ void __launch_bounds__(192, 1)
                 } else {
                     float* out = static_cast<float*>(a.out);
                     const int m = mt * 128 + tid;
+                    constexpr float kUnscale = kF16 ? 256.0f : 1.0f;   // undo the activations' 2^-8
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
                         const int t = n0 + c0 + j;
-                        if (t < a.T) out[(int64_t)t * a.ldo + m] = __uint_as_float(v[j]);
+                        if (t < a.T) out[(int64_t)t * a.ldo + m] = __uint_as_float(v[j]) * kUnscale;
                     }
                 }
             }
@@ -223,6 +230,23 @@ __global__ void __launch_bounds__(192, 1)
         tc::tc_fence_after();
         tc::tmem_dealloc(tmem, C::kTmemCols);
     }
+}
+
+// bf16 -> f16, eight values per thread (round to nearest even; exact for magnitudes 2^-14 .. 65504).
+__global__ void __launch_bounds__(256) k_bf16_to_f16(const uint4* __restrict__ in, uint4* __restrict__ out,
+                                                     int64_t n8) {
+    pdl_enter();
+    const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    if (i >= n8) return;
+    const uint4 v = in[i];
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const __half2 h = __floats2half2_rn(__uint_as_float(w[q] << 16), __uint_as_float(w[q] & 0xFFFF0000u));
+        o[q] = *reinterpret_cast<const uint32_t*>(&h);
+    }
+    out[i] = make_uint4(o[0], o[1], o[2], o[3]);
 }
 
 // ---- host side -----------------------------------------------------------------------------
@@ -244,19 +268,21 @@ inline bool make_map_bf16_3d(CUtensorMap* m, const void* base, uint64_t d0, uint
     return encode_tiled(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-template <bool kSwiGLU>
+// kF16: the plain instance as the shared down projection (f16 operands, output x 256); the router
+// logits use the plain bf16 instance.
+template <bool kSwiGLU, bool kF16 = false>
 int launch_gemm_bf16_ws(const Bf16GemmArgs& a, const void* act, const void* w0, const void* w1,
                         cudaStream_t stream) {
     constexpr int BN = 256;
     using C = Bf16Cfg<BN>;
     // plain instance: the weights' K extent Kw is a whole number of Ks-wide slices, and the
-    // activations' K a whole number of Kw (the shared down projection: two halves)
+    // activations' K a whole number of Kw
     if (!kSwiGLU && (a.Ks <= 0 || a.Kw <= 0 || a.Kw % a.Ks || a.K % a.Kw || a.Kw % 64))
         return MOE_ERR_INVALID_ARG;
     static int sms_cache[16] = {0};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
-    auto kern = k_gemm_bf16_ws<BN, kSwiGLU>;
+    auto kern = k_gemm_bf16_ws<BN, kSwiGLU, kF16>;
     if (sms_cache[dev & 15] == 0) {
         int sms = 0;
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kAlloc) != cudaSuccess ||

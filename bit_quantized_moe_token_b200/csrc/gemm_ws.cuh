@@ -613,8 +613,15 @@ inline bool ws_narrow(int BN) { return BN <= 32; }
 // A W4A8 layer on 128-row tiles (segments of 24 to 160 rows on average, typically skewed) runs
 // its segments of at most kShortRows rows on 32-row tiles, which widen unsigned and cost a
 // quarter of the integer work per weight: at T = 2048 with Zipf routing 84 of 184 128-row tiles
-// hold at most 32 rows (5 % of the rows).
-inline bool ws_split(int64_t P, int E) { return ws_tile_rows(P, E) == 128; }
+// hold at most 32 rows (5 % of the rows).  Only where both reductions span at least sixteen
+// K-groups (H, N >= 2048, the model's depths): the unsigned form's +8-biased sums lose up to half
+// an fp32 ulp each, which averages out over many groups but not over a few, and a requantized
+// code it tips over moves its token's outputs by ~1/N (measured on random layers: split, a
+// 256 x 128 layer put an output at 2.8 x the tolerance, 0.78 x unsplit; at 1024 x 1024 one
+// layer reached 1.36 x split; at 4096 x 2048 every case stays within 0.78 x).
+inline bool ws_split(int64_t P, int E, int H, int N) {
+    return H >= 16 * kGroup && N >= 16 * kGroup && ws_tile_rows(P, E) == 128;
+}
 
 // bn: the token-tile width (0: chosen from the average segment length, ws_tile_rows);
 // rows_sorted: a narrow gate/up launch reads expert-sorted activation rows instead of gathering

@@ -182,7 +182,8 @@ size_t moe_w4a8_workspace_bytes(const moe_w4a8_layer* layer, int64_t T, int k);
  * 32-row token tiles split a packed word into its even and odd nibbles; used for W4A8 and
  * hybrid layers whose tiles are that narrow); 2 when xq is in column order and the hq rows of
  * experts whose segment has at most 32 rows are in that K order, the other rows in column order
- * (a W4A8 layer on 128-row tiles, which runs its short segments on 32-row tiles). */
+ * (a W4A8 layer on 128-row tiles with H and N of at least 2048, which runs its short segments on
+ * 32-row tiles). */
 typedef struct {
     size_t topk_ids, topk_w, expert_offsets, sorted_pairs, row_of_pair;
     size_t xq, s_x, hq, s_h;

@@ -53,8 +53,10 @@ def _expected_records(x, logits, E, k, n_ranks):
     return rec, counts
 
 
-# (E, H, N, k, T): narrow 16- and 32-row token tiles, wide tiles, a ragged batch
-CASES = [(8, 256, 128, 2, 5), (8, 256, 128, 2, 37), (16, 256, 128, 4, 64), (8, 512, 256, 2, 700)]
+# (E, H, N, k, T): narrow 16- and 32-row token tiles, 192-row tiles, 128-row tiles with the short
+# segments (9 of 16 here) on 32-row tiles
+CASES = [(8, 256, 128, 2, 5), (8, 256, 128, 2, 37), (16, 256, 128, 4, 64), (8, 512, 256, 2, 700),
+         (16, 4096, 2048, 2, 260)]
 
 
 @pytest.mark.parametrize("E,H,N,k,T", CASES)

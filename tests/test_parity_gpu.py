@@ -291,22 +291,29 @@ def test_forward_ragged_shapes(E, H, N, k, T):
     _run_and_compare(hl, dl, x, logits, k)
 
 
-@pytest.mark.parametrize("E,H,N,k,T,skew", [(16, 512, 256, 2, 400, 3.0), (32, 256, 128, 4, 600, 2.0),
-                                              (8, 256, 256, 2, 600, 0.0)])
+@pytest.mark.parametrize("E,H,N,k,T,skew", [(16, 4096, 2048, 2, 400, 3.0), (32, 4096, 2048, 4, 600, 2.0),
+                                              (8, 4096, 2048, 2, 600, 0.0), (16, 256, 128, 2, 260, 0.0),
+                                              (8, 1024, 1024, 2, 600, 0.0)])
 def test_forward_split_short_segments(E, H, N, k, T, skew):
-    """Layers on 128-row tiles run their segments of at most 32 rows on 32-row tiles (unsigned
-    widening, sorted rows in its K order) and the others on 128-row tiles: skewed routing gives
-    both kinds in one layer (the last case, uniform, leaves the narrow launch empty)."""
+    """Layers on 128-row tiles at the model's depths (H, N >= 2048) run their segments of at most
+    32 rows on 32-row tiles (unsigned widening, sorted rows in its K order) and the others on
+    128-row tiles: skewed routing gives both kinds in one layer (the third case, uniform, leaves the
+    narrow launch empty).  The last two layers are too shallow for the split and stay on 128-row
+    tiles: the 256 x 128 one put an output at 2.8 x the tolerance when it split (0.78 x unsplit).
+    The 1024 x 1024 one has, split or not, one requantized code one step from the oracle's (rule 2),
+    which moves two outputs of its token to 1.2 x the tolerance: the only W4A8 case that needs the
+    named allowance (a step of one of N = 1024 activations weighs 2 x what it does at 2048)."""
     hl, dl = _host_layer_and_dev(E, H, N, seed=31 + E, n_shared=1, shared_N=128)
     x = synth.normal_bf16(33, 73_000, T * H, 1.0).reshape(T, H)
     logits = synth.normal_f32(33, 73_001, T * E, 1.0).reshape(T, E)
     logits += (skew * np.linspace(1.0, 0.0, E)).astype(np.float32)   # early experts preferred
     lay = moe.moe_w4a8_workspace_layout(dl, T, k)
-    assert lay["act_order"] == 2
-    r = _run_and_compare(hl, dl, x, logits, k)
+    assert lay["act_order"] == (2 if H >= 2048 and N >= 2048 else 0)
+    allow = ("w4a8 1024 x 1024 uniform, layer seed 39, inputs seed 33", 4) if (H, N) == (1024, 1024) else None
+    r = _run_and_compare(hl, dl, x, logits, k, allow=allow)
     seg = np.diff(oracle.moe_forward(hl, x, logits, k)["offsets"])
-    if skew > 0:
-        assert (seg[seg > 0] <= 32).any() and (seg > 32).any()
+    if skew > 0 or H < 1024:
+        assert (seg[seg > 0] <= 32).any() and (seg > 32).any()   # both kinds of segment
     _report(short_segments=int(((seg > 0) & (seg <= 32)).sum()), long_segments=int((seg > 32).sum()))
     assert r["hq_frac"] <= 1e-3
 
