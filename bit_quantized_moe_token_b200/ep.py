@@ -107,10 +107,13 @@ class EpLayer:
         send_counts = torch.empty(n, dtype=torch.int32, device=dev)
         send = torch.empty((T * k, rb), dtype=torch.uint8, device=dev)
         self.ops.dispatch(self.layer, x, logits, k, n, send_counts, send, ws_d)
-        # how many records go each way: one int per rank pair, then to the host for the splits
-        recv_counts = self._exchange(send_counts, n)
-        counts = torch.cat([send_counts, recv_counts]).cpu().tolist()
-        sc, rc = counts[:n], counts[n:]
+        if self.grouped:
+            # how many records go each way: one int per rank pair, then to the host for the splits
+            recv_counts = self._exchange(send_counts, n)
+            counts = torch.cat([send_counts, recv_counts]).cpu().tolist()
+            sc, rc = counts[:n], counts[n:]
+        else:
+            sc = rc = [T * k]   # alone: every record stays here, and nothing needs the host
         R = sum(rc)
         recv = self._exchange(send, R, rc, sc)
         y_rows = torch.empty((R, H), dtype=torch.float32, device=dev)
